@@ -1,0 +1,246 @@
+"""Oracle decoding procedures: AR steps, self-speculation rounds, block-diffusion steps.
+
+Test infrastructure only (see the package docstring).  Written from:
+* ranhao.site notes section 5.1 (AR: left-to-right p(x_i | x_<i)), 5.2 (a block starts as
+  [MASK] tokens and is denoised over several forwards, committing high-confidence positions),
+  5.3 (the diffusion pathway drafts k tokens in parallel, the AR pathway verifies, the
+  longest correct prefix is accepted and acceptance stops at the first mismatch);
+* r9-hu digest "Method", tri-mode inference (k drafts from one forward, a causal second
+  forward verifies them, 1 to k+1 tokens per round);
+* shilu.ai "Deploy and infer with SGLang" (32-token blocks; a confidence threshold decides
+  which tokens are committed each step; self-speculation is lossless against AR at
+  temperature 0).
+
+Readings where the pages are silent (each is listed with its reason in the design notes):
+* State between rounds: KV rows 0..n-1 are cached; the last committed token x_n is
+  "pending" (committed, no KV row yet) and sits at position n.
+* Shifted prediction in every mode: the output row at position i scores the token at i+1.
+  A draft block is [x_n, MASK x (k-1)] at positions n..n+k-1 and its k rows give the k
+  drafts d_1..d_k; with k == 1 the draft forward is exactly the AR step.
+* Verify input is [x_n, d_1..d_k] (k+1 rows, causal) giving v_1..v_{k+1}; a = the number of
+  leading i with d_i == v_i; the round commits v_1..v_{a+1}, KV rows n..n+a come from the
+  verify forward, pending becomes v_{a+1}.
+* Argmax ties resolve to the lowest token id; confidence is the largest softmax probability
+  over the V real tokens; a diffusion step commits every still-masked slot whose confidence
+  is >= tau, or else the single most confident one (lowest slot on ties).  A complete
+  block gets one causal forward over [x_n, b_1..b_{k-1}] that writes its KV rows; b_k
+  becomes the pending token.  With several sequences, a sequence whose block is complete
+  waits (its rows are computed and ignored) until every block is complete.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional, Tuple
+
+import torch
+
+
+def argmax_lowest(logits: torch.Tensor) -> torch.Tensor:
+    """Index of the largest logit along the last axis, the lowest index among equal maxima."""
+    mx = logits.max(dim=-1, keepdim=True).values
+    idx = torch.arange(logits.shape[-1]).expand_as(logits)
+    big = torch.full_like(idx, logits.shape[-1])
+    return torch.where(logits == mx, idx, big).min(dim=-1).values
+
+
+def confidence(logits: torch.Tensor) -> torch.Tensor:
+    """Largest softmax probability along the last axis: 1 / sum_v exp(l_v - max l)."""
+    mx = logits.max(dim=-1, keepdim=True).values
+    return 1.0 / torch.exp(logits - mx).sum(dim=-1)
+
+
+def accept_length(draft: List[int], verify: List[int]) -> int:
+    """Greedy longest matching prefix: the number of leading positions i (0-based, i < k)
+    with draft[i] == verify[i]; stops at the first mismatch."""
+    a = 0
+    for d, v in zip(draft, verify):
+        if d != v:
+            break
+        a += 1
+    return a
+
+
+def commit_after_verify(draft: List[int], verify: List[int],
+                        forced: Optional[int] = None) -> List[int]:
+    """Tokens a round commits: v_1..v_{a+1} (== d_1..d_a, v_{a+1}).  With a forced count c
+    (1..k+1) the round commits d_1..d_{c-1}, v_c instead: the tokens the verify forward's
+    first c KV rows belong to, closed by that forward's prediction."""
+    k = len(draft)
+    assert len(verify) == k + 1
+    if forced is None:
+        a = accept_length(draft, verify)
+        return list(verify[:a + 1])
+    assert 1 <= forced <= k + 1
+    return list(draft[:forced - 1]) + [verify[forced - 1]]
+
+
+def diffusion_commit(masked: List[bool], conf: List[float], tau: float) -> List[bool]:
+    """Slots committed by one confidence-threshold step: every masked slot with conf >= tau;
+    if none qualifies, the masked slot of highest confidence (lowest slot on ties)."""
+    pick = [mk and (cf >= tau) for mk, cf in zip(masked, conf)]
+    if any(pick) or not any(masked):
+        return pick
+    best = None
+    for i, (mk, cf) in enumerate(zip(masked, conf)):
+        if mk and (best is None or cf > conf[best]):
+            best = i
+    pick[best] = True
+    return pick
+
+
+@dataclasses.dataclass
+class SeqState:
+    cache: list               # OracleModel cache
+    lens: List[int]           # cached KV rows per sequence
+    pending: List[int]        # committed token without a KV row, at position lens[b]
+    block: Optional[List[List[int]]] = None   # diffusion block b_1..b_k (mask id = open)
+
+
+def prefill(model, prompt: torch.Tensor, capacity: int) -> SeqState:
+    """Causal forward over prompt[:, :P-1] writing KV rows 0..P-2; pending = prompt[:, P-1]."""
+    B, P = prompt.shape
+    cache = model.new_cache(B, capacity)
+    if P > 1:
+        model.forward(prompt[:, :P - 1], [0] * B, cache, block_size=1, write_kv=True,
+                      with_logits=False)
+    return SeqState(cache=cache, lens=[P - 1] * B, pending=[int(t) for t in prompt[:, P - 1]])
+
+
+def ar_forward(model, st: SeqState) -> torch.Tensor:
+    """Logits [B, 1, V] of the causal one-token forward over the pending tokens (writes KV)."""
+    toks = torch.tensor(st.pending, dtype=torch.int64)[:, None]
+    return model.forward(toks, st.lens, st.cache, block_size=1, write_kv=True)
+
+
+def ar_step(model, st: SeqState) -> List[int]:
+    logits = ar_forward(model, st)
+    nxt = argmax_lowest(logits[:, 0]).tolist()
+    for b in range(len(st.lens)):
+        st.lens[b] += 1
+        st.pending[b] = nxt[b]
+    return nxt
+
+
+def draft_forward(model, st: SeqState, k: int) -> torch.Tensor:
+    """Logits [B, k, V] of the diffusion draft forward over [x_n, MASK x (k-1)], one
+    bidirectional block over the cached prefix.  Draft KV rows are not kept."""
+    B = len(st.lens)
+    toks = torch.full((B, k), model.cfg.mask_id, dtype=torch.int64)
+    toks[:, 0] = torch.tensor(st.pending)
+    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False)
+
+
+def verify_forward(model, st: SeqState, drafts: List[List[int]]) -> torch.Tensor:
+    """Logits [B, k+1, V] of the causal forward over [x_n, d_1..d_k]; writes KV rows
+    n..n+k (only the accepted ones become part of the cache, by the length update)."""
+    toks = torch.tensor([[st.pending[b]] + list(drafts[b]) for b in range(len(st.lens))],
+                        dtype=torch.int64)
+    return model.forward(toks, st.lens, st.cache, block_size=1, write_kv=True)
+
+
+def apply_commit(st: SeqState, committed: List[List[int]]) -> None:
+    for b, toks in enumerate(committed):
+        st.lens[b] += len(toks)
+        st.pending[b] = toks[-1]
+
+
+def selfspec_round(model, st: SeqState, k: int, forced: Optional[List[int]] = None):
+    """One linear self-speculation round.  Returns (committed token lists, drafts, verify
+    argmaxes, draft logits, verify logits)."""
+    dl = draft_forward(model, st, k)
+    drafts = argmax_lowest(dl).tolist()
+    vl = verify_forward(model, st, drafts)
+    ver = argmax_lowest(vl).tolist()
+    committed = [commit_after_verify(drafts[b], ver[b], None if forced is None else forced[b])
+                 for b in range(len(st.lens))]
+    apply_commit(st, committed)
+    return committed, drafts, ver, dl, vl
+
+
+def diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
+    """Logits [B, k, V] of one denoising forward over [x_n, b_1..b_{k-1}] (open slots hold
+    the mask id), one bidirectional block; row i scores slot b_{i+1}."""
+    toks = torch.tensor([[st.pending[b]] + st.block[b][:k - 1] for b in range(len(st.lens))],
+                        dtype=torch.int64)
+    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False)
+
+
+def diffusion_step(model, st: SeqState, k: int, tau: float):
+    """One denoising step for every sequence (lockstep).  Returns a dict with
+    newly: per sequence the (slot, token) pairs committed this step,
+    conf [B,k], argmax [B,k] (row i scores slot i, i.e. b_{i+1}),
+    filled: whether the blocks completed and got their causal KV-fill forward,
+    blocks: the completed blocks (b_1..b_k per sequence) when filled, else None."""
+    mask_id = model.cfg.mask_id
+    B = len(st.lens)
+    if st.block is None:
+        st.block = [[mask_id] * k for _ in range(B)]
+    logits = diffusion_forward(model, st, k)
+    conf = confidence(logits)
+    am = argmax_lowest(logits)
+    newly = []
+    for b in range(B):
+        masked = [t == mask_id for t in st.block[b]]
+        pick = diffusion_commit(masked, conf[b].tolist(), tau)
+        got = []
+        for s in range(k):
+            if pick[s]:
+                st.block[b][s] = int(am[b, s])
+                got.append((s, int(am[b, s])))
+        newly.append(got)
+    filled = all(mask_id not in st.block[b] for b in range(B))
+    blocks = None
+    if filled:
+        blocks = [list(st.block[b]) for b in range(B)]
+        toks = torch.tensor([[st.pending[b]] + st.block[b][:k - 1] for b in range(B)],
+                            dtype=torch.int64)
+        model.forward(toks, st.lens, st.cache, block_size=1, write_kv=True, with_logits=False)
+        for b in range(B):
+            st.lens[b] += k
+            st.pending[b] = st.block[b][k - 1]
+        st.block = [[mask_id] * k for _ in range(B)]
+    return dict(newly=newly, conf=conf, argmax=am, filled=filled, blocks=blocks,
+                logits=logits)
+
+
+# ---- generation drivers (exactly N generated tokens; the last round is truncated) ----------
+
+def ar_generate(model, prompt: torch.Tensor, n_tokens: int, capacity: int) -> List[List[int]]:
+    st = prefill(model, prompt, capacity)
+    out = [[] for _ in range(prompt.shape[0])]
+    while len(out[0]) < n_tokens:
+        nxt = ar_step(model, st)
+        for b, t in enumerate(nxt):
+            out[b].append(t)
+    return out
+
+
+def selfspec_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, capacity: int
+                      ) -> Tuple[List[List[int]], List[List[int]]]:
+    """Returns (tokens per sequence, commits per round per sequence)."""
+    st = prefill(model, prompt, capacity)
+    B = prompt.shape[0]
+    out = [[] for _ in range(B)]
+    per_round = [[] for _ in range(B)]
+    while min(len(o) for o in out) < n_tokens:
+        committed, *_ = selfspec_round(model, st, k)
+        for b in range(B):
+            out[b].extend(committed[b])
+            per_round[b].append(len(committed[b]))
+    return [o[:n_tokens] for o in out], per_round
+
+
+def diffuse_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, tau: float,
+                     capacity: int) -> Tuple[List[List[int]], int]:
+    """Returns (tokens per sequence in position order, number of denoising steps)."""
+    st = prefill(model, prompt, capacity)
+    B = prompt.shape[0]
+    out = [[] for _ in range(B)]
+    steps = 0
+    while min(len(o) for o in out) < n_tokens:
+        r = diffusion_step(model, st, k, tau)
+        steps += 1
+        if r["filled"]:
+            for b in range(B):
+                out[b].extend(r["blocks"][b])
+    return [o[:n_tokens] for o in out], steps

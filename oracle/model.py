@@ -1,0 +1,189 @@
+"""Oracle decoder forward: a plain Llama-style transformer with explicit attention masks.
+
+Test infrastructure only (see the package docstring).  Everything here is the textbook
+definition written out with whole-tensor torch CPU ops (a matmul is the only library
+primitive used as a step); nothing is blocked, fused or reordered.
+
+Model (Llama-style decoder named for the workloads; weights from `synth`):
+  h0 = E[t]
+  per layer:  a = rmsnorm(h) * g1
+              q, k, v = a Wq^T, a Wk^T, a Wv^T ; RoPE on q and k at the absolute position
+              query head j reads kv head floor(j / (Hq/Hkv))
+              o = softmax(q k^T / sqrt(hd) + mask) v ;  h += o Wo^T
+              m = rmsnorm(h) * g2 ;  h += (silu(m Wg^T) * (m Wu^T)) Wd^T
+  logits = (rmsnorm(h) * gf) Wlm^T                          over the V real tokens
+  rmsnorm(x) = x / sqrt(mean(x^2) + eps)
+
+Attention mask (ranhao.site notes section 3.2 and r9-hu digest "Method": bidirectional
+inside a block, causal across blocks, the clean prefix reused as KV; section 4.3: the clean
+stream is strictly causal).  A forward covers positions n..n+m-1 of one sequence, cut into
+blocks of `block_size` starting at n.  A query sees every cached prefix key (j < n) and
+every key of the forward whose block index is not above its own.  block_size == 1 is the
+strictly causal mask.
+
+Precision modes
+  "f64"    float64 everywhere (the reference semantics).
+  "f32"    float32 everywhere.
+  "bf16io" float32 arithmetic with bf16 rounding where a bf16 library keeps activations in
+           storage: the matmul operand bf16(h), the stored q/k/v rows, the attention
+           output, the SwiGLU product.  The RMSNorm scale 1/rms is applied to the matmul
+           result instead of its operand (the same value in exact arithmetic, since the
+           norm scales each row by one number).  This is the rounding-matched mode the
+           tolerances of the bf16 parity tests are stated against.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import torch
+
+F32 = 0
+BF16 = 1
+
+
+def rmsnorm(x: torch.Tensor, eps: float) -> torch.Tensor:
+    """x / sqrt(mean(x^2) + eps) over the last axis (no gain)."""
+    return x / torch.sqrt((x * x).mean(dim=-1, keepdim=True) + eps)
+
+
+def inv_rms(x: torch.Tensor, eps: float) -> torch.Tensor:
+    return 1.0 / torch.sqrt((x * x).mean(dim=-1, keepdim=True) + eps)
+
+
+def rope_rotate(x: torch.Tensor, pos: torch.Tensor, theta: float) -> torch.Tensor:
+    """Rotary embedding, rotate-half pairing: element i is paired with i + hd/2 and the pair
+    is rotated by angle pos * theta^(-2i/hd).  x: [..., hd]; pos broadcasts against x[..., 0]."""
+    hd = x.shape[-1]
+    half = hd // 2
+    i = torch.arange(half, dtype=torch.float64)
+    inv_freq = theta ** (-2.0 * i / hd)                      # [half]
+    ang = pos.to(torch.float64)[..., None] * inv_freq        # [..., half]
+    c = torch.cos(ang).to(x.dtype)
+    s = torch.sin(ang).to(x.dtype)
+    x1 = x[..., :half]
+    x2 = x[..., half:]
+    return torch.cat([x1 * c - x2 * s, x2 * c + x1 * s], dim=-1)
+
+
+def causal_mask(m: int, n: int) -> torch.Tensor:
+    """[m, n+m] bool: query r (position n+r) sees key j iff j <= n+r."""
+    j = torch.arange(n + m)[None, :]
+    r = torch.arange(m)[:, None]
+    return j <= n + r
+
+
+def block_mask(m: int, n: int, block_size: int) -> torch.Tensor:
+    """[m, n+m] bool: prefix keys (j < n) always visible; keys of the forward are visible
+    when their block index (j-n)//block_size is not above the query's r//block_size."""
+    j = torch.arange(n + m)[None, :]
+    r = torch.arange(m)[:, None]
+    in_prefix = j < n
+    key_blk = torch.div(j - n, block_size, rounding_mode="floor")
+    q_blk = torch.div(r, block_size, rounding_mode="floor")
+    return in_prefix | ((j >= n) & (key_blk <= q_blk))
+
+
+def attention_explicit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       mask: torch.Tensor) -> torch.Tensor:
+    """Masked softmax attention written out: q [Hq, m, hd], k/v [Hkv, L, hd], mask [m, L].
+    Query head j uses kv head j // (Hq/Hkv).  Masked scores are -inf."""
+    Hq, m, hd = q.shape
+    Hkv = k.shape[0]
+    group = Hq // Hkv
+    kv_idx = torch.arange(Hq) // group
+    kk = k[kv_idx]                                            # [Hq, L, hd]
+    vv = v[kv_idx]
+    s = torch.matmul(q, kk.transpose(1, 2)) / math.sqrt(hd)  # [Hq, m, L]
+    s = s.masked_fill(~mask[None, :, :], float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    return torch.matmul(p, vv)
+
+
+def _bf16(x: torch.Tensor) -> torch.Tensor:
+    return x.to(torch.bfloat16).to(x.dtype)
+
+
+class OracleModel:
+    """Holds the weights (as given, bf16 or fp32 CPU tensors in the boundary's order) and
+    runs forwards with an explicit KV cache [B][layer] -> (K [Hkv, cap, hd], V ...)."""
+
+    def __init__(self, cfg, weights: List[Optional[torch.Tensor]], precision: str = "f64"):
+        assert precision in ("f64", "f32", "bf16io")
+        self.cfg = cfg
+        self.precision = precision
+        self.cdt = torch.float64 if precision == "f64" else torch.float32
+        w = [None if t is None else t.detach().cpu() for t in weights]
+        self.embed = w[0]
+        self.layers = []
+        for l in range(cfg.n_layers):
+            b = 1 + 9 * l
+            self.layers.append(dict(g1=w[b], wq=w[b + 1], wk=w[b + 2], wv=w[b + 3], wo=w[b + 4],
+                                    g2=w[b + 5], wg=w[b + 6], wu=w[b + 7], wd=w[b + 8]))
+        self.gf = w[1 + 9 * cfg.n_layers]
+        self.lm = w[2 + 9 * cfg.n_layers]
+
+    # -- helpers ------------------------------------------------------------------------
+    def _w(self, t: torch.Tensor) -> torch.Tensor:
+        return t.to(self.cdt)
+
+    def _mm(self, x: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
+        return torch.matmul(x, self._w(w).t())
+
+    def _normed_mm(self, h: torch.Tensor, g: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
+        """(rmsnorm(h) * g) W^T, in the rounding of the precision mode."""
+        eps = self.cfg.rms_eps
+        if self.precision == "bf16io":
+            return self._mm(_bf16(h) * self._w(g), w) * inv_rms(h, eps)
+        return self._mm(rmsnorm(h, eps) * self._w(g), w)
+
+    def _store(self, x: torch.Tensor) -> torch.Tensor:
+        return _bf16(x) if self.precision == "bf16io" else x
+
+    def new_cache(self, batch: int, capacity: int):
+        c = self.cfg
+        return [[(torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.cdt),
+                  torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.cdt))
+                 for _ in range(c.n_layers)] for _ in range(batch)]
+
+    # -- forward ------------------------------------------------------------------------
+    def forward(self, tokens: torch.Tensor, starts: List[int], cache, block_size: int,
+                write_kv: bool, layers: Optional[List[int]] = None,
+                with_logits: bool = True) -> Optional[torch.Tensor]:
+        """tokens [B, m] at positions starts[b]..starts[b]+m-1 over cached rows
+        [0, starts[b]).  block_size 1 = causal; block_size m = one bidirectional block.
+        write_kv stores this forward's K/V rows into the cache at their positions.
+        Returns logits [B, m, V] (compute dtype) or None."""
+        c = self.cfg
+        B, m = tokens.shape
+        hd, Hq, Hkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+        h = self._w(self.embed[tokens.long()])                # [B, m, d]
+        for li in (range(c.n_layers) if layers is None else layers):
+            L = self.layers[li]
+            q = self._normed_mm(h, L["g1"], L["wq"]).view(B, m, Hq, hd)
+            k = self._normed_mm(h, L["g1"], L["wk"]).view(B, m, Hkv, hd)
+            v = self._normed_mm(h, L["g1"], L["wv"]).view(B, m, Hkv, hd)
+            att = torch.empty(B, m, Hq, hd, dtype=self.cdt)
+            for b in range(B):
+                n = int(starts[b])
+                pos = torch.arange(n, n + m)
+                qb = self._store(rope_rotate(q[b], pos[:, None], c.rope_theta))   # [m, Hq, hd]
+                kb = self._store(rope_rotate(k[b], pos[:, None], c.rope_theta))   # [m, Hkv, hd]
+                vb = self._store(v[b])
+                Kc, Vc = cache[b][li]
+                keys = torch.cat([Kc[:, :n], kb.transpose(0, 1)], dim=1)          # [Hkv, n+m, hd]
+                vals = torch.cat([Vc[:, :n], vb.transpose(0, 1)], dim=1)
+                mask = block_mask(m, n, block_size)
+                o = attention_explicit(qb.transpose(0, 1), keys, vals, mask)      # [Hq, m, hd]
+                att[b] = self._store(o.transpose(0, 1))
+                if write_kv:
+                    Kc[:, n:n + m] = kb.transpose(0, 1)
+                    Vc[:, n:n + m] = vb.transpose(0, 1)
+            h = h + self._mm(att.reshape(B, m, Hq * hd), L["wo"])
+            g = self._normed_mm(h, L["g2"], L["wg"])
+            u = self._normed_mm(h, L["g2"], L["wu"])
+            act = self._store(g / (1.0 + torch.exp(-g)) * u)      # silu(g) * u
+            h = h + self._mm(act, L["wd"])
+        if not with_logits:
+            return None
+        return self._normed_mm(h, self.gf, self.lm)
