@@ -1,0 +1,205 @@
+/*
+ * nld.h -- C ABI of the tri-mode (AR / block diffusion / self-speculation) decode round.
+ *
+ * The operations follow the pages on Nemotron-Labs-Diffusion:
+ *   - AR step: ranhao.site technical-report notes, section 5.1 (left-to-right p(x_i|x_<i)).
+ *   - Draft forward: notes section 3.2 and the r9-hu digest, "Method" (one block, attention
+ *     bidirectional inside the block and causal over the cached clean prefix).
+ *   - Verify forward and acceptance: notes section 5.3 and r9-hu "Method" (k drafts, a
+ *     causal verification forward, the longest matching prefix is accepted, 1..k+1 tokens).
+ *   - Diffusion step: notes section 5.2 and shilu.ai "Deploy and infer with SGLang"
+ *     (32-token block of [MASK] ids denoised over several forwards; a confidence threshold
+ *     decides which positions commit).
+ *
+ * Conventions shared by every call
+ *   - All device pointers are CUDA device addresses on the context's device.  "h_" pointers
+ *     are host addresses.  Sizes are element counts unless stated.
+ *   - Every call is stream-ordered on the context's stream and returns without waiting for
+ *     the GPU unless its comment says it synchronises.  Outputs are valid once the stream
+ *     has reached the call.
+ *   - No call throws.  A call that fails argument or state validation launches nothing and
+ *     returns a status; nld_last_error() then describes the failure.  Device-side faults
+ *     detected by bounds checks (KV capacity exceeded, token id out of range, a bounded wait
+ *     that ran out) set an error word on the device; nld_sync() reports it.
+ *   - Sequence state lives in the context: per sequence the number of cached KV rows (len),
+ *     the pending token (committed, no KV row yet, at position len), the last drafts and
+ *     verifier argmaxes, and the diffusion block.  Predictions are shifted: the output row at
+ *     position i scores the token at position i+1.
+ *   - Token ids are int32 in [0, vocab); the [MASK] id is `vocab` (the embedding has
+ *     vocab+1 rows, the LM head vocab rows).
+ */
+#ifndef NLD_H
+#define NLD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct nld_ctx nld_ctx;
+
+typedef enum {
+  NLD_OK = 0,
+  NLD_ERR_ARG = 1,         /* invalid argument or configuration */
+  NLD_ERR_OOM = 2,         /* device allocation failed */
+  NLD_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  NLD_ERR_KV_FULL = 4,     /* the call would write past max_seq KV rows */
+  NLD_ERR_STATE = 5,       /* call out of order (e.g. a round before prefill) */
+  NLD_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (device error word) */
+  NLD_ERR_DEVICE = 7,      /* a device bounds check failed (device error word) */
+  NLD_ERR_UNSUPPORTED = 8  /* shape outside what the kernels implement */
+} nld_status;
+
+enum { NLD_F32 = 0, NLD_BF16 = 1 };
+
+/* Forward kinds accepted by nld_debug_logits. */
+enum { NLD_MODE_AR = 0, NLD_MODE_DRAFT = 1, NLD_MODE_VERIFY = 2, NLD_MODE_DIFFUSE = 3 };
+
+/* Device error word bits (reported by nld_sync). */
+enum { NLD_DEVERR_KV_OVERFLOW = 1, NLD_DEVERR_TIMEOUT = 2, NLD_DEVERR_TOKEN = 4 };
+
+/*
+ * Model and context configuration (Llama-style decoder: RMSNorm, RoPE with rotate-half
+ * pairing, GQA attention, SwiGLU MLP, untied LM head).
+ *   dtype        NLD_BF16: bf16 weights, activations and KV, fp32 accumulation, tensor-core
+ *                (tcgen05) GEMMs; NLD_F32: fp32 throughout on SIMT kernels.
+ *   head_dim     64 or 128 (bf16 requires 128).
+ *   d_model      multiple of 128; ffn_dim multiple of 64; n_q_heads*head_dim multiple of 128.
+ *   page_size    KV page length in tokens; must be 64.
+ *   block_k      draft / diffusion block length, 1..32.
+ *   max_seq      KV rows a sequence may hold (prompt + generated tokens).
+ */
+typedef struct {
+  int n_layers, d_model, n_q_heads, n_kv_heads, head_dim, ffn_dim, vocab;
+  int dtype;
+  int max_batch, max_seq, page_size, block_k;
+  float rms_eps, rope_theta;
+} nld_config;
+
+/* Create a context on the current CUDA device.  `cuda_stream` is a cudaStream_t that every
+ * later call is ordered on; NULL makes the context create (and own) a non-blocking stream,
+ * which nld_stream() returns.  The stream must not be the legacy default stream (decode calls
+ * are captured into CUDA graphs on it).  Allocates weights, the
+ * paged KV pool (max_batch * ceil((max_seq+block_k+1)/64) pages per layer) and scratch.
+ * Ownership: the context owns all of it until nld_destroy. */
+nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out);
+
+/* Synchronise the stream and free everything the context owns.  Accepts NULL. */
+nld_status nld_destroy(nld_ctx* ctx);
+
+/* Copy and repack the weights.  `tensors` holds 2 + 9*n_layers pointers in this order:
+ *   embed [vocab+1, d_model],
+ *   per layer: attn_norm [d], wq [Hq*hd, d], wk [Hkv*hd, d], wv [Hkv*hd, d], wo [d, Hq*hd],
+ *              mlp_norm [d], wg [ffn, d], wu [ffn, d], wd [d, ffn],
+ *   final_norm [d], lm_head [vocab, d].
+ * Matrices are row-major [out, in]; element type is the config dtype (bf16 as raw 16-bit
+ * patterns).  `on_device` = 1 if the pointers are device addresses, 0 for host.  The norm
+ * gains are folded into the following projection (W * diag(g), rounded to the dtype).
+ * The caller may free its buffers when the call returns (the call synchronises). */
+nld_status nld_init_weights(nld_ctx* ctx, const void* const* tensors, int n_tensors, int on_device);
+
+/* Start `batch` sequences from prompts d_tokens [batch, prompt_len] (device, int32).  Runs
+ * causal forwards over positions 0..prompt_len-2 (writing those KV rows) and makes
+ * prompt[prompt_len-1] the pending token, so len = prompt_len-1.  Resets drafts and
+ * diffusion blocks.  1 <= batch <= max_batch, 1 <= prompt_len <= max_seq. */
+nld_status nld_prefill(nld_ctx* ctx, const int32_t* d_tokens, int batch, int prompt_len);
+
+/* One AR step: causal one-token forward over the pending tokens; writes KV row len, then
+ * len += 1 and the argmax (lowest id on ties) becomes the pending token, also written to
+ * d_tokens_out [batch]. */
+nld_status nld_ar_step(nld_ctx* ctx, int32_t* d_tokens_out);
+
+/* Draft + verify forwards of one linear self-speculation round, without committing.
+ *   draft:  [x_n, MASK x (k-1)] at positions n..n+k-1, one bidirectional block; the k rows'
+ *           argmaxes are the drafts d_1..d_k.
+ *   verify: [x_n, d_1..d_k] at n..n+k, strictly causal; KV rows n..n+k are written in place
+ *           at their final slots; argmaxes v_1..v_{k+1}.
+ * Follow with nld_kv_commit. */
+nld_status nld_selfspec_draft_verify(nld_ctx* ctx);
+
+/* Commit path of a round (after nld_selfspec_draft_verify).  Per sequence b, c_b tokens
+ * commit: with d_nrows == NULL, c_b = a_b + 1 where a_b is the number of leading i with
+ * d_i == v_i (greedy longest matching prefix, warp-ballot computed); otherwise
+ * c_b = d_nrows[b] (forced count, 1..k+1).  The committed tokens are d_1..d_{c-1}, v_c,
+ * written to d_tokens_out [batch, k+1] (row b holds c_b tokens then -1 padding) and c_b to
+ * d_ncommit_out [batch].  KV rows n..n+c_b-1 written by the verify forward are kept where
+ * they are (the rows are already contiguous after the prefix: no copy); len += c_b;
+ * pending = v_c. */
+nld_status nld_kv_commit(nld_ctx* ctx, const int32_t* d_nrows, int32_t* d_tokens_out,
+                         int32_t* d_ncommit_out);
+
+/* One full round: nld_selfspec_draft_verify then nld_kv_commit(d_force_ncommit, ...),
+ * replayed from one captured CUDA graph per batch size. d_force_ncommit may be NULL. */
+nld_status nld_selfspec_round(nld_ctx* ctx, int32_t* d_tokens_out, int32_t* d_ncommit_out,
+                              const int32_t* d_force_ncommit);
+
+/* One block-diffusion denoising step for every sequence (lockstep).  Forward over
+ * [x_n, b_1..b_{k-1}] (open slots hold the [MASK] id), one bidirectional block; row i gives
+ * argmax and confidence (largest softmax probability over the vocab) for slot b_{i+1}.
+ * Among open slots, those with confidence >= threshold commit; if none does, the most
+ * confident one commits (lowest slot on ties).  Outputs: d_block_out [batch, k] the block
+ * after this step (open slots = vocab), d_conf_out [batch, k], d_ncommit_out [batch] slots
+ * committed this step.  Synchronises the stream once to learn whether every block is
+ * complete; if so it launches the causal KV-fill forward over [x_n, b_1..b_{k-1}] (KV rows
+ * n..n+k-1), sets len += k, pending = b_k, reopens the blocks, and sets *h_filled_out = 1
+ * (else 0). */
+nld_status nld_diffuse_block_step(nld_ctx* ctx, float threshold, int32_t* d_block_out,
+                                  float* d_conf_out, int32_t* d_ncommit_out, int32_t* h_filled_out);
+
+/* Test hook: run the forward of `mode` (NLD_MODE_*) from the current state and write its
+ * logits [batch, m, vocab] fp32 to d_logits_out (m = 1, k, k+1, k).  Sequence state is not
+ * advanced; a DRAFT call stores its argmaxes as the drafts a later VERIFY call reads.  The
+ * decode calls above never materialise logits. */
+nld_status nld_debug_logits(nld_ctx* ctx, int mode, float* d_logits_out);
+
+/* Test hook: copy state out (any pointer may be NULL): lens [batch], pending [batch],
+ * drafts [batch, k], verify argmaxes [batch, k+1]. */
+nld_status nld_debug_state(nld_ctx* ctx, int32_t* d_lens_out, int32_t* d_pending_out,
+                           int32_t* d_draft_out, int32_t* d_verify_out);
+
+/* Synchronise the context stream and report the device error word (then clear it):
+ * NLD_OK, NLD_ERR_KV_FULL, NLD_ERR_TIMEOUT or NLD_ERR_DEVICE. */
+nld_status nld_sync(nld_ctx* ctx);
+
+/* The cudaStream_t every call of this context is ordered on (created by nld_create when it
+ * was given NULL). */
+void* nld_stream(nld_ctx* ctx);
+
+/* Text of the last failure on this context (static storage when ctx is NULL). */
+const char* nld_last_error(const nld_ctx* ctx);
+
+/*
+ * Stand-alone block-causal GQA attention over a paged bf16 KV cache (the attention step of
+ * the forwards above, exposed for the attention micro-workload).  Notes section 3.2 / r9-hu
+ * "Method": a query sees every cached key and the keys of its own and earlier blocks.
+ *   d_q        [batch, m, Hq, hd] bf16: queries at positions lens[b]..lens[b]+m-1.
+ *   d_kv_pool  [n_pages][2][Hkv][64][hd] bf16 (K then V per page); the rows of the m query
+ *              positions must already be in the pool.
+ *   d_page_table [batch, pages_per_seq] int32 page ids (< n_pages).
+ *   d_lens     [batch] int32 cached rows before the m query rows.
+ *   block_size queries are cut into blocks of block_size from lens[b]; 1 = causal.
+ *   max_len    host upper bound of lens[b] + m (sizes the KV split), <= pages_per_seq*64.
+ *   d_out      [batch, m, Hq, hd] bf16.
+ *   d_workspace / workspace_bytes: scratch of at least nld_attention_workspace_size() bytes,
+ *              owned by the caller, 16-byte aligned, zero-filled once before its first use
+ *              (it starts with per-group arrival counters that every call leaves at zero;
+ *              the rest holds split-KV partials).  Calls sharing a workspace must not
+ *              overlap on the GPU.
+ *   Pool rows that no query may see must still hold finite values (zero-fill the pool).
+ * Requires head_dim == 128, page size 64.  Stream-ordered on `cuda_stream`.
+ */
+size_t nld_attention_workspace_size(int batch, int m, int n_q_heads, int n_kv_heads,
+                                    int head_dim, int max_len);
+nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* d_page_table,
+                         int pages_per_seq, int n_pages, const int32_t* d_lens, int batch, int m,
+                         int n_q_heads, int n_kv_heads, int head_dim, int block_size, int max_len,
+                         void* d_out, void* d_workspace, size_t workspace_bytes,
+                         void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NLD_H */

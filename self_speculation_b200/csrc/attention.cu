@@ -1,0 +1,450 @@
+// Block-causal GQA attention over the paged KV cache.
+//
+// Mask (ranhao.site notes section 3.2, r9-hu digest "Method"): the m rows of a forward sit at
+// positions len..len+m-1 and are cut into blocks of `block_size` starting at len; a row sees
+// every cached key and every key of its own and earlier blocks: key j is visible to row p
+// iff j <= len + min(floor(p/bs)*bs + bs, m) - 1.  block_size 1 is strictly causal (verify,
+// AR, prefill, KV fill); block_size m is one bidirectional block (draft, diffusion).  The
+// mask is computed from these indices and never stored.
+//
+// Tensor-core path (bf16, head_dim 128): one CTA per (KV split, kv head, sequence x query
+// tile).  Its rows are the G = Hq/Hkv query heads of that kv head times up to QT positions
+// (row = position*G + head), 16 rows per warp, so K and V tiles are read once for all the
+// heads that share them.  K/V tiles of 64 keys (one page) are staged by TMA with 128-byte
+// swizzle in a 3-deep ring; S = Q K^T and O += P V run on mma.sync m16n8k16 (bf16 in, fp32
+// accumulate); the softmax is online in registers (exp2 domain) with quad shuffles.  When the
+// keys are split over several CTAs (flash decoding), each writes unnormalised partials and
+// the last CTA of the group (atomic counter) merges them in split order.
+#include "common.cuh"
+
+namespace nld {
+
+namespace {
+
+constexpr int kAttStages = 3;
+constexpr int kHalfTile = kPage * 64 * 2;        // 8 KB: 64 keys x 64 dims bf16
+constexpr int kKVTile = 2 * kHalfTile;           // 16 KB: 64 keys x 128 dims
+constexpr int kMaxAttWarps = 12;
+
+NLD_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+NLD_DEV void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+NLD_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+NLD_DEV uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// Byte offset of 16-byte chunk `c` (0..15) of `row` in a [rows][128 dims] bf16 tile stored as
+// two TMA boxes of 64 dims with 128-byte swizzle.
+NLD_DEV uint32_t kv_off(int row, int c) {
+  return static_cast<uint32_t>((c >> 3) * kHalfTile + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+
+NLD_DEV int vis_end_of(int len, int p, int bs, int m) {
+  const int blk0 = (p / bs) * bs;
+  return len + min(blk0 + bs, m) - 1;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
+    attn_mma_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kAttStages * kKVTile;
+  uint8_t* sQ = smem + 2 * kAttStages * kKVTile;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sQ + a.NW * 16 * 256);
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nthr = blockDim.x;
+  const int split = blockIdx.x;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z / a.q_tiles;
+  const int qt = blockIdx.z - b * a.q_tiles;
+
+  if (tid == 0) {
+    for (int i = 0; i < kAttStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmKV);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+
+  int len = a.lens[b];
+  const int p0 = qt * a.QT;
+  const int np = min(a.QT, a.m - p0);
+  if (len < 0 || len + a.m > a.pps * kPage) {   // keys must stay inside the page table row
+    if (tid == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
+    len = max(0, min(len, a.pps * kPage - a.m));
+  }
+  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m) + 1;
+  const int n_tiles = (kv_end + kPage - 1) / kPage;
+  const int per = (n_tiles + a.S - 1) / a.S;
+  const int t_lo = split * per;
+  const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
+  __syncthreads();
+
+  auto issue = [&](int i) {
+    const int stage = i % kAttStages;
+    const int kt = t_lo + i;
+    const int page = a.page_table[b * a.pps + kt];
+    const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
+    const int row0v = row0 + a.Hkv * kPage;
+    mbar_arrive_expect_tx(&full[stage], 2 * kKVTile);
+    tma_load_2d(sK + stage * kKVTile, &tmKV, &full[stage], 0, row0);
+    tma_load_2d(sK + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0);
+    tma_load_2d(sV + stage * kKVTile, &tmKV, &full[stage], 0, row0v);
+    tma_load_2d(sV + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0v);
+  };
+  if (tid == 0)
+    for (int i = 0; i < min(kAttStages, ntile); ++i) issue(i);
+
+  // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row)
+  const int rows_pad = a.NW * 16;
+  for (int e = tid; e < rows_pad * 16; e += nthr) {
+    const int r = e >> 4, c = e & 15;
+    const int p = r / a.G, gq = r - p * a.G;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < a.rows && p < np) {
+      const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
+      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.q) +
+                                 ((tok * a.Hq) + g * a.G + gq) * 128 + c * 8;
+      val = *reinterpret_cast<const uint4*>(src);
+    }
+    *reinterpret_cast<uint4*>(sQ + r * 256 + ((c ^ (r & 7)) << 4)) = val;
+  }
+  __syncthreads();
+
+  // Q fragments for the warp's 16 rows, all 8 k-steps of head_dim 128
+  uint32_t qf[8][4];
+  {
+    const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int c = 2 * kk + (lane >> 4);
+      ldsm_x4(smem_u32(sQ + r * 256 + ((c ^ (r & 7)) << 4)), qf[kk][0], qf[kk][1], qf[kk][2],
+              qf[kk][3]);
+    }
+  }
+  const int ra = warp * 16 + (lane >> 2);
+  const int rb = ra + 8;
+  auto row_vis = [&](int r) {
+    const int p = r / a.G;
+    if (r >= a.rows || p >= np) return -1;
+    return vis_end_of(len, p0 + p, a.block_size, a.m);
+  };
+  const int vis_a = row_vis(ra), vis_b = row_vis(rb);
+
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+  bool timed_out = false;
+
+  for (int i = 0; i < ntile; ++i) {
+    const int stage = i % kAttStages;
+    if (!mbar_wait(&full[stage], static_cast<uint32_t>(i / kAttStages) & 1u, 2000000000ull)) {
+      timed_out = true;
+    }
+    if (__syncthreads_or(timed_out)) {
+      set_err(a.err, NLD_DEVERR_TIMEOUT);
+      break;
+    }
+    const int j0 = (t_lo + i) * kPage;
+    const uint32_t kb = smem_u32(sK + stage * kKVTile);
+    const uint32_t vb = smem_u32(sV + stage * kKVTile);
+
+    float sc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+    for (int kk2 = 0; kk2 < 4; ++kk2) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int key = nt * 8 + (lane & 7);
+        const int c = 4 * kk2 + (lane >> 3);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + kv_off(key, c), b0, b1, b2, b3);
+        mma_bf16_16816(sc[nt], qf[2 * kk2], b0, b1);
+        mma_bf16_16816(sc[nt], qf[2 * kk2 + 1], b2, b3);
+      }
+    }
+    // scale, mask, online softmax (log2 domain)
+    float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int key = j0 + nt * 8 + 2 * (lane & 3);
+#pragma unroll
+      for (int e2 = 0; e2 < 2; ++e2) {
+        float s0 = sc[nt][e2] * a.scale_log2;
+        float s1 = sc[nt][2 + e2] * a.scale_log2;
+        if (key + e2 > vis_a) s0 = -INFINITY;
+        if (key + e2 > vis_b) s1 = -INFINITY;
+        sc[nt][e2] = s0;
+        sc[nt][2 + e2] = s1;
+        mx_a = fmaxf(mx_a, s0);
+        mx_b = fmaxf(mx_b, s1);
+      }
+    }
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+    const float base_a = (mn_a == -INFINITY) ? 0.f : mn_a;
+    const float base_b = (mn_b == -INFINITY) ? 0.f : mn_b;
+    const float al_a = exp2f(m_a - base_a), al_b = exp2f(m_b - base_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      sc[nt][0] = exp2f(sc[nt][0] - base_a);
+      sc[nt][1] = exp2f(sc[nt][1] - base_a);
+      sc[nt][2] = exp2f(sc[nt][2] - base_b);
+      sc[nt][3] = exp2f(sc[nt][3] - base_b);
+      ps_a += sc[nt][0] + sc[nt][1];
+      ps_b += sc[nt][2] + sc[nt][3];
+    }
+    l_a = l_a * al_a + ps_a;
+    l_b = l_b * al_b + ps_b;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= al_a;
+      o[n][1] *= al_a;
+      o[n][2] *= al_b;
+      o[n][3] *= al_b;
+    }
+    // O += P V
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(sc[2 * j][0], sc[2 * j][1]);
+      pa[1] = pack_bf16(sc[2 * j][2], sc[2 * j][3]);
+      pa[2] = pack_bf16(sc[2 * j + 1][0], sc[2 * j + 1][1]);
+      pa[3] = pack_bf16(sc[2 * j + 1][2], sc[2 * j + 1][3]);
+      const int key = 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const int c = 2 * p + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + kv_off(key, c), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * p], pa, b0, b1);
+        mma_bf16_16816(o[2 * p + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && i + kAttStages < ntile) issue(i + kAttStages);
+  }
+
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+
+  auto out_ptr = [&](int r) -> __nv_bfloat16* {
+    const int p = r / a.G, gq = r - p * a.G;
+    const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
+    return static_cast<__nv_bfloat16*>(a.out) + ((tok * a.Hq) + g * a.G + gq) * 128;
+  };
+
+  if (a.S == 1) {
+    const float ia = (l_a > 0.f) ? 1.f / l_a : 0.f, ib = (l_b > 0.f) ? 1.f / l_b : 0.f;
+    if (vis_a >= 0) {
+      __nv_bfloat16* dst = out_ptr(ra);
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * (lane & 3)) = pack_bf16(o[n][0] * ia, o[n][1] * ia);
+    }
+    if (vis_b >= 0) {
+      __nv_bfloat16* dst = out_ptr(rb);
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * (lane & 3)) = pack_bf16(o[n][2] * ib, o[n][3] * ib);
+    }
+    return;
+  }
+
+  // split keys: write the unnormalised partial, the last CTA of the group merges
+  const int unit = blockIdx.z * a.Hkv + g;
+  const size_t base = (static_cast<size_t>(unit) * a.S + split) * rows_pad;
+  {
+    float* wo_a = a.ws_o + (base + ra) * 128;
+    float* wo_b = a.ws_o + (base + rb) * 128;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      *reinterpret_cast<float2*>(wo_a + n * 8 + 2 * (lane & 3)) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(wo_b + n * 8 + 2 * (lane & 3)) = make_float2(o[n][2], o[n][3]);
+    }
+    if ((lane & 3) == 0) {
+      *reinterpret_cast<float2*>(a.ws_ml + (base + ra) * 2) = make_float2(m_a, l_a);
+      *reinterpret_cast<float2*>(a.ws_ml + (base + rb) * 2) = make_float2(m_b, l_b);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int old = atomicAdd(&a.counters[unit], 1);
+    s_last = (old == a.S - 1) ? 1 : 0;
+    if (s_last) a.counters[unit] = 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const size_t base0 = static_cast<size_t>(unit) * a.S * rows_pad;
+  for (int e = tid; e < a.rows * 32; e += nthr) {
+    const int r = e >> 5, d4 = e & 31;
+    const int p = r / a.G;
+    if (p >= np) continue;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < a.S; ++s2)
+      M = fmaxf(M, __ldcg(a.ws_ml + (base0 + static_cast<size_t>(s2) * rows_pad + r) * 2));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s2 = 0; s2 < a.S; ++s2) {
+      const size_t rr = base0 + static_cast<size_t>(s2) * rows_pad + r;
+      const float ms = __ldcg(a.ws_ml + rr * 2);
+      if (ms == -INFINITY) continue;
+      const float w = exp2f(ms - M);
+      L += w * __ldcg(a.ws_ml + rr * 2 + 1);
+      const float4 ov = __ldcg(reinterpret_cast<const float4*>(a.ws_o + rr * 128) + d4);
+      acc.x += w * ov.x;
+      acc.y += w * ov.y;
+      acc.z += w * ov.z;
+      acc.w += w * ov.w;
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    __nv_bfloat16* dst = out_ptr(r) + d4 * 4;
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc.x * inv, acc.y * inv);
+    *reinterpret_cast<uint32_t*>(dst + 2) = pack_bf16(acc.z * inv, acc.w * inv);
+  }
+}
+
+// Plain per-(token, head) attention for any head_dim <= 128 and either storage type; used by
+// the fp32 configuration.  Scores go to shared memory (max_kv floats), two-pass softmax.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
+  extern __shared__ float sm[];
+  float* sq = sm;             // [hd]
+  float* sc = sm + 128;       // [max_kv]
+  __shared__ float red[4];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int tok = blockIdx.x, head = blockIdx.y;
+  const int b = tok / a.m, i = tok - b * a.m;
+  const int g = head / a.G;
+  int len = a.lens[b];
+  if (len < 0 || len + a.m > a.pps * kPage) {
+    if (threadIdx.x == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
+    len = max(0, min(len, a.pps * kPage - a.m));
+  }
+  const int nkeys = vis_end_of(len, i, a.block_size, a.m) + 1;
+  const T* q = static_cast<const T*>(a.q) + (static_cast<size_t>(tok) * a.Hq + head) * a.hd;
+  for (int d = threadIdx.x; d < a.hd; d += blockDim.x) sq[d] = to_f32<T>(q[d]);
+  __syncthreads();
+  const T* pool = static_cast<const T*>(a.pool);
+  const float scale = rsqrtf(static_cast<float>(a.hd));
+  for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+    const int page = a.page_table[b * a.pps + (j >> 6)];
+    const T* kr = pool + ((static_cast<size_t>(page) * 2) * a.Hkv + g) * kPage * a.hd +
+                  static_cast<size_t>(j & 63) * a.hd;
+    float acc = 0.f;
+    for (int d = 0; d < a.hd; ++d) acc += sq[d] * to_f32<T>(kr[d]);
+    sc[j] = acc * scale;
+  }
+  __syncthreads();
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j < nkeys; j += blockDim.x) mx = fmaxf(mx, sc[j]);
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+    const float p = expf(sc[j] - mx);
+    sc[j] = p;
+    sum += p;
+  }
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  sum = ((red[0] + red[1]) + red[2]) + red[3];
+  const float inv = 1.f / sum;
+  T* out = static_cast<T*>(a.out) + (static_cast<size_t>(tok) * a.Hq + head) * a.hd;
+  for (int d = threadIdx.x; d < a.hd; d += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < nkeys; ++j) {
+      const int page = a.page_table[b * a.pps + (j >> 6)];
+      const T* vr = pool + ((static_cast<size_t>(page) * 2 + 1) * a.Hkv + g) * kPage * a.hd +
+                    static_cast<size_t>(j & 63) * a.hd;
+      acc += sc[j] * to_f32<T>(vr[d]);
+    }
+    out[d] = from_f32<T>(acc * inv);
+  }
+}
+
+cudaError_t gemm_tc_init_attributes();
+
+// Shared-memory opt-ins of the large-smem kernels (host, once per process and device).
+cudaError_t init_kernel_attributes() {
+  cudaError_t e = gemm_tc_init_attributes();
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              227 * 1024);
+}
+
+size_t attn_mma_smem_bytes(int NW) {
+  return 1024 + 2 * kAttStages * kKVTile + static_cast<size_t>(NW) * 16 * 256 +
+         kAttStages * sizeof(uint64_t);
+}
+
+cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
+                                 int batch, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
+  cfg.blockDim = dim3(32 * a.NW);
+  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel, *tmKV, a);
+}
+
+cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,
+                                  int max_kv, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch * a.m, a.Hq);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = (128 + static_cast<size_t>(max_kv)) * sizeof(float);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (f32) return cudaLaunchKernelEx(&cfg, attn_simt_kernel<float>, a);
+  return cudaLaunchKernelEx(&cfg, attn_simt_kernel<__nv_bfloat16>, a);
+}
+
+}  // namespace nld

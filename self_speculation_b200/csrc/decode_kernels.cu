@@ -1,0 +1,282 @@
+// Per-forward small kernels: embedding gather (builds each mode's input block on the device),
+// the finalize step after the LM head (argmax/confidence combine over vocab tiles and the
+// mode's state update: drafts, AR commit, greedy acceptance, diffusion commit, KV-fill and
+// prefill bookkeeping), weight repacking and fills.
+#include <climits>
+
+#include "common.cuh"
+
+namespace nld {
+
+// ------------------------------------------------------------------------------ embedding --
+// Input block of each forward (shifted prediction; the pending token x_n sits at position n):
+//   AR      [x_n]                         DRAFT   [x_n, MASK x (k-1)]
+//   VERIFY  [x_n, d_1..d_k]               DIFFUSE / FILL [x_n, b_1..b_{k-1}]
+//   PREFILL prompt[chunk0 .. chunk0+m-1]
+// h = E[token] (fp32 residual), hb = the GEMM operand copy, and per 128-column tile the sum of
+// squares of h (the RMSNorm statistics the next GEMM epilogue turns into 1/rms).
+template <typename T>
+__global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = blockIdx.x;
+  const int b = t / a.m, i = t - b * a.m;
+  int id;
+  switch (a.mode) {
+    case FWD_PREFILL: id = a.prompt[static_cast<size_t>(b) * a.prompt_len + a.chunk0 + i]; break;
+    case FWD_AR: id = a.pending[b]; break;
+    case FWD_DRAFT: id = (i == 0) ? a.pending[b] : a.V; break;
+    case FWD_VERIFY: id = (i == 0) ? a.pending[b] : a.draft[b * a.k + i - 1]; break;
+    default: id = (i == 0) ? a.pending[b] : a.blk[b * a.k + i - 1]; break;
+  }
+  if (id < 0 || id > a.V) {
+    set_err(a.err, NLD_DEVERR_TOKEN);
+    id = 0;
+  }
+  const T* row = static_cast<const T*>(a.E) + static_cast<size_t>(id) * a.d;
+  float* h = a.h + static_cast<size_t>(t) * a.d;
+  T* hb = static_cast<T*>(a.hb) + static_cast<size_t>(t) * a.d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = a.d / kTileRows;
+  for (int tile = warp; tile < ntiles; tile += 8) {
+    float sq = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = tile * kTileRows + lane * 4 + q;
+      const float v = to_f32<T>(row[c]);
+      h[c] = v;
+      hb[c] = row[c];
+      sq += v * v;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if (lane == 0) a.ssq[static_cast<size_t>(tile) * a.ssq_ld + t] = sq;
+  }
+}
+
+cudaError_t launch_embed(cudaStream_t st, const EmbedArgs& a, int M, bool bf16, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (bf16) return cudaLaunchKernelEx(&cfg, embed_kernel<__nv_bfloat16>, a);
+  return cudaLaunchKernelEx(&cfg, embed_kernel<float>, a);
+}
+
+// ------------------------------------------------------------------------------- finalize --
+// One CTA per sequence.  For forwards with an LM head, warp w combines rows w, w+8, ... over
+// all vocab tiles: global max (lowest id on ties) and sum_t se_t * exp(mx_t - max), whose
+// inverse is the largest softmax probability (the confidence).
+__global__ void __launch_bounds__(256) finalize_kernel(const FinalizeArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ int s_arg[64];
+  __shared__ float s_conf[64];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool lm = (a.mode == FWD_AR || a.mode == FWD_DRAFT || a.mode == FWD_VERIFY ||
+                   a.mode == FWD_DIFFUSE);
+  if (lm) {
+    for (int i = warp; i < a.m; i += 8) {
+      const LmPart* row = a.lm_part + static_cast<size_t>(b * a.m + i) * a.lm_tiles;
+      float mx = -INFINITY;
+      int ix = INT_MAX;
+      for (int t = lane; t < a.lm_tiles; t += 32) {
+        const LmPart p = row[t];
+        if (p.mx > mx || (p.mx == mx && p.idx < ix)) {
+          mx = p.mx;
+          ix = p.idx;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float om = __shfl_xor_sync(0xffffffffu, mx, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, ix, off);
+        if (om > mx || (om == mx && oi < ix)) {
+          mx = om;
+          ix = oi;
+        }
+      }
+      float se = 0.f;
+      for (int t = lane; t < a.lm_tiles; t += 32) {
+        const LmPart p = row[t];
+        se += p.se * expf(p.mx - mx);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
+      if (lane == 0) {
+        s_arg[i] = ix;
+        s_conf[i] = 1.0f / se;
+      }
+    }
+    __syncthreads();
+  }
+  if (warp != 0) return;
+  const int k = a.k;
+  switch (a.mode) {
+    case FWD_AR: {
+      if (lane == 0) {
+        const int tok = s_arg[0];
+        if (a.commit) {
+          a.pending[b] = tok;
+          a.lens[b] += 1;
+          if (a.tokens_out) a.tokens_out[b] = tok;
+        }
+      }
+    } break;
+    case FWD_DRAFT: {
+      for (int i = lane; i < k; i += 32) a.draft[b * k + i] = s_arg[i];
+    } break;
+    case FWD_VERIFY: {
+      for (int i = lane; i < k + 1; i += 32) a.verify[b * (k + 1) + i] = s_arg[i];
+    } break;
+    case FWD_COMMIT: {
+      // greedy longest matching prefix: a = index of the first mismatch among d_i == v_i
+      const bool match = (lane < k) ? (a.draft[b * k + lane] == a.verify[b * (k + 1) + lane]) : true;
+      const unsigned bal = __ballot_sync(0xffffffffu, match);
+      int acc = (bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1);
+      acc = min(acc, k);
+      int c = acc + 1;
+      if (a.force) {
+        c = a.force[b];
+        if (c < 1 || c > k + 1) {
+          if (lane == 0) set_err(a.err, NLD_DEVERR_TOKEN);
+          c = max(1, min(c, k + 1));
+        }
+      }
+      for (int j = lane; j < k + 1; j += 32) {
+        int v;
+        if (j < c - 1) v = a.draft[b * k + j];
+        else if (j == c - 1) v = a.verify[b * (k + 1) + j];
+        else v = -1;
+        if (a.tokens_out) a.tokens_out[b * (k + 1) + j] = v;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (a.ncommit_out) a.ncommit_out[b] = c;
+        a.lens[b] += c;
+        a.pending[b] = a.verify[b * (k + 1) + c - 1];
+      }
+    } break;
+    case FWD_DIFFUSE: {
+      // confidence-threshold commit among open slots; at least one (the most confident)
+      const bool valid = lane < k;
+      const int cur = valid ? a.blk[b * k + lane] : 0;
+      const bool masked = valid && (cur == a.V);
+      const float conf = valid ? s_conf[lane] : 0.f;
+      const int tok = valid ? s_arg[lane] : 0;
+      bool pick = masked && (conf >= a.threshold);
+      const unsigned any_pick = __ballot_sync(0xffffffffu, pick);
+      const unsigned any_mask = __ballot_sync(0xffffffffu, masked);
+      if (any_pick == 0u && any_mask != 0u) {
+        float best = masked ? conf : -1.f;
+        int bi = masked ? lane : 64;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ob > best || (ob == best && oi < bi)) {
+            best = ob;
+            bi = oi;
+          }
+        }
+        pick = (lane == bi);
+      }
+      const unsigned picked = __ballot_sync(0xffffffffu, pick);
+      const unsigned still_open = __ballot_sync(0xffffffffu, masked && !pick);
+      const int nb = pick ? tok : cur;
+      if (valid) {
+        if (a.commit) a.blk[b * k + lane] = nb;
+        if (a.conf_out) a.conf_out[b * k + lane] = conf;
+        if (a.block_out) a.block_out[b * k + lane] = nb;
+      }
+      if (lane == 0) {
+        if (a.ncommit_out) a.ncommit_out[b] = __popc(picked);
+        if (a.commit && still_open != 0u && a.incomplete) atomicAdd(a.incomplete, 1);
+      }
+    } break;
+    case FWD_FILL: {
+      const int last = a.blk[b * k + k - 1];
+      __syncwarp();
+      for (int i = lane; i < k; i += 32) a.blk[b * k + i] = a.V;
+      if (lane == 0) {
+        a.lens[b] += k;
+        a.pending[b] = last;
+      }
+    } break;
+    case FWD_PREFILL: {
+      if (lane == 0) {
+        a.lens[b] += a.chunk;
+        if (a.prompt) a.pending[b] = a.prompt[static_cast<size_t>(b) * a.prompt_len + a.prompt_len - 1];
+      }
+    } break;
+    default:
+      break;
+  }
+}
+
+cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, finalize_kernel, a);
+}
+
+// -------------------------------------------------------------------------------- repack --
+// dst[r, c] = src[row_map[r], c] * gamma[c]  (gamma: RMSNorm gain folded into the projection
+// that follows the norm).
+template <typename T>
+__global__ void repack_kernel(T* __restrict__ dst, const T* __restrict__ src,
+                              const int* __restrict__ row_map, int n_rows, int K,
+                              const T* __restrict__ gamma) {
+  const size_t total = static_cast<size_t>(n_rows) * K;
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(idx / K);
+    const int c = static_cast<int>(idx - static_cast<size_t>(r) * K);
+    const int sr = row_map ? row_map[r] : r;
+    float v = to_f32<T>(src[static_cast<size_t>(sr) * K + c]);
+    if (gamma) v *= to_f32<T>(gamma[c]);
+    dst[idx] = from_f32<T>(v);
+  }
+}
+
+cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
+                          int n_rows, int K, const void* gamma, bool bf16) {
+  const int threads = 256;
+  const size_t total = static_cast<size_t>(n_rows) * K;
+  const int blocks = static_cast<int>(std::min<size_t>((total + threads - 1) / threads, 65536));
+  if (bf16)
+    repack_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+        static_cast<__nv_bfloat16*>(dst), static_cast<const __nv_bfloat16*>(src), row_map, n_rows,
+        K, static_cast<const __nv_bfloat16*>(gamma));
+  else
+    repack_kernel<float><<<blocks, threads, 0, st>>>(static_cast<float*>(dst),
+                                                     static_cast<const float*>(src), row_map,
+                                                     n_rows, K, static_cast<const float*>(gamma));
+  return cudaGetLastError();
+}
+
+__global__ void fill_i32_kernel(int* p, int value, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = value;
+}
+
+cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n) {
+  if (n <= 0) return cudaSuccess;
+  fill_i32_kernel<<<(n + 255) / 256, 256, 0, st>>>(p, value, n);
+  return cudaGetLastError();
+}
+
+}  // namespace nld

@@ -1,0 +1,197 @@
+// Fused epilogues of the projection GEMMs.  One thread owns one weight row (one output
+// feature) of a 128-row tile and 16 token columns of the accumulator.  The weight rows are
+// stored so that the two values an epilogue pairs sit in adjacent rows (lanes l and l^1):
+//   q/k rows of a head: row 2i = feature i, row 2i+1 = feature i + hd/2 (RoPE rotate-half
+//                       pairs; notes section 5 model: Llama-style RoPE);
+//   gate/up tile t:     row 2i = gate feature 64t+i, row 2i+1 = up feature 64t+i (SwiGLU).
+// so a single __shfl_xor(.., 1) brings the partner value.
+#pragma once
+
+#include "common.cuh"
+
+namespace nld {
+
+// red_f / red_i: shared scratch of at least 4*16 + 16 entries each.
+template <typename T>
+NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane, int ew,
+                       int tok0, const float* s_inv, int col0, float (&v)[16], float* red_f,
+                       int* red_i) {
+  const int row = row_tile * kTileRows + row_in_tile;
+  switch (e.kind) {
+    case EPI_QKV: {
+      const int qd = e.Hq * e.hd, kvd = e.Hkv * e.hd;
+      int sec, base;
+      if (row < qd) {
+        sec = 0; base = 0;
+      } else if (row < qd + kvd) {
+        sec = 1; base = qd;
+      } else {
+        sec = 2; base = qd + kvd;
+      }
+      const int rr = row - base;
+      const int head = rr / e.hd;
+      const int lr = rr - head * e.hd;
+      const int half = e.hd >> 1;
+      const int feat = (sec == 2) ? lr : ((lr & 1) ? (lr >> 1) + half : (lr >> 1));
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + j;
+        float x = v[j] * s_inv[col0 + j];
+        const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
+        if (tok >= e.M || row >= e.n_rows) continue;
+        const int b = tok / e.m;
+        const int pos = e.lens[b] + (tok - b * e.m);
+        if (pos >= e.kv_cap) {
+          set_err(e.err, NLD_DEVERR_KV_OVERFLOW);
+          continue;
+        }
+        if (sec < 2) {
+          const float2 cs = e.rope[static_cast<size_t>(pos) * half + (lr >> 1)];
+          x = (lr & 1) ? (x * cs.x + partner * cs.y) : (x * cs.x - partner * cs.y);
+        }
+        if (sec == 0) {
+          static_cast<T*>(e.q_out)[(static_cast<size_t>(tok) * e.Hq + head) * e.hd + feat] =
+              from_f32<T>(x);
+        } else {
+          const int page = e.page_table[b * e.pps + (pos >> 6)];
+          const size_t off =
+              ((static_cast<size_t>(page) * 2 + (sec - 1)) * e.Hkv + head) * kPage * e.hd +
+              static_cast<size_t>(pos & (kPage - 1)) * e.hd + feat;
+          static_cast<T*>(e.kv_layer)[off] = from_f32<T>(x);
+        }
+      }
+    } break;
+
+    case EPI_RESID: {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + j;
+        float hn = 0.f;
+        if (tok < e.M) {
+          float* hp = e.h + static_cast<size_t>(tok) * e.d + row;
+          hn = *hp + v[j];
+          *hp = hn;
+          static_cast<T*>(e.hb)[static_cast<size_t>(tok) * e.d + row] = from_f32<T>(hn);
+        }
+        float sq = hn * hn;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) red_f[ew * 16 + j] = sq;
+      }
+      named_bar_sync(1, 128);
+      if (row_in_tile < 16) {
+        const int j = row_in_tile;
+        const int tok = tok0 + j;
+        if (tok < e.M) {
+          const float s = ((red_f[j] + red_f[16 + j]) + red_f[32 + j]) + red_f[48 + j];
+          e.ssq_out[static_cast<size_t>(row_tile) * e.ssq_ld + tok] = s;
+        }
+      }
+      named_bar_sync(1, 128);
+    } break;
+
+    case EPI_SWIGLU: {
+      const int f = row_tile * (kTileRows / 2) + (row_in_tile >> 1);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + j;
+        const float x = v[j] * s_inv[col0 + j];
+        const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
+        if (tok < e.M && !(lane & 1)) {
+          const float g = x, u = partner;
+          const float act = g / (1.0f + expf(-g)) * u;
+          static_cast<T*>(e.u_out)[static_cast<size_t>(tok) * e.F + f] = from_f32<T>(act);
+        }
+      }
+    } break;
+
+    case EPI_LOGITS: {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + j;
+        if (tok < e.M && row < e.V)
+          e.logits[static_cast<size_t>(tok) * e.V + row] = v[j] * s_inv[col0 + j];
+      }
+    } break;
+
+    case EPI_LMHEAD: {
+      // pass 1: per column max and lowest argmax over the tile's 128 rows
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float l = (row < e.V) ? v[j] * s_inv[col0 + j] : -INFINITY;
+        v[j] = l;
+        float mx = l;
+        int ix = row;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float omx = __shfl_xor_sync(0xffffffffu, mx, off);
+          const int oix = __shfl_xor_sync(0xffffffffu, ix, off);
+          if (omx > mx || (omx == mx && oix < ix)) {
+            mx = omx;
+            ix = oix;
+          }
+        }
+        if (lane == 0) {
+          red_f[ew * 16 + j] = mx;
+          red_i[ew * 16 + j] = ix;
+        }
+      }
+      named_bar_sync(1, 128);
+      if (row_in_tile < 16) {
+        const int j = row_in_tile;
+        float mx = red_f[j];
+        int ix = red_i[j];
+#pragma unroll
+        for (int w = 1; w < 4; ++w) {
+          const float o = red_f[w * 16 + j];
+          if (o > mx) {   // earlier warps hold lower rows: strict > keeps the lowest index
+            mx = o;
+            ix = red_i[w * 16 + j];
+          }
+        }
+        red_f[64 + j] = mx;
+        red_i[64 + j] = ix;
+      }
+      named_bar_sync(1, 128);
+      // pass 2: sum over the tile of exp(l - tile max)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float mx = red_f[64 + j];
+        float s = (v[j] == -INFINITY) ? 0.f : expf(v[j] - mx);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) red_f[ew * 16 + j] = s;
+      }
+      named_bar_sync(1, 128);
+      if (row_in_tile < 16) {
+        const int j = row_in_tile;
+        const int tok = tok0 + j;
+        if (tok < e.M) {
+          LmPart p;
+          p.mx = red_f[64 + j];
+          p.se = ((red_f[j] + red_f[16 + j]) + red_f[32 + j]) + red_f[48 + j];
+          p.idx = red_i[64 + j];
+          p.pad = 0;
+          e.lm_part[static_cast<size_t>(tok) * e.lm_tiles + row_tile] = p;
+        }
+      }
+      named_bar_sync(1, 128);
+    } break;
+  }
+}
+
+// 1/rms for `n` token columns starting at tok0 into s_inv (threads et = 0..nthr-1 share it).
+NLD_DEV void compute_inv_rms(const EpiArgs& e, int tok0, int n, float* s_inv, int et, int nthr) {
+  for (int c = et; c < n; c += nthr) {
+    const int tok = tok0 + c;
+    float inv = 0.f;
+    if (tok < e.M) {
+      float acc = 0.f;
+      for (int t = 0; t < e.ssq_tiles; ++t) acc += e.ssq_in[static_cast<size_t>(t) * e.ssq_ld + tok];
+      inv = rsqrtf(acc * e.inv_d + e.eps);
+    }
+    s_inv[c] = inv;
+  }
+}
+
+}  // namespace nld

@@ -1,0 +1,1067 @@
+// C-ABI entry points and the host-side orchestration of a decode forward.
+//
+// A forward is: embedding gather -> per layer [QKV GEMM (+1/rms, RoPE, paged KV write),
+// attention, O GEMM (+residual), gate/up GEMM (+1/rms, SwiGLU), down GEMM (+residual)] ->
+// LM-head GEMM (+argmax/confidence partials) -> finalize (mode state update).  All kernels are
+// launched with programmatic dependent launch and each decode call is replayed from a CUDA
+// graph captured on first use, so the host crosses into the GPU once per call and lengths,
+// positions and tokens are read by the kernels from device memory (no host sync).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "nld_internal.h"
+
+using namespace nld;
+
+namespace nld {
+size_t gemm_tc_smem_bytes(const GemmShape& s);
+size_t attn_mma_smem_bytes(int NW);
+cudaError_t init_kernel_attributes();
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, inner] matrix, box [64 elements, box_rows],
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                   uint32_t box_rows) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+enum XBuf { XB_HB = 0, XB_ATTN = 1, XB_U = 2 };
+enum GemmWhich { GW_QKV = 0, GW_O = 1, GW_GU = 2, GW_D = 3, GW_LM = 4 };
+enum LmKind { LM_NONE = 0, LM_ARGMAX = 1, LM_LOGITS = 2 };
+
+std::string g_static_err;
+
+}  // namespace
+
+struct nld_ctx {
+  nld_config c{};
+  cudaStream_t stream = nullptr;
+  bool own_stream = false;
+  int dev = 0, sms = 148;
+  bool bf16 = true;
+  size_t el = 2;
+  int qd = 0, kvd = 0, qkv_rows = 0, gu_rows = 0, pps = 0, n_pages = 0, kv_cap = 0, M_max = 0;
+  int prefill_tokens = 2048;
+  std::vector<void*> allocs;
+  // weights (repacked)
+  void* embed = nullptr;
+  std::vector<void*> wqkv, wo, wgu, wd;
+  void* wlm = nullptr;
+  bool weights_ready = false;
+  // KV cache
+  void* pool = nullptr;
+  int* page_table = nullptr;
+  size_t layer_elems = 0;
+  // device state
+  int *lens = nullptr, *pending = nullptr, *draft = nullptr, *verify = nullptr, *blk = nullptr;
+  int *incomplete = nullptr, *err = nullptr, *prompt = nullptr;
+  // activations
+  float* h = nullptr;
+  void* hb = nullptr;
+  float* ssq = nullptr;
+  void* qbuf = nullptr;
+  void* attn = nullptr;
+  void* ubuf = nullptr;
+  LmPart* lm_part = nullptr;
+  int lm_tiles = 0;
+  float2* rope = nullptr;
+  // scratch
+  float* ws = nullptr;
+  int* counters = nullptr;
+  float* att_o = nullptr;
+  float* att_ml = nullptr;
+  int* att_counters = nullptr;
+  size_t att_o_floats = 0;
+  int att_units_max = 0;
+  int* h_pinned = nullptr;  // host: [0] error word, [1] incomplete, [2..] lens
+  // tensor maps
+  std::vector<CUtensorMap> tmWqkv, tmWo, tmWgu, tmWd;
+  CUtensorMap tmWlm{};
+  CUtensorMap tmKV{};
+  std::map<std::pair<int, int>, CUtensorMap> tmX;
+  // graphs
+  std::map<std::vector<uintptr_t>, cudaGraphExec_t> graphs;
+  // host-side sequence bookkeeping
+  int batch = 0;
+  bool started = false;
+  bool verify_fresh = false;
+  long long len_upper = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  std::string msg;
+};
+
+namespace {
+
+nld_status fail(nld_ctx* x, nld_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (x) x->msg = buf;
+  else g_static_err = buf;
+  return s;
+}
+
+#define CK(call)                                                                        \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(x, NLD_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                  __FILE__, __LINE__);                                                  \
+  } while (0)
+
+template <typename P>
+nld_status dalloc(nld_ctx* x, P** p, size_t bytes) {
+  void* q = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(&q, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(x, NLD_ERR_OOM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  x->allocs.push_back(q);
+  *p = static_cast<P*>(q);
+  return NLD_OK;
+}
+
+#define TRY(expr)                \
+  do {                           \
+    nld_status s_ = (expr);      \
+    if (s_ != NLD_OK) return s_; \
+  } while (0)
+
+nld_status validate(const nld_config* c, std::string& why) {
+  char b[256];
+  auto bad = [&](const char* m) {
+    why = m;
+    return NLD_ERR_ARG;
+  };
+  if (!c) return bad("config is NULL");
+  if (c->n_layers < 1 || c->d_model < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+      c->vocab < 2 || c->ffn_dim < 1 || c->max_batch < 1 || c->max_seq < 2)
+    return bad("non-positive dimension");
+  if (c->dtype != NLD_F32 && c->dtype != NLD_BF16) return bad("dtype must be NLD_F32 or NLD_BF16");
+  if (c->head_dim != 64 && c->head_dim != 128) return bad("head_dim must be 64 or 128");
+  if (c->dtype == NLD_BF16 && c->head_dim != 128) return bad("bf16 requires head_dim 128");
+  if (c->n_q_heads % c->n_kv_heads) return bad("n_q_heads must be a multiple of n_kv_heads");
+  if (c->d_model % 128) return bad("d_model must be a multiple of 128");
+  if (c->ffn_dim % 64) return bad("ffn_dim must be a multiple of 64");
+  if ((c->n_q_heads * c->head_dim) % 128) return bad("n_q_heads*head_dim must be a multiple of 128");
+  if ((c->n_kv_heads * c->head_dim) % 64) return bad("n_kv_heads*head_dim must be a multiple of 64");
+  if (c->page_size != kPage) return bad("page_size must be 64");
+  if (c->block_k < 1 || c->block_k > 32) return bad("block_k must be in 1..32");
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return bad("rms_eps > 0 and rope_theta > 1 required");
+  if (c->max_batch * (c->block_k + 1) > 65536) return bad("max_batch*(block_k+1) too large");
+  if (c->dtype == NLD_F32 && c->max_seq > 8192)
+    return bad("fp32 attention keeps a row of scores in shared memory: max_seq <= 8192");
+  (void)b;
+  return NLD_OK;
+}
+
+// ------------------------------------------------------------------------- GEMM dispatch --
+struct GemmPlan {
+  GemmShape s;
+};
+
+GemmShape plan_gemm(const nld_ctx* x, int n_rows, int K, int M) {
+  GemmShape s{};
+  s.n_rows = n_rows;
+  s.K = K;
+  s.M = M;
+  s.tok_tiles = (M + kMaxNT - 1) / kMaxNT;
+  int per = (M + s.tok_tiles - 1) / s.tok_tiles;
+  s.NT = std::max(16, (per + 15) / 16 * 16);
+  s.row_tiles = (n_rows + kTileRows - 1) / kTileRows;
+  s.KT = K / kTileK;
+  s.T = static_cast<long long>(s.row_tiles) * s.tok_tiles * s.KT;
+  s.G = static_cast<int>(std::min<long long>(x->sms, s.T));
+  const int stage_bytes = kTileRows * kTileK * 2 + s.NT * 128;
+  s.stages = std::max(2, std::min(8, (200 * 1024) / stage_bytes));
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(2 * s.NT)) cols <<= 1;
+  s.tmem_cols = cols;
+  s.ws_slot = kTileRows * s.NT;
+  return s;
+}
+
+const CUtensorMap* xmap(nld_ctx* x, int buf, int NT) {
+  auto key = std::make_pair(buf, NT);
+  auto it = x->tmX.find(key);
+  if (it != x->tmX.end()) return &it->second;
+  CUtensorMap m;
+  const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
+  const int inner = buf == XB_HB ? x->c.d_model : (buf == XB_ATTN ? x->qd : x->c.ffn_dim);
+  if (!make_map_bf16(&m, base, inner, x->M_max, NT)) return nullptr;
+  return &(x->tmX[key] = m);
+}
+
+nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool pdl) {
+  int n_rows, K, buf;
+  const void* W;
+  const CUtensorMap* tmW = nullptr;
+  switch (which) {
+    case GW_QKV: n_rows = x->qkv_rows; K = x->c.d_model; buf = XB_HB; W = x->wqkv[layer]; if (x->bf16) tmW = &x->tmWqkv[layer]; break;
+    case GW_O: n_rows = x->c.d_model; K = x->qd; buf = XB_ATTN; W = x->wo[layer]; if (x->bf16) tmW = &x->tmWo[layer]; break;
+    case GW_GU: n_rows = x->gu_rows; K = x->c.d_model; buf = XB_HB; W = x->wgu[layer]; if (x->bf16) tmW = &x->tmWgu[layer]; break;
+    case GW_D: n_rows = x->c.d_model; K = x->c.ffn_dim; buf = XB_U; W = x->wd[layer]; if (x->bf16) tmW = &x->tmWd[layer]; break;
+    default: n_rows = x->c.vocab; K = x->c.d_model; buf = XB_HB; W = x->wlm; if (x->bf16) tmW = &x->tmWlm; break;
+  }
+  EpiArgs ee = e;
+  ee.n_rows = n_rows;
+  if (!x->bf16) {
+    const void* X = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
+    CK(launch_gemm_simt(x->stream, static_cast<const float*>(W), static_cast<const float*>(X),
+                        n_rows, K, M, ee, pdl));
+    return NLD_OK;
+  }
+  GemmShape s = plan_gemm(x, n_rows, K, M);
+  const CUtensorMap* tmX = xmap(x, buf, s.NT);
+  if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
+  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->ws, x->counters, x->timeout_ns, pdl));
+  return NLD_OK;
+}
+
+void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a) {
+  a.G = Hq / Hkv;
+  a.QT = std::min(m, std::max(1, 144 / a.G));
+  a.q_tiles = (m + a.QT - 1) / a.QT;
+  a.rows = a.QT * a.G;
+  a.NW = (a.rows + 15) / 16;
+  const int units = batch * a.q_tiles * Hkv;
+  const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
+  a.S = 1;
+  if (units < 2 * sms) a.S = std::max(1, std::min(n_tiles, (2 * sms + units - 1) / units));
+}
+
+EpiArgs base_epi(nld_ctx* x, int M, int m) {
+  EpiArgs e{};
+  e.M = M;
+  e.m = m;
+  e.ssq_in = x->ssq;
+  e.ssq_tiles = x->c.d_model / kTileRows;
+  e.ssq_ld = x->M_max;
+  e.inv_d = 1.0f / static_cast<float>(x->c.d_model);
+  e.eps = x->c.rms_eps;
+  e.Hq = x->c.n_q_heads;
+  e.Hkv = x->c.n_kv_heads;
+  e.hd = x->c.head_dim;
+  e.page_table = x->page_table;
+  e.pps = x->pps;
+  e.lens = x->lens;
+  e.rope = x->rope;
+  e.kv_cap = x->kv_cap;
+  e.h = x->h;
+  e.hb = x->hb;
+  e.ssq_out = x->ssq;
+  e.d = x->c.d_model;
+  e.u_out = x->ubuf;
+  e.F = x->c.ffn_dim;
+  e.lm_part = x->lm_part;
+  e.lm_tiles = x->lm_tiles;
+  e.V = x->c.vocab;
+  e.q_out = x->qbuf;
+  e.err = x->err;
+  return e;
+}
+
+struct FwdSpec {
+  int mode;          // FwdMode of the embedding / finalize
+  int B, m, bs;      // sequences, rows per sequence, attention block size
+  int lm;            // LmKind
+  float* logits;     // LM_LOGITS target
+  int chunk0;        // prefill: first prompt position of this chunk
+  int prompt_len;
+  bool last_chunk;
+};
+
+// Launch one forward (no finalize).
+nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
+  const int M = f.B * f.m;
+  const bool pdl = true;
+  EmbedArgs ea{};
+  ea.E = x->embed;
+  ea.d = x->c.d_model;
+  ea.V = x->c.vocab;
+  ea.m = f.m;
+  ea.mode = f.mode;
+  ea.k = x->c.block_k;
+  ea.pending = x->pending;
+  ea.draft = x->draft;
+  ea.blk = x->blk;
+  ea.prompt = x->prompt;
+  ea.prompt_len = f.prompt_len;
+  ea.chunk0 = f.chunk0;
+  ea.lens = x->lens;
+  ea.h = x->h;
+  ea.hb = x->hb;
+  ea.ssq = x->ssq;
+  ea.ssq_ld = x->M_max;
+  ea.err = x->err;
+  CK(launch_embed(x->stream, ea, M, x->bf16, pdl));
+
+  const int max_len = static_cast<int>(std::min<long long>(x->kv_cap, x->len_upper + f.m));
+  AttnArgs aa{};
+  aa.q = x->qbuf;
+  aa.out = x->attn;
+  aa.m = f.m;
+  aa.Hq = x->c.n_q_heads;
+  aa.Hkv = x->c.n_kv_heads;
+  aa.hd = x->c.head_dim;
+  aa.lens = x->lens;
+  aa.page_table = x->page_table;
+  aa.pps = x->pps;
+  aa.block_size = f.bs;
+  aa.err = x->err;
+  aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
+  if (x->bf16) {
+    attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa);
+    const int units = f.B * aa.q_tiles * aa.Hkv;
+    if (aa.S > 1 && (units > x->att_units_max ||
+                     static_cast<size_t>(units) * aa.S * aa.NW * 16 * 128 > x->att_o_floats))
+      aa.S = 1;
+    aa.ws_o = x->att_o;
+    aa.ws_ml = x->att_ml;
+    aa.counters = x->att_counters;
+  } else {
+    aa.G = aa.Hq / aa.Hkv;
+  }
+
+  for (int l = 0; l < x->c.n_layers; ++l) {
+    EpiArgs e = base_epi(x, M, f.m);
+    e.kind = EPI_QKV;
+    e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
+    TRY(gemm(x, GW_QKV, l, M, e, pdl));
+    if (x->bf16) {
+      aa.layer_row0 = l * x->n_pages * 2 * x->c.n_kv_heads * kPage;
+      CK(launch_attention_mma(x->stream, &x->tmKV, aa, f.B, pdl));
+    } else {
+      aa.pool = e.kv_layer;
+      CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
+    }
+    e.kind = EPI_RESID;
+    TRY(gemm(x, GW_O, l, M, e, pdl));
+    e.kind = EPI_SWIGLU;
+    TRY(gemm(x, GW_GU, l, M, e, pdl));
+    e.kind = EPI_RESID;
+    TRY(gemm(x, GW_D, l, M, e, pdl));
+  }
+  if (f.lm != LM_NONE) {
+    EpiArgs e = base_epi(x, M, f.m);
+    e.kind = (f.lm == LM_LOGITS) ? EPI_LOGITS : EPI_LMHEAD;
+    e.logits = f.logits;
+    TRY(gemm(x, GW_LM, 0, M, e, pdl));
+  }
+  return NLD_OK;
+}
+
+FinalizeArgs base_fin(nld_ctx* x, int mode, int m) {
+  FinalizeArgs a{};
+  a.mode = mode;
+  a.m = m;
+  a.k = x->c.block_k;
+  a.V = x->c.vocab;
+  a.lm_tiles = x->lm_tiles;
+  a.lm_part = x->lm_part;
+  a.lens = x->lens;
+  a.pending = x->pending;
+  a.draft = x->draft;
+  a.verify = x->verify;
+  a.blk = x->blk;
+  a.incomplete = x->incomplete;
+  a.prompt = nullptr;
+  a.commit = 1;
+  a.kv_cap = x->kv_cap;
+  a.err = x->err;
+  return a;
+}
+
+nld_status finalize(nld_ctx* x, const FinalizeArgs& a) {
+  CK(launch_finalize(x->stream, a, x->batch, true));
+  return NLD_OK;
+}
+
+// Capture `body` into a graph keyed by `key` on first use, then replay it.
+template <typename F>
+nld_status run_graph(nld_ctx* x, const std::vector<uintptr_t>& key, F body) {
+  auto it = x->graphs.find(key);
+  if (it == x->graphs.end()) {
+    cudaGraph_t g = nullptr;
+    CK(cudaStreamBeginCapture(x->stream, cudaStreamCaptureModeThreadLocal));
+    nld_status s = body();
+    cudaError_t ce = cudaStreamEndCapture(x->stream, &g);
+    if (s != NLD_OK) {
+      if (g) cudaGraphDestroy(g);
+      cudaGetLastError();
+      return s;
+    }
+    if (ce != cudaSuccess) return fail(x, NLD_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ce));
+    cudaGraphExec_t ex = nullptr;
+    ce = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    if (ce != cudaSuccess) return fail(x, NLD_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(ce));
+    it = x->graphs.emplace(key, ex).first;
+  }
+  CK(cudaGraphLaunch(it->second, x->stream));
+  return NLD_OK;
+}
+
+// Make sure `grow` more committed rows fit; refresh the exact lengths from the device when
+// the host's upper bound says they might not.
+nld_status ensure_capacity(nld_ctx* x, long long grow) {
+  if (x->len_upper + grow <= x->c.max_seq) return NLD_OK;
+  CK(cudaMemcpyAsync(x->h_pinned + 2, x->lens, sizeof(int) * x->batch, cudaMemcpyDeviceToHost, x->stream));
+  CK(cudaStreamSynchronize(x->stream));
+  long long mx = 0;
+  for (int b = 0; b < x->batch; ++b) mx = std::max<long long>(mx, x->h_pinned[2 + b]);
+  x->len_upper = mx;
+  if (x->len_upper + grow > x->c.max_seq)
+    return fail(x, NLD_ERR_KV_FULL, "sequence length %lld + %lld would exceed max_seq %d", mx, grow,
+                x->c.max_seq);
+  return NLD_OK;
+}
+
+nld_status need_started(nld_ctx* x) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  if (!x->weights_ready) return fail(x, NLD_ERR_STATE, "weights not initialised");
+  if (!x->started) return fail(x, NLD_ERR_STATE, "no sequences: call nld_prefill first");
+  return NLD_OK;
+}
+
+}  // namespace
+
+// =================================================================================== API ===
+extern "C" {
+
+nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
+  if (!out) return fail(nullptr, NLD_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  std::string why;
+  if (validate(cfg, why) != NLD_OK) return fail(nullptr, NLD_ERR_ARG, "invalid config: %s", why.c_str());
+  nld_ctx* x = new nld_ctx();
+  x->c = *cfg;
+  const nld_config& c = x->c;
+  auto bail = [&](nld_status s) {
+    g_static_err = x->msg;
+    nld_destroy(x);
+    return s;
+  };
+  if (cudaGetDevice(&x->dev) != cudaSuccess) {
+    cudaGetLastError();
+    delete x;
+    return fail(nullptr, NLD_ERR_CUDA, "no CUDA device");
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, x->dev) != cudaSuccess) {
+    delete x;
+    return fail(nullptr, NLD_ERR_CUDA, "cudaGetDeviceProperties failed");
+  }
+  x->sms = prop.multiProcessorCount;
+  x->bf16 = (c.dtype == NLD_BF16);
+  if (x->bf16 && prop.major != 10) {
+    delete x;
+    return fail(nullptr, NLD_ERR_UNSUPPORTED, "bf16 kernels need an sm_100 GPU (found sm_%d%d)",
+                prop.major, prop.minor);
+  }
+  x->el = x->bf16 ? 2 : 4;
+  if (init_kernel_attributes() != cudaSuccess) {
+    cudaGetLastError();
+    delete x;
+    return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed");
+  }
+  if (cuda_stream) {
+    x->stream = static_cast<cudaStream_t>(cuda_stream);
+  } else {
+    if (cudaStreamCreateWithFlags(&x->stream, cudaStreamNonBlocking) != cudaSuccess) {
+      delete x;
+      return fail(nullptr, NLD_ERR_CUDA, "stream creation failed");
+    }
+    x->own_stream = true;
+  }
+  x->qd = c.n_q_heads * c.head_dim;
+  x->kvd = c.n_kv_heads * c.head_dim;
+  x->qkv_rows = x->qd + 2 * x->kvd;
+  x->gu_rows = 2 * c.ffn_dim;
+  x->pps = (c.max_seq + c.block_k + 1 + kPage - 1) / kPage;
+  x->kv_cap = x->pps * kPage;
+  x->n_pages = c.max_batch * x->pps;
+  x->prefill_tokens = 2048;
+  x->M_max = std::max(c.max_batch * (c.block_k + 1), x->prefill_tokens);
+  x->M_max = (x->M_max + 15) / 16 * 16;
+  x->lm_tiles = (c.vocab + kTileRows - 1) / kTileRows;
+  const size_t el = x->el;
+  const int d = c.d_model;
+
+  // KV pool [layer][page][2][Hkv][64][hd] and a page table that interleaves the sequences'
+  // pages (page j of sequence b is physical page j*max_batch + b), so kernels never rely on
+  // a sequence's pages being adjacent.
+  x->layer_elems = static_cast<size_t>(x->n_pages) * 2 * c.n_kv_heads * kPage * c.head_dim;
+  if (static_cast<long long>(c.n_layers) * x->n_pages * 2 * c.n_kv_heads * kPage > INT32_MAX)
+    return bail(fail(x, NLD_ERR_ARG, "KV pool too large for 32-bit TMA row coordinates"));
+  nld_status s;
+  if ((s = dalloc(x, &x->pool, x->layer_elems * c.n_layers * el)) != NLD_OK) return bail(s);
+  if (cudaMemsetAsync(x->pool, 0, x->layer_elems * c.n_layers * el, x->stream) != cudaSuccess)
+    return bail(fail(x, NLD_ERR_CUDA, "pool memset failed"));
+  {
+    std::vector<int> pt(static_cast<size_t>(c.max_batch) * x->pps);
+    for (int b = 0; b < c.max_batch; ++b)
+      for (int j = 0; j < x->pps; ++j) pt[static_cast<size_t>(b) * x->pps + j] = j * c.max_batch + b;
+    if ((s = dalloc(x, &x->page_table, pt.size() * sizeof(int))) != NLD_OK) return bail(s);
+    if (cudaMemcpy(x->page_table, pt.data(), pt.size() * sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(x, NLD_ERR_CUDA, "page table upload failed"));
+  }
+  // RoPE table [kv_cap][hd/2] of (cos, sin) of pos * theta^(-2i/hd), computed in double.
+  {
+    const int half = c.head_dim / 2;
+    std::vector<float2> tab(static_cast<size_t>(x->kv_cap) * half);
+    for (int p = 0; p < x->kv_cap; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double inv_freq = std::pow(static_cast<double>(c.rope_theta), -2.0 * i / c.head_dim);
+        const double ang = static_cast<double>(p) * inv_freq;
+        tab[static_cast<size_t>(p) * half + i] = make_float2(static_cast<float>(std::cos(ang)),
+                                                             static_cast<float>(std::sin(ang)));
+      }
+    if ((s = dalloc(x, &x->rope, tab.size() * sizeof(float2))) != NLD_OK) return bail(s);
+    if (cudaMemcpy(x->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(x, NLD_ERR_CUDA, "rope table upload failed"));
+  }
+  const int B = c.max_batch, k = c.block_k;
+  if ((s = dalloc(x, &x->lens, B * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->pending, B * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->draft, static_cast<size_t>(B) * k * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->verify, static_cast<size_t>(B) * (k + 1) * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->blk, static_cast<size_t>(B) * k * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->incomplete, 16)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->err, 16)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->prompt, static_cast<size_t>(B) * c.max_seq * sizeof(int))) != NLD_OK) return bail(s);
+  const size_t Mm = x->M_max;
+  if ((s = dalloc(x, &x->h, Mm * d * sizeof(float))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->hb, Mm * d * el)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->ssq, (d / kTileRows) * Mm * sizeof(float))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->qbuf, Mm * x->qd * el)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->attn, Mm * x->qd * el)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->ubuf, Mm * c.ffn_dim * el)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->lm_part, Mm * x->lm_tiles * sizeof(LmPart))) != NLD_OK) return bail(s);
+  // stream-K partial slots: two per CTA of at most 128 x 256 fp32
+  if ((s = dalloc(x, &x->ws, static_cast<size_t>(x->sms) * 2 * kTileRows * kMaxNT * sizeof(float))) != NLD_OK) return bail(s);
+  {
+    const int max_rows = std::max({x->qkv_rows, x->gu_rows, d, c.vocab});
+    const int n = ((max_rows + kTileRows - 1) / kTileRows) * ((x->M_max + kMaxNT - 1) / kMaxNT) + 64;
+    if ((s = dalloc(x, &x->counters, n * sizeof(int))) != NLD_OK) return bail(s);
+    if (cudaMemset(x->counters, 0, n * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  }
+  // attention split-KV partials: splits are only used while units*S <= ~2*SMs
+  x->att_units_max = 2 * x->sms;
+  x->att_o_floats = static_cast<size_t>(2 * x->sms + 64) * 12 * 16 * 128;
+  if ((s = dalloc(x, &x->att_o, x->att_o_floats * sizeof(float))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->att_ml, x->att_o_floats / 64 * sizeof(float))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->att_counters, x->att_units_max * sizeof(int))) != NLD_OK) return bail(s);
+  if (cudaMemset(x->att_counters, 0, x->att_units_max * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->err, 0, 16) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->lens, 0, B * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->h, 0, Mm * d * sizeof(float)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->hb, 0, Mm * d * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->attn, 0, Mm * x->qd * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->ubuf, 0, Mm * c.ffn_dim * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMallocHost(&x->h_pinned, (4 + B) * sizeof(int)) != cudaSuccess)
+    return bail(fail(x, NLD_ERR_OOM, "pinned host allocation failed"));
+  if (x->bf16) {
+    const uint64_t rows = static_cast<uint64_t>(c.n_layers) * x->n_pages * 2 * c.n_kv_heads * kPage;
+    if (!make_map_bf16(&x->tmKV, x->pool, c.head_dim, rows, kPage))
+      return bail(fail(x, NLD_ERR_CUDA, "tensor map encode failed (KV pool)"));
+  }
+  if (cudaStreamSynchronize(x->stream) != cudaSuccess)
+    return bail(fail(x, NLD_ERR_CUDA, "initialisation failed"));
+  *out = x;
+  return NLD_OK;
+}
+
+nld_status nld_destroy(nld_ctx* x) {
+  if (!x) return NLD_OK;
+  if (x->stream) cudaStreamSynchronize(x->stream);
+  for (auto& kv : x->graphs) cudaGraphExecDestroy(kv.second);
+  x->graphs.clear();
+  for (void* p : x->allocs) cudaFree(p);
+  x->allocs.clear();
+  if (x->h_pinned) cudaFreeHost(x->h_pinned);
+  if (x->own_stream && x->stream) cudaStreamDestroy(x->stream);
+  delete x;
+  return NLD_OK;
+}
+
+nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensors, int on_device) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  const nld_config& c = x->c;
+  const int L = c.n_layers;
+  if (!tensors || n_tensors != 2 + 9 * L)
+    return fail(x, NLD_ERR_ARG, "expected %d weight tensors, got %d", 2 + 9 * L, n_tensors);
+  for (int i = 0; i < n_tensors; ++i)
+    if (!tensors[i]) return fail(x, NLD_ERR_ARG, "weight tensor %d is NULL", i);
+  const size_t el = x->el;
+  const int d = c.d_model, F = c.ffn_dim, V = c.vocab, hd = c.head_dim;
+  if (x->weights_ready) return fail(x, NLD_ERR_STATE, "weights already initialised");
+  nld_status s;
+  // allocations
+  if ((s = dalloc(x, &x->embed, static_cast<size_t>(V + 1) * d * el)) != NLD_OK) return s;
+  x->wqkv.resize(L);
+  x->wo.resize(L);
+  x->wgu.resize(L);
+  x->wd.resize(L);
+  for (int l = 0; l < L; ++l) {
+    if ((s = dalloc(x, &x->wqkv[l], static_cast<size_t>(x->qkv_rows) * d * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wo[l], static_cast<size_t>(d) * x->qd * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wgu[l], static_cast<size_t>(x->gu_rows) * d * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wd[l], static_cast<size_t>(d) * F * el)) != NLD_OK) return s;
+  }
+  if ((s = dalloc(x, &x->wlm, static_cast<size_t>(V) * d * el)) != NLD_OK) return s;
+
+  // row maps: q/k heads interleave (i, i+hd/2); gate/up interleave per 64 features
+  std::vector<int> map_q(x->qd), map_kv(x->kvd), map_g(F), map_u(F);
+  for (int r = 0; r < x->qd; ++r) {
+    const int h = r / hd, lr = r % hd;
+    map_q[r] = h * hd + ((lr & 1) ? (lr >> 1) + hd / 2 : (lr >> 1));
+  }
+  for (int r = 0; r < x->kvd; ++r) {
+    const int h = r / hd, lr = r % hd;
+    map_kv[r] = h * hd + ((lr & 1) ? (lr >> 1) + hd / 2 : (lr >> 1));
+  }
+  int *d_map_q = nullptr, *d_map_kv = nullptr, *d_map_gu = nullptr;
+  std::vector<int> map_gu(2 * F);
+  // destination row 128t + 2i <- gate 64t+i ; 128t + 2i + 1 <- up 64t+i (sources concatenated
+  // as [Wg; Wu] in a staging buffer, so up rows are offset by F)
+  for (int t = 0; t < F / 64; ++t)
+    for (int i = 0; i < 64; ++i) {
+      map_gu[128 * t + 2 * i] = 64 * t + i;
+      map_gu[128 * t + 2 * i + 1] = F + 64 * t + i;
+    }
+  if ((s = dalloc(x, &d_map_q, x->qd * sizeof(int))) != NLD_OK) return s;
+  if ((s = dalloc(x, &d_map_kv, x->kvd * sizeof(int))) != NLD_OK) return s;
+  if ((s = dalloc(x, &d_map_gu, 2 * F * sizeof(int))) != NLD_OK) return s;
+  CK(cudaMemcpy(d_map_q, map_q.data(), x->qd * sizeof(int), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(d_map_kv, map_kv.data(), x->kvd * sizeof(int), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(d_map_gu, map_gu.data(), 2 * F * sizeof(int), cudaMemcpyHostToDevice));
+
+  // staging: the largest source (embed/lm head or [Wg;Wu]) plus one gain vector
+  size_t max_src = std::max({static_cast<size_t>(V + 1) * d, static_cast<size_t>(2) * F * d,
+                             static_cast<size_t>(x->qd) * d, static_cast<size_t>(d) * F});
+  void* stage = nullptr;
+  void* stage_g = nullptr;
+  if ((s = dalloc(x, &stage, max_src * el)) != NLD_OK) return s;
+  if ((s = dalloc(x, &stage_g, static_cast<size_t>(d) * el)) != NLD_OK) return s;
+  const cudaMemcpyKind kind = on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  auto up = [&](const void* src, size_t n, void* dst) -> nld_status {
+    CK(cudaMemcpyAsync(dst, src, n * el, kind, x->stream));
+    return NLD_OK;
+  };
+  // embedding: plain copy
+  TRY(up(tensors[0], static_cast<size_t>(V + 1) * d, x->embed));
+  for (int l = 0; l < L; ++l) {
+    const void* const* t = tensors + 1 + 9 * l;
+    TRY(up(t[0], d, stage_g));
+    char* qkv = static_cast<char*>(x->wqkv[l]);
+    TRY(up(t[1], static_cast<size_t>(x->qd) * d, stage));
+    CK(launch_repack(x->stream, qkv, stage, d_map_q, x->qd, d, stage_g, x->bf16));
+    TRY(up(t[2], static_cast<size_t>(x->kvd) * d, stage));
+    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd) * d * el, stage, d_map_kv, x->kvd, d, stage_g, x->bf16));
+    TRY(up(t[3], static_cast<size_t>(x->kvd) * d, stage));
+    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd + x->kvd) * d * el, stage, nullptr, x->kvd, d, stage_g, x->bf16));
+    TRY(up(t[4], static_cast<size_t>(d) * x->qd, x->wo[l]));
+    TRY(up(t[5], d, stage_g));
+    TRY(up(t[6], static_cast<size_t>(F) * d, stage));
+    TRY(up(t[7], static_cast<size_t>(F) * d, static_cast<char*>(stage) + static_cast<size_t>(F) * d * el));
+    CK(launch_repack(x->stream, x->wgu[l], stage, d_map_gu, 2 * F, d, stage_g, x->bf16));
+    TRY(up(t[8], static_cast<size_t>(d) * F, x->wd[l]));
+    CK(cudaStreamSynchronize(x->stream));   // staging reuse
+  }
+  TRY(up(tensors[1 + 9 * L], d, stage_g));
+  TRY(up(tensors[2 + 9 * L], static_cast<size_t>(V) * d, stage));
+  CK(launch_repack(x->stream, x->wlm, stage, nullptr, V, d, stage_g, x->bf16));
+  CK(cudaStreamSynchronize(x->stream));
+  // release staging (the last allocations)
+  for (void* p : {stage, stage_g, static_cast<void*>(d_map_q), static_cast<void*>(d_map_kv), static_cast<void*>(d_map_gu)}) {
+    cudaFree(p);
+    x->allocs.erase(std::remove(x->allocs.begin(), x->allocs.end(), p), x->allocs.end());
+  }
+  if (x->bf16) {
+    x->tmWqkv.resize(L);
+    x->tmWo.resize(L);
+    x->tmWgu.resize(L);
+    x->tmWd.resize(L);
+    bool ok = true;
+    for (int l = 0; l < L; ++l) {
+      ok &= make_map_bf16(&x->tmWqkv[l], x->wqkv[l], d, x->qkv_rows, kTileRows);
+      ok &= make_map_bf16(&x->tmWo[l], x->wo[l], x->qd, d, kTileRows);
+      ok &= make_map_bf16(&x->tmWgu[l], x->wgu[l], d, x->gu_rows, kTileRows);
+      ok &= make_map_bf16(&x->tmWd[l], x->wd[l], F, d, kTileRows);
+    }
+    ok &= make_map_bf16(&x->tmWlm, x->wlm, d, V, kTileRows);
+    if (!ok) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (weights)");
+  }
+  x->weights_ready = true;
+  return NLD_OK;
+}
+
+nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int prompt_len) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  if (!x->weights_ready) return fail(x, NLD_ERR_STATE, "weights not initialised");
+  if (!d_tokens) return fail(x, NLD_ERR_ARG, "tokens is NULL");
+  if (batch < 1 || batch > x->c.max_batch) return fail(x, NLD_ERR_ARG, "batch %d outside 1..%d", batch, x->c.max_batch);
+  if (prompt_len < 1 || prompt_len > x->c.max_seq) return fail(x, NLD_ERR_ARG, "prompt_len %d outside 1..%d", prompt_len, x->c.max_seq);
+  x->batch = batch;
+  const int k = x->c.block_k;
+  CK(cudaMemcpyAsync(x->prompt, d_tokens, static_cast<size_t>(batch) * prompt_len * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  CK(cudaMemsetAsync(x->lens, 0, batch * sizeof(int), x->stream));
+  CK(launch_fill_i32(x->stream, x->blk, x->c.vocab, batch * k));
+  CK(launch_fill_i32(x->stream, x->draft, x->c.vocab, batch * k));
+  CK(launch_fill_i32(x->stream, x->verify, -1, batch * (k + 1)));
+  x->len_upper = 0;
+  const int chunk = std::max(1, x->prefill_tokens / batch);
+  const int rows = prompt_len - 1;
+  int c0 = 0;
+  do {
+    const int m = std::min(chunk, rows - c0);
+    const bool last = (c0 + m >= rows);
+    if (m > 0) {
+      FwdSpec f{};
+      f.mode = FWD_PREFILL;
+      f.B = batch;
+      f.m = m;
+      f.bs = 1;
+      f.lm = LM_NONE;
+      f.chunk0 = c0;
+      f.prompt_len = prompt_len;
+      x->len_upper = c0;
+      TRY(launch_forward(x, f));
+    }
+    FinalizeArgs a = base_fin(x, FWD_PREFILL, std::max(m, 1));
+    a.chunk = m;
+    a.prompt = last ? x->prompt : nullptr;
+    a.prompt_len = prompt_len;
+    TRY(finalize(x, a));
+    c0 += m;
+    if (last) break;
+  } while (true);
+  x->len_upper = rows;
+  x->started = true;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+nld_status nld_ar_step(nld_ctx* x, int32_t* d_tokens_out) {
+  TRY(need_started(x));
+  TRY(ensure_capacity(x, 1));
+  std::vector<uintptr_t> key = {1, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_tokens_out)};
+  const long long saved = x->len_upper;
+  TRY(run_graph(x, key, [&]() -> nld_status {
+    FwdSpec f{};
+    f.mode = FWD_AR;
+    f.B = x->batch;
+    f.m = 1;
+    f.bs = 1;
+    f.lm = LM_ARGMAX;
+    x->len_upper = x->c.max_seq;   // graphs are sized for the longest sequence
+    nld_status s = launch_forward(x, f);
+    x->len_upper = saved;
+    if (s != NLD_OK) return s;
+    FinalizeArgs a = base_fin(x, FWD_AR, 1);
+    a.tokens_out = d_tokens_out;
+    return finalize(x, a);
+  }));
+  x->len_upper += 1;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+static nld_status draft_verify_body(nld_ctx* x) {
+  const int k = x->c.block_k;
+  const long long saved = x->len_upper;
+  x->len_upper = x->c.max_seq;
+  FwdSpec f{};
+  f.mode = FWD_DRAFT;
+  f.B = x->batch;
+  f.m = k;
+  f.bs = k;
+  f.lm = LM_ARGMAX;
+  nld_status s = launch_forward(x, f);
+  if (s == NLD_OK) s = finalize(x, base_fin(x, FWD_DRAFT, k));
+  if (s == NLD_OK) {
+    f.mode = FWD_VERIFY;
+    f.m = k + 1;
+    f.bs = 1;
+    s = launch_forward(x, f);
+  }
+  if (s == NLD_OK) s = finalize(x, base_fin(x, FWD_VERIFY, k + 1));
+  x->len_upper = saved;
+  return s;
+}
+
+nld_status nld_selfspec_draft_verify(nld_ctx* x) {
+  TRY(need_started(x));
+  TRY(ensure_capacity(x, x->c.block_k + 1));
+  std::vector<uintptr_t> key = {2, static_cast<uintptr_t>(x->batch)};
+  TRY(run_graph(x, key, [&]() { return draft_verify_body(x); }));
+  x->verify_fresh = true;
+  return NLD_OK;
+}
+
+nld_status nld_kv_commit(nld_ctx* x, const int32_t* d_nrows, int32_t* d_tokens_out, int32_t* d_ncommit_out) {
+  TRY(need_started(x));
+  if (!x->verify_fresh) return fail(x, NLD_ERR_STATE, "no uncommitted verify forward");
+  FinalizeArgs a = base_fin(x, FWD_COMMIT, x->c.block_k + 1);
+  a.force = d_nrows;
+  a.tokens_out = d_tokens_out;
+  a.ncommit_out = d_ncommit_out;
+  TRY(finalize(x, a));
+  x->len_upper += x->c.block_k + 1;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+nld_status nld_selfspec_round(nld_ctx* x, int32_t* d_tokens_out, int32_t* d_ncommit_out,
+                              const int32_t* d_force_ncommit) {
+  TRY(need_started(x));
+  TRY(ensure_capacity(x, x->c.block_k + 1));
+  std::vector<uintptr_t> key = {3, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_tokens_out),
+                                reinterpret_cast<uintptr_t>(d_ncommit_out), reinterpret_cast<uintptr_t>(d_force_ncommit)};
+  TRY(run_graph(x, key, [&]() -> nld_status {
+    TRY(draft_verify_body(x));
+    FinalizeArgs a = base_fin(x, FWD_COMMIT, x->c.block_k + 1);
+    a.force = d_force_ncommit;
+    a.tokens_out = d_tokens_out;
+    a.ncommit_out = d_ncommit_out;
+    return finalize(x, a);
+  }));
+  x->len_upper += x->c.block_k + 1;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_out, float* d_conf_out,
+                                  int32_t* d_ncommit_out, int32_t* h_filled_out) {
+  TRY(need_started(x));
+  const int k = x->c.block_k;
+  TRY(ensure_capacity(x, k));
+  uint32_t thr_bits;
+  std::memcpy(&thr_bits, &threshold, 4);
+  std::vector<uintptr_t> key = {4, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_block_out),
+                                reinterpret_cast<uintptr_t>(d_conf_out), reinterpret_cast<uintptr_t>(d_ncommit_out),
+                                thr_bits};
+  TRY(run_graph(x, key, [&]() -> nld_status {
+    CK(cudaMemsetAsync(x->incomplete, 0, sizeof(int), x->stream));
+    const long long saved = x->len_upper;
+    x->len_upper = x->c.max_seq;
+    FwdSpec f{};
+    f.mode = FWD_DIFFUSE;
+    f.B = x->batch;
+    f.m = k;
+    f.bs = k;
+    f.lm = LM_ARGMAX;
+    nld_status s = launch_forward(x, f);
+    x->len_upper = saved;
+    if (s != NLD_OK) return s;
+    FinalizeArgs a = base_fin(x, FWD_DIFFUSE, k);
+    a.threshold = threshold;
+    a.block_out = d_block_out;
+    a.conf_out = d_conf_out;
+    a.ncommit_out = d_ncommit_out;
+    TRY(finalize(x, a));
+    CK(cudaMemcpyAsync(x->h_pinned + 1, x->incomplete, sizeof(int), cudaMemcpyDeviceToHost, x->stream));
+    return NLD_OK;
+  }));
+  CK(cudaStreamSynchronize(x->stream));
+  const int open = x->h_pinned[1];
+  int filled = 0;
+  if (open == 0) {
+    std::vector<uintptr_t> fkey = {5, static_cast<uintptr_t>(x->batch)};
+    TRY(run_graph(x, fkey, [&]() -> nld_status {
+      const long long saved = x->len_upper;
+      x->len_upper = x->c.max_seq;
+      FwdSpec f{};
+      f.mode = FWD_FILL;
+      f.B = x->batch;
+      f.m = k;
+      f.bs = 1;
+      f.lm = LM_NONE;
+      nld_status s = launch_forward(x, f);
+      x->len_upper = saved;
+      if (s != NLD_OK) return s;
+      return finalize(x, base_fin(x, FWD_FILL, k));
+    }));
+    x->len_upper += k;
+    filled = 1;
+  }
+  if (h_filled_out) *h_filled_out = filled;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
+  TRY(need_started(x));
+  if (!d_logits_out) return fail(x, NLD_ERR_ARG, "logits is NULL");
+  const int k = x->c.block_k;
+  FwdSpec f{};
+  f.B = x->batch;
+  f.lm = LM_LOGITS;
+  f.logits = d_logits_out;
+  int fm;
+  switch (mode) {
+    case NLD_MODE_AR: fm = FWD_AR; f.m = 1; f.bs = 1; break;
+    case NLD_MODE_DRAFT: fm = FWD_DRAFT; f.m = k; f.bs = k; break;
+    case NLD_MODE_VERIFY: fm = FWD_VERIFY; f.m = k + 1; f.bs = 1; break;
+    case NLD_MODE_DIFFUSE: fm = FWD_DIFFUSE; f.m = k; f.bs = k; break;
+    default: return fail(x, NLD_ERR_ARG, "unknown mode %d", mode);
+  }
+  TRY(ensure_capacity(x, f.m));
+  f.mode = fm;
+  TRY(launch_forward(x, f));
+  // also record argmaxes (drafts / verify) through the argmax epilogue of the same forward
+  f.lm = LM_ARGMAX;
+  f.logits = nullptr;
+  TRY(launch_forward(x, f));
+  FinalizeArgs a = base_fin(x, fm, f.m);
+  a.commit = 0;
+  TRY(finalize(x, a));
+  if (mode == NLD_MODE_VERIFY) x->verify_fresh = true;
+  return NLD_OK;
+}
+
+nld_status nld_debug_state(nld_ctx* x, int32_t* d_lens_out, int32_t* d_pending_out, int32_t* d_draft_out,
+                           int32_t* d_verify_out) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  const int B = std::max(x->batch, 1), k = x->c.block_k;
+  if (d_lens_out) CK(cudaMemcpyAsync(d_lens_out, x->lens, B * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  if (d_pending_out) CK(cudaMemcpyAsync(d_pending_out, x->pending, B * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  if (d_draft_out) CK(cudaMemcpyAsync(d_draft_out, x->draft, static_cast<size_t>(B) * k * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  if (d_verify_out) CK(cudaMemcpyAsync(d_verify_out, x->verify, static_cast<size_t>(B) * (k + 1) * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  return NLD_OK;
+}
+
+nld_status nld_sync(nld_ctx* x) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  CK(cudaMemcpyAsync(x->h_pinned, x->err, sizeof(int), cudaMemcpyDeviceToHost, x->stream));
+  CK(cudaMemsetAsync(x->err, 0, sizeof(int), x->stream));
+  CK(cudaStreamSynchronize(x->stream));
+  const int e = x->h_pinned[0];
+  if (e & NLD_DEVERR_TIMEOUT) return fail(x, NLD_ERR_TIMEOUT, "a bounded device wait ran out (error word 0x%x)", e);
+  if (e & NLD_DEVERR_KV_OVERFLOW) return fail(x, NLD_ERR_KV_FULL, "a KV write past capacity was skipped (error word 0x%x)", e);
+  if (e) return fail(x, NLD_ERR_DEVICE, "device bounds check failed (error word 0x%x)", e);
+  return NLD_OK;
+}
+
+const char* nld_last_error(const nld_ctx* x) {
+  return x ? x->msg.c_str() : g_static_err.c_str();
+}
+
+void* nld_stream(nld_ctx* x) { return x ? static_cast<void*>(x->stream) : nullptr; }
+
+// ----------------------------------------------------------------- stand-alone attention --
+static void attn_ws_layout(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a,
+                           size_t& cnt_bytes, size_t& ml_bytes, size_t& o_bytes) {
+  attn_plan(batch, m, Hq, Hkv, max_len, sms, a);
+  const size_t units = static_cast<size_t>(batch) * a.q_tiles * Hkv;
+  const size_t rows_pad = static_cast<size_t>(a.NW) * 16;
+  cnt_bytes = (units * sizeof(int) + 255) / 256 * 256;
+  ml_bytes = a.S > 1 ? (units * a.S * rows_pad * 2 * sizeof(float) + 255) / 256 * 256 : 0;
+  o_bytes = a.S > 1 ? units * a.S * rows_pad * 128 * sizeof(float) : 0;
+}
+
+static int device_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  return n;
+}
+
+size_t nld_attention_workspace_size(int batch, int m, int n_q_heads, int n_kv_heads, int head_dim,
+                                    int max_len) {
+  if (batch < 1 || m < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || head_dim != 128) return 0;
+  AttnArgs a{};
+  size_t c, ml, o;
+  attn_ws_layout(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a, c, ml, o);
+  return c + ml + o;
+}
+
+nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* d_page_table,
+                         int pages_per_seq, int n_pages, const int32_t* d_lens, int batch, int m,
+                         int n_q_heads, int n_kv_heads, int head_dim, int block_size, int max_len,
+                         void* d_out, void* d_workspace, size_t workspace_bytes, void* cuda_stream) {
+  nld_ctx* x = nullptr;
+  if (!d_q || !d_kv_pool || !d_page_table || !d_lens || !d_out)
+    return fail(nullptr, NLD_ERR_ARG, "NULL pointer argument");
+  if (batch < 1 || m < 1 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads)
+    return fail(nullptr, NLD_ERR_ARG, "bad batch/m/head counts");
+  if (head_dim != 128) return fail(nullptr, NLD_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (block_size < 1) return fail(nullptr, NLD_ERR_ARG, "block_size must be >= 1");
+  if (max_len < m || max_len > pages_per_seq * kPage) return fail(nullptr, NLD_ERR_ARG, "max_len outside m..pages_per_seq*64");
+  if (static_cast<long long>(n_pages) * 2 * n_kv_heads * kPage > INT32_MAX) return fail(nullptr, NLD_ERR_ARG, "pool too large");
+  AttnArgs a{};
+  size_t cb, mlb, ob;
+  attn_ws_layout(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a, cb, mlb, ob);
+  if (!d_workspace || workspace_bytes < cb + mlb + ob)
+    return fail(nullptr, NLD_ERR_ARG, "workspace too small: need %zu bytes", cb + mlb + ob);
+  if (reinterpret_cast<uintptr_t>(d_workspace) % 16) return fail(nullptr, NLD_ERR_ARG, "workspace must be 16-byte aligned");
+  CUtensorMap map;
+  if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))
+    return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed (pool)");
+  a.q = d_q;
+  a.out = d_out;
+  a.m = m;
+  a.Hq = n_q_heads;
+  a.Hkv = n_kv_heads;
+  a.hd = 128;
+  a.lens = d_lens;
+  a.page_table = d_page_table;
+  a.pps = pages_per_seq;
+  a.layer_row0 = 0;
+  a.block_size = block_size;
+  a.counters = static_cast<int*>(d_workspace);
+  a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(d_workspace) + cb);
+  a.ws_o = reinterpret_cast<float*>(static_cast<char*>(d_workspace) + cb + mlb);
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  a.err = nullptr;
+  cudaError_t e = launch_attention_mma(static_cast<cudaStream_t>(cuda_stream), &map, a, batch, false);
+  if (e != cudaSuccess) return fail(x, NLD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  return NLD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+// Internal declarations shared by the kernels and the host orchestration.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nld.h"
+
+namespace nld {
+
+constexpr int kPage = 64;          // KV page length in tokens (one attention KV tile)
+constexpr int kTileRows = 128;     // GEMM weight rows per tile (tcgen05 M)
+constexpr int kTileK = 64;         // GEMM K per pipeline stage (128 bytes of bf16)
+constexpr int kMaxNT = 256;        // max token columns per GEMM tile (tcgen05 N)
+
+// Epilogue kinds of the projection GEMMs.
+enum EpiKind : int {
+  EPI_QKV = 0,     // * 1/rms, RoPE on q/k, q -> q buffer, k/v -> paged KV cache
+  EPI_RESID = 1,   // h += acc; hb = bf16(h); per-tile sum of squares of h
+  EPI_SWIGLU = 2,  // * 1/rms; silu(gate) * up -> u buffer
+  EPI_LMHEAD = 3,  // * 1/rms; per (token, vocab tile): max, argmax, sum exp(l - max)
+  EPI_LOGITS = 4,  // * 1/rms; logits -> fp32 buffer (test hook only)
+};
+
+// Forward kinds (which tokens the embedding gathers and what the finalize step does).
+enum FwdMode : int {
+  FWD_AR = 0, FWD_DRAFT = 1, FWD_VERIFY = 2, FWD_DIFFUSE = 3, FWD_FILL = 4, FWD_PREFILL = 5,
+  FWD_COMMIT = 6
+};
+
+// Per (token, vocab tile) partial of the LM-head reduction.
+struct LmPart {
+  float mx;    // max logit in the tile
+  float se;    // sum over the tile of exp(l - mx)
+  int idx;     // lowest vocab id attaining mx
+  int pad;
+};
+
+struct EpiArgs {
+  int kind;
+  int M;            // tokens in this forward (columns)
+  int m;            // rows per sequence
+  int n_rows;       // valid weight rows (GEMM outputs)
+  // RMSNorm of the GEMM input: 1/rms[tok] = rsqrt(sum_t ssq_in[t*ld + tok] / d + eps)
+  const float* ssq_in;
+  int ssq_tiles;
+  int ssq_ld;
+  float inv_d;
+  float eps;
+  // EPI_QKV
+  void* q_out;      // [M, Hq, hd]
+  int Hq, Hkv, hd;
+  void* kv_layer;   // pool base of this layer: [n_pages][2][Hkv][64][hd]
+  const int* page_table;  // [batch, pps]
+  int pps;
+  const int* lens;  // [batch]
+  const float2* rope;  // [kv_cap, hd/2] (cos, sin)
+  int kv_cap;
+  // EPI_RESID
+  float* h;         // [M, d]
+  void* hb;         // [M, d]
+  float* ssq_out;   // [d/128, ssq_ld]
+  int d;
+  // EPI_SWIGLU
+  void* u_out;      // [M, F]
+  int F;
+  // EPI_LMHEAD / EPI_LOGITS
+  LmPart* lm_part;  // [M, lm_tiles]
+  int lm_tiles;
+  float* logits;    // [M, V]
+  int V;
+  int* err;
+};
+
+struct GemmShape {
+  int n_rows;       // weight rows
+  int K;
+  int M;
+  int NT;           // token columns per tile (multiple of 16, <= 256)
+  int tok_tiles;
+  int row_tiles;
+  int KT;           // K / 64
+  long long T;      // row_tiles * tok_tiles * KT  (k-iterations over all tiles)
+  int G;            // CTAs (stream-K workers)
+  int stages;
+  uint32_t tmem_cols;  // power of two >= 2*NT
+  int ws_slot;      // floats per workspace slot (128 * NT)
+};
+
+struct AttnArgs {
+  const void* q;        // [M, Hq, hd]
+  void* out;            // [M, Hq, hd]
+  const void* pool;     // SIMT path: pool base of this layer
+  int m, Hq, Hkv, G, hd;
+  const int* lens;
+  const int* page_table;
+  int pps;
+  int layer_row0;       // row of this layer's first page in the 2D pool view
+  int block_size;
+  int QT, q_tiles, rows, S, NW;
+  float* ws_o;
+  float* ws_ml;
+  int* counters;
+  float scale_log2;     // log2(e) / sqrt(hd)
+  int* err;
+};
+
+// ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
+cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
+                           const GemmShape& s, const EpiArgs& e, float* ws, int* counters,
+                           uint64_t timeout_ns, bool pdl);
+cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
+                             int M, const EpiArgs& e, bool pdl);
+cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
+                                 int batch, bool pdl);
+cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,
+                                  int max_kv, bool pdl);
+
+struct EmbedArgs {
+  const void* E;        // [V+1, d]
+  int d, V, m, mode, k;
+  const int* pending; const int* draft; const int* blk;
+  const int* prompt; int prompt_len; int chunk0;
+  const int* lens;
+  float* h; void* hb; float* ssq; int ssq_ld;
+  int* err;
+};
+cudaError_t launch_embed(cudaStream_t st, const EmbedArgs& a, int M, bool bf16, bool pdl);
+
+struct FinalizeArgs {
+  int mode, m, k, V, lm_tiles;
+  const LmPart* lm_part;
+  int* lens; int* pending; int* draft; int* verify; int* blk;
+  int* tokens_out; int* ncommit_out; const int* force; float* conf_out; int* block_out;
+  float threshold;
+  int* incomplete;      // diffusion: count of sequences whose block is still open
+  const int* prompt; int prompt_len; int chunk;   // prefill
+  int commit;           // 0 = only record argmaxes (test hook)
+  int kv_cap;
+  int* err;
+};
+cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, bool pdl);
+
+cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
+                          int n_rows, int K, const void* gamma, bool bf16);
+cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
+
+}  // namespace nld
