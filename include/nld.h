@@ -89,7 +89,7 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out);
 /* Synchronise the stream and free everything the context owns.  Accepts NULL. */
 nld_status nld_destroy(nld_ctx* ctx);
 
-/* Copy and repack the weights.  `tensors` holds 2 + 9*n_layers pointers in this order:
+/* Copy and repack the weights.  `tensors` holds 3 + 9*n_layers pointers in this order:
  *   embed [vocab+1, d_model],
  *   per layer: attn_norm [d], wq [Hq*hd, d], wk [Hkv*hd, d], wv [Hkv*hd, d], wo [d, Hq*hd],
  *              mlp_norm [d], wg [ffn, d], wu [ffn, d], wd [d, ffn],

@@ -407,8 +407,14 @@ cudaError_t gemm_tc_init_attributes();
 cudaError_t init_kernel_attributes() {
   cudaError_t e = gemm_tc_init_attributes();
   if (e != cudaSuccess) return e;
+  int dev = 0, optin = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+    return e;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel)) != cudaSuccess) return e;
   return cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              227 * 1024);
+                              optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
 size_t attn_mma_smem_bytes(int NW) {

@@ -303,8 +303,16 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 cudaError_t gemm_tc_init_attributes() {
+  int dev = 0, optin = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+    return e;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, gemm_tc_kernel<__nv_bfloat16>)) != cudaSuccess) return e;
   return cudaFuncSetAttribute(gemm_tc_kernel<__nv_bfloat16>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
 size_t gemm_tc_smem_bytes(const GemmShape& s) {

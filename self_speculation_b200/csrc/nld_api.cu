@@ -504,10 +504,14 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
                 prop.major, prop.minor);
   }
   x->el = x->bf16 ? 2 : 4;
-  if (init_kernel_attributes() != cudaSuccess) {
-    cudaGetLastError();
-    delete x;
-    return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed");
+  {
+    cudaError_t ae = init_kernel_attributes();
+    if (ae != cudaSuccess) {
+      cudaGetLastError();
+      delete x;
+      return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed: %s",
+                  cudaGetErrorString(ae));
+    }
   }
   if (cuda_stream) {
     x->stream = static_cast<cudaStream_t>(cuda_stream);
@@ -633,8 +637,8 @@ nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensor
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   const nld_config& c = x->c;
   const int L = c.n_layers;
-  if (!tensors || n_tensors != 2 + 9 * L)
-    return fail(x, NLD_ERR_ARG, "expected %d weight tensors, got %d", 2 + 9 * L, n_tensors);
+  if (!tensors || n_tensors != 3 + 9 * L)
+    return fail(x, NLD_ERR_ARG, "expected %d weight tensors, got %d", 3 + 9 * L, n_tensors);
   for (int i = 0; i < n_tensors; ++i)
     if (!tensors[i]) return fail(x, NLD_ERR_ARG, "weight tensor %d is NULL", i);
   const size_t el = x->el;
@@ -1040,6 +1044,14 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   if (!d_workspace || workspace_bytes < cb + mlb + ob)
     return fail(nullptr, NLD_ERR_ARG, "workspace too small: need %zu bytes", cb + mlb + ob);
   if (reinterpret_cast<uintptr_t>(d_workspace) % 16) return fail(nullptr, NLD_ERR_ARG, "workspace must be 16-byte aligned");
+  {
+    cudaError_t ae = init_kernel_attributes();
+    if (ae != cudaSuccess) {
+      cudaGetLastError();
+      return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed: %s",
+                  cudaGetErrorString(ae));
+    }
+  }
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))
     return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed (pool)");
