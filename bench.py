@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the self-speculation decode round (8B-shaped decoder, batch 1 per GPU).
+
+A step is one linear self-speculation round through the C ABI: draft forward (one
+bidirectional block of k=32 positions over the cached prefix), causal verify forward (k+1
+positions), greedy acceptance and KV commit.  Weights are random-init bf16 of the 8B shape
+(36 layers, d 4096, 32/8 heads x 128, FFN 12288, vocab 151936); the prompt is 512 uniform
+random ids (synthetic stand-in for the benchmark prompts).  Every forward streams 15.1 GB of
+weights, far above the 126 MB L2, so no L2 flush is needed between steps.
+
+Multi-GPU: replicas only (every rank decodes its own sequence; there is no exchange step in
+the round).  Timing: CUDA events on the library's stream, max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "committed tokens/s & self-spec rounds/s at batch 1 (8B shape); % HBM roofline"
+PROMPT = 512
+K_BLOCK = 32
+HBM_FALLBACK_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return HBM_FALLBACK_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "epilogue.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "self_speculation_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce(vals, op, world):
+    import torch
+    if world == 1:
+        return vals
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return t.tolist()
+
+
+# ------------------------------------------------------------------------- CPU oracle leg --
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of one round of the 8B shape: draft (k rows) and
+    verify (k+1 rows) forwards over `n_layers_sample` of the 36 layers, timed with and without
+    the LM head, at 511 cached rows (zero-valued cache; values do not change the work)."""
+
+    def __init__(self, n_layers_sample: int, threads: int):
+        import torch
+
+        import oracle
+        import synth
+        torch.set_num_threads(threads)
+        self.cfg = synth.LLAMA8B
+        self.layers = list(range(n_layers_sample))
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        W = synth.model_weights(self.cfg, 0, device=dev, layers=self.layers)
+        W = [None if w is None else w.cpu() for w in W]
+        self.om = oracle.OracleModel(self.cfg, W, "f32")
+
+    def round(self):
+        """Returns (seconds for a full 36-layer round by layer-count scaling, wall seconds spent,
+        committed tokens of the sampled round)."""
+        import torch
+
+        from oracle import decode as odec
+        om, cfg, layers, k = self.om, self.cfg, self.layers, K_BLOCK
+        st = odec.SeqState(cache=om.new_cache(1, PROMPT + 2 * K_BLOCK + 2), lens=[PROMPT - 1],
+                           pending=[7])
+        t_all0 = time.perf_counter()
+        draft_toks = torch.full((1, k), cfg.mask_id, dtype=torch.int64)
+        draft_toks[0, 0] = st.pending[0]
+        t0 = time.perf_counter()
+        dl = om.forward(draft_toks, st.lens, st.cache, block_size=k, write_kv=False, layers=layers)
+        t1 = time.perf_counter()
+        om.forward(draft_toks, st.lens, st.cache, block_size=k, write_kv=False, layers=layers,
+                   with_logits=False)
+        t2 = time.perf_counter()
+        drafts = odec.argmax_lowest(dl).tolist()
+        ver_toks = torch.tensor([[st.pending[0]] + drafts[0]], dtype=torch.int64)
+        t3 = time.perf_counter()
+        vl = om.forward(ver_toks, st.lens, st.cache, block_size=1, write_kv=True, layers=layers)
+        t4 = time.perf_counter()
+        om.forward(ver_toks, st.lens, st.cache, block_size=1, write_kv=True, layers=layers,
+                   with_logits=False)
+        t5 = time.perf_counter()
+        committed = odec.commit_after_verify(drafts[0], odec.argmax_lowest(vl).tolist()[0])
+        scale = cfg.n_layers / len(layers)
+        lm_d = max(0.0, (t1 - t0) - (t2 - t1))
+        lm_v = max(0.0, (t4 - t3) - (t5 - t4))
+        round_s = (t2 - t1) * scale + lm_d + (t5 - t4) * scale + lm_v
+        return round_s, time.perf_counter() - t_all0, len(committed)
+
+
+# ------------------------------------------------------------------------------ our arm --
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import self_speculation_b200 as nb
+    import synth
+    from self_speculation_b200 import build as nbuild
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    nbuild.build()
+    K, W = args.steps, args.warmup
+    max_seq = (PROMPT + (K_BLOCK + 1) * (W + K + 2) + 63) // 64 * 64 + 64
+    cfg = synth.LLAMA8B.replace(max_seq=max_seq)
+    torch_stream = torch.cuda.Stream()          # owned by torch; the library orders on it
+    ctx = nb.Context(cfg, stream=torch_stream.cuda_stream)
+    weights = synth.model_weights(cfg, 0, device="cuda")
+    ctx.nld_init_weights(weights, on_device=True)
+    del weights
+    torch.cuda.empty_cache()
+    prompt = synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1 + rank)
+    ctx.nld_prefill(prompt.cuda())
+    toks = torch.empty(1, K_BLOCK + 1, dtype=torch.int32, device="cuda")
+    nc = torch.empty(1, dtype=torch.int32, device="cuda")
+    lens = torch.empty(1, dtype=torch.int32, device="cuda")
+    for _ in range(W):
+        ctx.nld_selfspec_round(toks, nc, None)
+    ctx.nld_sync()
+    ctx.nld_debug_state(lens)
+    ctx.nld_sync()
+    len0 = int(lens.item())
+    stream = torch_stream
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk = Clocks(local)
+    clk.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(K):
+        ctx.nld_selfspec_round(toks, nc, None)
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1)
+    ctx.nld_sync()
+    ctx.nld_debug_state(lens)
+    ctx.nld_sync()
+    len1 = int(lens.item())
+    committed = len1 - len0
+    max_ms, = reduce([ms], "max", world)
+    tot_committed, = reduce([float(committed)], "sum", world)
+    value = tot_committed / (max_ms / 1e3)
+    rounds_per_s = world * K / (max_ms / 1e3)
+
+    # round roofline: weight bytes of two forwards + KV rows read + KV rows written
+    hbm, peak_src = peaks()
+    wbytes = cfg.weight_bytes_per_forward()
+    kvb = cfg.kv_bytes_per_token()
+    L_avg = (len0 + len1) / 2.0
+    round_bytes = 2 * wbytes + (2 * L_avg + K_BLOCK + (K_BLOCK + 1)) * kvb \
+        + (2 * K_BLOCK + 1) * kvb
+    round_s = ms / 1e3 / K
+    round_gbs = round_bytes / round_s / 1e9
+
+    # dominant kernel: the fused gate/up GEMM of a verify forward (201 MB of weights / launch)
+    M = K_BLOCK + 1
+    kern = {}
+    names = ["qkv", "o", "gate_up", "down", "lm_head"]
+    n_rows = [cfg.q_dim + 2 * cfg.kv_dim, cfg.d_model, 2 * cfg.ffn_dim, cfg.d_model, cfg.vocab]
+    k_dim = [cfg.d_model, cfg.q_dim, cfg.d_model, cfg.ffn_dim, cfg.d_model]
+    for w, (nm, nr, kd) in enumerate(zip(names, n_rows, k_dim)):
+        reps = 10 if nm == "lm_head" else 40
+        t = ctx.nld_time_gemm(w, 0, M, reps)
+        byts = 2 * nr * kd + 2 * M * kd + (2 * M * nr // (2 if nm == "gate_up" else 1))
+        kern[nm] = {"ms": round(t, 5), "GB/s": round(byts / (t / 1e3) / 1e9, 1),
+                    "bytes": byts}
+    gu = kern["gate_up"]
+    roofline = {"bound": "hbm", "achieved": gu["GB/s"], "peak": hbm, "unit": "GB/s",
+                "frac": round(gu["GB/s"] / hbm, 4), "traffic": ncu_traffic("gemm_gate_up_8b_m33.txt"),
+                "kernel": "gemm_tc_kernel gate/up (8B, M=33 tokens), timed alone",
+                "peak_kind": f"{peak_src} HBM copy (burst)"}
+
+    # end to end through the public API: prompt H2D from pinned memory, prefill, K rounds, each
+    # followed by a D2H read of the committed tokens and counts
+    ctx2_tokens = 0
+    host_prompt = prompt.pin_memory()
+    h_toks = torch.empty(1, K_BLOCK + 1, dtype=torch.int32).pin_memory()
+    h_nc = torch.empty(1, dtype=torch.int32).pin_memory()
+    dev_prompt = torch.empty_like(prompt, device="cuda")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        dev_prompt.copy_(host_prompt, non_blocking=True)
+    stream.synchronize()
+    ctx.nld_prefill(dev_prompt)
+    for _ in range(K):
+        ctx.nld_selfspec_round(toks, nc, None)
+        with torch.cuda.stream(stream):
+            h_toks.copy_(toks, non_blocking=True)
+            h_nc.copy_(nc, non_blocking=True)
+        stream.synchronize()
+        ctx2_tokens += int(h_nc[0])
+    e2e_s = time.perf_counter() - t0
+    max_e2e, = reduce([e2e_s], "max", world)
+    tot_e2e, = reduce([float(ctx2_tokens)], "sum", world)
+    e2e = {"value": round(tot_e2e / max_e2e, 3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(PROMPT * 4 / K), "d2h_bytes_per_step": (K_BLOCK + 2) * 4,
+           "includes": "prompt upload + prefill of 512 tokens + K rounds with a D2H read each"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        round_est, spent, ncommit = OracleSample(2, threads).round()
+        cpu = {"value": round(ncommit / round_est, 5), "unit": "tokens/s", "cores": threads,
+               "kind": "oracle",
+               "sample": (f"one draft+verify round of the 8B shape at 511 cached rows over 2 of 36 "
+                          f"layers plus the LM head, scaled to 36 layers ({spent:.1f} s of CPU "
+                          f"work); {ncommit} committed token(s) in the sampled round"),
+               "round_s_est": round(round_est, 2)}
+
+    per_round = 2 * (1 + 5 * cfg.n_layers + 1 + 1) + 1
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "8B-shaped linear self-speculation round, batch 1 per GPU, k=32, "
+                               "prompt 512 random ids, random-init bf16 weights",
+                   "layers": cfg.n_layers, "d_model": cfg.d_model, "heads": "32q/8kv x 128",
+                   "ffn": cfg.ffn_dim, "vocab": cfg.vocab, "batch_per_gpu": 1, "block_k": K_BLOCK,
+                   "prompt": PROMPT, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: 15.1 GB of weights per forward exceed the 126 MB L2"},
+        "rounds_per_s": round(rounds_per_s, 3),
+        "tokens_per_forward": round(tot_committed / (2 * world * K), 4),
+        "round_roofline": {"bound": "hbm", "achieved": round(round_gbs, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(round_gbs / hbm, 4),
+                           "bytes_per_round": int(round_bytes)},
+        "roofline": roofline,
+        "kernels": kern,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": K * per_round,
+        "clocks": clocks,
+    }
+    ctx.close()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, world, rank, local):
+    """The oracle as it stands on the host cores (rank 0 only), each step one bounded sample
+    of a round (1 of 36 layers of a draft and a verify forward plus the LM head, scaled)."""
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    est, committed, spent = [], 0, 0.0
+    sample = OracleSample(1, threads)
+    for i in range(args.warmup + args.steps):
+        r, s, c = sample.round()
+        if i >= args.warmup:
+            est.append(r)
+            committed += c
+            spent += s
+    round_s = sum(est) / len(est)
+    value = committed / sum(est)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(round_s * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "8B-shaped linear self-speculation round, batch 1, k=32, "
+                               "prompt 512 random ids (CPU oracle)",
+                   "parallelism": "host cores of rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": "per step: draft+verify forwards over 1 of 36 layers plus the "
+                                   "LM head at 511 cached rows, scaled to 36 layers"},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_probe(args):
+    """Small case for ncu captures: a 2-layer model of the 8B layer shape (full vocab), prompt
+    512, then each projection GEMM launched alone at M=33 tokens (nld_time_gemm, reps=2) and one
+    self-speculation round."""
+    import torch
+
+    import self_speculation_b200 as nb
+    import synth
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    cfg = synth.LLAMA8B.replace(n_layers=2, max_seq=1024)
+    st = torch.cuda.Stream()
+    ctx = nb.Context(cfg, stream=st.cuda_stream)
+    ctx.nld_init_weights(synth.model_weights(cfg, 0, device="cuda"), on_device=True)
+    ctx.nld_prefill(synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1).cuda())
+    toks = torch.empty(1, K_BLOCK + 1, dtype=torch.int32, device="cuda")
+    nc = torch.empty(1, dtype=torch.int32, device="cuda")
+    ctx.nld_selfspec_round(toks, nc, None)
+    ctx.nld_sync()
+    out = {}
+    plans = {}
+    for w, nm in enumerate(["qkv", "o", "gate_up", "down", "lm_head"]):
+        out[nm] = ctx.nld_time_gemm(w, 0, K_BLOCK + 1, 2)
+        plans[nm] = ctx.nld_debug_gemm_plan(w, K_BLOCK + 1)
+    ctx.nld_selfspec_round(toks, nc, None)
+    ctx.nld_sync()
+    phases = ["start", "setup", "tma0", "tmaN", "mma0", "acc0", "acc1", "epi0", "epi1",
+              "epi0end", "epi1end", "exit", "fin_start", "fin_c0_loaded", "fin_c0_epi", "exit_epi"]
+    traces = {}
+    for w, nm in enumerate(["qkv", "o", "gate_up", "down", "lm_head"]):
+        tr = torch.zeros(148 * 16, dtype=torch.int64, device="cuda")
+        G = ctx.nld_trace_gemm(w, 0, K_BLOCK + 1, tr)
+        t = tr.view(148, 16)[:G, :16].cpu().double()
+        t0 = t[:, 0].min()
+        rel = {}
+        for i, ph in enumerate(phases):
+            col = t[:, i]
+            col = col[col > 0] - t0
+            if len(col):
+                rel[ph] = [round(float(col.min()) / 1e3, 2), round(float(col.median()) / 1e3, 2),
+                           round(float(col.max()) / 1e3, 2)]
+        traces[nm] = rel
+    ctx.close()
+    torch.cuda.synchronize()
+    print(json.dumps({"probe_ms": out}))
+    print(json.dumps({"plans": plans}))
+    print(json.dumps({"trace_us_min_med_max": traces}, indent=1))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe", action="store_true",
+                    help="small kernel-probe case for profiler captures (no JSON bench line)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.probe:
+        run_probe(args)
+    elif args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -159,6 +159,25 @@ nld_status nld_debug_logits(nld_ctx* ctx, int mode, float* d_logits_out);
 nld_status nld_debug_state(nld_ctx* ctx, int32_t* d_lens_out, int32_t* d_pending_out,
                            int32_t* d_draft_out, int32_t* d_verify_out);
 
+/* Profiling hook: launch the projection GEMM `which` (0 fused QKV, 1 O, 2 fused gate/up,
+ * 3 down, 4 LM head) of `layer` `reps` times back to back on the context stream over M token
+ * rows of the context's activation buffers (M a multiple of the batch), between two CUDA
+ * events; *ms_out = mean milliseconds per launch.  Synchronises.  Its epilogue writes only
+ * scratch (activations, partials, KV rows at positions >= len): decode state does not move. */
+nld_status nld_time_gemm(nld_ctx* ctx, int which, int layer, int M, int reps, float* ms_out);
+
+/* Profiling hook: like nld_time_gemm, one traced launch; d_trace receives, per CTA, 16
+ * globaltimer stamps (ns): 0 start, 1 setup done, 2/3 first/last TMA issue, 4 first MMA,
+ * 5/6 accumulator 0/1 committed, 7/8 epilogue 0/1 start, 9/10 epilogue 0/1 end, 11 exit.
+ * *grid_out = number of CTAs.  Synchronises. */
+nld_status nld_trace_gemm(nld_ctx* ctx, int which, int layer, int M, unsigned long long* d_trace,
+                          int* grid_out);
+
+/* Profiling hook: the tiling chosen for projection GEMM `which` (as in nld_time_gemm) over M
+ * token rows: out8 = {NT, token tiles, row tiles, k-iterations, split (cluster size),
+ * k-iterations per split, CTAs, pipeline stages}.  No GPU work. */
+nld_status nld_debug_gemm_plan(nld_ctx* ctx, int which, int M, int* out8);
+
 /* Synchronise the context stream and report the device error word (then clear it):
  * NLD_OK, NLD_ERR_KV_FULL, NLD_ERR_TIMEOUT or NLD_ERR_DEVICE. */
 nld_status nld_sync(nld_ctx* ctx);
@@ -176,27 +195,22 @@ const char* nld_last_error(const nld_ctx* ctx);
  * "Method": a query sees every cached key and the keys of its own and earlier blocks.
  *   d_q        [batch, m, Hq, hd] bf16: queries at positions lens[b]..lens[b]+m-1.
  *   d_kv_pool  [n_pages][2][Hkv][64][hd] bf16 (K then V per page); the rows of the m query
- *              positions must already be in the pool.
+ *              positions must already be in the pool.  Rows no query may see must still hold
+ *              finite values (zero-fill the pool once).
  *   d_page_table [batch, pages_per_seq] int32 page ids (< n_pages).
  *   d_lens     [batch] int32 cached rows before the m query rows.
  *   block_size queries are cut into blocks of block_size from lens[b]; 1 = causal.
- *   max_len    host upper bound of lens[b] + m (sizes the KV split), <= pages_per_seq*64.
+ *   max_len    host upper bound of lens[b] + m (sizes the KV split), <= pages_per_seq*64;
+ *              a longer sequence on the device is clamped and flagged.
  *   d_out      [batch, m, Hq, hd] bf16.
- *   d_workspace / workspace_bytes: scratch of at least nld_attention_workspace_size() bytes,
- *              owned by the caller, 16-byte aligned, zero-filled once before its first use
- *              (it starts with per-group arrival counters that every call leaves at zero;
- *              the rest holds split-KV partials).  Calls sharing a workspace must not
- *              overlap on the GPU.
- *   Pool rows that no query may see must still hold finite values (zero-fill the pool).
- * Requires head_dim == 128, page size 64.  Stream-ordered on `cuda_stream`.
+ * KV splits run as clusters of up to 8 CTAs that merge their partials in distributed shared
+ * memory, so the call needs no scratch.  Requires head_dim == 128, page size 64.
+ * Stream-ordered on `cuda_stream`; returns after the launch.
  */
-size_t nld_attention_workspace_size(int batch, int m, int n_q_heads, int n_kv_heads,
-                                    int head_dim, int max_len);
 nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* d_page_table,
                          int pages_per_seq, int n_pages, const int32_t* d_lens, int batch, int m,
                          int n_q_heads, int n_kv_heads, int head_dim, int block_size, int max_len,
-                         void* d_out, void* d_workspace, size_t workspace_bytes,
-                         void* cuda_stream);
+                         void* d_out, void* cuda_stream);
 
 #ifdef __cplusplus
 }

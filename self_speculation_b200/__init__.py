@@ -60,10 +60,12 @@ def load_library() -> ctypes.CDLL:
         "nld_debug_logits": ([P, I, P], I),
         "nld_debug_state": ([P, P, P, P, P], I),
         "nld_sync": ([P], I),
+        "nld_time_gemm": ([P, I, I, I, I, ctypes.POINTER(F)], I),
+        "nld_trace_gemm": ([P, I, I, I, P, ctypes.POINTER(I)], I),
+        "nld_debug_gemm_plan": ([P, I, I, ctypes.POINTER(I)], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
-        "nld_attention_workspace_size": ([I, I, I, I, I, I], S),
-        "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P, S, P], I),
+        "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -161,24 +163,36 @@ class Context:
         self._check(self.lib.nld_debug_state(self.h, _ptr(lens), _ptr(pending), _ptr(draft),
                                              _ptr(verify)), self.h)
 
+    def nld_time_gemm(self, which: int, layer: int, M: int, reps: int) -> float:
+        ms = ctypes.c_float(0.0)
+        self._check(self.lib.nld_time_gemm(self.h, which, layer, M, reps, ctypes.byref(ms)), self.h)
+        return ms.value
+
+    def nld_trace_gemm(self, which: int, layer: int, M: int, trace) -> int:
+        g = ctypes.c_int(0)
+        self._check(self.lib.nld_trace_gemm(self.h, which, layer, M, _ptr(trace), ctypes.byref(g)),
+                    self.h)
+        return g.value
+
+    def nld_debug_gemm_plan(self, which: int, M: int) -> dict:
+        v = (ctypes.c_int * 8)()
+        self._check(self.lib.nld_debug_gemm_plan(self.h, which, M, v), self.h)
+        keys = ["NT", "tok_tiles", "row_tiles", "KT", "split", "ks", "ctas", "stages"]
+        return dict(zip(keys, list(v)))
+
     def nld_sync(self) -> None:
         self._check(self.lib.nld_sync(self.h), self.h)
 
 
-def nld_attention_workspace_size(batch, m, n_q_heads, n_kv_heads, head_dim, max_len) -> int:
-    return load_library().nld_attention_workspace_size(batch, m, n_q_heads, n_kv_heads, head_dim,
-                                                       max_len)
-
-
-def nld_attention(q, kv_pool, page_table, lens, block_size: int, max_len: int, out, workspace,
+def nld_attention(q, kv_pool, page_table, lens, block_size: int, max_len: int, out,
                   stream: Optional[int] = None) -> None:
     """q [B, m, Hq, hd] bf16, kv_pool [n_pages, 2, Hkv, 64, hd] bf16, page_table [B, pps] int32,
-    lens [B] int32, out like q, workspace uint8 (zero-filled once)."""
+    lens [B] int32, out like q."""
     lib = load_library()
     B, m, Hq, hd = q.shape
     n_pages, _, Hkv, _, _ = kv_pool.shape
     st = lib.nld_attention(_ptr(q), _ptr(kv_pool), _ptr(page_table), page_table.shape[1], n_pages,
                            _ptr(lens), B, m, Hq, Hkv, hd, int(block_size), int(max_len), _ptr(out),
-                           _ptr(workspace), workspace.numel() * workspace.element_size(), stream)
+                           stream)
     if st != 0:
         raise NldError(st, lib.nld_last_error(None).decode())

@@ -13,8 +13,10 @@
 // heads that share them.  K/V tiles of 64 keys (one page) are staged by TMA with 128-byte
 // swizzle in a 3-deep ring; S = Q K^T and O += P V run on mma.sync m16n8k16 (bf16 in, fp32
 // accumulate); the softmax is online in registers (exp2 domain) with quad shuffles.  When the
-// keys are split over several CTAs (flash decoding), each writes unnormalised partials and
-// the last CTA of the group (atomic counter) merges them in split order.
+// keys are split over several CTAs (flash decoding), those CTAs form one thread-block cluster:
+// each leaves its unnormalised partial (O, running max, running sum) in its shared memory, and
+// after a cluster barrier every CTA merges a slice of the rows by reading all partials over
+// distributed shared memory, in split order.  No global scratch, no atomics.
 #include "common.cuh"
 
 namespace nld {
@@ -69,7 +71,6 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   uint8_t* sV = smem + kAttStages * kKVTile;
   uint8_t* sQ = smem + 2 * kAttStages * kKVTile;
   uint64_t* full = reinterpret_cast<uint64_t*>(sQ + a.NW * 16 * 256);
-  __shared__ int s_last;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmKV);
   }
+  __syncwarp();
   pdl_wait();
   pdl_launch_dependents();
 
@@ -96,7 +98,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   }
   const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m) + 1;
   const int n_tiles = (kv_end + kPage - 1) / kPage;
-  const int per = (n_tiles + a.S - 1) / a.S;
+  // at least two KV tiles per split: fewer, fuller splits keep the merge short
+  const int per = max(2, (n_tiles + a.S - 1) / a.S);
   const int t_lo = split * per;
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
   __syncthreads();
@@ -115,6 +118,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   };
   if (tid == 0)
     for (int i = 0; i < min(kAttStages, ntile); ++i) issue(i);
+  __syncwarp();
 
   // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row)
   const int rows_pad = a.NW * 16;
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     }
     __syncthreads();
     if (tid == 0 && i + kAttStages < ntile) issue(i + kAttStages);
+    __syncwarp();
   }
 
   l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
@@ -282,59 +287,68 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     return;
   }
 
-  // split keys: write the unnormalised partial, the last CTA of the group merges
-  const int unit = blockIdx.z * a.Hkv + g;
-  const size_t base = (static_cast<size_t>(unit) * a.S + split) * rows_pad;
+  // split keys: partials stay in shared memory (the K/V ring is free now), the cluster merges
+  __syncthreads();
+  float* sO = reinterpret_cast<float*>(sK);                  // [rows_pad][128]
+  float* sML = sO + static_cast<size_t>(rows_pad) * 128;     // [rows_pad][2]
   {
-    float* wo_a = a.ws_o + (base + ra) * 128;
-    float* wo_b = a.ws_o + (base + rb) * 128;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-      *reinterpret_cast<float2*>(wo_a + n * 8 + 2 * (lane & 3)) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(wo_b + n * 8 + 2 * (lane & 3)) = make_float2(o[n][2], o[n][3]);
+      *reinterpret_cast<float2*>(sO + ra * 128 + n * 8 + 2 * (lane & 3)) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(sO + rb * 128 + n * 8 + 2 * (lane & 3)) = make_float2(o[n][2], o[n][3]);
     }
     if ((lane & 3) == 0) {
-      *reinterpret_cast<float2*>(a.ws_ml + (base + ra) * 2) = make_float2(m_a, l_a);
-      *reinterpret_cast<float2*>(a.ws_ml + (base + rb) * 2) = make_float2(m_b, l_b);
+      *reinterpret_cast<float2*>(sML + ra * 2) = make_float2(m_a, l_a);
+      *reinterpret_cast<float2*>(sML + rb * 2) = make_float2(m_b, l_b);
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int old = atomicAdd(&a.counters[unit], 1);
-    s_last = (old == a.S - 1) ? 1 : 0;
-    if (s_last) a.counters[unit] = 0;
+  cluster_sync();
+  const int S = a.S;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int per_rank = (a.rows + S - 1) / S;
+  const int r0 = rank * per_rank, r1 = min(a.rows, r0 + per_rank);
+  const uint32_t o_base = smem_u32(sO), ml_base = smem_u32(sML);
+  uint32_t o_peer[8], ml_peer[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
+    ml_peer[q] = (q < S) ? dsmem_addr(ml_base, q) : 0u;
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const size_t base0 = static_cast<size_t>(unit) * a.S * rows_pad;
-  for (int e = tid; e < a.rows * 32; e += nthr) {
-    const int r = e >> 5, d4 = e & 31;
+  for (int e = tid; e < (r1 - r0) * 32; e += nthr) {
+    const int r = r0 + (e >> 5), d4 = e & 31;
     const int p = r / a.G;
     if (p >= np) continue;
+    float2 ml[8];
     float M = -INFINITY;
-    for (int s2 = 0; s2 < a.S; ++s2)
-      M = fmaxf(M, __ldcg(a.ws_ml + (base0 + static_cast<size_t>(s2) * rows_pad + r) * 2));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + r * 8) : make_float2(-INFINITY, 0.f);
+      M = fmaxf(M, ml[q].x);
+    }
+    float4 ov[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      ov[q] = (q < S && ml[q].x != -INFINITY) ? ld_dsmem_f4(o_peer[q] + (r * 128 + d4 * 4) * 4)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s2 = 0; s2 < a.S; ++s2) {
-      const size_t rr = base0 + static_cast<size_t>(s2) * rows_pad + r;
-      const float ms = __ldcg(a.ws_ml + rr * 2);
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      L += w * __ldcg(a.ws_ml + rr * 2 + 1);
-      const float4 ov = __ldcg(reinterpret_cast<const float4*>(a.ws_o + rr * 128) + d4);
-      acc.x += w * ov.x;
-      acc.y += w * ov.y;
-      acc.z += w * ov.z;
-      acc.w += w * ov.w;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < S && ml[q].x != -INFINITY) {
+        const float w = exp2f(ml[q].x - M);
+        L += w * ml[q].y;
+        acc.x += w * ov[q].x;
+        acc.y += w * ov[q].y;
+        acc.z += w * ov[q].z;
+        acc.w += w * ov[q].w;
+      }
     }
     const float inv = (L > 0.f) ? 1.f / L : 0.f;
     __nv_bfloat16* dst = out_ptr(r) + d4 * 4;
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc.x * inv, acc.y * inv);
     *reinterpret_cast<uint32_t*>(dst + 2) = pack_bf16(acc.z * inv, acc.w * inv);
   }
+  cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
 // Plain per-(token, head) attention for any head_dim <= 128 and either storage type; used by
@@ -432,8 +446,16 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchAttribute attrs[2];
+  int na = 0;
+  attrs[na].id = cudaLaunchAttributeClusterDimension;
+  attrs[na].val.clusterDim.x = a.S;
+  attrs[na].val.clusterDim.y = 1;
+  attrs[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl) attrs[na++] = attr[0];
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, attn_mma_kernel, *tmKV, a);
 }
 

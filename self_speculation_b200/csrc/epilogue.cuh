@@ -11,11 +11,16 @@
 
 namespace nld {
 
+// Per-column data of a tile, computed once per tile into shared memory (see
+// compute_tile_meta): s_inv = 1/rms of the token, s_pos = its position (-1: no KV row: column
+// past M or past the KV capacity), s_pg = the KV page holding that position.
 // red_f / red_i: shared scratch of at least 4*16 + 16 entries each.
+// Global loads of a 16-column chunk are issued together before any store of the chunk, so a
+// chunk costs one memory round trip rather than sixteen.
 template <typename T>
 NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane, int ew,
-                       int tok0, const float* s_inv, int col0, float (&v)[16], float* red_f,
-                       int* red_i) {
+                       int tok0, const float* s_inv, const int* s_pos, const int* s_pg, int col0,
+                       float (&v)[16], float* red_f, int* red_i) {
   const int row = row_tile * kTileRows + row_in_tile;
   switch (e.kind) {
     case EPI_QKV: {
@@ -33,29 +38,28 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
       const int lr = rr - head * e.hd;
       const int half = e.hd >> 1;
       const int feat = (sec == 2) ? lr : ((lr & 1) ? (lr >> 1) + half : (lr >> 1));
+      float2 cs[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int pos = s_pos[col0 + j];
+        cs[j] = (sec < 2 && pos >= 0) ? __ldg(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)])
+                                      : make_float2(1.f, 0.f);
+      }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int tok = tok0 + j;
         float x = v[j] * s_inv[col0 + j];
         const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
+        if (sec < 2) x = (lr & 1) ? (x * cs[j].x + partner * cs[j].y) : (x * cs[j].x - partner * cs[j].y);
         if (tok >= e.M || row >= e.n_rows) continue;
-        const int b = tok / e.m;
-        const int pos = e.lens[b] + (tok - b * e.m);
-        if (pos >= e.kv_cap) {
-          set_err(e.err, NLD_DEVERR_KV_OVERFLOW);
-          continue;
-        }
-        if (sec < 2) {
-          const float2 cs = e.rope[static_cast<size_t>(pos) * half + (lr >> 1)];
-          x = (lr & 1) ? (x * cs.x + partner * cs.y) : (x * cs.x - partner * cs.y);
-        }
         if (sec == 0) {
           static_cast<T*>(e.q_out)[(static_cast<size_t>(tok) * e.Hq + head) * e.hd + feat] =
               from_f32<T>(x);
         } else {
-          const int page = e.page_table[b * e.pps + (pos >> 6)];
+          const int pos = s_pos[col0 + j];
+          if (pos < 0) continue;
           const size_t off =
-              ((static_cast<size_t>(page) * 2 + (sec - 1)) * e.Hkv + head) * kPage * e.hd +
+              ((static_cast<size_t>(s_pg[col0 + j]) * 2 + (sec - 1)) * e.Hkv + head) * kPage * e.hd +
               static_cast<size_t>(pos & (kPage - 1)) * e.hd + feat;
           static_cast<T*>(e.kv_layer)[off] = from_f32<T>(x);
         }
@@ -63,14 +67,17 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
     } break;
 
     case EPI_RESID: {
+      float hv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        hv[j] = (tok0 + j < e.M) ? e.h[static_cast<size_t>(tok0 + j) * e.d + row] : 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int tok = tok0 + j;
         float hn = 0.f;
         if (tok < e.M) {
-          float* hp = e.h + static_cast<size_t>(tok) * e.d + row;
-          hn = *hp + v[j];
-          *hp = hn;
+          hn = hv[j] + v[j];
+          e.h[static_cast<size_t>(tok) * e.d + row] = hn;
           static_cast<T*>(e.hb)[static_cast<size_t>(tok) * e.d + row] = from_f32<T>(hn);
         }
         float sq = hn * hn;
@@ -180,17 +187,52 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
   }
 }
 
-// 1/rms for `n` token columns starting at tok0 into s_inv (threads et = 0..nthr-1 share it).
-NLD_DEV void compute_inv_rms(const EpiArgs& e, int tok0, int n, float* s_inv, int et, int nthr) {
-  for (int c = et; c < n; c += nthr) {
-    const int tok = tok0 + c;
-    float inv = 0.f;
-    if (tok < e.M) {
-      float acc = 0.f;
-      for (int t = 0; t < e.ssq_tiles; ++t) acc += e.ssq_in[static_cast<size_t>(t) * e.ssq_ld + tok];
-      inv = rsqrtf(acc * e.inv_d + e.eps);
+// Per-column data of a tile of n token columns starting at tok0 (see epi_chunk): 1/rms from
+// the RMSNorm statistics when `norm` (lane l of a warp sums tiles l, l+32, ... of 8 tokens at
+// once, then a shuffle reduction finishes each token), and for the QKV epilogue the position
+// and KV page of each token.  nthr threads (a multiple of 32) share the work.
+NLD_DEV void compute_tile_meta(const EpiArgs& e, int tok0, int n, bool norm, float* s_inv,
+                               int* s_pos, int* s_pg, int et, int nthr) {
+  const int nw = nthr >> 5, w = et >> 5, lane = et & 31;
+  if (norm) {
+    for (int c0 = w; c0 < n; c0 += nw * 8) {
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        acc[q] = 0.f;
+        const int c = c0 + q * nw;
+        const int tok = tok0 + c;
+        if (c < n && tok < e.M)
+          for (int t = lane; t < e.ssq_tiles; t += 32)
+            acc[q] += __ldg(&e.ssq_in[static_cast<size_t>(t) * e.ssq_ld + tok]);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float v = acc[q];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        const int c = c0 + q * nw;
+        if (lane == 0 && c < n) s_inv[c] = (tok0 + c < e.M) ? rsqrtf(v * e.inv_d + e.eps) : 0.f;
+      }
     }
-    s_inv[c] = inv;
+  }
+  if (e.kind == EPI_QKV) {
+    for (int c = et; c < n; c += nthr) {
+      const int tok = tok0 + c;
+      int pos = -1, pg = 0;
+      if (tok < e.M) {
+        const int b = tok / e.m;
+        pos = __ldg(&e.lens[b]) + (tok - b * e.m);
+        if (pos >= e.kv_cap || pos < 0) {
+          set_err(e.err, NLD_DEVERR_KV_OVERFLOW);
+          pos = -1;
+        } else {
+          pg = __ldg(&e.page_table[b * e.pps + (pos >> 6)]);
+        }
+      }
+      s_pos[c] = pos;
+      s_pg[c] = pg;
+    }
   }
 }
 

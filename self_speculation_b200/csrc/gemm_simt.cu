@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(128)
   __shared__ float Ws[kTileRows][33];
   __shared__ float Xs[16][33];
   __shared__ float s_inv[16];
+  __shared__ int s_pos[16];
+  __shared__ int s_pg[16];
   __shared__ float red_f[96];
   __shared__ int red_i[96];
   pdl_wait();
@@ -20,7 +22,7 @@ __global__ void __launch_bounds__(128)
   const int rt = blockIdx.x;
   const int tok0 = blockIdx.y * 16;
   const int tid = threadIdx.x;
-  if (e.kind != EPI_RESID) compute_inv_rms(e, tok0, 16, s_inv, tid, 128);
+  compute_tile_meta(e, tok0, 16, e.kind != EPI_RESID, s_inv, s_pos, s_pg, tid, 128);
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.f;
@@ -43,7 +45,7 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();
   }
-  epi_chunk<float>(e, rt, tid, tid & 31, tid >> 5, tok0, s_inv, 0, acc, red_f, red_i);
+  epi_chunk<float>(e, rt, tid, tid & 31, tid >> 5, tok0, s_inv, s_pos, s_pg, 0, acc, red_f, red_i);
 }
 
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,

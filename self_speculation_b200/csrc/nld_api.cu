@@ -24,7 +24,6 @@
 using namespace nld;
 
 namespace nld {
-size_t gemm_tc_smem_bytes(const GemmShape& s);
 size_t attn_mma_smem_bytes(int NW);
 cudaError_t init_kernel_attributes();
 }
@@ -105,14 +104,7 @@ struct nld_ctx {
   LmPart* lm_part = nullptr;
   int lm_tiles = 0;
   float2* rope = nullptr;
-  // scratch
-  float* ws = nullptr;
-  int* counters = nullptr;
-  float* att_o = nullptr;
-  float* att_ml = nullptr;
-  int* att_counters = nullptr;
-  size_t att_o_floats = 0;
-  int att_units_max = 0;
+  int max_clusters[9] = {0};
   int* h_pinned = nullptr;  // host: [0] error word, [1] incomplete, [2..] lens
   // tensor maps
   std::vector<CUtensorMap> tmWqkv, tmWo, tmWgu, tmWd;
@@ -204,24 +196,48 @@ struct GemmPlan {
   GemmShape s;
 };
 
+// Tiling of one projection GEMM.  Token columns: tiles of <= 256.  K: split over the CTAs of
+// a cluster (split 1..8, only for NT <= 64 where the fp32 staging buffers fit), chosen to
+// minimise waves x k-iterations per tile (+ a small per-tile cost) over the clusters that can
+// be resident at once.
 GemmShape plan_gemm(const nld_ctx* x, int n_rows, int K, int M) {
   GemmShape s{};
   s.n_rows = n_rows;
   s.K = K;
   s.M = M;
   s.tok_tiles = (M + kMaxNT - 1) / kMaxNT;
-  int per = (M + s.tok_tiles - 1) / s.tok_tiles;
+  const int per = (M + s.tok_tiles - 1) / s.tok_tiles;
   s.NT = std::max(16, (per + 15) / 16 * 16);
   s.row_tiles = (n_rows + kTileRows - 1) / kTileRows;
   s.KT = K / kTileK;
-  s.T = static_cast<long long>(s.row_tiles) * s.tok_tiles * s.KT;
-  s.G = static_cast<int>(std::min<long long>(x->sms, s.T));
+  const int tiles = s.row_tiles * s.tok_tiles;
+  long long best = -1;
+  // GEMMs with at least one tile per resident CTA keep split = 1: there the per-tile handoff
+  // of split partials would sit on every tile instead of hiding behind the next one.
+  const bool many = tiles >= x->max_clusters[1];
+  for (int split = 1; split <= 8; ++split) {
+    if (split > 1 && (s.NT > 64 || many)) break;
+    if (split > s.KT) break;
+    const int ks = (s.KT + split - 1) / split;
+    if ((split - 1) * ks >= s.KT) continue;
+    const int C = std::min(x->max_clusters[split], tiles);
+    if (C < 1) continue;
+    const long long waves = (tiles + C - 1) / C;
+    const long long cost = waves * (ks + 3);
+    if (best < 0 || cost < best) {
+      best = cost;
+      s.split = split;
+      s.ks = ks;
+      s.G = C * split;
+    }
+  }
   const int stage_bytes = kTileRows * kTileK * 2 + s.NT * 128;
-  s.stages = std::max(2, std::min(8, (200 * 1024) / stage_bytes));
+  const int staging = (s.split > 1) ? 2 * s.NT * kTileRows * 4 : 0;
+  s.stages = std::max(2, std::min(8, (216 * 1024 - staging - 4096) / stage_bytes));
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(2 * s.NT)) cols <<= 1;
   s.tmem_cols = cols;
-  s.ws_slot = kTileRows * s.NT;
+  s.trace = nullptr;
   return s;
 }
 
@@ -236,7 +252,8 @@ const CUtensorMap* xmap(nld_ctx* x, int buf, int NT) {
   return &(x->tmX[key] = m);
 }
 
-nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool pdl) {
+nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool pdl,
+                unsigned long long* trace = nullptr) {
   int n_rows, K, buf;
   const void* W;
   const CUtensorMap* tmW = nullptr;
@@ -256,9 +273,10 @@ nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool 
     return NLD_OK;
   }
   GemmShape s = plan_gemm(x, n_rows, K, M);
+  s.trace = trace;
   const CUtensorMap* tmX = xmap(x, buf, s.NT);
   if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
-  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->ws, x->counters, x->timeout_ns, pdl));
+  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->timeout_ns, pdl));
   return NLD_OK;
 }
 
@@ -268,10 +286,13 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   a.q_tiles = (m + a.QT - 1) / a.QT;
   a.rows = a.QT * a.G;
   a.NW = (a.rows + 15) / 16;
+  // KV splits of one (sequence, kv head, query tile) form a cluster of at most 8 CTAs; split
+  // only while the grid is short of two CTAs per SM, and keep >= 2 KV tiles per split
   const int units = batch * a.q_tiles * Hkv;
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   a.S = 1;
-  if (units < 2 * sms) a.S = std::max(1, std::min(n_tiles, (2 * sms + units - 1) / units));
+  if (units < 2 * sms)
+    a.S = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / 2)}));
 }
 
 EpiArgs base_epi(nld_ctx* x, int M, int m) {
@@ -356,13 +377,6 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa);
-    const int units = f.B * aa.q_tiles * aa.Hkv;
-    if (aa.S > 1 && (units > x->att_units_max ||
-                     static_cast<size_t>(units) * aa.S * aa.NW * 16 * 128 > x->att_o_floats))
-      aa.S = 1;
-    aa.ws_o = x->att_o;
-    aa.ws_ml = x->att_ml;
-    aa.counters = x->att_counters;
   } else {
     aa.G = aa.Hq / aa.Hkv;
   }
@@ -586,21 +600,9 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
   if ((s = dalloc(x, &x->attn, Mm * x->qd * el)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->ubuf, Mm * c.ffn_dim * el)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->lm_part, Mm * x->lm_tiles * sizeof(LmPart))) != NLD_OK) return bail(s);
-  // stream-K partial slots: two per CTA of at most 128 x 256 fp32
-  if ((s = dalloc(x, &x->ws, static_cast<size_t>(x->sms) * 2 * kTileRows * kMaxNT * sizeof(float))) != NLD_OK) return bail(s);
-  {
-    const int max_rows = std::max({x->qkv_rows, x->gu_rows, d, c.vocab});
-    const int n = ((max_rows + kTileRows - 1) / kTileRows) * ((x->M_max + kMaxNT - 1) / kMaxNT) + 64;
-    if ((s = dalloc(x, &x->counters, n * sizeof(int))) != NLD_OK) return bail(s);
-    if (cudaMemset(x->counters, 0, n * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
-  }
-  // attention split-KV partials: splits are only used while units*S <= ~2*SMs
-  x->att_units_max = 2 * x->sms;
-  x->att_o_floats = static_cast<size_t>(2 * x->sms + 64) * 12 * 16 * 128;
-  if ((s = dalloc(x, &x->att_o, x->att_o_floats * sizeof(float))) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->att_ml, x->att_o_floats / 64 * sizeof(float))) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->att_counters, x->att_units_max * sizeof(int))) != NLD_OK) return bail(s);
-  if (cudaMemset(x->att_counters, 0, x->att_units_max * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  // resident clusters of each split size (one GEMM CTA per SM)
+  if (x->bf16)
+    for (int sp = 1; sp <= 8; ++sp) x->max_clusters[sp] = gemm_tc_max_clusters(sp, 200 * 1024, x->sms);
   if (cudaMemset(x->err, 0, 16) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->lens, 0, B * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->h, 0, Mm * d * sizeof(float)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
@@ -969,6 +971,67 @@ nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
   return NLD_OK;
 }
 
+nld_status nld_time_gemm(nld_ctx* x, int which, int layer, int M, int reps, float* ms_out) {
+  TRY(need_started(x));
+  if (which < 0 || which > 4) return fail(x, NLD_ERR_ARG, "which must be 0..4");
+  if (layer < 0 || layer >= x->c.n_layers) return fail(x, NLD_ERR_ARG, "layer out of range");
+  if (M < 1 || M > x->M_max || M % x->batch) return fail(x, NLD_ERR_ARG, "M must be a multiple of the batch, <= %d", x->M_max);
+  if (reps < 1 || !ms_out) return fail(x, NLD_ERR_ARG, "reps >= 1 and ms_out required");
+  const int m = M / x->batch;
+  TRY(ensure_capacity(x, m));
+  EpiArgs e = base_epi(x, M, m);
+  static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
+  e.kind = kinds[which];
+  e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
+  cudaEvent_t a, b;
+  CK(cudaEventCreate(&a));
+  CK(cudaEventCreate(&b));
+  TRY(gemm(x, which, layer, M, e, false));   // warm (tensor maps, first-launch costs)
+  CK(cudaEventRecord(a, x->stream));
+  for (int i = 0; i < reps; ++i) TRY(gemm(x, which, layer, M, e, false));
+  CK(cudaEventRecord(b, x->stream));
+  CK(cudaEventSynchronize(b));
+  float ms = 0.f;
+  CK(cudaEventElapsedTime(&ms, a, b));
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  *ms_out = ms / reps;
+  return NLD_OK;
+}
+
+nld_status nld_trace_gemm(nld_ctx* x, int which, int layer, int M, unsigned long long* d_trace,
+                          int* grid_out) {
+  TRY(need_started(x));
+  if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
+  if (which < 0 || which > 4 || layer < 0 || layer >= x->c.n_layers || !d_trace || M < 1 ||
+      M > x->M_max || M % x->batch)
+    return fail(x, NLD_ERR_ARG, "bad trace arguments");
+  const int m = M / x->batch;
+  EpiArgs e = base_epi(x, M, m);
+  static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
+  e.kind = kinds[which];
+  e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
+  const int nr[5] = {x->qkv_rows, x->c.d_model, x->gu_rows, x->c.d_model, x->c.vocab};
+  const int kd[5] = {x->c.d_model, x->qd, x->c.d_model, x->c.ffn_dim, x->c.d_model};
+  if (grid_out) *grid_out = plan_gemm(x, nr[which], kd[which], M).G;
+  TRY(gemm(x, which, layer, M, e, false));
+  TRY(gemm(x, which, layer, M, e, false, d_trace));
+  CK(cudaStreamSynchronize(x->stream));
+  return NLD_OK;
+}
+
+nld_status nld_debug_gemm_plan(nld_ctx* x, int which, int M, int* out8) {
+  if (!x || !out8) return fail(x, NLD_ERR_ARG, "NULL argument");
+  if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
+  if (which < 0 || which > 4 || M < 1 || M > x->M_max) return fail(x, NLD_ERR_ARG, "bad plan arguments");
+  const int nr[5] = {x->qkv_rows, x->c.d_model, x->gu_rows, x->c.d_model, x->c.vocab};
+  const int kd[5] = {x->c.d_model, x->qd, x->c.d_model, x->c.ffn_dim, x->c.d_model};
+  const GemmShape s = plan_gemm(x, nr[which], kd[which], M);
+  const int v[8] = {s.NT, s.tok_tiles, s.row_tiles, s.KT, s.split, s.ks, s.G, s.stages};
+  for (int i = 0; i < 8; ++i) out8[i] = v[i];
+  return NLD_OK;
+}
+
 nld_status nld_debug_state(nld_ctx* x, int32_t* d_lens_out, int32_t* d_pending_out, int32_t* d_draft_out,
                            int32_t* d_verify_out) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
@@ -999,16 +1062,6 @@ const char* nld_last_error(const nld_ctx* x) {
 void* nld_stream(nld_ctx* x) { return x ? static_cast<void*>(x->stream) : nullptr; }
 
 // ----------------------------------------------------------------- stand-alone attention --
-static void attn_ws_layout(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a,
-                           size_t& cnt_bytes, size_t& ml_bytes, size_t& o_bytes) {
-  attn_plan(batch, m, Hq, Hkv, max_len, sms, a);
-  const size_t units = static_cast<size_t>(batch) * a.q_tiles * Hkv;
-  const size_t rows_pad = static_cast<size_t>(a.NW) * 16;
-  cnt_bytes = (units * sizeof(int) + 255) / 256 * 256;
-  ml_bytes = a.S > 1 ? (units * a.S * rows_pad * 2 * sizeof(float) + 255) / 256 * 256 : 0;
-  o_bytes = a.S > 1 ? units * a.S * rows_pad * 128 * sizeof(float) : 0;
-}
-
 static int device_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -1016,34 +1069,20 @@ static int device_sms() {
   return n;
 }
 
-size_t nld_attention_workspace_size(int batch, int m, int n_q_heads, int n_kv_heads, int head_dim,
-                                    int max_len) {
-  if (batch < 1 || m < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || head_dim != 128) return 0;
-  AttnArgs a{};
-  size_t c, ml, o;
-  attn_ws_layout(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a, c, ml, o);
-  return c + ml + o;
-}
-
 nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* d_page_table,
                          int pages_per_seq, int n_pages, const int32_t* d_lens, int batch, int m,
                          int n_q_heads, int n_kv_heads, int head_dim, int block_size, int max_len,
-                         void* d_out, void* d_workspace, size_t workspace_bytes, void* cuda_stream) {
-  nld_ctx* x = nullptr;
+                         void* d_out, void* cuda_stream) {
   if (!d_q || !d_kv_pool || !d_page_table || !d_lens || !d_out)
     return fail(nullptr, NLD_ERR_ARG, "NULL pointer argument");
   if (batch < 1 || m < 1 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads)
     return fail(nullptr, NLD_ERR_ARG, "bad batch/m/head counts");
   if (head_dim != 128) return fail(nullptr, NLD_ERR_UNSUPPORTED, "head_dim must be 128");
   if (block_size < 1) return fail(nullptr, NLD_ERR_ARG, "block_size must be >= 1");
-  if (max_len < m || max_len > pages_per_seq * kPage) return fail(nullptr, NLD_ERR_ARG, "max_len outside m..pages_per_seq*64");
-  if (static_cast<long long>(n_pages) * 2 * n_kv_heads * kPage > INT32_MAX) return fail(nullptr, NLD_ERR_ARG, "pool too large");
-  AttnArgs a{};
-  size_t cb, mlb, ob;
-  attn_ws_layout(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a, cb, mlb, ob);
-  if (!d_workspace || workspace_bytes < cb + mlb + ob)
-    return fail(nullptr, NLD_ERR_ARG, "workspace too small: need %zu bytes", cb + mlb + ob);
-  if (reinterpret_cast<uintptr_t>(d_workspace) % 16) return fail(nullptr, NLD_ERR_ARG, "workspace must be 16-byte aligned");
+  if (pages_per_seq < 1 || max_len < m || max_len > pages_per_seq * kPage)
+    return fail(nullptr, NLD_ERR_ARG, "max_len outside m..pages_per_seq*64");
+  if (n_pages < 1 || static_cast<long long>(n_pages) * 2 * n_kv_heads * kPage > INT32_MAX)
+    return fail(nullptr, NLD_ERR_ARG, "bad pool size");
   {
     cudaError_t ae = init_kernel_attributes();
     if (ae != cudaSuccess) {
@@ -1052,6 +1091,9 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
                   cudaGetErrorString(ae));
     }
   }
+  AttnArgs a{};
+  attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a);
+  if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))
     return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed (pool)");
@@ -1066,13 +1108,10 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   a.pps = pages_per_seq;
   a.layer_row0 = 0;
   a.block_size = block_size;
-  a.counters = static_cast<int*>(d_workspace);
-  a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(d_workspace) + cb);
-  a.ws_o = reinterpret_cast<float*>(static_cast<char*>(d_workspace) + cb + mlb);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   a.err = nullptr;
   cudaError_t e = launch_attention_mma(static_cast<cudaStream_t>(cuda_stream), &map, a, batch, false);
-  if (e != cudaSuccess) return fail(x, NLD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) return fail(nullptr, NLD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
   return NLD_OK;
 }
 

@@ -81,11 +81,12 @@ struct GemmShape {
   int tok_tiles;
   int row_tiles;
   int KT;           // K / 64
-  long long T;      // row_tiles * tok_tiles * KT  (k-iterations over all tiles)
-  int G;            // CTAs (stream-K workers)
+  int split;        // CTAs per cluster = K slices per tile (1..8)
+  int ks;           // k-iterations per slice
+  int G;            // CTAs = clusters * split
   int stages;
   uint32_t tmem_cols;  // power of two >= 2*NT
-  int ws_slot;      // floats per workspace slot (128 * NT)
+  unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
 };
 
 struct AttnArgs {
@@ -98,18 +99,16 @@ struct AttnArgs {
   int pps;
   int layer_row0;       // row of this layer's first page in the 2D pool view
   int block_size;
-  int QT, q_tiles, rows, S, NW;
-  float* ws_o;
-  float* ws_ml;
-  int* counters;
+  int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   float scale_log2;     // log2(e) / sqrt(hd)
   int* err;
 };
 
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
 cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
-                           const GemmShape& s, const EpiArgs& e, float* ws, int* counters,
-                           uint64_t timeout_ns, bool pdl);
+                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl);
+size_t gemm_tc_smem_bytes(const GemmShape& s);
+int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
                              int M, const EpiArgs& e, bool pdl);
 cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,

@@ -56,4 +56,4 @@ def test_null_arguments_rejected():
     assert lib.nld_prefill(None, None, 1, 1) == 1
     assert lib.nld_selfspec_round(None, None, None, None) == 1
     assert lib.nld_sync(None) == 1
-    assert lib.nld_attention_workspace_size(1, 32, 32, 8, 64, 128) == 0   # hd != 128
+    assert lib.nld_attention(None, None, None, 1, 1, None, 1, 32, 32, 8, 128, 1, 32, None, None) == 1

@@ -57,11 +57,9 @@ def _oracle(q, k, v, lens, m, bs):
 def _run(q, pool, perm, lens, m, bs, max_len):
     import self_speculation_b200 as nb
     B = q.shape[0]
-    ws_bytes = nb.nld_attention_workspace_size(B, m, HQ, HKV, HD, max_len)
-    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
     out = torch.empty(B, m, HQ, HD, dtype=torch.bfloat16, device="cuda")
     nb.nld_attention(q.cuda(), pool.cuda(), perm.cuda(), torch.tensor(lens, dtype=torch.int32).cuda(),
-                     bs, max_len, out, ws)
+                     bs, max_len, out)
     torch.cuda.synchronize()
     return out.cpu()
 
@@ -109,17 +107,11 @@ def test_attention_long_prefix_sampled():
         assert (got[b:b + 1].double() - want).abs().max().item() < TOL
 
 
-def test_workspace_counters_left_zero():
-    import self_speculation_b200 as nb
+def test_repeated_calls_identical():
+    """Deterministic merge order: repeated calls give bit-identical outputs."""
     lens = [500]
     m = 32
     q, k, v, pool, perm, pps = _setup(lens, m)
-    ws_bytes = nb.nld_attention_workspace_size(1, m, HQ, HKV, HD, 532)
-    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
-    out = torch.empty(1, m, HQ, HD, dtype=torch.bfloat16, device="cuda")
-    for _ in range(3):
-        nb.nld_attention(q.cuda(), pool.cuda(), perm.cuda(), torch.tensor(lens, dtype=torch.int32).cuda(),
-                         32, 532, out, ws)
-    torch.cuda.synchronize()
-    units = 1 * 1 * HKV
-    assert int(ws[:units * 4].view(torch.int32).abs().sum()) == 0
+    a = _run(q, pool, perm, lens, m, 32, 532)
+    b = _run(q, pool, perm, lens, m, 32, 532)
+    assert torch.equal(a, b)

@@ -217,7 +217,9 @@ def test_ar_steps_track_oracle_teacher_forced():
 
 
 def test_batch_rows_independent():
-    """A sequence's logits do not depend on the other sequences of the batch."""
+    """A sequence's logits do not depend on the other sequences of the batch beyond rounding:
+    a different batch changes the GEMM tiling (summation order, then bf16 activation rounding),
+    so the bar is the logit bar itself, plus argmax agreement where the margin is clear."""
     p = synth.prompt_tokens(3, 80, CFG.vocab, seed=10)
     ctx, _, _ = make_pair(CFG)
     ctx.nld_prefill(p.cuda())
@@ -225,4 +227,6 @@ def test_batch_rows_independent():
     ctx1, _, _ = make_pair(CFG)
     ctx1.nld_prefill(p[1:2].cuda())
     one = gpu_logits(ctx1, 1, 1, CFG.block_k)
-    assert (all3[1] - one[0]).abs().max().item() < 1e-3
+    assert (all3[1] - one[0]).abs().max().item() < TOL
+    sure = top2_margin(one[0]) > MARGIN
+    assert torch.equal(all3[1].argmax(-1)[sure], one[0].argmax(-1)[sure])
