@@ -118,11 +118,14 @@ def dist_setup():
 
 
 def reduce(vals, op, world):
+    """Replica timing reduction: max (time) or sum (tokens) over ranks.  The only collective of
+    a multi-GPU run; the decode round itself exchanges nothing between replicas."""
     import torch
     if world == 1:
         return vals
     import torch.distributed as dist
-    t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(vals, dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return t.tolist()
 

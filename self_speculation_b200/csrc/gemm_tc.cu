@@ -84,7 +84,8 @@ NLD_DEV bool epi_wait(uint64_t* bar, uint32_t parity, bool cluster_acquire, uint
 template <int EPI, typename T>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const GemmShape s, const EpiArgs e_in, const uint64_t timeout_ns) {
+                   const __grid_constant__ CUtensorMap tmWn, const GemmShape s, const EpiArgs e_in,
+                   const uint64_t timeout_ns) {
   EpiArgs e = e_in;
   e.kind = EPI;   // compile-time epilogue: each instantiation holds one kind's code
   extern __shared__ uint8_t smem_raw[];
@@ -183,6 +184,17 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_2d(sX + i * xbytes, &tmX, &tail->full[i], pre_k[i] * kTileK, pre_tt[i] * s.NT);
       }
       trace_mark(s, 3);
+      if (ok && s.next_valid && blockIdx.x < s.next_clusters * s.next_split) {
+        // warm L2 (and address translation) for this CTA index's first boxes of the next GEMM
+        const int nrank = blockIdx.x % s.next_split;
+        const int ncl = blockIdx.x / s.next_split;
+        if (ncl < s.next_tiles) {
+          const int nr = ncl / s.next_tok_tiles;
+          const int lo = nrank * s.next_ks;
+          const int hi = min(s.next_KT, min(lo + s.next_ks, lo + s.next_boxes));
+          for (int kt = lo; kt < hi; ++kt) tma_prefetch_l2_2d(&tmWn, kt * kTileK, nr * kTileRows);
+        }
+      }
       if (!ok) {
         // let every load already issued land before the CTA can exit
         const int first = it - S > 0 ? it - S : 0;
@@ -379,7 +391,9 @@ int gemm_tc_max_clusters(int split, size_t smem, int sms) {
 }
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
-                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl) {
+                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl,
+                           const CUtensorMap* tmW_next) {
+  const CUtensorMap* wn = tmW_next ? tmW_next : tmW;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s.G);
   cfg.blockDim = dim3(192);
@@ -401,19 +415,19 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtens
   cfg.numAttrs = na;
   switch (e.kind) {
     case EPI_QKV:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV, __nv_bfloat16>, *tmW, *tmX, s, e,
+      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
                                 timeout_ns);
     case EPI_RESID:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_RESID, __nv_bfloat16>, *tmW, *tmX, s, e,
+      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_RESID, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
                                 timeout_ns);
     case EPI_SWIGLU:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_SWIGLU, __nv_bfloat16>, *tmW, *tmX, s, e,
+      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_SWIGLU, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
                                 timeout_ns);
     case EPI_LMHEAD:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LMHEAD, __nv_bfloat16>, *tmW, *tmX, s, e,
+      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LMHEAD, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
                                 timeout_ns);
     default:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LOGITS, __nv_bfloat16>, *tmW, *tmX, s, e,
+      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LOGITS, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
                                 timeout_ns);
   }
 }

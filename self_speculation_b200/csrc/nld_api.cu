@@ -252,8 +252,26 @@ const CUtensorMap* xmap(nld_ctx* x, int buf, int NT) {
   return &(x->tmX[key] = m);
 }
 
+// Weight matrix, its tensor map and shape of projection `which` of `layer`.
+struct WInfo {
+  int n_rows, K, buf;
+  const void* W;
+  const CUtensorMap* map;
+};
+WInfo winfo(nld_ctx* x, int which, int layer) {
+  WInfo w{};
+  switch (which) {
+    case GW_QKV: w = {x->qkv_rows, x->c.d_model, XB_HB, x->wqkv[layer], x->bf16 ? &x->tmWqkv[layer] : nullptr}; break;
+    case GW_O: w = {x->c.d_model, x->qd, XB_ATTN, x->wo[layer], x->bf16 ? &x->tmWo[layer] : nullptr}; break;
+    case GW_GU: w = {x->gu_rows, x->c.d_model, XB_HB, x->wgu[layer], x->bf16 ? &x->tmWgu[layer] : nullptr}; break;
+    case GW_D: w = {x->c.d_model, x->c.ffn_dim, XB_U, x->wd[layer], x->bf16 ? &x->tmWd[layer] : nullptr}; break;
+    default: w = {x->c.vocab, x->c.d_model, XB_HB, x->wlm, x->bf16 ? &x->tmWlm : nullptr}; break;
+  }
+  return w;
+}
+
 nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool pdl,
-                unsigned long long* trace = nullptr) {
+                unsigned long long* trace = nullptr, int next_which = -1, int next_layer = 0) {
   int n_rows, K, buf;
   const void* W;
   const CUtensorMap* tmW = nullptr;
@@ -274,9 +292,23 @@ nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool 
   }
   GemmShape s = plan_gemm(x, n_rows, K, M);
   s.trace = trace;
+  const CUtensorMap* tmWn = nullptr;
+  if (next_which >= 0) {
+    const WInfo nw = winfo(x, next_which, next_layer);
+    const GemmShape n = plan_gemm(x, nw.n_rows, nw.K, M);
+    s.next_valid = 1;
+    s.next_split = n.split;
+    s.next_tok_tiles = n.tok_tiles;
+    s.next_ks = n.ks;
+    s.next_KT = n.KT;
+    s.next_clusters = n.G / n.split;
+    s.next_tiles = n.row_tiles * n.tok_tiles;
+    s.next_boxes = n.stages;
+    tmWn = nw.map;
+  }
   const CUtensorMap* tmX = xmap(x, buf, s.NT);
   if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
-  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->timeout_ns, pdl));
+  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->timeout_ns, pdl, tmWn));
   return NLD_OK;
 }
 
@@ -385,7 +417,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
     EpiArgs e = base_epi(x, M, f.m);
     e.kind = EPI_QKV;
     e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
-    TRY(gemm(x, GW_QKV, l, M, e, pdl));
+    TRY(gemm(x, GW_QKV, l, M, e, pdl, nullptr, GW_O, l));
     if (x->bf16) {
       aa.layer_row0 = l * x->n_pages * 2 * x->c.n_kv_heads * kPage;
       CK(launch_attention_mma(x->stream, &x->tmKV, aa, f.B, pdl));
@@ -393,12 +425,15 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
       aa.pool = e.kv_layer;
       CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
     }
+    const bool last = (l + 1 == x->c.n_layers);
     e.kind = EPI_RESID;
-    TRY(gemm(x, GW_O, l, M, e, pdl));
+    TRY(gemm(x, GW_O, l, M, e, pdl, nullptr, GW_GU, l));
     e.kind = EPI_SWIGLU;
-    TRY(gemm(x, GW_GU, l, M, e, pdl));
+    TRY(gemm(x, GW_GU, l, M, e, pdl, nullptr, GW_D, l));
     e.kind = EPI_RESID;
-    TRY(gemm(x, GW_D, l, M, e, pdl));
+    if (!last) TRY(gemm(x, GW_D, l, M, e, pdl, nullptr, GW_QKV, l + 1));
+    else if (f.lm != LM_NONE) TRY(gemm(x, GW_D, l, M, e, pdl, nullptr, GW_LM, 0));
+    else TRY(gemm(x, GW_D, l, M, e, pdl));
   }
   if (f.lm != LM_NONE) {
     EpiArgs e = base_epi(x, M, f.m);

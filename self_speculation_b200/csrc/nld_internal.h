@@ -87,6 +87,10 @@ struct GemmShape {
   int stages;
   uint32_t tmem_cols;  // power of two >= 2*NT
   unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
+  // the projection GEMM that runs next on the stream (its weights are independent of this
+  // one's output): each CTA prefetches into L2 the first weight boxes it will load there
+  int next_valid;
+  int next_split, next_tok_tiles, next_ks, next_KT, next_clusters, next_tiles, next_boxes;
 };
 
 struct AttnArgs {
@@ -106,7 +110,8 @@ struct AttnArgs {
 
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
 cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
-                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl);
+                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl,
+                           const CUtensorMap* tmW_next);
 size_t gemm_tc_smem_bytes(const GemmShape& s);
 int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
