@@ -407,27 +407,25 @@ def run_probe(args):
         plans[nm] = ctx.nld_debug_gemm_plan(w, K_BLOCK + 1)
     ctx.nld_selfspec_round(toks, nc, None)
     ctx.nld_sync()
-    phases = ["start", "setup", "tma0", "tmaN", "mma0", "acc0", "acc1", "epi0", "epi1",
-              "epi0end", "epi1end", "exit", "fin_start", "fin_c0_loaded", "fin_c0_epi", "exit_epi"]
-    traces = {}
-    for w, nm in enumerate(["qkv", "o", "gate_up", "down", "lm_head"]):
-        tr = torch.zeros(148 * 16, dtype=torch.int64, device="cuda")
-        G = ctx.nld_trace_gemm(w, 0, K_BLOCK + 1, tr)
-        t = tr.view(148, 16)[:G, :16].cpu().double()
-        t0 = t[:, 0].min()
-        rel = {}
-        for i, ph in enumerate(phases):
-            col = t[:, i]
-            col = col[col > 0] - t0
-            if len(col):
-                rel[ph] = [round(float(col.min()) / 1e3, 2), round(float(col.median()) / 1e3, 2),
-                           round(float(col.max()) / 1e3, 2)]
-        traces[nm] = rel
+    # full decode chain of layer 0 (O, gate/up, down, QKV of layer 1)
+    names = ["start", "setup"] + [f"{k}{p}" for p in range(4) for k in ("w0_", "epi_go_", "epi_done_")] \
+        + ["mma_last", "exit"]
+    tr = torch.zeros(148 * 16 + 256, dtype=torch.int64, device="cuda")
+    G = ctx.nld_trace_chain(0, K_BLOCK + 1, tr)
+    t = tr[:148 * 16].view(148, 16)[:G].cpu().double()
+    t0 = t[:, 0].min()
+    traces = {"ctas": G}
+    for i, ph in enumerate(names):
+        col = t[:, i]
+        col = col[col > 0] - t0
+        if len(col):
+            traces[ph] = [round(float(col.min()) / 1e3, 2), round(float(col.median()) / 1e3, 2),
+                          round(float(col.max()) / 1e3, 2)]
     ctx.close()
     torch.cuda.synchronize()
     print(json.dumps({"probe_ms": out}))
     print(json.dumps({"plans": plans}))
-    print(json.dumps({"trace_us_min_med_max": traces}, indent=1))
+    print(json.dumps({"chain_trace_us_min_med_max": traces}))
 
 
 def main():

@@ -173,6 +173,13 @@ nld_status nld_time_gemm(nld_ctx* ctx, int which, int layer, int M, int reps, fl
 nld_status nld_trace_gemm(nld_ctx* ctx, int which, int layer, int M, unsigned long long* d_trace,
                           int* grid_out);
 
+/* Profiling hook: one traced launch of the decode chain of `layer` (O-proj, gate/up, down,
+ * then layer+1's QKV) over M token rows (as nld_time_gemm, 0 <= layer < n_layers-1); d_trace
+ * receives per CTA 16 globaltimer stamps (ns): 0 start, 1 set-up done, for phase p = 0..3:
+ * 2+3p first weight load issued, 3+3p epilogue released by the phase counter, 4+3p epilogue
+ * done; 14 last MMA commit, 15 exit.  *grid_out = CTAs.  Synchronises. */
+nld_status nld_trace_chain(nld_ctx* ctx, int layer, int M, unsigned long long* d_trace, int* grid_out);
+
 /* Profiling hook: the tiling chosen for projection GEMM `which` (as in nld_time_gemm) over M
  * token rows: out8 = {NT, token tiles, row tiles, k-iterations, split (cluster size),
  * k-iterations per split, CTAs, pipeline stages}.  No GPU work. */

@@ -63,6 +63,7 @@ def load_library() -> ctypes.CDLL:
         "nld_time_gemm": ([P, I, I, I, I, ctypes.POINTER(F)], I),
         "nld_trace_gemm": ([P, I, I, I, P, ctypes.POINTER(I)], I),
         "nld_debug_gemm_plan": ([P, I, I, ctypes.POINTER(I)], I),
+        "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
@@ -172,6 +173,11 @@ class Context:
         g = ctypes.c_int(0)
         self._check(self.lib.nld_trace_gemm(self.h, which, layer, M, _ptr(trace), ctypes.byref(g)),
                     self.h)
+        return g.value
+
+    def nld_trace_chain(self, layer: int, M: int, trace) -> int:
+        g = ctypes.c_int(0)
+        self._check(self.lib.nld_trace_chain(self.h, layer, M, _ptr(trace), ctypes.byref(g)), self.h)
         return g.value
 
     def nld_debug_gemm_plan(self, which: int, M: int) -> dict:

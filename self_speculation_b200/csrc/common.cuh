@@ -213,6 +213,36 @@ NLD_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+NLD_DEV void mbar_arrive_remote_count(uint32_t cluster_addr, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+               "r"(count)
+               : "memory");
+}
+// Generic-proxy writes of other CTAs (made visible by a gpu-scope acquire) before this thread's
+// later async-proxy (TMA) reads of the same global memory.
+NLD_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+NLD_DEV unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait until *p >= target (gpu-scope acquire).  Returns false on timeout.
+NLD_DEV bool wait_counter(const unsigned* p, unsigned target, uint64_t timeout_ns) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (ld_acquire_gpu(p) >= target) return true;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+// L2 prefetch of a contiguous global range (16-byte aligned, size a multiple of 16).
+NLD_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
 NLD_DEV bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -234,37 +234,56 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 }
 
 // -------------------------------------------------------------------------------- repack --
-// dst[r, c] = src[row_map[r], c] * gamma[c]  (gamma: RMSNorm gain folded into the projection
-// that follows the norm).
+// dst <- src[row_map[r], c] * gamma[c]  (gamma: RMSNorm gain folded into the projection that
+// follows the norm).  Row-major dst[r, c], or, with `tiled`, the streaming layout of the
+// tensor-core GEMM: 128-row x 64-column blocks stored contiguously (16 KB of bf16 each), block
+// (row tile rt, k tile kt) at element offset (rt * KT + kt) * 8192, rows past n_rows zero.
 template <typename T>
 __global__ void repack_kernel(T* __restrict__ dst, const T* __restrict__ src,
                               const int* __restrict__ row_map, int n_rows, int K,
-                              const T* __restrict__ gamma) {
-  const size_t total = static_cast<size_t>(n_rows) * K;
+                              const T* __restrict__ gamma, int tiled) {
+  const int row_tiles = (n_rows + kTileRows - 1) / kTileRows;
+  const int KT = K / kTileK;
+  const size_t total = tiled ? static_cast<size_t>(row_tiles) * kTileRows * K
+                             : static_cast<size_t>(n_rows) * K;
   for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(idx / K);
-    const int c = static_cast<int>(idx - static_cast<size_t>(r) * K);
-    const int sr = row_map ? row_map[r] : r;
-    float v = to_f32<T>(src[static_cast<size_t>(sr) * K + c]);
-    if (gamma) v *= to_f32<T>(gamma[c]);
+    int r, c;
+    if (tiled) {
+      const size_t blk = idx / (kTileRows * kTileK);
+      const int in = static_cast<int>(idx - blk * (kTileRows * kTileK));
+      const int rt = static_cast<int>(blk / KT);
+      const int kt = static_cast<int>(blk - static_cast<size_t>(rt) * KT);
+      r = rt * kTileRows + in / kTileK;
+      c = kt * kTileK + in % kTileK;
+    } else {
+      r = static_cast<int>(idx / K);
+      c = static_cast<int>(idx - static_cast<size_t>(r) * K);
+    }
+    float v = 0.f;
+    if (r < n_rows) {
+      const int sr = row_map ? row_map[r] : r;
+      v = to_f32<T>(src[static_cast<size_t>(sr) * K + c]);
+      if (gamma) v *= to_f32<T>(gamma[c]);
+    }
     dst[idx] = from_f32<T>(v);
   }
 }
 
 cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
-                          int n_rows, int K, const void* gamma, bool bf16) {
+                          int n_rows, int K, const void* gamma, bool bf16, bool tiled) {
   const int threads = 256;
-  const size_t total = static_cast<size_t>(n_rows) * K;
+  const size_t total = static_cast<size_t>((n_rows + kTileRows - 1) / kTileRows) * kTileRows * K;
   const int blocks = static_cast<int>(std::min<size_t>((total + threads - 1) / threads, 65536));
   if (bf16)
     repack_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
         static_cast<__nv_bfloat16*>(dst), static_cast<const __nv_bfloat16*>(src), row_map, n_rows,
-        K, static_cast<const __nv_bfloat16*>(gamma));
+        K, static_cast<const __nv_bfloat16*>(gamma), tiled ? 1 : 0);
   else
     repack_kernel<float><<<blocks, threads, 0, st>>>(static_cast<float*>(dst),
                                                      static_cast<const float*>(src), row_map,
-                                                     n_rows, K, static_cast<const float*>(gamma));
+                                                     n_rows, K, static_cast<const float*>(gamma),
+                                                     tiled ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -14,13 +14,15 @@ namespace nld {
 // Per-column data of a tile, computed once per tile into shared memory (see
 // compute_tile_meta): s_inv = 1/rms of the token, s_pos = its position (-1: no KV row: column
 // past M or past the KV capacity), s_pg = the KV page holding that position.
-// red_f / red_i: shared scratch of at least 4*16 + 16 entries each.
+// red_f / red_i: shared scratch of at least 4*16 + 16 entries each, private to the 4 warps (one
+// per TMEM lane quarter, 128 threads) that call this together and synchronise on named
+// barrier `bar_id`.
 // Global loads of a 16-column chunk are issued together before any store of the chunk, so a
 // chunk costs one memory round trip rather than sixteen.
 template <typename T>
 NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane, int ew,
                        int tok0, const float* s_inv, const int* s_pos, const int* s_pg, int col0,
-                       float (&v)[16], float* red_f, int* red_i) {
+                       float (&v)[16], float* red_f, int* red_i, int bar_id) {
   const int row = row_tile * kTileRows + row_in_tile;
   switch (e.kind) {
     case EPI_QKV: {
@@ -85,7 +87,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
         if (lane == 0) red_f[ew * 16 + j] = sq;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
       if (row_in_tile < 16) {
         const int j = row_in_tile;
         const int tok = tok0 + j;
@@ -94,7 +96,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
           e.ssq_out[static_cast<size_t>(row_tile) * e.ssq_ld + tok] = s;
         }
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
     } break;
 
     case EPI_SWIGLU: {
@@ -106,7 +108,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
         if (tok < e.M && !(lane & 1)) {
           const float g = x, u = partner;
-          const float act = g / (1.0f + expf(-g)) * u;
+          const float act = __fdividef(g, 1.0f + __expf(-g)) * u;   // silu(g) * u
           static_cast<T*>(e.u_out)[static_cast<size_t>(tok) * e.F + f] = from_f32<T>(act);
         }
       }
@@ -143,7 +145,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
           red_i[ew * 16 + j] = ix;
         }
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
       if (row_in_tile < 16) {
         const int j = row_in_tile;
         float mx = red_f[j];
@@ -159,7 +161,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         red_f[64 + j] = mx;
         red_i[64 + j] = ix;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
       // pass 2: sum over the tile of exp(l - tile max)
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -169,7 +171,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) red_f[ew * 16 + j] = s;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
       if (row_in_tile < 16) {
         const int j = row_in_tile;
         const int tok = tok0 + j;
@@ -182,7 +184,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
           e.lm_part[static_cast<size_t>(tok) * e.lm_tiles + row_tile] = p;
         }
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(bar_id, 128);
     } break;
   }
 }

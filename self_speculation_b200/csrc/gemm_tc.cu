@@ -1,25 +1,29 @@
-// Projection GEMM on the 5th-generation tensor cores (tcgen05), Y^T = W * X^T.
+// Projection GEMMs on the 5th-generation tensor cores (tcgen05), Y^T = W * X^T, run as a
+// persistent chain: one launch executes up to four projections back to back (for a decode
+// layer: O-proj, gate/up, down, and the next layer's QKV).
 //
 // Swap-AB: the weight matrix W [n_rows, K] is the MMA's M=128 operand and the few token rows
-// X [M, K] are its N operand (N = 16..256), so a decode forward with 32 or 33 tokens per
-// sequence streams every weight byte exactly once.
+// X [M, K] are its N operand (N = 16..256), so a decode forward streams every weight byte once.
+// Weights are stored pre-tiled (128 x 64 blocks, 16 KB contiguous), so each TMA box is one
+// contiguous read and a CTA's K range is one contiguous stretch of HBM.
 //
-// Split-K across a thread-block cluster: the `split` CTAs of a cluster share each output tile
-// (128 weight rows x NT tokens); rank r streams the r-th K slice of the tile into its own
-// tensor-memory accumulator.  The partials meet in shared memory: every rank copies its
-// accumulator into a staging buffer, tells the other ranks with a remote mbarrier arrive, and
-// then reduces one slice of the tile's token columns by reading all ranks' staging buffers over
-// distributed shared memory (in rank order, so sums do not depend on timing) and runs the fused
-// epilogue on that slice.  Clusters are persistent: cluster c handles tiles c, c+C, ...  With
-// split = 1 (large token counts) a tile is finished straight from tensor memory.
+// Work split: the CTAs of a cluster (CS of them) share output tiles; in a phase with split s
+// (a divisor of CS) each group of s ranks splits the K range of a tile, each rank accumulating
+// its slice in tensor memory.  The partials meet in shared memory: every rank copies its
+// accumulator into a staging buffer, tells its group with remote mbarrier arrives, reduces one
+// slice of the tile's token columns by reading the group's staging buffers over distributed
+// shared memory (rank order: sums do not depend on timing) and runs the fused epilogue on it.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads (W with an evict-first L2 hint), warp 1
-// owns tensor memory and issues tcgen05.mma from one thread, warps 2..5 run the epilogue.  A
-// `stages`-deep ring of shared-memory stages (16 KB of W + NT*128 B of X each) is guarded by
-// full/empty mbarriers; two TMEM accumulators and two staging buffers let the epilogue of one
-// tile overlap the MMAs of the next.  Under programmatic dependent launch the first `stages`
-// weight tiles are requested before waiting for the previous kernel; activations are read only
-// after the wait.  Every wait is bounded (timeout -> device error word, orderly exit).
+// Phases: a CTA that finished its part of phase p adds one to a grid-wide arrival counter; the
+// next phase's activation loads and epilogue wait until every CTA has arrived.  Its weight
+// loads do not wait: the producer keeps the shared-memory ring full with the next phase's
+// weights across the transition, so HBM stays busy while the last tiles of a phase finish.
+// The first phase waits for the previous kernel the same way (programmatic dependent launch).
+//
+// Warp roles (320 threads): warp 0 issues TMA loads (W with an evict-first L2 hint), warp 1
+// owns tensor memory and issues tcgen05.mma from one thread, warps 2..9 run the epilogue: two
+// warps per TMEM lane quarter, alternating 16-column chunks.
+// Every wait is bounded (timeout -> device error word, orderly exit).
 #include <algorithm>
 
 #include "common.cuh"
@@ -32,14 +36,16 @@ namespace {
 constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB of bf16 weights per stage
 constexpr int kMaxStages = 8;
 constexpr int kMaxSplit = 8;
+constexpr int kEpiThreads = 256;   // 8 epilogue warps
+constexpr int kThreads = 64 + kEpiThreads;
 
 struct GemmTail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t sfull[2];    // staging buffer b holds every rank's partial (count: split)
-  uint64_t sempty[2];   // every rank has finished reading staging buffer b (count: split)
+  uint64_t sfull[2];    // staging buffer b holds every group rank's partial (count: CS)
+  uint64_t sempty[2];   // every group rank has finished reading staging buffer b (count: CS)
   uint32_t tmem_base;
   volatile int abort_flag;
   volatile int epi_abort;
@@ -47,13 +53,39 @@ struct GemmTail {
   float inv[kMaxNT];
   int pos[kMaxNT];
   int pg[kMaxNT];
-  float red_f[96];
-  int red_i[96];
+  float red_f[2][96];   // per epilogue half
+  int red_i[2][96];
 };
 
-// Phase timestamps of one CTA (profiling hook): slot i of trace[cta * 16 + i].
-NLD_DEV void trace_mark(const GemmShape& s, int slot) {
-  if (s.trace) s.trace[blockIdx.x * 16 + slot] = globaltimer_ns();
+// Work of one CTA in phase p: its group of s ranks, the group's tiles and this rank's K slice.
+struct Work {
+  int s, grank, grp, ngrp, tiles, k_lo, k_hi;
+};
+
+NLD_DEV Work work_of(const ChainArgs& A, int p, int cl, int rank, int C) {
+  const PhaseArgs& P = A.ph[p];
+  Work w;
+  w.s = P.s;
+  const int gpc = A.CS / P.s;
+  w.grank = rank % P.s;
+  w.grp = cl * gpc + rank / P.s;
+  w.ngrp = C * gpc;
+  w.tiles = P.row_tiles * P.tok_tiles;
+  w.k_lo = w.grank * P.ks;
+  w.k_hi = min(P.KT, w.k_lo + P.ks);
+  return w;
+}
+
+// Phase timestamps of one CTA (profiling hook), trace[cta * 16 + slot]: 0 start, 1 set-up
+// done, per phase p: 2+3p first weight load issued, 3+3p epilogue may start (after the phase
+// counter), 4+3p epilogue done; 14 last MMA commit, 15 exit.
+NLD_DEV void trace_mark(const ChainArgs& A, int slot) {
+  if (A.trace) A.trace[blockIdx.x * 16 + slot] = globaltimer_ns();
+}
+// Per-iteration pipeline stamps of CTA 0 (profiling hook): after the per-CTA slots.
+NLD_DEV void trace_iter(const ChainArgs& A, int kind, int it) {
+  if (A.trace && blockIdx.x == 0 && it >= 0 && it < 64)
+    A.trace[148 * 16 + kind * 64 + it] = globaltimer_ns();
 }
 
 NLD_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, GemmTail* tail,
@@ -66,7 +98,7 @@ NLD_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, 
 }
 
 // Epilogue-side wait: a thread whose wait ran out raises epi_abort before the barrier and every
-// epilogue thread reads it after the barrier, so they leave the tile loop together.
+// epilogue thread reads it after the barrier, so they leave together.
 NLD_DEV bool epi_wait(uint64_t* bar, uint32_t parity, bool cluster_acquire, uint64_t timeout_ns,
                       GemmTail* tail, int* err) {
   const bool ok = cluster_acquire ? mbar_wait_cluster(bar, parity, timeout_ns)
@@ -75,40 +107,36 @@ NLD_DEV bool epi_wait(uint64_t* bar, uint32_t parity, bool cluster_acquire, uint
     tail->epi_abort = 1;
     set_err(err, NLD_DEVERR_TIMEOUT);
   }
-  named_bar_sync(1, 128);
+  named_bar_sync(1, kEpiThreads);
   return tail->epi_abort == 0;
 }
 
 }  // namespace
 
-template <int EPI, typename T>
-__global__ void __launch_bounds__(192, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const __grid_constant__ CUtensorMap tmWn, const GemmShape s, const EpiArgs e_in,
-                   const uint64_t timeout_ns) {
-  EpiArgs e = e_in;
-  e.kind = EPI;   // compile-time epilogue: each instantiation holds one kind's code
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_chain_kernel(const __grid_constant__ ChainArgs A, const uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int S = s.stages;
-  const int xbytes = s.NT * 128;
-  const int split = s.split;
+  const int S = A.stages;
+  const int NT = A.NT;
+  const int xbytes = NT * 128;
+  const int CS = A.CS;
   uint8_t* sW = smem;
   uint8_t* sX = smem + S * kStageW;
-  float* staging = reinterpret_cast<float*>(sX + S * xbytes);          // [2][NT][128] if split>1
-  const int stg_floats = (split > 1) ? s.NT * kTileRows : 0;
+  float* staging = reinterpret_cast<float*>(sX + S * xbytes);          // [2][NT][128] if CS>1
+  const int stg_floats = (CS > 1) ? NT * kTileRows : 0;
   GemmTail* tail = reinterpret_cast<GemmTail*>(staging + 2 * stg_floats);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rank = (split > 1) ? static_cast<int>(cluster_ctarank()) : 0;
-  const int cl = blockIdx.x / split;
-  const int C = gridDim.x / split;
-  const int tiles = s.row_tiles * s.tok_tiles;
-  const int k_lo = rank * s.ks;
-  const int k_hi = min(s.KT, k_lo + s.ks);
-  if (threadIdx.x == 0) trace_mark(s, 0);
+  const int rank = (CS > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+  const int cl = blockIdx.x / CS;
+  const int C = gridDim.x / CS;
+  const unsigned G = gridDim.x;
+  int* err = A.ph[0].e.err;
+  if (threadIdx.x == 0) trace_mark(A, 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -117,82 +145,104 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tail->tfull[i], 1);
-      mbar_init(&tail->tempty[i], 128);
-      mbar_init(&tail->sfull[i], split);
-      mbar_init(&tail->sempty[i], split);
+      mbar_init(&tail->tempty[i], kEpiThreads);
+      mbar_init(&tail->sfull[i], CS);
+      mbar_init(&tail->sempty[i], CS);
     }
     tail->abort_flag = 0;
     tail->epi_abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmW);
-    tma_prefetch_desc(&tmX);
+    for (int p = 0; p < A.nph; ++p) {
+      tma_prefetch_desc(&A.ph[p].tmW);
+      tma_prefetch_desc(&A.ph[p].tmX);
+    }
   }
   __syncwarp();
   if (warp == 1) {
-    tmem_alloc(&tail->tmem_base, s.tmem_cols);
+    tmem_alloc(&tail->tmem_base, A.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (split > 1) cluster_sync();   // every rank's barriers exist before any remote arrive
+  if (CS > 1) cluster_sync();   // every rank's barriers exist before any remote arrive
   const uint32_t tmem = tail->tmem_base;
-  const uint32_t buf_cols = s.tmem_cols / 2;
+  const uint32_t buf_cols = A.tmem_cols / 2;
   pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------- TMA producer --
       const uint64_t pol = l2_policy_evict_first();
-      int pre_k[kMaxStages], pre_tt[kMaxStages];
-      int npre = 0;
-      bool waited = false;
+      int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages];
       int it = 0;
       bool ok = true;
-      for (int t = cl; ok && t < tiles; t += C) {
-        const int r = t / s.tok_tiles;
-        const int tt = t - r * s.tok_tiles;
-        for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
-          const int stage = it % S;
-          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-          if (!wait_or_abort(&tail->empty[stage], ph ^ 1u, timeout_ns, tail, e.err)) {
-            ok = false;
-            break;
-          }
-          if (it == 0) trace_mark(s, 2);
-          mbar_arrive_expect_tx(&tail->full[stage], kStageW + xbytes);
-          tma_load_2d_hint(sW + stage * kStageW, &tmW, &tail->full[stage], kt * kTileK,
-                           r * kTileRows, pol);
-          if (waited) {
-            tma_load_2d(sX + stage * xbytes, &tmX, &tail->full[stage], kt * kTileK, tt * s.NT);
+      for (int p = 0; ok && p < A.nph; ++p) {
+        const PhaseArgs& P = A.ph[p];
+        const Work w = work_of(A, p, cl, rank, C);
+        // activation loads of this phase wait for the previous kernel (p == 0) or for every
+        // CTA to finish phase p-1; weight loads run ahead into the free stages meanwhile
+        bool ready = false;
+        int nq = 0;
+        auto become_ready = [&]() -> bool {
+          if (p == 0) {
+            pdl_wait();
           } else {
-            pre_k[npre] = kt;
-            pre_tt[npre] = tt;
-            if (++npre == S) {
-              pdl_wait();
-              waited = true;
-              for (int i = 0; i < npre; ++i)
-                tma_load_2d(sX + i * xbytes, &tmX, &tail->full[i], pre_k[i] * kTileK,
-                            pre_tt[i] * s.NT);
+            if (!wait_counter(A.bar + (p - 1), G, timeout_ns)) {
+              tail->abort_flag = 1;
+              set_err(err, NLD_DEVERR_TIMEOUT);
+              return false;
+            }
+            fence_proxy_async_global();
+          }
+          for (int i = 0; i < nq; ++i)
+            tma_load_2d(sX + q_stage[i] * xbytes, &P.tmX, &tail->full[q_stage[i]], q_k[i] * kTileK,
+                        q_tt[i] * NT);
+          nq = 0;
+          ready = true;
+          return true;
+        };
+        for (int t = w.grp; ok && t < w.tiles; t += w.ngrp) {
+          const int r = t / P.tok_tiles;
+          const int tt = t - r * P.tok_tiles;
+          for (int kt = w.k_lo; kt < w.k_hi; ++kt, ++it) {
+            const int stage = it % S;
+            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+            // a slot still holding an earlier phase's stage frees without the grid counter; once
+            // the ring holds only this phase's stages (nq == S) the counter is waited on (below)
+            if (!wait_or_abort(&tail->empty[stage], ph ^ 1u, timeout_ns, tail, err)) {
+              ok = false;
+              break;
+            }
+            if (kt == w.k_lo && t == w.grp) trace_mark(A, 2 + 3 * p);
+            trace_iter(A, 2, it - S);
+            trace_iter(A, 0, it);
+            mbar_arrive_expect_tx(&tail->full[stage], kStageW + xbytes);
+            // weights are pre-tiled: block (r, kt) is one contiguous 16 KB box
+            tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], 0,
+                             (r * P.KT + kt) * kTileRows, pol);
+            if (ready) {
+              tma_load_2d(sX + stage * xbytes, &P.tmX, &tail->full[stage], kt * kTileK, tt * NT);
+            } else {
+              q_stage[nq] = stage;
+              q_k[nq] = kt;
+              q_tt[nq] = tt;
+              if (++nq == S && !become_ready()) { ok = false; break; }
             }
           }
         }
+        if (ok && !ready && !become_ready()) ok = false;
       }
-      if (!waited) {
-        pdl_wait();
-        for (int i = 0; i < npre; ++i)
-          tma_load_2d(sX + i * xbytes, &tmX, &tail->full[i], pre_k[i] * kTileK, pre_tt[i] * s.NT);
-      }
-      trace_mark(s, 3);
-      if (ok && s.next_valid && blockIdx.x < s.next_clusters * s.next_split) {
-        // warm L2 (and address translation) for this CTA index's first boxes of the next GEMM
-        const int nrank = blockIdx.x % s.next_split;
-        const int ncl = blockIdx.x / s.next_split;
-        if (ncl < s.next_tiles) {
-          const int nr = ncl / s.next_tok_tiles;
-          const int lo = nrank * s.next_ks;
-          const int hi = min(s.next_KT, min(lo + s.next_ks, lo + s.next_boxes));
-          for (int kt = lo; kt < hi; ++kt) tma_prefetch_l2_2d(&tmWn, kt * kTileK, nr * kTileRows);
+      if (ok && A.next_valid && static_cast<int>(blockIdx.x) < A.next_grid) {
+        // warm L2 (and address translation) for this CTA index's first boxes of the next chain
+        const int ncl = blockIdx.x / A.next_CS;
+        const int nrank = blockIdx.x % A.next_CS;
+        const int grp = ncl * (A.next_CS / A.next_s) + nrank / A.next_s;
+        if (grp < A.next_tiles) {
+          const int nr = grp / A.next_tok_tiles;
+          const int lo = (nrank % A.next_s) * A.next_ks;
+          const int hi = min(A.next_KT, min(lo + A.next_ks, lo + A.next_boxes));
+          for (int kt = lo; kt < hi; ++kt) tma_prefetch_l2_2d(&A.tmWn, 0, (nr * A.next_KT + kt) * kTileRows);
         }
       }
       if (!ok) {
@@ -206,154 +256,187 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer --
-      const uint32_t idesc = idesc_bf16_f32(kTileRows, s.NT);
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
       int it = 0, i = 0;
       bool ok = true;
-      for (int t = cl; ok && t < tiles; t += C, ++i) {
-        const int tb = i & 1;
-        const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!wait_or_abort(&tail->tempty[tb], (use & 1u) ^ 1u, timeout_ns, tail, e.err)) break;
-        tc_fence_after();
-        const uint32_t d = tmem + tb * buf_cols;
-        for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
-          const int stage = it % S;
-          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-          if (!wait_or_abort(&tail->full[stage], ph, timeout_ns, tail, e.err)) {
+      for (int p = 0; ok && p < A.nph; ++p) {
+        const Work w = work_of(A, p, cl, rank, C);
+        for (int t = w.grp; ok && t < w.tiles; t += w.ngrp, ++i) {
+          const int tb = i & 1;
+          const uint32_t use = static_cast<uint32_t>(i >> 1);
+          if (!wait_or_abort(&tail->tempty[tb], (use & 1u) ^ 1u, timeout_ns, tail, err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (it == 0) trace_mark(s, 4);
-          const uint64_t da = sdesc_k_sw128(smem_u32(sW + stage * kStageW));
-          const uint64_t db = sdesc_k_sw128(smem_u32(sX + stage * xbytes));
+          const uint32_t d = tmem + tb * buf_cols;
+          for (int kt = w.k_lo; kt < w.k_hi; ++kt, ++it) {
+            const int stage = it % S;
+            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+            if (!wait_or_abort(&tail->full[stage], ph, timeout_ns, tail, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            trace_iter(A, 1, it);
+            const uint64_t da = sdesc_k_sw128(smem_u32(sW + stage * kStageW));
+            const uint64_t db = sdesc_k_sw128(smem_u32(sX + stage * xbytes));
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk)
-            tc_mma_f16(d, da + 2 * kk, db + 2 * kk, idesc, (kt > k_lo || kk > 0) ? 1u : 0u);
-          tc_commit(&tail->empty[stage]);
+            for (int kk = 0; kk < kTileK / 16; ++kk)
+              tc_mma_f16(d, da + 2 * kk, db + 2 * kk, idesc, (kt > w.k_lo || kk > 0) ? 1u : 0u);
+            tc_commit(&tail->empty[stage]);
+          }
+          if (!ok) break;
+          tc_commit(&tail->tfull[tb]);
+          trace_mark(A, 14);
         }
-        if (!ok) break;
-        tc_commit(&tail->tfull[tb]);
-        trace_mark(s, 5 + (i < 2 ? i : 1));
       }
     }
     __syncwarp();
     // every epilogue read of tensor memory is done once the epilogue warps reach barrier 2
-    named_bar_sync(2, 160);
+    named_bar_sync(2, 32 + kEpiThreads);
     tc_fence_after();
-    tmem_dealloc(tmem, s.tmem_cols);
+    tmem_dealloc(tmem, A.tmem_cols);
   } else {
     // -------------------------------------------------------------------- epilogue --
     pdl_wait();
     const int et = threadIdx.x - 64;
     const int ew = warp & 3;              // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;     // which of the quarter's two warps: chunk parity
     const int row_in_tile = ew * 32 + lane;
-    const bool need_norm = (EPI != EPI_RESID);
+    float* red_f = tail->red_f[half];
+    int* red_i = tail->red_i[half];
+    const int hbar = 3 + half;            // named barrier of this half's 4 warps
     uint32_t stg_peer[kMaxSplit];
-    if (split > 1) {
 #pragma unroll
-      for (int q = 0; q < kMaxSplit; ++q)
-        stg_peer[q] = dsmem_addr(smem_u32(staging), static_cast<uint32_t>(q < split ? q : 0));
-    }
-    int i = 0;
-    for (int t = cl; t < tiles; t += C, ++i) {
-      const int r = t / s.tok_tiles;
-      const int tt = t - r * s.tok_tiles;
-      const int tok0 = tt * s.NT;
-      const int nvalid = min(s.NT, e.M - tok0);
-      const int nchunks = (nvalid + 15) >> 4;
-      const int tb = i & 1;
-      const uint32_t use = static_cast<uint32_t>(i >> 1);
-      named_bar_sync(1, 128);
-      compute_tile_meta(e, tok0, s.NT, need_norm, tail->inv, tail->pos, tail->pg, et, 128);
-      if (!epi_wait(&tail->tfull[tb], use & 1u, false, timeout_ns, tail, e.err)) break;
-      tc_fence_after();
-      if (et == 0) trace_mark(s, 7 + (i < 2 ? i : 1));
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(ew * 32) << 16) + tb * buf_cols;
-      if (split == 1) {
-        for (int c = 0; c < nchunks; ++c) {
-          float v[16];
-          tmem_ld16(tbase + c * 16, v);
-          epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
-                       c * 16, v, tail->red_f, tail->red_i);
+    for (int q = 0; q < kMaxSplit; ++q)
+      stg_peer[q] = (CS > 1) ? dsmem_addr(smem_u32(staging), static_cast<uint32_t>(q < CS ? q : 0)) : 0u;
+    int i = 0;    // tiles of this CTA so far (TMEM buffer parity)
+    int js = 0;   // split tiles so far (staging buffer parity)
+    bool ok = true;
+    for (int p = 0; ok && p < A.nph; ++p) {
+      const PhaseArgs& P = A.ph[p];
+      const EpiArgs& e = P.e;
+      const Work w = work_of(A, p, cl, rank, C);
+      const bool need_norm = (e.kind != EPI_RESID);
+      if (p > 0) {
+        // inputs of this epilogue (residual, RMS statistics) come from phase p-1
+        if (!wait_counter(A.bar + (p - 1), G, timeout_ns)) {
+          tail->epi_abort = 1;
+          set_err(err, NLD_DEVERR_TIMEOUT);
         }
-        tc_fence_before();
-        mbar_arrive(&tail->tempty[tb]);
-      } else {
-        // 1. this rank's partial -> staging buffer b, once every rank has read its last use
-        const int b = i & 1;
-        if (!epi_wait(&tail->sempty[b], (use & 1u) ^ 1u, true, timeout_ns, tail, e.err)) break;
-        float* stg = staging + b * stg_floats;
-        for (int c = 0; c < nchunks; ++c) {
-          float v[16];
-          tmem_ld16(tbase + c * 16, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) stg[(c * 16 + j) * kTileRows + row_in_tile] = v[j];
-        }
-        tc_fence_before();
-        mbar_arrive(&tail->tempty[tb]);
-        named_bar_sync(1, 128);
-        if (et == 0)
-          for (int q = 0; q < split; ++q)
-            mbar_arrive_remote(dsmem_addr(smem_u32(&tail->sfull[b]), static_cast<uint32_t>(q)));
-        // 2. every rank's partial is staged: reduce this rank's column slice over DSMEM
-        if (!epi_wait(&tail->sfull[b], use & 1u, true, timeout_ns, tail, e.err)) break;
-        if (et == 0) trace_mark(s, 12);
-        const int per = (nchunks + split - 1) / split;
-        const int c_lo = rank * per, c_hi = min(nchunks, c_lo + per);
-        const uint32_t off0 = static_cast<uint32_t>(b * stg_floats) * 4u;
-        for (int c = c_lo; c < c_hi; ++c) {
-          float part[kMaxSplit][16];
-          const uint32_t cofs = off0 + static_cast<uint32_t>((c * 16) * kTileRows + row_in_tile) * 4u;
-#pragma unroll
-          for (int q = 0; q < kMaxSplit; ++q) {
-            if (q < split) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                part[q][j] = ld_dsmem_f32(stg_peer[q] + cofs + static_cast<uint32_t>(j * kTileRows * 4));
-            }
-          }
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float acc = 0.f;
-#pragma unroll
-            for (int q = 0; q < kMaxSplit; ++q)
-              if (q < split) acc += part[q][j];
-            v[j] = acc;
-          }
-          epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
-                       c * 16, v, tail->red_f, tail->red_i);
-        }
-        // 3. this rank is done reading every rank's staging buffer b
-        named_bar_sync(1, 128);
-        if (et == 0)
-          for (int q = 0; q < split; ++q)
-            mbar_arrive_remote(dsmem_addr(smem_u32(&tail->sempty[b]), static_cast<uint32_t>(q)));
+        named_bar_sync(1, kEpiThreads);
+        if (tail->epi_abort) break;
       }
-      if (et == 0) trace_mark(s, 9 + (i < 2 ? i : 1));
+      if (et == 0) trace_mark(A, 3 + 3 * p);
+      const int g0 = (rank / w.s) * w.s;   // first cluster rank of this rank's group
+      for (int t = w.grp; t < w.tiles; t += w.ngrp, ++i) {
+        const int r = t / P.tok_tiles;
+        const int tt = t - r * P.tok_tiles;
+        const int tok0 = tt * NT;
+        const int nvalid = min(NT, e.M - tok0);
+        const int nchunks = (nvalid + 15) >> 4;
+        const int tb = i & 1;
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        named_bar_sync(1, kEpiThreads);
+        compute_tile_meta(e, tok0, NT, need_norm, tail->inv, tail->pos, tail->pg, et, kEpiThreads);
+        if (!epi_wait(&tail->tfull[tb], use & 1u, false, timeout_ns, tail, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(ew * 32) << 16) + tb * buf_cols;
+        if (w.s == 1) {
+          for (int c = half; c < nchunks; c += 2) {
+            float v[16];
+            tmem_ld16(tbase + c * 16, v);
+            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
+                         c * 16, v, red_f, red_i, hbar);
+          }
+          tc_fence_before();
+          mbar_arrive(&tail->tempty[tb]);
+        } else {
+          // 1. this rank's partial -> staging buffer b, once the group has read its last use
+          const int b = js & 1;
+          const uint32_t suse = static_cast<uint32_t>(js >> 1);
+          ++js;
+          if (!epi_wait(&tail->sempty[b], (suse & 1u) ^ 1u, true, timeout_ns, tail, err)) { ok = false; break; }
+          float* stg = staging + b * stg_floats;
+          for (int c = half; c < nchunks; c += 2) {
+            float v[16];
+            tmem_ld16(tbase + c * 16, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) stg[(c * 16 + j) * kTileRows + row_in_tile] = v[j];
+          }
+          tc_fence_before();
+          mbar_arrive(&tail->tempty[tb]);
+          named_bar_sync(1, kEpiThreads);
+          const uint32_t cnt = static_cast<uint32_t>(CS / w.s);
+          if (et == 0)
+            for (int q = 0; q < w.s; ++q)
+              mbar_arrive_remote_count(dsmem_addr(smem_u32(&tail->sfull[b]), static_cast<uint32_t>(g0 + q)), cnt);
+          // 2. the group's partials are staged: reduce this rank's column slice over DSMEM
+          if (!epi_wait(&tail->sfull[b], suse & 1u, true, timeout_ns, tail, err)) { ok = false; break; }
+          const int per = (nchunks + w.s - 1) / w.s;
+          const int c_lo = w.grank * per, c_hi = min(nchunks, c_lo + per);
+          const uint32_t off0 = static_cast<uint32_t>(b * stg_floats) * 4u;
+          for (int c = c_lo + half; c < c_hi; c += 2) {
+            const uint32_t cofs = off0 + static_cast<uint32_t>((c * 16) * kTileRows + row_in_tile) * 4u;
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            // ranks of the group in order, two at a time so that 32 loads are in flight
+            for (int q0 = 0; q0 < w.s; q0 += 2) {
+              float pa[16], pb[16];
+              const uint32_t a0 = stg_peer[g0 + q0] + cofs;
+              const bool two = (q0 + 1 < w.s);
+              const uint32_t a1 = two ? stg_peer[g0 + q0 + 1] + cofs : a0;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pa[j] = ld_dsmem_f32(a0 + static_cast<uint32_t>(j * kTileRows * 4));
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pb[j] = two ? ld_dsmem_f32(a1 + static_cast<uint32_t>(j * kTileRows * 4)) : 0.f;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = (v[j] + pa[j]) + pb[j];
+            }
+            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
+                         c * 16, v, red_f, red_i, hbar);
+          }
+          // 3. this rank is done reading the group's staging buffers b
+          named_bar_sync(1, kEpiThreads);
+          if (et == 0)
+            for (int q = 0; q < w.s; ++q)
+              mbar_arrive_remote_count(dsmem_addr(smem_u32(&tail->sempty[b]), static_cast<uint32_t>(g0 + q)), cnt);
+        }
+      }
+      if (!ok) break;
+      if (et == 0) trace_mark(A, 4 + 3 * p);
+      if (p + 1 < A.nph) {
+        // this CTA's outputs of phase p are written: publish them, then arrive
+        __threadfence();
+        fence_proxy_async_global();
+        named_bar_sync(1, kEpiThreads);
+        if (et == 0) atomicAdd(A.bar + p, 1u);
+      }
     }
     tc_fence_before();
-    named_bar_sync(2, 160);
-    if (et == 0) trace_mark(s, 15);
+    named_bar_sync(2, 32 + kEpiThreads);
   }
   // peers may still read this CTA's staging buffers or arrive on its barriers
-  if (split > 1) cluster_sync();
-  if (threadIdx.x == 0) trace_mark(s, 11);
+  if (CS > 1) cluster_sync();
+  __syncthreads();
+  if (A.nph > 1 && threadIdx.x == 0) {
+    // every thread of this CTA is past its last wait on the phase counters; the last CTA to
+    // get here zeroes them (and the exit counter) for the next launch that uses them
+    __threadfence();
+    const unsigned old = atomicAdd(A.bar + (kMaxPhases - 1), 1u);
+    if (old == G - 1) {
+      for (int p = 0; p < kMaxPhases; ++p) atomicExch(A.bar + p, 0u);
+      __threadfence();
+    }
+  }
+  if (threadIdx.x == 0) trace_mark(A, 15);
 }
 
-size_t gemm_tc_smem_bytes(const GemmShape& s) {
-  const size_t stg = (s.split > 1) ? 2ull * s.NT * kTileRows * sizeof(float) : 0;
-  return 1024 + static_cast<size_t>(s.stages) * (kStageW + s.NT * 128) + stg + sizeof(GemmTail);
-}
-
-template <int EPI>
-static cudaError_t set_smem_limit(int optin) {
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, gemm_tc_kernel<EPI, __nv_bfloat16>);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(gemm_tc_kernel<EPI, __nv_bfloat16>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              optin - static_cast<int>(fa.sharedSizeBytes));
+size_t gemm_chain_smem_bytes(int NT, int stages, int CS) {
+  const size_t stg = (CS > 1) ? 2ull * NT * kTileRows * sizeof(float) : 0;
+  return 1024 + static_cast<size_t>(stages) * (kStageW + NT * 128) + stg + sizeof(GemmTail);
 }
 
 cudaError_t gemm_tc_init_attributes() {
@@ -362,18 +445,18 @@ cudaError_t gemm_tc_init_attributes() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  if ((e = set_smem_limit<EPI_QKV>(optin)) != cudaSuccess) return e;
-  if ((e = set_smem_limit<EPI_RESID>(optin)) != cudaSuccess) return e;
-  if ((e = set_smem_limit<EPI_SWIGLU>(optin)) != cudaSuccess) return e;
-  if ((e = set_smem_limit<EPI_LMHEAD>(optin)) != cudaSuccess) return e;
-  return set_smem_limit<EPI_LOGITS>(optin);
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, gemm_chain_kernel<__nv_bfloat16>)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gemm_chain_kernel<__nv_bfloat16>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
 // Clusters of `split` CTAs (one CTA per SM at `smem` bytes) that can be resident at once.
 int gemm_tc_max_clusters(int split, size_t smem, int sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(split * (sms / split));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -383,26 +466,24 @@ int gemm_tc_max_clusters(int split, size_t smem, int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<EPI_QKV, __nv_bfloat16>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_chain_kernel<__nv_bfloat16>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return sms / split;
   }
   return n > 0 ? std::min(n, sms / split) : sms / split;
 }
 
-cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
-                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl,
-                           const CUtensorMap* tmW_next) {
-  const CUtensorMap* wn = tmW_next ? tmW_next : tmW;
+cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uint64_t timeout_ns,
+                              bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s.G);
-  cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = gemm_tc_smem_bytes(s);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.stages, A.CS);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;
   attr[na].id = cudaLaunchAttributeClusterDimension;
-  attr[na].val.clusterDim.x = s.split;
+  attr[na].val.clusterDim.x = A.CS;
   attr[na].val.clusterDim.y = 1;
   attr[na].val.clusterDim.z = 1;
   ++na;
@@ -413,23 +494,7 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtens
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  switch (e.kind) {
-    case EPI_QKV:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_QKV, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
-                                timeout_ns);
-    case EPI_RESID:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_RESID, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
-                                timeout_ns);
-    case EPI_SWIGLU:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_SWIGLU, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
-                                timeout_ns);
-    case EPI_LMHEAD:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LMHEAD, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
-                                timeout_ns);
-    default:
-      return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI_LOGITS, __nv_bfloat16>, *tmW, *tmX, *wn, s, e,
-                                timeout_ns);
-  }
+  return cudaLaunchKernelEx(&cfg, gemm_chain_kernel<__nv_bfloat16>, A, timeout_ns);
 }
 
 }  // namespace nld

@@ -64,6 +64,13 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a pre-tiled weight matrix: a 2D view [row_tiles * (K/64) * 128 rows, 64
+// elements] whose box {64, 128} is one contiguous 16 KB block.
+bool make_map_tiled(CUtensorMap* map, const void* base, int n_rows, int K) {
+  const uint64_t row_tiles = (n_rows + kTileRows - 1) / kTileRows;
+  return make_map_bf16(map, base, kTileK, row_tiles * (K / kTileK) * kTileRows, kTileRows);
+}
+
 enum XBuf { XB_HB = 0, XB_ATTN = 1, XB_U = 2 };
 enum GemmWhich { GW_QKV = 0, GW_O = 1, GW_GU = 2, GW_D = 3, GW_LM = 4 };
 enum LmKind { LM_NONE = 0, LM_ARGMAX = 1, LM_LOGITS = 2 };
@@ -105,6 +112,8 @@ struct nld_ctx {
   int lm_tiles = 0;
   float2* rope = nullptr;
   int max_clusters[9] = {0};
+  unsigned* bars = nullptr;   // chain phase-boundary counters: (1 + n_layers) x kMaxPhases
+  int n_bars = 0;
   int* h_pinned = nullptr;  // host: [0] error word, [1] incomplete, [2..] lens
   // tensor maps
   std::vector<CUtensorMap> tmWqkv, tmWo, tmWgu, tmWd;
@@ -192,54 +201,11 @@ nld_status validate(const nld_config* c, std::string& why) {
 }
 
 // ------------------------------------------------------------------------- GEMM dispatch --
-struct GemmPlan {
-  GemmShape s;
+// One projection of a chain: which weight, which layer, and its epilogue arguments.
+struct ProjRef {
+  int which, layer;
+  EpiArgs e;
 };
-
-// Tiling of one projection GEMM.  Token columns: tiles of <= 256.  K: split over the CTAs of
-// a cluster (split 1..8, only for NT <= 64 where the fp32 staging buffers fit), chosen to
-// minimise waves x k-iterations per tile (+ a small per-tile cost) over the clusters that can
-// be resident at once.
-GemmShape plan_gemm(const nld_ctx* x, int n_rows, int K, int M) {
-  GemmShape s{};
-  s.n_rows = n_rows;
-  s.K = K;
-  s.M = M;
-  s.tok_tiles = (M + kMaxNT - 1) / kMaxNT;
-  const int per = (M + s.tok_tiles - 1) / s.tok_tiles;
-  s.NT = std::max(16, (per + 15) / 16 * 16);
-  s.row_tiles = (n_rows + kTileRows - 1) / kTileRows;
-  s.KT = K / kTileK;
-  const int tiles = s.row_tiles * s.tok_tiles;
-  long long best = -1;
-  // GEMMs with at least one tile per resident CTA keep split = 1: there the per-tile handoff
-  // of split partials would sit on every tile instead of hiding behind the next one.
-  const bool many = tiles >= x->max_clusters[1];
-  for (int split = 1; split <= 8; ++split) {
-    if (split > 1 && (s.NT > 64 || many)) break;
-    if (split > s.KT) break;
-    const int ks = (s.KT + split - 1) / split;
-    if ((split - 1) * ks >= s.KT) continue;
-    const int C = std::min(x->max_clusters[split], tiles);
-    if (C < 1) continue;
-    const long long waves = (tiles + C - 1) / C;
-    const long long cost = waves * (ks + 3);
-    if (best < 0 || cost < best) {
-      best = cost;
-      s.split = split;
-      s.ks = ks;
-      s.G = C * split;
-    }
-  }
-  const int stage_bytes = kTileRows * kTileK * 2 + s.NT * 128;
-  const int staging = (s.split > 1) ? 2 * s.NT * kTileRows * 4 : 0;
-  s.stages = std::max(2, std::min(8, (216 * 1024 - staging - 4096) / stage_bytes));
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * s.NT)) cols <<= 1;
-  s.tmem_cols = cols;
-  s.trace = nullptr;
-  return s;
-}
 
 const CUtensorMap* xmap(nld_ctx* x, int buf, int NT) {
   auto key = std::make_pair(buf, NT);
@@ -270,45 +236,122 @@ WInfo winfo(nld_ctx* x, int which, int layer) {
   return w;
 }
 
-nld_status gemm(nld_ctx* x, int which, int layer, int M, const EpiArgs& e, bool pdl,
-                unsigned long long* trace = nullptr, int next_which = -1, int next_layer = 0) {
-  int n_rows, K, buf;
-  const void* W;
-  const CUtensorMap* tmW = nullptr;
-  switch (which) {
-    case GW_QKV: n_rows = x->qkv_rows; K = x->c.d_model; buf = XB_HB; W = x->wqkv[layer]; if (x->bf16) tmW = &x->tmWqkv[layer]; break;
-    case GW_O: n_rows = x->c.d_model; K = x->qd; buf = XB_ATTN; W = x->wo[layer]; if (x->bf16) tmW = &x->tmWo[layer]; break;
-    case GW_GU: n_rows = x->gu_rows; K = x->c.d_model; buf = XB_HB; W = x->wgu[layer]; if (x->bf16) tmW = &x->tmWgu[layer]; break;
-    case GW_D: n_rows = x->c.d_model; K = x->c.ffn_dim; buf = XB_U; W = x->wd[layer]; if (x->bf16) tmW = &x->tmWd[layer]; break;
-    default: n_rows = x->c.vocab; K = x->c.d_model; buf = XB_HB; W = x->wlm; if (x->bf16) tmW = &x->tmWlm; break;
+// Plan a chain of projections over M token rows.  Token columns: tiles of <= 256 (NT).  Cluster
+// size CS: 4 for multi-phase decode chains (NT <= 64, where the fp32 staging buffers fit), for
+// a single projection the best of 1, 2, 4, 8; 1 when NT > 64.  Per phase the K split s (a
+// divisor of CS) minimises waves x (k-iterations per tile + the cross-rank handoff of a split
+// tile, which measures at about six k-iterations) over the clusters that can be resident.
+ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_out, long long* cost_out = nullptr) {
+  ChainArgs best{};
+  long long best_cost = -1;
+  int best_grid = 0;
+  const int tok_tiles = (M + kMaxNT - 1) / kMaxNT;
+  const int per = (M + tok_tiles - 1) / tok_tiles;
+  const int NT = std::max(16, (per + 15) / 16 * 16);
+  int cands[4] = {1, 2, 4, 8};
+  int ncand = 4;
+  if (NT > 64) {
+    ncand = 1;
+  } else if (nph > 1) {
+    cands[0] = 4;
+    ncand = 1;
   }
-  EpiArgs ee = e;
-  ee.n_rows = n_rows;
+  for (int ci = 0; ci < ncand; ++ci) {
+    const int CS = cands[ci];
+    const int C = x->max_clusters[CS];
+    if (C < 1) continue;
+    ChainArgs A{};
+    A.nph = nph;
+    A.CS = CS;
+    A.NT = NT;
+    long long total = 0;
+    int need_clusters = 1;
+    for (int p = 0; p < nph; ++p) {
+      const WInfo w = winfo(x, pr[p].which, pr[p].layer);
+      PhaseArgs& P = A.ph[p];
+      P.tok_tiles = tok_tiles;
+      P.row_tiles = (w.n_rows + kTileRows - 1) / kTileRows;
+      P.KT = w.K / kTileK;
+      const int tiles = P.row_tiles * P.tok_tiles;
+      long long pbest = -1;
+      for (int sp = 1; sp <= CS; sp *= 2) {
+        if (sp > P.KT) break;
+        const int ks = (P.KT + sp - 1) / sp;
+        if ((sp - 1) * ks >= P.KT) continue;
+        const long long groups = static_cast<long long>(C) * (CS / sp);
+        const long long waves = (tiles + groups - 1) / groups;
+        const long long cost = waves * (ks + (sp > 1 ? 6 : 0));
+        if (pbest < 0 || cost < pbest) {
+          pbest = cost;
+          P.s = sp;
+          P.ks = ks;
+        }
+      }
+      total += pbest;
+      need_clusters = std::max(need_clusters, (tiles * P.s + CS - 1) / CS);
+    }
+    if (best_cost < 0 || total < best_cost) {
+      best_cost = total;
+      best = A;
+      best_grid = std::min(C, need_clusters) * CS;
+    }
+  }
+  const int stage_bytes = kTileRows * kTileK * 2 + NT * 128;
+  const int staging = (best.CS > 1) ? 2 * NT * kTileRows * 4 : 0;
+  best.stages = std::max(2, std::min(8, (216 * 1024 - staging - 4096) / stage_bytes));
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(2 * NT)) cols <<= 1;
+  best.tmem_cols = cols;
+  if (grid_out) *grid_out = best_grid;
+  if (cost_out) *cost_out = best_cost;
+  return best;
+}
+
+// Launch a chain of projections (the SIMT kernel one by one for the fp32 configuration).
+// `bar`: this launch's phase-boundary counters.  next_*: the projection after this launch
+// (L2 warm-up of its first weight boxes), or next_which < 0.
+nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsigned* bar,
+                 const ProjRef* next_pr, int next_nph, unsigned long long* trace = nullptr) {
   if (!x->bf16) {
-    const void* X = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
-    CK(launch_gemm_simt(x->stream, static_cast<const float*>(W), static_cast<const float*>(X),
-                        n_rows, K, M, ee, pdl));
+    for (int p = 0; p < nph; ++p) {
+      const WInfo w = winfo(x, pr[p].which, pr[p].layer);
+      EpiArgs e = pr[p].e;
+      e.n_rows = w.n_rows;
+      const void* X = w.buf == XB_HB ? x->hb : (w.buf == XB_ATTN ? x->attn : x->ubuf);
+      CK(launch_gemm_simt(x->stream, static_cast<const float*>(w.W), static_cast<const float*>(X),
+                          w.n_rows, w.K, M, e, pdl));
+    }
     return NLD_OK;
   }
-  GemmShape s = plan_gemm(x, n_rows, K, M);
-  s.trace = trace;
-  const CUtensorMap* tmWn = nullptr;
-  if (next_which >= 0) {
-    const WInfo nw = winfo(x, next_which, next_layer);
-    const GemmShape n = plan_gemm(x, nw.n_rows, nw.K, M);
-    s.next_valid = 1;
-    s.next_split = n.split;
-    s.next_tok_tiles = n.tok_tiles;
-    s.next_ks = n.ks;
-    s.next_KT = n.KT;
-    s.next_clusters = n.G / n.split;
-    s.next_tiles = n.row_tiles * n.tok_tiles;
-    s.next_boxes = n.stages;
-    tmWn = nw.map;
+  int grid = 0;
+  ChainArgs A = plan_chain(x, pr, nph, M, &grid);
+  for (int p = 0; p < nph; ++p) {
+    const WInfo w = winfo(x, pr[p].which, pr[p].layer);
+    A.ph[p].tmW = *w.map;
+    const CUtensorMap* tmX = xmap(x, w.buf, A.NT);
+    if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
+    A.ph[p].tmX = *tmX;
+    A.ph[p].e = pr[p].e;
+    A.ph[p].e.n_rows = w.n_rows;
   }
-  const CUtensorMap* tmX = xmap(x, buf, s.NT);
-  if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
-  CK(launch_gemm_tc(x->stream, tmW, tmX, s, ee, x->timeout_ns, pdl, tmWn));
+  A.bar = bar;
+  A.trace = trace;
+  A.tmWn = A.ph[0].tmW;
+  if (next_pr && next_nph > 0) {
+    int ngrid = 0;
+    const ChainArgs N = plan_chain(x, next_pr, next_nph, M, &ngrid);
+    A.next_valid = 1;
+    A.next_CS = N.CS;
+    A.next_s = N.ph[0].s;
+    A.next_tok_tiles = N.ph[0].tok_tiles;
+    A.next_ks = N.ph[0].ks;
+    A.next_KT = N.ph[0].KT;
+    A.next_grid = ngrid;
+    A.next_tiles = N.ph[0].row_tiles * N.ph[0].tok_tiles;
+    A.next_boxes = N.stages;
+    A.tmWn = *winfo(x, next_pr[0].which, next_pr[0].layer).map;
+  }
+  CK(launch_gemm_chain(x->stream, A, grid, x->timeout_ns, pdl));
   return NLD_OK;
 }
 
@@ -413,33 +456,51 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
     aa.G = aa.Hq / aa.Hkv;
   }
 
-  for (int l = 0; l < x->c.n_layers; ++l) {
-    EpiArgs e = base_epi(x, M, f.m);
-    e.kind = EPI_QKV;
-    e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
-    TRY(gemm(x, GW_QKV, l, M, e, pdl, nullptr, GW_O, l));
+  // projections: QKV(0) | per layer: attention, chain [O, gate/up, down, QKV(l+1)] | LM head
+  const int L = x->c.n_layers;
+  auto proj = [&](int which, int layer) {
+    ProjRef r{which, layer, base_epi(x, M, f.m)};
+    static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
+    r.e.kind = kinds[which];
+    if (which == GW_QKV)
+      r.e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
+    if (which == GW_LM) {
+      r.e.kind = (f.lm == LM_LOGITS) ? EPI_LOGITS : EPI_LMHEAD;
+      r.e.logits = f.logits;
+    }
+    return r;
+  };
+  auto layer_chain = [&](int l, ProjRef* out) {
+    int n = 0;
+    out[n++] = proj(GW_O, l);
+    out[n++] = proj(GW_GU, l);
+    out[n++] = proj(GW_D, l);
+    if (l + 1 < L) out[n++] = proj(GW_QKV, l + 1);
+    return n;
+  };
+  ProjRef cur[kMaxPhases], nxt[kMaxPhases];
+  {
+    const ProjRef q0 = proj(GW_QKV, 0);
+    const int nn = layer_chain(0, nxt);
+    TRY(chain(x, &q0, 1, M, pdl, x->bars, nxt, nn));
+  }
+  for (int l = 0; l < L; ++l) {
     if (x->bf16) {
       aa.layer_row0 = l * x->n_pages * 2 * x->c.n_kv_heads * kPage;
       CK(launch_attention_mma(x->stream, &x->tmKV, aa, f.B, pdl));
     } else {
-      aa.pool = e.kv_layer;
+      aa.pool = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
       CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
     }
-    const bool last = (l + 1 == x->c.n_layers);
-    e.kind = EPI_RESID;
-    TRY(gemm(x, GW_O, l, M, e, pdl, nullptr, GW_GU, l));
-    e.kind = EPI_SWIGLU;
-    TRY(gemm(x, GW_GU, l, M, e, pdl, nullptr, GW_D, l));
-    e.kind = EPI_RESID;
-    if (!last) TRY(gemm(x, GW_D, l, M, e, pdl, nullptr, GW_QKV, l + 1));
-    else if (f.lm != LM_NONE) TRY(gemm(x, GW_D, l, M, e, pdl, nullptr, GW_LM, 0));
-    else TRY(gemm(x, GW_D, l, M, e, pdl));
+    const int n = layer_chain(l, cur);
+    int nn = 0;
+    if (l + 1 < L) nn = layer_chain(l + 1, nxt);
+    else if (f.lm != LM_NONE) { nxt[0] = proj(GW_LM, 0); nn = 1; }
+    TRY(chain(x, cur, n, M, pdl, x->bars + (1 + l) * kMaxPhases, nn ? nxt : nullptr, nn));
   }
   if (f.lm != LM_NONE) {
-    EpiArgs e = base_epi(x, M, f.m);
-    e.kind = (f.lm == LM_LOGITS) ? EPI_LOGITS : EPI_LMHEAD;
-    e.logits = f.logits;
-    TRY(gemm(x, GW_LM, 0, M, e, pdl));
+    const ProjRef lm = proj(GW_LM, 0);
+    TRY(chain(x, &lm, 1, M, pdl, x->bars, nullptr, 0));
   }
   return NLD_OK;
 }
@@ -635,6 +696,9 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
   if ((s = dalloc(x, &x->attn, Mm * x->qd * el)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->ubuf, Mm * c.ffn_dim * el)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->lm_part, Mm * x->lm_tiles * sizeof(LmPart))) != NLD_OK) return bail(s);
+  x->n_bars = (2 + c.n_layers) * kMaxPhases;
+  if ((s = dalloc(x, &x->bars, x->n_bars * sizeof(unsigned))) != NLD_OK) return bail(s);
+  if (cudaMemset(x->bars, 0, x->n_bars * sizeof(unsigned)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   // resident clusters of each split size (one GEMM CTA per SM)
   if (x->bf16)
     for (int sp = 1; sp <= 8; ++sp) x->max_clusters[sp] = gemm_tc_max_clusters(sp, 200 * 1024, x->sms);
@@ -683,18 +747,21 @@ nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensor
   if (x->weights_ready) return fail(x, NLD_ERR_STATE, "weights already initialised");
   nld_status s;
   // allocations
+  // bf16 matrices are stored pre-tiled (16 KB blocks), with rows padded to a multiple of 128
+  auto pad = [&](int rows) { return x->bf16 ? (rows + kTileRows - 1) / kTileRows * kTileRows : rows; };
+  const bool tiled = x->bf16;
   if ((s = dalloc(x, &x->embed, static_cast<size_t>(V + 1) * d * el)) != NLD_OK) return s;
   x->wqkv.resize(L);
   x->wo.resize(L);
   x->wgu.resize(L);
   x->wd.resize(L);
   for (int l = 0; l < L; ++l) {
-    if ((s = dalloc(x, &x->wqkv[l], static_cast<size_t>(x->qkv_rows) * d * el)) != NLD_OK) return s;
-    if ((s = dalloc(x, &x->wo[l], static_cast<size_t>(d) * x->qd * el)) != NLD_OK) return s;
-    if ((s = dalloc(x, &x->wgu[l], static_cast<size_t>(x->gu_rows) * d * el)) != NLD_OK) return s;
-    if ((s = dalloc(x, &x->wd[l], static_cast<size_t>(d) * F * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wqkv[l], static_cast<size_t>(pad(x->qkv_rows)) * d * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wo[l], static_cast<size_t>(pad(d)) * x->qd * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wgu[l], static_cast<size_t>(pad(x->gu_rows)) * d * el)) != NLD_OK) return s;
+    if ((s = dalloc(x, &x->wd[l], static_cast<size_t>(pad(d)) * F * el)) != NLD_OK) return s;
   }
-  if ((s = dalloc(x, &x->wlm, static_cast<size_t>(V) * d * el)) != NLD_OK) return s;
+  if ((s = dalloc(x, &x->wlm, static_cast<size_t>(pad(V)) * d * el)) != NLD_OK) return s;
 
   // row maps: q/k heads interleave (i, i+hd/2); gate/up interleave per 64 features
   std::vector<int> map_q(x->qd), map_kv(x->kvd), map_g(F), map_u(F);
@@ -740,23 +807,27 @@ nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensor
     const void* const* t = tensors + 1 + 9 * l;
     TRY(up(t[0], d, stage_g));
     char* qkv = static_cast<char*>(x->wqkv[l]);
+    // q, k and v parts start on 128-row boundaries, where the tiled and row-major offsets agree
     TRY(up(t[1], static_cast<size_t>(x->qd) * d, stage));
-    CK(launch_repack(x->stream, qkv, stage, d_map_q, x->qd, d, stage_g, x->bf16));
+    CK(launch_repack(x->stream, qkv, stage, d_map_q, x->qd, d, stage_g, x->bf16, tiled));
     TRY(up(t[2], static_cast<size_t>(x->kvd) * d, stage));
-    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd) * d * el, stage, d_map_kv, x->kvd, d, stage_g, x->bf16));
+    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd) * d * el, stage, d_map_kv, x->kvd, d, stage_g, x->bf16, tiled));
     TRY(up(t[3], static_cast<size_t>(x->kvd) * d, stage));
-    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd + x->kvd) * d * el, stage, nullptr, x->kvd, d, stage_g, x->bf16));
-    TRY(up(t[4], static_cast<size_t>(d) * x->qd, x->wo[l]));
+    CK(launch_repack(x->stream, qkv + static_cast<size_t>(x->qd + x->kvd) * d * el, stage, nullptr, x->kvd, d, stage_g, x->bf16, tiled));
+    TRY(up(t[4], static_cast<size_t>(d) * x->qd, stage));
+    CK(launch_repack(x->stream, x->wo[l], stage, nullptr, d, x->qd, nullptr, x->bf16, tiled));
     TRY(up(t[5], d, stage_g));
     TRY(up(t[6], static_cast<size_t>(F) * d, stage));
     TRY(up(t[7], static_cast<size_t>(F) * d, static_cast<char*>(stage) + static_cast<size_t>(F) * d * el));
-    CK(launch_repack(x->stream, x->wgu[l], stage, d_map_gu, 2 * F, d, stage_g, x->bf16));
-    TRY(up(t[8], static_cast<size_t>(d) * F, x->wd[l]));
+    CK(launch_repack(x->stream, x->wgu[l], stage, d_map_gu, 2 * F, d, stage_g, x->bf16, tiled));
     CK(cudaStreamSynchronize(x->stream));   // staging reuse
+    TRY(up(t[8], static_cast<size_t>(d) * F, stage));
+    CK(launch_repack(x->stream, x->wd[l], stage, nullptr, d, F, nullptr, x->bf16, tiled));
+    CK(cudaStreamSynchronize(x->stream));
   }
   TRY(up(tensors[1 + 9 * L], d, stage_g));
   TRY(up(tensors[2 + 9 * L], static_cast<size_t>(V) * d, stage));
-  CK(launch_repack(x->stream, x->wlm, stage, nullptr, V, d, stage_g, x->bf16));
+  CK(launch_repack(x->stream, x->wlm, stage, nullptr, V, d, stage_g, x->bf16, tiled));
   CK(cudaStreamSynchronize(x->stream));
   // release staging (the last allocations)
   for (void* p : {stage, stage_g, static_cast<void*>(d_map_q), static_cast<void*>(d_map_kv), static_cast<void*>(d_map_gu)}) {
@@ -770,12 +841,12 @@ nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensor
     x->tmWd.resize(L);
     bool ok = true;
     for (int l = 0; l < L; ++l) {
-      ok &= make_map_bf16(&x->tmWqkv[l], x->wqkv[l], d, x->qkv_rows, kTileRows);
-      ok &= make_map_bf16(&x->tmWo[l], x->wo[l], x->qd, d, kTileRows);
-      ok &= make_map_bf16(&x->tmWgu[l], x->wgu[l], d, x->gu_rows, kTileRows);
-      ok &= make_map_bf16(&x->tmWd[l], x->wd[l], F, d, kTileRows);
+      ok &= make_map_tiled(&x->tmWqkv[l], x->wqkv[l], x->qkv_rows, d);
+      ok &= make_map_tiled(&x->tmWo[l], x->wo[l], d, x->qd);
+      ok &= make_map_tiled(&x->tmWgu[l], x->wgu[l], x->gu_rows, d);
+      ok &= make_map_tiled(&x->tmWd[l], x->wd[l], d, F);
     }
-    ok &= make_map_bf16(&x->tmWlm, x->wlm, d, V, kTileRows);
+    ok &= make_map_tiled(&x->tmWlm, x->wlm, V, d);
     if (!ok) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (weights)");
   }
   x->weights_ready = true;
@@ -1006,24 +1077,29 @@ nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
   return NLD_OK;
 }
 
+static ProjRef hook_proj(nld_ctx* x, int which, int layer, int M) {
+  const int m = M / x->batch;
+  ProjRef r{which, layer, base_epi(x, M, m)};
+  static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
+  r.e.kind = kinds[which];
+  r.e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
+  return r;
+}
+
 nld_status nld_time_gemm(nld_ctx* x, int which, int layer, int M, int reps, float* ms_out) {
   TRY(need_started(x));
   if (which < 0 || which > 4) return fail(x, NLD_ERR_ARG, "which must be 0..4");
   if (layer < 0 || layer >= x->c.n_layers) return fail(x, NLD_ERR_ARG, "layer out of range");
   if (M < 1 || M > x->M_max || M % x->batch) return fail(x, NLD_ERR_ARG, "M must be a multiple of the batch, <= %d", x->M_max);
   if (reps < 1 || !ms_out) return fail(x, NLD_ERR_ARG, "reps >= 1 and ms_out required");
-  const int m = M / x->batch;
-  TRY(ensure_capacity(x, m));
-  EpiArgs e = base_epi(x, M, m);
-  static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
-  e.kind = kinds[which];
-  e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
+  TRY(ensure_capacity(x, M / x->batch));
+  const ProjRef r = hook_proj(x, which, layer, M);
   cudaEvent_t a, b;
   CK(cudaEventCreate(&a));
   CK(cudaEventCreate(&b));
-  TRY(gemm(x, which, layer, M, e, false));   // warm (tensor maps, first-launch costs)
+  TRY(chain(x, &r, 1, M, false, x->bars, nullptr, 0));   // warm (tensor maps, first-launch costs)
   CK(cudaEventRecord(a, x->stream));
-  for (int i = 0; i < reps; ++i) TRY(gemm(x, which, layer, M, e, false));
+  for (int i = 0; i < reps; ++i) TRY(chain(x, &r, 1, M, false, x->bars, nullptr, 0));
   CK(cudaEventRecord(b, x->stream));
   CK(cudaEventSynchronize(b));
   float ms = 0.f;
@@ -1041,16 +1117,30 @@ nld_status nld_trace_gemm(nld_ctx* x, int which, int layer, int M, unsigned long
   if (which < 0 || which > 4 || layer < 0 || layer >= x->c.n_layers || !d_trace || M < 1 ||
       M > x->M_max || M % x->batch)
     return fail(x, NLD_ERR_ARG, "bad trace arguments");
-  const int m = M / x->batch;
-  EpiArgs e = base_epi(x, M, m);
-  static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
-  e.kind = kinds[which];
-  e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
-  const int nr[5] = {x->qkv_rows, x->c.d_model, x->gu_rows, x->c.d_model, x->c.vocab};
-  const int kd[5] = {x->c.d_model, x->qd, x->c.d_model, x->c.ffn_dim, x->c.d_model};
-  if (grid_out) *grid_out = plan_gemm(x, nr[which], kd[which], M).G;
-  TRY(gemm(x, which, layer, M, e, false));
-  TRY(gemm(x, which, layer, M, e, false, d_trace));
+  const ProjRef r = hook_proj(x, which, layer, M);
+  int grid = 0;
+  plan_chain(x, &r, 1, M, &grid);
+  if (grid_out) *grid_out = grid;
+  TRY(chain(x, &r, 1, M, false, x->bars, nullptr, 0));
+  TRY(chain(x, &r, 1, M, false, x->bars, nullptr, 0, d_trace));
+  CK(cudaStreamSynchronize(x->stream));
+  return NLD_OK;
+}
+
+nld_status nld_trace_chain(nld_ctx* x, int layer, int M, unsigned long long* d_trace, int* grid_out) {
+  TRY(need_started(x));
+  if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
+  if (layer < 0 || layer + 1 >= x->c.n_layers || !d_trace || M < 1 || M > x->M_max || M % x->batch)
+    return fail(x, NLD_ERR_ARG, "bad trace arguments");
+  TRY(ensure_capacity(x, M / x->batch));
+  ProjRef pr[4] = {hook_proj(x, GW_O, layer, M), hook_proj(x, GW_GU, layer, M),
+                   hook_proj(x, GW_D, layer, M), hook_proj(x, GW_QKV, layer + 1, M)};
+  int grid = 0;
+  plan_chain(x, pr, 4, M, &grid);
+  if (grid_out) *grid_out = grid;
+  unsigned* bar = x->bars + (1 + layer) * kMaxPhases;
+  TRY(chain(x, pr, 4, M, false, bar, nullptr, 0));
+  TRY(chain(x, pr, 4, M, false, bar, nullptr, 0, d_trace));
   CK(cudaStreamSynchronize(x->stream));
   return NLD_OK;
 }
@@ -1059,10 +1149,10 @@ nld_status nld_debug_gemm_plan(nld_ctx* x, int which, int M, int* out8) {
   if (!x || !out8) return fail(x, NLD_ERR_ARG, "NULL argument");
   if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
   if (which < 0 || which > 4 || M < 1 || M > x->M_max) return fail(x, NLD_ERR_ARG, "bad plan arguments");
-  const int nr[5] = {x->qkv_rows, x->c.d_model, x->gu_rows, x->c.d_model, x->c.vocab};
-  const int kd[5] = {x->c.d_model, x->qd, x->c.d_model, x->c.ffn_dim, x->c.d_model};
-  const GemmShape s = plan_gemm(x, nr[which], kd[which], M);
-  const int v[8] = {s.NT, s.tok_tiles, s.row_tiles, s.KT, s.split, s.ks, s.G, s.stages};
+  const ProjRef r{which, 0, base_epi(x, M, 1)};
+  int grid = 0;
+  const ChainArgs A = plan_chain(x, &r, 1, M, &grid);
+  const int v[8] = {A.NT, A.ph[0].tok_tiles, A.ph[0].row_tiles, A.ph[0].KT, A.ph[0].s, A.ph[0].ks, grid, A.stages};
   for (int i = 0; i < 8; ++i) out8[i] = v[i];
   return NLD_OK;
 }

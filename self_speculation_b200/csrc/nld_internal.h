@@ -73,24 +73,32 @@ struct EpiArgs {
   int* err;
 };
 
-struct GemmShape {
-  int n_rows;       // weight rows
-  int K;
-  int M;
+// One projection of a chain launch.
+constexpr int kMaxPhases = 4;
+struct alignas(64) PhaseArgs {
+  CUtensorMap tmW;  // pre-tiled weights: view [row_tiles * KT * 128, 64], box {64, 128}
+  CUtensorMap tmX;  // activations [M_max, K], box {64, NT}
+  EpiArgs e;
+  int tok_tiles, row_tiles, KT;
+  int s;            // ranks of a cluster splitting each tile's K range (divides CS)
+  int ks;           // k-iterations per rank
+};
+
+// A persistent launch running nph projections in order, separated by grid-wide arrivals.
+struct alignas(64) ChainArgs {
+  PhaseArgs ph[kMaxPhases];
+  CUtensorMap tmWn;  // weights of the projection that runs next on the stream (L2 warm-up)
+  int nph;
+  int CS;           // CTAs per cluster
   int NT;           // token columns per tile (multiple of 16, <= 256)
-  int tok_tiles;
-  int row_tiles;
-  int KT;           // K / 64
-  int split;        // CTAs per cluster = K slices per tile (1..8)
-  int ks;           // k-iterations per slice
-  int G;            // CTAs = clusters * split
   int stages;
-  uint32_t tmem_cols;  // power of two >= 2*NT
+  uint32_t tmem_cols;   // power of two >= 2*NT
+  unsigned* bar;    // [kMaxPhases] phase-boundary arrival counters + exit counter (last slot);
+                    // zero before the launch, left zero by it
   unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
-  // the projection GEMM that runs next on the stream (its weights are independent of this
-  // one's output): each CTA prefetches into L2 the first weight boxes it will load there
+  // the next chain launch's first phase (L2 warm-up of each CTA's first weight boxes there)
   int next_valid;
-  int next_split, next_tok_tiles, next_ks, next_KT, next_clusters, next_tiles, next_boxes;
+  int next_CS, next_s, next_tok_tiles, next_ks, next_KT, next_grid, next_tiles, next_boxes;
 };
 
 struct AttnArgs {
@@ -109,10 +117,9 @@ struct AttnArgs {
 };
 
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
-cudaError_t launch_gemm_tc(cudaStream_t st, const CUtensorMap* tmW, const CUtensorMap* tmX,
-                           const GemmShape& s, const EpiArgs& e, uint64_t timeout_ns, bool pdl,
-                           const CUtensorMap* tmW_next);
-size_t gemm_tc_smem_bytes(const GemmShape& s);
+cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uint64_t timeout_ns,
+                              bool pdl);
+size_t gemm_chain_smem_bytes(int NT, int stages, int CS);
 int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
                              int M, const EpiArgs& e, bool pdl);
@@ -147,7 +154,7 @@ struct FinalizeArgs {
 cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, bool pdl);
 
 cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
-                          int n_rows, int K, const void* gamma, bool bf16);
+                          int n_rows, int K, const void* gamma, bool bf16, bool tiled);
 cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
 
 }  // namespace nld
