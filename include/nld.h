@@ -197,6 +197,25 @@ void* nld_stream(nld_ctx* ctx);
 const char* nld_last_error(const nld_ctx* ctx);
 
 /*
+ * Stand-alone fused LM head + greedy token + confidence (the last step of every forward above),
+ * over caller buffers.  ranhao.site notes section 5.1 (greedy next token), 5.2 and shilu.ai
+ * SGLang (per-position confidence decides diffusion commits).  For each of M hidden rows h:
+ * logits = (h / sqrt(mean(h^2) + rms_eps)) W^T, never written out; d_argmax_out[i] = the index
+ * of the largest logit (lowest on ties), d_conf_out[i] = the largest softmax probability
+ * 1 / sum_v exp(l_v - max).
+ *   d_hidden     [M, d] bf16 row-major, 16-byte aligned; 1 <= M <= 4096, d a multiple of 128.
+ *   d_lm_weight  [vocab, d] bf16 row-major (RMSNorm gain already folded in), 16-byte aligned.
+ *   d_workspace  caller scratch of nld_lm_head_workspace_size() bytes, 256-byte aligned: per
+ *                128-column tile RMS sums, then per (row, 128-row vocab tile) partials.
+ * Stream-ordered on `cuda_stream`; returns after the launches.  Calls sharing a workspace must
+ * not overlap on the GPU.
+ */
+size_t nld_lm_head_workspace_size(int M, int d, int vocab);
+nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int M, int d, int vocab,
+                              float rms_eps, int32_t* d_argmax_out, float* d_conf_out,
+                              void* d_workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * Stand-alone block-causal GQA attention over a paged bf16 KV cache (the attention step of
  * the forwards above, exposed for the attention micro-workload).  Notes section 3.2 / r9-hu
  * "Method": a query sees every cached key and the keys of its own and earlier blocks.

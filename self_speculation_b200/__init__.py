@@ -67,6 +67,8 @@ def load_library() -> ctypes.CDLL:
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
+        "nld_lm_head_workspace_size": ([I, I, I], S),
+        "nld_lm_head_argmax": ([P, P, I, I, I, F, P, P, P, S, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -200,5 +202,23 @@ def nld_attention(q, kv_pool, page_table, lens, block_size: int, max_len: int, o
     st = lib.nld_attention(_ptr(q), _ptr(kv_pool), _ptr(page_table), page_table.shape[1], n_pages,
                            _ptr(lens), B, m, Hq, Hkv, hd, int(block_size), int(max_len), _ptr(out),
                            stream)
+    if st != 0:
+        raise NldError(st, lib.nld_last_error(None).decode())
+
+
+def nld_lm_head_workspace_size(M: int, d: int, vocab: int) -> int:
+    return load_library().nld_lm_head_workspace_size(M, d, vocab)
+
+
+def nld_lm_head_argmax(hidden, lm_weight, rms_eps: float, argmax_out, conf_out, workspace,
+                       stream: Optional[int] = None) -> None:
+    """hidden [M, d] bf16, lm_weight [vocab, d] bf16, argmax_out [M] int32, conf_out [M] fp32,
+    workspace uint8 of nld_lm_head_workspace_size bytes."""
+    lib = load_library()
+    M, d = hidden.shape
+    vocab = lm_weight.shape[0]
+    st = lib.nld_lm_head_argmax(_ptr(hidden), _ptr(lm_weight), M, d, vocab, float(rms_eps),
+                                _ptr(argmax_out), _ptr(conf_out), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), stream)
     if st != 0:
         raise NldError(st, lib.nld_last_error(None).decode())

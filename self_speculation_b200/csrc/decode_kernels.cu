@@ -287,6 +287,74 @@ cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int
   return cudaGetLastError();
 }
 
+// ----------------------------------------------------------- stand-alone LM-head helpers --
+// ssq[t * M + row] = sum over columns 128t..128t+127 of h[row, c]^2 (fp32), one warp per tile.
+__global__ void __launch_bounds__(256) rms_stats_kernel(const __nv_bfloat16* __restrict__ h, int M,
+                                                        int d, float* __restrict__ ssq) {
+  const int row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* hr = h + static_cast<size_t>(row) * d;
+  for (int t = warp; t < d / kTileRows; t += 8) {
+    float sq = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float v = __bfloat162float(hr[t * kTileRows + lane * 4 + q]);
+      sq += v * v;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if (lane == 0) ssq[static_cast<size_t>(t) * M + row] = sq;
+  }
+}
+
+cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq) {
+  rms_stats_kernel<<<M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), M, d, ssq);
+  return cudaGetLastError();
+}
+
+// One warp per token: max over vocab tiles (lowest id on ties), then sum_t se_t exp(mx_t - max);
+// the confidence is its inverse (largest softmax probability).
+__global__ void __launch_bounds__(256) lm_combine_kernel(const LmPart* __restrict__ part, int M,
+                                                         int tiles, int* __restrict__ argmax,
+                                                         float* __restrict__ conf) {
+  const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= M) return;
+  const LmPart* row = part + static_cast<size_t>(tok) * tiles;
+  float mx = -INFINITY;
+  int ix = INT_MAX;
+  for (int t = lane; t < tiles; t += 32) {
+    const LmPart p = row[t];
+    if (p.mx > mx || (p.mx == mx && p.idx < ix)) {
+      mx = p.mx;
+      ix = p.idx;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, mx, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, ix, off);
+    if (om > mx || (om == mx && oi < ix)) {
+      mx = om;
+      ix = oi;
+    }
+  }
+  float se = 0.f;
+  for (int t = lane; t < tiles; t += 32) se += row[t].se * expf(row[t].mx - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
+  if (lane == 0) {
+    argmax[tok] = ix;
+    conf[tok] = 1.0f / se;
+  }
+}
+
+cudaError_t launch_lm_combine(cudaStream_t st, const LmPart* part, int M, int tiles, int* argmax,
+                              float* conf) {
+  lm_combine_kernel<<<(M + 7) / 8, 256, 0, st>>>(part, M, tiles, argmax, conf);
+  return cudaGetLastError();
+}
+
 __global__ void fill_i32_kernel(int* p, int value, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = value;

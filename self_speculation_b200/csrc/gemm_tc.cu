@@ -218,9 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             trace_iter(A, 2, it - S);
             trace_iter(A, 0, it);
             mbar_arrive_expect_tx(&tail->full[stage], kStageW + xbytes);
-            // weights are pre-tiled: block (r, kt) is one contiguous 16 KB box
-            tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], 0,
-                             (r * P.KT + kt) * kTileRows, pol);
+            // pre-tiled weights: block (r, kt) is one contiguous 16 KB box
+            if (P.w_rowmajor)
+              tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], kt * kTileK,
+                               r * kTileRows, pol);
+            else
+              tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], 0,
+                               (r * P.KT + kt) * kTileRows, pol);
             if (ready) {
               tma_load_2d(sX + stage * xbytes, &P.tmX, &tail->full[stage], kt * kTileK, tt * NT);
             } else {

@@ -241,7 +241,8 @@ WInfo winfo(nld_ctx* x, int which, int layer) {
 // a single projection the best of 1, 2, 4, 8; 1 when NT > 64.  Per phase the K split s (a
 // divisor of CS) minimises waves x (k-iterations per tile + the cross-rank handoff of a split
 // tile, which measures at about six k-iterations) over the clusters that can be resident.
-ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_out, long long* cost_out = nullptr) {
+ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const int* K, int nph, int M,
+                            int* grid_out) {
   ChainArgs best{};
   long long best_cost = -1;
   int best_grid = 0;
@@ -258,7 +259,7 @@ ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_ou
   }
   for (int ci = 0; ci < ncand; ++ci) {
     const int CS = cands[ci];
-    const int C = x->max_clusters[CS];
+    const int C = max_clusters[CS];
     if (C < 1) continue;
     ChainArgs A{};
     A.nph = nph;
@@ -267,11 +268,10 @@ ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_ou
     long long total = 0;
     int need_clusters = 1;
     for (int p = 0; p < nph; ++p) {
-      const WInfo w = winfo(x, pr[p].which, pr[p].layer);
       PhaseArgs& P = A.ph[p];
       P.tok_tiles = tok_tiles;
-      P.row_tiles = (w.n_rows + kTileRows - 1) / kTileRows;
-      P.KT = w.K / kTileK;
+      P.row_tiles = (n_rows[p] + kTileRows - 1) / kTileRows;
+      P.KT = K[p] / kTileK;
       const int tiles = P.row_tiles * P.tok_tiles;
       long long pbest = -1;
       for (int sp = 1; sp <= CS; sp *= 2) {
@@ -303,8 +303,17 @@ ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_ou
   while (cols < static_cast<uint32_t>(2 * NT)) cols <<= 1;
   best.tmem_cols = cols;
   if (grid_out) *grid_out = best_grid;
-  if (cost_out) *cost_out = best_cost;
   return best;
+}
+
+ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_out) {
+  int nr[kMaxPhases], kd[kMaxPhases];
+  for (int p = 0; p < nph; ++p) {
+    const WInfo w = winfo(x, pr[p].which, pr[p].layer);
+    nr[p] = w.n_rows;
+    kd[p] = w.K;
+  }
+  return plan_chain_shapes(x->max_clusters, nr, kd, nph, M, grid_out);
 }
 
 // Launch a chain of projections (the SIMT kernel one by one for the fp32 configuration).
@@ -1185,6 +1194,99 @@ const char* nld_last_error(const nld_ctx* x) {
 }
 
 void* nld_stream(nld_ctx* x) { return x ? static_cast<void*>(x->stream) : nullptr; }
+
+// -------------------------------------------------------------- stand-alone LM head (a8) --
+// Resident clusters per split size on the current device (one GEMM CTA per SM), cached.
+static const int* device_max_clusters() {
+  static int cache[64][9];
+  static bool ready[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  if (!ready[dev]) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaGetLastError();
+    cache[dev][0] = 0;
+    for (int sp = 1; sp <= 8; ++sp) cache[dev][sp] = gemm_tc_max_clusters(sp, 200 * 1024, sms);
+    ready[dev] = true;
+  }
+  return cache[dev];
+}
+
+static size_t lm_ssq_bytes(int M, int d) { return (static_cast<size_t>(d / kTileRows) * M * sizeof(float) + 255) / 256 * 256; }
+static size_t lm_part_bytes(int M, int vocab) {
+  return static_cast<size_t>(M) * ((vocab + kTileRows - 1) / kTileRows) * sizeof(LmPart);
+}
+
+static nld_status lm_head_check(const void* h, const void* w, int M, int d, int vocab, const int32_t* am,
+                                const float* cf) {
+  if (!h || !w || !am || !cf) return fail(nullptr, NLD_ERR_ARG, "NULL pointer argument");
+  if (M < 1 || M > 4096) return fail(nullptr, NLD_ERR_ARG, "M must be in 1..4096");
+  if (d < 128 || d % 128) return fail(nullptr, NLD_ERR_ARG, "d must be a positive multiple of 128");
+  if (vocab < 1) return fail(nullptr, NLD_ERR_ARG, "vocab must be >= 1");
+  if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(w)) % 16)
+    return fail(nullptr, NLD_ERR_ARG, "hidden and weight must be 16-byte aligned");
+  return NLD_OK;
+}
+
+// Launch the a8 path over caller buffers with scratch at ws (ssq then LM-head partials).
+static nld_status lm_head_launch(const void* d_hidden, const void* d_lm_weight, int M, int d, int vocab,
+                                 float rms_eps, int32_t* d_argmax_out, float* d_conf_out, char* ws,
+                                 cudaStream_t st) {
+  cudaError_t ae = init_kernel_attributes();
+  if (ae != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed: %s", cudaGetErrorString(ae));
+  }
+  float* ssq = reinterpret_cast<float*>(ws);
+  LmPart* part = reinterpret_cast<LmPart*>(ws + lm_ssq_bytes(M, d));
+  int grid = 0;
+  const int nr = vocab, kd = d;
+  ChainArgs A = plan_chain_shapes(device_max_clusters(), &nr, &kd, 1, M, &grid);
+  PhaseArgs& P = A.ph[0];
+  if (!make_map_bf16(&P.tmW, d_lm_weight, d, vocab, kTileRows) ||
+      !make_map_bf16(&P.tmX, d_hidden, d, M, A.NT))
+    return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed");
+  P.w_rowmajor = 1;
+  EpiArgs& e = P.e;
+  e.kind = EPI_LMHEAD;
+  e.M = M;
+  e.m = M;
+  e.n_rows = vocab;
+  e.ssq_in = ssq;
+  e.ssq_tiles = d / kTileRows;
+  e.ssq_ld = M;
+  e.inv_d = 1.0f / static_cast<float>(d);
+  e.eps = rms_eps;
+  e.lm_part = part;
+  e.lm_tiles = (vocab + kTileRows - 1) / kTileRows;
+  e.V = vocab;
+  A.tmWn = P.tmW;
+  cudaError_t ce = launch_rms_stats(st, d_hidden, M, d, ssq);
+  if (ce == cudaSuccess) ce = launch_gemm_chain(st, A, grid, 2000000000ull, false);
+  if (ce == cudaSuccess) ce = launch_lm_combine(st, part, M, e.lm_tiles, d_argmax_out, d_conf_out);
+  if (ce != cudaSuccess) return fail(nullptr, NLD_ERR_CUDA, "LM-head launch failed: %s", cudaGetErrorString(ce));
+  return NLD_OK;
+}
+
+size_t nld_lm_head_workspace_size(int M, int d, int vocab) {
+  if (M < 1 || d < 128 || d % 128 || vocab < 1) return 0;
+  return lm_ssq_bytes(M, d) + lm_part_bytes(M, vocab);
+}
+
+nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int M, int d, int vocab,
+                              float rms_eps, int32_t* d_argmax_out, float* d_conf_out,
+                              void* d_workspace, size_t workspace_bytes, void* cuda_stream) {
+  TRY(lm_head_check(d_hidden, d_lm_weight, M, d, vocab, d_argmax_out, d_conf_out));
+  const size_t need = nld_lm_head_workspace_size(M, d, vocab);
+  if (!d_workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(d_workspace) % 256)
+    return fail(nullptr, NLD_ERR_ARG, "workspace must be 256-byte aligned and at least %zu bytes", need);
+  return lm_head_launch(d_hidden, d_lm_weight, M, d, vocab, rms_eps, d_argmax_out, d_conf_out,
+                        static_cast<char*>(d_workspace), static_cast<cudaStream_t>(cuda_stream));
+}
 
 // ----------------------------------------------------------------- stand-alone attention --
 static int device_sms() {

@@ -82,6 +82,8 @@ struct alignas(64) PhaseArgs {
   int tok_tiles, row_tiles, KT;
   int s;            // ranks of a cluster splitting each tile's K range (divides CS)
   int ks;           // k-iterations per rank
+  int w_rowmajor;   // 1: tmW views a plain row-major [n_rows, K] matrix (box {64, 128} at
+                    // (k*64, row)); 0: the pre-tiled layout
 };
 
 // A persistent launch running nph projections in order, separated by grid-wide arrivals.
@@ -156,5 +158,10 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
                           int n_rows, int K, const void* gamma, bool bf16, bool tiled);
 cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
+// Per 128-column tile sums of squares of bf16 rows h [M, d] into ssq [d/128, M].
+cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq);
+// Per token: argmax (lowest id on ties) and largest softmax probability from LM-head partials.
+cudaError_t launch_lm_combine(cudaStream_t st, const LmPart* part, int M, int tiles, int* argmax,
+                              float* conf);
 
 }  // namespace nld
