@@ -216,6 +216,26 @@ nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int
                               void* d_workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * nld_lm_head_argmax without a caller workspace, for callers that cannot allocate device
+ * memory: code inside a framework that owns every device allocation through its own pool, and
+ * latency-critical paths where cudaMalloc / cudaFree would synchronise the device.  The paper
+ * has no counterpart; this is a deployment convenience.
+ *   Same arguments, results and stream ordering as nld_lm_head_argmax, minus the workspace.
+ *   Scratch: a fixed array built into the library (nld_lm_head_static_max_bytes() = 8 MiB per
+ *   GPU, held from library load until process exit).  Shapes needing more scratch than that,
+ *   M * (d/128 * 4 + ceil(vocab/128) * 16) bytes plus alignment, fail with NLD_ERR_ARG and
+ *   launch nothing.  Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ *   make that first call before any stream capture on that device.
+ *   Every call shares the one array and leaves its contents behind (each call overwrites all
+ *   it reads, so nothing needs clearing); calls that overlap on the GPU race on it.
+ */
+size_t nld_lm_head_static_max_bytes(void);
+nld_status nld_lm_head_argmax_static(const void* d_hidden, const void* d_lm_weight, int M, int d,
+                                     int vocab, float rms_eps, int32_t* d_argmax_out,
+                                     float* d_conf_out, void* cuda_stream);
+
+/*
  * Stand-alone block-causal GQA attention over a paged bf16 KV cache (the attention step of
  * the forwards above, exposed for the attention micro-workload).  Notes section 3.2 / r9-hu
  * "Method": a query sees every cached key and the keys of its own and earlier blocks.

@@ -69,6 +69,8 @@ def load_library() -> ctypes.CDLL:
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
         "nld_lm_head_workspace_size": ([I, I, I], S),
         "nld_lm_head_argmax": ([P, P, I, I, I, F, P, P, P, S, P], I),
+        "nld_lm_head_static_max_bytes": ([], S),
+        "nld_lm_head_argmax_static": ([P, P, I, I, I, F, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -220,5 +222,17 @@ def nld_lm_head_argmax(hidden, lm_weight, rms_eps: float, argmax_out, conf_out, 
     st = lib.nld_lm_head_argmax(_ptr(hidden), _ptr(lm_weight), M, d, vocab, float(rms_eps),
                                 _ptr(argmax_out), _ptr(conf_out), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), stream)
+    if st != 0:
+        raise NldError(st, lib.nld_last_error(None).decode())
+
+
+def nld_lm_head_argmax_static(hidden, lm_weight, rms_eps: float, argmax_out, conf_out,
+                              stream: Optional[int] = None) -> None:
+    """nld_lm_head_argmax with the library's built-in scratch (allocates nothing)."""
+    lib = load_library()
+    M, d = hidden.shape
+    vocab = lm_weight.shape[0]
+    st = lib.nld_lm_head_argmax_static(_ptr(hidden), _ptr(lm_weight), M, d, vocab, float(rms_eps),
+                                       _ptr(argmax_out), _ptr(conf_out), stream)
     if st != 0:
         raise NldError(st, lib.nld_last_error(None).decode())

@@ -15,6 +15,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -1286,6 +1287,56 @@ nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int
     return fail(nullptr, NLD_ERR_ARG, "workspace must be 256-byte aligned and at least %zu bytes", need);
   return lm_head_launch(d_hidden, d_lm_weight, M, d, vocab, rms_eps, d_argmax_out, d_conf_out,
                         static_cast<char*>(d_workspace), static_cast<cudaStream_t>(cuda_stream));
+}
+
+// ------------------------------------------- LM head with built-in scratch (no allocation) --
+// For callers that cannot allocate device memory: code running inside a framework that owns
+// all device memory through its own pool (a raw cudaMalloc would bypass its budget), and
+// latency-critical paths where cudaMalloc / cudaFree would synchronise the device.  The
+// scratch of nld_lm_head_argmax lives in this fixed array instead; every GPU that loads the
+// library holds it until the process exits.
+constexpr size_t kStaticLmScratchBytes = 8u << 20;
+static __device__ __align__(256) unsigned char g_lm_scratch[kStaticLmScratchBytes];
+
+// Device address of g_lm_scratch per device (host code may not use the symbol itself as an
+// address): looked up with cudaGetSymbolAddress on the first call made on each device.
+static std::mutex g_lm_scratch_mu;
+static void* g_lm_scratch_addr[64] = {nullptr};
+
+size_t nld_lm_head_static_max_bytes(void) { return kStaticLmScratchBytes; }
+
+nld_status nld_lm_head_argmax_static(const void* d_hidden, const void* d_lm_weight, int M, int d,
+                                     int vocab, float rms_eps, int32_t* d_argmax_out,
+                                     float* d_conf_out, void* cuda_stream) {
+  TRY(lm_head_check(d_hidden, d_lm_weight, M, d, vocab, d_argmax_out, d_conf_out));
+  const size_t need = nld_lm_head_workspace_size(M, d, vocab);
+  if (need > kStaticLmScratchBytes)
+    return fail(nullptr, NLD_ERR_ARG,
+                "scratch of %zu bytes exceeds the built-in %zu bytes: M * (d/128 * 4 + ceil(vocab/128) * 16) "
+                "must stay within it (use nld_lm_head_argmax with a caller workspace)",
+                need, kStaticLmScratchBytes);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return fail(nullptr, NLD_ERR_CUDA, "no usable current CUDA device");
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_lm_scratch_mu);
+    if (!g_lm_scratch_addr[dev]) {
+      void* ptr = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&ptr, g_lm_scratch);
+      if (e != cudaSuccess || !ptr) {
+        cudaGetLastError();
+        return fail(nullptr, NLD_ERR_CUDA, "cudaGetSymbolAddress of the built-in scratch failed: %s",
+                    cudaGetErrorString(e));
+      }
+      g_lm_scratch_addr[dev] = ptr;
+    }
+    scratch = g_lm_scratch_addr[dev];
+  }
+  return lm_head_launch(d_hidden, d_lm_weight, M, d, vocab, rms_eps, d_argmax_out, d_conf_out,
+                        static_cast<char*>(scratch), static_cast<cudaStream_t>(cuda_stream));
 }
 
 // ----------------------------------------------------------------- stand-alone attention --
