@@ -43,7 +43,7 @@ def peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "epilogue.cuh", "common.cuh"):
+    for f in ("gemm_tc.cu", "epilogue.cuh", "common.cuh", "nld_internal.h"):
         h.update(open(os.path.join(ROOT, "self_speculation_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -270,10 +270,17 @@ def run_ours(args, world, rank, local):
         byts = 2 * nr * kd + 2 * M * kd + (2 * M * nr // (2 if nm == "gate_up" else 1))
         kern[nm] = {"ms": round(t, 5), "GB/s": round(byts / (t / 1e3) / 1e9, 1),
                     "bytes": byts}
-    gu = kern["gate_up"]
-    roofline = {"bound": "hbm", "achieved": gu["GB/s"], "peak": hbm, "unit": "GB/s",
-                "frac": round(gu["GB/s"] / hbm, 4), "traffic": ncu_traffic("gemm_gate_up_8b_m33.txt"),
-                "kernel": "gemm_tc_kernel gate/up (8B, M=33 tokens), timed alone",
+    # dominant kernel: the decode chain of a layer (O, gate/up, down, next layer's QKV in one
+    # persistent launch), timed alone over the verify forward's M = k+1 rows
+    ch_ms = ctx.nld_time_chain(0, M, 20)
+    ch_bytes = sum(kern[n]["bytes"] for n in ("o", "gate_up", "down", "qkv"))
+    ch_gbs = ch_bytes / (ch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(ch_gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ch_gbs / hbm, 4),
+                "traffic": ncu_traffic("gemm_chain_layer_8b_m32.txt"),
+                "kernel": "gemm_chain_kernel: one decode layer (O, gate/up, down, next QKV), "
+                          "8B shape, M=33 tokens, timed alone with CUDA events",
+                "bytes_per_launch": ch_bytes, "ms_per_launch": round(ch_ms, 5),
                 "peak_kind": f"{peak_src} HBM copy (burst)"}
 
     # end to end through the public API: prompt H2D from pinned memory, prefill, K rounds, each

@@ -173,6 +173,11 @@ nld_status nld_time_gemm(nld_ctx* ctx, int which, int layer, int M, int reps, fl
 nld_status nld_trace_gemm(nld_ctx* ctx, int which, int layer, int M, unsigned long long* d_trace,
                           int* grid_out);
 
+/* Profiling hook: the decode chain of `layer` (O-proj, gate/up, down, then layer+1's QKV; one
+ * launch) `reps` times back to back on the context stream over M token rows, between two CUDA
+ * events; *ms_out = mean milliseconds per launch.  Synchronises; writes only scratch. */
+nld_status nld_time_chain(nld_ctx* ctx, int layer, int M, int reps, float* ms_out);
+
 /* Profiling hook: one traced launch of the decode chain of `layer` (O-proj, gate/up, down,
  * then layer+1's QKV) over M token rows (as nld_time_gemm, 0 <= layer < n_layers-1); d_trace
  * receives per CTA 16 globaltimer stamps (ns): 0 start, 1 set-up done, for phase p = 0..3:

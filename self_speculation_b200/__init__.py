@@ -64,6 +64,7 @@ def load_library() -> ctypes.CDLL:
         "nld_trace_gemm": ([P, I, I, I, P, ctypes.POINTER(I)], I),
         "nld_debug_gemm_plan": ([P, I, I, ctypes.POINTER(I)], I),
         "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
+        "nld_time_chain": ([P, I, I, I, ctypes.POINTER(F)], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
@@ -178,6 +179,11 @@ class Context:
         self._check(self.lib.nld_trace_gemm(self.h, which, layer, M, _ptr(trace), ctypes.byref(g)),
                     self.h)
         return g.value
+
+    def nld_time_chain(self, layer: int, M: int, reps: int) -> float:
+        ms = ctypes.c_float(0.0)
+        self._check(self.lib.nld_time_chain(self.h, layer, M, reps, ctypes.byref(ms)), self.h)
+        return ms.value
 
     def nld_trace_chain(self, layer: int, M: int, trace) -> int:
         g = ctypes.c_int(0)

@@ -1155,6 +1155,31 @@ nld_status nld_trace_chain(nld_ctx* x, int layer, int M, unsigned long long* d_t
   return NLD_OK;
 }
 
+nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out) {
+  TRY(need_started(x));
+  if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
+  if (layer < 0 || layer + 1 >= x->c.n_layers || M < 1 || M > x->M_max || M % x->batch || reps < 1 || !ms_out)
+    return fail(x, NLD_ERR_ARG, "bad timing arguments");
+  TRY(ensure_capacity(x, M / x->batch));
+  ProjRef pr[4] = {hook_proj(x, GW_O, layer, M), hook_proj(x, GW_GU, layer, M),
+                   hook_proj(x, GW_D, layer, M), hook_proj(x, GW_QKV, layer + 1, M)};
+  unsigned* bar = x->bars + (1 + layer) * kMaxPhases;
+  cudaEvent_t a, b;
+  CK(cudaEventCreate(&a));
+  CK(cudaEventCreate(&b));
+  TRY(chain(x, pr, 4, M, false, bar, nullptr, 0));
+  CK(cudaEventRecord(a, x->stream));
+  for (int i = 0; i < reps; ++i) TRY(chain(x, pr, 4, M, false, bar, nullptr, 0));
+  CK(cudaEventRecord(b, x->stream));
+  CK(cudaEventSynchronize(b));
+  float ms = 0.f;
+  CK(cudaEventElapsedTime(&ms, a, b));
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  *ms_out = ms / reps;
+  return NLD_OK;
+}
+
 nld_status nld_debug_gemm_plan(nld_ctx* x, int which, int M, int* out8) {
   if (!x || !out8) return fail(x, NLD_ERR_ARG, "NULL argument");
   if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
