@@ -388,6 +388,201 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def _events_ms(fn, stream, reps, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_attention(args):
+    """Attention micro-workload: 32 q / 8 kv heads x 128, a block of 32 queries per sequence after
+    a cached prefix of 1k/4k/16k/32k, batch 1/8/32, modes block-bidirectional (block 32), strict
+    causal and block size 1.  Q/K/V ~ N(0,1) bf16 (seed 2) in a paged pool.  HBM bytes per call:
+    B*(L+32)*8*128*2*2 (K and V) + 2*B*32*32*128*2 (Q and O)."""
+    import torch
+
+    import self_speculation_b200 as nb
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    hbm, peak_src = peaks()
+    Hq, Hkv, hd, m = 32, 8, 128, 32
+    stream = torch.cuda.current_stream()
+    points = []
+    for L in (1024, 4096, 16384, 32768):
+        for B in (1, 8, 32):
+            pps = (L + m + 63) // 64
+            n_pages = B * pps
+            g = torch.Generator(device="cuda").manual_seed(2)
+            pool = torch.randn((n_pages, 2, Hkv, 64, hd), generator=g, device="cuda").to(torch.bfloat16)
+            q = torch.randn((B, m, Hq, hd), generator=g, device="cuda").to(torch.bfloat16)
+            perm = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).view(B, pps)
+            lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+            out = torch.empty_like(q)
+            byts = B * (L + m) * Hkv * hd * 2 * 2 + 2 * B * m * Hq * hd * 2
+            for mode, bs in (("block", 32), ("causal", 1), ("block_size_1", 1)):
+                ms = _events_ms(lambda: nb.nld_attention(q, pool, perm, lens, bs, L + m, out,
+                                                         stream.cuda_stream), stream, reps=20)
+                gbs = byts / (ms / 1e3) / 1e9
+                points.append({"prefix": L, "batch": B, "mode": mode, "us": round(ms * 1e3, 2),
+                               "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                               "l2_resident": byts < 126e6})
+            del pool, q, perm, out
+            torch.cuda.empty_cache()
+    big = [p for p in points if not p["l2_resident"]]
+    best = max(big, key=lambda p: p["GB/s"])
+    print(json.dumps({
+        "metric": "attention HBM throughput (block-causal GQA over paged bf16 KV)",
+        "value": best["GB/s"], "unit": "GB/s", "n_gpus": 1, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "attention micro-workload: 32q/8kv x 128, 32 queries per sequence",
+                   "l2": "not flushed: points under 126 MB are marked l2_resident"},
+        "roofline": {"bound": "hbm", "achieved": best["GB/s"], "peak": hbm, "unit": "GB/s",
+                     "frac": best["frac"], "traffic": None, "peak_kind": f"{peak_src} HBM copy"},
+        "points": points}), flush=True)
+
+
+def _model_ctx(cfg, seed=0):
+    import torch
+
+    import self_speculation_b200 as nb
+    import synth
+    st = torch.cuda.Stream()
+    ctx = nb.Context(cfg, stream=st.cuda_stream)
+    w = synth.model_weights(cfg, seed, device="cuda")
+    ctx.nld_init_weights(w, on_device=True)
+    del w
+    torch.cuda.empty_cache()
+    return ctx, st
+
+
+def run_diffusion(args):
+    """8B-shaped block diffusion: block 32 of [MASK], confidence threshold 0.9 (at least one commit
+    per step), batch 1/4/16, prompt 2048 random ids; steps until 512 tokens per sequence are
+    committed (lockstep; the causal KV fill runs when every block is complete)."""
+    import torch
+
+    import synth
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    hbm, peak_src = peaks()
+    P, N = 2048, 512
+    pts = []
+    for B in (1, 4, 16):
+        cfg = synth.LLAMA8B.replace(max_batch=B, max_seq=P + N + 128)
+        ctx, st = _model_ctx(cfg)
+        ctx.nld_prefill(synth.prompt_tokens(B, P, cfg.vocab, seed=1).cuda())
+        k = cfg.block_k
+        blk = torch.empty(B, k, dtype=torch.int32, device="cuda")
+        conf = torch.empty(B, k, dtype=torch.float32, device="cuda")
+        nc = torch.empty(B, dtype=torch.int32, device="cuda")
+        for _ in range(3):
+            ctx.nld_diffuse_block_step(0.9, blk, conf, nc)
+        lens = torch.empty(B, dtype=torch.int32, device="cuda")
+        ctx.nld_debug_state(lens)
+        ctx.nld_sync()
+        l0 = lens.clone()
+        torch.cuda.synchronize()
+        steps, fills, t0 = 0, 0, time.perf_counter()
+        committed = 0
+        while committed < N and steps < 4 * N:
+            fills += int(ctx.nld_diffuse_block_step(0.9, blk, conf, nc))
+            committed += int(nc.min())
+            steps += 1
+        ctx.nld_sync()
+        dt = time.perf_counter() - t0
+        ctx.nld_debug_state(lens)
+        ctx.nld_sync()
+        tok = int((lens - l0).sum()) + int((blk != cfg.vocab).sum()) * 0
+        step_bytes = cfg.weight_bytes_per_forward() + B * (P + N / 2) * cfg.kv_bytes_per_token()
+        fwd = steps + fills
+        pts.append({"batch": B, "steps": steps, "kv_fills": fills, "s": round(dt, 3),
+                    "committed_tokens": committed * B, "tokens_per_s": round(committed * B / dt, 2),
+                    "steps_per_s": round(steps / dt, 2),
+                    "hbm_frac": round(step_bytes * fwd / dt / 1e9 / hbm, 4)})
+        ctx.close()
+        del ctx
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    print(json.dumps({
+        "metric": "committed tokens/s, 8B-shaped block diffusion (tau 0.9)", "value": pts[-1]["tokens_per_s"],
+        "unit": "tokens/s", "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "8B-shaped diffusion mode, block 32, prompt 2048, 512 tokens",
+                   "timing": "host wall clock per step (each step synchronises once by design)"},
+        "points": pts}), flush=True)
+
+
+def run_sweep14b(args):
+    """14B-shaped concurrency sweep: 40 layers, d 5120, 40/8 heads x 128, FFN 17408, vocab 151936;
+    4k-token random prefixes; batch 1/4/16/64; AR step vs self-spec round (k=32) vs diffusion
+    step; tokens/s per user and aggregate."""
+    import torch
+
+    import synth
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    hbm, peak_src = peaks()
+    P = 4096
+    reps = max(3, args.steps // 10)
+    pts = []
+    for B in (1, 4, 16, 64):
+        cfg = synth.LLAMA14B.replace(max_batch=B, max_seq=P + 33 * (3 * reps + 12) + 64)
+        ctx, st = _model_ctx(cfg)
+        ctx.nld_prefill(synth.prompt_tokens(B, P, cfg.vocab, seed=1).cuda())
+        k = cfg.block_k
+        t1 = torch.empty(B, dtype=torch.int32, device="cuda")
+        tk = torch.empty(B, k + 1, dtype=torch.int32, device="cuda")
+        nc = torch.empty(B, dtype=torch.int32, device="cuda")
+        lens = torch.empty(B, dtype=torch.int32, device="cuda")
+        ar_ms = _events_ms(lambda: ctx.nld_ar_step(t1), st, reps)
+        ctx.nld_debug_state(lens)
+        ctx.nld_sync()
+        l0 = int(lens.sum())
+        ss_ms = _events_ms(lambda: ctx.nld_selfspec_round(tk, nc, None), st, reps, warm=2)
+        ctx.nld_debug_state(lens)
+        ctx.nld_sync()
+        ss_tok = (int(lens.sum()) - l0) / (reps + 2)
+        blk = torch.empty(B, k, dtype=torch.int32, device="cuda")
+        cf = torch.empty(B, k, dtype=torch.float32, device="cuda")
+        t0 = time.perf_counter()
+        dsteps, dtok = 0, 0
+        for _ in range(reps):
+            ctx.nld_diffuse_block_step(0.9, blk, cf, nc)
+            dtok += int(nc.sum())
+            dsteps += 1
+        d_s = (time.perf_counter() - t0) / dsteps
+        wb = cfg.weight_bytes_per_forward()
+        kvb = B * P * cfg.kv_bytes_per_token()
+        pts.append({
+            "batch": B,
+            "ar": {"ms": round(ar_ms, 3), "tokens_per_s": round(B / (ar_ms / 1e3), 1),
+                   "per_user": round(1 / (ar_ms / 1e3), 1),
+                   "hbm_frac": round((wb + kvb) / (ar_ms / 1e3) / 1e9 / hbm, 4)},
+            "selfspec": {"ms": round(ss_ms, 3), "tokens_per_s": round(ss_tok / (ss_ms / 1e3), 1),
+                         "per_user": round(ss_tok / B / (ss_ms / 1e3), 1),
+                         "hbm_frac": round(2 * (wb + kvb) / (ss_ms / 1e3) / 1e9 / hbm, 4)},
+            "diffusion": {"ms": round(d_s * 1e3, 3), "tokens_per_s": round(dtok / dsteps / d_s, 1),
+                          "per_user": round(dtok / dsteps / B / d_s, 1)}})
+        ctx.close()
+        del ctx
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    print(json.dumps({
+        "metric": "tokens/s per user and aggregate, 14B shape (AR / self-spec / diffusion)",
+        "value": pts[-1]["ar"]["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "14B-shaped concurrency sweep, 4k prefixes, batch 1/4/16/64"},
+        "points": pts}), flush=True)
+
+
 def run_probe(args):
     """Small case for ncu captures: a 2-layer model of the 8B layer shape (full vocab), prompt
     512, then each projection GEMM launched alone at M=33 tokens (nld_time_gemm, reps=2) and one
@@ -442,6 +637,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b"],
+                    default="selfspec8b")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
     args = ap.parse_args()
@@ -450,6 +647,12 @@ def main():
     world, rank, local = dist_setup()
     if args.probe:
         run_probe(args)
+    elif args.workload == "attention":
+        run_attention(args)
+    elif args.workload == "diffusion8b":
+        run_diffusion(args)
+    elif args.workload == "sweep14b":
+        run_sweep14b(args)
     elif args.impl == "reference":
         run_reference(args, world, rank, local)
     else:
