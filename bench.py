@@ -323,7 +323,10 @@ def run_ours(args, world, rank, local):
                           f"work); {ncommit} committed token(s) in the sampled round"),
                "round_s_est": round(round_est, 2)}
 
-    per_round = 2 * (1 + 5 * cfg.n_layers + 1 + 1) + 1
+    # two forwards (draft, verify), each: embed, QKV chain of layer 0, per layer one attention
+    # and one chain (O, gate/up, down, next QKV), LM-head chain; then finalize for draft,
+    # verify and commit
+    per_round = 2 * (1 + 1 + 2 * cfg.n_layers + 1) + 3
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
