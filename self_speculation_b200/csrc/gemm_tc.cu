@@ -121,11 +121,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int S = A.stages;
   const int NT = A.NT;
-  const int xbytes = NT * 128;
+  const int KPS = A.kps;
+  const int xbytes = A.xr * 128;       // one k-tile of activations: xr token rows x 128 B
+  const int wst = KPS * kStageW;       // one stage: KPS k-tiles of weights ...
+  const int xst = KPS * xbytes;        // ... and of activations
   const int CS = A.CS;
   uint8_t* sW = smem;
-  uint8_t* sX = smem + S * kStageW;
-  float* staging = reinterpret_cast<float*>(sX + S * xbytes);          // [2][NT][128] if CS>1
+  uint8_t* sX = smem + S * wst;
+  float* staging = reinterpret_cast<float*>(sX + S * xst);             // [2][NT][128] if CS>1
   const int stg_floats = (CS > 1) ? NT * kTileRows : 0;
   GemmTail* tail = reinterpret_cast<GemmTail*>(staging + 2 * stg_floats);
 
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------- TMA producer --
       const uint64_t pol = l2_policy_evict_first();
-      int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages];
+      int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages], q_nk[kMaxStages];
       int it = 0;
       bool ok = true;
       for (int p = 0; ok && p < A.nph; ++p) {
@@ -196,8 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_global();
           }
           for (int i = 0; i < nq; ++i)
-            tma_load_2d(sX + q_stage[i] * xbytes, &P.tmX, &tail->full[q_stage[i]], q_k[i] * kTileK,
-                        q_tt[i] * NT);
+            for (int j = 0; j < q_nk[i]; ++j)
+              tma_load_2d(sX + q_stage[i] * xst + j * xbytes, &P.tmX, &tail->full[q_stage[i]],
+                          (q_k[i] + j) * kTileK, q_tt[i] * NT);
           nq = 0;
           ready = true;
           return true;
@@ -205,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = w.grp; ok && t < w.tiles; t += w.ngrp) {
           const int r = t / P.tok_tiles;
           const int tt = t - r * P.tok_tiles;
-          for (int kt = w.k_lo; kt < w.k_hi; ++kt, ++it) {
+          for (int kt = w.k_lo; kt < w.k_hi; kt += KPS, ++it) {
+            const int nk = min(KPS, w.k_hi - kt);
             const int stage = it % S;
             const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
             // a slot still holding an earlier phase's stage frees without the grid counter; once
@@ -217,20 +222,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kt == w.k_lo && t == w.grp) trace_mark(A, 2 + 3 * p);
             trace_iter(A, 2, it - S);
             trace_iter(A, 0, it);
-            mbar_arrive_expect_tx(&tail->full[stage], kStageW + xbytes);
+            mbar_arrive_expect_tx(&tail->full[stage], nk * (kStageW + xbytes));
             // pre-tiled weights: block (r, kt) is one contiguous 16 KB box
-            if (P.w_rowmajor)
-              tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], kt * kTileK,
-                               r * kTileRows, pol);
-            else
-              tma_load_2d_hint(sW + stage * kStageW, &P.tmW, &tail->full[stage], 0,
-                               (r * P.KT + kt) * kTileRows, pol);
+            for (int j = 0; j < nk; ++j) {
+              if (P.w_rowmajor)
+                tma_load_2d_hint(sW + stage * wst + j * kStageW, &P.tmW, &tail->full[stage],
+                                 (kt + j) * kTileK, r * kTileRows, pol);
+              else
+                tma_load_2d_hint(sW + stage * wst + j * kStageW, &P.tmW, &tail->full[stage], 0,
+                                 (r * P.KT + kt + j) * kTileRows, pol);
+            }
             if (ready) {
-              tma_load_2d(sX + stage * xbytes, &P.tmX, &tail->full[stage], kt * kTileK, tt * NT);
+              for (int j = 0; j < nk; ++j)
+                tma_load_2d(sX + stage * xst + j * xbytes, &P.tmX, &tail->full[stage],
+                            (kt + j) * kTileK, tt * NT);
             } else {
               q_stage[nq] = stage;
               q_k[nq] = kt;
               q_tt[nq] = tt;
+              q_nk[nq] = nk;
               if (++nq == S && !become_ready()) { ok = false; break; }
             }
           }
@@ -274,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t d = tmem + tb * buf_cols;
-          for (int kt = w.k_lo; kt < w.k_hi; ++kt, ++it) {
+          for (int kt = w.k_lo; kt < w.k_hi; kt += KPS, ++it) {
+            const int nk = min(KPS, w.k_hi - kt);
             const int stage = it % S;
             const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
             if (!wait_or_abort(&tail->full[stage], ph, timeout_ns, tail, err)) {
@@ -283,11 +294,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             trace_iter(A, 1, it);
-            const uint64_t da = sdesc_k_sw128(smem_u32(sW + stage * kStageW));
-            const uint64_t db = sdesc_k_sw128(smem_u32(sX + stage * xbytes));
+            for (int j = 0; j < nk; ++j) {
+              // B reads NT token rows from an xr-row block: rows past xr are padding columns of
+              // the tile (stale shared memory, never used by the epilogue)
+              const uint64_t da = sdesc_k_sw128(smem_u32(sW + stage * wst + j * kStageW));
+              const uint64_t db = sdesc_k_sw128(smem_u32(sX + stage * xst + j * xbytes));
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk)
-              tc_mma_f16(d, da + 2 * kk, db + 2 * kk, idesc, (kt > w.k_lo || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kTileK / 16; ++kk)
+                tc_mma_f16(d, da + 2 * kk, db + 2 * kk, idesc, (kt > w.k_lo || j > 0 || kk > 0) ? 1u : 0u);
+            }
             tc_commit(&tail->empty[stage]);
           }
           if (!ok) break;
@@ -438,10 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_mark(A, 15);
 }
 
-size_t gemm_chain_smem_bytes(int NT, int stages, int CS) {
+size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS) {
   const size_t stg = (CS > 1) ? 2ull * NT * kTileRows * sizeof(float) : 0;
-  return 1024 + static_cast<size_t>(stages) * (kStageW + NT * 128) + stg + sizeof(GemmTail);
+  return 1024 + static_cast<size_t>(stages) * kps * (kStageW + xr * 128) + stg + sizeof(GemmTail);
 }
+int gemm_chain_max_stages() { return kMaxStages; }
 
 cudaError_t gemm_tc_init_attributes() {
   int dev = 0, optin = 0;
@@ -482,7 +498,7 @@ cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uin
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.stages, A.CS);
+  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;

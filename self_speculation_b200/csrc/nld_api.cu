@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -208,14 +209,14 @@ struct ProjRef {
   EpiArgs e;
 };
 
-const CUtensorMap* xmap(nld_ctx* x, int buf, int NT) {
-  auto key = std::make_pair(buf, NT);
+const CUtensorMap* xmap(nld_ctx* x, int buf, int rows) {
+  auto key = std::make_pair(buf, rows);
   auto it = x->tmX.find(key);
   if (it != x->tmX.end()) return &it->second;
   CUtensorMap m;
   const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
   const int inner = buf == XB_HB ? x->c.d_model : (buf == XB_ATTN ? x->qd : x->c.ffn_dim);
-  if (!make_map_bf16(&m, base, inner, x->M_max, NT)) return nullptr;
+  if (!make_map_bf16(&m, base, inner, x->M_max, rows)) return nullptr;
   return &(x->tmX[key] = m);
 }
 
@@ -297,9 +298,19 @@ ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const in
       best_grid = std::min(C, need_clusters) * CS;
     }
   }
-  const int stage_bytes = kTileRows * kTileK * 2 + NT * 128;
-  const int staging = (best.CS > 1) ? 2 * NT * kTileRows * 4 : 0;
-  best.stages = std::max(2, std::min(8, (216 * 1024 - staging - 4096) / stage_bytes));
+  // activations: the token tile's rows rounded up to 8 (a multiple of the 128-byte swizzle
+  // atom's 8 rows), so a decode tile of 33 tokens moves 40 rows per k-tile, not NT = 48
+  // (several token tiles: every tile but the last is full, so all NT rows)
+  best.xr = (tok_tiles == 1) ? std::min(NT, (M + 7) / 8 * 8) : NT;
+  // two k-tiles (32 KB of weights) per stage: the producer/MMA barrier round trip, not HBM,
+  // bounds a ring of 16 KB stages; as many stages as fit the shared-memory budget
+  best.kps = 2;
+  best.stages = 2;
+  for (int st = gemm_chain_max_stages(); st > 2; --st)
+    if (gemm_chain_smem_bytes(NT, best.xr, best.kps, st, best.CS) <= kChainSmemBudget) {
+      best.stages = st;
+      break;
+    }
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(2 * NT)) cols <<= 1;
   best.tmem_cols = cols;
@@ -338,7 +349,7 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
   for (int p = 0; p < nph; ++p) {
     const WInfo w = winfo(x, pr[p].which, pr[p].layer);
     A.ph[p].tmW = *w.map;
-    const CUtensorMap* tmX = xmap(x, w.buf, A.NT);
+    const CUtensorMap* tmX = xmap(x, w.buf, A.xr);
     if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
     A.ph[p].tmX = *tmX;
     A.ph[p].e = pr[p].e;
@@ -358,7 +369,7 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
     A.next_KT = N.ph[0].KT;
     A.next_grid = ngrid;
     A.next_tiles = N.ph[0].row_tiles * N.ph[0].tok_tiles;
-    A.next_boxes = N.stages;
+    A.next_boxes = N.stages * N.kps;
     A.tmWn = *winfo(x, next_pr[0].which, next_pr[0].layer).map;
   }
   CK(launch_gemm_chain(x->stream, A, grid, x->timeout_ns, pdl));
@@ -1274,7 +1285,7 @@ static nld_status lm_head_launch(const void* d_hidden, const void* d_lm_weight, 
   ChainArgs A = plan_chain_shapes(device_max_clusters(), &nr, &kd, 1, M, &grid);
   PhaseArgs& P = A.ph[0];
   if (!make_map_bf16(&P.tmW, d_lm_weight, d, vocab, kTileRows) ||
-      !make_map_bf16(&P.tmX, d_hidden, d, M, A.NT))
+      !make_map_bf16(&P.tmX, d_hidden, d, M, A.xr))
     return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed");
   P.w_rowmajor = 1;
   EpiArgs& e = P.e;

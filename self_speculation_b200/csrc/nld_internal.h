@@ -12,6 +12,7 @@ namespace nld {
 constexpr int kPage = 64;          // KV page length in tokens (one attention KV tile)
 constexpr int kTileRows = 128;     // GEMM weight rows per tile (tcgen05 M)
 constexpr int kTileK = 64;         // GEMM K per pipeline stage (128 bytes of bf16)
+constexpr int kChainSmemBudget = 227 * 1024;   // dynamic shared memory of one chain CTA (sm_100 opt-in)
 constexpr int kMaxNT = 256;        // max token columns per GEMM tile (tcgen05 N)
 
 // Epilogue kinds of the projection GEMMs.
@@ -93,7 +94,11 @@ struct alignas(64) ChainArgs {
   int nph;
   int CS;           // CTAs per cluster
   int NT;           // token columns per tile (multiple of 16, <= 256)
-  int stages;
+  int stages;       // shared-memory ring depth
+  int kps;          // k-tiles (of 64) per stage: one barrier round trip moves kps x 16 KB of weights
+  int xr;           // activation rows loaded per k-tile of a token tile: the tile's token count
+                    // rounded up to 8 (<= NT); the MMA's N = NT columns read past them into
+                    // padding columns that the epilogue never uses
   uint32_t tmem_cols;   // power of two >= 2*NT
   unsigned* bar;    // [kMaxPhases] phase-boundary arrival counters + exit counter (last slot);
                     // zero before the launch, left zero by it
@@ -121,7 +126,8 @@ struct AttnArgs {
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
 cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uint64_t timeout_ns,
                               bool pdl);
-size_t gemm_chain_smem_bytes(int NT, int stages, int CS);
+size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS);
+int gemm_chain_max_stages();
 int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
                              int M, const EpiArgs& e, bool pdl);
