@@ -631,6 +631,11 @@ def run_probe(args):
     print(json.dumps({"probe_ms": out}))
     print(json.dumps({"plans": plans}))
     print(json.dumps({"chain_trace_us_min_med_max": traces}))
+    # CTA 0's pipeline: per stage iteration issue / MMA start / slot freed, per tile epilogue
+    it = tr[148 * 16:148 * 16 + 256].view(4, 64).cpu().double()
+    rel = lambda v: [round((float(x) - float(t0)) / 1e3, 2) if x > 0 else None for x in v]
+    print(json.dumps({"cta0_pipeline_us": {"issue": rel(it[0]), "mma": rel(it[1]), "freed": rel(it[2]),
+                                           "epi_tiles": [rel(it[3][8 * i:8 * i + 7]) for i in range(8)]}}))
 
 
 def main():

@@ -218,6 +218,31 @@ NLD_DEV void mbar_arrive_remote_count(uint32_t cluster_addr, uint32_t count) {
                "r"(count)
                : "memory");
 }
+// Asynchronous 16-byte store into another cluster CTA's shared memory; the bytes count against
+// the transaction count of that CTA's mbarrier at remote_bar (both shared::cluster addresses).
+NLD_DEV void st_async_f4(uint32_t remote_addr, float4 v, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          remote_addr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar)
+      : "memory");
+}
+NLD_DEV uint32_t ld_dsmem_u32_relaxed(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.relaxed.cluster.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+NLD_DEV void st_shared_u32_relaxed_cluster(void* p, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+// Same without release semantics: for a signal that publishes no data of this thread (e.g.
+// "done reading your buffer", once the loaded values have been consumed), so the arrive does
+// not wait for this thread's outstanding global stores.
+NLD_DEV void mbar_arrive_remote_count_relaxed(uint32_t cluster_addr, uint32_t count) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+               "r"(count)
+               : "memory");
+}
 // Generic-proxy writes of other CTAs (made visible by a gpu-scope acquire) before this thread's
 // later async-proxy (TMA) reads of the same global memory.
 NLD_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }

@@ -17,42 +17,69 @@ namespace nld {
 // red_f / red_i: shared scratch of at least 4*16 + 16 entries each, private to the 4 warps (one
 // per TMEM lane quarter, 128 threads) that call this together and synchronise on named
 // barrier `bar_id`.
-// Global loads of a 16-column chunk are issued together before any store of the chunk, so a
-// chunk costs one memory round trip rather than sixteen.
+// The global operands of a 16-column chunk (epi_preload) are loaded together, ahead of the
+// accumulator values where the caller can (a split tile loads them before waiting for its
+// group's partials), so a chunk costs at most one memory round trip.
+struct EpiPre {
+  float a[32];   // EPI_RESID: residual h of the 16 tokens; EPI_QKV: RoPE (cos, sin) of each
+};
+
+NLD_DEV void qkv_row_info(const EpiArgs& e, int row, int& sec, int& head, int& lr, int& feat) {
+  const int qd = e.Hq * e.hd, kvd = e.Hkv * e.hd;
+  int base;
+  if (row < qd) {
+    sec = 0; base = 0;
+  } else if (row < qd + kvd) {
+    sec = 1; base = qd;
+  } else {
+    sec = 2; base = qd + kvd;
+  }
+  const int rr = row - base;
+  head = rr / e.hd;
+  lr = rr - head * e.hd;
+  const int half = e.hd >> 1;
+  feat = (sec == 2) ? lr : ((lr & 1) ? (lr >> 1) + half : (lr >> 1));
+}
+
+NLD_DEV void epi_preload(const EpiArgs& e, int row_tile, int row_in_tile, int tok0,
+                         const int* s_pos, int col0, EpiPre& p) {
+  const int row = row_tile * kTileRows + row_in_tile;
+  if (e.kind == EPI_RESID) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      p.a[j] = (tok0 + j < e.M) ? e.h[static_cast<size_t>(tok0 + j) * e.d + row] : 0.f;
+  } else if (e.kind == EPI_QKV) {
+    int sec, head, lr, feat;
+    qkv_row_info(e, row, sec, head, lr, feat);
+    const int half = e.hd >> 1;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int pos = s_pos[col0 + j];
+      const float2 cs = (sec < 2 && pos >= 0)
+                            ? __ldg(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)])
+                            : make_float2(1.f, 0.f);
+      p.a[2 * j] = cs.x;
+      p.a[2 * j + 1] = cs.y;
+    }
+  }
+}
+
 template <typename T>
 NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane, int ew,
                        int tok0, const float* s_inv, const int* s_pos, const int* s_pg, int col0,
-                       float (&v)[16], float* red_f, int* red_i, int bar_id) {
+                       float (&v)[16], const EpiPre& pre, float* red_f, int* red_i, int bar_id) {
   const int row = row_tile * kTileRows + row_in_tile;
   switch (e.kind) {
     case EPI_QKV: {
-      const int qd = e.Hq * e.hd, kvd = e.Hkv * e.hd;
-      int sec, base;
-      if (row < qd) {
-        sec = 0; base = 0;
-      } else if (row < qd + kvd) {
-        sec = 1; base = qd;
-      } else {
-        sec = 2; base = qd + kvd;
-      }
-      const int rr = row - base;
-      const int head = rr / e.hd;
-      const int lr = rr - head * e.hd;
-      const int half = e.hd >> 1;
-      const int feat = (sec == 2) ? lr : ((lr & 1) ? (lr >> 1) + half : (lr >> 1));
-      float2 cs[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int pos = s_pos[col0 + j];
-        cs[j] = (sec < 2 && pos >= 0) ? __ldg(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)])
-                                      : make_float2(1.f, 0.f);
-      }
+      int sec, head, lr, feat;
+      qkv_row_info(e, row, sec, head, lr, feat);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int tok = tok0 + j;
         float x = v[j] * s_inv[col0 + j];
         const float partner = __shfl_xor_sync(0xffffffffu, x, 1);
-        if (sec < 2) x = (lr & 1) ? (x * cs[j].x + partner * cs[j].y) : (x * cs[j].x - partner * cs[j].y);
+        const float c = pre.a[2 * j], sn = pre.a[2 * j + 1];
+        if (sec < 2) x = (lr & 1) ? (x * c + partner * sn) : (x * c - partner * sn);
         if (tok >= e.M || row >= e.n_rows) continue;
         if (sec == 0) {
           static_cast<T*>(e.q_out)[(static_cast<size_t>(tok) * e.Hq + head) * e.hd + feat] =
@@ -69,16 +96,12 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
     } break;
 
     case EPI_RESID: {
-      float hv[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        hv[j] = (tok0 + j < e.M) ? e.h[static_cast<size_t>(tok0 + j) * e.d + row] : 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int tok = tok0 + j;
         float hn = 0.f;
         if (tok < e.M) {
-          hn = hv[j] + v[j];
+          hn = pre.a[j] + v[j];
           e.h[static_cast<size_t>(tok) * e.d + row] = hn;
           static_cast<T*>(e.hb)[static_cast<size_t>(tok) * e.d + row] = from_f32<T>(hn);
         }

@@ -45,7 +45,9 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();
   }
-  epi_chunk<float>(e, rt, tid, tid & 31, tid >> 5, tok0, s_inv, s_pos, s_pg, 0, acc, red_f, red_i, 1);
+  EpiPre pre;
+  epi_preload(e, rt, tid, tok0, s_pos, 0, pre);
+  epi_chunk<float>(e, rt, tid, tid & 31, tid >> 5, tok0, s_inv, s_pos, s_pg, 0, acc, pre, red_f, red_i, 1);
 }
 
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,

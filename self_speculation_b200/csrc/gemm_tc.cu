@@ -9,10 +9,10 @@
 //
 // Work split: the CTAs of a cluster (CS of them) share output tiles; in a phase with split s
 // (a divisor of CS) each group of s ranks splits the K range of a tile, each rank accumulating
-// its slice in tensor memory.  The partials meet in shared memory: every rank copies its
-// accumulator into a staging buffer, tells its group with remote mbarrier arrives, reduces one
-// slice of the tile's token columns by reading the group's staging buffers over distributed
-// shared memory (rank order: sums do not depend on timing) and runs the fused epilogue on it.
+// its slice in tensor memory.  The tile's 16-column chunks are divided among the group; every
+// rank sends its partial of each chunk to the chunk's owner with st.async (a one-way write into
+// the owner's shared memory, counted by the owner's mbarrier), and the owner sums the partials
+// in rank order (sums do not depend on timing) and runs the fused epilogue on them.
 //
 // Phases: a CTA that finished its part of phase p adds one to a grid-wide arrival counter; the
 // next phase's activation loads and epilogue wait until every CTA has arrived.  Its weight
@@ -35,7 +35,10 @@ namespace {
 
 constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB of bf16 weights per stage
 constexpr int kMaxStages = 8;
-constexpr int kMaxSplit = 8;
+constexpr int kBoundaryPrefetch = 16;   // weight boxes prefetched into L2 per phase boundary
+constexpr int kSlotLd = 20;              // floats per row of a split-K slot: 16 + 4 (16-byte
+                                         // accesses of 8 consecutive rows hit distinct banks)
+constexpr int kSlotFloats = kTileRows * kSlotLd;
 constexpr int kEpiThreads = 256;   // 8 epilogue warps
 constexpr int kThreads = 64 + kEpiThreads;
 
@@ -44,8 +47,9 @@ struct GemmTail {
   uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t sfull[2];    // staging buffer b holds every group rank's partial (count: CS)
-  uint64_t sempty[2];   // every group rank has finished reading staging buffer b (count: CS)
+  uint64_t rfull;       // the group's partials of this CTA's chunks have arrived (count 1 + tx)
+  uint32_t done[kMaxPhases];   // split tiles of phase p whose chunks this CTA has reduced (read
+                               // by the group's other ranks before they write its slot area)
   uint32_t tmem_base;
   volatile int abort_flag;
   volatile int epi_abort;
@@ -76,13 +80,37 @@ NLD_DEV Work work_of(const ChainArgs& A, int p, int cl, int rank, int C) {
   return w;
 }
 
+// Transaction bytes of the next split tile after tile t_prev of phase p (t_prev = -1: from the
+// start of phase p) in which this CTA owns chunks: every other rank of the group sends it 64
+// bytes per row per owned chunk.  0 if there is none.
+NLD_DEV uint32_t next_owned_bytes(const ChainArgs& A, int p, int t_prev, int cl, int rank, int C) {
+  for (int q = p; q < A.nph; ++q) {
+    const PhaseArgs& P = A.ph[q];
+    const Work w = work_of(A, q, cl, rank, C);
+    if (w.s <= 1) continue;
+    for (int t = (q == p && t_prev >= 0) ? t_prev + w.ngrp : w.grp; t < w.tiles; t += w.ngrp) {
+      const int tt = t - (t / P.tok_tiles) * P.tok_tiles;
+      const int nvalid = min(A.NT, P.e.M - tt * A.NT);
+      const int nchunks = (nvalid + 15) >> 4;
+      const int per = (nchunks + w.s - 1) / w.s;
+      const int n_own = min(nchunks, (w.grank + 1) * per) - w.grank * per;
+      if (n_own > 0) return static_cast<uint32_t>((w.s - 1) * n_own * kTileRows * 64);
+    }
+  }
+  return 0;
+}
+
 // Phase timestamps of one CTA (profiling hook), trace[cta * 16 + slot]: 0 start, 1 set-up
 // done, per phase p: 2+3p first weight load issued, 3+3p epilogue may start (after the phase
 // counter), 4+3p epilogue done; 14 last MMA commit, 15 exit.
 NLD_DEV void trace_mark(const ChainArgs& A, int slot) {
   if (A.trace) A.trace[blockIdx.x * 16 + slot] = globaltimer_ns();
 }
-// Per-iteration pipeline stamps of CTA 0 (profiling hook): after the per-CTA slots.
+// Per-iteration pipeline stamps of CTA 0 (profiling hook), after the per-CTA slots: kind 0
+// stage `it` issued, 1 stage `it` consumed by the MMA, 2 stage `it` freed; kind 3 at 8i + k
+// for the epilogue of tile i: k = 0 accumulator ready, 1 partials sent, 2 the group's partials
+// received, 3 reduced and written (all threads), 4 done, 5 / 6 thread 0's sums formed / its
+// chunk written.
 NLD_DEV void trace_iter(const ChainArgs& A, int kind, int it) {
   if (A.trace && blockIdx.x == 0 && it >= 0 && it < 64)
     A.trace[148 * 16 + kind * 64 + it] = globaltimer_ns();
@@ -128,9 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int CS = A.CS;
   uint8_t* sW = smem;
   uint8_t* sX = smem + S * wst;
-  float* staging = reinterpret_cast<float*>(sX + S * xst);             // [2][NT][128] if CS>1
-  const int stg_floats = (CS > 1) ? NT * kTileRows : 0;
-  GemmTail* tail = reinterpret_cast<GemmTail*>(staging + 2 * stg_floats);
+  // split-K slot area (CS > 1): [A.slots][128 rows][kSlotLd] floats; for a split tile of group
+  // size s, slot (q * per + c) holds group rank q's partial of this CTA's c-th owned chunk
+  float* slots = reinterpret_cast<float*>(sX + S * xst);
+  GemmTail* tail = reinterpret_cast<GemmTail*>(slots + (CS > 1 ? A.slots * kSlotFloats : 0));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -149,12 +178,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tail->tfull[i], 1);
       mbar_init(&tail->tempty[i], kEpiThreads);
-      mbar_init(&tail->sfull[i], CS);
-      mbar_init(&tail->sempty[i], CS);
     }
+    mbar_init(&tail->rfull, 1);
+    for (int p = 0; p < kMaxPhases; ++p) tail->done[p] = 0;
     tail->abort_flag = 0;
     tail->epi_abort = 0;
     fence_mbar_init();
+    // the first split tile whose chunks this CTA owns: its transaction count is armed before
+    // any rank of the cluster can send (they all pass the cluster barrier below first)
+    if (CS > 1) {
+      const uint32_t b0 = next_owned_bytes(A, 0, -1, blockIdx.x / CS, static_cast<int>(cluster_ctarank()),
+                                           static_cast<int>(gridDim.x) / CS);
+      if (b0) mbar_arrive_expect_tx(&tail->rfull, b0);
+    }
     for (int p = 0; p < A.nph; ++p) {
       tma_prefetch_desc(&A.ph[p].tmW);
       tma_prefetch_desc(&A.ph[p].tmX);
@@ -187,14 +223,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         // CTA to finish phase p-1; weight loads run ahead into the free stages meanwhile
         bool ready = false;
         int nq = 0;
-        auto become_ready = [&]() -> bool {
+        // (tn, ktn): the next weight box this CTA loads after the ring's queued stages; while
+        // the phase boundary is waited on, the TMA unit is idle, so it prefetches the following
+        // boxes into L2 and HBM keeps streaming through the boundary
+        auto become_ready = [&](int tn, int ktn) -> bool {
           if (p == 0) {
             pdl_wait();
           } else {
-            if (!wait_counter(A.bar + (p - 1), G, timeout_ns)) {
-              tail->abort_flag = 1;
-              set_err(err, NLD_DEVERR_TIMEOUT);
-              return false;
+            const uint64_t t0 = globaltimer_ns();
+            int npf = 0;
+            while (ld_acquire_gpu(A.bar + (p - 1)) < G) {
+              if (npf < kBoundaryPrefetch && tn < w.tiles) {
+                const int rn = tn / P.tok_tiles;
+                if (P.w_rowmajor)
+                  tma_prefetch_l2_2d(&P.tmW, ktn * kTileK, rn * kTileRows);
+                else
+                  tma_prefetch_l2_2d(&P.tmW, 0, (rn * P.KT + ktn) * kTileRows);
+                ++npf;
+                if (++ktn >= w.k_hi) {
+                  tn += w.ngrp;
+                  ktn = w.k_lo;
+                }
+              } else if (globaltimer_ns() - t0 > timeout_ns) {
+                tail->abort_flag = 1;
+                set_err(err, NLD_DEVERR_TIMEOUT);
+                return false;
+              }
             }
             fence_proxy_async_global();
           }
@@ -241,11 +295,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               q_k[nq] = kt;
               q_tt[nq] = tt;
               q_nk[nq] = nk;
-              if (++nq == S && !become_ready()) { ok = false; break; }
+              if (++nq == S) {
+                const bool last_k = kt + nk >= w.k_hi;
+                if (!become_ready(last_k ? t + w.ngrp : t, last_k ? w.k_lo : kt + nk)) {
+                  ok = false;
+                  break;
+                }
+              }
             }
           }
         }
-        if (ok && !ready && !become_ready()) ok = false;
+        if (ok && !ready && !become_ready(w.tiles, 0)) ok = false;
       }
       if (ok && A.next_valid && static_cast<int>(blockIdx.x) < A.next_grid) {
         // warm L2 (and address translation) for this CTA index's first boxes of the next chain
@@ -326,12 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* red_f = tail->red_f[half];
     int* red_i = tail->red_i[half];
     const int hbar = 3 + half;            // named barrier of this half's 4 warps
-    uint32_t stg_peer[kMaxSplit];
-#pragma unroll
-    for (int q = 0; q < kMaxSplit; ++q)
-      stg_peer[q] = (CS > 1) ? dsmem_addr(smem_u32(staging), static_cast<uint32_t>(q < CS ? q : 0)) : 0u;
     int i = 0;    // tiles of this CTA so far (TMEM buffer parity)
-    int js = 0;   // split tiles so far (staging buffer parity)
+    int ru = 0;   // split tiles in which this CTA owned chunks (rfull phases)
     bool ok = true;
     for (int p = 0; ok && p < A.nph; ++p) {
       const PhaseArgs& P = A.ph[p];
@@ -349,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (et == 0) trace_mark(A, 3 + 3 * p);
       const int g0 = (rank / w.s) * w.s;   // first cluster rank of this rank's group
+      int kp = 0;                          // split tiles of this phase so far (same in the group)
       for (int t = w.grp; t < w.tiles; t += w.ngrp, ++i) {
         const int r = t / P.tok_tiles;
         const int tt = t - r * P.tok_tiles;
@@ -359,70 +416,116 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         named_bar_sync(1, kEpiThreads);
         compute_tile_meta(e, tok0, NT, need_norm, tail->inv, tail->pos, tail->pg, et, kEpiThreads);
+        // Split tile: the group's s ranks each hold a partial sum of the whole tile.  Rank g
+        // owns chunks [g*per, (g+1)*per): every rank sends its partial of those chunks to g with
+        // st.async (one-way, counted by g's rfull transaction count) and g sums the s partials
+        // in rank order from its own shared memory.  Prepared while the tile's MMAs run: the
+        // chunk's global operands, and the other owners' readiness for this tile.
+        const int per = (nchunks + w.s - 1) / w.s;
+        const int c_lo = w.grank * per, c_hi = min(nchunks, c_lo + per);
+        const int n_own = max(0, c_hi - c_lo);
+        const int cm = c_lo + half;
+        EpiPre pre;
+        if (w.s > 1) {
+          named_bar_sync(1, kEpiThreads);   // the tile's positions (QKV) are in shared memory
+          if (cm < c_hi) epi_preload(e, r, row_in_tile, tok0 + cm * 16, tail->pos, cm * 16, pre);
+          // every other owner of this tile has reduced the group's previous split tile of this
+          // phase (earlier phases: the grid-wide phase counter), so its slots are free
+          if (et < w.s && et != w.grank && et * per < nchunks) {
+            const uint32_t a = dsmem_addr(smem_u32(&tail->done[p]), static_cast<uint32_t>(g0 + et));
+            const uint64_t t0 = globaltimer_ns();
+            while (static_cast<int>(ld_dsmem_u32_relaxed(a)) < kp) {
+              if (globaltimer_ns() - t0 > timeout_ns) {
+                tail->epi_abort = 1;
+                set_err(err, NLD_DEVERR_TIMEOUT);
+                break;
+              }
+            }
+          }
+        }
+        // (epi_wait's barrier also publishes a timed-out readiness wait above)
         if (!epi_wait(&tail->tfull[tb], use & 1u, false, timeout_ns, tail, err)) { ok = false; break; }
         tc_fence_after();
+        if (et == 0) trace_iter(A, 3, 8 * i);
         const uint32_t tbase = tmem + (static_cast<uint32_t>(ew * 32) << 16) + tb * buf_cols;
         if (w.s == 1) {
           for (int c = half; c < nchunks; c += 2) {
+            EpiPre pre;
+            epi_preload(e, r, row_in_tile, tok0 + c * 16, tail->pos, c * 16, pre);
             float v[16];
             tmem_ld16(tbase + c * 16, v);
             epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
-                         c * 16, v, red_f, red_i, hbar);
+                         c * 16, v, pre, red_f, red_i, hbar);
           }
           tc_fence_before();
           mbar_arrive(&tail->tempty[tb]);
         } else {
-          // 1. this rank's partial -> staging buffer b, once the group has read its last use
-          const int b = js & 1;
-          const uint32_t suse = static_cast<uint32_t>(js >> 1);
-          ++js;
-          if (!epi_wait(&tail->sempty[b], (suse & 1u) ^ 1u, true, timeout_ns, tail, err)) { ok = false; break; }
-          float* stg = staging + b * stg_floats;
+          // 2. partial -> owners (own chunks by plain stores)
           for (int c = half; c < nchunks; c += 2) {
             float v[16];
             tmem_ld16(tbase + c * 16, v);
+            const int o = c / per;
+            const uint32_t off = static_cast<uint32_t>(((w.grank * per + (c - o * per)) * kTileRows + row_in_tile) * kSlotLd) * 4u;
+            if (o == w.grank) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(slots) + off);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) stg[(c * 16 + j) * kTileRows + row_in_tile] = v[j];
+              for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            } else {
+              const uint32_t peer = static_cast<uint32_t>(g0 + o);
+              const uint32_t dst = dsmem_addr(smem_u32(slots), peer) + off;
+              const uint32_t bar = dsmem_addr(smem_u32(&tail->rfull), peer);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                st_async_f4(dst + 16u * q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]), bar);
+            }
           }
           tc_fence_before();
           mbar_arrive(&tail->tempty[tb]);
-          named_bar_sync(1, kEpiThreads);
-          const uint32_t cnt = static_cast<uint32_t>(CS / w.s);
-          if (et == 0)
-            for (int q = 0; q < w.s; ++q)
-              mbar_arrive_remote_count(dsmem_addr(smem_u32(&tail->sfull[b]), static_cast<uint32_t>(g0 + q)), cnt);
-          // 2. the group's partials are staged: reduce this rank's column slice over DSMEM
-          if (!epi_wait(&tail->sfull[b], suse & 1u, true, timeout_ns, tail, err)) { ok = false; break; }
-          const int per = (nchunks + w.s - 1) / w.s;
-          const int c_lo = w.grank * per, c_hi = min(nchunks, c_lo + per);
-          const uint32_t off0 = static_cast<uint32_t>(b * stg_floats) * 4u;
-          for (int c = c_lo + half; c < c_hi; c += 2) {
-            const uint32_t cofs = off0 + static_cast<uint32_t>((c * 16) * kTileRows + row_in_tile) * 4u;
+          if (et == 0) trace_iter(A, 3, 8 * i + 1);
+          // 3. the other ranks' partials of this CTA's chunks have landed
+          if (n_own > 0) {
+            const uint32_t rp = static_cast<uint32_t>(ru++);
+            if (!epi_wait(&tail->rfull, rp & 1u, true, timeout_ns, tail, err)) { ok = false; break; }
+            // arm the next owned split tile now: its senders first wait for done[] below
+            if (et == 0) {
+              const uint32_t nb = next_owned_bytes(A, p, t, cl, rank, C);
+              if (nb) mbar_arrive_expect_tx(&tail->rfull, nb);
+            }
+          } else {
+            named_bar_sync(1, kEpiThreads);
+          }
+          if (et == 0) trace_iter(A, 3, 8 * i + 2);
+          // 4. reduce this thread's chunk in rank order
+          if (cm < c_hi) {
+            const float* src = slots + static_cast<size_t>((cm - c_lo) * kTileRows + row_in_tile) * kSlotLd;
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            // ranks of the group in order, two at a time so that 32 loads are in flight
-            for (int q0 = 0; q0 < w.s; q0 += 2) {
-              float pa[16], pb[16];
-              const uint32_t a0 = stg_peer[g0 + q0] + cofs;
-              const bool two = (q0 + 1 < w.s);
-              const uint32_t a1 = two ? stg_peer[g0 + q0 + 1] + cofs : a0;
+            for (int q = 0; q < w.s; ++q) {
+              const float4* pq = reinterpret_cast<const float4*>(src + static_cast<size_t>(q * per) * kSlotFloats);
 #pragma unroll
-              for (int j = 0; j < 16; ++j) pa[j] = ld_dsmem_f32(a0 + static_cast<uint32_t>(j * kTileRows * 4));
-#pragma unroll
-              for (int j = 0; j < 16; ++j) pb[j] = two ? ld_dsmem_f32(a1 + static_cast<uint32_t>(j * kTileRows * 4)) : 0.f;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] = (v[j] + pa[j]) + pb[j];
+              for (int k4 = 0; k4 < 4; ++k4) {
+                const float4 a4 = pq[k4];
+                v[4 * k4] += a4.x;
+                v[4 * k4 + 1] += a4.y;
+                v[4 * k4 + 2] += a4.z;
+                v[4 * k4 + 3] += a4.w;
+              }
             }
-            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
-                         c * 16, v, red_f, red_i, hbar);
+            if (et == 0) trace_iter(A, 3, 8 * i + 5);
+            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + cm * 16, tail->inv, tail->pos, tail->pg,
+                         cm * 16, v, pre, red_f, red_i, hbar);
+            if (et == 0) trace_iter(A, 3, 8 * i + 6);
           }
-          // 3. this rank is done reading the group's staging buffers b
+          // 5. this CTA's slots are free again (relaxed: the loaded values were consumed)
           named_bar_sync(1, kEpiThreads);
-          if (et == 0)
-            for (int q = 0; q < w.s; ++q)
-              mbar_arrive_remote_count(dsmem_addr(smem_u32(&tail->sempty[b]), static_cast<uint32_t>(g0 + q)), cnt);
+          ++kp;
+          if (et == 0) {
+            trace_iter(A, 3, 8 * i + 3);
+            st_shared_u32_relaxed_cluster(&tail->done[p], static_cast<uint32_t>(kp));
+          }
         }
+        if (et == 0) trace_iter(A, 3, 8 * i + 4);
       }
       if (!ok) break;
       if (et == 0) trace_mark(A, 4 + 3 * p);
@@ -437,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     named_bar_sync(2, 32 + kEpiThreads);
   }
-  // peers may still read this CTA's staging buffers or arrive on its barriers
+  // peers may still write into this CTA's slot area or arrive on its barriers
   if (CS > 1) cluster_sync();
   __syncthreads();
   if (A.nph > 1 && threadIdx.x == 0) {
@@ -453,8 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_mark(A, 15);
 }
 
-size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS) {
-  const size_t stg = (CS > 1) ? 2ull * NT * kTileRows * sizeof(float) : 0;
+size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS, int slots) {
+  const size_t stg = (CS > 1) ? static_cast<size_t>(slots) * kSlotFloats * sizeof(float) : 0;
   return 1024 + static_cast<size_t>(stages) * kps * (kStageW + xr * 128) + stg + sizeof(GemmTail);
 }
 int gemm_chain_max_stages() { return kMaxStages; }
@@ -498,7 +601,7 @@ cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uin
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS);
+  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS, A.slots);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;

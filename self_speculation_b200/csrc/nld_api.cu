@@ -305,9 +305,15 @@ ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const in
   // two k-tiles (32 KB of weights) per stage: the producer/MMA barrier round trip, not HBM,
   // bounds a ring of 16 KB stages; as many stages as fit the shared-memory budget
   best.kps = 2;
+  best.slots = 0;
+  for (int p = 0; p < nph; ++p)
+    if (best.ph[p].s > 1) {
+      const int nch = NT / 16, s = best.ph[p].s;
+      best.slots = std::max(best.slots, s * ((nch + s - 1) / s));
+    }
   best.stages = 2;
   for (int st = gemm_chain_max_stages(); st > 2; --st)
-    if (gemm_chain_smem_bytes(NT, best.xr, best.kps, st, best.CS) <= kChainSmemBudget) {
+    if (gemm_chain_smem_bytes(NT, best.xr, best.kps, st, best.CS, best.slots) <= kChainSmemBudget) {
       best.stages = st;
       break;
     }
@@ -369,7 +375,7 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
     A.next_KT = N.ph[0].KT;
     A.next_grid = ngrid;
     A.next_tiles = N.ph[0].row_tiles * N.ph[0].tok_tiles;
-    A.next_boxes = N.stages * N.kps;
+    A.next_boxes = N.stages * N.kps + 8;
     A.tmWn = *winfo(x, next_pr[0].which, next_pr[0].layer).map;
   }
   CK(launch_gemm_chain(x->stream, A, grid, x->timeout_ns, pdl));

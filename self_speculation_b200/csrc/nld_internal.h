@@ -99,6 +99,7 @@ struct alignas(64) ChainArgs {
   int xr;           // activation rows loaded per k-tile of a token tile: the tile's token count
                     // rounded up to 8 (<= NT); the MMA's N = NT columns read past them into
                     // padding columns that the epilogue never uses
+  int slots;        // split-K slot area: max over split phases of s * ceil(NT/16 / s) chunks
   uint32_t tmem_cols;   // power of two >= 2*NT
   unsigned* bar;    // [kMaxPhases] phase-boundary arrival counters + exit counter (last slot);
                     // zero before the launch, left zero by it
@@ -126,7 +127,7 @@ struct AttnArgs {
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
 cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uint64_t timeout_ns,
                               bool pdl);
-size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS);
+size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS, int slots);
 int gemm_chain_max_stages();
 int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,
