@@ -252,6 +252,11 @@ NLD_DEV unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 // Bounded wait until *p >= target (gpu-scope acquire).  Returns false on timeout.
+// Add to a global counter without returning the old value, with release semantics at gpu
+// scope (the arriving side of a grid-wide phase counter).
+NLD_DEV void red_add_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 NLD_DEV bool wait_counter(const unsigned* p, unsigned target, uint64_t timeout_ns) {
   if (ld_acquire_gpu(p) >= target) return true;
   const uint64_t t0 = globaltimer_ns();

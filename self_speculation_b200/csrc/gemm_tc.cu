@@ -395,8 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Work w = work_of(A, p, cl, rank, C);
       const bool need_norm = (e.kind != EPI_RESID);
       if (p > 0) {
-        // inputs of this epilogue (residual, RMS statistics) come from phase p-1
-        if (!wait_counter(A.bar + (p - 1), G, timeout_ns)) {
+        // inputs of this epilogue (residual, RMS statistics) come from phase p-1; one thread
+        // polls the counter (acquire), the barrier orders the others' reads after it
+        if (et == 0 && !wait_counter(A.bar + (p - 1), G, timeout_ns)) {
           tail->epi_abort = 1;
           set_err(err, NLD_DEVERR_TIMEOUT);
         }
@@ -530,11 +531,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (et == 0) trace_mark(A, 4 + 3 * p);
       if (p + 1 < A.nph) {
-        // this CTA's outputs of phase p are written: publish them, then arrive
-        __threadfence();
-        fence_proxy_async_global();
+        // this CTA's outputs of phase p are written: after the barrier one thread publishes
+        // them (its gpu-scope fence covers the stores the barrier ordered before it) and arrives
         named_bar_sync(1, kEpiThreads);
-        if (et == 0) atomicAdd(A.bar + p, 1u);
+        if (et == 0) {
+          __threadfence();
+          fence_proxy_async_global();
+          red_add_release_gpu(A.bar + p, 1u);
+        }
       }
     }
     tc_fence_before();
