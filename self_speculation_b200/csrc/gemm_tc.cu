@@ -514,8 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             if (et == 0) trace_iter(A, 3, 8 * i + 5);
+            // slot `half` (rank 0's partial of this half's chunk) is read only by this half:
+            // once all four of its warps have summed, it is the chunk's transpose buffer
+            named_bar_sync(hbar, 128);
             epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + cm * 16, tail->inv, tail->pos, tail->pg,
-                         cm * 16, v, pre, red_f, red_i, hbar);
+                         cm * 16, v, pre, red_f, red_i, hbar, slots + static_cast<size_t>(half) * kSlotFloats);
             if (et == 0) trace_iter(A, 3, 8 * i + 6);
           }
           // 5. this CTA's slots are free again (relaxed: the loaded values were consumed)
