@@ -86,9 +86,11 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     tma_prefetch_desc(&tmKV);
   }
   __syncwarp();
-  pdl_wait();
-  pdl_launch_dependents();
 
+  // The sequence length, the page table and the cached KV rows below len were written by
+  // earlier forwards (kernels that completed before the one this launch may overlap: that one
+  // writes only rows len..len+m-1), so the first KV tiles lying wholly in the cached prefix are
+  // requested before waiting for the previous kernel.
   int len = a.lens[b];
   const int p0 = qt * a.QT;
   const int np = min(a.QT, a.m - p0);
@@ -116,8 +118,15 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     tma_load_2d(sV + stage * kKVTile, &tmKV, &full[stage], 0, row0v);
     tma_load_2d(sV + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0v);
   };
+  int n_pre = 0;
+  if (tid == 0) {
+    for (; n_pre < min(kAttStages, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
+  }
+  __syncwarp();
+  pdl_wait();
+  pdl_launch_dependents();
   if (tid == 0)
-    for (int i = 0; i < min(kAttStages, ntile); ++i) issue(i);
+    for (int i = n_pre; i < min(kAttStages, ntile); ++i) issue(i);
   __syncwarp();
 
   // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row)

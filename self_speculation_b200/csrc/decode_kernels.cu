@@ -8,6 +8,8 @@
 
 namespace nld {
 
+constexpr int kFinalizeThreads = 1024;   // one warp per LM-head row of a sequence (m <= 64)
+
 // ------------------------------------------------------------------------------ embedding --
 // Input block of each forward (shifted prediction; the pending token x_n sits at position n):
 //   AR      [x_n]                         DRAFT   [x_n, MASK x (k-1)]
@@ -72,7 +74,19 @@ cudaError_t launch_embed(cudaStream_t st, const EmbedArgs& a, int M, bool bf16, 
 // One CTA per sequence.  For forwards with an LM head, warp w combines rows w, w+8, ... over
 // all vocab tiles: global max (lowest id on ties) and sum_t se_t * exp(mx_t - max), whose
 // inverse is the largest softmax probability (the confidence).
-__global__ void __launch_bounds__(256) finalize_kernel(const FinalizeArgs a) {
+// Merge of two LM-head partials (max, sum of exp(l - max), lowest argmax) into a.
+NLD_DEV void lm_merge(float& mx, float& se, int& ix, float bmx, float bse, int bix) {
+  if (bmx == -INFINITY) return;
+  if (bmx > mx || (bmx == mx && bix < ix)) {
+    se = bse + ((mx == -INFINITY) ? 0.f : se * expf(mx - bmx));
+    mx = bmx;
+    ix = bix;
+  } else {
+    se += bse * expf(bmx - mx);
+  }
+}
+
+__global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const FinalizeArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ int s_arg[64];
@@ -82,33 +96,35 @@ __global__ void __launch_bounds__(256) finalize_kernel(const FinalizeArgs a) {
   const bool lm = (a.mode == FWD_AR || a.mode == FWD_DRAFT || a.mode == FWD_VERIFY ||
                    a.mode == FWD_DIFFUSE);
   if (lm) {
-    for (int i = warp; i < a.m; i += 8) {
+    // one warp per row; one pass over the row's vocab tiles with 8 loads in flight per lane,
+    // merging (max, sum exp, argmax) online, then across the warp
+    for (int i = warp; i < a.m; i += kFinalizeThreads / 32) {
       const LmPart* row = a.lm_part + static_cast<size_t>(b * a.m + i) * a.lm_tiles;
-      float mx = -INFINITY;
+      float mx = -INFINITY, se = 0.f;
       int ix = INT_MAX;
-      for (int t = lane; t < a.lm_tiles; t += 32) {
-        const LmPart p = row[t];
-        if (p.mx > mx || (p.mx == mx && p.idx < ix)) {
-          mx = p.mx;
-          ix = p.idx;
+      for (int t0 = lane; t0 < a.lm_tiles; t0 += 32 * 8) {
+        LmPart p[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = t0 + 32 * u;
+          if (t < a.lm_tiles) {
+            p[u] = row[t];
+          } else {
+            p[u].mx = -INFINITY;
+            p[u].se = 0.f;
+            p[u].idx = INT_MAX;
+          }
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) lm_merge(mx, se, ix, p[u].mx, p[u].se, p[u].idx);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         const float om = __shfl_xor_sync(0xffffffffu, mx, off);
+        const float os = __shfl_xor_sync(0xffffffffu, se, off);
         const int oi = __shfl_xor_sync(0xffffffffu, ix, off);
-        if (om > mx || (om == mx && oi < ix)) {
-          mx = om;
-          ix = oi;
-        }
+        lm_merge(mx, se, ix, om, os, oi);
       }
-      float se = 0.f;
-      for (int t = lane; t < a.lm_tiles; t += 32) {
-        const LmPart p = row[t];
-        se += p.se * expf(p.mx - mx);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
       if (lane == 0) {
         s_arg[i] = ix;
         s_conf[i] = 1.0f / se;
@@ -223,7 +239,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(const FinalizeArgs a) {
 cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kFinalizeThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
