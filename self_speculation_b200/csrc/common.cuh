@@ -207,17 +207,6 @@ NLD_DEV float2 ld_dsmem_f2(uint32_t addr) {
   return v;
 }
 
-// Arrive (release, cluster scope) on an mbarrier of another CTA of the cluster, addressed by
-// its shared::cluster address (dsmem_addr).
-NLD_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-NLD_DEV void mbar_arrive_remote_count(uint32_t cluster_addr, uint32_t count) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
-               "r"(count)
-               : "memory");
-}
 // Asynchronous 16-byte store into another cluster CTA's shared memory; the bytes count against
 // the transaction count of that CTA's mbarrier at remote_bar (both shared::cluster addresses).
 NLD_DEV void st_async_f4(uint32_t remote_addr, float4 v, uint32_t remote_bar) {
@@ -234,14 +223,6 @@ NLD_DEV uint32_t ld_dsmem_u32_relaxed(uint32_t addr) {
 }
 NLD_DEV void st_shared_u32_relaxed_cluster(void* p, uint32_t v) {
   asm volatile("st.relaxed.cluster.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-// Same without release semantics: for a signal that publishes no data of this thread (e.g.
-// "done reading your buffer", once the loaded values have been consumed), so the arrive does
-// not wait for this thread's outstanding global stores.
-NLD_DEV void mbar_arrive_remote_count_relaxed(uint32_t cluster_addr, uint32_t count) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
-               "r"(count)
-               : "memory");
 }
 // Generic-proxy writes of other CTAs (made visible by a gpu-scope acquire) before this thread's
 // later async-proxy (TMA) reads of the same global memory.
@@ -267,12 +248,6 @@ NLD_DEV bool wait_counter(const unsigned* p, unsigned target, uint64_t timeout_n
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
 }
-// L2 prefetch of a contiguous global range (16-byte aligned, size a multiple of 16).
-NLD_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
-}
 NLD_DEV bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -294,11 +269,6 @@ NLD_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t timeout_
       if (mbar_try_wait_acq_cluster(bar, parity)) return true;
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
-}
-NLD_DEV float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 // -------------------------------------------------------------------------- misc helpers --
