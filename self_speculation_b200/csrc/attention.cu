@@ -447,6 +447,7 @@ size_t attn_mma_smem_bytes(int NW) {
 
 cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
                                  int batch, bool pdl) {
+  if (a.NW < 1 || a.NW > kMaxAttWarps) return cudaErrorInvalidValue;   // launch bound
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
   cfg.blockDim = dim3(32 * a.NW);

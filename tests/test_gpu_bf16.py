@@ -1,8 +1,9 @@
 """bf16 path (tcgen05 GEMMs, tensor-core attention) against the rounding-matched oracle.
 
 Shape: 2 layers, d 512, 8 q / 2 kv heads x 128 (GQA group 4), FFN 1536, vocab 5000 (a ragged
-last LM-head tile), k = 32, batch up to 4: every GEMM spans several row tiles and stream-K
-splits; prompt lengths put the KV prefix off page boundaries.
+last LM-head tile), k = 32, batch up to 4: every projection spans several row tiles, batch 1
+runs the cluster split-K path (M = 32/33 tokens) and batch 3 the wide-tile path (M = 96/99);
+prompt lengths put the KV prefix off page boundaries.
 
 Bars (stated for the decode round): logits max-abs error <= 2e-2; argmax equal wherever the
 oracle's top-2 margin exceeds 5e-2; acceptance lengths, committed ids and lengths bit-exact given
