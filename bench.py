@@ -324,9 +324,9 @@ def run_ours(args, world, rank, local):
                "round_s_est": round(round_est, 2)}
 
     # two forwards (draft, verify), each: embed, QKV chain of layer 0, per layer one attention
-    # and one chain (O, gate/up, down, next QKV), LM-head chain; then finalize for draft,
-    # verify and commit
-    per_round = 2 * (1 + 1 + 2 * cfg.n_layers + 1) + 3
+    # and one chain (O, gate/up, down, then the next QKV or, last, the LM head); then finalize
+    # for draft, verify and commit
+    per_round = 2 * (1 + 1 + 2 * cfg.n_layers) + 3
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
@@ -635,7 +635,7 @@ def run_probe(args):
     it = tr[148 * 16:148 * 16 + 256].view(4, 64).cpu().double()
     rel = lambda v: [round((float(x) - float(t0)) / 1e3, 2) if x > 0 else None for x in v]
     print(json.dumps({"cta0_pipeline_us": {"issue": rel(it[0]), "mma": rel(it[1]), "freed": rel(it[2]),
-                                           "epi_tiles": [rel(it[3][8 * i:8 * i + 7]) for i in range(8)]}}))
+                                           "epi_tiles": [rel(it[3][8 * i:8 * i + 8]) for i in range(8)]}}))
 
 
 def main():

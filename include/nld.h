@@ -166,10 +166,13 @@ nld_status nld_debug_state(nld_ctx* ctx, int32_t* d_lens_out, int32_t* d_pending
  * scratch (activations, partials, KV rows at positions >= len): decode state does not move. */
 nld_status nld_time_gemm(nld_ctx* ctx, int which, int layer, int M, int reps, float* ms_out);
 
-/* Profiling hook: like nld_time_gemm, one traced launch; d_trace receives, per CTA, 16
- * globaltimer stamps (ns): 0 start, 1 setup done, 2/3 first/last TMA issue, 4 first MMA,
- * 5/6 accumulator 0/1 committed, 7/8 epilogue 0/1 start, 9/10 epilogue 0/1 end, 11 exit.
- * *grid_out = number of CTAs.  Synchronises. */
+/* Profiling hook: like nld_time_gemm, one traced launch (a one-phase chain, see
+ * nld_trace_chain).  d_trace: at least 148*16 + 256 uint64 entries, zeroed by the caller; it
+ * receives per CTA 16 globaltimer stamps (ns): 0 start, 1 set-up done, 2 first weight load
+ * issued, 3 epilogue released, 4 epilogue done, 14 last MMA commit, 15 exit; then, from entry
+ * 148*16, CTA 0's pipeline: 4 x 64 stamps (stage issued, stage consumed by the MMA, stage
+ * freed, and per tile i at 8i+k the epilogue steps).  *grid_out = number of CTAs.
+ * Synchronises. */
 nld_status nld_trace_gemm(nld_ctx* ctx, int which, int layer, int M, unsigned long long* d_trace,
                           int* grid_out);
 
@@ -180,9 +183,10 @@ nld_status nld_time_chain(nld_ctx* ctx, int layer, int M, int reps, float* ms_ou
 
 /* Profiling hook: one traced launch of the decode chain of `layer` (O-proj, gate/up, down,
  * then layer+1's QKV) over M token rows (as nld_time_gemm, 0 <= layer < n_layers-1); d_trace
- * receives per CTA 16 globaltimer stamps (ns): 0 start, 1 set-up done, for phase p = 0..3:
- * 2+3p first weight load issued, 3+3p epilogue released by the phase counter, 4+3p epilogue
- * done; 14 last MMA commit, 15 exit.  *grid_out = CTAs.  Synchronises. */
+ * (at least 148*16 + 256 uint64 entries, zeroed) receives per CTA 16 globaltimer stamps (ns):
+ * 0 start, 1 set-up done, for phase p = 0..3: 2+3p first weight load issued, 3+3p epilogue
+ * released by the phase counter, 4+3p epilogue done; 14 last MMA commit, 15 exit; then CTA 0's
+ * pipeline stamps as in nld_trace_gemm.  *grid_out = CTAs.  Synchronises. */
 nld_status nld_trace_chain(nld_ctx* ctx, int layer, int M, unsigned long long* d_trace, int* grid_out);
 
 /* Profiling hook: the tiling chosen for projection GEMM `which` (as in nld_time_gemm) over M

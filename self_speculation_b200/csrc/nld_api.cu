@@ -483,7 +483,8 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
     aa.G = aa.Hq / aa.Hkv;
   }
 
-  // projections: QKV(0) | per layer: attention, chain [O, gate/up, down, QKV(l+1)] | LM head
+  // projections: QKV(0) | per layer: attention, chain [O, gate/up, down, QKV(l+1) or, for the
+  // last layer, the LM head]
   const int L = x->c.n_layers;
   auto proj = [&](int which, int layer) {
     ProjRef r{which, layer, base_epi(x, M, f.m)};
@@ -519,15 +520,16 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
       aa.pool = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
       CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
     }
-    const int n = layer_chain(l, cur);
+    int n = layer_chain(l, cur);
     int nn = 0;
-    if (l + 1 < L) nn = layer_chain(l + 1, nxt);
-    else if (f.lm != LM_NONE) { nxt[0] = proj(GW_LM, 0); nn = 1; }
+    if (l + 1 < L) {
+      nn = layer_chain(l + 1, nxt);
+    } else if (f.lm != LM_NONE) {
+      // the last layer's chain ends with the final norm + LM head: its weights stream in across
+      // the phase boundary instead of after a kernel boundary
+      cur[n++] = proj(GW_LM, 0);
+    }
     TRY(chain(x, cur, n, M, pdl, x->bars + (1 + l) * kMaxPhases, nn ? nxt : nullptr, nn));
-  }
-  if (f.lm != LM_NONE) {
-    const ProjRef lm = proj(GW_LM, 0);
-    TRY(chain(x, &lm, 1, M, pdl, x->bars, nullptr, 0));
   }
   return NLD_OK;
 }
