@@ -26,6 +26,12 @@ Readings where the pages are silent (each is listed with its reason in the desig
   block gets one causal forward over [x_n, b_1..b_{k-1}] that writes its KV rows; b_k
   becomes the pending token.  With several sequences, a sequence whose block is complete
   waits (its rows are computed and ignored) until every block is complete.
+* Fused fill (the deferred form of the KV fill): the causal forward over the complete block
+  and the first denoising forward of the next block run as one forward of 2k rows,
+  [x_n, b_1..b_{k-1}, b_k, MASK x (k-1)] at positions n..n+2k-1, whose first k rows are
+  causal and whose last k rows are one bidirectional block that sees the first k.  In exact
+  arithmetic its KV rows n..n+k-1 and its last k logit rows equal those of the fill followed
+  by the plain denoising forward.
 """
 from __future__ import annotations
 
@@ -203,6 +209,52 @@ def diffusion_step(model, st: SeqState, k: int, tau: float):
                 logits=logits)
 
 
+def fill_diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
+    """The fused fill: st.block is complete.  One forward over
+    [x_n, b_1..b_{k-1}, b_k, MASK x (k-1)] (first k rows causal, last k rows one block) writes
+    the complete block's KV rows; then lens += k, pending = b_k, a fresh block of masks.
+    Returns the logits [B, k, V] of the last k rows (the new block's first denoising step)."""
+    mask_id = model.cfg.mask_id
+    B = len(st.lens)
+    toks = torch.tensor([[st.pending[b]] + st.block[b] + [mask_id] * (k - 1) for b in range(B)],
+                        dtype=torch.int64)
+    logits = model.forward(toks, st.lens, st.cache, block_size=k, write_kv=True,
+                           causal_rows=k)
+    for b in range(B):
+        st.lens[b] += k
+        st.pending[b] = st.block[b][k - 1]
+    st.block = [[mask_id] * k for _ in range(B)]
+    return logits[:, k:]
+
+
+def diffusion_step_fused(model, st: SeqState, k: int, tau: float, fill_pending: bool):
+    """One denoising step with the deferred fill: when fill_pending (the previous step
+    completed the block), the fill and this step are the one fused forward; a block completed
+    by this step is not filled now (returned fill_pending = True).  Same commit rule as
+    diffusion_step.  Returns (dict as diffusion_step without the fill, fill_pending)."""
+    mask_id = model.cfg.mask_id
+    B = len(st.lens)
+    if st.block is None:
+        st.block = [[mask_id] * k for _ in range(B)]
+    logits = fill_diffusion_forward(model, st, k) if fill_pending else diffusion_forward(model, st, k)
+    conf = confidence(logits)
+    am = argmax_lowest(logits)
+    newly = []
+    for b in range(B):
+        masked = [t == mask_id for t in st.block[b]]
+        pick = diffusion_commit(masked, conf[b].tolist(), tau)
+        got = []
+        for s in range(k):
+            if pick[s]:
+                st.block[b][s] = int(am[b, s])
+                got.append((s, int(am[b, s])))
+        newly.append(got)
+    complete = all(mask_id not in st.block[b] for b in range(B))
+    blocks = [list(st.block[b]) for b in range(B)] if complete else None
+    return dict(newly=newly, conf=conf, argmax=am, complete=complete, blocks=blocks,
+                logits=logits), complete
+
+
 # ---- generation drivers (exactly N generated tokens; the last round is truncated) ----------
 
 def ar_generate(model, prompt: torch.Tensor, n_tokens: int, capacity: int) -> List[List[int]]:
@@ -228,6 +280,26 @@ def selfspec_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, capaci
             out[b].extend(committed[b])
             per_round[b].append(len(committed[b]))
     return [o[:n_tokens] for o in out], per_round
+
+
+def diffuse_generate_fused(model, prompt: torch.Tensor, n_tokens: int, k: int, tau: float,
+                           capacity: int) -> Tuple[List[List[int]], int, int]:
+    """diffuse_generate with the deferred, fused fill.  Returns (tokens per sequence in
+    position order, number of forwards, number of denoising steps); a fill still pending at
+    the end is not run (its tokens are committed)."""
+    st = prefill(model, prompt, capacity)
+    B = prompt.shape[0]
+    out = [[] for _ in range(B)]
+    steps = forwards = 0
+    pending = False
+    while min(len(o) for o in out) < n_tokens:
+        r, pending = diffusion_step_fused(model, st, k, tau, pending)
+        steps += 1
+        forwards += 1
+        if r["complete"]:
+            for b in range(B):
+                out[b].extend(r["blocks"][b])
+    return [o[:n_tokens] for o in out], forwards, steps
 
 
 def diffuse_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, tau: float,

@@ -73,15 +73,28 @@ def causal_mask(m: int, n: int) -> torch.Tensor:
     return j <= n + r
 
 
-def block_mask(m: int, n: int, block_size: int) -> torch.Tensor:
+def block_mask(m: int, n: int, block_size: int, causal_rows: int = 0) -> torch.Tensor:
     """[m, n+m] bool: prefix keys (j < n) always visible; keys of the forward are visible
-    when their block index (j-n)//block_size is not above the query's r//block_size."""
+    when their block index (j-n)//block_size is not above the query's r//block_size.
+
+    causal_rows = c > 0 (the fused diffusion KV fill): the first c rows of the forward are
+    strictly causal (a complete block being written into the clean prefix), and the blocks
+    of block_size start after them: row r >= c sees the prefix, all c causal rows, and the
+    keys of its own and earlier blocks counted from c."""
     j = torch.arange(n + m)[None, :]
     r = torch.arange(m)[:, None]
     in_prefix = j < n
-    key_blk = torch.div(j - n, block_size, rounding_mode="floor")
-    q_blk = torch.div(r, block_size, rounding_mode="floor")
-    return in_prefix | ((j >= n) & (key_blk <= q_blk))
+    if causal_rows == 0:
+        key_blk = torch.div(j - n, block_size, rounding_mode="floor")
+        q_blk = torch.div(r, block_size, rounding_mode="floor")
+        return in_prefix | ((j >= n) & (key_blk <= q_blk))
+    c = causal_rows
+    causal_part = (r < c) & (j <= n + r)
+    in_fill = (j >= n) & (j < n + c)
+    key_blk = torch.div(j - n - c, block_size, rounding_mode="floor")
+    q_blk = torch.div(r - c, block_size, rounding_mode="floor")
+    block_part = (r >= c) & (in_fill | ((j >= n + c) & (key_blk <= q_blk)))
+    return (in_prefix & (r >= 0)) | causal_part | block_part
 
 
 def attention_explicit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -149,7 +162,7 @@ class OracleModel:
     # -- forward ------------------------------------------------------------------------
     def forward(self, tokens: torch.Tensor, starts: List[int], cache, block_size: int,
                 write_kv: bool, layers: Optional[List[int]] = None,
-                with_logits: bool = True) -> Optional[torch.Tensor]:
+                with_logits: bool = True, causal_rows: int = 0) -> Optional[torch.Tensor]:
         """tokens [B, m] at positions starts[b]..starts[b]+m-1 over cached rows
         [0, starts[b]).  block_size 1 = causal; block_size m = one bidirectional block.
         write_kv stores this forward's K/V rows into the cache at their positions.
@@ -173,7 +186,7 @@ class OracleModel:
                 Kc, Vc = cache[b][li]
                 keys = torch.cat([Kc[:, :n], kb.transpose(0, 1)], dim=1)          # [Hkv, n+m, hd]
                 vals = torch.cat([Vc[:, :n], vb.transpose(0, 1)], dim=1)
-                mask = block_mask(m, n, block_size)
+                mask = block_mask(m, n, block_size, causal_rows)
                 o = attention_explicit(qb.transpose(0, 1), keys, vals, mask)      # [Hq, m, hd]
                 att[b] = self._store(o.transpose(0, 1))
                 if write_kv:

@@ -405,3 +405,66 @@ def test_mlp_branch_closed_form():
     h1 = h0 + u @ W[9].double().t()
     want = (h1 / torch.sqrt((h1 * h1).mean(-1, keepdim=True) + cfg.rms_eps)) @ W[-1].double().t()
     assert torch.allclose(logits[0], want, atol=1e-12)
+
+
+# ---------------------------------------------- fused KV fill (deferred fill, next row f1) --
+
+def test_fused_fill_mask_reduces_to_causal_and_block_masks():
+    n, c, bs = 5, 4, 4
+    m = c + bs
+    full = omod.block_mask(m, n, bs, causal_rows=c)
+    # the first c rows are the causal mask's rows
+    assert torch.equal(full[:c, :n + c], omod.causal_mask(c, n))
+    assert not full[:c, n + c:].any()
+    # the block rows see the prefix, every fill row and their whole block
+    assert full[c:].all()
+    # no causal rows: unchanged
+    assert torch.equal(omod.block_mask(m, n, bs, 0), omod.block_mask(m, n, bs))
+
+
+def _state_with_complete_block(mdl, k, seed):
+    st = odec.prefill(mdl, synth.prompt_tokens(2, 11, mdl.cfg.vocab, seed=seed), 96)
+    st.block = [[mdl.cfg.mask_id] * k for _ in range(2)]
+    st.block = [list(odec.argmax_lowest(odec.diffusion_forward(mdl, st, k))[b].tolist())
+                for b in range(2)]
+    return st
+
+
+def test_fused_fill_equals_fill_then_denoise():
+    """The fused forward's KV rows and last k logit rows equal the causal fill forward
+    followed by the plain denoising forward of the next block (fp64, exact up to rounding)."""
+    import copy
+    cfg = _tiny(n_layers=2)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0), "f64")
+    k = 4
+    st = _state_with_complete_block(mdl, k, seed=3)
+    a, b = copy.deepcopy(st), copy.deepcopy(st)
+    # separate: fill (causal, writes KV) then the new block's first denoising forward
+    toks = torch.tensor([[a.pending[i]] + a.block[i][:k - 1] for i in range(2)], dtype=torch.int64)
+    mdl.forward(toks, a.lens, a.cache, block_size=1, write_kv=True, with_logits=False)
+    for i in range(2):
+        a.lens[i] += k
+        a.pending[i] = a.block[i][k - 1]
+    a.block = [[cfg.mask_id] * k for _ in range(2)]
+    la = odec.diffusion_forward(mdl, a, k)
+    # fused
+    lb = odec.fill_diffusion_forward(mdl, b, k)
+    assert (la - lb).abs().max().item() < 1e-10
+    assert a.lens == b.lens and a.pending == b.pending and a.block == b.block
+    for i in range(2):
+        for layer in range(cfg.n_layers):
+            for t in range(2):
+                x, y = a.cache[i][layer][t][:, :a.lens[i]], b.cache[i][layer][t][:, :b.lens[i]]
+                assert (x - y).abs().max().item() < 1e-12
+
+
+@pytest.mark.parametrize("tau", [0.9, 0.0, 1.5])
+def test_fused_fill_generation_equals_unfused(tau):
+    cfg = _tiny(n_layers=1)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0, lm_head_scale=30.0), "f64")
+    p = synth.prompt_tokens(2, 10, cfg.vocab, seed=5)
+    k = 4
+    ref, steps = odec.diffuse_generate(mdl, p, 12, k, tau, 96)
+    got, forwards, fsteps = odec.diffuse_generate_fused(mdl, p, 12, k, tau, 96)
+    assert got == ref
+    assert fsteps == steps and forwards == steps   # no separate fill forwards
