@@ -148,6 +148,22 @@ nld_status nld_selfspec_round(nld_ctx* ctx, int32_t* d_tokens_out, int32_t* d_nc
 nld_status nld_diffuse_block_step(nld_ctx* ctx, float threshold, int32_t* d_block_out,
                                   float* d_conf_out, int32_t* d_ncommit_out, int32_t* h_filled_out);
 
+/* nld_diffuse_block_step with the KV fill deferred and fused.  When a step completes every
+ * block, the fill is not launched; the next call of this function runs it together with the
+ * new block's first denoising step as ONE forward of 2k rows per sequence,
+ * [x_n, b_1..b_k, MASK x (k-1)] at positions n..n+2k-1, whose first k rows are causal (they
+ * write KV rows n..n+k-1 of the complete block) and whose last k rows are one bidirectional
+ * block that sees them (ranhao.site notes §4.3: the clean prefix is causal; reading: the two
+ * forwards are equal in exact arithmetic to this one).  One forward less per block.  Same
+ * outputs as nld_diffuse_block_step; *h_filled_out = 1 when this call performed a deferred
+ * fill (len += k, pending = b_k happened here).  A fill still deferred runs alone at the start
+ * of the next nld_diffuse_block_step, nld_ar_step, nld_selfspec_* or nld_debug_logits call
+ * (nld_debug_state reports the state before it).  Needs 2k <= 64 and batch*2k token rows
+ * (NLD_ERR_UNSUPPORTED otherwise). */
+nld_status nld_diffuse_block_step_fused(nld_ctx* ctx, float threshold, int32_t* d_block_out,
+                                        float* d_conf_out, int32_t* d_ncommit_out,
+                                        int32_t* h_filled_out);
+
 /* Test hook: run the forward of `mode` (NLD_MODE_*) from the current state and write its
  * logits [batch, m, vocab] fp32 to d_logits_out (m = 1, k, k+1, k).  Sequence state is not
  * advanced; a DRAFT call stores its argmaxes as the drafts a later VERIFY call reads.  The

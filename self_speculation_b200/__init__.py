@@ -57,6 +57,7 @@ def load_library() -> ctypes.CDLL:
         "nld_kv_commit": ([P, P, P, P], I),
         "nld_selfspec_round": ([P, P, P, P], I),
         "nld_diffuse_block_step": ([P, F, P, P, P, P], I),
+        "nld_diffuse_block_step_fused": ([P, F, P, P, P, P], I),
         "nld_debug_logits": ([P, I, P], I),
         "nld_debug_state": ([P, P, P, P, P], I),
         "nld_sync": ([P], I),
@@ -160,6 +161,13 @@ class Context:
         self._check(self.lib.nld_diffuse_block_step(self.h, float(threshold), _ptr(block_out),
                                                     _ptr(conf_out), _ptr(ncommit_out),
                                                     ctypes.byref(filled)), self.h)
+        return bool(filled.value)
+
+    def nld_diffuse_block_step_fused(self, threshold: float, block_out, conf_out, ncommit_out) -> bool:
+        filled = ctypes.c_int32(0)
+        self._check(self.lib.nld_diffuse_block_step_fused(self.h, float(threshold), _ptr(block_out),
+                                                          _ptr(conf_out), _ptr(ncommit_out),
+                                                          ctypes.byref(filled)), self.h)
         return bool(filled.value)
 
     def nld_debug_logits(self, mode: int, logits_out) -> None:

@@ -55,8 +55,11 @@ NLD_DEV uint32_t kv_off(int row, int c) {
   return static_cast<uint32_t>((c >> 3) * kHalfTile + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
-NLD_DEV int vis_end_of(int len, int p, int bs, int m) {
-  const int blk0 = (p / bs) * bs;
+// Last key row visible to query row p (0-based in the forward): rows p < c are strictly
+// causal; the blocks of bs rows start at row c (c = 0: the plain block mask).
+NLD_DEV int vis_end_of(int len, int p, int bs, int m, int c) {
+  if (p < c) return len + p;
+  const int blk0 = c + ((p - c) / bs) * bs;
   return len + min(blk0 + bs, m) - 1;
 }
 
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     if (tid == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
     len = max(0, min(len, a.pps * kPage - a.m));
   }
-  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m) + 1;
+  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m, a.causal_rows) + 1;
   const int n_tiles = (kv_end + kPage - 1) / kPage;
   // at least two KV tiles per split: fewer, fuller splits keep the merge short
   const int per = max(2, (n_tiles + a.S - 1) / a.S);
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   auto row_vis = [&](int r) {
     const int p = r / a.G;
     if (r >= a.rows || p >= np) return -1;
-    return vis_end_of(len, p0 + p, a.block_size, a.m);
+    return vis_end_of(len, p0 + p, a.block_size, a.m, a.causal_rows);
   };
   const int vis_a = row_vis(ra), vis_b = row_vis(rb);
 
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
     if (threadIdx.x == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
     len = max(0, min(len, a.pps * kPage - a.m));
   }
-  const int nkeys = vis_end_of(len, i, a.block_size, a.m) + 1;
+  const int nkeys = vis_end_of(len, i, a.block_size, a.m, a.causal_rows) + 1;
   const T* q = static_cast<const T*>(a.q) + (static_cast<size_t>(tok) * a.Hq + head) * a.hd;
   for (int d = threadIdx.x; d < a.hd; d += blockDim.x) sq[d] = to_f32<T>(q[d]);
   __syncthreads();

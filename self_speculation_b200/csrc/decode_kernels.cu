@@ -29,6 +29,9 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
     case FWD_AR: id = a.pending[b]; break;
     case FWD_DRAFT: id = (i == 0) ? a.pending[b] : a.V; break;
     case FWD_VERIFY: id = (i == 0) ? a.pending[b] : a.draft[b * a.k + i - 1]; break;
+    case FWD_FILLDIFF:   // the complete block (causal rows), then b_k and k-1 masks
+      id = (i == 0) ? a.pending[b] : (i <= a.k ? a.blk[b * a.k + i - 1] : a.V);
+      break;
     default: id = (i == 0) ? a.pending[b] : a.blk[b * a.k + i - 1]; break;
   }
   if (id < 0 || id > a.V) {
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool lm = (a.mode == FWD_AR || a.mode == FWD_DRAFT || a.mode == FWD_VERIFY ||
-                   a.mode == FWD_DIFFUSE);
+                   a.mode == FWD_DIFFUSE || a.mode == FWD_FILLDIFF);
   if (lm) {
     // one warp per row; one pass over the row's vocab tiles with 8 loads in flight per lane,
     // merging (max, sum exp, argmax) online, then across the warp
@@ -179,13 +182,30 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
         a.pending[b] = a.verify[b * (k + 1) + c - 1];
       }
     } break;
+    case FWD_FILLDIFF:
     case FWD_DIFFUSE: {
+      // FWD_FILLDIFF: the complete block's KV rows were written by this forward's first k
+      // (causal) rows: len += k, pending = b_k, and the new block (all masks) is denoised by
+      // the last k rows
+      const bool fused = (a.mode == FWD_FILLDIFF);
+      const int row0 = fused ? k : 0;
+      if (fused) {
+        const int last = a.blk[b * k + k - 1];
+        __syncwarp();
+        if (a.commit)
+          for (int i = lane; i < k; i += 32) a.blk[b * k + i] = a.V;
+        __syncwarp();
+        if (lane == 0 && a.commit) {
+          a.lens[b] += k;
+          a.pending[b] = last;
+        }
+      }
       // confidence-threshold commit among open slots; at least one (the most confident)
       const bool valid = lane < k;
-      const int cur = valid ? a.blk[b * k + lane] : 0;
+      const int cur = valid ? (fused ? a.V : a.blk[b * k + lane]) : 0;
       const bool masked = valid && (cur == a.V);
-      const float conf = valid ? s_conf[lane] : 0.f;
-      const int tok = valid ? s_arg[lane] : 0;
+      const float conf = valid ? s_conf[row0 + lane] : 0.f;
+      const int tok = valid ? s_arg[row0 + lane] : 0;
       bool pick = masked && (conf >= a.threshold);
       const unsigned any_pick = __ballot_sync(0xffffffffu, pick);
       const unsigned any_mask = __ballot_sync(0xffffffffu, masked);

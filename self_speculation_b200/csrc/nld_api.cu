@@ -128,6 +128,7 @@ struct nld_ctx {
   int batch = 0;
   bool started = false;
   bool verify_fresh = false;
+  bool fill_pending = false;   // a complete diffusion block whose causal KV fill is deferred
   long long len_upper = 0;
   uint64_t timeout_ns = 2000000000ull;
   std::string msg;
@@ -436,6 +437,7 @@ struct FwdSpec {
   int chunk0;        // prefill: first prompt position of this chunk
   int prompt_len;
   bool last_chunk;
+  int causal_rows;   // attention: leading strictly causal rows (fused diffusion fill)
 };
 
 // Launch one forward (no finalize).
@@ -475,6 +477,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.page_table = x->page_table;
   aa.pps = x->pps;
   aa.block_size = f.bs;
+  aa.causal_rows = f.causal_rows;
   aa.err = x->err;
   aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
   if (x->bf16) {
@@ -882,6 +885,10 @@ nld_status nld_init_weights(nld_ctx* x, const void* const* tensors, int n_tensor
   return NLD_OK;
 }
 
+namespace {
+nld_status flush_fill(nld_ctx* x);   // (diffusion, below)
+}  // namespace
+
 nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int prompt_len) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (!x->weights_ready) return fail(x, NLD_ERR_STATE, "weights not initialised");
@@ -925,11 +932,13 @@ nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int promp
   x->len_upper = rows;
   x->started = true;
   x->verify_fresh = false;
+  x->fill_pending = false;
   return NLD_OK;
 }
 
 nld_status nld_ar_step(nld_ctx* x, int32_t* d_tokens_out) {
   TRY(need_started(x));
+  TRY(flush_fill(x));
   TRY(ensure_capacity(x, 1));
   std::vector<uintptr_t> key = {1, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_tokens_out)};
   const long long saved = x->len_upper;
@@ -978,6 +987,7 @@ static nld_status draft_verify_body(nld_ctx* x) {
 
 nld_status nld_selfspec_draft_verify(nld_ctx* x) {
   TRY(need_started(x));
+  TRY(flush_fill(x));
   TRY(ensure_capacity(x, x->c.block_k + 1));
   std::vector<uintptr_t> key = {2, static_cast<uintptr_t>(x->batch)};
   TRY(run_graph(x, key, [&]() { return draft_verify_body(x); }));
@@ -1001,6 +1011,7 @@ nld_status nld_kv_commit(nld_ctx* x, const int32_t* d_nrows, int32_t* d_tokens_o
 nld_status nld_selfspec_round(nld_ctx* x, int32_t* d_tokens_out, int32_t* d_ncommit_out,
                               const int32_t* d_force_ncommit) {
   TRY(need_started(x));
+  TRY(flush_fill(x));
   TRY(ensure_capacity(x, x->c.block_k + 1));
   std::vector<uintptr_t> key = {3, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_tokens_out),
                                 reinterpret_cast<uintptr_t>(d_ncommit_out), reinterpret_cast<uintptr_t>(d_force_ncommit)};
@@ -1017,30 +1028,61 @@ nld_status nld_selfspec_round(nld_ctx* x, int32_t* d_tokens_out, int32_t* d_ncom
   return NLD_OK;
 }
 
-nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_out, float* d_conf_out,
-                                  int32_t* d_ncommit_out, int32_t* h_filled_out) {
-  TRY(need_started(x));
+namespace {
+
+// The causal KV-fill forward of a complete diffusion block: len += k, pending = b_k.
+nld_status run_fill(nld_ctx* x) {
   const int k = x->c.block_k;
   TRY(ensure_capacity(x, k));
+  std::vector<uintptr_t> fkey = {5, static_cast<uintptr_t>(x->batch)};
+  TRY(run_graph(x, fkey, [&]() -> nld_status {
+    const long long saved = x->len_upper;
+    x->len_upper = x->c.max_seq;
+    FwdSpec f{};
+    f.mode = FWD_FILL;
+    f.B = x->batch;
+    f.m = k;
+    f.bs = 1;
+    f.lm = LM_NONE;
+    nld_status s = launch_forward(x, f);
+    x->len_upper = saved;
+    if (s != NLD_OK) return s;
+    return finalize(x, base_fin(x, FWD_FILL, k));
+  }));
+  x->len_upper += k;
+  x->fill_pending = false;
+  return NLD_OK;
+}
+
+// A deferred fill runs alone before any other decode call.
+nld_status flush_fill(nld_ctx* x) { return x->fill_pending ? run_fill(x) : NLD_OK; }
+
+// One denoising forward + commit (fused = the deferred fill of the previous block and the new
+// block's first step in one forward of 2k rows); returns the number of sequences whose block
+// is still open.
+nld_status run_denoise(nld_ctx* x, bool fused, float threshold, int32_t* d_block_out, float* d_conf_out,
+                       int32_t* d_ncommit_out, int* open_out) {
+  const int k = x->c.block_k;
   uint32_t thr_bits;
   std::memcpy(&thr_bits, &threshold, 4);
-  std::vector<uintptr_t> key = {4, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_block_out),
-                                reinterpret_cast<uintptr_t>(d_conf_out), reinterpret_cast<uintptr_t>(d_ncommit_out),
-                                thr_bits};
+  std::vector<uintptr_t> key = {static_cast<uintptr_t>(fused ? 6 : 4), static_cast<uintptr_t>(x->batch),
+                                reinterpret_cast<uintptr_t>(d_block_out), reinterpret_cast<uintptr_t>(d_conf_out),
+                                reinterpret_cast<uintptr_t>(d_ncommit_out), thr_bits};
   TRY(run_graph(x, key, [&]() -> nld_status {
     CK(cudaMemsetAsync(x->incomplete, 0, sizeof(int), x->stream));
     const long long saved = x->len_upper;
     x->len_upper = x->c.max_seq;
     FwdSpec f{};
-    f.mode = FWD_DIFFUSE;
+    f.mode = fused ? FWD_FILLDIFF : FWD_DIFFUSE;
     f.B = x->batch;
-    f.m = k;
+    f.m = fused ? 2 * k : k;
     f.bs = k;
+    f.causal_rows = fused ? k : 0;
     f.lm = LM_ARGMAX;
     nld_status s = launch_forward(x, f);
     x->len_upper = saved;
     if (s != NLD_OK) return s;
-    FinalizeArgs a = base_fin(x, FWD_DIFFUSE, k);
+    FinalizeArgs a = base_fin(x, f.mode, f.m);
     a.threshold = threshold;
     a.block_out = d_block_out;
     a.conf_out = d_conf_out;
@@ -1050,25 +1092,22 @@ nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_
     return NLD_OK;
   }));
   CK(cudaStreamSynchronize(x->stream));
-  const int open = x->h_pinned[1];
+  *open_out = x->h_pinned[1];
+  return NLD_OK;
+}
+
+}  // namespace
+
+nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_out, float* d_conf_out,
+                                  int32_t* d_ncommit_out, int32_t* h_filled_out) {
+  TRY(need_started(x));
+  TRY(flush_fill(x));
+  TRY(ensure_capacity(x, x->c.block_k));
+  int open = 1;
+  TRY(run_denoise(x, false, threshold, d_block_out, d_conf_out, d_ncommit_out, &open));
   int filled = 0;
   if (open == 0) {
-    std::vector<uintptr_t> fkey = {5, static_cast<uintptr_t>(x->batch)};
-    TRY(run_graph(x, fkey, [&]() -> nld_status {
-      const long long saved = x->len_upper;
-      x->len_upper = x->c.max_seq;
-      FwdSpec f{};
-      f.mode = FWD_FILL;
-      f.B = x->batch;
-      f.m = k;
-      f.bs = 1;
-      f.lm = LM_NONE;
-      nld_status s = launch_forward(x, f);
-      x->len_upper = saved;
-      if (s != NLD_OK) return s;
-      return finalize(x, base_fin(x, FWD_FILL, k));
-    }));
-    x->len_upper += k;
+    TRY(run_fill(x));
     filled = 1;
   }
   if (h_filled_out) *h_filled_out = filled;
@@ -1076,8 +1115,29 @@ nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_
   return NLD_OK;
 }
 
+nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_block_out,
+                                        float* d_conf_out, int32_t* d_ncommit_out, int32_t* h_filled_out) {
+  TRY(need_started(x));
+  const int k = x->c.block_k;
+  const bool fused = x->fill_pending;
+  if (fused && (2 * k > 64 || x->batch * 2 * k > x->M_max))
+    return fail(x, NLD_ERR_UNSUPPORTED, "fused fill needs 2k <= 64 and batch*2k <= %d rows", x->M_max);
+  TRY(ensure_capacity(x, fused ? 2 * k : k));
+  int open = 1;
+  TRY(run_denoise(x, fused, threshold, d_block_out, d_conf_out, d_ncommit_out, &open));
+  if (fused) {
+    x->len_upper += k;
+    x->fill_pending = false;
+  }
+  if (open == 0) x->fill_pending = true;   // this block's fill joins the next step
+  if (h_filled_out) *h_filled_out = fused ? 1 : 0;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
 nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
   TRY(need_started(x));
+  TRY(flush_fill(x));
   if (!d_logits_out) return fail(x, NLD_ERR_ARG, "logits is NULL");
   const int k = x->c.block_k;
   FwdSpec f{};

@@ -27,7 +27,8 @@ enum EpiKind : int {
 // Forward kinds (which tokens the embedding gathers and what the finalize step does).
 enum FwdMode : int {
   FWD_AR = 0, FWD_DRAFT = 1, FWD_VERIFY = 2, FWD_DIFFUSE = 3, FWD_FILL = 4, FWD_PREFILL = 5,
-  FWD_COMMIT = 6
+  FWD_COMMIT = 6,
+  FWD_FILLDIFF = 7   // fused diffusion KV fill: [x_n, b_1..b_k, MASK x (k-1)], 2k rows
 };
 
 // Per (token, vocab tile) partial of the LM-head reduction.
@@ -119,6 +120,8 @@ struct AttnArgs {
   int pps;
   int layer_row0;       // row of this layer's first page in the 2D pool view
   int block_size;
+  int causal_rows;      // the first causal_rows rows of each sequence are strictly causal and
+                        // the blocks of block_size start after them (fused diffusion fill)
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   float scale_log2;     // log2(e) / sqrt(hd)
   int* err;
