@@ -1,11 +1,14 @@
 // Projection GEMMs on the 5th-generation tensor cores (tcgen05), Y^T = W * X^T, run as a
 // persistent chain: one launch executes up to four projections back to back (for a decode
-// layer: O-proj, gate/up, down, and the next layer's QKV).
+// layer: O-proj, gate/up, down, and the next layer's QKV, or for the last layer the final
+// norm + LM head).
 //
 // Swap-AB: the weight matrix W [n_rows, K] is the MMA's M=128 operand and the few token rows
 // X [M, K] are its N operand (N = 16..256), so a decode forward streams every weight byte once.
 // Weights are stored pre-tiled (128 x 64 blocks, 16 KB contiguous), so each TMA box is one
-// contiguous read and a CTA's K range is one contiguous stretch of HBM.
+// contiguous read and a CTA's K range is one contiguous stretch of HBM.  A pipeline stage holds
+// two k-tiles (32 KB of weights plus the activation rows), so one producer -> MMA -> producer
+// barrier round trip moves 32 KB.
 //
 // Work split: the CTAs of a cluster (CS of them) share output tiles; in a phase with split s
 // (a divisor of CS) each group of s ranks splits the K range of a tile, each rank accumulating
@@ -17,7 +20,8 @@
 // Phases: a CTA that finished its part of phase p adds one to a grid-wide arrival counter; the
 // next phase's activation loads and epilogue wait until every CTA has arrived.  Its weight
 // loads do not wait: the producer keeps the shared-memory ring full with the next phase's
-// weights across the transition, so HBM stays busy while the last tiles of a phase finish.
+// weights across the transition and, while it waits, prefetches the following boxes into L2,
+// so HBM stays busy while the last tiles of a phase finish.
 // The first phase waits for the previous kernel the same way (programmatic dependent launch).
 //
 // Warp roles (320 threads): warp 0 issues TMA loads (W with an evict-first L2 hint), warp 1
@@ -33,7 +37,7 @@ namespace nld {
 
 namespace {
 
-constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB of bf16 weights per stage
+constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB: one k-tile of bf16 weights
 constexpr int kMaxStages = 8;
 constexpr int kBoundaryPrefetch = 16;   // weight boxes prefetched into L2 per phase boundary
 constexpr int kSlotLd = 20;              // floats per row of a split-K slot: 16 + 4 (16-byte
