@@ -26,6 +26,9 @@ Readings where the pages are silent (each is listed with its reason in the desig
   block gets one causal forward over [x_n, b_1..b_{k-1}] that writes its KV rows; b_k
   becomes the pending token.  With several sequences, a sequence whose block is complete
   waits (its rows are computed and ignored) until every block is complete.
+* LoRA drafter (optional, OracleModel.set_lora): the low-rank o_proj delta applies to the
+  block-bidirectional forwards (draft, diffusion denoising) only; causal forwards (verify, AR,
+  prefill, KV fill) use the frozen weights, so committed KV rows never contain it.
 * Fused fill (the deferred form of the KV fill): the causal forward over the complete block
   and the first denoising forward of the next block run as one forward of 2k rows,
   [x_n, b_1..b_{k-1}, b_k, MASK x (k-1)] at positions n..n+2k-1, whose first k rows are
@@ -133,7 +136,7 @@ def draft_forward(model, st: SeqState, k: int) -> torch.Tensor:
     B = len(st.lens)
     toks = torch.full((B, k), model.cfg.mask_id, dtype=torch.int64)
     toks[:, 0] = torch.tensor(st.pending)
-    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False)
+    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False, lora=True)
 
 
 def verify_forward(model, st: SeqState, drafts: List[List[int]]) -> torch.Tensor:
@@ -168,7 +171,7 @@ def diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
     the mask id), one bidirectional block; row i scores slot b_{i+1}."""
     toks = torch.tensor([[st.pending[b]] + st.block[b][:k - 1] for b in range(len(st.lens))],
                         dtype=torch.int64)
-    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False)
+    return model.forward(toks, st.lens, st.cache, block_size=k, write_kv=False, lora=True)
 
 
 def diffusion_step(model, st: SeqState, k: int, tau: float):
@@ -214,6 +217,7 @@ def fill_diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
     [x_n, b_1..b_{k-1}, b_k, MASK x (k-1)] (first k rows causal, last k rows one block) writes
     the complete block's KV rows; then lens += k, pending = b_k, a fresh block of masks.
     Returns the logits [B, k, V] of the last k rows (the new block's first denoising step)."""
+    assert model.lora is None, "the fused fill mixes causal and drafter rows: no LoRA drafter"
     mask_id = model.cfg.mask_id
     B = len(st.lens)
     toks = torch.tensor([[st.pending[b]] + st.block[b] + [mask_id] * (k - 1) for b in range(B)],

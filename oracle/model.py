@@ -135,6 +135,14 @@ class OracleModel:
                                     g2=w[b + 5], wg=w[b + 6], wu=w[b + 7], wd=w[b + 8]))
         self.gf = w[1 + 9 * cfg.n_layers]
         self.lm = w[2 + 9 * cfg.n_layers]
+        self.lora = None
+
+    def set_lora(self, A: List[torch.Tensor], B: List[torch.Tensor], scale: float) -> None:
+        """Low-rank delta on o_proj for the diffusion drafter (ranhao.site notes section 6:
+        LoRA of rank 128 on o_proj, trained for the diffusion pathway while the AR verifier
+        stays frozen): per layer A [r, Hq*hd], B [d, r]; a block-bidirectional forward adds
+        scale * B (A att) to the residual next to o_proj's output."""
+        self.lora = (list(A), list(B), float(scale))
 
     # -- helpers ------------------------------------------------------------------------
     def _w(self, t: torch.Tensor) -> torch.Tensor:
@@ -162,7 +170,8 @@ class OracleModel:
     # -- forward ------------------------------------------------------------------------
     def forward(self, tokens: torch.Tensor, starts: List[int], cache, block_size: int,
                 write_kv: bool, layers: Optional[List[int]] = None,
-                with_logits: bool = True, causal_rows: int = 0) -> Optional[torch.Tensor]:
+                with_logits: bool = True, causal_rows: int = 0,
+                lora: bool = False) -> Optional[torch.Tensor]:
         """tokens [B, m] at positions starts[b]..starts[b]+m-1 over cached rows
         [0, starts[b]).  block_size 1 = causal; block_size m = one bidirectional block.
         write_kv stores this forward's K/V rows into the cache at their positions.
@@ -192,7 +201,12 @@ class OracleModel:
                 if write_kv:
                     Kc[:, n:n + m] = kb.transpose(0, 1)
                     Vc[:, n:n + m] = vb.transpose(0, 1)
-            h = h + self._mm(att.reshape(B, m, Hq * hd), L["wo"])
+            a2 = att.reshape(B, m, Hq * hd)
+            if lora and self.lora is not None:
+                # z = A att is stored like any activation; the delta joins the residual first
+                LA, LB, sc = self.lora[0][li], self.lora[1][li], self.lora[2]
+                h = h + sc * self._mm(self._store(self._mm(a2, LA)), LB)
+            h = h + self._mm(a2, L["wo"])
             g = self._normed_mm(h, L["g2"], L["wg"])
             u = self._normed_mm(h, L["g2"], L["wu"])
             act = self._store(g / (1.0 + torch.exp(-g)) * u)      # silu(g) * u

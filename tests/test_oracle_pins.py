@@ -468,3 +468,52 @@ def test_fused_fill_generation_equals_unfused(tau):
     got, forwards, fsteps = odec.diffuse_generate_fused(mdl, p, 12, k, tau, 96)
     assert got == ref
     assert fsteps == steps and forwards == steps   # no separate fill forwards
+
+
+# ------------------------------------------------------------ LoRA drafter (next row f3) --
+
+def _lora(cfg, r, seed, std=0.02):
+    g = torch.Generator().manual_seed(seed)
+    qd = cfg.n_q_heads * cfg.head_dim
+    A = [torch.randn(r, qd, generator=g, dtype=torch.float64) * std for _ in range(cfg.n_layers)]
+    B = [torch.randn(cfg.d_model, r, generator=g, dtype=torch.float64) * std for _ in range(cfg.n_layers)]
+    return A, B
+
+
+def test_lora_equals_merged_o_proj_in_draft():
+    """The LoRA forward equals the plain forward with W_o + scale * B A (the merge identity of a
+    low-rank adapter), in fp64."""
+    cfg = _tiny(n_layers=2)
+    W = synth.model_weights(cfg, 0)
+    A, B = _lora(cfg, 8, seed=3)
+    sc = 5.0
+    lo = oracle.OracleModel(cfg, W, "f64")
+    lo.set_lora(A, B, sc)
+    Wm = list(W)
+    for l in range(cfg.n_layers):
+        Wm[1 + 9 * l + 4] = W[1 + 9 * l + 4].double() + sc * (B[l] @ A[l])
+    merged = oracle.OracleModel(cfg, Wm, "f64")
+    plain = oracle.OracleModel(cfg, W, "f64")
+    p = synth.prompt_tokens(2, 20, cfg.vocab, seed=4)
+    # the clean prefix is written by the frozen (plain) weights; only the draft differs
+    st = odec.prefill(plain, p, 96)
+    a, b = odec.draft_forward(lo, st, 8), odec.draft_forward(merged, st, 8)
+    assert (a - b).abs().max().item() < 1e-10
+    # and the delta is not negligible at this scale
+    assert (a - odec.draft_forward(plain, st, 8)).abs().max().item() > 1e-3
+
+
+def test_lora_only_in_drafter_forwards():
+    cfg = _tiny(n_layers=2)
+    W = synth.model_weights(cfg, 0)
+    A, B = _lora(cfg, 8, seed=3)
+    lo, pl = oracle.OracleModel(cfg, W, "f64"), oracle.OracleModel(cfg, W, "f64")
+    lo.set_lora(A, B, 5.0)
+    p = synth.prompt_tokens(1, 20, cfg.vocab, seed=4)
+    s1, s2 = odec.prefill(lo, p, 96), odec.prefill(pl, p, 96)
+    drafts = [[3, 7, 11, 2, 5, 9, 1, 4]]
+    assert torch.equal(odec.verify_forward(lo, s1, drafts), odec.verify_forward(pl, s2, drafts))
+    assert torch.equal(odec.ar_forward(lo, s1), odec.ar_forward(pl, s2))
+    zero = [torch.zeros_like(b) for b in B]
+    lo.set_lora(A, zero, 5.0)
+    assert torch.equal(odec.draft_forward(lo, s1, 8), odec.draft_forward(pl, s2, 8))
