@@ -100,6 +100,20 @@ nld_status nld_destroy(nld_ctx* ctx);
  * The caller may free its buffers when the call returns (the call synchronises). */
 nld_status nld_init_weights(nld_ctx* ctx, const void* const* tensors, int n_tensors, int on_device);
 
+/* Optional LoRA drafter (Nemotron-Labs-Diffusion notes, ranhao.site, section 6: a rank-128
+ * adapter on o_proj trained for the diffusion pathway while the AR verifier stays frozen).
+ * `tensors` holds 2*n_layers pointers: per layer A [rank, Hq*hd] then B [d_model, rank],
+ * row-major, config dtype, host or device as `on_device` says.  Every block-bidirectional
+ * forward (the self-speculation draft, each diffusion denoising step, the block rows of the
+ * fused fill) then adds scale * B (A att) to the residual beside W_o att, with z = A att
+ * rounded to the activation type; causal forwards (prefill, AR, verify, the KV fill) are
+ * unchanged.  rank 0 (tensors may be NULL) switches the adapter off.  The first load fixes
+ * the rank (1..256); later loads replace the weights and scale and must use the same rank
+ * (else NLD_ERR_STATE).  Requires nld_init_weights first.  Synchronises; the caller may free
+ * its buffers on return.  Two extra launches per layer in those forwards. */
+nld_status nld_init_lora(nld_ctx* ctx, int rank, float scale, const void* const* tensors, int n_tensors,
+                         int on_device);
+
 /* Start `batch` sequences from prompts d_tokens [batch, prompt_len] (device, int32).  Runs
  * causal forwards over positions 0..prompt_len-2 (writing those KV rows) and makes
  * prompt[prompt_len-1] the pending token, so len = prompt_len-1.  Resets drafts and

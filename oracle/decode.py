@@ -216,14 +216,13 @@ def fill_diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
     """The fused fill: st.block is complete.  One forward over
     [x_n, b_1..b_{k-1}, b_k, MASK x (k-1)] (first k rows causal, last k rows one block) writes
     the complete block's KV rows; then lens += k, pending = b_k, a fresh block of masks.
-    Returns the logits [B, k, V] of the last k rows (the new block's first denoising step)."""
-    assert model.lora is None, "the fused fill mixes causal and drafter rows: no LoRA drafter"
+    A LoRA drafter applies to the last k (block) rows only.  Returns the logits [B, k, V] of the last k rows (the new block's first denoising step)."""
     mask_id = model.cfg.mask_id
     B = len(st.lens)
     toks = torch.tensor([[st.pending[b]] + st.block[b] + [mask_id] * (k - 1) for b in range(B)],
                         dtype=torch.int64)
     logits = model.forward(toks, st.lens, st.cache, block_size=k, write_kv=True,
-                           causal_rows=k)
+                           causal_rows=k, lora=True)
     for b in range(B):
         st.lens[b] += k
         st.pending[b] = st.block[b][k - 1]

@@ -203,9 +203,13 @@ class OracleModel:
                     Vc[:, n:n + m] = vb.transpose(0, 1)
             a2 = att.reshape(B, m, Hq * hd)
             if lora and self.lora is not None:
-                # z = A att is stored like any activation; the delta joins the residual first
+                # z = A att is stored like any activation; the delta joins the residual first.
+                # Only rows that attend block-bidirectionally are drafter rows: the leading
+                # causal rows (the fused KV fill) take the frozen path.
                 LA, LB, sc = self.lora[0][li], self.lora[1][li], self.lora[2]
-                h = h + sc * self._mm(self._store(self._mm(a2, LA)), LB)
+                delta = sc * self._mm(self._store(self._mm(a2, LA)), LB)
+                delta[:, :causal_rows] = 0
+                h = h + delta
             h = h + self._mm(a2, L["wo"])
             g = self._normed_mm(h, L["g2"], L["wg"])
             u = self._normed_mm(h, L["g2"], L["wu"])

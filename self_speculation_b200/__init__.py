@@ -51,6 +51,7 @@ def load_library() -> ctypes.CDLL:
         "nld_create": ([ctypes.POINTER(nld_config), P, ctypes.POINTER(P)], I),
         "nld_destroy": ([P], I),
         "nld_init_weights": ([P, ctypes.POINTER(P), I, I], I),
+        "nld_init_lora": ([P, I, F, ctypes.POINTER(P), I, I], I),
         "nld_prefill": ([P, P, I, I], I),
         "nld_ar_step": ([P, P], I),
         "nld_selfspec_draft_verify": ([P], I),
@@ -137,6 +138,15 @@ class Context:
             on_device = tensors[0].is_cuda
         arr = (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
         self._check(self.lib.nld_init_weights(self.h, arr, len(tensors), int(on_device)), self.h)
+
+    def nld_init_lora(self, rank: int, scale: float, tensors: Optional[Sequence] = None,
+                      on_device: Optional[bool] = None) -> None:
+        tensors = [t.contiguous() for t in (tensors or [])]
+        if on_device is None:
+            on_device = bool(tensors) and tensors[0].is_cuda
+        arr = (ctypes.c_void_p * max(1, len(tensors)))(*[t.data_ptr() for t in tensors])
+        self._check(self.lib.nld_init_lora(self.h, rank, scale, arr if tensors else None,
+                                           len(tensors), int(on_device)), self.h)
 
     def nld_prefill(self, tokens) -> None:
         B, P = tokens.shape

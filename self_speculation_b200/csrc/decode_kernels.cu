@@ -2,6 +2,7 @@
 // the finalize step after the LM head (argmax/confidence combine over vocab tiles and the
 // mode's state update: drafts, AR commit, greedy acceptance, diffusion commit, KV-fill and
 // prefill bookkeeping), weight repacking and fills.
+#include <algorithm>
 #include <climits>
 
 #include "common.cuh"
@@ -267,6 +268,119 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, finalize_kernel, a);
+}
+
+// ------------------------------------------------------------------------- LoRA drafter --
+// Low-rank delta on o_proj in the block-bidirectional (drafter) forwards: h += scale * B (A att),
+// added to the residual before the layer chain adds W_o att.  A [r, qd], Bt = B^T [r, d].
+// z = A att: one CTA per adapter row j with that A row in shared memory, one warp per token;
+// stored in the activation type (like every activation between kernels).
+template <typename T>
+__global__ void __launch_bounds__(256) lora_down_kernel(const T* A, const T* att, T* z, int M,
+                                                        int qd, int r) {
+  extern __shared__ float s_a[];   // [qd]
+  pdl_wait();
+  pdl_launch_dependents();
+  const int j = blockIdx.x;
+  for (int c = threadIdx.x; c < qd; c += blockDim.x) s_a[c] = to_f32<T>(A[static_cast<size_t>(j) * qd + c]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < M; t += blockDim.x >> 5) {
+    const T* row = att + static_cast<size_t>(t) * qd;
+    float acc = 0.f;
+    for (int c = lane; c < qd; c += 32) acc += s_a[c] * to_f32<T>(row[c]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) z[static_cast<size_t>(t) * r + j] = from_f32<T>(acc);
+  }
+}
+
+// h[t][i] += scale * sum_j B[i][j] z[t][j]: a CTA per 128 outputs i and 8 tokens, z rows of
+// the tokens in shared memory, Bt read coalesced over i.  Rows t with t mod m < causal_rows
+// (the fused fill's causal rows) are not drafter rows and keep h unchanged.
+template <typename T>
+__global__ void __launch_bounds__(128) lora_up_kernel(const T* Bt, const T* z, float* h, int M,
+                                                      int d, int r, float scale, int m,
+                                                      int causal_rows) {
+  extern __shared__ float s_z[];   // [8][r]
+  pdl_wait();
+  pdl_launch_dependents();
+  const int i = blockIdx.x * 128 + threadIdx.x;
+  const int t0 = blockIdx.y * 8;
+  const int nt = min(8, M - t0);
+  for (int e = threadIdx.x; e < 8 * r; e += 128) {
+    const int tt = e / r, j = e - tt * r;
+    s_z[e] = (tt < nt) ? to_f32<T>(z[static_cast<size_t>(t0 + tt) * r + j]) : 0.f;
+  }
+  __syncthreads();
+  if (i >= d) return;
+  float acc[8];
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) acc[tt] = 0.f;
+  for (int j = 0; j < r; ++j) {
+    const float b = to_f32<T>(Bt[static_cast<size_t>(j) * d + i]);
+#pragma unroll
+    for (int tt = 0; tt < 8; ++tt) acc[tt] += b * s_z[tt * r + j];
+  }
+  for (int tt = 0; tt < nt; ++tt)
+    if ((t0 + tt) % m >= causal_rows) h[static_cast<size_t>(t0 + tt) * d + i] += scale * acc[tt];
+}
+
+// dst [cols, rows] = src [rows, cols]^T (LoRA B -> Bt at load time)
+template <typename T>
+__global__ void transpose_kernel(const T* src, T* dst, int rows, int cols) {
+  const size_t n = static_cast<size_t>(rows) * cols;
+  for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t rr = e / cols, cc = e - rr * cols;
+    dst[cc * rows + rr] = src[e];
+  }
+}
+
+cudaError_t launch_lora(cudaStream_t st, const void* A, const void* Bt, const void* att, void* z,
+                        float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
+                        bool bf16, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c1 = {};
+  c1.gridDim = dim3(r);
+  c1.blockDim = dim3(256);
+  c1.dynamicSmemBytes = static_cast<size_t>(qd) * sizeof(float);
+  c1.stream = st;
+  c1.attrs = attr;
+  c1.numAttrs = pdl ? 1 : 0;
+  cudaLaunchConfig_t c2 = c1;
+  c2.gridDim = dim3((d + 127) / 128, (M + 7) / 8);
+  c2.blockDim = dim3(128);
+  c2.dynamicSmemBytes = static_cast<size_t>(8) * r * sizeof(float);
+  cudaError_t e;
+  if (bf16) {
+    using T = __nv_bfloat16;
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T>, static_cast<const T*>(A), static_cast<const T*>(att),
+                           static_cast<T*>(z), M, qd, r);
+    if (e == cudaSuccess)
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T>, static_cast<const T*>(Bt), static_cast<const T*>(z), h,
+                             M, d, r, scale, m, causal_rows);
+  } else {
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<float>, static_cast<const float*>(A),
+                           static_cast<const float*>(att), static_cast<float*>(z), M, qd, r);
+    if (e == cudaSuccess)
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<float>, static_cast<const float*>(Bt),
+                             static_cast<const float*>(z), h, M, d, r, scale, m, causal_rows);
+  }
+  return e;
+}
+
+cudaError_t launch_transpose(cudaStream_t st, const void* src, void* dst, int rows, int cols, bool bf16) {
+  const int blocks = std::max(1, std::min(4096, (rows * cols + 255) / 256));
+  if (bf16)
+    transpose_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
+                                                            static_cast<__nv_bfloat16*>(dst), rows, cols);
+  else
+    transpose_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst),
+                                                    rows, cols);
+  return cudaGetLastError();
 }
 
 // -------------------------------------------------------------------------------- repack --

@@ -430,12 +430,17 @@ def _state_with_complete_block(mdl, k, seed):
     return st
 
 
-def test_fused_fill_equals_fill_then_denoise():
+@pytest.mark.parametrize("with_lora", [False, True])
+def test_fused_fill_equals_fill_then_denoise(with_lora):
     """The fused forward's KV rows and last k logit rows equal the causal fill forward
-    followed by the plain denoising forward of the next block (fp64, exact up to rounding)."""
+    followed by the plain denoising forward of the next block (fp64, exact up to rounding).
+    With a LoRA drafter the fill rows stay on the frozen path and the block rows take it."""
     import copy
     cfg = _tiny(n_layers=2)
     mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0), "f64")
+    if with_lora:
+        A, B = _lora(cfg, 8, seed=3)
+        mdl.set_lora(A, B, 5.0)
     k = 4
     st = _state_with_complete_block(mdl, k, seed=3)
     a, b = copy.deepcopy(st), copy.deepcopy(st)
