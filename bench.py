@@ -207,6 +207,9 @@ def run_ours(args, world, rank, local):
     weights = synth.model_weights(cfg, 0, device="cuda")
     ctx.nld_init_weights(weights, on_device=True)
     del weights
+    if args.lora:
+        # optional drafter adapter on o_proj (seeded random, scale 1): draft forwards only
+        ctx.nld_init_lora(args.lora, 1.0, synth.lora_weights(cfg, args.lora, 0, device="cuda"))
     torch.cuda.empty_cache()
     prompt = synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1 + rank)
     ctx.nld_prefill(prompt.cuda())
@@ -254,7 +257,7 @@ def run_ours(args, world, rank, local):
     kvb = cfg.kv_bytes_per_token()
     L_avg = (len0 + len1) / 2.0
     round_bytes = 2 * wbytes + (2 * L_avg + K_BLOCK + (K_BLOCK + 1)) * kvb \
-        + (2 * K_BLOCK + 1) * kvb
+        + (2 * K_BLOCK + 1) * kvb + 2 * cfg.n_layers * args.lora * (cfg.q_dim + cfg.d_model)
     round_s = ms / 1e3 / K
     round_gbs = round_bytes / round_s / 1e9
 
@@ -326,7 +329,7 @@ def run_ours(args, world, rank, local):
     # two forwards (draft, verify), each: embed, QKV chain of layer 0, per layer one attention
     # and one chain (O, gate/up, down, then the next QKV or, last, the LM head); then finalize
     # for draft, verify and commit
-    per_round = 2 * (1 + 1 + 2 * cfg.n_layers) + 3
+    per_round = 2 * (1 + 1 + 2 * cfg.n_layers) + 3 + (2 * cfg.n_layers if args.lora else 0)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
@@ -336,6 +339,7 @@ def run_ours(args, world, rank, local):
                    "layers": cfg.n_layers, "d_model": cfg.d_model, "heads": "32q/8kv x 128",
                    "ffn": cfg.ffn_dim, "vocab": cfg.vocab, "batch_per_gpu": 1, "block_k": K_BLOCK,
                    "prompt": PROMPT, "parallelism": f"replicas x{world}",
+                   "lora_rank": args.lora,
                    "l2": "no flush: 15.1 GB of weights per forward exceed the 126 MB L2"},
         "rounds_per_s": round(rounds_per_s, 3),
         "tokens_per_forward": round(tot_committed / (2 * world * K), 4),
@@ -651,6 +655,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lora", type=int, default=0,
+                    help="rank of a seeded random o_proj adapter in the draft forwards (0: none)")
     ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b"],
                     default="selfspec8b")
     ap.add_argument("--probe", action="store_true",

@@ -108,7 +108,7 @@ nld_status nld_init_weights(nld_ctx* ctx, const void* const* tensors, int n_tens
  * fused fill) then adds scale * B (A att) to the residual beside W_o att, with z = A att
  * rounded to the activation type; causal forwards (prefill, AR, verify, the KV fill) are
  * unchanged.  rank 0 (tensors may be NULL) switches the adapter off.  The first load fixes
- * the rank (1..256); later loads replace the weights and scale and must use the same rank
+ * the rank (a multiple of 8 in 8..256; else NLD_ERR_ARG); later loads replace the weights and scale and must use the same rank
  * (else NLD_ERR_STATE).  Requires nld_init_weights first.  Synchronises; the caller may free
  * its buffers on return.  Two extra launches per layer in those forwards. */
 nld_status nld_init_lora(nld_ctx* ctx, int rank, float scale, const void* const* tensors, int n_tensors,

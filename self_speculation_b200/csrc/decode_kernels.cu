@@ -272,37 +272,96 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 
 // ------------------------------------------------------------------------- LoRA drafter --
 // Low-rank delta on o_proj in the block-bidirectional (drafter) forwards: h += scale * B (A att),
-// added to the residual before the layer chain adds W_o att.  A [r, qd], Bt = B^T [r, d].
-// z = A att: one CTA per adapter row j with that A row in shared memory, one warp per token;
-// stored in the activation type (like every activation between kernels).
+// added to the residual before the layer chain adds W_o att.  A [r, qd], B [d, r] row-major
+// (the caller's layout); rank r a multiple of 8.  Two launches, both latency-bound at decode
+// sizes (1 MB of adapter weights per matrix at r 128, d 4096), so every global load of a CTA
+// is a 16-byte vector load issued before any arithmetic.
+//
+// z partials: CTA (jg, ks, tg) takes 16 adapter rows x one 512-byte column slice of qd x 32
+// tokens, stages the A and att slices in shared memory (rows padded so that the per-token
+// reads of a warp hit distinct banks) and writes zp[ks][t][j] = sum over its slice (fp32).
+// The slices are summed in a fixed order by lora_up: deterministic, no atomics.
+constexpr int kLoraJ = 16, kLoraT = 32, kLoraThreads = 256;
+template <typename T> struct LoraCols { static constexpr int n = 512 / sizeof(T); };
+
 template <typename T>
-__global__ void __launch_bounds__(256) lora_down_kernel(const T* A, const T* att, T* z, int M,
-                                                        int qd, int r) {
-  extern __shared__ float s_a[];   // [qd]
+__global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, const T* att, float* zp,
+                                                                 int M, int qd, int r) {
+  constexpr int C = LoraCols<T>::n, LD = C + 2, V = 16 / sizeof(T);
+  __shared__ __align__(16) T sA[kLoraJ][LD];
+  __shared__ __align__(16) T sX[kLoraT][LD];
   pdl_wait();
   pdl_launch_dependents();
-  const int j = blockIdx.x;
-  for (int c = threadIdx.x; c < qd; c += blockDim.x) s_a[c] = to_f32<T>(A[static_cast<size_t>(j) * qd + c]);
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < M; t += blockDim.x >> 5) {
-    const T* row = att + static_cast<size_t>(t) * qd;
-    float acc = 0.f;
-    for (int c = lane; c < qd; c += 32) acc += s_a[c] * to_f32<T>(row[c]);
+  const int j0 = blockIdx.x * kLoraJ, c0 = blockIdx.y * C, t0 = blockIdx.z * kLoraT;
+  // stage: 16 + 32 rows of C/V vectors; out-of-range rows and columns read as zero
+  constexpr int kVecRow = C / V, kVecs = (kLoraJ + kLoraT) * kVecRow;
+  uint4 v[(kVecs + kLoraThreads - 1) / kLoraThreads];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) z[static_cast<size_t>(t) * r + j] = from_f32<T>(acc);
+  for (int u = 0; u < (kVecs + kLoraThreads - 1) / kLoraThreads; ++u) {
+    const int e = u * kLoraThreads + threadIdx.x;
+    const int row = e / kVecRow, c = c0 + (e % kVecRow) * V;
+    v[u] = make_uint4(0, 0, 0, 0);
+    if (e < kVecs && c < qd) {
+      if (row < kLoraJ) {
+        if (j0 + row < r) v[u] = *reinterpret_cast<const uint4*>(A + static_cast<size_t>(j0 + row) * qd + c);
+      } else if (t0 + row - kLoraJ < M) {
+        v[u] = *reinterpret_cast<const uint4*>(att + static_cast<size_t>(t0 + row - kLoraJ) * qd + c);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < (kVecs + kLoraThreads - 1) / kLoraThreads; ++u) {
+    const int e = u * kLoraThreads + threadIdx.x;
+    if (e < kVecs) {
+      const int row = e / kVecRow, cc = (e % kVecRow) * V;
+      T* dst = (row < kLoraJ) ? &sA[row][cc] : &sX[row - kLoraJ][cc];
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) reinterpret_cast<uint32_t*>(dst)[q] = w[q];   // rows 4-byte aligned
+    }
+  }
+  __syncthreads();
+  // lane = token, warp = adapter rows 2w, 2w+1
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < C; c += 2) {
+    float x0, x1, p0, p1, q0, q1;
+    if constexpr (sizeof(T) == 2) {
+      const float2 xx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sX[lane][c]));
+      const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sA[2 * w][c]));
+      const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sA[2 * w + 1][c]));
+      x0 = xx.x; x1 = xx.y; p0 = pp.x; p1 = pp.y; q0 = qq.x; q1 = qq.y;
+    } else {
+      const float2 xx = *reinterpret_cast<const float2*>(&sX[lane][c]);
+      const float2 pp = *reinterpret_cast<const float2*>(&sA[2 * w][c]);
+      const float2 qq = *reinterpret_cast<const float2*>(&sA[2 * w + 1][c]);
+      x0 = xx.x; x1 = xx.y; p0 = pp.x; p1 = pp.y; q0 = qq.x; q1 = qq.y;
+    }
+    a0 = fmaf(p0, x0, a0);
+    a0 = fmaf(p1, x1, a0);
+    a1 = fmaf(q0, x0, a1);
+    a1 = fmaf(q1, x1, a1);
+  }
+  const int t = t0 + lane, j = j0 + 2 * w;
+  if (t < M) {
+    float* out = zp + (static_cast<size_t>(blockIdx.y) * M + t) * r;
+    if (j < r) out[j] = a0;
+    if (j + 1 < r) out[j + 1] = a1;
   }
 }
 
-// h[t][i] += scale * sum_j B[i][j] z[t][j]: a CTA per 128 outputs i and 8 tokens, z rows of
-// the tokens in shared memory, Bt read coalesced over i.  Rows t with t mod m < causal_rows
-// (the fused fill's causal rows) are not drafter rows and keep h unchanged.
+// h[t][i] += scale * sum_j B[i][j] z[t][j], z = the activation-type rounding of the summed
+// partials.  A CTA per 128 outputs i and 8 tokens; thread i reads its own row of B in 64-column
+// chunks of 16-byte loads (all issued before the chunk's arithmetic); z rows broadcast from
+// shared memory.  Rows t with t mod m < causal_rows (the fused fill's causal rows) are not
+// drafter rows and keep h unchanged.
 template <typename T>
-__global__ void __launch_bounds__(128) lora_up_kernel(const T* Bt, const T* z, float* h, int M,
-                                                      int d, int r, float scale, int m,
+__global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* zp, float* h, int M,
+                                                      int d, int r, int n_ks, float scale, int m,
                                                       int causal_rows) {
-  extern __shared__ float s_z[];   // [8][r]
+  constexpr int kChunk = 64, V = 16 / sizeof(T), kLd = kChunk / V;
+  __shared__ __align__(16) float s_z[8][256];
   pdl_wait();
   pdl_launch_dependents();
   const int i = blockIdx.x * 128 + threadIdx.x;
@@ -310,77 +369,84 @@ __global__ void __launch_bounds__(128) lora_up_kernel(const T* Bt, const T* z, f
   const int nt = min(8, M - t0);
   for (int e = threadIdx.x; e < 8 * r; e += 128) {
     const int tt = e / r, j = e - tt * r;
-    s_z[e] = (tt < nt) ? to_f32<T>(z[static_cast<size_t>(t0 + tt) * r + j]) : 0.f;
+    float acc = 0.f;
+    if (tt < nt)
+      for (int ks = 0; ks < n_ks; ++ks) acc += zp[(static_cast<size_t>(ks) * M + t0 + tt) * r + j];
+    s_z[tt][j] = to_f32<T>(from_f32<T>(acc));
   }
   __syncthreads();
   if (i >= d) return;
   float acc[8];
 #pragma unroll
   for (int tt = 0; tt < 8; ++tt) acc[tt] = 0.f;
-  for (int j = 0; j < r; ++j) {
-    const float b = to_f32<T>(Bt[static_cast<size_t>(j) * d + i]);
+  const T* brow = B + static_cast<size_t>(i) * r;
+  for (int j0 = 0; j0 < r; j0 += kChunk) {
+    uint4 v[kLd];
 #pragma unroll
-    for (int tt = 0; tt < 8; ++tt) acc[tt] += b * s_z[tt * r + j];
+    for (int u = 0; u < kLd; ++u)
+      v[u] = (j0 + u * V < r) ? *reinterpret_cast<const uint4*>(brow + j0 + u * V) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const T* bv = reinterpret_cast<const T*>(&v[u]);
+      const int jb = j0 + u * V;
+      if (jb >= r) break;
+#pragma unroll
+      for (int q = 0; q < V; q += 4) {
+        const float b0 = to_f32<T>(bv[q]), b1 = to_f32<T>(bv[q + 1]);
+        const float b2 = to_f32<T>(bv[q + 2]), b3 = to_f32<T>(bv[q + 3]);
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+          const float4 z4 = *reinterpret_cast<const float4*>(&s_z[tt][jb + q]);
+          acc[tt] = fmaf(b0, z4.x, acc[tt]);
+          acc[tt] = fmaf(b1, z4.y, acc[tt]);
+          acc[tt] = fmaf(b2, z4.z, acc[tt]);
+          acc[tt] = fmaf(b3, z4.w, acc[tt]);
+        }
+      }
+    }
   }
   for (int tt = 0; tt < nt; ++tt)
     if ((t0 + tt) % m >= causal_rows) h[static_cast<size_t>(t0 + tt) * d + i] += scale * acc[tt];
 }
 
-// dst [cols, rows] = src [rows, cols]^T (LoRA B -> Bt at load time)
-template <typename T>
-__global__ void transpose_kernel(const T* src, T* dst, int rows, int cols) {
-  const size_t n = static_cast<size_t>(rows) * cols;
-  for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < n;
-       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t rr = e / cols, cc = e - rr * cols;
-    dst[cc * rows + rr] = src[e];
-  }
+int lora_n_ks(int qd, bool bf16) {
+  const int C = bf16 ? LoraCols<__nv_bfloat16>::n : LoraCols<float>::n;
+  return (qd + C - 1) / C;
 }
 
-cudaError_t launch_lora(cudaStream_t st, const void* A, const void* Bt, const void* att, void* z,
+cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
                         bool bf16, bool pdl) {
+  if (r < 8 || r > 256 || r % 8 || M < 1) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int n_ks = lora_n_ks(qd, bf16);
   cudaLaunchConfig_t c1 = {};
-  c1.gridDim = dim3(r);
-  c1.blockDim = dim3(256);
-  c1.dynamicSmemBytes = static_cast<size_t>(qd) * sizeof(float);
+  c1.gridDim = dim3((r + kLoraJ - 1) / kLoraJ, n_ks, (M + kLoraT - 1) / kLoraT);
+  c1.blockDim = dim3(kLoraThreads);
   c1.stream = st;
   c1.attrs = attr;
   c1.numAttrs = pdl ? 1 : 0;
   cudaLaunchConfig_t c2 = c1;
   c2.gridDim = dim3((d + 127) / 128, (M + 7) / 8);
   c2.blockDim = dim3(128);
-  c2.dynamicSmemBytes = static_cast<size_t>(8) * r * sizeof(float);
   cudaError_t e;
   if (bf16) {
     using T = __nv_bfloat16;
-    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T>, static_cast<const T*>(A), static_cast<const T*>(att),
-                           static_cast<T*>(z), M, qd, r);
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T>, static_cast<const T*>(A), static_cast<const T*>(att), zp,
+                           M, qd, r);
     if (e == cudaSuccess)
-      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T>, static_cast<const T*>(Bt), static_cast<const T*>(z), h,
-                             M, d, r, scale, m, causal_rows);
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T>, static_cast<const T*>(B), static_cast<const float*>(zp),
+                             h, M, d, r, n_ks, scale, m, causal_rows);
   } else {
     e = cudaLaunchKernelEx(&c1, lora_down_kernel<float>, static_cast<const float*>(A),
-                           static_cast<const float*>(att), static_cast<float*>(z), M, qd, r);
+                           static_cast<const float*>(att), zp, M, qd, r);
     if (e == cudaSuccess)
-      e = cudaLaunchKernelEx(&c2, lora_up_kernel<float>, static_cast<const float*>(Bt),
-                             static_cast<const float*>(z), h, M, d, r, scale, m, causal_rows);
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<float>, static_cast<const float*>(B),
+                             static_cast<const float*>(zp), h, M, d, r, n_ks, scale, m, causal_rows);
   }
   return e;
-}
-
-cudaError_t launch_transpose(cudaStream_t st, const void* src, void* dst, int rows, int cols, bool bf16) {
-  const int blocks = std::max(1, std::min(4096, (rows * cols + 255) / 256));
-  if (bf16)
-    transpose_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
-                                                            static_cast<__nv_bfloat16*>(dst), rows, cols);
-  else
-    transpose_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst),
-                                                    rows, cols);
-  return cudaGetLastError();
 }
 
 // -------------------------------------------------------------------------------- repack --

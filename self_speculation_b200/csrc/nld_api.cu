@@ -96,11 +96,11 @@ struct nld_ctx {
   std::vector<void*> wqkv, wo, wgu, wd;
   void* wlm = nullptr;
   bool weights_ready = false;
-  // LoRA drafter (optional): per layer A [r, qd] and Bt = B^T [r, d]; z [M_max, r]
+  // LoRA drafter (optional): per layer A [r, qd] and B [d, r]; fp32 z partials
   int lora_r = 0, lora_r_alloc = 0;
   float lora_scale = 0.f;
-  std::vector<void*> lora_A, lora_Bt;
-  void* lora_z = nullptr;
+  std::vector<void*> lora_A, lora_B;
+  float* lora_zp = nullptr;
   // KV cache
   void* pool = nullptr;
   int* page_table = nullptr;
@@ -530,7 +530,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
     }
     // LoRA drafter: the block-bidirectional rows (the fused fill's causal rows excluded)
     if (x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF))
-      CK(launch_lora(x->stream, x->lora_A[l], x->lora_Bt[l], x->attn, x->lora_z, x->h, M, x->qd,
+      CK(launch_lora(x->stream, x->lora_A[l], x->lora_B[l], x->attn, x->lora_zp, x->h, M, x->qd,
                      x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, x->bf16, pdl));
     int n = layer_chain(l, cur);
     int nn = 0;
@@ -780,7 +780,9 @@ nld_status nld_init_lora(nld_ctx* x, int rank, float scale, const void* const* t
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (!x->weights_ready) return fail(x, NLD_ERR_STATE, "weights not initialised");
   const int L = x->c.n_layers, d = x->c.d_model;
-  if (rank < 0 || rank > 256) return fail(x, NLD_ERR_ARG, "LoRA rank %d outside [0, 256]", rank);
+  if (rank < 0 || rank > 256 || rank % 8)
+    return fail(x, NLD_ERR_ARG, "LoRA rank %d: a multiple of 8 in [8, 256] (0 switches off)", rank);
+  if (x->qd % 8) return fail(x, NLD_ERR_UNSUPPORTED, "LoRA needs Hq*hd a multiple of 8");
   if (!std::isfinite(scale)) return fail(x, NLD_ERR_ARG, "LoRA scale is not finite");
   if (rank > 0) {
     if (!tensors || n_tensors != 2 * L)
@@ -800,30 +802,21 @@ nld_status nld_init_lora(nld_ctx* x, int rank, float scale, const void* const* t
   nld_status s;
   if (x->lora_A.empty()) {
     x->lora_A.assign(L, nullptr);
-    x->lora_Bt.assign(L, nullptr);
+    x->lora_B.assign(L, nullptr);
     for (int l = 0; l < L; ++l) {
       if ((s = dalloc(x, &x->lora_A[l], static_cast<size_t>(rank) * x->qd * el)) != NLD_OK) return s;
-      if ((s = dalloc(x, &x->lora_Bt[l], static_cast<size_t>(rank) * d * el)) != NLD_OK) return s;
+      if ((s = dalloc(x, &x->lora_B[l], static_cast<size_t>(d) * rank * el)) != NLD_OK) return s;
     }
-    if ((s = dalloc(x, &x->lora_z, static_cast<size_t>(x->M_max) * rank * el)) != NLD_OK) return s;
+    const size_t zp = static_cast<size_t>(lora_n_ks(x->qd, x->bf16)) * x->M_max * rank;
+    if ((s = dalloc(x, &x->lora_zp, zp * sizeof(float))) != NLD_OK) return s;
     x->lora_r_alloc = rank;
   }
-  void* stage = nullptr;
-  if ((s = dalloc(x, &stage, static_cast<size_t>(rank) * d * el)) != NLD_OK) return s;
   const cudaMemcpyKind kind = on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
-  nld_status rs = NLD_OK;
-  for (int l = 0; l < L && rs == NLD_OK; ++l) {
-    cudaError_t e = cudaMemcpyAsync(x->lora_A[l], tensors[2 * l], static_cast<size_t>(rank) * x->qd * el, kind,
-                                    x->stream);
-    if (e == cudaSuccess)
-      e = cudaMemcpyAsync(stage, tensors[2 * l + 1], static_cast<size_t>(d) * rank * el, kind, x->stream);
-    if (e == cudaSuccess) e = launch_transpose(x->stream, stage, x->lora_Bt[l], d, rank, x->bf16);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(x->stream);   // staging reuse
-    if (e != cudaSuccess) rs = fail(x, NLD_ERR_CUDA, "LoRA upload failed: %s", cudaGetErrorString(e));
+  for (int l = 0; l < L; ++l) {
+    CK(cudaMemcpyAsync(x->lora_A[l], tensors[2 * l], static_cast<size_t>(rank) * x->qd * el, kind, x->stream));
+    CK(cudaMemcpyAsync(x->lora_B[l], tensors[2 * l + 1], static_cast<size_t>(d) * rank * el, kind, x->stream));
   }
-  cudaFree(stage);
-  x->allocs.erase(std::remove(x->allocs.begin(), x->allocs.end(), stage), x->allocs.end());
-  if (rs != NLD_OK) return rs;
+  CK(cudaStreamSynchronize(x->stream));
   x->lora_r = rank;
   x->lora_scale = scale;
   return NLD_OK;

@@ -168,12 +168,13 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int* row_map,
                           int n_rows, int K, const void* gamma, bool bf16, bool tiled);
 cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
-// LoRA drafter: z = A att [M, r] (activation type), then h += scale * B z (two launches) on
-// the rows t with t mod m >= causal_rows.
-cudaError_t launch_lora(cudaStream_t st, const void* A, const void* Bt, const void* att, void* z,
+// LoRA drafter: fp32 partials zp [lora_n_ks][M][r] of z = A att, then h += scale * B z on
+// the rows t with t mod m >= causal_rows (z rounded to the activation type).  A [r, qd],
+// B [d, r] row-major; 8 <= r <= 256, r % 8 == 0; qd a multiple of 8.
+int lora_n_ks(int qd, bool bf16);
+cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
                         bool bf16, bool pdl);
-cudaError_t launch_transpose(cudaStream_t st, const void* src, void* dst, int rows, int cols, bool bf16);
 // Per 128-column tile sums of squares of bf16 rows h [M, d] into ssq [d/128, M].
 cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq);
 // Per token: argmax (lowest id on ties) and largest softmax probability from LM-head partials.

@@ -145,6 +145,20 @@ def model_weights(cfg: ModelConfig, seed: int = 0, device: str = "cpu",
     return out
 
 
+def lora_weights(cfg: ModelConfig, rank: int, seed: int, std: float = 0.02,
+                 device: str = "cpu") -> List[torch.Tensor]:
+    """An o_proj adapter in the boundary's order: per layer A [rank, Hq*hd] then B [d, rank],
+    N(0, std^2) drawn in fp32 from one CPU generator seeded with `seed` (A_0, B_0, A_1, ...),
+    stored in the config dtype and moved to `device`."""
+    g = torch.Generator().manual_seed(seed)
+    dt = _storage_dtype(cfg)
+    out: List[torch.Tensor] = []
+    for _ in range(cfg.n_layers):
+        out.append((torch.randn(rank, cfg.q_dim, generator=g) * std).to(dt).to(device))
+        out.append((torch.randn(cfg.d_model, rank, generator=g) * std).to(dt).to(device))
+    return out
+
+
 def prompt_tokens(batch: int, length: int, vocab: int, seed: int = 1) -> torch.Tensor:
     """Uniform-random real token ids in [0, vocab), int32 [batch, length] (stand-in for the
     benchmark prompts, which are not available)."""

@@ -20,13 +20,9 @@ pytestmark = pytest.mark.gpu
 
 
 def _adapter(cfg, r, seed, std):
-    """A [r, Hq*hd], B [d, r] per layer, already representable in the config dtype."""
-    g = torch.Generator().manual_seed(seed)
-    qd = cfg.n_q_heads * cfg.head_dim
-    dt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
-    A = [(torch.randn(r, qd, generator=g) * std).to(dt) for _ in range(cfg.n_layers)]
-    B = [(torch.randn(cfg.d_model, r, generator=g) * std).to(dt) for _ in range(cfg.n_layers)]
-    return A, B
+    """A [r, Hq*hd], B [d, r] per layer, in the config dtype."""
+    flat = synth.lora_weights(cfg, r, seed, std)
+    return flat[0::2], flat[1::2]
 
 
 def _load(ctx, om, A, B, scale):
