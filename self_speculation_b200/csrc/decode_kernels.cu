@@ -367,12 +367,24 @@ __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* z
   const int i = blockIdx.x * 128 + threadIdx.x;
   const int t0 = blockIdx.y * 8;
   const int nt = min(8, M - t0);
-  for (int e = threadIdx.x; e < 8 * r; e += 128) {
-    const int tt = e / r, j = e - tt * r;
-    float acc = 0.f;
-    if (tt < nt)
-      for (int ks = 0; ks < n_ks; ++ks) acc += zp[(static_cast<size_t>(ks) * M + t0 + tt) * r + j];
-    s_z[tt][j] = to_f32<T>(from_f32<T>(acc));
+  // the 8 token rows of a partial are contiguous (8*r floats): element e = tt*r + j; each
+  // slice's loads of all of a thread's elements are independent, summed in slice order
+  constexpr int kQ = 8 * 256 / 128;
+  float za[kQ];
+#pragma unroll
+  for (int q = 0; q < kQ; ++q) za[q] = 0.f;
+  for (int ks = 0; ks < n_ks; ++ks) {
+    const float* zk = zp + (static_cast<size_t>(ks) * M + t0) * r;
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      const int e = q * 128 + threadIdx.x;
+      if (e < nt * r) za[q] += zk[e];
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kQ; ++q) {
+    const int e = q * 128 + threadIdx.x;
+    if (e < 8 * r) s_z[e / r][e % r] = to_f32<T>(from_f32<T>(za[q]));   // rows >= nt: zero
   }
   __syncthreads();
   if (i >= d) return;
