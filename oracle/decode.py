@@ -35,6 +35,10 @@ Readings where the pages are silent (each is listed with its reason in the desig
   causal and whose last k rows are one bidirectional block that sees the first k.  In exact
   arithmetic its KV rows n..n+k-1 and its last k logit rows equal those of the fill followed
   by the plain denoising forward.
+* Per-sequence (non-lockstep) diffusion: a sequence whose block completed runs its causal KV
+  fill in its next step while the other sequences of the batch keep denoising; each step is
+  one forward of k rows per sequence.  Sequences never see one another, so every sequence's
+  tokens equal those it would generate alone.
 """
 from __future__ import annotations
 
@@ -256,6 +260,77 @@ def diffusion_step_fused(model, st: SeqState, k: int, tau: float, fill_pending: 
     blocks = [list(st.block[b]) for b in range(B)] if complete else None
     return dict(newly=newly, conf=conf, argmax=am, complete=complete, blocks=blocks,
                 logits=logits), complete
+
+
+def _one(st: SeqState, b: int) -> SeqState:
+    """Sequence b of st as a batch of one: its cache and block lists are shared with st, its
+    length and pending token copied."""
+    return SeqState(cache=[st.cache[b]], lens=[st.lens[b]], pending=[st.pending[b]],
+                    block=None if st.block is None else [st.block[b]])
+
+
+def diffusion_step_nonlockstep(model, st: SeqState, k: int, tau: float, fill_next: List[bool]):
+    """One step of per-sequence (non-lockstep) diffusion: every sequence takes k rows of one
+    forward.  A sequence whose block completed in an earlier step (fill_next[b]) runs its
+    causal KV fill over [x_n, b_1..b_{k-1}] (then len += k, pending = b_k, a fresh block of
+    masks); every other sequence takes one denoising step with the commit rule of
+    diffusion_step.  No sequence waits for the others.  Sequences are independent, so each is
+    computed as a batch of one.  Returns (newly [B] (slot, token) lists, state [B]: 0 block
+    still open, 1 block completed by this step, 2 filled in this step; blocks [B]: the
+    completed block where state is 1, else None; the new fill_next)."""
+    mask_id = model.cfg.mask_id
+    B = len(st.lens)
+    if st.block is None:
+        st.block = [[mask_id] * k for _ in range(B)]
+    newly, state, blocks, nxt = [], [], [], []
+    for b in range(B):
+        one = _one(st, b)
+        if fill_next[b]:
+            toks = torch.tensor([[one.pending[0]] + one.block[0][:k - 1]], dtype=torch.int64)
+            model.forward(toks, one.lens, one.cache, block_size=1, write_kv=True, with_logits=False)
+            st.lens[b] += k
+            st.pending[b] = st.block[b][k - 1]
+            st.block[b] = [mask_id] * k
+            newly.append([])
+            state.append(2)
+            blocks.append(None)
+            nxt.append(False)
+            continue
+        logits = diffusion_forward(model, one, k)
+        conf = confidence(logits)[0]
+        am = argmax_lowest(logits)[0]
+        masked = [t == mask_id for t in st.block[b]]
+        pick = diffusion_commit(masked, conf.tolist(), tau)
+        got = []
+        for slot in range(k):
+            if pick[slot]:
+                st.block[b][slot] = int(am[slot])
+                got.append((slot, int(am[slot])))
+        newly.append(got)
+        done = mask_id not in st.block[b]
+        state.append(1 if done else 0)
+        blocks.append(list(st.block[b]) if done else None)
+        nxt.append(done)
+    return newly, state, blocks, nxt
+
+
+def diffuse_generate_nonlockstep(model, prompt: torch.Tensor, n_tokens: int, k: int, tau: float,
+                                 capacity: int) -> Tuple[List[List[int]], int, List[List[int]]]:
+    """Per-sequence diffusion until every sequence has n_tokens.  Returns (tokens per sequence
+    in position order, number of forwards (= steps: one batched forward each), the per-step
+    state lists)."""
+    st = prefill(model, prompt, capacity)
+    B = prompt.shape[0]
+    out = [[] for _ in range(B)]
+    fill_next = [False] * B
+    states = []
+    while min(len(o) for o in out) < n_tokens:
+        _, state, blocks, fill_next = diffusion_step_nonlockstep(model, st, k, tau, fill_next)
+        states.append(state)
+        for b in range(B):
+            if state[b] == 1:
+                out[b].extend(blocks[b])
+    return [o[:n_tokens] for o in out], len(states), states
 
 
 # ---- generation drivers (exactly N generated tokens; the last round is truncated) ----------

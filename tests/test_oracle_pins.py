@@ -522,3 +522,52 @@ def test_lora_only_in_drafter_forwards():
     zero = [torch.zeros_like(b) for b in B]
     lo.set_lora(A, zero, 5.0)
     assert torch.equal(odec.draft_forward(lo, s1, 8), odec.draft_forward(pl, s2, 8))
+
+
+# ---------------------------------------------- per-sequence diffusion (next row f4) --
+
+def _varied_prompts(cfg, B, P, seed):
+    return synth.prompt_tokens(B, P, cfg.vocab, seed=seed)
+
+
+@pytest.mark.parametrize("tau", [0.9, 0.6, 0.3])
+def test_nonlockstep_tokens_equal_each_sequence_alone(tau):
+    """Sequences are independent: per-sequence diffusion of a batch gives every sequence the
+    tokens the lockstep driver gives it alone (fp64)."""
+    cfg = _tiny(n_layers=1)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0, lm_head_scale=30.0), "f64")
+    p = _varied_prompts(cfg, 3, 10, seed=6)
+    k = 4
+    got, forwards, states = odec.diffuse_generate_nonlockstep(mdl, p, 12, k, tau, 96)
+    for b in range(3):
+        alone, _ = odec.diffuse_generate(mdl, p[b:b + 1], 12, k, tau, 96)
+        assert got[b] == alone[0]
+    # every step is one forward; a fill always follows the step that completed the block
+    assert forwards == len(states)
+    for b in range(3):
+        seq = [st[b] for st in states]
+        for i, v in enumerate(seq[:-1]):
+            assert (seq[i + 1] == 2) == (v == 1)
+
+
+def test_nonlockstep_saves_forwards_when_progress_differs():
+    """With sequences that finish their blocks at different steps, lockstep runs every block
+    as long as the slowest sequence; per-sequence scheduling does not wait (forwards counted
+    for the same number of generated tokens)."""
+    cfg = _tiny(n_layers=1)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0, lm_head_scale=30.0), "f64")
+    p = _varied_prompts(cfg, 3, 10, seed=6)
+    k, tau, n = 4, 0.6, 12
+    _, nl_forwards, states = odec.diffuse_generate_nonlockstep(mdl, p, n, k, tau, 96)
+    # lockstep: each step is one forward, plus one fill forward per completed set of blocks
+    _, ls_steps = odec.diffuse_generate(mdl, p, n, k, tau, 96)
+    ls_forwards = ls_steps + n // k
+    # per sequence, the steps it needs alone (denoising + one fill per block)
+    alone = []
+    for b in range(3):
+        _, s1 = odec.diffuse_generate(mdl, p[b:b + 1], n, k, tau, 96)
+        alone.append(s1 + n // k)
+    assert len(set(alone)) > 1                        # the sequences progress differently
+    assert nl_forwards < ls_forwards
+    # the batch runs until its slowest sequence is done, give or take its last fill
+    assert max(alone) - 1 <= nl_forwards <= max(alone) + 1
