@@ -178,6 +178,23 @@ nld_status nld_diffuse_block_step_fused(nld_ctx* ctx, float threshold, int32_t* 
                                         float* d_conf_out, int32_t* d_ncommit_out,
                                         int32_t* h_filled_out);
 
+/* Per-sequence (non-lockstep) diffusion step: one forward of k rows per sequence in which a
+ * sequence whose block completed in an earlier call runs its causal KV fill over
+ * [x_n, b_1..b_{k-1}] (all its rows causal; then len += k, pending = b_k, a fresh block of
+ * masks) while every other sequence takes one denoising step with the commit rule of
+ * nld_diffuse_block_step.  No sequence waits for the batch and the call does not synchronise
+ * (the decision is a device-side flag per sequence).  A reading of the Nemotron-Labs-Diffusion
+ * pages, which state block progress only for one sequence and pitch the modes at workloads of
+ * unpredictable batch size (shilu.ai blog, the three generation modes): progress is per
+ * sequence, each sequence's tokens are those it would generate alone.  Outputs (device, may be NULL): block [batch, k]
+ * after the step (mask id = open; all masks after a fill), conf [batch, k] (0 after a fill),
+ * ncommit [batch] (0 after a fill), state [batch]: 0 block still open, 1 block completed by
+ * this step (its tokens are in block; the fill runs in the next call), 2 filled in this call.
+ * A fill still due when another decode call comes runs first, in one forward (after a host
+ * read of the flags). */
+nld_status nld_diffuse_step_nonlockstep(nld_ctx* ctx, float threshold, int32_t* d_block_out,
+                                        float* d_conf_out, int32_t* d_ncommit_out, int32_t* d_state_out);
+
 /* Test hook: run the forward of `mode` (NLD_MODE_*) from the current state and write its
  * logits [batch, m, vocab] fp32 to d_logits_out (m = 1, k, k+1, k).  Sequence state is not
  * advanced; a DRAFT call stores its argmaxes as the drafts a later VERIFY call reads.  The

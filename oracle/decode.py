@@ -269,6 +269,23 @@ def _one(st: SeqState, b: int) -> SeqState:
                     block=None if st.block is None else [st.block[b]])
 
 
+def _fill_one(model, st: SeqState, b: int, k: int) -> None:
+    """Causal KV fill of sequence b's complete block: len += k, pending = b_k, fresh masks."""
+    one = _one(st, b)
+    toks = torch.tensor([[one.pending[0]] + one.block[0][:k - 1]], dtype=torch.int64)
+    model.forward(toks, one.lens, one.cache, block_size=1, write_kv=True, with_logits=False)
+    st.lens[b] += k
+    st.pending[b] = st.block[b][k - 1]
+    st.block[b] = [model.cfg.mask_id] * k
+
+
+def flush_fills(model, st: SeqState, k: int, fill_next: List[bool]) -> None:
+    """Run the fills that per-sequence diffusion left due (before another decode mode)."""
+    for b in range(len(st.lens)):
+        if fill_next[b]:
+            _fill_one(model, st, b, k)
+
+
 def diffusion_step_nonlockstep(model, st: SeqState, k: int, tau: float, fill_next: List[bool]):
     """One step of per-sequence (non-lockstep) diffusion: every sequence takes k rows of one
     forward.  A sequence whose block completed in an earlier step (fill_next[b]) runs its
@@ -286,11 +303,7 @@ def diffusion_step_nonlockstep(model, st: SeqState, k: int, tau: float, fill_nex
     for b in range(B):
         one = _one(st, b)
         if fill_next[b]:
-            toks = torch.tensor([[one.pending[0]] + one.block[0][:k - 1]], dtype=torch.int64)
-            model.forward(toks, one.lens, one.cache, block_size=1, write_kv=True, with_logits=False)
-            st.lens[b] += k
-            st.pending[b] = st.block[b][k - 1]
-            st.block[b] = [mask_id] * k
+            _fill_one(model, st, b, k)
             newly.append([])
             state.append(2)
             blocks.append(None)

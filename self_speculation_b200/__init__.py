@@ -59,6 +59,7 @@ def load_library() -> ctypes.CDLL:
         "nld_selfspec_round": ([P, P, P, P], I),
         "nld_diffuse_block_step": ([P, F, P, P, P, P], I),
         "nld_diffuse_block_step_fused": ([P, F, P, P, P, P], I),
+        "nld_diffuse_step_nonlockstep": ([P, F, P, P, P, P], I),
         "nld_debug_logits": ([P, I, P], I),
         "nld_debug_state": ([P, P, P, P, P], I),
         "nld_sync": ([P], I),
@@ -179,6 +180,12 @@ class Context:
                                                           _ptr(conf_out), _ptr(ncommit_out),
                                                           ctypes.byref(filled)), self.h)
         return bool(filled.value)
+
+    def nld_diffuse_step_nonlockstep(self, threshold: float, block_out=None, conf_out=None,
+                                     ncommit_out=None, state_out=None) -> None:
+        self._check(self.lib.nld_diffuse_step_nonlockstep(self.h, float(threshold), _ptr(block_out),
+                                                          _ptr(conf_out), _ptr(ncommit_out),
+                                                          _ptr(state_out)), self.h)
 
     def nld_debug_logits(self, mode: int, logits_out) -> None:
         self._check(self.lib.nld_debug_logits(self.h, int(mode), _ptr(logits_out)), self.h)

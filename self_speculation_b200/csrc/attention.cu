@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     if (tid == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
     len = max(0, min(len, a.pps * kPage - a.m));
   }
-  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m, a.causal_rows) + 1;
+  const int crow = (a.causal_seq && a.causal_seq[b]) ? a.m : a.causal_rows;
+  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m, crow) + 1;
   const int n_tiles = (kv_end + kPage - 1) / kPage;
   // at least two KV tiles per split: fewer, fuller splits keep the merge short
   const int per = max(2, (n_tiles + a.S - 1) / a.S);
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   auto row_vis = [&](int r) {
     const int p = r / a.G;
     if (r >= a.rows || p >= np) return -1;
-    return vis_end_of(len, p0 + p, a.block_size, a.m, a.causal_rows);
+    return vis_end_of(len, p0 + p, a.block_size, a.m, crow);
   };
   const int vis_a = row_vis(ra), vis_b = row_vis(rb);
 
@@ -381,7 +382,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
     if (threadIdx.x == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
     len = max(0, min(len, a.pps * kPage - a.m));
   }
-  const int nkeys = vis_end_of(len, i, a.block_size, a.m, a.causal_rows) + 1;
+  const int crow = (a.causal_seq && a.causal_seq[b]) ? a.m : a.causal_rows;
+  const int nkeys = vis_end_of(len, i, a.block_size, a.m, crow) + 1;
   const T* q = static_cast<const T*>(a.q) + (static_cast<size_t>(tok) * a.Hq + head) * a.hd;
   for (int d = threadIdx.x; d < a.hd; d += blockDim.x) sq[d] = to_f32<T>(q[d]);
   __syncthreads();

@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool lm = (a.mode == FWD_AR || a.mode == FWD_DRAFT || a.mode == FWD_VERIFY ||
-                   a.mode == FWD_DIFFUSE || a.mode == FWD_FILLDIFF);
+                   a.mode == FWD_DIFFUSE || a.mode == FWD_FILLDIFF || a.mode == FWD_NLDIFF);
   if (lm) {
     // one warp per row; one pass over the row's vocab tiles with 8 loads in flight per lane,
     // merging (max, sum exp, argmax) online, then across the warp
@@ -183,8 +183,32 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
         a.pending[b] = a.verify[b * (k + 1) + c - 1];
       }
     } break;
+    case FWD_NLFILL:
+    case FWD_NLDIFF:
     case FWD_FILLDIFF:
     case FWD_DIFFUSE: {
+      // FWD_NLDIFF / FWD_NLFILL (per-sequence diffusion): a sequence flagged in fillnext ran its
+      // causal KV fill in this forward (all its rows causal): len += k, pending = b_k, a fresh
+      // block of masks.  The others denoise (FWD_NLFILL: keep their state).
+      const bool nl = (a.mode == FWD_NLDIFF || a.mode == FWD_NLFILL);
+      if (nl && a.fillnext[b] != 0) {
+        const int last = a.blk[b * k + k - 1];
+        __syncwarp();
+        for (int i = lane; i < k; i += 32) {
+          a.blk[b * k + i] = a.V;
+          if (a.block_out) a.block_out[b * k + i] = a.V;
+          if (a.conf_out) a.conf_out[b * k + i] = 0.f;
+        }
+        if (lane == 0) {
+          a.lens[b] += k;
+          a.pending[b] = last;
+          a.fillnext[b] = 0;
+          if (a.ncommit_out) a.ncommit_out[b] = 0;
+          if (a.state_out) a.state_out[b] = 2;
+        }
+        break;
+      }
+      if (a.mode == FWD_NLFILL) break;
       // FWD_FILLDIFF: the complete block's KV rows were written by this forward's first k
       // (causal) rows: len += k, pending = b_k, and the new block (all masks) is denoised by
       // the last k rows
@@ -235,6 +259,10 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
       if (lane == 0) {
         if (a.ncommit_out) a.ncommit_out[b] = __popc(picked);
         if (a.commit && still_open != 0u && a.incomplete) atomicAdd(a.incomplete, 1);
+        if (nl) {   // a completed block is filled by this sequence's next step
+          if (a.commit) a.fillnext[b] = (still_open == 0u) ? 1 : 0;
+          if (a.state_out) a.state_out[b] = (still_open == 0u) ? 1 : 0;
+        }
       }
     } break;
     case FWD_FILL: {
@@ -354,12 +382,13 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
 // h[t][i] += scale * sum_j B[i][j] z[t][j], z = the activation-type rounding of the summed
 // partials.  A CTA per 128 outputs i and 8 tokens; thread i reads its own row of B in 64-column
 // chunks of 16-byte loads (all issued before the chunk's arithmetic); z rows broadcast from
-// shared memory.  Rows t with t mod m < causal_rows (the fused fill's causal rows) are not
-// drafter rows and keep h unchanged.
+// shared memory.  Rows t with t mod m < causal_rows (the fused fill's causal rows) and the
+// rows of sequences flagged in causal_seq (a per-sequence fill) are not drafter rows and keep h
+// unchanged.
 template <typename T>
 __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* zp, float* h, int M,
                                                       int d, int r, int n_ks, float scale, int m,
-                                                      int causal_rows) {
+                                                      int causal_rows, const int* causal_seq) {
   constexpr int kChunk = 64, V = 16 / sizeof(T), kLd = kChunk / V;
   __shared__ __align__(16) float s_z[8][256];
   pdl_wait();
@@ -418,7 +447,8 @@ __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* z
     }
   }
   for (int tt = 0; tt < nt; ++tt)
-    if ((t0 + tt) % m >= causal_rows) h[static_cast<size_t>(t0 + tt) * d + i] += scale * acc[tt];
+    if ((t0 + tt) % m >= causal_rows && !(causal_seq && causal_seq[(t0 + tt) / m]))
+      h[static_cast<size_t>(t0 + tt) * d + i] += scale * acc[tt];
 }
 
 int lora_n_ks(int qd, bool bf16) {
@@ -428,7 +458,7 @@ int lora_n_ks(int qd, bool bf16) {
 
 cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
-                        bool bf16, bool pdl) {
+                        const int* causal_seq, bool bf16, bool pdl) {
   if (r < 8 || r > 256 || r % 8 || M < 1) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -450,13 +480,14 @@ cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const voi
                            M, qd, r);
     if (e == cudaSuccess)
       e = cudaLaunchKernelEx(&c2, lora_up_kernel<T>, static_cast<const T*>(B), static_cast<const float*>(zp),
-                             h, M, d, r, n_ks, scale, m, causal_rows);
+                             h, M, d, r, n_ks, scale, m, causal_rows, causal_seq);
   } else {
     e = cudaLaunchKernelEx(&c1, lora_down_kernel<float>, static_cast<const float*>(A),
                            static_cast<const float*>(att), zp, M, qd, r);
     if (e == cudaSuccess)
       e = cudaLaunchKernelEx(&c2, lora_up_kernel<float>, static_cast<const float*>(B),
-                             static_cast<const float*>(zp), h, M, d, r, n_ks, scale, m, causal_rows);
+                             static_cast<const float*>(zp), h, M, d, r, n_ks, scale, m, causal_rows,
+                             causal_seq);
   }
   return e;
 }

@@ -108,6 +108,7 @@ struct nld_ctx {
   // device state
   int *lens = nullptr, *pending = nullptr, *draft = nullptr, *verify = nullptr, *blk = nullptr;
   int *incomplete = nullptr, *err = nullptr, *prompt = nullptr;
+  int* fillnext = nullptr;   // per-sequence diffusion: block complete, causal fill due next step
   // activations
   float* h = nullptr;
   void* hb = nullptr;
@@ -121,7 +122,7 @@ struct nld_ctx {
   int max_clusters[9] = {0};
   unsigned* bars = nullptr;   // chain phase-boundary counters: (1 + n_layers) x kMaxPhases
   int n_bars = 0;
-  int* h_pinned = nullptr;  // host: [0] error word, [1] incomplete, [2..] lens
+  int* h_pinned = nullptr;  // host: [0] error word, [1] incomplete, [2..2+B) lens, then fillnext
   // tensor maps
   std::vector<CUtensorMap> tmWqkv, tmWo, tmWgu, tmWd;
   CUtensorMap tmWlm{};
@@ -134,6 +135,7 @@ struct nld_ctx {
   bool started = false;
   bool verify_fresh = false;
   bool fill_pending = false;   // a complete diffusion block whose causal KV fill is deferred
+  bool nl_active = false;      // per-sequence diffusion ran: fills may be due on the device
   long long len_upper = 0;
   uint64_t timeout_ns = 2000000000ull;
   std::string msg;
@@ -443,6 +445,7 @@ struct FwdSpec {
   int prompt_len;
   bool last_chunk;
   int causal_rows;   // attention: leading strictly causal rows (fused diffusion fill)
+  const int* causal_seq;   // per-sequence diffusion: sequences whose rows are all causal
 };
 
 // Launch one forward (no finalize).
@@ -483,6 +486,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.pps = x->pps;
   aa.block_size = f.bs;
   aa.causal_rows = f.causal_rows;
+  aa.causal_seq = f.causal_seq;
   aa.err = x->err;
   aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
   if (x->bf16) {
@@ -529,9 +533,11 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
       CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
     }
     // LoRA drafter: the block-bidirectional rows (the fused fill's causal rows excluded)
-    if (x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF))
+    if (x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF ||
+                          f.mode == FWD_NLDIFF))
       CK(launch_lora(x->stream, x->lora_A[l], x->lora_B[l], x->attn, x->lora_zp, x->h, M, x->qd,
-                     x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, x->bf16, pdl));
+                     x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, f.causal_seq,
+                     x->bf16, pdl));
     int n = layer_chain(l, cur);
     int nn = 0;
     if (l + 1 < L) {
@@ -564,6 +570,8 @@ FinalizeArgs base_fin(nld_ctx* x, int mode, int m) {
   a.commit = 1;
   a.kv_cap = x->kv_cap;
   a.err = x->err;
+  a.fillnext = x->fillnext;
+  a.state_out = nullptr;
   return a;
 }
 
@@ -749,7 +757,9 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
   if (cudaMemset(x->hb, 0, Mm * d * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->attn, 0, Mm * x->qd * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->ubuf, 0, Mm * c.ffn_dim * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
-  if (cudaMallocHost(&x->h_pinned, (4 + B) * sizeof(int)) != cudaSuccess)
+  if ((s = dalloc(x, &x->fillnext, B * sizeof(int))) != NLD_OK) return bail(s);
+  if (cudaMemset(x->fillnext, 0, B * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMallocHost(&x->h_pinned, (4 + 2 * B) * sizeof(int)) != cudaSuccess)
     return bail(fail(x, NLD_ERR_OOM, "pinned host allocation failed"));
   if (x->bf16) {
     const uint64_t rows = static_cast<uint64_t>(c.n_layers) * x->n_pages * 2 * c.n_kv_heads * kPage;
@@ -958,6 +968,8 @@ nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int promp
   CK(launch_fill_i32(x->stream, x->blk, x->c.vocab, batch * k));
   CK(launch_fill_i32(x->stream, x->draft, x->c.vocab, batch * k));
   CK(launch_fill_i32(x->stream, x->verify, -1, batch * (k + 1)));
+  CK(cudaMemsetAsync(x->fillnext, 0, batch * sizeof(int), x->stream));
+  x->nl_active = false;
   x->len_upper = 0;
   const int chunk = std::max(1, x->prefill_tokens / batch);
   const int rows = prompt_len - 1;
@@ -1110,8 +1122,62 @@ nld_status run_fill(nld_ctx* x) {
   return NLD_OK;
 }
 
-// A deferred fill runs alone before any other decode call.
-nld_status flush_fill(nld_ctx* x) { return x->fill_pending ? run_fill(x) : NLD_OK; }
+// One forward of per-sequence diffusion: sequences flagged in fillnext run their causal KV
+// fill, the others denoise (fill_only: keep their state, no LM head).
+nld_status run_nl(nld_ctx* x, bool fill_only, float threshold, int32_t* d_block_out, float* d_conf_out,
+                  int32_t* d_ncommit_out, int32_t* d_state_out) {
+  const int k = x->c.block_k;
+  TRY(ensure_capacity(x, k));
+  uint32_t thr_bits;
+  std::memcpy(&thr_bits, &threshold, 4);
+  std::vector<uintptr_t> key = {static_cast<uintptr_t>(fill_only ? 9 : 8), static_cast<uintptr_t>(x->batch),
+                                reinterpret_cast<uintptr_t>(d_block_out), reinterpret_cast<uintptr_t>(d_conf_out),
+                                reinterpret_cast<uintptr_t>(d_ncommit_out), reinterpret_cast<uintptr_t>(d_state_out),
+                                thr_bits};
+  TRY(run_graph(x, key, [&]() -> nld_status {
+    const long long saved = x->len_upper;
+    x->len_upper = x->c.max_seq;
+    FwdSpec f{};
+    f.mode = fill_only ? FWD_NLFILL : FWD_NLDIFF;
+    f.B = x->batch;
+    f.m = k;
+    f.bs = k;
+    f.causal_seq = x->fillnext;
+    f.lm = fill_only ? LM_NONE : LM_ARGMAX;
+    nld_status s = launch_forward(x, f);
+    x->len_upper = saved;
+    if (s != NLD_OK) return s;
+    FinalizeArgs a = base_fin(x, f.mode, k);
+    a.threshold = threshold;
+    a.block_out = d_block_out;
+    a.conf_out = d_conf_out;
+    a.ncommit_out = d_ncommit_out;
+    a.state_out = d_state_out;
+    a.incomplete = nullptr;
+    return finalize(x, a);
+  }));
+  x->len_upper += k;   // upper bound: a fill grows a sequence by k
+  return NLD_OK;
+}
+
+// Fills that per-sequence diffusion left due run before any other decode call: one forward,
+// only if some sequence is flagged.
+nld_status flush_nl(nld_ctx* x) {
+  if (!x->nl_active) return NLD_OK;
+  x->nl_active = false;
+  int* flags = x->h_pinned + 2 + x->batch;
+  CK(cudaMemcpyAsync(flags, x->fillnext, sizeof(int) * x->batch, cudaMemcpyDeviceToHost, x->stream));
+  CK(cudaStreamSynchronize(x->stream));
+  bool any = false;
+  for (int b = 0; b < x->batch; ++b) any = any || flags[b] != 0;
+  return any ? run_nl(x, true, 0.f, nullptr, nullptr, nullptr, nullptr) : NLD_OK;
+}
+
+// A deferred fill (lockstep or per-sequence) runs alone before any other decode call.
+nld_status flush_fill(nld_ctx* x) {
+  TRY(flush_nl(x));
+  return x->fill_pending ? run_fill(x) : NLD_OK;
+}
 
 // One denoising forward + commit (fused = the deferred fill of the previous block and the new
 // block's first step in one forward of 2k rows); returns the number of sequences whose block
@@ -1174,6 +1240,7 @@ nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_
 nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_block_out,
                                         float* d_conf_out, int32_t* d_ncommit_out, int32_t* h_filled_out) {
   TRY(need_started(x));
+  TRY(flush_nl(x));
   const int k = x->c.block_k;
   const bool fused = x->fill_pending;
   if (fused && (2 * k > 64 || x->batch * 2 * k > x->M_max))
@@ -1187,6 +1254,16 @@ nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_
   }
   if (open == 0) x->fill_pending = true;   // this block's fill joins the next step
   if (h_filled_out) *h_filled_out = fused ? 1 : 0;
+  x->verify_fresh = false;
+  return NLD_OK;
+}
+
+nld_status nld_diffuse_step_nonlockstep(nld_ctx* x, float threshold, int32_t* d_block_out, float* d_conf_out,
+                                        int32_t* d_ncommit_out, int32_t* d_state_out) {
+  TRY(need_started(x));
+  if (x->fill_pending) TRY(run_fill(x));   // a lockstep block's deferred fill
+  TRY(run_nl(x, false, threshold, d_block_out, d_conf_out, d_ncommit_out, d_state_out));
+  x->nl_active = true;
   x->verify_fresh = false;
   return NLD_OK;
 }

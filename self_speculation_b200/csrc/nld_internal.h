@@ -28,7 +28,9 @@ enum EpiKind : int {
 enum FwdMode : int {
   FWD_AR = 0, FWD_DRAFT = 1, FWD_VERIFY = 2, FWD_DIFFUSE = 3, FWD_FILL = 4, FWD_PREFILL = 5,
   FWD_COMMIT = 6,
-  FWD_FILLDIFF = 7   // fused diffusion KV fill: [x_n, b_1..b_k, MASK x (k-1)], 2k rows
+  FWD_FILLDIFF = 7,  // fused diffusion KV fill: [x_n, b_1..b_k, MASK x (k-1)], 2k rows
+  FWD_NLDIFF = 8,    // per-sequence diffusion: flagged sequences fill, the others denoise
+  FWD_NLFILL = 9     // per-sequence diffusion: flagged sequences fill, the others keep state
 };
 
 // Per (token, vocab tile) partial of the LM-head reduction.
@@ -122,6 +124,7 @@ struct AttnArgs {
   int block_size;
   int causal_rows;      // the first causal_rows rows of each sequence are strictly causal and
                         // the blocks of block_size start after them (fused diffusion fill)
+  const int* causal_seq;  // optional [batch]: nonzero makes all m rows of that sequence causal
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   float scale_log2;     // log2(e) / sqrt(hd)
   int* err;
@@ -162,6 +165,8 @@ struct FinalizeArgs {
   int commit;           // 0 = only record argmaxes (test hook)
   int kv_cap;
   int* err;
+  int* fillnext;        // per-sequence diffusion: [batch] fill flags (read and updated)
+  int* state_out;       // per-sequence diffusion: 0 open, 1 completed now, 2 filled now
 };
 cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, bool pdl);
 
@@ -169,12 +174,13 @@ cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int
                           int n_rows, int K, const void* gamma, bool bf16, bool tiled);
 cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
 // LoRA drafter: fp32 partials zp [lora_n_ks][M][r] of z = A att, then h += scale * B z on
-// the rows t with t mod m >= causal_rows (z rounded to the activation type).  A [r, qd],
+// the rows t with t mod m >= causal_rows of sequences b = t / m whose causal_seq flag (if
+// given) is zero (z rounded to the activation type).  A [r, qd],
 // B [d, r] row-major; 8 <= r <= 256, r % 8 == 0; qd a multiple of 8.
 int lora_n_ks(int qd, bool bf16);
 cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
-                        bool bf16, bool pdl);
+                        const int* causal_seq, bool bf16, bool pdl);
 // Per 128-column tile sums of squares of bf16 rows h [M, d] into ssq [d/128, M].
 cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq);
 // Per token: argmax (lowest id on ties) and largest softmax probability from LM-head partials.
