@@ -40,6 +40,7 @@ def test_generation_and_states_token_exact_f32(scale, tau):
     states = []
     while min(len(o) for o in out) < n:
         ctx.nld_diffuse_step_nonlockstep(tau, blk, conf, nc, state)
+        ctx.nld_sync()          # the call does not synchronise; outputs are read next
         s = state.cpu().tolist()
         states.append(s)
         g = blk.cpu().tolist()
@@ -66,6 +67,7 @@ def test_due_fill_runs_before_ar_f32():
     # step until some sequence has a completed block whose fill is due and another has not
     for _ in range(20):
         ctx.nld_diffuse_step_nonlockstep(tau, blk, conf, nc, state)
+        ctx.nld_sync()          # the call does not synchronise; outputs are read next
         _, wstate, _, fill_next = odec.diffusion_step_nonlockstep(om, st, k, tau, fill_next)
         assert state.cpu().tolist() == wstate
         if any(fill_next) and not all(fill_next):
@@ -93,6 +95,7 @@ def test_bookkeeping_and_commit_rule_bf16():
     # threshold 0 commits every open slot: blocks complete at steps 2 and 5, fill at 3 and 6
     for tau in [0.9, 0.9, 0.0, 0.9, 0.9, 0.0, 0.9]:
         ctx.nld_diffuse_step_nonlockstep(tau, blk, conf, nc, state)
+        ctx.nld_sync()          # the call does not synchronise; outputs are read next
         s = state.cpu().tolist()
         lens, pend, _, _ = gpu_state(ctx, B)
         g_blk, g_conf = blk.cpu().tolist(), conf.cpu()
