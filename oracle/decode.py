@@ -35,6 +35,12 @@ Readings where the pages are silent (each is listed with its reason in the desig
   causal and whose last k rows are one bidirectional block that sees the first k.  In exact
   arithmetic its KV rows n..n+k-1 and its last k logit rows equal those of the fill followed
   by the plain denoising forward.
+* Quadratic self-speculation (named by the pages, not defined there): one forward per round
+  holds the causal verify rows of the current drafts and, for each possible acceptance
+  length a = 0..k, a pre-draft block of the next round (k mask rows at n+a+1..n+a+k that see
+  the prefix, the verify rows of x_n, d_1..d_a and each other).  The round commits as the
+  linear round does; the next drafts come from the block of the outcome that happened.
+  (k+1)^2 rows per forward: quadratic in k.  See quadratic_layout.
 * Per-sequence (non-lockstep) diffusion: a sequence whose block completed runs its causal KV
   fill in its next step while the other sequences of the batch keep denoising; each step is
   one forward of k rows per sequence.  Sequences never see one another, so every sequence's
@@ -168,6 +174,70 @@ def selfspec_round(model, st: SeqState, k: int, forced: Optional[List[int]] = No
                  for b in range(len(st.lens))]
     apply_commit(st, committed)
     return committed, drafts, ver, dl, vl
+
+
+def quadratic_layout(n: int, k: int):
+    """Rows, positions and mask of the quadratic self-speculation forward at cached length n.
+
+    Rows 0..k are the verify rows V_i (inputs x_n, d_1..d_k at positions n..n+k, causal).
+    Then, for every acceptance outcome a = 0..k, a pre-draft block P_a of k rows: the mask id
+    at positions n+a+1 .. n+a+k.  P_a stands for the next round's draft block
+    [v_{a+1}, MASK x (k-1)] with v_{a+1} not yet known (it is being computed by V_a in the
+    same forward), so its first slot is a mask too.  P_a sees the cached prefix, the verify
+    rows V_0..V_a (the tokens x_n, d_1..d_a that outcome a keeps) and all of its own rows;
+    nothing else.  Returns (m, positions [m], mask [m, n+m])."""
+    m = (k + 1) + (k + 1) * k
+    pos = torch.empty(m, dtype=torch.int64)
+    mask = torch.zeros(m, n + m, dtype=torch.bool)
+    mask[:, :n] = True
+    for i in range(k + 1):
+        pos[i] = n + i
+        mask[i, n:n + i + 1] = True
+    for a in range(k + 1):
+        r0 = (k + 1) + a * k
+        pos[r0:r0 + k] = torch.arange(n + a + 1, n + a + 1 + k)
+        mask[r0:r0 + k, n:n + a + 1] = True
+        mask[r0:r0 + k, n + r0:n + r0 + k] = True
+    return m, pos, mask
+
+
+def quadratic_forward(model, st: SeqState, drafts: List[List[int]]):
+    """One forward of quadratic self-speculation: the verify rows of the current drafts and
+    the k+1 pre-draft blocks of the next round.  Writes the verify rows' KV at n..n+k (the
+    pre-draft rows' K/V are not kept); the LoRA drafter, if any, applies to the pre-draft
+    rows only.  Returns (verify logits [B, k+1, V], pre-draft logits [B, k+1, k, V])."""
+    B = len(st.lens)
+    k = len(drafts[0])
+    mask_id = model.cfg.mask_id
+    m = (k + 1) * (k + 1)
+    toks = torch.tensor([[st.pending[b]] + list(drafts[b]) + [mask_id] * ((k + 1) * k)
+                         for b in range(B)], dtype=torch.int64)
+    positions, masks = [], []
+    for b in range(B):
+        _, pos, mask = quadratic_layout(st.lens[b], k)
+        positions.append(pos)
+        masks.append(mask)
+    lora_rows = torch.zeros(B, m, dtype=torch.bool)
+    lora_rows[:, k + 1:] = True
+    logits = model.forward_rows(toks, torch.stack(positions), st.lens, st.cache, masks,
+                                write_kv_rows=k + 1, lora_rows=lora_rows)
+    V = logits.shape[-1]
+    return logits[:, :k + 1], logits[:, k + 1:].reshape(B, k + 1, k, V)
+
+
+def quadratic_round(model, st: SeqState, drafts: List[List[int]]):
+    """One quadratic round: verify the drafts and commit as in the linear round (greedy
+    longest matching prefix, 1..k+1 tokens); the next round's drafts are the argmaxes of the
+    pre-draft block of the outcome that happened.  Returns (committed, next drafts)."""
+    vl, pl = quadratic_forward(model, st, drafts)
+    ver = argmax_lowest(vl).tolist()
+    committed, nxt = [], []
+    for b in range(len(st.lens)):
+        c = commit_after_verify(drafts[b], ver[b])
+        committed.append(c)
+        nxt.append(argmax_lowest(pl[b, len(c) - 1]).tolist())
+    apply_commit(st, committed)
+    return committed, nxt
 
 
 def diffusion_forward(model, st: SeqState, k: int) -> torch.Tensor:
@@ -371,6 +441,25 @@ def selfspec_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, capaci
             out[b].extend(committed[b])
             per_round[b].append(len(committed[b]))
     return [o[:n_tokens] for o in out], per_round
+
+
+def quadratic_generate(model, prompt: torch.Tensor, n_tokens: int, k: int, capacity: int
+                       ) -> Tuple[List[List[int]], int, List[List[int]]]:
+    """Quadratic self-speculation: one diffusion draft forward to start, then one forward per
+    round.  Returns (tokens per sequence, forwards, commits per round per sequence)."""
+    st = prefill(model, prompt, capacity)
+    B = prompt.shape[0]
+    drafts = argmax_lowest(draft_forward(model, st, k)).tolist()
+    forwards = 1
+    out = [[] for _ in range(B)]
+    per_round = [[] for _ in range(B)]
+    while min(len(o) for o in out) < n_tokens:
+        committed, drafts = quadratic_round(model, st, drafts)
+        forwards += 1
+        for b in range(B):
+            out[b].extend(committed[b])
+            per_round[b].append(len(committed[b]))
+    return [o[:n_tokens] for o in out], forwards, per_round
 
 
 def diffuse_generate_fused(model, prompt: torch.Tensor, n_tokens: int, k: int, tau: float,

@@ -175,10 +175,38 @@ class OracleModel:
         """tokens [B, m] at positions starts[b]..starts[b]+m-1 over cached rows
         [0, starts[b]).  block_size 1 = causal; block_size m = one bidirectional block.
         write_kv stores this forward's K/V rows into the cache at their positions.
+        lora: the adapter (if set) applies to the rows that attend block-bidirectionally,
+        i.e. all rows but the leading causal_rows.
         Returns logits [B, m, V] (compute dtype) or None."""
+        B, m = tokens.shape
+        positions = torch.stack([torch.arange(int(starts[b]), int(starts[b]) + m) for b in range(B)])
+        masks = [block_mask(m, int(starts[b]), block_size, causal_rows) for b in range(B)]
+        lora_rows = None
+        if lora:
+            lora_rows = torch.zeros(B, m, dtype=torch.bool)
+            lora_rows[:, causal_rows:] = True
+        return self.forward_rows(tokens, positions, starts, cache, masks,
+                                 write_kv_rows=m if write_kv else 0, lora_rows=lora_rows,
+                                 layers=layers, with_logits=with_logits)
+
+    def forward_rows(self, tokens: torch.Tensor, positions: torch.Tensor, starts: List[int],
+                     cache, masks: List[torch.Tensor], write_kv_rows: int = 0,
+                     lora_rows: Optional[torch.Tensor] = None,
+                     layers: Optional[List[int]] = None,
+                     with_logits: bool = True) -> Optional[torch.Tensor]:
+        """The general forward: row r of sequence b has token tokens[b, r] at absolute
+        position positions[b, r] (RoPE); its keys are the cached rows [0, starts[b]) followed
+        by this forward's m rows, and masks[b] [m, starts[b]+m] says which it sees.  The
+        first write_kv_rows rows store their K/V into the cache at their positions (which
+        must be starts[b]+r).  lora_rows [B, m] (bool) picks the rows that take the adapter's
+        delta when one is set.  Returns logits [B, m, V] (compute dtype) or None."""
         c = self.cfg
         B, m = tokens.shape
         hd, Hq, Hkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+        for b in range(B):
+            n = int(starts[b])
+            assert masks[b].shape == (m, n + m)
+            assert all(int(positions[b, r]) == n + r for r in range(write_kv_rows))
         h = self._w(self.embed[tokens.long()])                # [B, m, d]
         for li in (range(c.n_layers) if layers is None else layers):
             L = self.layers[li]
@@ -188,28 +216,26 @@ class OracleModel:
             att = torch.empty(B, m, Hq, hd, dtype=self.cdt)
             for b in range(B):
                 n = int(starts[b])
-                pos = torch.arange(n, n + m)
+                pos = positions[b]
                 qb = self._store(rope_rotate(q[b], pos[:, None], c.rope_theta))   # [m, Hq, hd]
                 kb = self._store(rope_rotate(k[b], pos[:, None], c.rope_theta))   # [m, Hkv, hd]
                 vb = self._store(v[b])
                 Kc, Vc = cache[b][li]
                 keys = torch.cat([Kc[:, :n], kb.transpose(0, 1)], dim=1)          # [Hkv, n+m, hd]
                 vals = torch.cat([Vc[:, :n], vb.transpose(0, 1)], dim=1)
-                mask = block_mask(m, n, block_size, causal_rows)
-                o = attention_explicit(qb.transpose(0, 1), keys, vals, mask)      # [Hq, m, hd]
+                o = attention_explicit(qb.transpose(0, 1), keys, vals, masks[b])  # [Hq, m, hd]
                 att[b] = self._store(o.transpose(0, 1))
-                if write_kv:
-                    Kc[:, n:n + m] = kb.transpose(0, 1)
-                    Vc[:, n:n + m] = vb.transpose(0, 1)
+                w = write_kv_rows
+                if w:
+                    Kc[:, n:n + w] = kb[:w].transpose(0, 1)
+                    Vc[:, n:n + w] = vb[:w].transpose(0, 1)
             a2 = att.reshape(B, m, Hq * hd)
-            if lora and self.lora is not None:
-                # z = A att is stored like any activation; the delta joins the residual first.
-                # Only rows that attend block-bidirectionally are drafter rows: the leading
-                # causal rows (the fused KV fill) take the frozen path.
+            if lora_rows is not None and self.lora is not None:
+                # z = A att is stored like any activation; the delta joins the residual first,
+                # on the drafter rows only
                 LA, LB, sc = self.lora[0][li], self.lora[1][li], self.lora[2]
                 delta = sc * self._mm(self._store(self._mm(a2, LA)), LB)
-                delta[:, :causal_rows] = 0
-                h = h + delta
+                h = h + torch.where(lora_rows[..., None], delta, torch.zeros_like(delta))
             h = h + self._mm(a2, L["wo"])
             g = self._normed_mm(h, L["g2"], L["wg"])
             u = self._normed_mm(h, L["g2"], L["wu"])

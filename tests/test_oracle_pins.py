@@ -571,3 +571,103 @@ def test_nonlockstep_saves_forwards_when_progress_differs():
     assert nl_forwards < ls_forwards
     # the batch runs until its slowest sequence is done, give or take its last fill
     assert max(alone) - 1 <= nl_forwards <= max(alone) + 1
+
+
+# ------------------------------------------ quadratic self-speculation (next row f2) --
+
+def test_quadratic_layout_small_case_by_hand():
+    """n = 2 cached rows, k = 1: rows V0 (x_n at 2), V1 (d_1 at 3), P0 (mask at 3), P1 (mask
+    at 4); keys are the 2 cached rows then the 4 rows of the forward."""
+    m, pos, mask = odec.quadratic_layout(2, 1)
+    assert m == 4 and pos.tolist() == [2, 3, 3, 4]
+    T, F = True, False
+    want = [[T, T, T, F, F, F],     # V0: prefix, itself
+             [T, T, T, T, F, F],    # V1: prefix, V0, itself
+             [T, T, T, F, T, F],    # P0: prefix, V0 (outcome a = 0 keeps x_n), itself
+             [T, T, T, T, F, T]]    # P1: prefix, V0, V1, itself
+    assert mask.tolist() == want
+
+
+@pytest.mark.parametrize("k", [2, 4])
+def test_quadratic_layout_invariants(k):
+    n = 5
+    m, pos, mask = odec.quadratic_layout(n, k)
+    assert m == (k + 1) ** 2                    # quadratic in k
+    assert mask[:, :n].all()
+    assert torch.equal(mask[:k + 1, :n + k + 1], omod.causal_mask(k + 1, n))
+    assert not mask[:k + 1, n + k + 1:].any()   # verify rows never see a pre-draft row
+    for a in range(k + 1):
+        r0 = k + 1 + a * k
+        rows = mask[r0:r0 + k]
+        assert rows[:, n:n + a + 1].all() and not rows[:, n + a + 1:n + k + 1].any()
+        assert rows[:, n + r0:n + r0 + k].all()
+        assert rows[:, n + k + 1:].sum().item() == k * k     # no other block's rows
+        assert pos[r0:r0 + k].tolist() == list(range(n + a + 1, n + a + 1 + k))
+
+
+def test_quadratic_forward_equals_verify_and_separate_predrafts():
+    """The verify rows equal the linear verify forward (logits and KV rows), and pre-draft
+    block a equals a block forward of k masks at n+a+1 over the prefix extended by the causal
+    rows of x_n, d_1..d_a: the two constructions agree in fp64."""
+    import copy
+    cfg = _tiny(n_layers=2)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0), "f64")
+    A, B = _lora(cfg, 8, seed=3)
+    mdl.set_lora(A, B, 5.0)                     # the pre-draft rows are drafter rows
+    k = 3
+    st = odec.prefill(mdl, synth.prompt_tokens(2, 9, cfg.vocab, seed=2), 96)
+    drafts = [[5, 17, 3], [8, 8, 2]]
+    s_lin, s_quad = copy.deepcopy(st), copy.deepcopy(st)
+    vl = odec.verify_forward(mdl, s_lin, drafts)
+    ql, pl = odec.quadratic_forward(mdl, s_quad, drafts)
+    assert (ql - vl).abs().max().item() < 1e-10
+    for b in range(2):
+        n = st.lens[b]
+        for layer in range(cfg.n_layers):
+            for t in range(2):
+                x = s_lin.cache[b][layer][t][:, n:n + k + 1]
+                y = s_quad.cache[b][layer][t][:, n:n + k + 1]
+                assert (x - y).abs().max().item() < 1e-12
+    for a in range(k + 1):
+        sep = copy.deepcopy(st)
+        toks = torch.tensor([[sep.pending[b]] + drafts[b][:a] for b in range(2)], dtype=torch.int64)
+        mdl.forward(toks, sep.lens, sep.cache, block_size=1, write_kv=True, with_logits=False)
+        starts = [sep.lens[b] + a + 1 for b in range(2)]
+        masks = torch.full((2, k), cfg.mask_id, dtype=torch.int64)
+        want = mdl.forward(masks, starts, sep.cache, block_size=k, write_kv=False, lora=True)
+        assert (pl[:, a] - want).abs().max().item() < 1e-10
+
+
+@pytest.mark.parametrize("seed", [9, 4])
+def test_quadratic_generation_is_lossless_and_one_forward_per_round(seed):
+    cfg = _tiny(n_layers=1)
+    W = synth.model_weights(cfg, 5)
+    W[-1] = W[0][:cfg.vocab].clone() * 50.0      # peaky head tied to the embedding: drafts hit
+    mdl = oracle.OracleModel(cfg, W, "f64")
+    p = synth.prompt_tokens(2, 12, cfg.vocab, seed=seed)
+    k, n = 4, 24
+    got, forwards, per = odec.quadratic_generate(mdl, p, n, k, 128)
+    assert got == odec.ar_generate(mdl, p, n, 128)
+    rounds = len(per[0])
+    assert forwards == 1 + rounds
+    assert all(1 <= c <= k + 1 for row in per for c in row)
+    assert max(c for row in per for c in row) > 1        # multi-token commits happen
+
+
+def test_quadratic_round_picks_the_block_of_the_outcome():
+    """Drafts equal to the AR continuation are all accepted (k+1 commits) and the next drafts
+    come from block P_k; drafts that miss at once commit 1 token and use block P_0."""
+    import copy
+    cfg = _tiny(n_layers=1)
+    mdl = oracle.OracleModel(cfg, synth.model_weights(cfg, 0), "f64")
+    k = 3
+    p = synth.prompt_tokens(1, 10, cfg.vocab, seed=7)
+    cont = odec.ar_generate(mdl, p, k + 1, 64)[0]
+    st = odec.prefill(mdl, p, 64)
+    for drafts, a in (([cont[:k]], k), ([[(cont[0] + 1) % cfg.vocab] * k], 0)):
+        s1, s2 = copy.deepcopy(st), copy.deepcopy(st)
+        _, pl = odec.quadratic_forward(mdl, s1, drafts)
+        committed, nxt = odec.quadratic_round(mdl, s2, drafts)
+        assert committed[0] == cont[:a + 1]
+        assert nxt[0] == odec.argmax_lowest(pl[0, a]).tolist()
+        assert s2.lens[0] == st.lens[0] + a + 1 and s2.pending[0] == cont[a]
