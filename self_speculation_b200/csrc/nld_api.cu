@@ -811,14 +811,19 @@ nld_status nld_init_lora(nld_ctx* x, int rank, float scale, const void* const* t
   const size_t el = x->el;
   nld_status s;
   if (x->lora_A.empty()) {
-    x->lora_A.assign(L, nullptr);
-    x->lora_B.assign(L, nullptr);
+    // allocate into locals; the context takes them only when all succeeded (a failed first
+    // load leaves no half-made adapter behind; what was allocated is freed with the context)
+    std::vector<void*> A(L, nullptr), Bm(L, nullptr);
+    float* zp = nullptr;
     for (int l = 0; l < L; ++l) {
-      if ((s = dalloc(x, &x->lora_A[l], static_cast<size_t>(rank) * x->qd * el)) != NLD_OK) return s;
-      if ((s = dalloc(x, &x->lora_B[l], static_cast<size_t>(d) * rank * el)) != NLD_OK) return s;
+      if ((s = dalloc(x, &A[l], static_cast<size_t>(rank) * x->qd * el)) != NLD_OK) return s;
+      if ((s = dalloc(x, &Bm[l], static_cast<size_t>(d) * rank * el)) != NLD_OK) return s;
     }
-    const size_t zp = static_cast<size_t>(lora_n_ks(x->qd, x->bf16)) * x->M_max * rank;
-    if ((s = dalloc(x, &x->lora_zp, zp * sizeof(float))) != NLD_OK) return s;
+    const size_t nzp = static_cast<size_t>(lora_n_ks(x->qd, x->bf16)) * x->M_max * rank;
+    if ((s = dalloc(x, &zp, nzp * sizeof(float))) != NLD_OK) return s;
+    x->lora_A.swap(A);
+    x->lora_B.swap(Bm);
+    x->lora_zp = zp;
     x->lora_r_alloc = rank;
   }
   const cudaMemcpyKind kind = on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
@@ -1164,13 +1169,14 @@ nld_status run_nl(nld_ctx* x, bool fill_only, float threshold, int32_t* d_block_
 // only if some sequence is flagged.
 nld_status flush_nl(nld_ctx* x) {
   if (!x->nl_active) return NLD_OK;
-  x->nl_active = false;
   int* flags = x->h_pinned + 2 + x->batch;
   CK(cudaMemcpyAsync(flags, x->fillnext, sizeof(int) * x->batch, cudaMemcpyDeviceToHost, x->stream));
   CK(cudaStreamSynchronize(x->stream));
   bool any = false;
   for (int b = 0; b < x->batch; ++b) any = any || flags[b] != 0;
-  return any ? run_nl(x, true, 0.f, nullptr, nullptr, nullptr, nullptr) : NLD_OK;
+  if (any) TRY(run_nl(x, true, 0.f, nullptr, nullptr, nullptr, nullptr));
+  x->nl_active = false;   // only once the due fills ran: a failed flush is retried next call
+  return NLD_OK;
 }
 
 // A deferred fill (lockstep or per-sequence) runs alone before any other decode call.
