@@ -4,8 +4,11 @@
 // positions len..len+m-1 and are cut into blocks of `block_size` starting at len; a row sees
 // every cached key and every key of its own and earlier blocks: key j is visible to row p
 // iff j <= len + min(floor(p/bs)*bs + bs, m) - 1.  block_size 1 is strictly causal (verify,
-// AR, prefill, KV fill); block_size m is one bidirectional block (draft, diffusion).  The
-// mask is computed from these indices and never stored.
+// AR, prefill, KV fill); block_size m is one bidirectional block (draft, diffusion).  Two
+// extensions: the first causal_rows rows of every sequence are strictly causal and the blocks
+// start after them (the fused diffusion fill), and a per-sequence flag (causal_seq) makes all
+// rows of that sequence causal (per-sequence diffusion, where a sequence fills while the others
+// denoise).  The mask is computed from these indices and never stored.
 //
 // Tensor-core path (bf16, head_dim 128): one CTA per (KV split, kv head, sequence x query
 // tile).  Its rows are the G = Hq/Hkv query heads of that kv head times up to QT positions

@@ -1,7 +1,8 @@
 // Per-forward small kernels: embedding gather (builds each mode's input block on the device),
 // the finalize step after the LM head (argmax/confidence combine over vocab tiles and the
-// mode's state update: drafts, AR commit, greedy acceptance, diffusion commit, KV-fill and
-// prefill bookkeeping), weight repacking and fills.
+// mode's state update: drafts, AR commit, greedy acceptance, diffusion commit in lockstep,
+// fused or per-sequence form, KV-fill and prefill bookkeeping), the optional LoRA drafter's two
+// kernels, weight repacking and fills.
 #include <algorithm>
 #include <climits>
 
