@@ -241,6 +241,23 @@ nld_status nld_trace_chain(nld_ctx* ctx, int layer, int M, unsigned long long* d
  * k-iterations per split, CTAs, pipeline stages}.  No GPU work. */
 nld_status nld_debug_gemm_plan(nld_ctx* ctx, int which, int M, int* out8);
 
+/* Test hook, pure host (no CUDA call, no context): the plan of a projection chain of nph
+ * phases (1..4) over M token rows, phase p computing n_rows[p] outputs over K[p] inputs (a
+ * multiple of 64), given the clusters of each size that can be resident at once
+ * (max_clusters[cs] for cs = 1, 2, 4, 8; an occupancy query on the device).
+ * out20 = {cluster size, NT (token columns per tile), activation rows per k-tile box, k-tiles
+ * per stage, stages, split-K slots, TMEM columns, grid CTAs, shared-memory bytes, token
+ * tiles, then per phase p < 4: split s at 10+2p and k-tiles per split at 11+2p}.
+ * NLD_ERR_ARG on bad sizes, NLD_ERR_UNSUPPORTED if no cluster size can be resident. */
+nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const int* max_clusters,
+                          int* out20);
+
+/* Test hook, pure host: the attention launch plan for batch sequences of m rows, Hq/Hkv heads,
+ * keys up to max_len, on sms SMs.  out6 = {G = Hq/Hkv, query positions per CTA, query tiles,
+ * rows per CTA (positions x G), warps per CTA, KV splits (= cluster size)}.  NLD_ERR_ARG on
+ * bad sizes. */
+nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out6);
+
 /* Synchronise the context stream and report the device error word (then clear it):
  * NLD_OK, NLD_ERR_KV_FULL, NLD_ERR_TIMEOUT or NLD_ERR_DEVICE. */
 nld_status nld_sync(nld_ctx* ctx);

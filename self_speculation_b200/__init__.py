@@ -66,6 +66,9 @@ def load_library() -> ctypes.CDLL:
         "nld_time_gemm": ([P, I, I, I, I, ctypes.POINTER(F)], I),
         "nld_trace_gemm": ([P, I, I, I, P, ctypes.POINTER(I)], I),
         "nld_debug_gemm_plan": ([P, I, I, ctypes.POINTER(I)], I),
+        "nld_plan_chain": ([I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I),
+                            ctypes.POINTER(I)], I),
+        "nld_plan_attention": ([I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
         "nld_time_chain": ([P, I, I, I, ctypes.POINTER(F)], I),
         "nld_stream": ([P], P),

@@ -1398,6 +1398,49 @@ nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out)
   return NLD_OK;
 }
 
+nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const int* max_clusters,
+                          int* out20) {
+  if (!n_rows || !K || !max_clusters || !out20) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
+  if (M < 1 || nph < 1 || nph > kMaxPhases) return fail(nullptr, NLD_ERR_ARG, "bad plan sizes");
+  for (int p = 0; p < nph; ++p)
+    if (n_rows[p] < 1 || K[p] < kTileK || K[p] % kTileK)
+      return fail(nullptr, NLD_ERR_ARG, "phase %d: rows %d, K %d", p, n_rows[p], K[p]);
+  int grid = 0;
+  const ChainArgs A = plan_chain_shapes(max_clusters, n_rows, K, nph, M, &grid);
+  if (A.CS < 1) return fail(nullptr, NLD_ERR_UNSUPPORTED, "no cluster size can be resident");
+  for (int i = 0; i < 20; ++i) out20[i] = 0;
+  out20[0] = A.CS;
+  out20[1] = A.NT;
+  out20[2] = A.xr;
+  out20[3] = A.kps;
+  out20[4] = A.stages;
+  out20[5] = A.slots;
+  out20[6] = static_cast<int>(A.tmem_cols);
+  out20[7] = grid;
+  out20[8] = static_cast<int>(gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS, A.slots));
+  out20[9] = A.ph[0].tok_tiles;
+  for (int p = 0; p < nph; ++p) {
+    out20[10 + 2 * p] = A.ph[p].s;
+    out20[11 + 2 * p] = A.ph[p].ks;
+  }
+  return NLD_OK;
+}
+
+nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out6) {
+  if (!out6) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
+  if (batch < 1 || m < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_len < 1 || sms < 1)
+    return fail(nullptr, NLD_ERR_ARG, "bad attention plan sizes");
+  AttnArgs a{};
+  attn_plan(batch, m, Hq, Hkv, max_len, sms, a);
+  out6[0] = a.G;
+  out6[1] = a.QT;
+  out6[2] = a.q_tiles;
+  out6[3] = a.rows;
+  out6[4] = a.NW;
+  out6[5] = a.S;
+  return NLD_OK;
+}
+
 nld_status nld_debug_gemm_plan(nld_ctx* x, int which, int M, int* out8) {
   if (!x || !out8) return fail(x, NLD_ERR_ARG, "NULL argument");
   if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");

@@ -1,0 +1,142 @@
+"""Host logic of the launch planners, on CPU through the pure-host hooks nld_plan_chain and
+nld_plan_attention: every plan the library can make for the benchmark and test shapes keeps
+the kernels' limits (227 KB of shared memory, TMEM columns a power of two covering the
+double-buffered accumulator, split-K factors that give every rank work, <= 12 attention warps,
+<= 8 KV splits), and the plans at the benchmarked decode shape are the ones the committed
+launch list records (layer chain 132 CTAs in clusters of 4, layer-0 QKV 96 CTAs in clusters
+of 2, attention 7 x 8 CTAs of 288 / 256 threads in clusters of 7)."""
+import ctypes
+
+import pytest
+
+import self_speculation_b200 as nb
+import synth
+
+SMEM_BUDGET = 227 * 1024
+MAX_STAGES = 8
+# clusters of each size resident at once with one ~200 KB CTA per SM on 148 SMs (the device
+# reports these through an occupancy query; 33 clusters of 4 is the measured figure)
+B200_CLUSTERS = [0, 148, 74, 0, 33, 0, 0, 0, 16]
+
+
+def plan_chain(M, phases, clusters=B200_CLUSTERS):
+    lib = nb.load_library()
+    n = len(phases)
+    rows = (ctypes.c_int * n)(*[r for r, _ in phases])
+    K = (ctypes.c_int * n)(*[k for _, k in phases])
+    mc = (ctypes.c_int * 9)(*clusters)
+    out = (ctypes.c_int * 20)()
+    st = lib.nld_plan_chain(M, n, rows, K, mc, out)
+    assert st == 0, lib.nld_last_error(None)
+    o = list(out)
+    return dict(CS=o[0], NT=o[1], xr=o[2], kps=o[3], stages=o[4], slots=o[5], tmem=o[6],
+                grid=o[7], smem=o[8], tok_tiles=o[9],
+                split=[(o[10 + 2 * p], o[11 + 2 * p]) for p in range(n)])
+
+
+def plan_attention(batch, m, Hq, Hkv, max_len, sms=148):
+    lib = nb.load_library()
+    out = (ctypes.c_int * 6)()
+    assert lib.nld_plan_attention(batch, m, Hq, Hkv, max_len, sms, out) == 0
+    return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S"], list(out)))
+
+
+def chains(cfg):
+    """The projection chains of a forward: layer-0 QKV, a decode layer, the last layer with the
+    LM head, and the stand-alone LM head."""
+    qd, kvd, d, F, V = cfg.q_dim, cfg.kv_dim, cfg.d_model, cfg.ffn_dim, cfg.vocab
+    o, gu, dn, qkv, lm = (d, qd), (2 * F, d), (d, F), (qd + 2 * kvd, d), (V, d)
+    return {"qkv0": [qkv], "layer": [o, gu, dn, qkv], "last": [o, gu, dn, lm], "lm": [lm]}
+
+
+def decode_Ms(cfg):
+    k = cfg.block_k
+    Ms = {1, 2048}
+    for B in {1, 2, 4, cfg.max_batch}:
+        Ms |= {B, B * k, B * (k + 1), B * 2 * k}
+    return sorted(m for m in Ms if m <= max(2048, cfg.max_batch * (k + 1)))
+
+
+SHAPES = [("8b", synth.LLAMA8B.replace(max_batch=64)), ("14b", synth.LLAMA14B.replace(max_batch=64)),
+          ("small", synth.SMALL_BF16)]
+
+
+@pytest.mark.parametrize("name,cfg", SHAPES, ids=[s[0] for s in SHAPES])
+def test_chain_plans_keep_kernel_limits(name, cfg):
+    for M in decode_Ms(cfg):
+        for kind, phases in chains(cfg).items():
+            for clusters in (B200_CLUSTERS, [0, 100, 50, 0, 20, 0, 0, 0, 8]):
+                P = plan_chain(M, phases, clusters)
+                where = (name, kind, M, clusters[4])
+                assert P["smem"] <= SMEM_BUDGET, where
+                assert 2 <= P["stages"] <= MAX_STAGES and P["kps"] == 2, where
+                assert P["CS"] in (1, 2, 4, 8) and clusters[P["CS"]] >= 1, where
+                NT = P["NT"]
+                assert NT % 16 == 0 and 16 <= NT <= 256 and NT * P["tok_tiles"] >= M, where
+                assert P["xr"] % 8 == 0 and P["xr"] <= NT, where
+                if P["tok_tiles"] == 1:
+                    assert P["xr"] >= M, where
+                t = P["tmem"]
+                assert t & (t - 1) == 0 and 2 * NT <= t <= 512, where
+                assert P["grid"] % P["CS"] == 0 and P["grid"] <= P["CS"] * clusters[P["CS"]], where
+                if len(phases) > 1 and NT <= 64:
+                    assert P["CS"] == 4, where
+                for (rows, K), (s, ks) in zip(phases, P["split"]):
+                    KT = K // 64
+                    assert P["CS"] % s == 0 and s * ks >= KT and (s - 1) * ks < KT, where
+                if any(s > 1 for s, _ in P["split"]):
+                    assert P["slots"] >= NT // 16, where
+
+
+def test_decode_plans_match_the_recorded_launch_list():
+    cfg = synth.LLAMA8B
+    ch = chains(cfg)
+    for M, NT, xr in ((33, 48, 40), (32, 32, 32)):
+        P = plan_chain(M, ch["layer"])
+        assert (P["CS"], P["NT"], P["xr"], P["stages"], P["grid"]) == (4, NT, xr, 4, 132)
+        L = plan_chain(M, ch["last"])
+        assert (L["CS"], L["grid"]) == (4, 132)
+    Q = plan_chain(33, ch["qkv0"])
+    assert (Q["CS"], Q["grid"]) == (2, 96)
+
+
+@pytest.mark.parametrize("name,cfg", SHAPES, ids=[s[0] for s in SHAPES])
+def test_attention_plans_keep_kernel_limits(name, cfg):
+    for M in decode_Ms(cfg):
+        for B in {1, 4, cfg.max_batch}:
+            if M % B:
+                continue
+            m = M // B
+            if m > 2 * cfg.block_k + 1:
+                continue
+            for max_len in (m, 64, 900, 4096 + m, 32768):
+                A = plan_attention(B, m, cfg.n_q_heads, cfg.n_kv_heads, max_len)
+                where = (name, B, m, max_len)
+                assert A["G"] * cfg.n_kv_heads == cfg.n_q_heads, where
+                assert 1 <= A["QT"] <= m and A["QT"] * A["q_tiles"] >= m, where
+                assert A["rows"] == A["QT"] * A["G"] and A["rows"] <= 16 * A["NW"], where
+                assert 1 <= A["NW"] <= 12, where
+                assert 1 <= A["S"] <= 8, where
+                if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
+                    assert A["S"] == 1, where
+
+
+def test_attention_plan_of_the_benchmarked_round():
+    # verify forward (m = 33) and draft forward (m = 32) at ~865 keys: 7 x 8 CTAs in clusters of 7
+    v = plan_attention(1, 33, 32, 8, 865)
+    d = plan_attention(1, 32, 32, 8, 865)
+    assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"]) == (4, 33, 1, 9, 7)
+    assert (d["NW"], d["S"]) == (8, 7)
+
+
+def test_plan_hooks_reject_bad_sizes():
+    lib = nb.load_library()
+    out = (ctypes.c_int * 20)()
+    rows = (ctypes.c_int * 1)(4096)
+    bad_k = (ctypes.c_int * 1)(100)
+    mc = (ctypes.c_int * 9)(*B200_CLUSTERS)
+    assert lib.nld_plan_chain(33, 1, rows, bad_k, mc, out) == 1
+    assert lib.nld_plan_chain(0, 1, rows, (ctypes.c_int * 1)(4096), mc, out) == 1
+    none = (ctypes.c_int * 9)(*([0] * 9))
+    assert lib.nld_plan_chain(33, 1, rows, (ctypes.c_int * 1)(4096), none, out) == 8   # unsupported
+    assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 6)()) == 1
