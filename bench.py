@@ -555,6 +555,58 @@ def run_diffusion(args):
         "points": pts}), flush=True)
 
 
+def run_commit_sweep(args):
+    """8B-shaped commit-path sweep: after a draft+verify pair, nld_kv_commit with a forced count
+    c = 1..k+1 (random weights accept nothing on their own), timed alone with CUDA events on the
+    library stream.  The commit moves no KV row (the verify forward wrote rows n..n+k at their
+    final slots), so its time should not depend on c."""
+    import torch
+
+    import synth
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    reps = 5
+    cs = [1, 2, 4, 8, 16, 24, 32, 33]
+    cfg = synth.LLAMA8B.replace(max_seq=PROMPT + reps * (sum(cs) + 3 * 33) + 256)
+    ctx, stream = _model_ctx(cfg)
+    ctx.nld_prefill(synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1).cuda())
+    k = cfg.block_k
+    toks = torch.empty(1, k + 1, dtype=torch.int32, device="cuda")
+    nc = torch.empty(1, dtype=torch.int32, device="cuda")
+    force = torch.empty(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):                                   # warm-up: graphs captured
+        ctx.nld_selfspec_draft_verify()
+        force.fill_(1)
+        torch.cuda.synchronize()
+        ctx.nld_kv_commit(force, toks, nc)
+    ctx.nld_sync()
+    points = []
+    for c in cs:
+        force.fill_(c)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            ctx.nld_selfspec_draft_verify()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ctx.nld_kv_commit(force, toks, nc)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+            assert int(nc.item()) == c
+        points.append({"c": c, "us_median": round(sorted(ts)[len(ts) // 2], 2),
+                       "us_min": round(min(ts), 2)})
+    ctx.close()
+    print(json.dumps({
+        "metric": "commit-path time vs forced commit count, 8B shape, batch 1, k=32",
+        "unit": "us", "higher_is_better": False, "n_gpus": 1, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "8B-shaped nld_kv_commit after a draft+verify pair, forced c",
+                   "timing": "CUDA events on the library stream around the commit call only"},
+        "points": points}), flush=True)
+
+
 def run_sweep14b(args):
     """14B-shaped concurrency sweep: 40 layers, d 5120, 40/8 heads x 128, FFN 17408, vocab 151936;
     4k-token random prefixes; batch 1/4/16/64; AR step vs self-spec round (k=32) vs diffusion
@@ -679,7 +731,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a seeded random o_proj adapter in the draft forwards (0: none)")
-    ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b"],
+    ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b",
+                                           "commit8b"],
                     default="selfspec8b")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
@@ -695,6 +748,8 @@ def main():
         run_diffusion(args)
     elif args.workload == "sweep14b":
         run_sweep14b(args)
+    elif args.workload == "commit8b":
+        run_commit_sweep(args)
     elif args.impl == "reference":
         run_reference(args, world, rank, local)
     else:
