@@ -671,3 +671,23 @@ def test_quadratic_round_picks_the_block_of_the_outcome():
         assert committed[0] == cont[:a + 1]
         assert nxt[0] == odec.argmax_lowest(pl[0, a]).tolist()
         assert s2.lens[0] == st.lens[0] + a + 1 and s2.pending[0] == cont[a]
+
+
+def _golden_rows(name):
+    return [l.split() for l in open(os.path.join(GOLD, name))
+            if l.strip() and not l.startswith("#")]
+
+
+def test_fused_fill_mask_golden():
+    want = torch.tensor([[int(x) for x in r] for r in _golden_rows("mask_fill_n2_c2_bs2_m6.txt")],
+                        dtype=torch.bool)
+    assert torch.equal(omod.block_mask(6, 2, 2, causal_rows=2), want)
+
+
+def test_quadratic_layout_golden():
+    rows = _golden_rows("quadratic_n1_k2.txt")
+    assert rows[0][0] == "positions"
+    m, pos, mask = odec.quadratic_layout(1, 2)
+    assert pos.tolist() == [int(x) for x in rows[0][1:]]
+    want = torch.tensor([[int(x) for x in r] for r in rows[1:]], dtype=torch.bool)
+    assert m == 9 and torch.equal(mask, want)
