@@ -7,7 +7,8 @@ the oracle's per-sequence driver (itself pinned to every sequence's stand-alone 
 tests/test_oracle_pins.py), with the same per-step state of every sequence (open, completed,
 filled); a fill left due when AR decoding resumes runs first and the AR tokens match the
 oracle's.  bf16 small model, batch 4: a fill moves len by k and makes b_k pending, the others
-follow the commit rule on the GPU's own confidences.
+follow the commit rule on the GPU's own confidences.  This file is collected after the other
+GPU tests so that a failure here does not hide theirs.
 """
 import pytest
 import torch
