@@ -114,13 +114,25 @@ nld_status nld_init_weights(nld_ctx* ctx, const void* const* tensors, int n_tens
 nld_status nld_init_lora(nld_ctx* ctx, int rank, float scale, const void* const* tensors, int n_tensors,
                          int on_device);
 
-/* Start `batch` sequences from prompts d_tokens [batch, prompt_len] (device, int32).  Runs
- * causal forwards over positions 0..prompt_len-2 (writing those KV rows) and makes
- * prompt[prompt_len-1] the pending token, so len = prompt_len-1.  Resets drafts and
- * diffusion blocks.  1 <= batch <= max_batch, 1 <= prompt_len <= max_seq. */
-nld_status nld_prefill(nld_ctx* ctx, const int32_t* d_tokens, int batch, int prompt_len);
+/* Start `batch` sequences from their prompts (the clean prefix the AR pathway reads causally:
+ * ranhao.site notes section 5.1; r9-hu digest "Method", the cached clean prefix every later
+ * draft and verify forward attends to).
+ *   d_tokens       [batch, stride] int32 device, row b holding prompt b in its first lens[b]
+ *                  entries (the rest is ignored).
+ *   d_lens         [batch] int32 device prompt lengths, 1..stride; NULL = every prompt is
+ *                  `stride` long.  A length outside 1..stride is clamped and sets the device
+ *                  error word (NLD_ERR_DEVICE from nld_sync).
+ *   d_pending_out  [batch] int32 device or NULL: receives each sequence's pending token.
+ * Runs causal forwards over positions 0..stride-2 (rows at or past a shorter prompt's last
+ * position are padding whose KV rows lie past that sequence's length and are overwritten
+ * before any query sees them); then per sequence len = lens[b]-1 KV rows are cached and
+ * prompt[b][lens[b]-1] is the pending token.  Resets drafts and diffusion blocks.
+ * 1 <= batch <= max_batch, 1 <= stride <= max_seq. */
+nld_status nld_prefill(nld_ctx* ctx, const int32_t* d_tokens, int stride, const int32_t* d_lens,
+                       int batch, int32_t* d_pending_out);
 
-/* One AR step: causal one-token forward over the pending tokens; writes KV row len, then
+/* One AR step (ranhao.site notes section 5.1: left-to-right decoding with p(x_i | x_<i); greedy
+ * at temperature 0): causal one-token forward over the pending tokens; writes KV row len, then
  * len += 1 and the argmax (lowest id on ties) becomes the pending token, also written to
  * d_tokens_out [batch]. */
 nld_status nld_ar_step(nld_ctx* ctx, int32_t* d_tokens_out);
@@ -133,7 +145,11 @@ nld_status nld_ar_step(nld_ctx* ctx, int32_t* d_tokens_out);
  * Follow with nld_kv_commit. */
 nld_status nld_selfspec_draft_verify(nld_ctx* ctx);
 
-/* Commit path of a round (after nld_selfspec_draft_verify).  Per sequence b, c_b tokens
+/* Commit path of a round (after nld_selfspec_draft_verify): ranhao.site notes section 5.3 and
+ * the r9-hu digest "Method" (the longest prefix of drafts the verifier agrees with is accepted,
+ * stopping at the first mismatch; the round commits 1..k+1 tokens, the verifier's own token at
+ * the first mismatch included, and the KV rows of the committed tokens join the clean prefix).
+ * Per sequence b, c_b tokens
  * commit: with d_nrows == NULL, c_b = a_b + 1 where a_b is the number of leading i with
  * d_i == v_i (greedy longest matching prefix, warp-ballot computed); otherwise
  * c_b = d_nrows[b] (forced count, 1..k+1).  The committed tokens are d_1..d_{c-1}, v_c,
@@ -144,8 +160,12 @@ nld_status nld_selfspec_draft_verify(nld_ctx* ctx);
 nld_status nld_kv_commit(nld_ctx* ctx, const int32_t* d_nrows, int32_t* d_tokens_out,
                          int32_t* d_ncommit_out);
 
-/* One full round: nld_selfspec_draft_verify then nld_kv_commit(d_force_ncommit, ...),
- * replayed from one captured CUDA graph per batch size. d_force_ncommit may be NULL. */
+/* One full linear self-speculation round (r9-hu digest "Method", tri-mode inference; shilu.ai
+ * "Deploy and infer with SGLang": drafts from the diffusion pathway, verification by the AR
+ * pathway, lossless against AR at temperature 0): nld_selfspec_draft_verify then
+ * nld_kv_commit(d_force_ncommit, ...), replayed from one captured CUDA graph per (batch, output
+ * pointers).  d_force_ncommit may be NULL.  Outputs: d_tokens_out [batch, k+1] (the committed
+ * tokens, then -1), d_ncommit_out [batch] in 1..k+1. */
 nld_status nld_selfspec_round(nld_ctx* ctx, int32_t* d_tokens_out, int32_t* d_ncommit_out,
                               const int32_t* d_force_ncommit);
 
@@ -244,19 +264,35 @@ nld_status nld_debug_gemm_plan(nld_ctx* ctx, int which, int M, int* out8);
 /* Test hook, pure host (no CUDA call, no context): the plan of a projection chain of nph
  * phases (1..4) over M token rows, phase p computing n_rows[p] outputs over K[p] inputs (a
  * multiple of 64), given the clusters of each size that can be resident at once
- * (max_clusters[cs] for cs = 1, 2, 4, 8; an occupancy query on the device).
+ * (max_clusters[cs] for cs = 1, 2, 4, 8; an occupancy query on the device).  hilo = 1: the
+ * activations are (hi, lo) bf16 row pairs (the context's chains), 0: plain bf16 rows (the
+ * stand-alone LM head).
  * out20 = {cluster size, NT (token columns per tile), activation rows per k-tile box, k-tiles
  * per stage, stages, split-K slots, TMEM columns, grid CTAs, shared-memory bytes, token
  * tiles, then per phase p < 4: split s at 10+2p and k-tiles per split at 11+2p}.
  * NLD_ERR_ARG on bad sizes, NLD_ERR_UNSUPPORTED if no cluster size can be resident. */
 nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const int* max_clusters,
-                          int* out20);
+                          int hilo, int* out20);
 
 /* Test hook, pure host: the attention launch plan for batch sequences of m rows, Hq/Hkv heads,
  * keys up to max_len, on sms SMs.  out6 = {G = Hq/Hkv, query positions per CTA, query tiles,
  * rows per CTA (positions x G), warps per CTA, KV splits (= cluster size)}.  NLD_ERR_ARG on
  * bad sizes. */
 nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out6);
+
+/* Profiling hook: tuning of the projection chains' pipeline.  stage_cap = 0 lets the planner
+ * use as many shared-memory stages as fit, else at most stage_cap (3..8); k_tiles_per_stage =
+ * 1 or 2 weight boxes (16 KB each) per ring stage (0 = the planner's choice).  Synchronises and
+ * drops the captured graphs; later calls use the new values. */
+nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_stage);
+
+/* Test hook for failure detection: one launch of layer 0's four-phase chain over the current
+ * batch (scratch buffers only, as nld_time_chain) with every bounded wait limited to timeout_ns
+ * (1 us..2 s), in which CTA 0 withholds its arrival on the first phase counter, so every wait on
+ * that counter runs out.  Each CTA then lets its issued copies land, frees its tensor memory and
+ * exits; the device error word gets NLD_DEVERR_TIMEOUT, which the next nld_sync reports as
+ * NLD_ERR_TIMEOUT (and clears).  The context stays usable.  Returns after the launch. */
+nld_status nld_debug_timeout_chain(nld_ctx* ctx, unsigned long long timeout_ns);
 
 /* Synchronise the context stream and report the device error word (then clear it):
  * NLD_OK, NLD_ERR_KV_FULL, NLD_ERR_TIMEOUT or NLD_ERR_DEVICE. */
@@ -278,10 +314,12 @@ const char* nld_last_error(const nld_ctx* ctx);
  * 1 / sum_v exp(l_v - max).
  *   d_hidden     [M, d] bf16 row-major, 16-byte aligned; 1 <= M <= 4096, d a multiple of 128.
  *   d_lm_weight  [vocab, d] bf16 row-major (RMSNorm gain already folded in), 16-byte aligned.
- *   d_workspace  caller scratch of nld_lm_head_workspace_size() bytes, 256-byte aligned: per
- *                128-column tile RMS sums, then per (row, 128-row vocab tile) partials.
+ *   d_workspace  caller scratch of nld_lm_head_workspace_size() bytes, 256-byte aligned: a
+ *                256-byte block with the device error word, per 128-column tile RMS sums, then
+ *                per (row, 128-row vocab tile) partials.
  * Stream-ordered on `cuda_stream`; returns after the launches.  Calls sharing a workspace must
- * not overlap on the GPU.
+ * not overlap on the GPU.  If a bounded wait of the GEMM runs out (2 s), every row gets
+ * d_argmax_out = -1 and d_conf_out = 0 instead of results computed from unwritten partials.
  */
 size_t nld_lm_head_workspace_size(int M, int d, int vocab);
 nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int M, int d, int vocab,
@@ -296,10 +334,11 @@ nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int
  *   Same arguments, results and stream ordering as nld_lm_head_argmax, minus the workspace.
  *   Scratch: a fixed array built into the library (nld_lm_head_static_max_bytes() = 8 MiB per
  *   GPU, held from library load until process exit).  Shapes needing more scratch than that,
- *   M * (d/128 * 4 + ceil(vocab/128) * 16) bytes plus alignment, fail with NLD_ERR_ARG and
+ *   256 + M * (d/128 * 4 + ceil(vocab/128) * 16) bytes plus alignment, fail with NLD_ERR_ARG and
  *   launch nothing.  Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
- *   The first call on a device looks up the array's device address (cudaGetSymbolAddress);
- *   make that first call before any stream capture on that device.
+ *   Each call made outside stream capture looks up the array's device address
+ *   (cudaGetSymbolAddress); a call under capture reuses the last address found on that device,
+ *   so make one call on each device before capturing one.
  *   Every call shares the one array and leaves its contents behind (each call overwrites all
  *   it reads, so nothing needs clearing); calls that overlap on the GPU race on it.
  */

@@ -24,12 +24,11 @@ strictly causal mask.
 Precision modes
   "f64"    float64 everywhere (the reference semantics).
   "f32"    float32 everywhere.
-  "bf16io" float32 arithmetic with bf16 rounding where a bf16 library keeps activations in
-           storage: the matmul operand bf16(h), the stored q/k/v rows, the attention
-           output, the SwiGLU product.  The RMSNorm scale 1/rms is applied to the matmul
-           result instead of its operand (the same value in exact arithmetic, since the
-           norm scales each row by one number).  This is the rounding-matched mode the
-           tolerances of the bf16 parity tests are stated against.
+  "f32kv"  float32 everywhere, with a bf16 KV cache: the key and value rows are stored in a
+           bfloat16 cache and every attention reads them back from it (a forward's own rows
+           included).  Together with weights given as bf16 values this is the bf16
+           configuration as specified (bf16 weights and KV cache, fp32 accumulation and fp32
+           activations); the bf16 parity tests state their tolerances against it.
 """
 from __future__ import annotations
 
@@ -45,10 +44,6 @@ BF16 = 1
 def rmsnorm(x: torch.Tensor, eps: float) -> torch.Tensor:
     """x / sqrt(mean(x^2) + eps) over the last axis (no gain)."""
     return x / torch.sqrt((x * x).mean(dim=-1, keepdim=True) + eps)
-
-
-def inv_rms(x: torch.Tensor, eps: float) -> torch.Tensor:
-    return 1.0 / torch.sqrt((x * x).mean(dim=-1, keepdim=True) + eps)
 
 
 def rope_rotate(x: torch.Tensor, pos: torch.Tensor, theta: float) -> torch.Tensor:
@@ -113,16 +108,12 @@ def attention_explicit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return torch.matmul(p, vv)
 
 
-def _bf16(x: torch.Tensor) -> torch.Tensor:
-    return x.to(torch.bfloat16).to(x.dtype)
-
-
 class OracleModel:
     """Holds the weights (as given, bf16 or fp32 CPU tensors in the boundary's order) and
     runs forwards with an explicit KV cache [B][layer] -> (K [Hkv, cap, hd], V ...)."""
 
     def __init__(self, cfg, weights: List[Optional[torch.Tensor]], precision: str = "f64"):
-        assert precision in ("f64", "f32", "bf16io")
+        assert precision in ("f64", "f32", "f32kv")
         self.cfg = cfg
         self.precision = precision
         self.cdt = torch.float64 if precision == "f64" else torch.float32
@@ -152,19 +143,22 @@ class OracleModel:
         return torch.matmul(x, self._w(w).t())
 
     def _normed_mm(self, h: torch.Tensor, g: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
-        """(rmsnorm(h) * g) W^T, in the rounding of the precision mode."""
-        eps = self.cfg.rms_eps
-        if self.precision == "bf16io":
-            return self._mm(_bf16(h) * self._w(g), w) * inv_rms(h, eps)
-        return self._mm(rmsnorm(h, eps) * self._w(g), w)
+        """(rmsnorm(h) * g) W^T."""
+        return self._mm(rmsnorm(h, self.cfg.rms_eps) * self._w(g), w)
 
-    def _store(self, x: torch.Tensor) -> torch.Tensor:
-        return _bf16(x) if self.precision == "bf16io" else x
+    @property
+    def kv_dtype(self):
+        """Element type of the KV cache: bfloat16 in "f32kv", else the compute type."""
+        return torch.bfloat16 if self.precision == "f32kv" else self.cdt
+
+    def _kv(self, x: torch.Tensor) -> torch.Tensor:
+        """A key or value row as the cache holds it (stored in kv_dtype, read back)."""
+        return x.to(self.kv_dtype).to(self.cdt)
 
     def new_cache(self, batch: int, capacity: int):
         c = self.cfg
-        return [[(torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.cdt),
-                  torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.cdt))
+        return [[(torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.kv_dtype),
+                  torch.zeros(c.n_kv_heads, capacity, c.head_dim, dtype=self.kv_dtype))
                  for _ in range(c.n_layers)] for _ in range(batch)]
 
     # -- forward ------------------------------------------------------------------------
@@ -217,29 +211,28 @@ class OracleModel:
             for b in range(B):
                 n = int(starts[b])
                 pos = positions[b]
-                qb = self._store(rope_rotate(q[b], pos[:, None], c.rope_theta))   # [m, Hq, hd]
-                kb = self._store(rope_rotate(k[b], pos[:, None], c.rope_theta))   # [m, Hkv, hd]
-                vb = self._store(v[b])
+                qb = rope_rotate(q[b], pos[:, None], c.rope_theta)                # [m, Hq, hd]
+                kb = self._kv(rope_rotate(k[b], pos[:, None], c.rope_theta))      # [m, Hkv, hd]
+                vb = self._kv(v[b])
                 Kc, Vc = cache[b][li]
-                keys = torch.cat([Kc[:, :n], kb.transpose(0, 1)], dim=1)          # [Hkv, n+m, hd]
-                vals = torch.cat([Vc[:, :n], vb.transpose(0, 1)], dim=1)
+                keys = torch.cat([Kc[:, :n].to(self.cdt), kb.transpose(0, 1)], dim=1)   # [Hkv, n+m, hd]
+                vals = torch.cat([Vc[:, :n].to(self.cdt), vb.transpose(0, 1)], dim=1)
                 o = attention_explicit(qb.transpose(0, 1), keys, vals, masks[b])  # [Hq, m, hd]
-                att[b] = self._store(o.transpose(0, 1))
+                att[b] = o.transpose(0, 1)
                 w = write_kv_rows
                 if w:
-                    Kc[:, n:n + w] = kb[:w].transpose(0, 1)
-                    Vc[:, n:n + w] = vb[:w].transpose(0, 1)
+                    Kc[:, n:n + w] = kb[:w].transpose(0, 1).to(self.kv_dtype)
+                    Vc[:, n:n + w] = vb[:w].transpose(0, 1).to(self.kv_dtype)
             a2 = att.reshape(B, m, Hq * hd)
             if lora_rows is not None and self.lora is not None:
-                # z = A att is stored like any activation; the delta joins the residual first,
-                # on the drafter rows only
+                # the delta joins the residual first, on the drafter rows only
                 LA, LB, sc = self.lora[0][li], self.lora[1][li], self.lora[2]
-                delta = sc * self._mm(self._store(self._mm(a2, LA)), LB)
+                delta = sc * self._mm(self._mm(a2, LA), LB)
                 h = h + torch.where(lora_rows[..., None], delta, torch.zeros_like(delta))
             h = h + self._mm(a2, L["wo"])
             g = self._normed_mm(h, L["g2"], L["wg"])
             u = self._normed_mm(h, L["g2"], L["wu"])
-            act = self._store(g / (1.0 + torch.exp(-g)) * u)      # silu(g) * u
+            act = g / (1.0 + torch.exp(-g)) * u                     # silu(g) * u
             h = h + self._mm(act, L["wd"])
         if not with_logits:
             return None

@@ -52,7 +52,7 @@ def load_library() -> ctypes.CDLL:
         "nld_destroy": ([P], I),
         "nld_init_weights": ([P, ctypes.POINTER(P), I, I], I),
         "nld_init_lora": ([P, I, F, ctypes.POINTER(P), I, I], I),
-        "nld_prefill": ([P, P, I, I], I),
+        "nld_prefill": ([P, P, I, P, I, P], I),
         "nld_ar_step": ([P, P], I),
         "nld_selfspec_draft_verify": ([P], I),
         "nld_kv_commit": ([P, P, P, P], I),
@@ -66,11 +66,13 @@ def load_library() -> ctypes.CDLL:
         "nld_time_gemm": ([P, I, I, I, I, ctypes.POINTER(F)], I),
         "nld_trace_gemm": ([P, I, I, I, P, ctypes.POINTER(I)], I),
         "nld_debug_gemm_plan": ([P, I, I, ctypes.POINTER(I)], I),
-        "nld_plan_chain": ([I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I),
+        "nld_plan_chain": ([I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), I,
                             ctypes.POINTER(I)], I),
         "nld_plan_attention": ([I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
         "nld_time_chain": ([P, I, I, I, ctypes.POINTER(F)], I),
+        "nld_debug_chain_tuning": ([P, I, I], I),
+        "nld_debug_timeout_chain": ([P, ctypes.c_ulonglong], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
@@ -152,9 +154,12 @@ class Context:
         self._check(self.lib.nld_init_lora(self.h, rank, scale, arr if tensors else None,
                                            len(tensors), int(on_device)), self.h)
 
-    def nld_prefill(self, tokens) -> None:
+    def nld_prefill(self, tokens, lens=None, pending_out=None) -> None:
+        """tokens [B, stride] int32 (device); lens [B] int32 prompt lengths (None: all stride);
+        pending_out [B] int32 receives the pending tokens."""
         B, P = tokens.shape
-        self._check(self.lib.nld_prefill(self.h, _ptr(tokens), B, P), self.h)
+        self._check(self.lib.nld_prefill(self.h, _ptr(tokens), P, _ptr(lens), B, _ptr(pending_out)),
+                    self.h)
 
     def nld_ar_step(self, tokens_out) -> None:
         self._check(self.lib.nld_ar_step(self.h, _ptr(tokens_out)), self.h)
@@ -218,6 +223,13 @@ class Context:
         self._check(self.lib.nld_trace_chain(self.h, layer, M, _ptr(trace), ctypes.byref(g)), self.h)
         return g.value
 
+    def nld_debug_chain_tuning(self, stage_cap: int, k_tiles_per_stage: int = 0) -> None:
+        self._check(self.lib.nld_debug_chain_tuning(self.h, int(stage_cap), int(k_tiles_per_stage)),
+                    self.h)
+
+    def nld_debug_timeout_chain(self, timeout_ns: int) -> None:
+        self._check(self.lib.nld_debug_timeout_chain(self.h, int(timeout_ns)), self.h)
+
     def nld_debug_gemm_plan(self, which: int, M: int) -> dict:
         v = (ctypes.c_int * 8)()
         self._check(self.lib.nld_debug_gemm_plan(self.h, which, M, v), self.h)
@@ -246,13 +258,36 @@ def nld_lm_head_workspace_size(M: int, d: int, vocab: int) -> int:
     return load_library().nld_lm_head_workspace_size(M, d, vocab)
 
 
+def _current_stream(stream: Optional[int]) -> int:
+    """The caller's stream, else torch's current stream on the current device (not the legacy
+    default stream, so inputs produced on a side stream are ordered before the launches)."""
+    if stream is not None:
+        return stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _lm_head_args(hidden, lm_weight, argmax_out, conf_out):
+    import torch
+    for name, t, dt in (("hidden", hidden, torch.bfloat16), ("lm_weight", lm_weight, torch.bfloat16),
+                        ("argmax_out", argmax_out, torch.int32), ("conf_out", conf_out, torch.float32)):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == dt):
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    if hidden.dim() != 2 or lm_weight.dim() != 2 or lm_weight.shape[1] != hidden.shape[1]:
+        raise ValueError("hidden [M, d] and lm_weight [vocab, d] expected")
+    M = hidden.shape[0]
+    if argmax_out.numel() < M or conf_out.numel() < M:
+        raise ValueError(f"argmax_out and conf_out must hold at least M = {M} elements")
+    return M, hidden.shape[1], lm_weight.shape[0]
+
+
 def nld_lm_head_argmax(hidden, lm_weight, rms_eps: float, argmax_out, conf_out, workspace,
                        stream: Optional[int] = None) -> None:
     """hidden [M, d] bf16, lm_weight [vocab, d] bf16, argmax_out [M] int32, conf_out [M] fp32,
     workspace uint8 of nld_lm_head_workspace_size bytes."""
     lib = load_library()
-    M, d = hidden.shape
-    vocab = lm_weight.shape[0]
+    M, d, vocab = _lm_head_args(hidden, lm_weight, argmax_out, conf_out)
+    stream = _current_stream(stream)
     st = lib.nld_lm_head_argmax(_ptr(hidden), _ptr(lm_weight), M, d, vocab, float(rms_eps),
                                 _ptr(argmax_out), _ptr(conf_out), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), stream)
@@ -264,8 +299,8 @@ def nld_lm_head_argmax_static(hidden, lm_weight, rms_eps: float, argmax_out, con
                               stream: Optional[int] = None) -> None:
     """nld_lm_head_argmax with the library's built-in scratch (allocates nothing)."""
     lib = load_library()
-    M, d = hidden.shape
-    vocab = lm_weight.shape[0]
+    M, d, vocab = _lm_head_args(hidden, lm_weight, argmax_out, conf_out)
+    stream = _current_stream(stream)
     st = lib.nld_lm_head_argmax_static(_ptr(hidden), _ptr(lm_weight), M, d, vocab, float(rms_eps),
                                        _ptr(argmax_out), _ptr(conf_out), stream)
     if st != 0:

@@ -29,7 +29,7 @@ namespace {
 constexpr int kAttStages = 3;
 constexpr int kHalfTile = kPage * 64 * 2;        // 8 KB: 64 keys x 64 dims bf16
 constexpr int kKVTile = 2 * kHalfTile;           // 16 KB: 64 keys x 128 dims
-constexpr int kMaxAttWarps = 12;
+constexpr int kMaxAttWarps = 9;   // rows = positions x G <= 144 (the planner's query tile)
 
 NLD_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -52,6 +52,13 @@ NLD_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// The bf16 pair (x0, x1) as hi and lo halves: hi = bf16(x), lo = bf16(x - hi).
+NLD_DEV void pack_bf16_hilo(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
 // Byte offset of 16-byte chunk `c` (0..15) of `row` in a [rows][128 dims] bf16 tile stored as
 // two TMA boxes of 64 dims with 128-byte swizzle.
 NLD_DEV uint32_t kv_off(int row, int c) {
@@ -68,6 +75,12 @@ NLD_DEV int vis_end_of(int len, int p, int bs, int m, int c) {
 
 }  // namespace
 
+// kHiLo (the model's forwards): q arrives in fp32 and is split into bf16 hi and lo halves, the
+// probabilities P likewise, and S = (Q_hi + Q_lo) K^T, O = (P_hi + P_lo) V take two MMAs each,
+// so only the bf16 K/V cache rounds; the output is written as (hi, lo) bf16 row pairs, the
+// operand layout of the O projection.  Otherwise (the stand-alone entry point) q and the output
+// are plain bf16 and P is rounded to bf16 for its MMA.
+template <bool kHiLo>
 __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -76,7 +89,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   uint8_t* sK = smem;
   uint8_t* sV = smem + kAttStages * kKVTile;
   uint8_t* sQ = smem + 2 * kAttStages * kKVTile;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sQ + a.NW * 16 * 256);
+  uint8_t* sQl = sQ + a.NW * 16 * 256;           // lo halves of Q (kHiLo)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sQ + (kHiLo ? 2 : 1) * a.NW * 16 * 256);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -141,25 +155,33 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   for (int e = tid; e < rows_pad * 16; e += nthr) {
     const int r = e >> 4, c = e & 15;
     const int p = r / a.G, gq = r - p * a.G;
-    uint4 val = make_uint4(0, 0, 0, 0);
+    uint4 val = make_uint4(0, 0, 0, 0), vlo = make_uint4(0, 0, 0, 0);
     if (r < a.rows && p < np) {
       const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
-      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.q) +
-                                 ((tok * a.Hq) + g * a.G + gq) * 128 + c * 8;
-      val = *reinterpret_cast<const uint4*>(src);
+      const size_t off = ((tok * a.Hq) + g * a.G + gq) * 128 + c * 8;
+      if constexpr (kHiLo) {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
+        const float4 x0 = src[0], x1 = src[1];
+        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        split8(xs, val, vlo);
+      } else {
+        val = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+      }
     }
     *reinterpret_cast<uint4*>(sQ + r * 256 + ((c ^ (r & 7)) << 4)) = val;
+    if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQl + r * 256 + ((c ^ (r & 7)) << 4)) = vlo;
   }
   __syncthreads();
 
-  // Q fragments for the warp's 16 rows, all 8 k-steps of head_dim 128
+  // Q fragments for the warp's 16 rows, all 8 k-steps of head_dim 128 (the lo halves are
+  // read from shared memory per k-step inside the tile loop)
   uint32_t qf[8][4];
+  const int qr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
   {
-    const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const int c = 2 * kk + (lane >> 4);
-      ldsm_x4(smem_u32(sQ + r * 256 + ((c ^ (r & 7)) << 4)), qf[kk][0], qf[kk][1], qf[kk][2],
+      ldsm_x4(smem_u32(sQ + qr * 256 + ((c ^ (qr & 7)) << 4)), qf[kk][0], qf[kk][1], qf[kk][2],
               qf[kk][3]);
     }
   }
@@ -196,6 +218,12 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
     for (int kk2 = 0; kk2 < 4; ++kk2) {
+      uint32_t ql0[4], ql1[4];
+      if constexpr (kHiLo) {
+        const int c0 = 4 * kk2 + (lane >> 4), c1 = c0 + 2;
+        ldsm_x4(smem_u32(sQl + qr * 256 + ((c0 ^ (qr & 7)) << 4)), ql0[0], ql0[1], ql0[2], ql0[3]);
+        ldsm_x4(smem_u32(sQl + qr * 256 + ((c1 ^ (qr & 7)) << 4)), ql1[0], ql1[1], ql1[2], ql1[3]);
+      }
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int key = nt * 8 + (lane & 7);
@@ -204,6 +232,10 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
         ldsm_x4(kb + kv_off(key, c), b0, b1, b2, b3);
         mma_bf16_16816(sc[nt], qf[2 * kk2], b0, b1);
         mma_bf16_16816(sc[nt], qf[2 * kk2 + 1], b2, b3);
+        if constexpr (kHiLo) {
+          mma_bf16_16816(sc[nt], ql0, b0, b1);
+          mma_bf16_16816(sc[nt], ql1, b2, b3);
+        }
       }
     }
     // scale, mask, online softmax (log2 domain)
@@ -255,11 +287,18 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     // O += P V
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16(sc[2 * j][0], sc[2 * j][1]);
-      pa[1] = pack_bf16(sc[2 * j][2], sc[2 * j][3]);
-      pa[2] = pack_bf16(sc[2 * j + 1][0], sc[2 * j + 1][1]);
-      pa[3] = pack_bf16(sc[2 * j + 1][2], sc[2 * j + 1][3]);
+      uint32_t pa[4], pl[4];
+      if constexpr (kHiLo) {
+        pack_bf16_hilo(sc[2 * j][0], sc[2 * j][1], pa[0], pl[0]);
+        pack_bf16_hilo(sc[2 * j][2], sc[2 * j][3], pa[1], pl[1]);
+        pack_bf16_hilo(sc[2 * j + 1][0], sc[2 * j + 1][1], pa[2], pl[2]);
+        pack_bf16_hilo(sc[2 * j + 1][2], sc[2 * j + 1][3], pa[3], pl[3]);
+      } else {
+        pa[0] = pack_bf16(sc[2 * j][0], sc[2 * j][1]);
+        pa[1] = pack_bf16(sc[2 * j][2], sc[2 * j][3]);
+        pa[2] = pack_bf16(sc[2 * j + 1][0], sc[2 * j + 1][1]);
+        pa[3] = pack_bf16(sc[2 * j + 1][2], sc[2 * j + 1][3]);
+      }
       const int key = 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
@@ -268,6 +307,10 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
         ldsm_x4_t(vb + kv_off(key, c), b0, b1, b2, b3);
         mma_bf16_16816(o[2 * p], pa, b0, b1);
         mma_bf16_16816(o[2 * p + 1], pa, b2, b3);
+        if constexpr (kHiLo) {
+          mma_bf16_16816(o[2 * p], pl, b0, b1);
+          mma_bf16_16816(o[2 * p + 1], pl, b2, b3);
+        }
       }
     }
     __syncthreads();
@@ -280,25 +323,34 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
 
-  auto out_ptr = [&](int r) -> __nv_bfloat16* {
+  // output row r of this CTA (part 1: the lo row of a (hi, lo) pair)
+  auto out_ptr = [&](int r, int part) -> __nv_bfloat16* {
     const int p = r / a.G, gq = r - p * a.G;
     const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
-    return static_cast<__nv_bfloat16*>(a.out) + ((tok * a.Hq) + g * a.G + gq) * 128;
+    const size_t orow = kHiLo ? 2 * tok + part : tok;
+    return static_cast<__nv_bfloat16*>(a.out) + ((orow * a.Hq) + g * a.G + gq) * 128;
+  };
+  // store the pair (x0, x1) at column d of output row r
+  auto store2 = [&](int r, int d, float x0, float x1) {
+    if constexpr (kHiLo) {
+      uint32_t hi, lo;
+      pack_bf16_hilo(x0, x1, hi, lo);
+      *reinterpret_cast<uint32_t*>(out_ptr(r, 0) + d) = hi;
+      *reinterpret_cast<uint32_t*>(out_ptr(r, 1) + d) = lo;
+    } else {
+      *reinterpret_cast<uint32_t*>(out_ptr(r, 0) + d) = pack_bf16(x0, x1);
+    }
   };
 
   if (a.S == 1) {
     const float ia = (l_a > 0.f) ? 1.f / l_a : 0.f, ib = (l_b > 0.f) ? 1.f / l_b : 0.f;
     if (vis_a >= 0) {
-      __nv_bfloat16* dst = out_ptr(ra);
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
-        *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * (lane & 3)) = pack_bf16(o[n][0] * ia, o[n][1] * ia);
+      for (int n = 0; n < 16; ++n) store2(ra, n * 8 + 2 * (lane & 3), o[n][0] * ia, o[n][1] * ia);
     }
     if (vis_b >= 0) {
-      __nv_bfloat16* dst = out_ptr(rb);
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
-        *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * (lane & 3)) = pack_bf16(o[n][2] * ib, o[n][3] * ib);
+      for (int n = 0; n < 16; ++n) store2(rb, n * 8 + 2 * (lane & 3), o[n][2] * ib, o[n][3] * ib);
     }
     return;
   }
@@ -360,9 +412,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
       }
     }
     const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    __nv_bfloat16* dst = out_ptr(r) + d4 * 4;
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc.x * inv, acc.y * inv);
-    *reinterpret_cast<uint32_t*>(dst + 2) = pack_bf16(acc.z * inv, acc.w * inv);
+    store2(r, d4 * 4, acc.x * inv, acc.y * inv);
+    store2(r, d4 * 4 + 2, acc.z * inv, acc.w * inv);
   }
   cluster_sync();   // peers may still be reading this CTA's shared memory
 }
@@ -443,13 +494,17 @@ cudaError_t init_kernel_attributes() {
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
   cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel)) != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel<false>)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(attn_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - static_cast<int>(fa.sharedSizeBytes))) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel<true>)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
-size_t attn_mma_smem_bytes(int NW) {
-  return 1024 + 2 * kAttStages * kKVTile + static_cast<size_t>(NW) * 16 * 256 +
+size_t attn_mma_smem_bytes(int NW, bool hilo) {
+  return 1024 + 2 * kAttStages * kKVTile + static_cast<size_t>(hilo ? 2 : 1) * NW * 16 * 256 +
          kAttStages * sizeof(uint64_t);
 }
 
@@ -459,7 +514,7 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
   cfg.blockDim = dim3(32 * a.NW);
-  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW);
+  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW, a.hilo != 0);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -474,7 +529,8 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   if (pdl) attrs[na++] = attr[0];
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_mma_kernel, *tmKV, a);
+  if (a.hilo) return cudaLaunchKernelEx(&cfg, attn_mma_kernel<true>, *tmKV, a);
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<false>, *tmKV, a);
 }
 
 cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,

@@ -286,6 +286,28 @@ NLD_DEV float from_f32<float>(float x) { return x; }
 template <>
 NLD_DEV __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// hi/lo split of an fp32 value into two bf16 numbers: hi = bf16(x), lo = bf16(x - hi).  hi + lo
+// carries 16 significand bits (relative error <= 2^-17), so a tensor-core product summed over
+// the two halves equals the fp32-operand product to that precision.
+NLD_DEV void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+// Eight fp32 values as two 16-byte pieces of bf16: their hi halves and their lo halves.
+NLD_DEV void split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(x[2 * q], h0, l0);
+    split_bf16(x[2 * q + 1], h1, l1);
+    h[q] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+    l[q] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 NLD_DEV void set_err(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }

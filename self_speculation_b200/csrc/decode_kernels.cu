@@ -27,7 +27,13 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
   const int b = t / a.m, i = t - b * a.m;
   int id;
   switch (a.mode) {
-    case FWD_PREFILL: id = a.prompt[static_cast<size_t>(b) * a.prompt_len + a.chunk0 + i]; break;
+    case FWD_PREFILL:
+      // rows at or past the sequence's own last prompt position are padding of a ragged batch
+      // (their KV rows lie past its length and are overwritten before any query sees them)
+      id = (a.plens && a.chunk0 + i >= a.plens[b] - 1)
+               ? 0
+               : a.prompt[static_cast<size_t>(b) * a.prompt_len + a.chunk0 + i];
+      break;
     case FWD_AR: id = a.pending[b]; break;
     case FWD_DRAFT: id = (i == 0) ? a.pending[b] : a.V; break;
     case FWD_VERIFY: id = (i == 0) ? a.pending[b] : a.draft[b * a.k + i - 1]; break;
@@ -42,7 +48,9 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
   }
   const T* row = static_cast<const T*>(a.E) + static_cast<size_t>(id) * a.d;
   float* h = a.h + static_cast<size_t>(t) * a.d;
-  T* hb = static_cast<T*>(a.hb) + static_cast<size_t>(t) * a.d;
+  // bf16 operands: the (hi, lo) row pair of token t; an embedding row is exact in bf16, so lo = 0
+  const bool hl = (sizeof(T) == 2) && a.hilo;
+  T* hb = static_cast<T*>(a.hb) + static_cast<size_t>(hl ? 2 * t : t) * a.d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = a.d / kTileRows;
   for (int tile = warp; tile < ntiles; tile += 8) {
@@ -53,6 +61,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
       const float v = to_f32<T>(row[c]);
       h[c] = v;
       hb[c] = row[c];
+      if (hl) hb[a.d + c] = from_f32<T>(0.f);
       sq += v * v;
     }
 #pragma unroll
@@ -277,8 +286,20 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
     } break;
     case FWD_PREFILL: {
       if (lane == 0) {
-        a.lens[b] += a.chunk;
-        if (a.prompt) a.pending[b] = a.prompt[static_cast<size_t>(b) * a.prompt_len + a.prompt_len - 1];
+        if (a.prompt) {
+          // last chunk: the sequence's own length and pending token
+          int plen = a.plens ? a.plens[b] : a.prompt_len;
+          if (plen < 1 || plen > a.prompt_len) {
+            set_err(a.err, NLD_DEVERR_TOKEN);
+            plen = max(1, min(plen, a.prompt_len));
+          }
+          const int tok = a.prompt[static_cast<size_t>(b) * a.prompt_len + plen - 1];
+          a.lens[b] = plen - 1;
+          a.pending[b] = tok;
+          if (a.pending_out) a.pending_out[b] = tok;
+        } else {
+          a.lens[b] += a.chunk;
+        }
       }
     } break;
     default:
@@ -313,17 +334,18 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 constexpr int kLoraJ = 16, kLoraT = 32, kLoraThreads = 256;
 template <typename T> struct LoraCols { static constexpr int n = 512 / sizeof(T); };
 
-template <typename T>
+template <typename T, bool kHiLo>
 __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, const T* att, float* zp,
                                                                  int M, int qd, int r) {
   constexpr int C = LoraCols<T>::n, LD = C + 2, V = 16 / sizeof(T);
+  constexpr int kXRows = kHiLo ? 2 * kLoraT : kLoraT;   // with hi/lo: rows 2t, 2t+1 per token
   __shared__ __align__(16) T sA[kLoraJ][LD];
-  __shared__ __align__(16) T sX[kLoraT][LD];
+  __shared__ __align__(16) T sX[kXRows][LD];
   pdl_wait();
   pdl_launch_dependents();
   const int j0 = blockIdx.x * kLoraJ, c0 = blockIdx.y * C, t0 = blockIdx.z * kLoraT;
-  // stage: 16 + 32 rows of C/V vectors; out-of-range rows and columns read as zero
-  constexpr int kVecRow = C / V, kVecs = (kLoraJ + kLoraT) * kVecRow;
+  // stage: 16 + 32 (64 with hi/lo) rows of C/V vectors; out-of-range rows and columns read as zero
+  constexpr int kVecRow = C / V, kVecs = (kLoraJ + kXRows) * kVecRow;
   uint4 v[(kVecs + kLoraThreads - 1) / kLoraThreads];
 #pragma unroll
   for (int u = 0; u < (kVecs + kLoraThreads - 1) / kLoraThreads; ++u) {
@@ -333,8 +355,10 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
     if (e < kVecs && c < qd) {
       if (row < kLoraJ) {
         if (j0 + row < r) v[u] = *reinterpret_cast<const uint4*>(A + static_cast<size_t>(j0 + row) * qd + c);
-      } else if (t0 + row - kLoraJ < M) {
-        v[u] = *reinterpret_cast<const uint4*>(att + static_cast<size_t>(t0 + row - kLoraJ) * qd + c);
+      } else if (((row - kLoraJ) >> (kHiLo ? 1 : 0)) + t0 < M) {
+        // att row index: token t0 + i (plain) or row 2 t0 + i of the (hi, lo) pairs
+        const size_t arow = (kHiLo ? 2 * static_cast<size_t>(t0) : static_cast<size_t>(t0)) + (row - kLoraJ);
+        v[u] = *reinterpret_cast<const uint4*>(att + arow * qd + c);
       }
     }
   }
@@ -357,7 +381,14 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
   for (int c = 0; c < C; c += 2) {
     float x0, x1, p0, p1, q0, q1;
     if constexpr (sizeof(T) == 2) {
-      const float2 xx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sX[lane][c]));
+      float2 xx;
+      if constexpr (kHiLo) {
+        const float2 xh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sX[2 * lane][c]));
+        const float2 xl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sX[2 * lane + 1][c]));
+        xx = make_float2(xh.x + xl.x, xh.y + xl.y);
+      } else {
+        xx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sX[lane][c]));
+      }
       const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sA[2 * w][c]));
       const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sA[2 * w + 1][c]));
       x0 = xx.x; x1 = xx.y; p0 = pp.x; p1 = pp.y; q0 = qq.x; q1 = qq.y;
@@ -386,7 +417,7 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
 // shared memory.  Rows t with t mod m < causal_rows (the fused fill's causal rows) and the
 // rows of sequences flagged in causal_seq (a per-sequence fill) are not drafter rows and keep h
 // unchanged.
-template <typename T>
+template <typename T, bool kHiLo>
 __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* zp, float* h, int M,
                                                       int d, int r, int n_ks, float scale, int m,
                                                       int causal_rows, const int* causal_seq) {
@@ -414,7 +445,7 @@ __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* z
 #pragma unroll
   for (int q = 0; q < kQ; ++q) {
     const int e = q * 128 + threadIdx.x;
-    if (e < 8 * r) s_z[e / r][e % r] = to_f32<T>(from_f32<T>(za[q]));   // rows >= nt: zero
+    if (e < 8 * r) s_z[e / r][e % r] = kHiLo ? za[q] : to_f32<T>(from_f32<T>(za[q]));   // rows >= nt: zero
   }
   __syncthreads();
   if (i >= d) return;
@@ -459,7 +490,7 @@ int lora_n_ks(int qd, bool bf16) {
 
 cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
-                        const int* causal_seq, bool bf16, bool pdl) {
+                        const int* causal_seq, bool bf16, bool hilo, bool pdl) {
   if (r < 8 || r > 256 || r % 8 || M < 1) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -475,18 +506,25 @@ cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const voi
   c2.gridDim = dim3((d + 127) / 128, (M + 7) / 8);
   c2.blockDim = dim3(128);
   cudaError_t e;
-  if (bf16) {
+  if (bf16 && hilo) {
     using T = __nv_bfloat16;
-    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T>, static_cast<const T*>(A), static_cast<const T*>(att), zp,
-                           M, qd, r);
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T, true>, static_cast<const T*>(A), static_cast<const T*>(att),
+                           zp, M, qd, r);
     if (e == cudaSuccess)
-      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T>, static_cast<const T*>(B), static_cast<const float*>(zp),
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T, true>, static_cast<const T*>(B), static_cast<const float*>(zp),
+                             h, M, d, r, n_ks, scale, m, causal_rows, causal_seq);
+  } else if (bf16) {
+    using T = __nv_bfloat16;
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<T, false>, static_cast<const T*>(A), static_cast<const T*>(att),
+                           zp, M, qd, r);
+    if (e == cudaSuccess)
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<T, false>, static_cast<const T*>(B), static_cast<const float*>(zp),
                              h, M, d, r, n_ks, scale, m, causal_rows, causal_seq);
   } else {
-    e = cudaLaunchKernelEx(&c1, lora_down_kernel<float>, static_cast<const float*>(A),
+    e = cudaLaunchKernelEx(&c1, lora_down_kernel<float, false>, static_cast<const float*>(A),
                            static_cast<const float*>(att), zp, M, qd, r);
     if (e == cudaSuccess)
-      e = cudaLaunchKernelEx(&c2, lora_up_kernel<float>, static_cast<const float*>(B),
+      e = cudaLaunchKernelEx(&c2, lora_up_kernel<float, false>, static_cast<const float*>(B),
                              static_cast<const float*>(zp), h, M, d, r, n_ks, scale, m, causal_rows,
                              causal_seq);
   }
@@ -550,8 +588,9 @@ cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int
 // ----------------------------------------------------------- stand-alone LM-head helpers --
 // ssq[t * M + row] = sum over columns 128t..128t+127 of h[row, c]^2 (fp32), one warp per tile.
 __global__ void __launch_bounds__(256) rms_stats_kernel(const __nv_bfloat16* __restrict__ h, int M,
-                                                        int d, float* __restrict__ ssq) {
+                                                        int d, float* __restrict__ ssq, int* err) {
   const int row = blockIdx.x;
+  if (row == 0 && threadIdx.x == 0) *err = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const __nv_bfloat16* hr = h + static_cast<size_t>(row) * d;
   for (int t = warp; t < d / kTileRows; t += 8) {
@@ -567,8 +606,8 @@ __global__ void __launch_bounds__(256) rms_stats_kernel(const __nv_bfloat16* __r
   }
 }
 
-cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq) {
-  rms_stats_kernel<<<M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), M, d, ssq);
+cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq, int* err) {
+  rms_stats_kernel<<<M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), M, d, ssq, err);
   return cudaGetLastError();
 }
 
@@ -576,10 +615,17 @@ cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float
 // the confidence is its inverse (largest softmax probability).
 __global__ void __launch_bounds__(256) lm_combine_kernel(const LmPart* __restrict__ part, int M,
                                                          int tiles, int* __restrict__ argmax,
-                                                         float* __restrict__ conf) {
+                                                         float* __restrict__ conf, const int* err) {
   const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= M) return;
+  if (*err) {   // a wait of the LM-head GEMM ran out: its partials are incomplete
+    if (lane == 0) {
+      argmax[tok] = -1;
+      conf[tok] = 0.f;
+    }
+    return;
+  }
   const LmPart* row = part + static_cast<size_t>(tok) * tiles;
   float mx = -INFINITY;
   int ix = INT_MAX;
@@ -610,8 +656,8 @@ __global__ void __launch_bounds__(256) lm_combine_kernel(const LmPart* __restric
 }
 
 cudaError_t launch_lm_combine(cudaStream_t st, const LmPart* part, int M, int tiles, int* argmax,
-                              float* conf) {
-  lm_combine_kernel<<<(M + 7) / 8, 256, 0, st>>>(part, M, tiles, argmax, conf);
+                              float* conf, const int* err) {
+  lm_combine_kernel<<<(M + 7) / 8, 256, 0, st>>>(part, M, tiles, argmax, conf, err);
   return cudaGetLastError();
 }
 

@@ -64,14 +64,54 @@ NLD_DEV void epi_preload(const EpiArgs& e, int row_tile, int row_in_tile, int to
   }
 }
 
+// Eight fp32 values as one 16-byte piece of bf16 (round to nearest even).
+NLD_DEV uint4 pack8_bf16(const float* x) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+    w[q] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Store of one bf16 activation value: with hi/lo operands (hl) the row pair (2 tok, 2 tok + 1)
+// of a [2 M, ld] buffer receives bf16(x) and bf16(x - bf16(x)); otherwise row tok of [M, ld].
+template <typename T>
+NLD_DEV void store_act(void* buf, bool hl, int tok, int ld, int col, float x) {
+  if (hl) {
+    __nv_bfloat16 hi, lo;
+    split_bf16(x, hi, lo);
+    __nv_bfloat16* b = static_cast<__nv_bfloat16*>(buf);
+    b[static_cast<size_t>(2 * tok) * ld + col] = hi;
+    b[static_cast<size_t>(2 * tok + 1) * ld + col] = lo;
+  } else {
+    static_cast<T*>(buf)[static_cast<size_t>(tok) * ld + col] = from_f32<T>(x);
+  }
+}
+// Same for eight consecutive values (one 16-byte piece per stored row; bf16 storage only).
+NLD_DEV void store_act8(void* buf, bool hl, int tok, int ld, int col, const float* x) {
+  __nv_bfloat16* b = static_cast<__nv_bfloat16*>(buf);
+  if (hl) {
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4*>(b + static_cast<size_t>(2 * tok) * ld + col) = hi;
+    *reinterpret_cast<uint4*>(b + static_cast<size_t>(2 * tok + 1) * ld + col) = lo;
+  } else {
+    *reinterpret_cast<uint4*>(b + static_cast<size_t>(tok) * ld + col) = pack8_bf16(x);
+  }
+}
+
 // Every per-column loop below runs stage by stage over all 16 columns (all loads, then all
 // multiplies, then all shuffles of one butterfly level, ...): a column-at-a-time loop is a
 // chain of dependent shared-memory and shuffle latencies 16 times over (~1.3-2 us per chunk
 // measured), while the stage-wise form keeps 16 independent operations in flight.
 //
-// Vector stores (xbuf != nullptr, bf16 outputs, 128-row tiles aligned to heads): the 128
-// threads first write the chunk transposed, [16 tokens][row], into xbuf (16 x 132 floats,
-// private to these 4 warps), then each thread stores whole 16-byte pieces of token rows.
+// Vector stores (xbuf != nullptr, bf16 storage, 128-row tiles aligned to heads): the 128
+// threads first write the chunk's fp32 outputs transposed, [16 tokens][row], into xbuf (16 x
+// 132 floats, private to these 4 warps), then each thread stores whole 16-byte pieces of token
+// rows.  With hi/lo activations (e.hilo) the bf16 activation outputs (hb, u) are written as
+// row pairs (hi, lo) and q is kept in fp32.
 template <typename T>
 NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane, int ew,
                        int tok0, const float* s_inv, const int* s_pos, const int* s_pg, int col0,
@@ -80,6 +120,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
   const int row = row_tile * kTileRows + row_in_tile;
   constexpr int kXld = 132;   // floats per token row of xbuf
   const bool vec = (xbuf != nullptr) && sizeof(T) == 2;
+  const bool hl = (sizeof(T) == 2) && e.hilo;
   switch (e.kind) {
     case EPI_QKV: {
       int sec, head, lr, feat;
@@ -99,18 +140,32 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         }
       }
       if (vec && e.hd == kTileRows) {
-        // one tile = one head of q, k or v: the token's 128 features are one 256-byte row
-        __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(xbuf);
+        // one tile = one head of q, k or v: the token's 128 features are one row of xbuf
 #pragma unroll
-        for (int j = 0; j < 16; ++j) xb[j * (2 * kXld) + feat] = __float2bfloat16_rn(x[j]);
+        for (int j = 0; j < 16; ++j) xbuf[j * kXld + feat] = x[j];
         named_bar_sync(bar_id, 128);
+        if (row_tile * kTileRows >= e.n_rows) break;
+        if (sec == 0 && hl) {
+          // q in fp32: 16 tokens x 32 pieces of 4 floats
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int idx = row_in_tile + 128 * q;
+            const int j = idx >> 5, c4 = idx & 31;
+            const int tok = tok0 + j;
+            if (tok < e.M)
+              *reinterpret_cast<float4*>(static_cast<float*>(e.q_out) +
+                                         (static_cast<size_t>(tok) * e.Hq + head) * e.hd + c4 * 4) =
+                  *reinterpret_cast<const float4*>(xbuf + j * kXld + c4 * 4);
+          }
+          break;
+        }
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int idx = row_in_tile + 128 * q;
           const int j = idx >> 4, c8 = idx & 15;
           const int tok = tok0 + j;
-          if (tok >= e.M || row_tile * kTileRows >= e.n_rows) continue;
-          const uint4 val = *reinterpret_cast<const uint4*>(xb + j * (2 * kXld) + c8 * 8);
+          if (tok >= e.M) continue;
+          const uint4 val = pack8_bf16(xbuf + j * kXld + c8 * 8);
           if (sec == 0) {
             *reinterpret_cast<uint4*>(static_cast<T*>(e.q_out) +
                                       (static_cast<size_t>(tok) * e.Hq + head) * e.hd + c8 * 8) = val;
@@ -130,8 +185,11 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         const int tok = tok0 + j;
         if (tok >= e.M || row >= e.n_rows) continue;
         if (sec == 0) {
-          static_cast<T*>(e.q_out)[(static_cast<size_t>(tok) * e.Hq + head) * e.hd + feat] =
-              from_f32<T>(x[j]);
+          const size_t qi = (static_cast<size_t>(tok) * e.Hq + head) * e.hd + feat;
+          if (hl)
+            static_cast<float*>(e.q_out)[qi] = x[j];
+          else
+            static_cast<T*>(e.q_out)[qi] = from_f32<T>(x[j]);
         } else {
           const int pos = s_pos[col0 + j];
           if (pos < 0) continue;
@@ -154,7 +212,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
           xbuf[j * kXld + row_in_tile] = hn[j];
         } else {
           e.h[static_cast<size_t>(tok0 + j) * e.d + row] = hn[j];
-          static_cast<T*>(e.hb)[static_cast<size_t>(tok0 + j) * e.d + row] = from_f32<T>(hn[j]);
+          store_act<T>(e.hb, hl, tok0 + j, e.d, row, hn[j]);
         }
       }
 #pragma unroll
@@ -178,7 +236,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         }
       }
       if (vec && row_tile * kTileRows < e.n_rows) {
-        // h: 16 tokens x 128 fp32 = 512 16-byte pieces; hb: 256 pieces of 8 bf16
+        // h: 16 tokens x 128 fp32 = 512 16-byte pieces; hb: 256 pieces of 8 bf16 per stored row
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int idx = row_in_tile + 128 * q;
@@ -191,19 +249,8 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
         for (int q = 0; q < 2; ++q) {
           const int idx = row_in_tile + 128 * q;
           const int j = idx >> 4, c8 = idx & 15;
-          if (tok0 + j < e.M) {
-            const float4 a = *reinterpret_cast<const float4*>(xbuf + j * kXld + c8 * 8);
-            const float4 b = *reinterpret_cast<const float4*>(xbuf + j * kXld + c8 * 8 + 4);
-            __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
-            __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-            uint4 o;
-            o.x = *reinterpret_cast<uint32_t*>(&p0);
-            o.y = *reinterpret_cast<uint32_t*>(&p1);
-            o.z = *reinterpret_cast<uint32_t*>(&p2);
-            o.w = *reinterpret_cast<uint32_t*>(&p3);
-            *reinterpret_cast<uint4*>(static_cast<T*>(e.hb) + static_cast<size_t>(tok0 + j) * e.d +
-                                      row_tile * kTileRows + c8 * 8) = o;
-          }
+          if (tok0 + j < e.M)
+            store_act8(e.hb, hl, tok0 + j, e.d, row_tile * kTileRows + c8 * 8, xbuf + j * kXld + c8 * 8);
         }
       }
       named_bar_sync(bar_id, 128);
@@ -221,24 +268,21 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
 #pragma unroll
       for (int j = 0; j < 16; ++j) x[j] = __fdividef(x[j], 1.0f + __expf(-x[j])) * pt[j];   // silu(g) * u
       if (vec) {
-        // 16 tokens x 64 outputs of bf16: one 16-byte piece per thread
-        __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(xbuf);
+        // 16 tokens x 64 outputs: one 16-byte piece (per stored row) per thread
         if (!(lane & 1)) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) xb[j * (2 * kXld) + (row_in_tile >> 1)] = __float2bfloat16_rn(x[j]);
+          for (int j = 0; j < 16; ++j) xbuf[j * kXld + (row_in_tile >> 1)] = x[j];
         }
         named_bar_sync(bar_id, 128);
         const int j = row_in_tile >> 3, c8 = row_in_tile & 7;
         if (tok0 + j < e.M && row_tile * kTileRows < e.n_rows)
-          *reinterpret_cast<uint4*>(static_cast<T*>(e.u_out) + static_cast<size_t>(tok0 + j) * e.F +
-                                    row_tile * (kTileRows / 2) + c8 * 8) =
-              *reinterpret_cast<const uint4*>(xb + j * (2 * kXld) + c8 * 8);
+          store_act8(e.u_out, hl, tok0 + j, e.F, row_tile * (kTileRows / 2) + c8 * 8, xbuf + j * kXld + c8 * 8);
         break;
       }
       if (!(lane & 1)) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          if (tok0 + j < e.M) static_cast<T*>(e.u_out)[static_cast<size_t>(tok0 + j) * e.F + f] = from_f32<T>(x[j]);
+          if (tok0 + j < e.M) store_act<T>(e.u_out, hl, tok0 + j, e.F, f, x[j]);
       }
     } break;
 

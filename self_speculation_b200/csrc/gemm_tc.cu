@@ -5,6 +5,10 @@
 //
 // Swap-AB: the weight matrix W [n_rows, K] is the MMA's M=128 operand and the few token rows
 // X [M, K] are its N operand (N = 16..256), so a decode forward streams every weight byte once.
+// Activations are fp32 values held as two bf16 rows each (hi = bf16(x), lo = bf16(x - hi),
+// interleaved: row 2t, 2t+1 for token t), so one MMA of N = 2 x tokens multiplies both halves by
+// the same weights and the epilogue adds column pairs: the product has the precision of fp32
+// operands against bf16 weights (the stand-alone LM head over caller bf16 rows uses N = tokens).
 // Weights are stored pre-tiled (128 x 64 blocks, 16 KB contiguous), so each TMA box is one
 // contiguous read and a CTA's K range is one contiguous stretch of HBM.  A pipeline stage holds
 // two k-tiles (32 KB of weights plus the activation rows), so one producer -> MMA -> producer
@@ -120,6 +124,24 @@ NLD_DEV void trace_iter(const ChainArgs& A, int kind, int it) {
     A.trace[148 * 16 + kind * 64 + it] = globaltimer_ns();
 }
 
+// The accumulator of chunk c (16 tokens) of a tile.  With hi/lo activations (rows 2t, 2t+1 =
+// bf16(x_t), bf16(x_t - bf16(x_t))) columns 2t and 2t+1 hold W x_hi and W x_lo of token t, and
+// their sum is W x_t to fp32-operand precision.
+NLD_DEV void tmem_ld_chunk(uint32_t tbase, int c, int hilo, float (&v)[16]) {
+  if (!hilo) {
+    tmem_ld16(tbase + c * 16, v);
+    return;
+  }
+  float a[16], b[16];
+  tmem_ld16(tbase + c * 32, a);
+  tmem_ld16(tbase + c * 32 + 16, b);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[j] = a[2 * j] + a[2 * j + 1];
+    v[8 + j] = b[2 * j] + b[2 * j + 1];
+  }
+}
+
 NLD_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, GemmTail* tail,
                            int* err) {
   if (tail->abort_flag) return false;
@@ -153,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int S = A.stages;
   const int NT = A.NT;
+  const int NN = NT << A.hilo;         // MMA N: activation rows of a token tile (hi/lo pairs)
   const int KPS = A.kps;
   const int xbytes = A.xr * 128;       // one k-tile of activations: xr token rows x 128 B
   const int wst = KPS * kStageW;       // one stage: KPS k-tiles of weights ...
@@ -219,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = l2_policy_evict_first();
       int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages], q_nk[kMaxStages];
       int it = 0;
+      int n_issued = 0;   // stages whose loads were issued
       bool ok = true;
       for (int p = 0; ok && p < A.nph; ++p) {
         const PhaseArgs& P = A.ph[p];
@@ -259,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < nq; ++i)
             for (int j = 0; j < q_nk[i]; ++j)
               tma_load_2d(sX + q_stage[i] * xst + j * xbytes, &P.tmX, &tail->full[q_stage[i]],
-                          (q_k[i] + j) * kTileK, q_tt[i] * NT);
+                          (q_k[i] + j) * kTileK, q_tt[i] * NN);
           nq = 0;
           ready = true;
           return true;
@@ -290,10 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d_hint(sW + stage * wst + j * kStageW, &P.tmW, &tail->full[stage], 0,
                                  (r * P.KT + kt + j) * kTileRows, pol);
             }
+            n_issued = it + 1;
             if (ready) {
               for (int j = 0; j < nk; ++j)
                 tma_load_2d(sX + stage * xst + j * xbytes, &P.tmX, &tail->full[stage],
-                            (kt + j) * kTileK, tt * NT);
+                            (kt + j) * kTileK, tt * NN);
             } else {
               q_stage[nq] = stage;
               q_k[nq] = kt;
@@ -325,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // let every load already issued land before the CTA can exit
-        const int first = it - S > 0 ? it - S : 0;
-        for (int j = first; j < it; ++j)
+        const int first = n_issued - S > 0 ? n_issued - S : 0;
+        for (int j = first; j < n_issued; ++j)
           mbar_wait(&tail->full[j % S], static_cast<uint32_t>(j / S) & 1u, timeout_ns);
       }
     }
@@ -334,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer --
-      const uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, NN);
       int it = 0, i = 0;
       bool ok = true;
       for (int p = 0; ok && p < A.nph; ++p) {
@@ -458,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             EpiPre pre;
             epi_preload(e, r, row_in_tile, tok0 + c * 16, tail->pos, c * 16, pre);
             float v[16];
-            tmem_ld16(tbase + c * 16, v);
+            tmem_ld_chunk(tbase, c, A.hilo, v);
             epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
                          c * 16, v, pre, red_f, red_i, hbar);
           }
@@ -468,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 2. partial -> owners (own chunks by plain stores)
           for (int c = half; c < nchunks; c += 2) {
             float v[16];
-            tmem_ld16(tbase + c * 16, v);
+            tmem_ld_chunk(tbase, c, A.hilo, v);
             const int o = c / per;
             const uint32_t off = static_cast<uint32_t>(((w.grank * per + (c - o * per)) * kTileRows + row_in_tile) * kSlotLd) * 4u;
             if (o == w.grank) {
@@ -541,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this CTA's outputs of phase p are written: after the barrier one thread publishes
         // them (its gpu-scope fence covers the stores the barrier ordered before it) and arrives
         named_bar_sync(1, kEpiThreads);
-        if (et == 0) {
+        if (et == 0 && !(A.dbg_skip_arrive && blockIdx.x == 0 && p == 0)) {
           __threadfence();
           fence_proxy_async_global();
           red_add_release_gpu(A.bar + p, 1u);

@@ -26,7 +26,7 @@
 using namespace nld;
 
 namespace nld {
-size_t attn_mma_smem_bytes(int NW);
+size_t attn_mma_smem_bytes(int NW, bool hilo);
 cudaError_t init_kernel_attributes();
 }
 
@@ -108,6 +108,7 @@ struct nld_ctx {
   // device state
   int *lens = nullptr, *pending = nullptr, *draft = nullptr, *verify = nullptr, *blk = nullptr;
   int *incomplete = nullptr, *err = nullptr, *prompt = nullptr;
+  int* plens = nullptr;      // prompt length of each sequence (ragged prefill)
   int* fillnext = nullptr;   // per-sequence diffusion: block complete, causal fill due next step
   // activations
   float* h = nullptr;
@@ -128,8 +129,17 @@ struct nld_ctx {
   CUtensorMap tmWlm{};
   CUtensorMap tmKV{};
   std::map<std::pair<int, int>, CUtensorMap> tmX;
-  // graphs
-  std::map<std::vector<uintptr_t>, cudaGraphExec_t> graphs;
+  // graphs: one per (call, batch, output pointers), at most kMaxGraphs (least recently used
+  // evicted); tick = the call count at each graph's last replay
+  struct GraphEntry {
+    cudaGraphExec_t exec;
+    unsigned long long tick;
+  };
+  std::map<std::vector<uintptr_t>, GraphEntry> graphs;
+  unsigned long long graph_tick = 0;
+  // chain tuning (profiling hook): stage cap (0 = as many as fit), k-tiles per stage
+  int chain_stage_cap = 0;
+  int chain_kps = 0;   // k-tiles per stage (0 = the planner's choice)
   // host-side sequence bookkeeping
   int batch = 0;
   bool started = false;
@@ -224,7 +234,8 @@ const CUtensorMap* xmap(nld_ctx* x, int buf, int rows) {
   CUtensorMap m;
   const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
   const int inner = buf == XB_HB ? x->c.d_model : (buf == XB_ATTN ? x->qd : x->c.ffn_dim);
-  if (!make_map_bf16(&m, base, inner, x->M_max, rows)) return nullptr;
+  // bf16 activations are (hi, lo) row pairs: 2 M_max rows
+  if (!make_map_bf16(&m, base, inner, 2ull * x->M_max, rows)) return nullptr;
   return &(x->tmX[key] = m);
 }
 
@@ -252,11 +263,13 @@ WInfo winfo(nld_ctx* x, int which, int layer) {
 // divisor of CS) minimises waves x (k-iterations per tile + the cross-rank handoff of a split
 // tile, which measures at about six k-iterations) over the clusters that can be resident.
 ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const int* K, int nph, int M,
-                            int* grid_out) {
+                            int hilo, int* grid_out, int stage_cap = 0, int kps_force = 0) {
   ChainArgs best{};
   long long best_cost = -1;
   int best_grid = 0;
-  const int tok_tiles = (M + kMaxNT - 1) / kMaxNT;
+  // with hi/lo activation rows a token takes two MMA columns: at most 128 tokens per tile
+  const int max_tok = hilo ? kMaxNT / 2 : kMaxNT;
+  const int tok_tiles = (M + max_tok - 1) / max_tok;
   const int per = (M + tok_tiles - 1) / tok_tiles;
   const int NT = std::max(16, (per + 15) / 16 * 16);
   int cands[4] = {1, 2, 4, 8};
@@ -309,24 +322,34 @@ ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const in
   // activations: the token tile's rows rounded up to 8 (a multiple of the 128-byte swizzle
   // atom's 8 rows), so a decode tile of 33 tokens moves 40 rows per k-tile, not NT = 48
   // (several token tiles: every tile but the last is full, so all NT rows)
-  best.xr = (tok_tiles == 1) ? std::min(NT, (M + 7) / 8 * 8) : NT;
+  best.hilo = hilo ? 1 : 0;
+  const int NN = NT << best.hilo;
+  best.xr = (tok_tiles == 1) ? std::min(NN, ((M << best.hilo) + 7) / 8 * 8) : NN;
   // two k-tiles (32 KB of weights) per stage: the producer/MMA barrier round trip, not HBM,
   // bounds a ring of 16 KB stages; as many stages as fit the shared-memory budget
-  best.kps = 2;
   best.slots = 0;
   for (int p = 0; p < nph; ++p)
     if (best.ph[p].s > 1) {
       const int nch = NT / 16, s = best.ph[p].s;
       best.slots = std::max(best.slots, s * ((nch + s - 1) / s));
     }
-  best.stages = 2;
-  for (int st = gemm_chain_max_stages(); st > 2; --st)
-    if (gemm_chain_smem_bytes(NT, best.xr, best.kps, st, best.CS, best.slots) <= kChainSmemBudget) {
-      best.stages = st;
-      break;
-    }
+  // ring: two k-tiles (32 KB of weights) per stage, so one producer/MMA barrier round trip moves
+  // 32 KB, with as many stages as fit the shared-memory budget; when wide activation boxes leave
+  // room for fewer than three such stages, one k-tile per stage (more, smaller stages)
+  const int st_max = stage_cap > 0 ? std::min(stage_cap, gemm_chain_max_stages()) : gemm_chain_max_stages();
+  auto fit = [&](int kps) {
+    for (int st = st_max; st > 2; --st)
+      if (gemm_chain_smem_bytes(NT, best.xr, kps, st, best.CS, best.slots) <= kChainSmemBudget) return st;
+    return 2;
+  };
+  best.kps = (kps_force > 0) ? kps_force : 2;
+  best.stages = fit(best.kps);
+  if (kps_force <= 0 && best.stages < 3) {
+    best.kps = 1;
+    best.stages = fit(1);
+  }
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * NT)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(2 * NN)) cols <<= 1;
   best.tmem_cols = cols;
   if (grid_out) *grid_out = best_grid;
   return best;
@@ -339,7 +362,8 @@ ChainArgs plan_chain(nld_ctx* x, const ProjRef* pr, int nph, int M, int* grid_ou
     nr[p] = w.n_rows;
     kd[p] = w.K;
   }
-  return plan_chain_shapes(x->max_clusters, nr, kd, nph, M, grid_out);
+  return plan_chain_shapes(x->max_clusters, nr, kd, nph, M, x->bf16 ? 1 : 0, grid_out, x->chain_stage_cap,
+                           x->chain_kps);
 }
 
 // Launch a chain of projections (the SIMT kernel one by one for the fp32 configuration).
@@ -432,6 +456,7 @@ EpiArgs base_epi(nld_ctx* x, int M, int m) {
   e.lm_tiles = x->lm_tiles;
   e.V = x->c.vocab;
   e.q_out = x->qbuf;
+  e.hilo = x->bf16 ? 1 : 0;
   e.err = x->err;
   return e;
 }
@@ -465,11 +490,13 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   ea.prompt = x->prompt;
   ea.prompt_len = f.prompt_len;
   ea.chunk0 = f.chunk0;
+  ea.plens = (f.mode == FWD_PREFILL) ? x->plens : nullptr;
   ea.lens = x->lens;
   ea.h = x->h;
   ea.hb = x->hb;
   ea.ssq = x->ssq;
   ea.ssq_ld = x->M_max;
+  ea.hilo = x->bf16 ? 1 : 0;
   ea.err = x->err;
   CK(launch_embed(x->stream, ea, M, x->bf16, pdl));
 
@@ -489,6 +516,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.causal_seq = f.causal_seq;
   aa.err = x->err;
   aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
+  aa.hilo = x->bf16 ? 1 : 0;
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa);
   } else {
@@ -537,7 +565,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
                           f.mode == FWD_NLDIFF))
       CK(launch_lora(x->stream, x->lora_A[l], x->lora_B[l], x->attn, x->lora_zp, x->h, M, x->qd,
                      x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, f.causal_seq,
-                     x->bf16, pdl));
+                     x->bf16, x->bf16, pdl));
     int n = layer_chain(l, cur);
     int nn = 0;
     if (l + 1 < L) {
@@ -580,11 +608,28 @@ nld_status finalize(nld_ctx* x, const FinalizeArgs& a) {
   return NLD_OK;
 }
 
-// Capture `body` into a graph keyed by `key` on first use, then replay it.
+constexpr size_t kMaxGraphs = 64;
+
+void drop_graphs(nld_ctx* x) {
+  for (auto& kv : x->graphs) cudaGraphExecDestroy(kv.second.exec);
+  x->graphs.clear();
+}
+
+// Capture `body` into a graph keyed by `key` on first use, then replay it.  A caller that keeps
+// passing fresh output buffers makes new keys: past kMaxGraphs graphs the least recently
+// replayed one is destroyed (after the stream drains, so no replay of it is in flight).
 template <typename F>
 nld_status run_graph(nld_ctx* x, const std::vector<uintptr_t>& key, F body) {
   auto it = x->graphs.find(key);
   if (it == x->graphs.end()) {
+    if (x->graphs.size() >= kMaxGraphs) {
+      auto victim = x->graphs.begin();
+      for (auto g = x->graphs.begin(); g != x->graphs.end(); ++g)
+        if (g->second.tick < victim->second.tick) victim = g;
+      CK(cudaStreamSynchronize(x->stream));
+      cudaGraphExecDestroy(victim->second.exec);
+      x->graphs.erase(victim);
+    }
     cudaGraph_t g = nullptr;
     CK(cudaStreamBeginCapture(x->stream, cudaStreamCaptureModeThreadLocal));
     nld_status s = body();
@@ -599,9 +644,10 @@ nld_status run_graph(nld_ctx* x, const std::vector<uintptr_t>& key, F body) {
     ce = cudaGraphInstantiate(&ex, g, 0);
     cudaGraphDestroy(g);
     if (ce != cudaSuccess) return fail(x, NLD_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(ce));
-    it = x->graphs.emplace(key, ex).first;
+    it = x->graphs.emplace(key, nld_ctx::GraphEntry{ex, 0}).first;
   }
-  CK(cudaGraphLaunch(it->second, x->stream));
+  it->second.tick = ++x->graph_tick;
+  CK(cudaGraphLaunch(it->second.exec, x->stream));
   return NLD_OK;
 }
 
@@ -737,13 +783,17 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
   if ((s = dalloc(x, &x->incomplete, 16)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->err, 16)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->prompt, static_cast<size_t>(B) * c.max_seq * sizeof(int))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->plens, B * sizeof(int))) != NLD_OK) return bail(s);
   const size_t Mm = x->M_max;
   if ((s = dalloc(x, &x->h, Mm * d * sizeof(float))) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->hb, Mm * d * el)) != NLD_OK) return bail(s);
+  // activation operands: fp32 values (fp32 path) or (hi, lo) bf16 row pairs: 4 bytes each;
+  // q is fp32 in both (the bf16 attention splits it itself)
+  const size_t ael = 4;
+  if ((s = dalloc(x, &x->hb, Mm * d * ael)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->ssq, (d / kTileRows) * Mm * sizeof(float))) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->qbuf, Mm * x->qd * el)) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->attn, Mm * x->qd * el)) != NLD_OK) return bail(s);
-  if ((s = dalloc(x, &x->ubuf, Mm * c.ffn_dim * el)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->qbuf, Mm * x->qd * sizeof(float))) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->attn, Mm * x->qd * ael)) != NLD_OK) return bail(s);
+  if ((s = dalloc(x, &x->ubuf, Mm * c.ffn_dim * ael)) != NLD_OK) return bail(s);
   if ((s = dalloc(x, &x->lm_part, Mm * x->lm_tiles * sizeof(LmPart))) != NLD_OK) return bail(s);
   x->n_bars = (2 + c.n_layers) * kMaxPhases;
   if ((s = dalloc(x, &x->bars, x->n_bars * sizeof(unsigned))) != NLD_OK) return bail(s);
@@ -754,9 +804,9 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
   if (cudaMemset(x->err, 0, 16) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->lens, 0, B * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMemset(x->h, 0, Mm * d * sizeof(float)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
-  if (cudaMemset(x->hb, 0, Mm * d * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
-  if (cudaMemset(x->attn, 0, Mm * x->qd * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
-  if (cudaMemset(x->ubuf, 0, Mm * c.ffn_dim * el) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->hb, 0, Mm * d * ael) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->attn, 0, Mm * x->qd * ael) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
+  if (cudaMemset(x->ubuf, 0, Mm * c.ffn_dim * ael) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if ((s = dalloc(x, &x->fillnext, B * sizeof(int))) != NLD_OK) return bail(s);
   if (cudaMemset(x->fillnext, 0, B * sizeof(int)) != cudaSuccess) return bail(fail(x, NLD_ERR_CUDA, "memset"));
   if (cudaMallocHost(&x->h_pinned, (4 + 2 * B) * sizeof(int)) != cudaSuccess)
@@ -775,8 +825,7 @@ nld_status nld_create(const nld_config* cfg, void* cuda_stream, nld_ctx** out) {
 nld_status nld_destroy(nld_ctx* x) {
   if (!x) return NLD_OK;
   if (x->stream) cudaStreamSynchronize(x->stream);
-  for (auto& kv : x->graphs) cudaGraphExecDestroy(kv.second);
-  x->graphs.clear();
+  drop_graphs(x);
   for (void* p : x->allocs) cudaFree(p);
   x->allocs.clear();
   if (x->h_pinned) cudaFreeHost(x->h_pinned);
@@ -804,8 +853,7 @@ nld_status nld_init_lora(nld_ctx* x, int rank, float scale, const void* const* t
   }
   CK(cudaStreamSynchronize(x->stream));
   // the captured graphs hold the old launch sequence (or none of the LoRA launches)
-  for (auto& kv : x->graphs) cudaGraphExecDestroy(kv.second);
-  x->graphs.clear();
+  drop_graphs(x);
   x->lora_r = 0;
   if (rank == 0) return NLD_OK;
   const size_t el = x->el;
@@ -960,15 +1008,20 @@ namespace {
 nld_status flush_fill(nld_ctx* x);   // (diffusion, below)
 }  // namespace
 
-nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int prompt_len) {
+nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int stride, const int32_t* d_lens, int batch,
+                       int32_t* d_pending_out) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (!x->weights_ready) return fail(x, NLD_ERR_STATE, "weights not initialised");
   if (!d_tokens) return fail(x, NLD_ERR_ARG, "tokens is NULL");
   if (batch < 1 || batch > x->c.max_batch) return fail(x, NLD_ERR_ARG, "batch %d outside 1..%d", batch, x->c.max_batch);
-  if (prompt_len < 1 || prompt_len > x->c.max_seq) return fail(x, NLD_ERR_ARG, "prompt_len %d outside 1..%d", prompt_len, x->c.max_seq);
+  if (stride < 1 || stride > x->c.max_seq) return fail(x, NLD_ERR_ARG, "prompt stride %d outside 1..%d", stride, x->c.max_seq);
   x->batch = batch;
   const int k = x->c.block_k;
-  CK(cudaMemcpyAsync(x->prompt, d_tokens, static_cast<size_t>(batch) * prompt_len * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  CK(cudaMemcpyAsync(x->prompt, d_tokens, static_cast<size_t>(batch) * stride * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  if (d_lens)
+    CK(cudaMemcpyAsync(x->plens, d_lens, batch * sizeof(int), cudaMemcpyDeviceToDevice, x->stream));
+  else
+    CK(launch_fill_i32(x->stream, x->plens, stride, batch));
   CK(cudaMemsetAsync(x->lens, 0, batch * sizeof(int), x->stream));
   CK(launch_fill_i32(x->stream, x->blk, x->c.vocab, batch * k));
   CK(launch_fill_i32(x->stream, x->draft, x->c.vocab, batch * k));
@@ -976,8 +1029,11 @@ nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int promp
   CK(cudaMemsetAsync(x->fillnext, 0, batch * sizeof(int), x->stream));
   x->nl_active = false;
   x->len_upper = 0;
+  // causal forwards over positions 0..stride-2 in chunks of up to prefill_tokens rows; every
+  // sequence advances by the chunk (rows past its own prompt are padding), and the last
+  // finalize sets each sequence's length and pending token from its own prompt length
   const int chunk = std::max(1, x->prefill_tokens / batch);
-  const int rows = prompt_len - 1;
+  const int rows = stride - 1;
   int c0 = 0;
   do {
     const int m = std::min(chunk, rows - c0);
@@ -990,14 +1046,16 @@ nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int batch, int promp
       f.bs = 1;
       f.lm = LM_NONE;
       f.chunk0 = c0;
-      f.prompt_len = prompt_len;
+      f.prompt_len = stride;
       x->len_upper = c0;
       TRY(launch_forward(x, f));
     }
     FinalizeArgs a = base_fin(x, FWD_PREFILL, std::max(m, 1));
     a.chunk = m;
     a.prompt = last ? x->prompt : nullptr;
-    a.prompt_len = prompt_len;
+    a.prompt_len = stride;
+    a.plens = x->plens;
+    a.pending_out = last ? d_pending_out : nullptr;
     TRY(finalize(x, a));
     c0 += m;
     if (last) break;
@@ -1398,15 +1456,54 @@ nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out)
   return NLD_OK;
 }
 
+nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  if (stage_cap < 0 || stage_cap == 1 || stage_cap == 2 || stage_cap > gemm_chain_max_stages() ||
+      k_tiles_per_stage < 0 || k_tiles_per_stage > 2)
+    return fail(x, NLD_ERR_ARG, "stage cap 0 or 3..%d, k-tiles per stage 0..2", gemm_chain_max_stages());
+  CK(cudaStreamSynchronize(x->stream));
+  drop_graphs(x);   // captured graphs hold the old launch parameters
+  x->chain_stage_cap = stage_cap;
+  x->chain_kps = k_tiles_per_stage;
+  return NLD_OK;
+}
+
+nld_status nld_debug_timeout_chain(nld_ctx* x, unsigned long long timeout_ns) {
+  TRY(need_started(x));
+  if (!x->bf16) return fail(x, NLD_ERR_UNSUPPORTED, "tensor-core GEMM only");
+  if (x->c.n_layers < 2) return fail(x, NLD_ERR_UNSUPPORTED, "needs two layers (a four-phase chain)");
+  if (timeout_ns < 1000 || timeout_ns > 2000000000ull) return fail(x, NLD_ERR_ARG, "timeout outside 1 us..2 s");
+  const int M = x->batch;
+  TRY(ensure_capacity(x, 1));
+  ProjRef pr[4] = {hook_proj(x, GW_O, 0, M), hook_proj(x, GW_GU, 0, M), hook_proj(x, GW_D, 0, M),
+                   hook_proj(x, GW_QKV, 1, M)};
+  int grid = 0;
+  ChainArgs A = plan_chain(x, pr, 4, M, &grid);
+  for (int p = 0; p < 4; ++p) {
+    const WInfo w = winfo(x, pr[p].which, pr[p].layer);
+    A.ph[p].tmW = *w.map;
+    const CUtensorMap* tmX = xmap(x, w.buf, A.xr);
+    if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
+    A.ph[p].tmX = *tmX;
+    A.ph[p].e = pr[p].e;
+    A.ph[p].e.n_rows = w.n_rows;
+  }
+  A.bar = x->bars + kMaxPhases;   // layer 0's counters (left zero by every launch)
+  A.tmWn = A.ph[0].tmW;
+  A.dbg_skip_arrive = 1;
+  CK(launch_gemm_chain(x->stream, A, grid, timeout_ns, false));
+  return NLD_OK;
+}
+
 nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const int* max_clusters,
-                          int* out20) {
+                          int hilo, int* out20) {
   if (!n_rows || !K || !max_clusters || !out20) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
   if (M < 1 || nph < 1 || nph > kMaxPhases) return fail(nullptr, NLD_ERR_ARG, "bad plan sizes");
   for (int p = 0; p < nph; ++p)
     if (n_rows[p] < 1 || K[p] < kTileK || K[p] % kTileK)
       return fail(nullptr, NLD_ERR_ARG, "phase %d: rows %d, K %d", p, n_rows[p], K[p]);
   int grid = 0;
-  const ChainArgs A = plan_chain_shapes(max_clusters, n_rows, K, nph, M, &grid);
+  const ChainArgs A = plan_chain_shapes(max_clusters, n_rows, K, nph, M, hilo ? 1 : 0, &grid);
   if (A.CS < 1) return fail(nullptr, NLD_ERR_UNSUPPORTED, "no cluster size can be resident");
   for (int i = 0; i < 20; ++i) out20[i] = 0;
   out20[0] = A.CS;
@@ -1487,11 +1584,13 @@ void* nld_stream(nld_ctx* x) { return x ? static_cast<void*>(x->stream) : nullpt
 static const int* device_max_clusters() {
   static int cache[64][9];
   static bool ready[64] = {false};
+  static std::mutex mu;   // callers may come from several threads
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     dev = 0;
   }
+  std::lock_guard<std::mutex> lock(mu);
   if (!ready[dev]) {
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1503,6 +1602,9 @@ static const int* device_max_clusters() {
   return cache[dev];
 }
 
+// Workspace layout of the stand-alone LM head: a 256-byte block holding the device error word
+// (bounded waits that ran out), then the per-tile RMS sums, then the per-(row, vocab tile) partials.
+constexpr size_t kLmErrBytes = 256;
 static size_t lm_ssq_bytes(int M, int d) { return (static_cast<size_t>(d / kTileRows) * M * sizeof(float) + 255) / 256 * 256; }
 static size_t lm_part_bytes(int M, int vocab) {
   return static_cast<size_t>(M) * ((vocab + kTileRows - 1) / kTileRows) * sizeof(LmPart);
@@ -1528,11 +1630,12 @@ static nld_status lm_head_launch(const void* d_hidden, const void* d_lm_weight, 
     cudaGetLastError();
     return fail(nullptr, NLD_ERR_CUDA, "setting kernel shared-memory limits failed: %s", cudaGetErrorString(ae));
   }
-  float* ssq = reinterpret_cast<float*>(ws);
-  LmPart* part = reinterpret_cast<LmPart*>(ws + lm_ssq_bytes(M, d));
+  int* err = reinterpret_cast<int*>(ws);
+  float* ssq = reinterpret_cast<float*>(ws + kLmErrBytes);
+  LmPart* part = reinterpret_cast<LmPart*>(ws + kLmErrBytes + lm_ssq_bytes(M, d));
   int grid = 0;
   const int nr = vocab, kd = d;
-  ChainArgs A = plan_chain_shapes(device_max_clusters(), &nr, &kd, 1, M, &grid);
+  ChainArgs A = plan_chain_shapes(device_max_clusters(), &nr, &kd, 1, M, 0, &grid);
   PhaseArgs& P = A.ph[0];
   if (!make_map_bf16(&P.tmW, d_lm_weight, d, vocab, kTileRows) ||
       !make_map_bf16(&P.tmX, d_hidden, d, M, A.xr))
@@ -1551,17 +1654,20 @@ static nld_status lm_head_launch(const void* d_hidden, const void* d_lm_weight, 
   e.lm_part = part;
   e.lm_tiles = (vocab + kTileRows - 1) / kTileRows;
   e.V = vocab;
+  e.err = err;
   A.tmWn = P.tmW;
-  cudaError_t ce = launch_rms_stats(st, d_hidden, M, d, ssq);
+  // rms_stats clears the error word, the chain sets it when a wait runs out, and the combine
+  // then writes argmax -1 and confidence 0 for every row instead of partials never written
+  cudaError_t ce = launch_rms_stats(st, d_hidden, M, d, ssq, err);
   if (ce == cudaSuccess) ce = launch_gemm_chain(st, A, grid, 2000000000ull, false);
-  if (ce == cudaSuccess) ce = launch_lm_combine(st, part, M, e.lm_tiles, d_argmax_out, d_conf_out);
+  if (ce == cudaSuccess) ce = launch_lm_combine(st, part, M, e.lm_tiles, d_argmax_out, d_conf_out, err);
   if (ce != cudaSuccess) return fail(nullptr, NLD_ERR_CUDA, "LM-head launch failed: %s", cudaGetErrorString(ce));
   return NLD_OK;
 }
 
 size_t nld_lm_head_workspace_size(int M, int d, int vocab) {
   if (M < 1 || d < 128 || d % 128 || vocab < 1) return 0;
-  return lm_ssq_bytes(M, d) + lm_part_bytes(M, vocab);
+  return kLmErrBytes + lm_ssq_bytes(M, d) + lm_part_bytes(M, vocab);
 }
 
 nld_status nld_lm_head_argmax(const void* d_hidden, const void* d_lm_weight, int M, int d, int vocab,
@@ -1598,7 +1704,7 @@ nld_status nld_lm_head_argmax_static(const void* d_hidden, const void* d_lm_weig
   const size_t need = nld_lm_head_workspace_size(M, d, vocab);
   if (need > kStaticLmScratchBytes)
     return fail(nullptr, NLD_ERR_ARG,
-                "scratch of %zu bytes exceeds the built-in %zu bytes: M * (d/128 * 4 + ceil(vocab/128) * 16) "
+                "scratch of %zu bytes exceeds the built-in %zu bytes: 256 + M * (d/128 * 4 + ceil(vocab/128) * 16) "
                 "must stay within it (use nld_lm_head_argmax with a caller workspace)",
                 need, kStaticLmScratchBytes);
   int dev = 0;
@@ -1608,8 +1714,16 @@ nld_status nld_lm_head_argmax_static(const void* d_hidden, const void* d_lm_weig
   }
   void* scratch = nullptr;
   {
+    // outside stream capture the address is looked up on every call (cheap), so a device whose
+    // context was reset and whose module was reloaded gets the array's new address; under
+    // capture the last looked-up address is used
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(cuda_stream), &cap) != cudaSuccess) {
+      cudaGetLastError();
+      cap = cudaStreamCaptureStatusNone;
+    }
     std::lock_guard<std::mutex> lock(g_lm_scratch_mu);
-    if (!g_lm_scratch_addr[dev]) {
+    if (!g_lm_scratch_addr[dev] || cap == cudaStreamCaptureStatusNone) {
       void* ptr = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&ptr, g_lm_scratch);
       if (e != cudaSuccess || !ptr) {
@@ -1673,6 +1787,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   a.layer_row0 = 0;
   a.block_size = block_size;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  a.hilo = 0;   // caller's bf16 q and output
   a.err = nullptr;
   cudaError_t e = launch_attention_mma(static_cast<cudaStream_t>(cuda_stream), &map, a, batch, false);
   if (e != cudaSuccess) return fail(nullptr, NLD_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));

@@ -74,6 +74,7 @@ struct EpiArgs {
   int lm_tiles;
   float* logits;    // [M, V]
   int V;
+  int hilo;         // bf16 storage: hb / u written as (hi, lo) row pairs [2M, ld], q in fp32
   int* err;
 };
 
@@ -96,17 +97,20 @@ struct alignas(64) ChainArgs {
   CUtensorMap tmWn;  // weights of the projection that runs next on the stream (L2 warm-up)
   int nph;
   int CS;           // CTAs per cluster
-  int NT;           // token columns per tile (multiple of 16, <= 256)
+  int NT;           // tokens per tile (multiple of 16; MMA N = NT << hilo <= 256)
   int stages;       // shared-memory ring depth
   int kps;          // k-tiles (of 64) per stage: one barrier round trip moves kps x 16 KB of weights
-  int xr;           // activation rows loaded per k-tile of a token tile: the tile's token count
-                    // rounded up to 8 (<= NT); the MMA's N = NT columns read past them into
+  int xr;           // activation rows loaded per k-tile of a token tile: the tile's rows (2 per
+                    // token with hilo) rounded up to 8 (<= MMA N); the MMA reads past them into
                     // padding columns that the epilogue never uses
   int slots;        // split-K slot area: max over split phases of s * ceil(NT/16 / s) chunks
-  uint32_t tmem_cols;   // power of two >= 2*NT
+  int hilo;         // activation rows come in (hi, lo) pairs: MMA N = 2 NT, chunk sums of pairs
+  uint32_t tmem_cols;   // power of two >= 2 * MMA N
   unsigned* bar;    // [kMaxPhases] phase-boundary arrival counters + exit counter (last slot);
                     // zero before the launch, left zero by it
   unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
+  int dbg_skip_arrive;   // test hook: CTA 0 withholds its phase-0 arrival, so every wait on that
+                         // counter runs into its time limit (the failure-detection test)
   // the next chain launch's first phase (L2 warm-up of each CTA's first weight boxes there)
   int next_valid;
   int next_CS, next_s, next_tok_tiles, next_ks, next_KT, next_grid, next_tiles, next_boxes;
@@ -127,6 +131,7 @@ struct AttnArgs {
   const int* causal_seq;  // optional [batch]: nonzero makes all m rows of that sequence causal
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   float scale_log2;     // log2(e) / sqrt(hd)
+  int hilo;             // tensor-core path: q fp32 [M, Hq, hd], out (hi, lo) bf16 rows [2M, Hq, hd]
   int* err;
 };
 
@@ -148,8 +153,10 @@ struct EmbedArgs {
   int d, V, m, mode, k;
   const int* pending; const int* draft; const int* blk;
   const int* prompt; int prompt_len; int chunk0;
+  const int* plens;     // prefill: [batch] prompt lengths (rows at or past plens[b]-1 are padding)
   const int* lens;
   float* h; void* hb; float* ssq; int ssq_ld;
+  int hilo;             // bf16: hb rows in (hi, lo) pairs (the embedding row, then zeros)
   int* err;
 };
 cudaError_t launch_embed(cudaStream_t st, const EmbedArgs& a, int M, bool bf16, bool pdl);
@@ -162,6 +169,8 @@ struct FinalizeArgs {
   float threshold;
   int* incomplete;      // diffusion: count of sequences whose block is still open
   const int* prompt; int prompt_len; int chunk;   // prefill
+  const int* plens;     // prefill: [batch] prompt lengths (<= prompt_len, the row stride)
+  int* pending_out;     // prefill: [batch] the pending token of each sequence, or null
   int commit;           // 0 = only record argmaxes (test hook)
   int kv_cap;
   int* err;
@@ -175,16 +184,18 @@ cudaError_t launch_repack(cudaStream_t st, void* dst, const void* src, const int
 cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
 // LoRA drafter: fp32 partials zp [lora_n_ks][M][r] of z = A att, then h += scale * B z on
 // the rows t with t mod m >= causal_rows of sequences b = t / m whose causal_seq flag (if
-// given) is zero (z rounded to the activation type).  A [r, qd],
-// B [d, r] row-major; 8 <= r <= 256, r % 8 == 0; qd a multiple of 8.
+// given) is zero.  With hilo, att holds (hi, lo) bf16 row pairs [2M, qd] whose sums are the
+// attention output, and z stays fp32; otherwise z is rounded to the activation type.
+// A [r, qd], B [d, r] row-major; 8 <= r <= 256, r % 8 == 0; qd a multiple of 8.
 int lora_n_ks(int qd, bool bf16);
 cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
-                        const int* causal_seq, bool bf16, bool pdl);
-// Per 128-column tile sums of squares of bf16 rows h [M, d] into ssq [d/128, M].
-cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq);
-// Per token: argmax (lowest id on ties) and largest softmax probability from LM-head partials.
+                        const int* causal_seq, bool bf16, bool hilo, bool pdl);
+// Per 128-column tile sums of squares of bf16 rows h [M, d] into ssq [d/128, M]; zeroes *err.
+cudaError_t launch_rms_stats(cudaStream_t st, const void* h, int M, int d, float* ssq, int* err);
+// Per token: argmax (lowest id on ties) and largest softmax probability from LM-head partials;
+// argmax -1 and confidence 0 when *err is set (the partials were not all written).
 cudaError_t launch_lm_combine(cudaStream_t st, const LmPart* part, int M, int tiles, int* argmax,
-                              float* conf);
+                              float* conf, const int* err);
 
 }  // namespace nld

@@ -19,7 +19,7 @@ def make_pair(cfg, seed=0, precision=None, weights=None, device_weights=False):
     else:
         ctx.nld_init_weights(W, on_device=False)
     if precision is None:
-        precision = "f64" if cfg.dtype == synth.F32 else "bf16io"
+        precision = "f64" if cfg.dtype == synth.F32 else "f32kv"
     om = oracle.OracleModel(cfg, W, precision)
     return ctx, om, W
 

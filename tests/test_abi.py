@@ -53,12 +53,14 @@ def test_null_arguments_rejected():
     lib = nb.load_library()
     assert lib.nld_create(None, None, None) == 1
     assert lib.nld_destroy(None) == 0
-    assert lib.nld_prefill(None, None, 1, 1) == 1
+    assert lib.nld_prefill(None, None, 1, None, 1, None) == 1
+    assert lib.nld_debug_chain_tuning(None, 0, 0) == 1
+    assert lib.nld_debug_timeout_chain(None, 1000000) == 1
     assert lib.nld_selfspec_round(None, None, None, None) == 1
     assert lib.nld_sync(None) == 1
     assert lib.nld_attention(None, None, None, 1, 1, None, 1, 32, 32, 8, 128, 1, 32, None, None) == 1
     assert lib.nld_init_lora(None, 8, 1.0, None, 0, 0) == 1
     assert lib.nld_diffuse_block_step_fused(None, 0.9, None, None, None, None) == 1
     assert lib.nld_diffuse_step_nonlockstep(None, 0.9, None, None, None, None) == 1
-    assert lib.nld_plan_chain(1, 1, None, None, None, None) == 1
+    assert lib.nld_plan_chain(1, 1, None, None, None, 1, None) == 1
     assert lib.nld_plan_attention(1, 1, 8, 8, 1, 148, None) == 1

@@ -115,3 +115,31 @@ def test_repeated_calls_identical():
     a = _run(q, pool, perm, lens, m, 32, 532)
     b = _run(q, pool, perm, lens, m, 32, 532)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("L,bs", [(16384, 32), (16384, 1), (16384, 8), (32768, 32), (32768, 1)])
+def test_attention_microbench_prefix_batch32_sampled(L, bs):
+    """The attention micro-workload's largest points: batch 32, prefixes 16k and 32k, block
+    (32), causal (1) and block size 8 masks; operands built on the GPU, pages scattered by a
+    random page table; the oracle runs on sequences 0 and 31."""
+    B, m = 32, 32
+    q, k, v = synth.attention_operands(B, m, HQ, HKV, HD, L, seed=5, device="cuda")
+    pps = (L + m + 63) // 64
+    n_pages = B * pps
+    g = torch.Generator(device="cuda").manual_seed(7)
+    perm = torch.randperm(n_pages, generator=g, device="cuda").view(B, pps).to(torch.int32)
+    pool = torch.zeros(n_pages, 2, HKV, 64, HD, dtype=torch.bfloat16, device="cuda")
+    j = torch.arange(L + m, device="cuda")
+    pg = perm[:, j // 64].long()                       # [B, L+m] page of key row j
+    sl = (j % 64)[None, :].expand(B, -1)               # its slot in the page
+    pool_k, pool_v = pool[:, 0], pool[:, 1]
+    pool_k[pg, :, sl, :] = k.permute(0, 2, 1, 3)
+    pool_v[pg, :, sl, :] = v.permute(0, 2, 1, 3)
+    lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    import self_speculation_b200 as nb
+    out = torch.empty(B, m, HQ, HD, dtype=torch.bfloat16, device="cuda")
+    nb.nld_attention(q, pool, perm, lens, bs, L + m, out)
+    torch.cuda.synchronize()
+    for b in (0, B - 1):
+        want = _oracle(q[b:b + 1].cpu(), k[b:b + 1].cpu(), v[b:b + 1].cpu(), [L], m, bs)
+        assert (out[b:b + 1].cpu().double() - want).abs().max().item() < TOL

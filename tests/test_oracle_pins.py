@@ -378,16 +378,28 @@ def test_confidence_and_argmax_closed_forms():
     assert abs(float(odec.confidence(l)[0]) - 3.0 / 8.0) < 1e-15
 
 
-def test_bf16io_mode_close_to_f64():
-    """The rounding-matched mode differs from the exact forward only by bf16 rounding."""
+def test_f32kv_mode_is_fp32_over_a_bf16_cache():
+    """"f32kv" is the fp32 forward whose KV cache holds bf16 numbers: the rows it caches are
+    bf16 values within one bf16 spacing of the exact (f64) rows, and its logits differ from the
+    exact forward by the effect of that rounding (nonzero, well under the 2e-2 bar), while the
+    plain fp32 forward differs only by fp32 rounding."""
     cfg = synth.SMALL_BF16.replace(n_layers=1)
     W = synth.model_weights(cfg, 0)
     toks = synth.prompt_tokens(1, 9, cfg.vocab, seed=3).long()
-    a = oracle.OracleModel(cfg, W, "f64").forward(toks, [0], None or oracle.OracleModel(cfg, W, "f64").new_cache(1, 16), 1, False)
-    mb = oracle.OracleModel(cfg, W, "bf16io")
-    b = mb.forward(toks, [0], mb.new_cache(1, 16), 1, False)
-    err = (a - b.double()).abs().max().item()
-    assert 1e-6 < err < 5e-2
+    models = {p: oracle.OracleModel(cfg, W, p) for p in ("f64", "f32", "f32kv")}
+    caches = {p: m.new_cache(1, 16) for p, m in models.items()}
+    logits = {p: m.forward(toks, [0], caches[p], 1, True).double() for p, m in models.items()}
+    for kv in (0, 1):
+        exact = caches["f64"][0][0][kv][:, :9]
+        held = caches["f32kv"][0][0][kv][:, :9]
+        assert held.dtype == torch.bfloat16
+        # bf16 has 8 significand bits: neighbouring values are at most 2^-7 |x| apart
+        assert ((held.double() - exact).abs() <= 2.0 ** -7 * exact.abs() + 1e-30).all()
+        assert not torch.equal(held.double(), exact)
+    e32 = (logits["f32"] - logits["f64"]).abs().max().item()
+    ekv = (logits["f32kv"] - logits["f64"]).abs().max().item()
+    assert e32 < 1e-4
+    assert 1e-4 < ekv < 1e-2
 
 
 def test_mlp_branch_closed_form():

@@ -19,14 +19,14 @@ MAX_STAGES = 8
 B200_CLUSTERS = [0, 148, 74, 0, 33, 0, 0, 0, 16]
 
 
-def plan_chain(M, phases, clusters=B200_CLUSTERS):
+def plan_chain(M, phases, clusters=B200_CLUSTERS, hilo=1):
     lib = nb.load_library()
     n = len(phases)
     rows = (ctypes.c_int * n)(*[r for r, _ in phases])
     K = (ctypes.c_int * n)(*[k for _, k in phases])
     mc = (ctypes.c_int * 9)(*clusters)
     out = (ctypes.c_int * 20)()
-    st = lib.nld_plan_chain(M, n, rows, K, mc, out)
+    st = lib.nld_plan_chain(M, n, rows, K, mc, hilo, out)
     assert st == 0, lib.nld_last_error(None)
     o = list(out)
     return dict(CS=o[0], NT=o[1], xr=o[2], kps=o[3], stages=o[4], slots=o[5], tmem=o[6],
@@ -65,19 +65,24 @@ SHAPES = [("8b", synth.LLAMA8B.replace(max_batch=64)), ("14b", synth.LLAMA14B.re
 def test_chain_plans_keep_kernel_limits(name, cfg):
     for M in decode_Ms(cfg):
         for kind, phases in chains(cfg).items():
+            # the context's chains take (hi, lo) activation row pairs; the stand-alone LM head
+            # takes the caller's plain bf16 rows
+            hilo = 0 if kind == "lm" else 1
             for clusters in (B200_CLUSTERS, [0, 100, 50, 0, 20, 0, 0, 0, 8]):
-                P = plan_chain(M, phases, clusters)
+                P = plan_chain(M, phases, clusters, hilo)
                 where = (name, kind, M, clusters[4])
                 assert P["smem"] <= SMEM_BUDGET, where
-                assert 2 <= P["stages"] <= MAX_STAGES and P["kps"] == 2, where
+                assert 2 <= P["stages"] <= MAX_STAGES and P["kps"] in (1, 2), where
+                assert P["stages"] >= 3 or P["kps"] == 1, where
                 assert P["CS"] in (1, 2, 4, 8) and clusters[P["CS"]] >= 1, where
                 NT = P["NT"]
-                assert NT % 16 == 0 and 16 <= NT <= 256 and NT * P["tok_tiles"] >= M, where
-                assert P["xr"] % 8 == 0 and P["xr"] <= NT, where
+                NN = NT << hilo            # MMA N: activation rows of a token tile
+                assert NT % 16 == 0 and 16 <= NT and NN <= 256 and NT * P["tok_tiles"] >= M, where
+                assert P["xr"] % 8 == 0 and P["xr"] <= NN, where
                 if P["tok_tiles"] == 1:
-                    assert P["xr"] >= M, where
+                    assert P["xr"] >= M << hilo, where
                 t = P["tmem"]
-                assert t & (t - 1) == 0 and 2 * NT <= t <= 512, where
+                assert t & (t - 1) == 0 and 2 * NN <= t <= 512, where
                 assert P["grid"] % P["CS"] == 0 and P["grid"] <= P["CS"] * clusters[P["CS"]], where
                 if len(phases) > 1 and NT <= 64:
                     assert P["CS"] == 4, where
@@ -91,9 +96,10 @@ def test_chain_plans_keep_kernel_limits(name, cfg):
 def test_decode_plans_match_the_recorded_launch_list():
     cfg = synth.LLAMA8B
     ch = chains(cfg)
-    for M, NT, xr in ((33, 48, 40), (32, 32, 32)):
+    # (hi, lo) activation rows: 66 / 64 rows per k-tile box, MMA N = 96 / 64
+    for M, NT, xr in ((33, 48, 72), (32, 32, 64)):
         P = plan_chain(M, ch["layer"])
-        assert (P["CS"], P["NT"], P["xr"], P["stages"], P["grid"]) == (4, NT, xr, 4, 132)
+        assert (P["CS"], P["NT"], P["xr"], P["stages"], P["grid"]) == (4, NT, xr, 3, 132)
         L = plan_chain(M, ch["last"])
         assert (L["CS"], L["grid"]) == (4, 132)
     Q = plan_chain(33, ch["qkv0"])
@@ -115,7 +121,7 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
                 assert A["G"] * cfg.n_kv_heads == cfg.n_q_heads, where
                 assert 1 <= A["QT"] <= m and A["QT"] * A["q_tiles"] >= m, where
                 assert A["rows"] == A["QT"] * A["G"] and A["rows"] <= 16 * A["NW"], where
-                assert 1 <= A["NW"] <= 12, where
+                assert 1 <= A["NW"] <= 9, where
                 assert 1 <= A["S"] <= 8, where
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
                     assert A["S"] == 1, where
@@ -135,8 +141,8 @@ def test_plan_hooks_reject_bad_sizes():
     rows = (ctypes.c_int * 1)(4096)
     bad_k = (ctypes.c_int * 1)(100)
     mc = (ctypes.c_int * 9)(*B200_CLUSTERS)
-    assert lib.nld_plan_chain(33, 1, rows, bad_k, mc, out) == 1
-    assert lib.nld_plan_chain(0, 1, rows, (ctypes.c_int * 1)(4096), mc, out) == 1
+    assert lib.nld_plan_chain(33, 1, rows, bad_k, mc, 1, out) == 1
+    assert lib.nld_plan_chain(0, 1, rows, (ctypes.c_int * 1)(4096), mc, 1, out) == 1
     none = (ctypes.c_int * 9)(*([0] * 9))
-    assert lib.nld_plan_chain(33, 1, rows, (ctypes.c_int * 1)(4096), none, out) == 8   # unsupported
+    assert lib.nld_plan_chain(33, 1, rows, (ctypes.c_int * 1)(4096), none, 1, out) == 8   # unsupported
     assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 6)()) == 1
