@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 METRIC = "committed tokens/s & self-spec rounds/s at batch 1 (8B shape); % HBM roofline"
 PROMPT = 512
 K_BLOCK = 32
+GEN_TOKENS = 1024      # the generation length of the 8B self-speculation workload
 HBM_FALLBACK_GBS = 6650.0
 
 
@@ -42,8 +43,10 @@ def peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the layer-chain kernel's own sources (the kernel, its epilogues and the device
+    helpers it includes)."""
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "epilogue.cuh", "common.cuh", "nld_internal.h"):
+    for f in ("gemm_tc.cu", "epilogue.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "self_speculation_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -132,56 +135,42 @@ def reduce(vals, op, world):
 
 # ------------------------------------------------------------------------- CPU oracle leg --
 
-class OracleSample:
-    """The CPU oracle on a bounded sample of one round of the 8B shape: draft (k rows) and
-    verify (k+1 rows) forwards over `n_layers_sample` of the 36 layers, timed with and without
-    the LM head, at 511 cached rows (zero-valued cache; values do not change the work)."""
+class OracleRounds:
+    """The CPU oracle as it stands running whole linear self-speculation rounds of the 8B shape:
+    all 36 layers and the LM head, fp32 arithmetic with a bf16 KV cache, weights held as bf16
+    and widened per matmul.  The cache holds 511 zero-valued rows (the work of a round does not
+    depend on the cached values), so no 511-token prefill is run on the host.  Each call of
+    round() is one draft forward (k rows), one verify forward (k+1 rows) and the commit, timed
+    with the host clock."""
 
-    def __init__(self, n_layers_sample: int, threads: int):
+    def __init__(self, threads: int, n_layers: int = 36):
         import torch
 
         import oracle
         import synth
         torch.set_num_threads(threads)
-        self.cfg = synth.LLAMA8B
-        self.layers = list(range(n_layers_sample))
+        self.cfg = synth.LLAMA8B.replace(n_layers=n_layers)
         dev = "cuda" if torch.cuda.is_available() else "cpu"
-        W = synth.model_weights(self.cfg, 0, device=dev, layers=self.layers)
-        W = [None if w is None else w.cpu() for w in W]
-        self.om = oracle.OracleModel(self.cfg, W, "f32")
+        W = [w.cpu() for w in synth.model_weights(self.cfg, 0, device=dev)]
+        self.om = oracle.OracleModel(self.cfg, W, "f32kv")
+        self.cap = PROMPT + 8 * (K_BLOCK + 1)
 
     def round(self):
-        """Returns (seconds for a full 36-layer round by layer-count scaling, wall seconds spent,
-        committed tokens of the sampled round)."""
+        """Seconds of one measured round and the tokens it committed."""
         import torch
 
         from oracle import decode as odec
-        om, cfg, layers, k = self.om, self.cfg, self.layers, K_BLOCK
-        st = odec.SeqState(cache=om.new_cache(1, PROMPT + 2 * K_BLOCK + 2), lens=[PROMPT - 1],
-                           pending=[7])
-        t_all0 = time.perf_counter()
+        om, cfg, k = self.om, self.cfg, K_BLOCK
+        st = odec.SeqState(cache=om.new_cache(1, self.cap), lens=[PROMPT - 1], pending=[7])
+        t0 = time.perf_counter()
         draft_toks = torch.full((1, k), cfg.mask_id, dtype=torch.int64)
         draft_toks[0, 0] = st.pending[0]
-        t0 = time.perf_counter()
-        dl = om.forward(draft_toks, st.lens, st.cache, block_size=k, write_kv=False, layers=layers)
-        t1 = time.perf_counter()
-        om.forward(draft_toks, st.lens, st.cache, block_size=k, write_kv=False, layers=layers,
-                   with_logits=False)
-        t2 = time.perf_counter()
+        dl = om.forward(draft_toks, st.lens, st.cache, block_size=k, write_kv=False)
         drafts = odec.argmax_lowest(dl).tolist()
         ver_toks = torch.tensor([[st.pending[0]] + drafts[0]], dtype=torch.int64)
-        t3 = time.perf_counter()
-        vl = om.forward(ver_toks, st.lens, st.cache, block_size=1, write_kv=True, layers=layers)
-        t4 = time.perf_counter()
-        om.forward(ver_toks, st.lens, st.cache, block_size=1, write_kv=True, layers=layers,
-                   with_logits=False)
-        t5 = time.perf_counter()
+        vl = om.forward(ver_toks, st.lens, st.cache, block_size=1, write_kv=True)
         committed = odec.commit_after_verify(drafts[0], odec.argmax_lowest(vl).tolist()[0])
-        scale = cfg.n_layers / len(layers)
-        lm_d = max(0.0, (t1 - t0) - (t2 - t1))
-        lm_v = max(0.0, (t4 - t3) - (t5 - t4))
-        round_s = (t2 - t1) * scale + lm_d + (t5 - t4) * scale + lm_v
-        return round_s, time.perf_counter() - t_all0, len(committed)
+        return time.perf_counter() - t0, len(committed)
 
 
 # ------------------------------------------------------------------------------ our arm --
@@ -201,6 +190,7 @@ def run_ours(args, world, rank, local):
     nbuild.build()
     K, W = args.steps, args.warmup
     max_seq = (PROMPT + (K_BLOCK + 1) * (W + K + 2) + 63) // 64 * 64 + 64
+    max_seq = max(max_seq, PROMPT + GEN_TOKENS + 4 * (K_BLOCK + 1))
     cfg = synth.LLAMA8B.replace(max_seq=max_seq)
     torch_stream = torch.cuda.Stream()          # owned by torch; the library orders on it
     ctx = nb.Context(cfg, stream=torch_stream.cuda_stream)
@@ -315,16 +305,48 @@ def run_ours(args, world, rank, local):
            "h2d_bytes_per_step": int(PROMPT * 4 / K), "d2h_bytes_per_step": (K_BLOCK + 2) * 4,
            "includes": "prompt upload + prefill of 512 tokens + K rounds with a D2H read each"}
 
+    # generation of config 3's length: a fresh 512-token prompt, rounds until 1024 tokens are
+    # committed (the cached prefix grows 512 -> 1536), timed with CUDA events on the stream
+    gen = None
+    if not args.no_generation:
+        ctx.nld_prefill(prompt.cuda())
+        ctx.nld_sync()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        rounds, done = 0, 0
+        while done < GEN_TOKENS:
+            burst = max(1, min(64, (GEN_TOKENS - done + K_BLOCK) // (K_BLOCK + 1)))
+            for _ in range(burst):
+                ctx.nld_selfspec_round(toks, nc, None)
+            rounds += burst
+            ctx.nld_debug_state(lens)
+            ctx.nld_sync()
+            done = int(lens.item()) - (PROMPT - 1)
+        g1.record(stream)
+        g1.synchronize()
+        gms = g0.elapsed_time(g1)
+        gen = {"tokens": done, "rounds": rounds, "ms": round(gms, 2),
+               "tokens_per_s": round(done / (gms / 1e3), 3),
+               "ms_per_round": round(gms / rounds, 4),
+               "prefix": f"{PROMPT} -> {PROMPT + done}",
+               "note": "host reads the length every up to 64 rounds to stop at 1024 tokens"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        round_est, spent, ncommit = OracleSample(2, threads).round()
-        cpu = {"value": round(ncommit / round_est, 5), "unit": "tokens/s", "cores": threads,
+        ref = OracleRounds(threads)
+        secs, ncommit = [], 0
+        for _ in range(2):
+            s_round, c = ref.round()
+            secs.append(s_round)
+            ncommit += c
+        cpu = {"value": round(ncommit / sum(secs), 5), "unit": "tokens/s", "cores": threads,
                "kind": "oracle",
-               "sample": (f"one draft+verify round of the 8B shape at 511 cached rows over 2 of 36 "
-                          f"layers plus the LM head, scaled to 36 layers ({spent:.1f} s of CPU "
-                          f"work); {ncommit} committed token(s) in the sampled round"),
-               "round_s_est": round(round_est, 2)}
+               "sample": (f"2 whole self-speculation rounds of the 8B shape (36 layers + LM head, "
+                          f"fp32 with a bf16 KV cache, 511 cached rows), measured: "
+                          f"{', '.join(f'{x:.2f}' for x in secs)} s; {ncommit} committed tokens"),
+               "round_s": round(sum(secs) / len(secs), 3)}
 
     # two forwards (draft, verify), each: embed, QKV chain of layer 0, per layer one attention
     # and one chain (O, gate/up, down, then the next QKV or, last, the LM head); then finalize
@@ -350,6 +372,7 @@ def run_ours(args, world, rank, local):
         "kernels": kern,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "generation_1024": gen,
         "gpu_launches": K * per_round,
         "clocks": clocks,
     }
@@ -362,33 +385,32 @@ def run_ours(args, world, rank, local):
 
 
 def run_reference(args, world, rank, local):
-    """The oracle as it stands on the host cores (rank 0 only), each step one bounded sample
-    of a round (1 of 36 layers of a draft and a verify forward plus the LM head, scaled)."""
+    """The oracle as it stands on the host cores (rank 0 only): every step is one whole round of
+    the 8B shape (both forwards over all 36 layers and the LM head), timed with the host clock."""
     if rank != 0:
         return
     threads = os.cpu_count() or 1
-    est, committed, spent = [], 0, 0.0
-    sample = OracleSample(1, threads)
+    ref = OracleRounds(threads, args.ref_layers)
+    secs, committed = [], 0
     for i in range(args.warmup + args.steps):
-        r, s, c = sample.round()
+        s_round, c = ref.round()
         if i >= args.warmup:
-            est.append(r)
+            secs.append(s_round)
             committed += c
-            spent += s
-    round_s = sum(est) / len(est)
-    value = committed / sum(est)
+    value = committed / sum(secs)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(round_s * 1e3, 2), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "ms_per_step": round(1e3 * sum(secs) / len(secs), 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "8B-shaped linear self-speculation round, batch 1, k=32, "
                                "prompt 512 random ids (CPU oracle)",
-                   "parallelism": "host cores of rank 0"},
+                   "layers": args.ref_layers, "parallelism": "host cores of rank 0"},
         "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": threads,
                          "kind": "oracle",
-                         "sample": "per step: draft+verify forwards over 1 of 36 layers plus the "
-                                   "LM head at 511 cached rows, scaled to 36 layers"},
+                         "sample": "per step: one whole round (draft and verify forwards over all "
+                                   "36 layers plus the LM head, fp32 with a bf16 KV cache) at 511 "
+                                   "cached rows, measured"},
         "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -424,27 +446,30 @@ def run_attention(args):
     Hq, Hkv, hd, m = 32, 8, 128, 32
     stream = torch.cuda.current_stream()
     points = []
-    for L in (1024, 4096, 16384, 32768):
-        for B in (1, 8, 32):
-            pps = (L + m + 63) // 64
-            n_pages = B * pps
-            g = torch.Generator(device="cuda").manual_seed(2)
-            pool = torch.randn((n_pages, 2, Hkv, 64, hd), generator=g, device="cuda").to(torch.bfloat16)
-            q = torch.randn((B, m, Hq, hd), generator=g, device="cuda").to(torch.bfloat16)
-            perm = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).view(B, pps)
-            lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
-            out = torch.empty_like(q)
-            byts = B * (L + m) * Hkv * hd * 2 * 2 + 2 * B * m * Hq * hd * 2
-            for mode, bs in (("block", 32), ("causal", 1), ("block_size_1", 1)):
-                ms = _events_ms(lambda: nb.nld_attention(q, pool, perm, lens, bs, L + m, out,
-                                                         stream.cuda_stream), stream, reps=20)
-                gbs = byts / (ms / 1e3) / 1e9
-                points.append({"prefix": L, "batch": B, "mode": mode, "us": round(ms * 1e3, 2),
-                               "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
-                               "l2_resident": byts < 126e6})
-            del pool, q, perm, out
-            torch.cuda.empty_cache()
-    big = [p for p in points if not p["l2_resident"]]
+    grid = [(L, B) for L in (1024, 4096, 16384, 32768) for B in (1, 8, 32)]
+    if args.attn_point:
+        L, B = (int(v) for v in args.attn_point.split(","))
+        grid = [(L, B)]
+    for L, B in grid:
+        pps = (L + m + 63) // 64
+        n_pages = B * pps
+        g = torch.Generator(device="cuda").manual_seed(2)
+        pool = torch.randn((n_pages, 2, Hkv, 64, hd), generator=g, device="cuda").to(torch.bfloat16)
+        q = torch.randn((B, m, Hq, hd), generator=g, device="cuda").to(torch.bfloat16)
+        perm = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).view(B, pps)
+        lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+        out = torch.empty_like(q)
+        byts = B * (L + m) * Hkv * hd * 2 * 2 + 2 * B * m * Hq * hd * 2
+        for mode, bs in (("block", 32), ("causal", 1), ("block_size_1", 1)):
+            ms = _events_ms(lambda: nb.nld_attention(q, pool, perm, lens, bs, L + m, out,
+                                                     stream.cuda_stream), stream, reps=20)
+            gbs = byts / (ms / 1e3) / 1e9
+            points.append({"prefix": L, "batch": B, "mode": mode, "us": round(ms * 1e3, 2),
+                           "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                           "l2_resident": byts < 126e6})
+        del pool, q, perm, out
+        torch.cuda.empty_cache()
+    big = [p for p in points if not p["l2_resident"]] or points
     best = max(big, key=lambda p: p["GB/s"])
     print(json.dumps({
         "metric": "attention HBM throughput (block-causal GQA over paged bf16 KV)",
@@ -684,6 +709,8 @@ def run_probe(args):
     st = torch.cuda.Stream()
     ctx = nb.Context(cfg, stream=st.cuda_stream)
     ctx.nld_init_weights(synth.model_weights(cfg, 0, device="cuda"), on_device=True)
+    if args.lora:
+        ctx.nld_init_lora(args.lora, 1.0, synth.lora_weights(cfg, args.lora, 0, device="cuda"))
     ctx.nld_prefill(synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1).cuda())
     toks = torch.empty(1, K_BLOCK + 1, dtype=torch.int32, device="cuda")
     nc = torch.empty(1, dtype=torch.int32, device="cuda")
@@ -729,11 +756,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-layers", type=int, default=36,
+                    help="layers of the reference arm's model (36 = the 8B shape; fewer only to "
+                         "exercise the arm's output quickly)")
+    ap.add_argument("--no-generation", action="store_true",
+                    help="skip the 1024-token generation measured after the timed rounds")
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a seeded random o_proj adapter in the draft forwards (0: none)")
     ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b",
                                            "commit8b"],
                     default="selfspec8b")
+    ap.add_argument("--attn-point", default="",
+                    help="attention workload: one point 'prefix,batch' instead of the whole grid")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
     args = ap.parse_args()

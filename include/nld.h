@@ -55,7 +55,7 @@ typedef enum {
 enum { NLD_F32 = 0, NLD_BF16 = 1 };
 
 /* Forward kinds accepted by nld_debug_logits. */
-enum { NLD_MODE_AR = 0, NLD_MODE_DRAFT = 1, NLD_MODE_VERIFY = 2, NLD_MODE_DIFFUSE = 3 };
+enum { NLD_MODE_AR = 0, NLD_MODE_DRAFT = 1, NLD_MODE_VERIFY = 2, NLD_MODE_DIFFUSE = 3, NLD_MODE_QUAD = 4 };
 
 /* Device error word bits (reported by nld_sync). */
 enum { NLD_DEVERR_KV_OVERFLOW = 1, NLD_DEVERR_TIMEOUT = 2, NLD_DEVERR_TOKEN = 4 };
@@ -169,6 +169,25 @@ nld_status nld_kv_commit(nld_ctx* ctx, const int32_t* d_nrows, int32_t* d_tokens
 nld_status nld_selfspec_round(nld_ctx* ctx, int32_t* d_tokens_out, int32_t* d_ncommit_out,
                               const int32_t* d_force_ncommit);
 
+/* One quadratic self-speculation round (ranhao.site notes section 8.1 and the shilu.ai blog's
+ * performance highlights name the mode and give it more tokens per forward than the linear
+ * round; the pages do not define it.  Reading taken: ONE forward per round).  The forward holds,
+ * per sequence, (k+1)^2 rows:
+ *   rows 0..k     the causal verify rows [x_n, d_1..d_k] at positions n..n+k (KV rows n..n+k
+ *                 written at their final slots, as in the linear verify forward);
+ *   rows k+1+a*k+j, a = 0..k, j = 0..k-1: pre-draft block a, the next round's draft block for
+ *                 the outcome "a drafts accepted": mask ids at positions n+a+1+j, seeing the
+ *                 cached prefix, the verify rows 0..a and its own k rows, nothing else (their
+ *                 K/V go to scratch slots n+k+1.. that later forwards overwrite).
+ * The round then commits exactly like nld_selfspec_round (greedy longest matching prefix,
+ * c = a+1 tokens into d_tokens_out [batch, k+1] and d_ncommit_out [batch]), and the argmaxes
+ * of block a become the next round's drafts, so a run of rounds costs one forward each.  The
+ * first round after any other decode call starts from one linear draft forward.  Needs
+ * batch * (k+1)^2 <= 2048 token rows and (k+1)^2 KV slots past each sequence (max_seq must
+ * leave k*(k+1) rows of room beyond the committed tokens; else NLD_ERR_KV_FULL).  The LoRA
+ * drafter, if loaded, applies to the pre-draft rows. */
+nld_status nld_quadratic_round(nld_ctx* ctx, int32_t* d_tokens_out, int32_t* d_ncommit_out);
+
 /* One block-diffusion denoising step for every sequence (lockstep).  Forward over
  * [x_n, b_1..b_{k-1}] (open slots hold the [MASK] id), one bidirectional block; row i gives
  * argmax and confidence (largest softmax probability over the vocab) for slot b_{i+1}.
@@ -216,9 +235,10 @@ nld_status nld_diffuse_step_nonlockstep(nld_ctx* ctx, float threshold, int32_t* 
                                         float* d_conf_out, int32_t* d_ncommit_out, int32_t* d_state_out);
 
 /* Test hook: run the forward of `mode` (NLD_MODE_*) from the current state and write its
- * logits [batch, m, vocab] fp32 to d_logits_out (m = 1, k, k+1, k).  Sequence state is not
- * advanced; a DRAFT call stores its argmaxes as the drafts a later VERIFY call reads.  The
- * decode calls above never materialise logits. */
+ * logits [batch, m, vocab] fp32 to d_logits_out (m = 1, k, k+1, k, (k+1)^2 for AR, DRAFT,
+ * VERIFY, DIFFUSE, QUAD).  Sequence state is not advanced; a DRAFT call stores its argmaxes as
+ * the drafts a later VERIFY or QUAD call reads (QUAD records nothing).  The decode calls above
+ * never materialise logits. */
 nld_status nld_debug_logits(nld_ctx* ctx, int mode, float* d_logits_out);
 
 /* Test hook: copy state out (any pointer may be NULL): lens [batch], pending [batch],
@@ -282,9 +302,12 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
 
 /* Profiling hook: tuning of the projection chains' pipeline.  stage_cap = 0 lets the planner
  * use as many shared-memory stages as fit, else at most stage_cap (3..8); k_tiles_per_stage =
- * 1 or 2 weight boxes (16 KB each) per ring stage (0 = the planner's choice).  Synchronises and
- * drops the captured graphs; later calls use the new values. */
-nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_stage);
+ * 1 or 2 weight boxes (16 KB each) per ring stage (0 = the planner's choice);
+ * boundary_prefetch = weight boxes each CTA prefetches into L2 while it waits at a phase
+ * boundary (0..256; 16 at creation).  Synchronises and drops the captured graphs; later calls
+ * use the new values. */
+nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_stage,
+                                  int boundary_prefetch);
 
 /* Test hook for failure detection: one launch of layer 0's four-phase chain over the current
  * batch (scratch buffers only, as nld_time_chain) with every bounded wait limited to timeout_ns

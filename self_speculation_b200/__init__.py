@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libnld.so")
 HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "nld.h")
 
 NLD_F32, NLD_BF16 = 0, 1
-NLD_MODE_AR, NLD_MODE_DRAFT, NLD_MODE_VERIFY, NLD_MODE_DIFFUSE = 0, 1, 2, 3
+NLD_MODE_AR, NLD_MODE_DRAFT, NLD_MODE_VERIFY, NLD_MODE_DIFFUSE, NLD_MODE_QUAD = 0, 1, 2, 3, 4
 STATUS = {0: "NLD_OK", 1: "NLD_ERR_ARG", 2: "NLD_ERR_OOM", 3: "NLD_ERR_CUDA", 4: "NLD_ERR_KV_FULL",
           5: "NLD_ERR_STATE", 6: "NLD_ERR_TIMEOUT", 7: "NLD_ERR_DEVICE", 8: "NLD_ERR_UNSUPPORTED"}
 
@@ -57,6 +57,7 @@ def load_library() -> ctypes.CDLL:
         "nld_selfspec_draft_verify": ([P], I),
         "nld_kv_commit": ([P, P, P, P], I),
         "nld_selfspec_round": ([P, P, P, P], I),
+        "nld_quadratic_round": ([P, P, P], I),
         "nld_diffuse_block_step": ([P, F, P, P, P, P], I),
         "nld_diffuse_block_step_fused": ([P, F, P, P, P, P], I),
         "nld_diffuse_step_nonlockstep": ([P, F, P, P, P, P], I),
@@ -71,7 +72,7 @@ def load_library() -> ctypes.CDLL:
         "nld_plan_attention": ([I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
         "nld_time_chain": ([P, I, I, I, ctypes.POINTER(F)], I),
-        "nld_debug_chain_tuning": ([P, I, I], I),
+        "nld_debug_chain_tuning": ([P, I, I, I], I),
         "nld_debug_timeout_chain": ([P, ctypes.c_ulonglong], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
@@ -175,6 +176,9 @@ class Context:
         self._check(self.lib.nld_selfspec_round(self.h, _ptr(tokens_out), _ptr(ncommit_out),
                                                 _ptr(force)), self.h)
 
+    def nld_quadratic_round(self, tokens_out, ncommit_out) -> None:
+        self._check(self.lib.nld_quadratic_round(self.h, _ptr(tokens_out), _ptr(ncommit_out)), self.h)
+
     def nld_diffuse_block_step(self, threshold: float, block_out, conf_out, ncommit_out) -> bool:
         filled = ctypes.c_int32(0)
         self._check(self.lib.nld_diffuse_block_step(self.h, float(threshold), _ptr(block_out),
@@ -223,9 +227,10 @@ class Context:
         self._check(self.lib.nld_trace_chain(self.h, layer, M, _ptr(trace), ctypes.byref(g)), self.h)
         return g.value
 
-    def nld_debug_chain_tuning(self, stage_cap: int, k_tiles_per_stage: int = 0) -> None:
-        self._check(self.lib.nld_debug_chain_tuning(self.h, int(stage_cap), int(k_tiles_per_stage)),
-                    self.h)
+    def nld_debug_chain_tuning(self, stage_cap: int = 0, k_tiles_per_stage: int = 0,
+                               boundary_prefetch: int = 16) -> None:
+        self._check(self.lib.nld_debug_chain_tuning(self.h, int(stage_cap), int(k_tiles_per_stage),
+                                                    int(boundary_prefetch)), self.h)
 
     def nld_debug_timeout_chain(self, timeout_ns: int) -> None:
         self._check(self.lib.nld_debug_timeout_chain(self.h, int(timeout_ns)), self.h)

@@ -73,6 +73,24 @@ NLD_DEV int vis_end_of(int len, int p, int bs, int m, int c) {
   return len + min(blk0 + bs, m) - 1;
 }
 
+// Keys visible to row p: [0, v1] and [l2, h2] (an empty second interval unless p is a
+// pre-draft row of the quadratic self-speculation forward with block k = quad_k: rows 0..k are
+// the causal verify rows; row k+1+a*k+j sees the cached prefix, the verify rows 0..a, i.e. keys
+// up to len+a, and the k rows of its own block at slots len+k+1+a*k ..).
+NLD_DEV void row_keys(int len, int p, int bs, int m, int c, int quad_k, int& v1, int& l2, int& h2) {
+  if (quad_k > 0 && p > quad_k) {
+    const int blk = (p - quad_k - 1) / quad_k;
+    v1 = len + blk;
+    l2 = len + quad_k + 1 + blk * quad_k;
+    h2 = l2 + quad_k - 1;
+  } else {
+    v1 = vis_end_of(len, p, bs, m, c);
+    l2 = 0x7fffffff;
+    h2 = -1;
+  }
+}
+NLD_DEV bool key_visible(int key, int v1, int l2, int h2) { return key <= v1 || (key >= l2 && key <= h2); }
+
 }  // namespace
 
 // kHiLo (the model's forwards): q arrives in fp32 and is split into bf16 hi and lo halves, the
@@ -119,7 +137,13 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     len = max(0, min(len, a.pps * kPage - a.m));
   }
   const int crow = (a.causal_seq && a.causal_seq[b]) ? a.m : a.causal_rows;
-  const int kv_end = vis_end_of(len, p0 + np - 1, a.block_size, a.m, crow) + 1;
+  int kv_end;
+  {
+    // the CTA's last row sees the furthest key (both intervals grow with the row)
+    int v1, l2, h2;
+    row_keys(len, p0 + np - 1, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
+    kv_end = max(v1, h2) + 1;
+  }
   const int n_tiles = (kv_end + kPage - 1) / kPage;
   // at least two KV tiles per split: fewer, fuller splits keep the merge short
   const int per = max(2, (n_tiles + a.S - 1) / a.S);
@@ -187,12 +211,11 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   }
   const int ra = warp * 16 + (lane >> 2);
   const int rb = ra + 8;
-  auto row_vis = [&](int r) {
-    const int p = r / a.G;
-    if (r >= a.rows || p >= np) return -1;
-    return vis_end_of(len, p0 + p, a.block_size, a.m, crow);
-  };
-  const int vis_a = row_vis(ra), vis_b = row_vis(rb);
+  int vis_a = -1, la2 = 0x7fffffff, ha2 = -1, vis_b = -1, lb2 = 0x7fffffff, hb2 = -1;
+  if (ra < a.rows && ra / a.G < np)
+    row_keys(len, p0 + ra / a.G, a.block_size, a.m, crow, a.quad_k, vis_a, la2, ha2);
+  if (rb < a.rows && rb / a.G < np)
+    row_keys(len, p0 + rb / a.G, a.block_size, a.m, crow, a.quad_k, vis_b, lb2, hb2);
 
   float o[16][4];
 #pragma unroll
@@ -247,8 +270,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
       for (int e2 = 0; e2 < 2; ++e2) {
         float s0 = sc[nt][e2] * a.scale_log2;
         float s1 = sc[nt][2 + e2] * a.scale_log2;
-        if (key + e2 > vis_a) s0 = -INFINITY;
-        if (key + e2 > vis_b) s1 = -INFINITY;
+        if (!key_visible(key + e2, vis_a, la2, ha2)) s0 = -INFINITY;
+        if (!key_visible(key + e2, vis_b, lb2, hb2)) s1 = -INFINITY;
         sc[nt][e2] = s0;
         sc[nt][2 + e2] = s1;
         mx_a = fmaxf(mx_a, s0);
@@ -437,7 +460,9 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
     len = max(0, min(len, a.pps * kPage - a.m));
   }
   const int crow = (a.causal_seq && a.causal_seq[b]) ? a.m : a.causal_rows;
-  const int nkeys = vis_end_of(len, i, a.block_size, a.m, crow) + 1;
+  int v1, l2, h2;
+  row_keys(len, i, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
+  const int nkeys = max(v1, h2) + 1;
   const T* q = static_cast<const T*>(a.q) + (static_cast<size_t>(tok) * a.Hq + head) * a.hd;
   for (int d = threadIdx.x; d < a.hd; d += blockDim.x) sq[d] = to_f32<T>(q[d]);
   __syncthreads();
@@ -449,7 +474,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
                   static_cast<size_t>(j & 63) * a.hd;
     float acc = 0.f;
     for (int d = 0; d < a.hd; ++d) acc += sq[d] * to_f32<T>(kr[d]);
-    sc[j] = acc * scale;
+    sc[j] = key_visible(j, v1, l2, h2) ? acc * scale : -INFINITY;
   }
   __syncthreads();
   float mx = -INFINITY;

@@ -40,6 +40,9 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedArgs a) {
     case FWD_FILLDIFF:   // the complete block (causal rows), then b_k and k-1 masks
       id = (i == 0) ? a.pending[b] : (i <= a.k ? a.blk[b * a.k + i - 1] : a.V);
       break;
+    case FWD_QUAD:       // verify rows [x_n, d_1..d_k], then (k+1) pre-draft blocks of masks
+      id = (i == 0) ? a.pending[b] : (i <= a.k ? a.draft[b * a.k + i - 1] : a.V);
+      break;
     default: id = (i == 0) ? a.pending[b] : a.blk[b * a.k + i - 1]; break;
   }
   if (id < 0 || id > a.V) {
@@ -100,6 +103,81 @@ NLD_DEV void lm_merge(float& mx, float& se, int& ix, float bmx, float bse, int b
   }
 }
 
+// Combine the LM-head partials of row `row` of sequence b (one warp): argmax (lowest id on ties)
+// and confidence, valid in every lane.
+NLD_DEV void combine_row(const FinalizeArgs& a, int b, int row, int lane, int& ix_out, float& conf_out) {
+  const LmPart* part = a.lm_part + static_cast<size_t>(b * a.m + row) * a.lm_tiles;
+  float mx = -INFINITY, se = 0.f;
+  int ix = INT_MAX;
+  for (int t0 = lane; t0 < a.lm_tiles; t0 += 32 * 8) {
+    LmPart p[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + 32 * u;
+      if (t < a.lm_tiles) {
+        p[u] = part[t];
+      } else {
+        p[u].mx = -INFINITY;
+        p[u].se = 0.f;
+        p[u].idx = INT_MAX;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) lm_merge(mx, se, ix, p[u].mx, p[u].se, p[u].idx);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, mx, off);
+    const float os = __shfl_xor_sync(0xffffffffu, se, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, ix, off);
+    lm_merge(mx, se, ix, om, os, oi);
+  }
+  ix_out = ix;
+  conf_out = 1.0f / se;
+}
+
+// Quadratic self-speculation round (one CTA per sequence): the verify rows 0..k give v_1..v_{k+1};
+// the round commits as the linear round does (greedy longest matching prefix, c = a+1 tokens
+// d_1..d_a, v_{a+1}); the next drafts are the argmaxes of pre-draft block a (rows
+// k+1+a*k .. k+1+a*k+k-1), the block whose rows assumed exactly this outcome.
+NLD_DEV void finalize_quad(const FinalizeArgs& a, int b, int warp, int lane, int* s_arg) {
+  const int k = a.k;
+  __shared__ int s_c;
+  for (int i = warp; i <= k; i += kFinalizeThreads / 32) {
+    int ix;
+    float cf;
+    combine_row(a, b, i, lane, ix, cf);
+    if (lane == 0) s_arg[i] = ix;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const bool match = (lane < k) ? (a.draft[b * k + lane] == s_arg[lane]) : true;
+    const unsigned bal = __ballot_sync(0xffffffffu, match);
+    const int acc = min((bal == 0xffffffffu) ? 32 : (__ffs(~bal) - 1), k);
+    const int c = acc + 1;
+    for (int j = lane; j < k + 1; j += 32) {
+      const int v = (j < c - 1) ? a.draft[b * k + j] : (j == c - 1 ? s_arg[j] : -1);
+      if (a.tokens_out) a.tokens_out[b * (k + 1) + j] = v;
+      a.verify[b * (k + 1) + j] = s_arg[j];
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (a.ncommit_out) a.ncommit_out[b] = c;
+      a.lens[b] += c;
+      a.pending[b] = s_arg[c - 1];
+      s_c = c;
+    }
+  }
+  __syncthreads();
+  const int r0 = k + 1 + (s_c - 1) * k;
+  for (int i = warp; i < k; i += kFinalizeThreads / 32) {
+    int ix;
+    float cf;
+    combine_row(a, b, r0 + i, lane, ix, cf);
+    if (lane == 0) a.draft[b * k + i] = ix;   // the old drafts were read by warp 0 above
+  }
+}
+
 __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const FinalizeArgs a) {
   pdl_wait();
   pdl_launch_dependents();
@@ -107,41 +185,22 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
   __shared__ float s_conf[64];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (a.mode == FWD_QUAD) {
+    finalize_quad(a, b, warp, lane, s_arg);
+    return;
+  }
   const bool lm = (a.mode == FWD_AR || a.mode == FWD_DRAFT || a.mode == FWD_VERIFY ||
                    a.mode == FWD_DIFFUSE || a.mode == FWD_FILLDIFF || a.mode == FWD_NLDIFF);
   if (lm) {
     // one warp per row; one pass over the row's vocab tiles with 8 loads in flight per lane,
     // merging (max, sum exp, argmax) online, then across the warp
     for (int i = warp; i < a.m; i += kFinalizeThreads / 32) {
-      const LmPart* row = a.lm_part + static_cast<size_t>(b * a.m + i) * a.lm_tiles;
-      float mx = -INFINITY, se = 0.f;
-      int ix = INT_MAX;
-      for (int t0 = lane; t0 < a.lm_tiles; t0 += 32 * 8) {
-        LmPart p[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = t0 + 32 * u;
-          if (t < a.lm_tiles) {
-            p[u] = row[t];
-          } else {
-            p[u].mx = -INFINITY;
-            p[u].se = 0.f;
-            p[u].idx = INT_MAX;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) lm_merge(mx, se, ix, p[u].mx, p[u].se, p[u].idx);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float om = __shfl_xor_sync(0xffffffffu, mx, off);
-        const float os = __shfl_xor_sync(0xffffffffu, se, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, ix, off);
-        lm_merge(mx, se, ix, om, os, oi);
-      }
+      int ix;
+      float cf;
+      combine_row(a, b, i, lane, ix, cf);
       if (lane == 0) {
         s_arg[i] = ix;
-        s_conf[i] = 1.0f / se;
+        s_conf[i] = cf;
       }
     }
     __syncthreads();

@@ -12,8 +12,9 @@
 namespace nld {
 
 // Per-column data of a tile, computed once per tile into shared memory (see
-// compute_tile_meta): s_inv = 1/rms of the token, s_pos = its position (-1: no KV row: column
-// past M or past the KV capacity), s_pg = the KV page holding that position.
+// compute_tile_meta): s_inv = 1/rms of the token, s_pos = its KV slot (-1: no KV row: column
+// past M or past the KV capacity), s_pg = the KV page holding that slot, s_rpos = its RoPE
+// position (the slot itself except in the quadratic self-speculation forward).
 // red_f / red_i: shared scratch of at least 4*16 + 16 entries each, private to the 4 warps (one
 // per TMEM lane quarter, 128 threads) that call this together and synchronise on named
 // barrier `bar_id`.
@@ -42,7 +43,7 @@ NLD_DEV void qkv_row_info(const EpiArgs& e, int row, int& sec, int& head, int& l
 }
 
 NLD_DEV void epi_preload(const EpiArgs& e, int row_tile, int row_in_tile, int tok0,
-                         const int* s_pos, int col0, EpiPre& p) {
+                         const int* s_rpos, int col0, EpiPre& p) {
   const int row = row_tile * kTileRows + row_in_tile;
   if (e.kind == EPI_RESID) {
 #pragma unroll
@@ -54,7 +55,7 @@ NLD_DEV void epi_preload(const EpiArgs& e, int row_tile, int row_in_tile, int to
     const int half = e.hd >> 1;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const int pos = s_pos[col0 + j];
+      const int pos = s_rpos[col0 + j];
       const float2 cs = (sec < 2 && pos >= 0)
                             ? __ldg(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)])
                             : make_float2(1.f, 0.f);
@@ -376,12 +377,22 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
   }
 }
 
+// RoPE position of row r (0-based in its sequence's forward) relative to the first row's
+// position.  Plain forwards: r.  Quadratic self-speculation (quad_k = k): rows 0..k verify
+// [x_n, d_1..d_k] at offsets 0..k; row k+1+a*k+j (pre-draft block a = 0..k, slot j = 0..k-1)
+// sits at offset a+1+j, while its K/V goes to slot r like every row.
+NLD_DEV int rope_offset(int r, int quad_k) {
+  if (quad_k <= 0 || r <= quad_k) return r;
+  const int q = r - quad_k - 1;
+  return q / quad_k + 1 + q % quad_k;
+}
+
 // Per-column data of a tile of n token columns starting at tok0 (see epi_chunk): 1/rms from
 // the RMSNorm statistics when `norm` (lane l of a warp sums tiles l, l+32, ... of 8 tokens at
-// once, then a shuffle reduction finishes each token), and for the QKV epilogue the position
-// and KV page of each token.  nthr threads (a multiple of 32) share the work.
+// once, then a shuffle reduction finishes each token), and for the QKV epilogue the KV slot, its
+// page and the RoPE position of each token.  nthr threads (a multiple of 32) share the work.
 NLD_DEV void compute_tile_meta(const EpiArgs& e, int tok0, int n, bool norm, float* s_inv,
-                               int* s_pos, int* s_pg, int et, int nthr) {
+                               int* s_pos, int* s_pg, int* s_rpos, int et, int nthr) {
   const int nw = nthr >> 5, w = et >> 5, lane = et & 31;
   if (norm) {
     for (int c0 = w; c0 < n; c0 += nw * 8) {
@@ -408,19 +419,22 @@ NLD_DEV void compute_tile_meta(const EpiArgs& e, int tok0, int n, bool norm, flo
   if (e.kind == EPI_QKV) {
     for (int c = et; c < n; c += nthr) {
       const int tok = tok0 + c;
-      int pos = -1, pg = 0;
+      int pos = -1, pg = 0, rpos = -1;
       if (tok < e.M) {
         const int b = tok / e.m;
-        pos = __ldg(&e.lens[b]) + (tok - b * e.m);
+        const int len = __ldg(&e.lens[b]);
+        pos = len + (tok - b * e.m);
+        rpos = len + rope_offset(tok - b * e.m, e.quad_k);
         if (pos >= e.kv_cap || pos < 0) {
           set_err(e.err, NLD_DEVERR_KV_OVERFLOW);
-          pos = -1;
+          pos = rpos = -1;
         } else {
           pg = __ldg(&e.page_table[b * e.pps + (pos >> 6)]);
         }
       }
       s_pos[c] = pos;
       s_pg[c] = pg;
+      s_rpos[c] = rpos;
     }
   }
 }

@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(128)
   __shared__ float s_inv[16];
   __shared__ int s_pos[16];
   __shared__ int s_pg[16];
+  __shared__ int s_rpos[16];
   __shared__ float red_f[96];
   __shared__ int red_i[96];
   pdl_wait();
@@ -22,7 +23,7 @@ __global__ void __launch_bounds__(128)
   const int rt = blockIdx.x;
   const int tok0 = blockIdx.y * 16;
   const int tid = threadIdx.x;
-  compute_tile_meta(e, tok0, 16, e.kind != EPI_RESID, s_inv, s_pos, s_pg, tid, 128);
+  compute_tile_meta(e, tok0, 16, e.kind != EPI_RESID, s_inv, s_pos, s_pg, s_rpos, tid, 128);
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.f;
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(128)
     __syncthreads();
   }
   EpiPre pre;
-  epi_preload(e, rt, tid, tok0, s_pos, 0, pre);
+  epi_preload(e, rt, tid, tok0, s_rpos, 0, pre);
   epi_chunk<float>(e, rt, tid, tid & 31, tid >> 5, tok0, s_inv, s_pos, s_pg, 0, acc, pre, red_f, red_i, 1);
 }
 

@@ -43,7 +43,6 @@ namespace {
 
 constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB: one k-tile of bf16 weights
 constexpr int kMaxStages = 8;
-constexpr int kBoundaryPrefetch = 16;   // weight boxes prefetched into L2 per phase boundary
 constexpr int kSlotLd = 20;              // floats per row of a split-K slot: 16 + 4 (16-byte
                                          // accesses of 8 consecutive rows hit distinct banks)
 constexpr int kSlotFloats = kTileRows * kSlotLd;
@@ -65,6 +64,7 @@ struct GemmTail {
   float inv[kMaxNT];
   int pos[kMaxNT];
   int pg[kMaxNT];
+  int rpos[kMaxNT];
   float red_f[2][96];   // per epilogue half
   int red_i[2][96];
 };
@@ -132,13 +132,14 @@ NLD_DEV void tmem_ld_chunk(uint32_t tbase, int c, int hilo, float (&v)[16]) {
     tmem_ld16(tbase + c * 16, v);
     return;
   }
-  float a[16], b[16];
-  tmem_ld16(tbase + c * 32, a);
-  tmem_ld16(tbase + c * 32 + 16, b);
+  uint32_t a[16], b[16];
+  tmem_ld16_nowait(tbase + c * 32, a);
+  tmem_ld16_nowait(tbase + c * 32 + 16, b);
+  tmem_ld_wait();
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    v[j] = a[2 * j] + a[2 * j + 1];
-    v[8 + j] = b[2 * j] + b[2 * j + 1];
+    v[j] = __uint_as_float(a[2 * j]) + __uint_as_float(a[2 * j + 1]);
+    v[8 + j] = __uint_as_float(b[2 * j]) + __uint_as_float(b[2 * j + 1]);
   }
 }
 
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t t0 = globaltimer_ns();
             int npf = 0;
             while (ld_acquire_gpu(A.bar + (p - 1)) < G) {
-              if (npf < kBoundaryPrefetch && tn < w.tiles) {
+              if (npf < A.boundary_pf && tn < w.tiles) {
                 const int rn = tn / P.tok_tiles;
                 if (P.w_rowmajor)
                   tma_prefetch_l2_2d(&P.tmW, ktn * kTileK, rn * kTileRows);
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tb = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         named_bar_sync(1, kEpiThreads);
-        compute_tile_meta(e, tok0, NT, need_norm, tail->inv, tail->pos, tail->pg, et, kEpiThreads);
+        compute_tile_meta(e, tok0, NT, need_norm, tail->inv, tail->pos, tail->pg, tail->rpos, et, kEpiThreads);
         // Split tile: the group's s ranks each hold a partial sum of the whole tile.  Rank g
         // owns chunks [g*per, (g+1)*per): every rank sends its partial of those chunks to g with
         // st.async (one-way, counted by g's rfull transaction count) and g sums the s partials
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         EpiPre pre;
         if (w.s > 1) {
           named_bar_sync(1, kEpiThreads);   // the tile's positions (QKV) are in shared memory
-          if (cm < c_hi) epi_preload(e, r, row_in_tile, tok0 + cm * 16, tail->pos, cm * 16, pre);
+          if (cm < c_hi) epi_preload(e, r, row_in_tile, tok0 + cm * 16, tail->rpos, cm * 16, pre);
           // every other owner of this tile has reduced the group's previous split tile of this
           // phase (earlier phases: the grid-wide phase counter), so its slots are free
           if (et < w.s && et != w.grank && et * per < nchunks) {
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w.s == 1) {
           for (int c = half; c < nchunks; c += 2) {
             EpiPre pre;
-            epi_preload(e, r, row_in_tile, tok0 + c * 16, tail->pos, c * 16, pre);
+            epi_preload(e, r, row_in_tile, tok0 + c * 16, tail->rpos, c * 16, pre);
             float v[16];
             tmem_ld_chunk(tbase, c, A.hilo, v);
             epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,

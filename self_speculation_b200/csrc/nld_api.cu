@@ -140,12 +140,14 @@ struct nld_ctx {
   // chain tuning (profiling hook): stage cap (0 = as many as fit), k-tiles per stage
   int chain_stage_cap = 0;
   int chain_kps = 0;   // k-tiles per stage (0 = the planner's choice)
+  int chain_boundary_pf = 16;   // weight boxes prefetched into L2 per CTA at a phase boundary
   // host-side sequence bookkeeping
   int batch = 0;
   bool started = false;
   bool verify_fresh = false;
   bool fill_pending = false;   // a complete diffusion block whose causal KV fill is deferred
   bool nl_active = false;      // per-sequence diffusion ran: fills may be due on the device
+  bool quad_ready = false;     // the drafts on the device came from the last quadratic round
   long long len_upper = 0;
   uint64_t timeout_ns = 2000000000ull;
   std::string msg;
@@ -395,6 +397,7 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
   }
   A.bar = bar;
   A.trace = trace;
+  A.boundary_pf = x->chain_boundary_pf;
   A.tmWn = A.ph[0].tmW;
   if (next_pr && next_nph > 0) {
     int ngrid = 0;
@@ -471,6 +474,7 @@ struct FwdSpec {
   bool last_chunk;
   int causal_rows;   // attention: leading strictly causal rows (fused diffusion fill)
   const int* causal_seq;   // per-sequence diffusion: sequences whose rows are all causal
+  int quad_k;        // quadratic self-speculation forward with block k (0 = off)
 };
 
 // Launch one forward (no finalize).
@@ -517,6 +521,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.err = x->err;
   aa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(x->c.head_dim)));
   aa.hilo = x->bf16 ? 1 : 0;
+  aa.quad_k = f.quad_k;
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa);
   } else {
@@ -528,6 +533,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   const int L = x->c.n_layers;
   auto proj = [&](int which, int layer) {
     ProjRef r{which, layer, base_epi(x, M, f.m)};
+    r.e.quad_k = f.quad_k;
     static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
     r.e.kind = kinds[which];
     if (which == GW_QKV)
@@ -562,7 +568,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
     }
     // LoRA drafter: the block-bidirectional rows (the fused fill's causal rows excluded)
     if (x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF ||
-                          f.mode == FWD_NLDIFF))
+                          f.mode == FWD_NLDIFF || f.mode == FWD_QUAD))
       CK(launch_lora(x->stream, x->lora_A[l], x->lora_B[l], x->attn, x->lora_zp, x->h, M, x->qd,
                      x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, f.causal_seq,
                      x->bf16, x->bf16, pdl));
@@ -1063,6 +1069,7 @@ nld_status nld_prefill(nld_ctx* x, const int32_t* d_tokens, int stride, const in
   x->len_upper = rows;
   x->started = true;
   x->verify_fresh = false;
+  x->quad_ready = false;
   x->fill_pending = false;
   return NLD_OK;
 }
@@ -1090,6 +1097,7 @@ nld_status nld_ar_step(nld_ctx* x, int32_t* d_tokens_out) {
   }));
   x->len_upper += 1;
   x->verify_fresh = false;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1123,6 +1131,7 @@ nld_status nld_selfspec_draft_verify(nld_ctx* x) {
   std::vector<uintptr_t> key = {2, static_cast<uintptr_t>(x->batch)};
   TRY(run_graph(x, key, [&]() { return draft_verify_body(x); }));
   x->verify_fresh = true;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1136,6 +1145,7 @@ nld_status nld_kv_commit(nld_ctx* x, const int32_t* d_nrows, int32_t* d_tokens_o
   TRY(finalize(x, a));
   x->len_upper += x->c.block_k + 1;
   x->verify_fresh = false;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1156,6 +1166,75 @@ nld_status nld_selfspec_round(nld_ctx* x, int32_t* d_tokens_out, int32_t* d_ncom
   }));
   x->len_upper += x->c.block_k + 1;
   x->verify_fresh = false;
+  x->quad_ready = false;
+  return NLD_OK;
+}
+
+// The quadratic self-speculation forward over the current drafts (no finalize): (k+1)^2 rows per
+// sequence, the verify rows and the k+1 pre-draft blocks.
+static nld_status quad_forward(nld_ctx* x, int lm, float* logits) {
+  const int k = x->c.block_k;
+  FwdSpec f{};
+  f.mode = FWD_QUAD;
+  f.B = x->batch;
+  f.m = (k + 1) * (k + 1);
+  f.bs = 1;
+  f.causal_rows = k + 1;   // the verify rows; the LoRA drafter takes the pre-draft rows
+  f.quad_k = k;
+  f.lm = lm;
+  f.logits = logits;
+  return launch_forward(x, f);
+}
+
+// Checks shared by the quadratic entry points: the forward's batch x (k+1)^2 rows fit the
+// activation buffers, and its rows' K/V slots (len .. len+(k+1)^2-1) fit the KV capacity.
+static nld_status quad_check(nld_ctx* x) {
+  const int k = x->c.block_k, m = (k + 1) * (k + 1);
+  if (static_cast<long long>(x->batch) * m > x->M_max)
+    return fail(x, NLD_ERR_UNSUPPORTED, "a quadratic forward needs batch x (k+1)^2 = %d x %d rows <= %d",
+                x->batch, m, x->M_max);
+  return ensure_capacity(x, m - k - 1);   // kv_cap >= max_seq + k + 1
+}
+
+nld_status nld_quadratic_round(nld_ctx* x, int32_t* d_tokens_out, int32_t* d_ncommit_out) {
+  TRY(need_started(x));
+  TRY(flush_fill(x));
+  TRY(quad_check(x));
+  const int k = x->c.block_k;
+  if (!x->quad_ready) {
+    // the first round after any other call starts from one linear draft forward
+    std::vector<uintptr_t> dkey = {11, static_cast<uintptr_t>(x->batch)};
+    TRY(run_graph(x, dkey, [&]() -> nld_status {
+      const long long saved = x->len_upper;
+      x->len_upper = x->c.max_seq;
+      FwdSpec f{};
+      f.mode = FWD_DRAFT;
+      f.B = x->batch;
+      f.m = k;
+      f.bs = k;
+      f.lm = LM_ARGMAX;
+      nld_status s = launch_forward(x, f);
+      x->len_upper = saved;
+      if (s != NLD_OK) return s;
+      return finalize(x, base_fin(x, FWD_DRAFT, k));
+    }));
+  }
+  std::vector<uintptr_t> key = {10, static_cast<uintptr_t>(x->batch), reinterpret_cast<uintptr_t>(d_tokens_out),
+                                reinterpret_cast<uintptr_t>(d_ncommit_out)};
+  TRY(run_graph(x, key, [&]() -> nld_status {
+    const long long saved = x->len_upper;
+    x->len_upper = x->c.max_seq;
+    nld_status s = quad_forward(x, LM_ARGMAX, nullptr);
+    x->len_upper = saved;
+    if (s != NLD_OK) return s;
+    FinalizeArgs a = base_fin(x, FWD_QUAD, (k + 1) * (k + 1));
+    a.tokens_out = d_tokens_out;
+    a.ncommit_out = d_ncommit_out;
+    return finalize(x, a);
+  }));
+  x->len_upper += k + 1;
+  x->verify_fresh = false;
+  x->quad_ready = true;
   return NLD_OK;
 }
 
@@ -1298,6 +1377,7 @@ nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_
   }
   if (h_filled_out) *h_filled_out = filled;
   x->verify_fresh = false;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1319,6 +1399,7 @@ nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_
   if (open == 0) x->fill_pending = true;   // this block's fill joins the next step
   if (h_filled_out) *h_filled_out = fused ? 1 : 0;
   x->verify_fresh = false;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1329,6 +1410,7 @@ nld_status nld_diffuse_step_nonlockstep(nld_ctx* x, float threshold, int32_t* d_
   TRY(run_nl(x, false, threshold, d_block_out, d_conf_out, d_ncommit_out, d_state_out));
   x->nl_active = true;
   x->verify_fresh = false;
+  x->quad_ready = false;
   return NLD_OK;
 }
 
@@ -1337,6 +1419,13 @@ nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
   TRY(flush_fill(x));
   if (!d_logits_out) return fail(x, NLD_ERR_ARG, "logits is NULL");
   const int k = x->c.block_k;
+  if (mode == NLD_MODE_QUAD) {
+    // the quadratic forward over the current drafts; nothing is recorded or committed
+    TRY(quad_check(x));
+    TRY(quad_forward(x, LM_LOGITS, d_logits_out));
+    x->quad_ready = false;
+    return NLD_OK;
+  }
   FwdSpec f{};
   f.B = x->batch;
   f.lm = LM_LOGITS;
@@ -1359,6 +1448,7 @@ nld_status nld_debug_logits(nld_ctx* x, int mode, float* d_logits_out) {
   FinalizeArgs a = base_fin(x, fm, f.m);
   a.commit = 0;
   TRY(finalize(x, a));
+  x->quad_ready = false;
   if (mode == NLD_MODE_VERIFY) x->verify_fresh = true;
   return NLD_OK;
 }
@@ -1456,15 +1546,17 @@ nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out)
   return NLD_OK;
 }
 
-nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage) {
+nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage, int boundary_prefetch) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (stage_cap < 0 || stage_cap == 1 || stage_cap == 2 || stage_cap > gemm_chain_max_stages() ||
-      k_tiles_per_stage < 0 || k_tiles_per_stage > 2)
-    return fail(x, NLD_ERR_ARG, "stage cap 0 or 3..%d, k-tiles per stage 0..2", gemm_chain_max_stages());
+      k_tiles_per_stage < 0 || k_tiles_per_stage > 2 || boundary_prefetch < 0 || boundary_prefetch > 256)
+    return fail(x, NLD_ERR_ARG, "stage cap 0 or 3..%d, k-tiles per stage 0..2, boundary prefetch 0..256",
+                gemm_chain_max_stages());
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);   // captured graphs hold the old launch parameters
   x->chain_stage_cap = stage_cap;
   x->chain_kps = k_tiles_per_stage;
+  x->chain_boundary_pf = boundary_prefetch;
   return NLD_OK;
 }
 
@@ -1489,6 +1581,7 @@ nld_status nld_debug_timeout_chain(nld_ctx* x, unsigned long long timeout_ns) {
     A.ph[p].e.n_rows = w.n_rows;
   }
   A.bar = x->bars + kMaxPhases;   // layer 0's counters (left zero by every launch)
+  A.boundary_pf = x->chain_boundary_pf;
   A.tmWn = A.ph[0].tmW;
   A.dbg_skip_arrive = 1;
   CK(launch_gemm_chain(x->stream, A, grid, timeout_ns, false));

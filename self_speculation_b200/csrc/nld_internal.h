@@ -30,7 +30,8 @@ enum FwdMode : int {
   FWD_COMMIT = 6,
   FWD_FILLDIFF = 7,  // fused diffusion KV fill: [x_n, b_1..b_k, MASK x (k-1)], 2k rows
   FWD_NLDIFF = 8,    // per-sequence diffusion: flagged sequences fill, the others denoise
-  FWD_NLFILL = 9     // per-sequence diffusion: flagged sequences fill, the others keep state
+  FWD_NLFILL = 9,    // per-sequence diffusion: flagged sequences fill, the others keep state
+  FWD_QUAD = 10      // quadratic self-speculation: verify rows + (k+1) pre-draft blocks, (k+1)^2 rows
 };
 
 // Per (token, vocab tile) partial of the LM-head reduction.
@@ -75,6 +76,8 @@ struct EpiArgs {
   float* logits;    // [M, V]
   int V;
   int hilo;         // bf16 storage: hb / u written as (hi, lo) row pairs [2M, ld], q in fp32
+  int quad_k;       // quadratic self-speculation forward with block k: RoPE positions of the
+                    // pre-draft rows differ from their KV slots (0 = every other forward)
   int* err;
 };
 
@@ -109,6 +112,7 @@ struct alignas(64) ChainArgs {
   unsigned* bar;    // [kMaxPhases] phase-boundary arrival counters + exit counter (last slot);
                     // zero before the launch, left zero by it
   unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
+  int boundary_pf;  // weight boxes each CTA prefetches into L2 while it waits at a phase boundary
   int dbg_skip_arrive;   // test hook: CTA 0 withholds its phase-0 arrival, so every wait on that
                          // counter runs into its time limit (the failure-detection test)
   // the next chain launch's first phase (L2 warm-up of each CTA's first weight boxes there)
@@ -132,6 +136,8 @@ struct AttnArgs {
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   float scale_log2;     // log2(e) / sqrt(hd)
   int hilo;             // tensor-core path: q fp32 [M, Hq, hd], out (hi, lo) bf16 rows [2M, Hq, hd]
+  int quad_k;           // quadratic self-speculation forward with block k (0 = off): rows 0..k are
+                        // causal; pre-draft row k+1+a*k+j sees the prefix, rows 0..a and its block
   int* err;
 };
 

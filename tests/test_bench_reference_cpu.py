@@ -12,9 +12,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _run(env_extra):
     env = dict(os.environ, **env_extra)
+    # one layer of the 8B shape keeps the host work of this check to seconds; the arm itself
+    # runs all 36 layers by default
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
-                        "--warmup", "3"], cwd=ROOT, env=env, capture_output=True, text=True,
-                       timeout=600)
+                        "--warmup", "3", "--ref-layers", "1"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     return [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
 
@@ -33,7 +35,7 @@ def test_reference_line_keys_and_values():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
-    assert "workload" in d["config"]
+    assert "workload" in d["config"] and d["config"]["layers"] == 1
 
 
 def test_reference_other_ranks_print_nothing():
