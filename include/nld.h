@@ -304,10 +304,18 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
  * use as many shared-memory stages as fit, else at most stage_cap (3..8); k_tiles_per_stage =
  * 1 or 2 weight boxes (16 KB each) per ring stage (0 = the planner's choice);
  * boundary_prefetch = weight boxes each CTA prefetches into L2 while it waits at a phase
- * boundary (0..256; 16 at creation).  Synchronises and drops the captured graphs; later calls
- * use the new values. */
+ * boundary (0..256; 16 at creation); act_3d = 1 loads a stage's activation k-tiles with one
+ * 3D box (the default), 0 with one 2D box per k-tile; runahead_stages = D > 0 prefetches the
+ * weights of the stage D ahead of each load into L2 (0..16; 0 = off).  Synchronises and drops
+ * the captured graphs; later calls use the new values. */
 nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_stage,
-                                  int boundary_prefetch);
+                                  int boundary_prefetch, int act_3d, int runahead_stages);
+
+/* Profiling hook: attention planning.  rows_per_cta (16..144) caps the query rows (positions x
+ * query heads of one kv head) a CTA holds, so smaller values give more, lighter CTAs;
+ * min_tiles_per_split (1..8) is the fewest 64-key tiles a KV split takes (more splits merge more
+ * partials).  Defaults 144 and 2.  Synchronises and drops the captured graphs. */
+nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
 
 /* Test hook for failure detection: one launch of layer 0's four-phase chain over the current
  * batch (scratch buffers only, as nld_time_chain) with every bounded wait limited to timeout_ns

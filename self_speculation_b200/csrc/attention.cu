@@ -145,8 +145,8 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     kv_end = max(v1, h2) + 1;
   }
   const int n_tiles = (kv_end + kPage - 1) / kPage;
-  // at least two KV tiles per split: fewer, fuller splits keep the merge short
-  const int per = max(2, (n_tiles + a.S - 1) / a.S);
+  // at least min_tiles KV tiles per split: fewer, fuller splits keep the merge short
+  const int per = max(a.min_tiles, (n_tiles + a.S - 1) / a.S);
   const int t_lo = split * per;
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
   __syncthreads();
@@ -174,26 +174,47 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     for (int i = n_pre; i < min(kAttStages, ntile); ++i) issue(i);
   __syncwarp();
 
-  // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row)
+  // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row); each
+  // thread issues the global loads of kQB chunks before storing any, so they are in flight together
   const int rows_pad = a.NW * 16;
-  for (int e = tid; e < rows_pad * 16; e += nthr) {
-    const int r = e >> 4, c = e & 15;
-    const int p = r / a.G, gq = r - p * a.G;
-    uint4 val = make_uint4(0, 0, 0, 0), vlo = make_uint4(0, 0, 0, 0);
-    if (r < a.rows && p < np) {
-      const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
-      const size_t off = ((tok * a.Hq) + g * a.G + gq) * 128 + c * 8;
-      if constexpr (kHiLo) {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
-        const float4 x0 = src[0], x1 = src[1];
-        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        split8(xs, val, vlo);
-      } else {
-        val = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+  constexpr int kQB = 4;
+  for (int e0 = tid; e0 < rows_pad * 16; e0 += kQB * nthr) {
+    float4 x0[kQB], x1[kQB];
+    uint4 xb[kQB];
+    bool ok[kQB];
+#pragma unroll
+    for (int u = 0; u < kQB; ++u) {
+      const int e = e0 + u * nthr;
+      const int r = e >> 4, c = e & 15;
+      const int p = r / a.G, gq = r - p * a.G;
+      ok[u] = (e < rows_pad * 16) && r < a.rows && p < np;
+      x0[u] = x1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      xb[u] = make_uint4(0, 0, 0, 0);
+      if (ok[u]) {
+        const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
+        const size_t off = ((tok * a.Hq) + g * a.G + gq) * 128 + c * 8;
+        if constexpr (kHiLo) {
+          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
+          x0[u] = src[0];
+          x1[u] = src[1];
+        } else {
+          xb[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+        }
       }
     }
-    *reinterpret_cast<uint4*>(sQ + r * 256 + ((c ^ (r & 7)) << 4)) = val;
-    if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQl + r * 256 + ((c ^ (r & 7)) << 4)) = vlo;
+#pragma unroll
+    for (int u = 0; u < kQB; ++u) {
+      const int e = e0 + u * nthr;
+      if (e >= rows_pad * 16) break;
+      const int r = e >> 4, c = e & 15;
+      uint4 val = xb[u], vlo = make_uint4(0, 0, 0, 0);
+      if constexpr (kHiLo) {
+        const float xs[8] = {x0[u].x, x0[u].y, x0[u].z, x0[u].w, x1[u].x, x1[u].y, x1[u].z, x1[u].w};
+        split8(xs, val, vlo);
+      }
+      *reinterpret_cast<uint4*>(sQ + r * 256 + ((c ^ (r & 7)) << 4)) = val;
+      if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQl + r * 256 + ((c ^ (r & 7)) << 4)) = vlo;
+    }
   }
   __syncthreads();
 

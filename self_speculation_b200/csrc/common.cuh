@@ -84,6 +84,14 @@ NLD_DEV void tma_load_2d(void* dst, const void* map, uint64_t* bar, int c0, int 
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// 3D tiled load (no multicast) of box [c0.., c1.., c2..] into shared memory, completing on `bar`.
+NLD_DEV void tma_load_3d(void* dst, const void* map, uint64_t* bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // Same with an L2 eviction-priority hint (evict_first for data read once: weights).
 NLD_DEV void tma_load_2d_hint(void* dst, const void* map, uint64_t* bar, int c0, int c1,
                               uint64_t policy) {
@@ -92,6 +100,21 @@ NLD_DEV void tma_load_2d_hint(void* dst, const void* map, uint64_t* bar, int c0,
       "cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
+}
+// Plain bulk copy (no tensor map) of `bytes` contiguous bytes global -> shared, completing on
+// `bar`, with an L2 eviction-priority hint.  Both addresses 16-byte aligned, bytes a multiple of 16.
+NLD_DEV void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// Prefetch `bytes` contiguous bytes into L2 (16-byte aligned, a multiple of 16).
+NLD_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
 }
 // Prefetch a 2D tensor box into L2 (no shared-memory destination, no completion tracking).
 NLD_DEV void tma_prefetch_l2_2d(const void* map, int c0, int c1) {

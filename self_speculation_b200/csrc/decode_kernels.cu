@@ -487,19 +487,28 @@ __global__ void __launch_bounds__(128) lora_up_kernel(const T* B, const float* z
   const int i = blockIdx.x * 128 + threadIdx.x;
   const int t0 = blockIdx.y * 8;
   const int nt = min(8, M - t0);
-  // the 8 token rows of a partial are contiguous (8*r floats): element e = tt*r + j; each
-  // slice's loads of all of a thread's elements are independent, summed in slice order
-  constexpr int kQ = 8 * 256 / 128;
+  // the 8 token rows of a partial are contiguous (8*r floats): element e = tt*r + j.  Four
+  // slices' loads of all of a thread's elements are issued before any is summed (64 loads in
+  // flight), and the sums run in slice order (deterministic)
+  constexpr int kQ = 8 * 256 / 128, kS = 4;
   float za[kQ];
 #pragma unroll
   for (int q = 0; q < kQ; ++q) za[q] = 0.f;
-  for (int ks = 0; ks < n_ks; ++ks) {
-    const float* zk = zp + (static_cast<size_t>(ks) * M + t0) * r;
+  for (int ks0 = 0; ks0 < n_ks; ks0 += kS) {
+    float t[kS][kQ];
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) {
-      const int e = q * 128 + threadIdx.x;
-      if (e < nt * r) za[q] += zk[e];
+    for (int u = 0; u < kS; ++u) {
+      const float* zk = zp + (static_cast<size_t>(ks0 + u) * M + t0) * r;
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        const int e = q * 128 + threadIdx.x;
+        t[u][q] = (ks0 + u < n_ks && e < nt * r) ? zk[e] : 0.f;
+      }
     }
+#pragma unroll
+    for (int u = 0; u < kS; ++u)
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) za[q] += t[u][q];
   }
 #pragma unroll
   for (int q = 0; q < kQ; ++q) {
@@ -595,6 +604,10 @@ cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const voi
 // follows the norm).  Row-major dst[r, c], or, with `tiled`, the streaming layout of the
 // tensor-core GEMM: 128-row x 64-column blocks stored contiguously (16 KB of bf16 each), block
 // (row tile rt, k tile kt) at element offset (rt * KT + kt) * 8192, rows past n_rows zero.
+// Each block holds the byte image the MMA reads from shared memory: row r of the block is 128
+// bytes at r * 128 whose eight 16-byte pieces are permuted by the 128-byte swizzle (piece p of
+// the row stored at position p ^ (r & 7)), so one plain bulk copy of consecutive blocks into a
+// 1024-byte-aligned buffer gives the K-major swizzled operand.
 template <typename T>
 __global__ void repack_kernel(T* __restrict__ dst, const T* __restrict__ src,
                               const int* __restrict__ row_map, int n_rows, int K,
@@ -611,8 +624,11 @@ __global__ void repack_kernel(T* __restrict__ dst, const T* __restrict__ src,
       const int in = static_cast<int>(idx - blk * (kTileRows * kTileK));
       const int rt = static_cast<int>(blk / KT);
       const int kt = static_cast<int>(blk - static_cast<size_t>(rt) * KT);
-      r = rt * kTileRows + in / kTileK;
-      c = kt * kTileK + in % kTileK;
+      // position `in` of the block: row in / 64, 16-byte piece (in % 64) / 8 holds the source
+      // piece ((in % 64) / 8) ^ (row & 7)
+      const int rr = in / kTileK, pc = ((in % kTileK) >> 3) ^ (rr & 7);
+      r = rt * kTileRows + rr;
+      c = kt * kTileK + pc * 8 + (in & 7);
     } else {
       r = static_cast<int>(idx / K);
       c = static_cast<int>(idx - static_cast<size_t>(r) * K);

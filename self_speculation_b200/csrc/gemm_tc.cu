@@ -245,6 +245,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       int n_issued = 0;   // stages whose loads were issued
       bool ok = true;
+      // L2 run-ahead (A.pf_stages = D > 0, pre-tiled weights): after the load of stage `it` is
+      // issued, the weights of stage it + D are prefetched into L2 with one bulk prefetch of their
+      // contiguous blocks, so the load of that stage finds them there.  The cursor walks the
+      // same (phase, tile, k) order as the loads; divisions only where it enters a phase.
+      struct PfCursor {
+        int p, t, kt, k_lo, k_hi, ngrp, tiles, tok_tiles, KT;
+        const uint8_t* W;
+        bool live;
+      } pf{};
+      auto pf_phase = [&](int q) {
+        pf.live = false;
+        for (; q < A.nph; ++q) {
+          const PhaseArgs& Q = A.ph[q];
+          if (Q.w_rowmajor) return;
+          const Work wq = work_of(A, q, cl, rank, C);
+          if (wq.grp < wq.tiles) {
+            pf = {q, wq.grp, wq.k_lo, wq.k_lo, wq.k_hi, wq.ngrp, wq.tiles, Q.tok_tiles, Q.KT,
+                  static_cast<const uint8_t*>(Q.W), true};
+            return;
+          }
+        }
+      };
+      auto pf_step = [&](bool issue) {
+        if (!pf.live) return;
+        if (issue) {
+          const int r = (pf.tok_tiles == 1) ? pf.t : pf.t / pf.tok_tiles;
+          bulk_prefetch_l2(pf.W + (static_cast<size_t>(r) * pf.KT + pf.kt) * kStageW,
+                           static_cast<uint32_t>(min(KPS, pf.k_hi - pf.kt) * kStageW));
+        }
+        pf.kt += KPS;
+        if (pf.kt >= pf.k_hi) {
+          pf.kt = pf.k_lo;
+          pf.t += pf.ngrp;
+          if (pf.t >= pf.tiles) pf_phase(pf.p + 1);
+        }
+      };
+      if (A.pf_stages > 0) {
+        // the first S stages fill the ring at once: the run-ahead starts after them
+        pf_phase(0);
+        for (int i = 0; i < S; ++i) pf_step(false);
+        for (int i = 0; i < A.pf_stages; ++i) pf_step(true);
+      }
       for (int p = 0; ok && p < A.nph; ++p) {
         const PhaseArgs& P = A.ph[p];
         const Work w = work_of(A, p, cl, rank, C);
@@ -267,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (P.w_rowmajor)
                   tma_prefetch_l2_2d(&P.tmW, ktn * kTileK, rn * kTileRows);
                 else
-                  tma_prefetch_l2_2d(&P.tmW, 0, (rn * P.KT + ktn) * kTileRows);
+                  bulk_prefetch_l2(static_cast<const uint8_t*>(P.W) +
+                                       (static_cast<size_t>(rn) * P.KT + ktn) * kStageW, kStageW);
                 ++npf;
                 if (++ktn >= w.k_hi) {
                   tn += w.ngrp;
@@ -281,10 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_global();
           }
-          for (int i = 0; i < nq; ++i)
-            for (int j = 0; j < q_nk[i]; ++j)
-              tma_load_2d(sX + q_stage[i] * xst + j * xbytes, &P.tmX, &tail->full[q_stage[i]],
-                          (q_k[i] + j) * kTileK, q_tt[i] * NN);
+          for (int i = 0; i < nq; ++i) {
+            if (P.x3d) {
+              tma_load_3d(sX + q_stage[i] * xst, &P.tmX, &tail->full[q_stage[i]], 0, q_tt[i] * NN, q_k[i]);
+            } else {
+              for (int j = 0; j < q_nk[i]; ++j)
+                tma_load_2d(sX + q_stage[i] * xst + j * xbytes, &P.tmX, &tail->full[q_stage[i]],
+                            (q_k[i] + j) * kTileK, q_tt[i] * NN);
+            }
+          }
           nq = 0;
           ready = true;
           return true;
@@ -305,21 +353,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kt == w.k_lo && t == w.grp) trace_mark(A, 2 + 3 * p);
             trace_iter(A, 2, it - S);
             trace_iter(A, 0, it);
-            mbar_arrive_expect_tx(&tail->full[stage], nk * (kStageW + xbytes));
-            // pre-tiled weights: block (r, kt) is one contiguous 16 KB box
-            for (int j = 0; j < nk; ++j) {
-              if (P.w_rowmajor)
+            // a 3D activation box always moves KPS k-tiles (zero-filled past the tensor)
+            mbar_arrive_expect_tx(&tail->full[stage], nk * kStageW + (P.x3d ? KPS : nk) * xbytes);
+            // pre-tiled weights: blocks (r, kt..kt+nk-1) are one contiguous stretch of nk x 16 KB
+            // stored as the swizzled shared-memory image, so one plain bulk copy loads the stage
+            if (P.w_rowmajor) {
+              for (int j = 0; j < nk; ++j)
                 tma_load_2d_hint(sW + stage * wst + j * kStageW, &P.tmW, &tail->full[stage],
                                  (kt + j) * kTileK, r * kTileRows, pol);
-              else
-                tma_load_2d_hint(sW + stage * wst + j * kStageW, &P.tmW, &tail->full[stage], 0,
-                                 (r * P.KT + kt + j) * kTileRows, pol);
+            } else {
+              bulk_load_hint(sW + stage * wst,
+                             static_cast<const uint8_t*>(P.W) + (static_cast<size_t>(r) * P.KT + kt) * kStageW,
+                             static_cast<uint32_t>(nk * kStageW), &tail->full[stage], pol);
             }
             n_issued = it + 1;
+            if (A.pf_stages > 0 && it >= S) pf_step(true);
             if (ready) {
-              for (int j = 0; j < nk; ++j)
-                tma_load_2d(sX + stage * xst + j * xbytes, &P.tmX, &tail->full[stage],
-                            (kt + j) * kTileK, tt * NN);
+              if (P.x3d) {
+                tma_load_3d(sX + stage * xst, &P.tmX, &tail->full[stage], 0, tt * NN, kt);
+              } else {
+                for (int j = 0; j < nk; ++j)
+                  tma_load_2d(sX + stage * xst + j * xbytes, &P.tmX, &tail->full[stage],
+                              (kt + j) * kTileK, tt * NN);
+              }
             } else {
               q_stage[nq] = stage;
               q_k[nq] = kt;
@@ -346,7 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nr = grp / A.next_tok_tiles;
           const int lo = (nrank % A.next_s) * A.next_ks;
           const int hi = min(A.next_KT, min(lo + A.next_ks, lo + A.next_boxes));
-          for (int kt = lo; kt < hi; ++kt) tma_prefetch_l2_2d(&A.tmWn, 0, (nr * A.next_KT + kt) * kTileRows);
+          if (hi > lo)
+            bulk_prefetch_l2(static_cast<const uint8_t*>(A.Wn) + (static_cast<size_t>(nr) * A.next_KT + lo) * kStageW,
+                             static_cast<uint32_t>((hi - lo) * kStageW));
         }
       }
       if (!ok) {

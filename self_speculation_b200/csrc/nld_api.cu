@@ -128,7 +128,10 @@ struct nld_ctx {
   std::vector<CUtensorMap> tmWqkv, tmWo, tmWgu, tmWd;
   CUtensorMap tmWlm{};
   CUtensorMap tmKV{};
-  std::map<std::pair<int, int>, CUtensorMap> tmX;
+  std::map<std::tuple<int, int, int>, std::pair<CUtensorMap, int>> tmX;   // (buffer, rows, kps) -> map, 3D
+  int chain_x3d = 1;   // activation loads of a stage as one 3D box (0: per k-tile 2D boxes)
+  int attn_rows_cap = 144;   // attention planning (profiling hook): query rows per CTA at most
+  int attn_min_tiles = 2;    // and KV tiles per split at least
   // graphs: one per (call, batch, output pointers), at most kMaxGraphs (least recently used
   // evicted); tick = the call count at each graph's last replay
   struct GraphEntry {
@@ -141,6 +144,7 @@ struct nld_ctx {
   int chain_stage_cap = 0;
   int chain_kps = 0;   // k-tiles per stage (0 = the planner's choice)
   int chain_boundary_pf = 16;   // weight boxes prefetched into L2 per CTA at a phase boundary
+  int chain_pf_stages = 0;      // L2 run-ahead distance in stages (0 = off)
   // host-side sequence bookkeeping
   int batch = 0;
   bool started = false;
@@ -229,16 +233,47 @@ struct ProjRef {
   EpiArgs e;
 };
 
-const CUtensorMap* xmap(nld_ctx* x, int buf, int rows) {
-  auto key = std::make_pair(buf, rows);
+// 3D bf16 tensor map over a row-major [rows, inner] matrix seen as [inner/64 blocks][rows][64]
+// (strides: a row inner*2 bytes, a block 128 bytes), box {64, box_rows, box_blocks}, 128-byte
+// swizzle: one load brings box_blocks consecutive 64-column k-tiles of box_rows rows, stored one
+// after the other ([block][row][64]), each as a 2D box would store it.
+bool make_map_act3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
+                    uint32_t box_blocks) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc || inner % 64) return false;
+  cuuint64_t dims[3] = {64, rows, inner / 64};
+  cuuint64_t strides[2] = {inner * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Tensor map of an activation buffer for loads of `rows` rows x `kps` k-tiles: the 3D form (one
+// load per stage) when the encoder accepts it, else the 2D form; *is3d tells which.
+const CUtensorMap* xmap(nld_ctx* x, int buf, int rows, int kps, int* is3d) {
+  auto key = std::make_tuple(buf, rows, kps);
   auto it = x->tmX.find(key);
-  if (it != x->tmX.end()) return &it->second;
+  if (it != x->tmX.end()) {
+    *is3d = it->second.second;
+    return &it->second.first;
+  }
   CUtensorMap m;
   const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
   const int inner = buf == XB_HB ? x->c.d_model : (buf == XB_ATTN ? x->qd : x->c.ffn_dim);
   // bf16 activations are (hi, lo) row pairs: 2 M_max rows
-  if (!make_map_bf16(&m, base, inner, 2ull * x->M_max, rows)) return nullptr;
-  return &(x->tmX[key] = m);
+  int d3 = 0;
+  if (x->chain_x3d && make_map_act3d(&m, base, inner, 2ull * x->M_max, rows, kps)) {
+    d3 = 1;
+  } else if (!make_map_bf16(&m, base, inner, 2ull * x->M_max, rows)) {
+    return nullptr;
+  }
+  auto& slot = x->tmX[key];
+  slot = std::make_pair(m, d3);
+  *is3d = d3;
+  return &slot.first;
 }
 
 // Weight matrix, its tensor map and shape of projection `which` of `layer`.
@@ -389,15 +424,19 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
   for (int p = 0; p < nph; ++p) {
     const WInfo w = winfo(x, pr[p].which, pr[p].layer);
     A.ph[p].tmW = *w.map;
-    const CUtensorMap* tmX = xmap(x, w.buf, A.xr);
+    A.ph[p].W = w.W;
+    int is3d = 0;
+    const CUtensorMap* tmX = xmap(x, w.buf, A.xr, A.kps, &is3d);
     if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
     A.ph[p].tmX = *tmX;
+    A.ph[p].x3d = is3d;
     A.ph[p].e = pr[p].e;
     A.ph[p].e.n_rows = w.n_rows;
   }
   A.bar = bar;
   A.trace = trace;
   A.boundary_pf = x->chain_boundary_pf;
+  A.pf_stages = x->chain_pf_stages;
   A.tmWn = A.ph[0].tmW;
   if (next_pr && next_nph > 0) {
     int ngrid = 0;
@@ -412,14 +451,22 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
     A.next_tiles = N.ph[0].row_tiles * N.ph[0].tok_tiles;
     A.next_boxes = N.stages * N.kps + 8;
     A.tmWn = *winfo(x, next_pr[0].which, next_pr[0].layer).map;
+    A.Wn = winfo(x, next_pr[0].which, next_pr[0].layer).W;
   }
   CK(launch_gemm_chain(x->stream, A, grid, x->timeout_ns, pdl));
   return NLD_OK;
 }
 
-void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a) {
+// rows_cap: query rows (positions x heads) per CTA at most (<= 144: 9 warps); min_tiles: KV tiles
+// a split takes at least.
+void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, int rows_cap = 144,
+               int min_tiles = 2) {
   a.G = Hq / Hkv;
-  a.QT = std::min(m, std::max(1, 144 / a.G));
+  a.min_tiles = min_tiles;
+  // query positions per CTA: as many as rows_cap allows, spread evenly over the query tiles
+  const int qt_max = std::min(m, std::max(1, rows_cap / a.G));
+  const int nq = (m + qt_max - 1) / qt_max;
+  a.QT = (m + nq - 1) / nq;
   a.q_tiles = (m + a.QT - 1) / a.QT;
   a.rows = a.QT * a.G;
   a.NW = (a.rows + 15) / 16;
@@ -429,7 +476,7 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   a.S = 1;
   if (units < 2 * sms)
-    a.S = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / 2)}));
+    a.S = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / min_tiles)}));
 }
 
 EpiArgs base_epi(nld_ctx* x, int M, int m) {
@@ -523,7 +570,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.hilo = x->bf16 ? 1 : 0;
   aa.quad_k = f.quad_k;
   if (x->bf16) {
-    attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa);
+    attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa, x->attn_rows_cap, x->attn_min_tiles);
   } else {
     aa.G = aa.Hq / aa.Hkv;
   }
@@ -1546,17 +1593,34 @@ nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out)
   return NLD_OK;
 }
 
-nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage, int boundary_prefetch) {
+nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage, int boundary_prefetch,
+                                  int act_3d, int runahead_stages) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (stage_cap < 0 || stage_cap == 1 || stage_cap == 2 || stage_cap > gemm_chain_max_stages() ||
-      k_tiles_per_stage < 0 || k_tiles_per_stage > 2 || boundary_prefetch < 0 || boundary_prefetch > 256)
-    return fail(x, NLD_ERR_ARG, "stage cap 0 or 3..%d, k-tiles per stage 0..2, boundary prefetch 0..256",
+      k_tiles_per_stage < 0 || k_tiles_per_stage > 2 || boundary_prefetch < 0 || boundary_prefetch > 256 ||
+      (act_3d != 0 && act_3d != 1) || runahead_stages < 0 || runahead_stages > 16)
+    return fail(x, NLD_ERR_ARG,
+                "stage cap 0 or 3..%d, k-tiles per stage 0..2, boundary prefetch 0..256, act_3d 0/1, run-ahead 0..16",
                 gemm_chain_max_stages());
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);   // captured graphs hold the old launch parameters
   x->chain_stage_cap = stage_cap;
   x->chain_kps = k_tiles_per_stage;
   x->chain_boundary_pf = boundary_prefetch;
+  if (x->chain_x3d != act_3d) x->tmX.clear();   // activation maps of the other form
+  x->chain_x3d = act_3d;
+  x->chain_pf_stages = runahead_stages;
+  return NLD_OK;
+}
+
+nld_status nld_debug_attention_tuning(nld_ctx* x, int rows_per_cta, int min_tiles_per_split) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  if (rows_per_cta < 16 || rows_per_cta > 144 || min_tiles_per_split < 1 || min_tiles_per_split > 8)
+    return fail(x, NLD_ERR_ARG, "rows per CTA 16..144, KV tiles per split 1..8");
+  CK(cudaStreamSynchronize(x->stream));
+  drop_graphs(x);
+  x->attn_rows_cap = rows_per_cta;
+  x->attn_min_tiles = min_tiles_per_split;
   return NLD_OK;
 }
 
@@ -1574,14 +1638,18 @@ nld_status nld_debug_timeout_chain(nld_ctx* x, unsigned long long timeout_ns) {
   for (int p = 0; p < 4; ++p) {
     const WInfo w = winfo(x, pr[p].which, pr[p].layer);
     A.ph[p].tmW = *w.map;
-    const CUtensorMap* tmX = xmap(x, w.buf, A.xr);
+    A.ph[p].W = w.W;
+    int is3d = 0;
+    const CUtensorMap* tmX = xmap(x, w.buf, A.xr, A.kps, &is3d);
     if (!tmX) return fail(x, NLD_ERR_CUDA, "tensor map encode failed (activation buffer)");
     A.ph[p].tmX = *tmX;
+    A.ph[p].x3d = is3d;
     A.ph[p].e = pr[p].e;
     A.ph[p].e.n_rows = w.n_rows;
   }
   A.bar = x->bars + kMaxPhases;   // layer 0's counters (left zero by every launch)
   A.boundary_pf = x->chain_boundary_pf;
+  A.pf_stages = x->chain_pf_stages;
   A.tmWn = A.ph[0].tmW;
   A.dbg_skip_arrive = 1;
   CK(launch_gemm_chain(x->stream, A, grid, timeout_ns, false));

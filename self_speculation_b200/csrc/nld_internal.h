@@ -84,20 +84,26 @@ struct EpiArgs {
 // One projection of a chain launch.
 constexpr int kMaxPhases = 4;
 struct alignas(64) PhaseArgs {
-  CUtensorMap tmW;  // pre-tiled weights: view [row_tiles * KT * 128, 64], box {64, 128}
+  CUtensorMap tmW;  // row-major weights (w_rowmajor): box {64, 128} at (k * 64, row)
   CUtensorMap tmX;  // activations [M_max, K], box {64, NT}
+  const void* W;    // pre-tiled weights (w_rowmajor == 0): block (row tile r, k-tile kt) is the
+                    // 16 KB swizzled shared-memory image at byte offset (r * KT + kt) * 16384
   EpiArgs e;
   int tok_tiles, row_tiles, KT;
   int s;            // ranks of a cluster splitting each tile's K range (divides CS)
   int ks;           // k-iterations per rank
   int w_rowmajor;   // 1: tmW views a plain row-major [n_rows, K] matrix (box {64, 128} at
                     // (k*64, row)); 0: the pre-tiled layout
+  int x3d;          // 1: tmX views the activations as [K/64 blocks][rows][64] with box
+                    // {64, xr, kps}: one load brings a stage's kps k-tiles of a token tile
+                    // (rows past the tensor fill with zeros); 0: 2D [rows, K], box {64, xr}
 };
 
 // A persistent launch running nph projections in order, separated by grid-wide arrivals.
 struct alignas(64) ChainArgs {
   PhaseArgs ph[kMaxPhases];
-  CUtensorMap tmWn;  // weights of the projection that runs next on the stream (L2 warm-up)
+  CUtensorMap tmWn;  // (unused by the pre-tiled path)
+  const void* Wn;    // pre-tiled weights of the projection that runs next on the stream (L2 warm-up)
   int nph;
   int CS;           // CTAs per cluster
   int NT;           // tokens per tile (multiple of 16; MMA N = NT << hilo <= 256)
@@ -113,6 +119,7 @@ struct alignas(64) ChainArgs {
                     // zero before the launch, left zero by it
   unsigned long long* trace;   // optional per-CTA phase timestamps (profiling hook), or null
   int boundary_pf;  // weight boxes each CTA prefetches into L2 while it waits at a phase boundary
+  int pf_stages;    // L2 run-ahead: stages between a weight prefetch and its load (0 = off)
   int dbg_skip_arrive;   // test hook: CTA 0 withholds its phase-0 arrival, so every wait on that
                          // counter runs into its time limit (the failure-detection test)
   // the next chain launch's first phase (L2 warm-up of each CTA's first weight boxes there)
@@ -134,6 +141,7 @@ struct AttnArgs {
                         // the blocks of block_size start after them (fused diffusion fill)
   const int* causal_seq;  // optional [batch]: nonzero makes all m rows of that sequence causal
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
+  int min_tiles;        // KV tiles a split takes at least (1..)
   float scale_log2;     // log2(e) / sqrt(hd)
   int hilo;             // tensor-core path: q fp32 [M, Hq, hd], out (hi, lo) bf16 rows [2M, Hq, hd]
   int quad_k;           // quadratic self-speculation forward with block k (0 = off): rows 0..k are
