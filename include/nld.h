@@ -58,7 +58,7 @@ enum { NLD_F32 = 0, NLD_BF16 = 1 };
 enum { NLD_MODE_AR = 0, NLD_MODE_DRAFT = 1, NLD_MODE_VERIFY = 2, NLD_MODE_DIFFUSE = 3, NLD_MODE_QUAD = 4 };
 
 /* Device error word bits (reported by nld_sync). */
-enum { NLD_DEVERR_KV_OVERFLOW = 1, NLD_DEVERR_TIMEOUT = 2, NLD_DEVERR_TOKEN = 4 };
+enum { NLD_DEVERR_KV_OVERFLOW = 1, NLD_DEVERR_TIMEOUT = 2, NLD_DEVERR_TOKEN = 4, NLD_DEVERR_LAUNCH = 8 };
 
 /*
  * Model and context configuration (Llama-style decoder: RMSNorm, RoPE with rotate-half

@@ -110,7 +110,7 @@ NLD_DEV void store_act8(void* buf, bool hl, int tok, int ld, int col, const floa
 //
 // Vector stores (xbuf != nullptr, bf16 storage, 128-row tiles aligned to heads): the 128
 // threads first write the chunk's fp32 outputs transposed, [16 tokens][row], into xbuf (16 x
-// 132 floats, private to these 4 warps), then each thread stores whole 16-byte pieces of token
+// 128 floats, private to these 4 warps), then each thread stores whole 16-byte pieces of token
 // rows.  With hi/lo activations (e.hilo) the bf16 activation outputs (hb, u) are written as
 // row pairs (hi, lo) and q is kept in fp32.
 template <typename T>
@@ -119,7 +119,7 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
                        float (&v)[16], const EpiPre& pre, float* red_f, int* red_i, int bar_id,
                        float* xbuf = nullptr) {
   const int row = row_tile * kTileRows + row_in_tile;
-  constexpr int kXld = 132;   // floats per token row of xbuf
+  constexpr int kXld = 128;   // floats per token row of xbuf (one split-K slot: 16 x 128 floats)
   const bool vec = (xbuf != nullptr) && sizeof(T) == 2;
   const bool hl = (sizeof(T) == 2) && e.hilo;
   switch (e.kind) {

@@ -43,9 +43,13 @@ namespace {
 
 constexpr int kStageW = kTileRows * kTileK * 2;   // 16 KB: one k-tile of bf16 weights
 constexpr int kMaxStages = 8;
-constexpr int kSlotLd = 20;              // floats per row of a split-K slot: 16 + 4 (16-byte
-                                         // accesses of 8 consecutive rows hit distinct banks)
+constexpr int kSlotLd = 16;              // floats per row of a split-K slot (one 16-column chunk)
 constexpr int kSlotFloats = kTileRows * kSlotLd;
+// Byte offset of 16-byte piece q (0..3) of `row` in a slot: the pieces of a row are permuted by
+// (row >> 1) & 3 so that the 16-byte accesses of 8 consecutive rows hit distinct bank groups.
+NLD_DEV uint32_t slot_off(int row, int q) {
+  return static_cast<uint32_t>(row * kSlotLd * 4 + ((q ^ ((row >> 1) & 3)) << 4));
+}
 constexpr int kEpiThreads = 256;   // 8 epilogue warps
 constexpr int kThreads = 64 + kEpiThreads;
 
@@ -61,12 +65,9 @@ struct GemmTail {
   volatile int abort_flag;
   volatile int epi_abort;
   int pad;
-  float inv[kMaxNT];
-  int pos[kMaxNT];
-  int pg[kMaxNT];
-  int rpos[kMaxNT];
-  float red_f[2][96];   // per epilogue half
-  int red_i[2][96];
+  float red_f[2][80];   // per epilogue half (4 x 16 partials + 16 results)
+  int red_i[2][80];
+  // followed in shared memory by the tile's per-column data: inv[NT], pos[NT], pg[NT], rpos[NT]
 };
 
 // Work of one CTA in phase p: its group of s ranks, the group's tiles and this rank's K slice.
@@ -171,9 +172,15 @@ NLD_DEV bool epi_wait(uint64_t* bar, uint32_t parity, bool cluster_acquire, uint
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_chain_kernel(const __grid_constant__ ChainArgs A, const uint64_t timeout_ns) {
+  // the launch asks for no alignment slack: the dynamic shared memory of a CTA without static
+  // shared memory starts 1024-byte aligned, which the 128-byte swizzle of the ring needs; a launch
+  // where it does not leaves at once (error word) before any barrier or tensor-memory use
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) set_err(A.ph[0].e.err, NLD_DEVERR_LAUNCH);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int S = A.stages;
   const int NT = A.NT;
   const int NN = NT << A.hilo;         // MMA N: activation rows of a token tile (hi/lo pairs)
@@ -185,9 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sW = smem;
   uint8_t* sX = smem + S * wst;
   // split-K slot area (CS > 1): [A.slots][128 rows][kSlotLd] floats; for a split tile of group
-  // size s, slot (q * per + c) holds group rank q's partial of this CTA's c-th owned chunk
+  // size s, slot (q' * per + c) holds the partial of this CTA's c-th owned chunk from the q'-th
+  // other rank of the group (q' = q for ranks q below this one, q - 1 above); the owner keeps
+  // its own partial in registers
   float* slots = reinterpret_cast<float*>(sX + S * xst);
   GemmTail* tail = reinterpret_cast<GemmTail*>(slots + (CS > 1 ? A.slots * kSlotFloats : 0));
+  float* const s_inv = reinterpret_cast<float*>(tail + 1);
+  int* const s_pos = reinterpret_cast<int*>(s_inv + NT);
+  int* const s_pg = s_pos + NT;
+  int* const s_rpos = s_pg + NT;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -504,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tb = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         named_bar_sync(1, kEpiThreads);
-        compute_tile_meta(e, tok0, NT, need_norm, tail->inv, tail->pos, tail->pg, tail->rpos, et, kEpiThreads);
+        compute_tile_meta(e, tok0, NT, need_norm, s_inv, s_pos, s_pg, s_rpos, et, kEpiThreads);
         // Split tile: the group's s ranks each hold a partial sum of the whole tile.  Rank g
         // owns chunks [g*per, (g+1)*per): every rank sends its partial of those chunks to g with
         // st.async (one-way, counted by g's rfull transaction count) and g sums the s partials
@@ -513,11 +526,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int per = (nchunks + w.s - 1) / w.s;
         const int c_lo = w.grank * per, c_hi = min(nchunks, c_lo + per);
         const int n_own = max(0, c_hi - c_lo);
-        const int cm = c_lo + half;
+        // the half whose chunk parity matches reduces an owned chunk (per <= 2): the thread that
+        // loads that chunk's accumulator in step 2 is the one that sums it in step 4
+        const int cm = ((c_lo & 1) == half) ? c_lo : c_lo + 1;
         EpiPre pre;
         if (w.s > 1) {
           named_bar_sync(1, kEpiThreads);   // the tile's positions (QKV) are in shared memory
-          if (cm < c_hi) epi_preload(e, r, row_in_tile, tok0 + cm * 16, tail->rpos, cm * 16, pre);
+          if (cm < c_hi) epi_preload(e, r, row_in_tile, tok0 + cm * 16, s_rpos, cm * 16, pre);
           // every other owner of this tile has reduced the group's previous split tile of this
           // phase (earlier phases: the grid-wide phase counter), so its slots are free
           if (et < w.s && et != w.grank && et * per < nchunks) {
@@ -540,32 +555,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w.s == 1) {
           for (int c = half; c < nchunks; c += 2) {
             EpiPre pre;
-            epi_preload(e, r, row_in_tile, tok0 + c * 16, tail->rpos, c * 16, pre);
+            epi_preload(e, r, row_in_tile, tok0 + c * 16, s_rpos, c * 16, pre);
             float v[16];
             tmem_ld_chunk(tbase, c, A.hilo, v);
-            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, tail->inv, tail->pos, tail->pg,
+            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + c * 16, s_inv, s_pos, s_pg,
                          c * 16, v, pre, red_f, red_i, hbar);
           }
           tc_fence_before();
           mbar_arrive(&tail->tempty[tb]);
         } else {
-          // 2. partial -> owners (own chunks by plain stores)
+          // 2. partial -> owners; the own chunk's partial stays in registers (v_own)
+          float v_own[16];
           for (int c = half; c < nchunks; c += 2) {
             float v[16];
             tmem_ld_chunk(tbase, c, A.hilo, v);
             const int o = c / per;
-            const uint32_t off = static_cast<uint32_t>(((w.grank * per + (c - o * per)) * kTileRows + row_in_tile) * kSlotLd) * 4u;
             if (o == w.grank) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(slots) + off);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              for (int j = 0; j < 16; ++j) v_own[j] = v[j];
             } else {
+              const int qs = (w.grank < o) ? w.grank : w.grank - 1;   // this rank among o's senders
               const uint32_t peer = static_cast<uint32_t>(g0 + o);
-              const uint32_t dst = dsmem_addr(smem_u32(slots), peer) + off;
+              const uint32_t base = dsmem_addr(smem_u32(slots), peer) +
+                                    static_cast<uint32_t>((qs * per + (c - o * per)) * kSlotFloats * 4);
               const uint32_t bar = dsmem_addr(smem_u32(&tail->rfull), peer);
 #pragma unroll
               for (int q = 0; q < 4; ++q)
-                st_async_f4(dst + 16u * q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]), bar);
+                st_async_f4(base + slot_off(row_in_tile, q),
+                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]), bar);
             }
           }
           tc_fence_before();
@@ -584,17 +601,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             named_bar_sync(1, kEpiThreads);
           }
           if (et == 0) trace_iter(A, 3, 8 * i + 2);
-          // 4. reduce this thread's chunk in rank order
+          // 4. reduce this thread's chunk in rank order (its own partial at its rank's place)
           if (cm < c_hi) {
-            const float* src = slots + static_cast<size_t>((cm - c_lo) * kTileRows + row_in_tile) * kSlotLd;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(slots) +
+                                 static_cast<size_t>(cm - c_lo) * kSlotFloats * 4;
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
             for (int q = 0; q < w.s; ++q) {
-              const float4* pq = reinterpret_cast<const float4*>(src + static_cast<size_t>(q * per) * kSlotFloats);
+              if (q == w.grank) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += v_own[j];
+                continue;
+              }
+              const int qs = (q < w.grank) ? q : q - 1;
+              const uint8_t* pq = src + static_cast<size_t>(qs * per) * kSlotFloats * 4;
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4) {
-                const float4 a4 = pq[k4];
+                const float4 a4 = *reinterpret_cast<const float4*>(pq + slot_off(row_in_tile, k4));
                 v[4 * k4] += a4.x;
                 v[4 * k4 + 1] += a4.y;
                 v[4 * k4 + 2] += a4.z;
@@ -602,11 +626,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             if (et == 0) trace_iter(A, 3, 8 * i + 5);
-            // slot `half` (rank 0's partial of this half's chunk) is read only by this half:
-            // once all four of its warps have summed, it is the chunk's transpose buffer
+            // slot (cm - c_lo) (the first sender's partial of this half's chunk) is read only by
+            // this half: once all four of its warps have summed, it is the chunk's transpose buffer
             named_bar_sync(hbar, 128);
-            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + cm * 16, tail->inv, tail->pos, tail->pg,
-                         cm * 16, v, pre, red_f, red_i, hbar, slots + static_cast<size_t>(half) * kSlotFloats);
+            epi_chunk<T>(e, r, row_in_tile, lane, ew, tok0 + cm * 16, s_inv, s_pos, s_pg,
+                         cm * 16, v, pre, red_f, red_i, hbar,
+                         slots + static_cast<size_t>(cm - c_lo) * kSlotFloats);
             if (et == 0) trace_iter(A, 3, 8 * i + 6);
           }
           // 5. this CTA's slots are free again (relaxed: the loaded values were consumed)
@@ -651,9 +676,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_mark(A, 15);
 }
 
-size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS, int slots) {
+// Dynamic shared memory of a chain launch: the ring, then the split-K slots, the tail and the
+// per-column tile data.  The MMA reads NN = MMA N activation rows from each xr-row box, so the
+// last box of the ring is read (nn - xr) * 128 bytes past its end: that much must still lie in
+// the allocation (the bytes after the ring are read as padding columns the epilogue ignores).
+size_t gemm_chain_smem_bytes(int NT, int nn, int xr, int kps, int stages, int CS, int slots) {
   const size_t stg = (CS > 1) ? static_cast<size_t>(slots) * kSlotFloats * sizeof(float) : 0;
-  return 1024 + static_cast<size_t>(stages) * kps * (kStageW + xr * 128) + stg + sizeof(GemmTail);
+  const size_t after = stg + sizeof(GemmTail) + static_cast<size_t>(NT) * 16;
+  const size_t overread = static_cast<size_t>(nn > xr ? nn - xr : 0) * 128;
+  return static_cast<size_t>(stages) * kps * (kStageW + xr * 128) + (after > overread ? after : overread);
 }
 int gemm_chain_max_stages() { return kMaxStages; }
 
@@ -696,7 +727,7 @@ cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uin
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS, A.slots);
+  cfg.dynamicSmemBytes = gemm_chain_smem_bytes(A.NT, A.NT << A.hilo, A.xr, A.kps, A.stages, A.CS, A.slots);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;

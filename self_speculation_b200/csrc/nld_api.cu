@@ -367,8 +367,9 @@ ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const in
   best.slots = 0;
   for (int p = 0; p < nph; ++p)
     if (best.ph[p].s > 1) {
+      // (s - 1) senders x the chunks a rank owns (the owner keeps its own partial in registers)
       const int nch = NT / 16, s = best.ph[p].s;
-      best.slots = std::max(best.slots, s * ((nch + s - 1) / s));
+      best.slots = std::max(best.slots, (s - 1) * ((nch + s - 1) / s));
     }
   // ring: two k-tiles (32 KB of weights) per stage, so one producer/MMA barrier round trip moves
   // 32 KB, with as many stages as fit the shared-memory budget; when wide activation boxes leave
@@ -376,7 +377,7 @@ ChainArgs plan_chain_shapes(const int* max_clusters, const int* n_rows, const in
   const int st_max = stage_cap > 0 ? std::min(stage_cap, gemm_chain_max_stages()) : gemm_chain_max_stages();
   auto fit = [&](int kps) {
     for (int st = st_max; st > 2; --st)
-      if (gemm_chain_smem_bytes(NT, best.xr, kps, st, best.CS, best.slots) <= kChainSmemBudget) return st;
+      if (gemm_chain_smem_bytes(NT, NN, best.xr, kps, st, best.CS, best.slots) <= kChainSmemBudget) return st;
     return 2;
   };
   best.kps = (kps_force > 0) ? kps_force : 2;
@@ -1675,7 +1676,7 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
   out20[5] = A.slots;
   out20[6] = static_cast<int>(A.tmem_cols);
   out20[7] = grid;
-  out20[8] = static_cast<int>(gemm_chain_smem_bytes(A.NT, A.xr, A.kps, A.stages, A.CS, A.slots));
+  out20[8] = static_cast<int>(gemm_chain_smem_bytes(A.NT, A.NT << A.hilo, A.xr, A.kps, A.stages, A.CS, A.slots));
   out20[9] = A.ph[0].tok_tiles;
   for (int p = 0; p < nph; ++p) {
     out20[10 + 2 * p] = A.ph[p].s;

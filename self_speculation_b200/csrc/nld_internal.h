@@ -152,7 +152,7 @@ struct AttnArgs {
 // ---- host-side launchers (each returns cudaError_t of the launch) -----------------------
 cudaError_t launch_gemm_chain(cudaStream_t st, const ChainArgs& A, int grid, uint64_t timeout_ns,
                               bool pdl);
-size_t gemm_chain_smem_bytes(int NT, int xr, int kps, int stages, int CS, int slots);
+size_t gemm_chain_smem_bytes(int NT, int nn, int xr, int kps, int stages, int CS, int slots);
 int gemm_chain_max_stages();
 int gemm_tc_max_clusters(int split, size_t smem, int sms);
 cudaError_t launch_gemm_simt(cudaStream_t st, const float* W, const float* X, int n_rows, int K,

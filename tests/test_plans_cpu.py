@@ -1,7 +1,7 @@
 """Host logic of the launch planners, on CPU through the pure-host hooks nld_plan_chain and
 nld_plan_attention: every plan the library can make for the benchmark and test shapes keeps
 the kernels' limits (227 KB of shared memory, TMEM columns a power of two covering the
-double-buffered accumulator, split-K factors that give every rank work, <= 12 attention warps,
+double-buffered accumulator, split-K factors that give every rank work, <= 9 attention warps,
 <= 8 KV splits), and the plans at the benchmarked decode shape are the ones the committed
 launch list records (layer chain 132 CTAs in clusters of 4, layer-0 QKV 96 CTAs in clusters
 of 2, attention 7 x 8 CTAs of 288 / 256 threads in clusters of 7)."""
@@ -83,14 +83,20 @@ def test_chain_plans_keep_kernel_limits(name, cfg):
                     assert P["xr"] >= M << hilo, where
                 t = P["tmem"]
                 assert t & (t - 1) == 0 and 2 * NN <= t <= 512, where
+                # the MMA reads NN activation rows from each xr-row box: the last box of the
+                # ring is read (NN - xr) rows past its end, which must stay in the allocation
+                ring = P["stages"] * P["kps"] * (16384 + P["xr"] * 128)
+                assert P["smem"] >= ring + (NN - P["xr"]) * 128, where
                 assert P["grid"] % P["CS"] == 0 and P["grid"] <= P["CS"] * clusters[P["CS"]], where
                 if len(phases) > 1 and NT <= 64:
                     assert P["CS"] == 4, where
                 for (rows, K), (s, ks) in zip(phases, P["split"]):
                     KT = K // 64
                     assert P["CS"] % s == 0 and s * ks >= KT and (s - 1) * ks < KT, where
-                if any(s > 1 for s, _ in P["split"]):
-                    assert P["slots"] >= NT // 16, where
+                # split-K receive slots: (s - 1) senders x the 16-token chunks a rank owns
+                for s, _ in P["split"]:
+                    if s > 1:
+                        assert P["slots"] >= (s - 1) * -(-(NT // 16) // s), where
 
 
 def test_decode_plans_match_the_recorded_launch_list():
@@ -99,7 +105,7 @@ def test_decode_plans_match_the_recorded_launch_list():
     # (hi, lo) activation rows: 66 / 64 rows per k-tile box, MMA N = 96 / 64
     for M, NT, xr in ((33, 48, 72), (32, 32, 64)):
         P = plan_chain(M, ch["layer"])
-        assert (P["CS"], P["NT"], P["xr"], P["stages"], P["grid"]) == (4, NT, xr, 3, 132)
+        assert (P["CS"], P["NT"], P["xr"], P["stages"], P["grid"]) == (4, NT, xr, 4, 132)
         L = plan_chain(M, ch["last"])
         assert (L["CS"], L["grid"]) == (4, 132)
     Q = plan_chain(33, ch["qkv0"])
