@@ -306,16 +306,30 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
  * boundary_prefetch = weight boxes each CTA prefetches into L2 while it waits at a phase
  * boundary (0..256; 16 at creation); act_3d = 1 loads a stage's activation k-tiles with one
  * 3D box (the default), 0 with one 2D box per k-tile; runahead_stages = D > 0 prefetches the
- * weights of the stage D ahead of each load into L2 (0..16; 0 = off).  Synchronises and drops
- * the captured graphs; later calls use the new values. */
+ * weights of the stage D ahead of each load into L2 (0..16; 0 = off); warm_next = weight boxes
+ * of the next chain launch's second phase that each CTA prefetches into L2 before it exits, on
+ * top of that launch's first-phase boxes (0..256; 0 at creation).  Synchronises and drops the
+ * captured graphs; later calls use the new values. */
 nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_stage,
-                                  int boundary_prefetch, int act_3d, int runahead_stages);
+                                  int boundary_prefetch, int act_3d, int runahead_stages,
+                                  int warm_next);
 
-/* Profiling hook: attention planning.  rows_per_cta (16..144) caps the query rows (positions x
+/* Profiling hook: attention planning.  rows_per_cta (16..128) caps the query rows (positions x
  * query heads of one kv head) a CTA holds, so smaller values give more, lighter CTAs;
  * min_tiles_per_split (1..8) is the fewest 64-key tiles a KV split takes (more splits merge more
- * partials).  Defaults 144 and 2.  Synchronises and drops the captured graphs. */
+ * partials).  0 for either restores the planner's choice (the default): 64 rows and single-tile
+ * splits when a few sequences leave most SMs idle, else 128 rows and 2 tiles.  Synchronises and
+ * drops the captured graphs. */
 nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
+
+/* Profiling hook: while d_trace (device, n entries of 8 bytes, caller-owned) is set, every
+ * tensor-core attention launch of the model's forwards whose grid fits (16 entries per CTA)
+ * writes per CTA, at entry (CTA linear index) * 16 + i, the global timer in ns at: entry (0),
+ * dependency on the previous kernel met (1), query tile staged (2), KV tile t done (3 + t,
+ * t < 6), split partials published to the cluster (10), output written (11); later launches
+ * overwrite earlier ones.  d_trace = NULL with n = 0 turns it off.  Synchronises and drops the
+ * captured graphs. */
+nld_status nld_debug_attention_trace(nld_ctx* ctx, unsigned long long* d_trace, size_t n);
 
 /* Test hook for failure detection: one launch of layer 0's four-phase chain over the current
  * batch (scratch buffers only, as nld_time_chain) with every bounded wait limited to timeout_ns

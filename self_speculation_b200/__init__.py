@@ -72,9 +72,10 @@ def load_library() -> ctypes.CDLL:
         "nld_plan_attention": ([I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "nld_trace_chain": ([P, I, I, P, ctypes.POINTER(I)], I),
         "nld_time_chain": ([P, I, I, I, ctypes.POINTER(F)], I),
-        "nld_debug_chain_tuning": ([P, I, I, I, I, I], I),
+        "nld_debug_chain_tuning": ([P, I, I, I, I, I, I], I),
         "nld_debug_timeout_chain": ([P, ctypes.c_ulonglong], I),
         "nld_debug_attention_tuning": ([P, I, I], I),
+        "nld_debug_attention_trace": ([P, P, S], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
@@ -230,12 +231,18 @@ class Context:
 
     def nld_debug_chain_tuning(self, stage_cap: int = 0, k_tiles_per_stage: int = 0,
                                boundary_prefetch: int = 16, act_3d: int = 1,
-                               runahead_stages: int = 0) -> None:
+                               runahead_stages: int = 0, warm_next: int = 0) -> None:
         self._check(self.lib.nld_debug_chain_tuning(self.h, int(stage_cap), int(k_tiles_per_stage),
                                                     int(boundary_prefetch), int(act_3d),
-                                                    int(runahead_stages)), self.h)
+                                                    int(runahead_stages), int(warm_next)), self.h)
 
-    def nld_debug_attention_tuning(self, rows_per_cta: int = 144, min_tiles_per_split: int = 2) -> None:
+    def nld_debug_attention_trace(self, trace=None) -> None:
+        """trace: int64 device tensor (16 entries per CTA) or None to turn the hook off."""
+        n = 0 if trace is None else trace.numel()
+        self._check(self.lib.nld_debug_attention_trace(self.h, _ptr(trace) if trace is not None else None, n),
+                    self.h)
+
+    def nld_debug_attention_tuning(self, rows_per_cta: int = 0, min_tiles_per_split: int = 0) -> None:
         self._check(self.lib.nld_debug_attention_tuning(self.h, int(rows_per_cta), int(min_tiles_per_split)),
                     self.h)
 

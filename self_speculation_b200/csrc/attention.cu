@@ -26,10 +26,11 @@ namespace nld {
 
 namespace {
 
-constexpr int kAttStages = 3;
+constexpr int kMaxAttStages = 3;   // K/V ring depth: 2 or 3 (AttnArgs::stages)
 constexpr int kHalfTile = kPage * 64 * 2;        // 8 KB: 64 keys x 64 dims bf16
 constexpr int kKVTile = 2 * kHalfTile;           // 16 KB: 64 keys x 128 dims
-constexpr int kMaxAttWarps = 9;   // rows = positions x G <= 144 (the planner's query tile)
+constexpr int kMaxAttWarps = 8;   // rows = positions x G <= 128 (the planner's query tile); at
+                                  // most two warps per SM sub-partition, so 255 registers each
 
 NLD_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -41,8 +42,10 @@ NLD_DEV void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, 
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
+// (not volatile: a pure function of its operands, so the compiler may interleave independent
+// accumulators)
 NLD_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -105,10 +108,14 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
-  uint8_t* sV = smem + kAttStages * kKVTile;
-  uint8_t* sQ = smem + 2 * kAttStages * kKVTile;
+  const int NS = a.stages;
+  uint8_t* sV = smem + NS * kKVTile;
+  uint8_t* sQ = smem + 2 * NS * kKVTile;
   uint8_t* sQl = sQ + a.NW * 16 * 256;           // lo halves of Q (kHiLo)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sQ + (kHiLo ? 2 : 1) * a.NW * 16 * 256);
+  // ring barriers past both the ring + query tile and the split partials that overlay them
+  const int ring_q = 2 * NS * kKVTile + (kHiLo ? 2 : 1) * a.NW * 16 * 256;
+  const int partials = a.NW * 16 * (128 + 2) * 4;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + max(ring_q, partials));
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -117,9 +124,17 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   const int g = blockIdx.y;
   const int b = blockIdx.z / a.q_tiles;
   const int qt = blockIdx.z - b * a.q_tiles;
+  // profiling hook: slot i of this CTA's 16 timestamps (entry 0, dependency met 1, Q staged 2,
+  // KV tile t done 3+t for t < 6, partials published 10, done 11)
+  auto stamp = [&](int i) {
+    if (a.trace && tid == 0)
+      a.trace[((static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 16 + i] =
+          globaltimer_ns();
+  };
+  stamp(0);
 
   if (tid == 0) {
-    for (int i = 0; i < kAttStages; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < NS; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmKV);
   }
@@ -152,7 +167,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   __syncthreads();
 
   auto issue = [&](int i) {
-    const int stage = i % kAttStages;
+    const int stage = i % NS;
     const int kt = t_lo + i;
     const int page = a.page_table[b * a.pps + kt];
     const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
@@ -165,19 +180,19 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   };
   int n_pre = 0;
   if (tid == 0) {
-    for (; n_pre < min(kAttStages, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
+    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
   }
   __syncwarp();
   pdl_wait();
-  pdl_launch_dependents();
+  stamp(1);
   if (tid == 0)
-    for (int i = n_pre; i < min(kAttStages, ntile); ++i) issue(i);
+    for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
   __syncwarp();
 
   // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row); each
   // thread issues the global loads of kQB chunks before storing any, so they are in flight together
   const int rows_pad = a.NW * 16;
-  constexpr int kQB = 4;
+  constexpr int kQB = 8;   // 8 warps x 32 threads x 8 chunks = 128 rows x 16: one round
   for (int e0 = tid; e0 < rows_pad * 16; e0 += kQB * nthr) {
     float4 x0[kQB], x1[kQB];
     uint4 xb[kQB];
@@ -217,6 +232,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     }
   }
   __syncthreads();
+  stamp(2);
 
   // Q fragments for the warp's 16 rows, all 8 k-steps of head_dim 128 (the lo halves are
   // read from shared memory per k-step inside the tile loop)
@@ -245,14 +261,18 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
   bool timed_out = false;
 
   for (int i = 0; i < ntile; ++i) {
-    const int stage = i % kAttStages;
-    if (!mbar_wait(&full[stage], static_cast<uint32_t>(i / kAttStages) & 1u, 2000000000ull)) {
+    const int stage = i % NS;
+    if (!mbar_wait(&full[stage], static_cast<uint32_t>(i / NS) & 1u, 2000000000ull)) {
       timed_out = true;
     }
     if (__syncthreads_or(timed_out)) {
       set_err(a.err, NLD_DEVERR_TIMEOUT);
       break;
     }
+    // the next kernel (a projection chain that starts by streaming weights) may launch once
+    // every CTA holds its query tile and first KV tile: launched earlier, its loads queue ahead
+    // of these latency-critical ones
+    if (i == 0) pdl_launch_dependents();
     const int j0 = (t_lo + i) * kPage;
     const uint32_t kb = smem_u32(sK + stage * kKVTile);
     const uint32_t vb = smem_u32(sV + stage * kKVTile);
@@ -260,26 +280,31 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     float sc[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    // per 32 dims: the K fragments of all 8 key groups first, then the MMAs grouped so that
+    // consecutive ones go to the 8 independent accumulators (each accumulator still takes its
+    // terms in the order hi k-step 0, hi k-step 1, lo k-step 0, lo k-step 1)
 #pragma unroll
     for (int kk2 = 0; kk2 < 4; ++kk2) {
-      uint32_t ql0[4], ql1[4];
-      if constexpr (kHiLo) {
-        const int c0 = 4 * kk2 + (lane >> 4), c1 = c0 + 2;
-        ldsm_x4(smem_u32(sQl + qr * 256 + ((c0 ^ (qr & 7)) << 4)), ql0[0], ql0[1], ql0[2], ql0[3]);
-        ldsm_x4(smem_u32(sQl + qr * 256 + ((c1 ^ (qr & 7)) << 4)), ql1[0], ql1[1], ql1[2], ql1[3]);
-      }
+      uint32_t kf[8][4];
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         const int key = nt * 8 + (lane & 7);
         const int c = 4 * kk2 + (lane >> 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + kv_off(key, c), b0, b1, b2, b3);
-        mma_bf16_16816(sc[nt], qf[2 * kk2], b0, b1);
-        mma_bf16_16816(sc[nt], qf[2 * kk2 + 1], b2, b3);
-        if constexpr (kHiLo) {
-          mma_bf16_16816(sc[nt], ql0, b0, b1);
-          mma_bf16_16816(sc[nt], ql1, b2, b3);
-        }
+        ldsm_x4(kb + kv_off(key, c), kf[nt][0], kf[nt][1], kf[nt][2], kf[nt][3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(sc[nt], qf[2 * kk2], kf[nt][0], kf[nt][1]);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(sc[nt], qf[2 * kk2 + 1], kf[nt][2], kf[nt][3]);
+      if constexpr (kHiLo) {
+        uint32_t ql0[4], ql1[4];
+        const int c0 = 4 * kk2 + (lane >> 4), c1 = c0 + 2;
+        ldsm_x4(smem_u32(sQl + qr * 256 + ((c0 ^ (qr & 7)) << 4)), ql0[0], ql0[1], ql0[2], ql0[3]);
+        ldsm_x4(smem_u32(sQl + qr * 256 + ((c1 ^ (qr & 7)) << 4)), ql1[0], ql1[1], ql1[2], ql1[3]);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(sc[nt], ql0, kf[nt][0], kf[nt][1]);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(sc[nt], ql1, kf[nt][2], kf[nt][3]);
       }
     }
     // scale, mask, online softmax (log2 domain)
@@ -344,24 +369,34 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
         pa[3] = pack_bf16(sc[2 * j + 1][2], sc[2 * j + 1][3]);
       }
       const int key = 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
+      // the V fragments of all 128 dims first, then 16 independent accumulators per pass (each
+      // takes P_hi then P_lo)
+      uint32_t vf[8][4];
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         const int c = 2 * p + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + kv_off(key, c), b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * p], pa, b0, b1);
-        mma_bf16_16816(o[2 * p + 1], pa, b2, b3);
-        if constexpr (kHiLo) {
-          mma_bf16_16816(o[2 * p], pl, b0, b1);
-          mma_bf16_16816(o[2 * p + 1], pl, b2, b3);
+        ldsm_x4_t(vb + kv_off(key, c), vf[p][0], vf[p][1], vf[p][2], vf[p][3]);
+      }
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        mma_bf16_16816(o[2 * p], pa, vf[p][0], vf[p][1]);
+        mma_bf16_16816(o[2 * p + 1], pa, vf[p][2], vf[p][3]);
+      }
+      if constexpr (kHiLo) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          mma_bf16_16816(o[2 * p], pl, vf[p][0], vf[p][1]);
+          mma_bf16_16816(o[2 * p + 1], pl, vf[p][2], vf[p][3]);
         }
       }
     }
     __syncthreads();
-    if (tid == 0 && i + kAttStages < ntile) issue(i + kAttStages);
+    if (i < 6) stamp(3 + i);
+    if (tid == 0 && i + NS < ntile) issue(i + NS);
     __syncwarp();
   }
 
+  if (ntile == 0 || timed_out) pdl_launch_dependents();
   l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
   l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
@@ -396,6 +431,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
 #pragma unroll
       for (int n = 0; n < 16; ++n) store2(rb, n * 8 + 2 * (lane & 3), o[n][2] * ib, o[n][3] * ib);
     }
+    stamp(11);
     return;
   }
 
@@ -415,6 +451,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     }
   }
   cluster_sync();
+  stamp(10);
   const int S = a.S;
   const int rank = static_cast<int>(cluster_ctarank());
   const int per_rank = (a.rows + S - 1) / S;
@@ -430,18 +467,18 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     const int r = r0 + (e >> 5), d4 = e & 31;
     const int p = r / a.G;
     if (p >= np) continue;
+    // every split published (m, l) and O for every row (zeros and -inf where it saw no key),
+    // so all loads are issued before any is used
     float2 ml[8];
-    float M = -INFINITY;
+    float4 ov[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + r * 8) : make_float2(-INFINITY, 0.f);
-      M = fmaxf(M, ml[q].x);
+      ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + (r * 128 + d4 * 4) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float4 ov[8];
+    float M = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      ov[q] = (q < S && ml[q].x != -INFINITY) ? ld_dsmem_f4(o_peer[q] + (r * 128 + d4 * 4) * 4)
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < 8; ++q) M = fmaxf(M, ml[q].x);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -459,6 +496,7 @@ __global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
     store2(r, d4 * 4, acc.x * inv, acc.y * inv);
     store2(r, d4 * 4 + 2, acc.z * inv, acc.w * inv);
   }
+  stamp(11);
   cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
@@ -549,18 +587,46 @@ cudaError_t init_kernel_attributes() {
                               optin - static_cast<int>(fa.sharedSizeBytes));
 }
 
-size_t attn_mma_smem_bytes(int NW, bool hilo) {
-  return 1024 + 2 * kAttStages * kKVTile + static_cast<size_t>(hilo ? 2 : 1) * NW * 16 * 256 +
-         kAttStages * sizeof(uint64_t);
+// Dynamic shared memory of a launch: the K/V ring and the query tile (hi and lo halves with
+// hilo), then the ring's barriers; the split partials (fp32 O and (m, l) per row) overlay the
+// ring and the query tile once the KV loop is done.
+size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
+  const size_t ring_q = 2 * static_cast<size_t>(stages) * kKVTile + static_cast<size_t>(hilo ? 2 : 1) * NW * 16 * 256;
+  const size_t partials = static_cast<size_t>(NW) * 16 * (128 + 2) * sizeof(float);
+  return 1024 + std::max(ring_q, partials) + kMaxAttStages * sizeof(uint64_t);
+}
+
+// Clusters of S CTAs (NW warps, the shared memory above) that can be resident at once.
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S * (sms / S));
+  cfg.blockDim = dim3(32 * NW);
+  cfg.dynamicSmemBytes = attn_mma_smem_bytes(NW, hilo, stages);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = hilo ? cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<true>, &cfg)
+                             : cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<false>, &cfg);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return sms / S;
+  }
+  return n > 0 ? n : 1;
 }
 
 cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
                                  int batch, bool pdl) {
-  if (a.NW < 1 || a.NW > kMaxAttWarps) return cudaErrorInvalidValue;   // launch bound
+  if (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages)
+    return cudaErrorInvalidValue;   // launch bound, ring depth
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
   cfg.blockDim = dim3(32 * a.NW);
-  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW, a.hilo != 0);
+  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW, a.hilo != 0, a.stages);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -410,13 +410,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warm L2 (and address translation) for this CTA index's first boxes of the next chain
         const int ncl = blockIdx.x / A.next_CS;
         const int nrank = blockIdx.x % A.next_CS;
-        const int grp = ncl * (A.next_CS / A.next_s) + nrank / A.next_s;
-        if (grp < A.next_tiles) {
-          const int nr = grp / A.next_tok_tiles;
-          const int lo = (nrank % A.next_s) * A.next_ks;
-          const int hi = min(A.next_KT, min(lo + A.next_ks, lo + A.next_boxes));
+        for (int j = 0; j < 2; ++j) {
+          const WarmPhase& N = A.next[j];
+          if (N.boxes <= 0) continue;
+          const int grp = ncl * (A.next_CS / N.s) + nrank / N.s;
+          if (grp >= N.tiles) continue;
+          const int nr = grp / N.tok_tiles;
+          const int lo = (nrank % N.s) * N.ks;
+          const int hi = min(N.KT, min(lo + N.ks, lo + N.boxes));
           if (hi > lo)
-            bulk_prefetch_l2(static_cast<const uint8_t*>(A.Wn) + (static_cast<size_t>(nr) * A.next_KT + lo) * kStageW,
+            bulk_prefetch_l2(static_cast<const uint8_t*>(N.W) + (static_cast<size_t>(nr) * N.KT + lo) * kStageW,
                              static_cast<uint32_t>((hi - lo) * kStageW));
         }
       }

@@ -17,6 +17,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <functional>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -26,7 +27,8 @@
 using namespace nld;
 
 namespace nld {
-size_t attn_mma_smem_bytes(int NW, bool hilo);
+size_t attn_mma_smem_bytes(int NW, bool hilo, int stages);
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms);
 cudaError_t init_kernel_attributes();
 }
 
@@ -130,8 +132,8 @@ struct nld_ctx {
   CUtensorMap tmKV{};
   std::map<std::tuple<int, int, int>, std::pair<CUtensorMap, int>> tmX;   // (buffer, rows, kps) -> map, 3D
   int chain_x3d = 1;   // activation loads of a stage as one 3D box (0: per k-tile 2D boxes)
-  int attn_rows_cap = 144;   // attention planning (profiling hook): query rows per CTA at most
-  int attn_min_tiles = 2;    // and KV tiles per split at least
+  int attn_rows_cap = 0;     // attention planning (profiling hook): query rows per CTA at most
+  int attn_min_tiles = 0;    // and KV tiles per split at least (0: the planner's choice)
   // graphs: one per (call, batch, output pointers), at most kMaxGraphs (least recently used
   // evicted); tick = the call count at each graph's last replay
   struct GraphEntry {
@@ -145,6 +147,9 @@ struct nld_ctx {
   int chain_kps = 0;   // k-tiles per stage (0 = the planner's choice)
   int chain_boundary_pf = 16;   // weight boxes prefetched into L2 per CTA at a phase boundary
   int chain_pf_stages = 0;      // L2 run-ahead distance in stages (0 = off)
+  int chain_warm_next = 0;      // boxes of the next chain's second phase each CTA warms in L2
+  unsigned long long* attn_trace = nullptr;   // profiling hook: attention timestamps (or null)
+  size_t attn_trace_n = 0;
   // host-side sequence bookkeeping
   int batch = 0;
   bool started = false;
@@ -156,6 +161,14 @@ struct nld_ctx {
   uint64_t timeout_ns = 2000000000ull;
   std::string msg;
 };
+
+// SMs of the current device.
+static int device_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  return n;
+}
 
 namespace {
 
@@ -438,46 +451,83 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
   A.trace = trace;
   A.boundary_pf = x->chain_boundary_pf;
   A.pf_stages = x->chain_pf_stages;
-  A.tmWn = A.ph[0].tmW;
   if (next_pr && next_nph > 0) {
     int ngrid = 0;
     const ChainArgs N = plan_chain(x, next_pr, next_nph, M, &ngrid);
     A.next_valid = 1;
     A.next_CS = N.CS;
-    A.next_s = N.ph[0].s;
-    A.next_tok_tiles = N.ph[0].tok_tiles;
-    A.next_ks = N.ph[0].ks;
-    A.next_KT = N.ph[0].KT;
     A.next_grid = ngrid;
-    A.next_tiles = N.ph[0].row_tiles * N.ph[0].tok_tiles;
-    A.next_boxes = N.stages * N.kps + 8;
-    A.tmWn = *winfo(x, next_pr[0].which, next_pr[0].layer).map;
-    A.Wn = winfo(x, next_pr[0].which, next_pr[0].layer).W;
+    for (int j = 0; j < 2 && j < next_nph; ++j) {
+      WarmPhase& wp = A.next[j];
+      wp.W = winfo(x, next_pr[j].which, next_pr[j].layer).W;
+      wp.s = N.ph[j].s;
+      wp.tok_tiles = N.ph[j].tok_tiles;
+      wp.ks = N.ph[j].ks;
+      wp.KT = N.ph[j].KT;
+      wp.tiles = N.ph[j].row_tiles * N.ph[j].tok_tiles;
+      wp.boxes = j == 0 ? N.stages * N.kps + 8 : x->chain_warm_next;
+    }
   }
   CK(launch_gemm_chain(x->stream, A, grid, x->timeout_ns, pdl));
   return NLD_OK;
 }
 
-// rows_cap: query rows (positions x heads) per CTA at most (<= 144: 9 warps); min_tiles: KV tiles
-// a split takes at least.
-void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, int rows_cap = 144,
-               int min_tiles = 2) {
+// Clusters of S attention CTAs (NW warps, `stages` ring stages) resident at once.
+using AttnCapacity = std::function<int(int S, int NW, int stages)>;
+
+// rows_cap: query rows (positions x heads) per CTA at most (16..128: 8 warps); min_tiles: KV
+// tiles a split takes at least; 0 = the planner's choice for either.
+void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
+               int rows_cap = 0, int min_tiles = 0) {
   a.G = Hq / Hkv;
+  const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
+  auto q_tiles_for = [&](int c) {
+    const int qt_max = std::min(m, std::max(1, c / a.G));
+    return (m + qt_max - 1) / qt_max;
+  };
+  // Latency regime (a few sequences): even split 8 ways, whole query tiles would leave most SMs
+  // idle, so the query positions are cut into tiles of <= 64 rows (one warp per SM
+  // sub-partition: a KV tile then costs a quarter of the MMA time of an 8-warp CTA), the keys
+  // into splits of single tiles, and the ring holds 2 stages (about 100 KB, two CTAs per SM).
+  // Otherwise tiles of up to 128 rows read each K/V tile once for as many query rows as
+  // possible, through a 3-stage ring.
+  const bool latency = batch * Hkv * q_tiles_for(128) * 8 < 2 * sms;
+  if (rows_cap <= 0) rows_cap = latency ? 64 : 128;
+  if (min_tiles <= 0) min_tiles = latency ? 1 : 2;
   a.min_tiles = min_tiles;
+  a.stages = latency ? 2 : 3;
   // query positions per CTA: as many as rows_cap allows, spread evenly over the query tiles
-  const int qt_max = std::min(m, std::max(1, rows_cap / a.G));
-  const int nq = (m + qt_max - 1) / qt_max;
+  const int nq = q_tiles_for(rows_cap);
   a.QT = (m + nq - 1) / nq;
   a.q_tiles = (m + a.QT - 1) / a.QT;
   a.rows = a.QT * a.G;
   a.NW = (a.rows + 15) / 16;
-  // KV splits of one (sequence, kv head, query tile) form a cluster of at most 8 CTAs; split
-  // only while the grid is short of two CTAs per SM, and keep >= 2 KV tiles per split
+  // KV splits of one (sequence, kv head, query tile) form a cluster of at most 8 CTAs.  Split
+  // only while the grid is short of two CTAs per SM, keep >= min_tiles KV tiles per split, take
+  // no more splits than lets every cluster be resident at once (a second wave doubles the
+  // latency), and launch no split that the tiles per split leave empty.
   const int units = batch * a.q_tiles * Hkv;
-  const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   a.S = 1;
-  if (units < 2 * sms)
-    a.S = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / min_tiles)}));
+  if (units < 2 * sms) {
+    int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / min_tiles)}));
+    while (s_max > 1 && units > cap(s_max, a.NW, a.stages)) --s_max;
+    const int per = std::max(min_tiles, (n_tiles + s_max - 1) / s_max);
+    a.S = std::max(1, (n_tiles + per - 1) / per);
+  }
+}
+
+// The device's cluster capacity for the attention kernel (occupancy query, cached).
+int attn_device_capacity(bool hilo, int S, int NW, int stages) {
+  static int cache[16][9][9][2][4];   // [device][S][NW][hilo][stages]; 0 = not yet queried
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 16 || S < 1 || S > 8 || NW < 1 || NW > 8 || stages < 2 ||
+      stages > 3) {
+    cudaGetLastError();
+    return 1;
+  }
+  int& c = cache[dev][S][NW][hilo ? 1 : 0][stages];
+  if (c == 0) c = attn_mma_max_clusters(S, NW, hilo, stages, device_sms());
+  return c;
 }
 
 EpiArgs base_epi(nld_ctx* x, int M, int m) {
@@ -571,7 +621,11 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.hilo = x->bf16 ? 1 : 0;
   aa.quad_k = f.quad_k;
   if (x->bf16) {
-    attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa, x->attn_rows_cap, x->attn_min_tiles);
+    attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa,
+              [](int S, int NW, int stages) { return attn_device_capacity(true, S, NW, stages); },
+              x->attn_rows_cap, x->attn_min_tiles);
+    const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
+    if (x->attn_trace && ctas * 16 <= x->attn_trace_n) aa.trace = x->attn_trace;
   } else {
     aa.G = aa.Hq / aa.Hkv;
   }
@@ -1595,13 +1649,15 @@ nld_status nld_time_chain(nld_ctx* x, int layer, int M, int reps, float* ms_out)
 }
 
 nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_stage, int boundary_prefetch,
-                                  int act_3d, int runahead_stages) {
+                                  int act_3d, int runahead_stages, int warm_next) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if (stage_cap < 0 || stage_cap == 1 || stage_cap == 2 || stage_cap > gemm_chain_max_stages() ||
       k_tiles_per_stage < 0 || k_tiles_per_stage > 2 || boundary_prefetch < 0 || boundary_prefetch > 256 ||
-      (act_3d != 0 && act_3d != 1) || runahead_stages < 0 || runahead_stages > 16)
+      (act_3d != 0 && act_3d != 1) || runahead_stages < 0 || runahead_stages > 16 || warm_next < 0 ||
+      warm_next > 256)
     return fail(x, NLD_ERR_ARG,
-                "stage cap 0 or 3..%d, k-tiles per stage 0..2, boundary prefetch 0..256, act_3d 0/1, run-ahead 0..16",
+                "stage cap 0 or 3..%d, k-tiles per stage 0..2, boundary prefetch 0..256, act_3d 0/1, "
+                "run-ahead 0..16, warm-next 0..256",
                 gemm_chain_max_stages());
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);   // captured graphs hold the old launch parameters
@@ -1611,13 +1667,25 @@ nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_sta
   if (x->chain_x3d != act_3d) x->tmX.clear();   // activation maps of the other form
   x->chain_x3d = act_3d;
   x->chain_pf_stages = runahead_stages;
+  x->chain_warm_next = warm_next;
+  return NLD_OK;
+}
+
+nld_status nld_debug_attention_trace(nld_ctx* x, unsigned long long* d_trace, size_t n) {
+  if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
+  if ((d_trace == nullptr) != (n == 0)) return fail(x, NLD_ERR_ARG, "trace buffer and size: both or neither");
+  CK(cudaStreamSynchronize(x->stream));
+  drop_graphs(x);   // captured graphs hold the old launch parameters
+  x->attn_trace = d_trace;
+  x->attn_trace_n = n;
   return NLD_OK;
 }
 
 nld_status nld_debug_attention_tuning(nld_ctx* x, int rows_per_cta, int min_tiles_per_split) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
-  if (rows_per_cta < 16 || rows_per_cta > 144 || min_tiles_per_split < 1 || min_tiles_per_split > 8)
-    return fail(x, NLD_ERR_ARG, "rows per CTA 16..144, KV tiles per split 1..8");
+  if ((rows_per_cta != 0 && (rows_per_cta < 16 || rows_per_cta > 128)) || min_tiles_per_split < 0 ||
+      min_tiles_per_split > 8)
+    return fail(x, NLD_ERR_ARG, "rows per CTA 0 or 16..128, KV tiles per split 0..8");
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);
   x->attn_rows_cap = rows_per_cta;
@@ -1651,7 +1719,6 @@ nld_status nld_debug_timeout_chain(nld_ctx* x, unsigned long long timeout_ns) {
   A.bar = x->bars + kMaxPhases;   // layer 0's counters (left zero by every launch)
   A.boundary_pf = x->chain_boundary_pf;
   A.pf_stages = x->chain_pf_stages;
-  A.tmWn = A.ph[0].tmW;
   A.dbg_skip_arrive = 1;
   CK(launch_gemm_chain(x->stream, A, grid, timeout_ns, false));
   return NLD_OK;
@@ -1690,7 +1757,12 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
   if (batch < 1 || m < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_len < 1 || sms < 1)
     return fail(nullptr, NLD_ERR_ARG, "bad attention plan sizes");
   AttnArgs a{};
-  attn_plan(batch, m, Hq, Hkv, max_len, sms, a);
+  // pure host: clusters of S resident at once as if every SM held as many CTAs as its 228 KB of
+  // shared memory allows (one block reserves 1 KB)
+  attn_plan(batch, m, Hq, Hkv, max_len, sms, a, [sms](int S, int NW, int stages) {
+    const int per_sm = static_cast<int>(233472 / (attn_mma_smem_bytes(NW, true, stages) + 1024));
+    return std::max(1, sms * per_sm / S);
+  });
   out6[0] = a.G;
   out6[1] = a.QT;
   out6[2] = a.q_tiles;
@@ -1817,7 +1889,6 @@ static nld_status lm_head_launch(const void* d_hidden, const void* d_lm_weight, 
   e.lm_tiles = (vocab + kTileRows - 1) / kTileRows;
   e.V = vocab;
   e.err = err;
-  A.tmWn = P.tmW;
   // rms_stats clears the error word, the chain sets it when a wait runs out, and the combine
   // then writes argmax -1 and confidence 0 for every row instead of partials never written
   cudaError_t ce = launch_rms_stats(st, d_hidden, M, d, ssq, err);
@@ -1902,12 +1973,6 @@ nld_status nld_lm_head_argmax_static(const void* d_hidden, const void* d_lm_weig
 }
 
 // ----------------------------------------------------------------- stand-alone attention --
-static int device_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  cudaGetLastError();
-  return n;
-}
 
 nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* d_page_table,
                          int pages_per_seq, int n_pages, const int32_t* d_lens, int batch, int m,
@@ -1932,7 +1997,8 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
     }
   }
   AttnArgs a{};
-  attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a);
+  attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
+            [](int S, int NW, int stages) { return attn_device_capacity(false, S, NW, stages); });
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))

@@ -99,11 +99,16 @@ struct alignas(64) PhaseArgs {
                     // (rows past the tensor fill with zeros); 0: 2D [rows, K], box {64, xr}
 };
 
+// One phase of the next chain launch, as far as the L2 warm-up needs it.
+struct WarmPhase {
+  const void* W;    // pre-tiled weights of that phase
+  int s, tok_tiles, ks, KT, tiles;
+  int boxes;        // 16 KB weight boxes to prefetch per CTA (0 = none)
+};
+
 // A persistent launch running nph projections in order, separated by grid-wide arrivals.
 struct alignas(64) ChainArgs {
   PhaseArgs ph[kMaxPhases];
-  CUtensorMap tmWn;  // (unused by the pre-tiled path)
-  const void* Wn;    // pre-tiled weights of the projection that runs next on the stream (L2 warm-up)
   int nph;
   int CS;           // CTAs per cluster
   int NT;           // tokens per tile (multiple of 16; MMA N = NT << hilo <= 256)
@@ -122,9 +127,12 @@ struct alignas(64) ChainArgs {
   int pf_stages;    // L2 run-ahead: stages between a weight prefetch and its load (0 = off)
   int dbg_skip_arrive;   // test hook: CTA 0 withholds its phase-0 arrival, so every wait on that
                          // counter runs into its time limit (the failure-detection test)
-  // the next chain launch's first phase (L2 warm-up of each CTA's first weight boxes there)
+  // the next chain launch on the stream: before exiting, each CTA prefetches into L2 the first
+  // weight boxes that the CTA of the same index loads in that launch's first two phases, so HBM
+  // streams them while the kernels in between (attention) run
   int next_valid;
-  int next_CS, next_s, next_tok_tiles, next_ks, next_KT, next_grid, next_tiles, next_boxes;
+  int next_CS, next_grid;
+  WarmPhase next[2];
 };
 
 struct AttnArgs {
@@ -142,10 +150,12 @@ struct AttnArgs {
   const int* causal_seq;  // optional [batch]: nonzero makes all m rows of that sequence causal
   int QT, q_tiles, rows, S, NW;   // S = KV splits = cluster size (1..8)
   int min_tiles;        // KV tiles a split takes at least (1..)
+  int stages;           // K/V ring depth of the tensor-core path (2 or 3)
   float scale_log2;     // log2(e) / sqrt(hd)
   int hilo;             // tensor-core path: q fp32 [M, Hq, hd], out (hi, lo) bf16 rows [2M, Hq, hd]
   int quad_k;           // quadratic self-speculation forward with block k (0 = off): rows 0..k are
                         // causal; pre-draft row k+1+a*k+j sees the prefix, rows 0..a and its block
+  unsigned long long* trace;   // optional per-CTA timestamps (profiling hook), or null
   int* err;
 };
 

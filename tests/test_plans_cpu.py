@@ -1,10 +1,11 @@
 """Host logic of the launch planners, on CPU through the pure-host hooks nld_plan_chain and
 nld_plan_attention: every plan the library can make for the benchmark and test shapes keeps
 the kernels' limits (227 KB of shared memory, TMEM columns a power of two covering the
-double-buffered accumulator, split-K factors that give every rank work, <= 9 attention warps,
-<= 8 KV splits), and the plans at the benchmarked decode shape are the ones the committed
-launch list records (layer chain 132 CTAs in clusters of 4, layer-0 QKV 96 CTAs in clusters
-of 2, attention 7 x 8 CTAs of 288 / 256 threads in clusters of 7)."""
+double-buffered accumulator, split-K factors that give every rank work, <= 8 attention warps,
+<= 8 KV splits, no KV split left without a tile), and the plans at the benchmarked decode shape
+are the ones the committed launch list records (layer chain 132 CTAs in clusters of 4, layer-0
+QKV 96 CTAs in clusters of 2, attention in query tiles of <= 64 rows and single-tile KV
+splits)."""
 import ctypes
 
 import pytest
@@ -127,18 +128,25 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
                 assert A["G"] * cfg.n_kv_heads == cfg.n_q_heads, where
                 assert 1 <= A["QT"] <= m and A["QT"] * A["q_tiles"] >= m, where
                 assert A["rows"] == A["QT"] * A["G"] and A["rows"] <= 16 * A["NW"], where
-                assert 1 <= A["NW"] <= 9, where
+                assert 1 <= A["NW"] <= 8, where
                 assert 1 <= A["S"] <= 8, where
+                assert A["S"] <= -(-max_len // 64), where   # every split has a KV tile
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
                     assert A["S"] == 1, where
 
 
 def test_attention_plan_of_the_benchmarked_round():
-    # verify forward (m = 33) and draft forward (m = 32) at ~865 keys: 7 x 8 CTAs in clusters of 7
-    v = plan_attention(1, 33, 32, 8, 865)
-    d = plan_attention(1, 32, 32, 8, 865)
-    assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"]) == (4, 33, 1, 9, 7)
-    assert (d["NW"], d["S"]) == (8, 7)
+    # verify forward (m = 33: 3 query tiles of 11 positions x 4 heads, 3 warps) and draft forward
+    # (m = 32: 2 tiles of 16 positions, 4 warps); 545 keys = 9 tiles in 5 splits of <= 2 tiles,
+    # 865 keys = 14 tiles in 7 splits
+    for keys, S in ((545, 5), (865, 7)):
+        v = plan_attention(1, 33, 32, 8, keys)
+        d = plan_attention(1, 32, 32, 8, keys)
+        assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"]) == (4, 11, 3, 3, S)
+        assert (d["QT"], d["q_tiles"], d["NW"], d["S"]) == (16, 2, 4, S)
+    # many sequences: whole 128-row query tiles, no split
+    b = plan_attention(64, 33, 32, 8, 4096 + 33)
+    assert (b["QT"], b["NW"], b["S"]) == (17, 5, 1)
 
 
 def test_plan_hooks_reject_bad_sizes():
