@@ -322,14 +322,18 @@ nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_s
  * drops the captured graphs. */
 nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
 
-/* Profiling hook: while d_trace (device, n entries of 8 bytes, caller-owned) is set, every
- * tensor-core attention launch of the model's forwards whose grid fits (16 entries per CTA)
- * writes per CTA, at entry (CTA linear index) * 16 + i, the global timer in ns at: entry (0),
- * dependency on the previous kernel met (1), query tile staged (2), KV tile t done (3 + t,
- * t < 6), split partials published to the cluster (10), output written (11); later launches
- * overwrite earlier ones.  d_trace = NULL with n = 0 turns it off.  Synchronises and drops the
- * captured graphs. */
-nld_status nld_debug_attention_trace(nld_ctx* ctx, unsigned long long* d_trace, size_t n);
+/* Profiling hook: timestamps of one layer inside the model's own forwards (graph launches
+ * included).  While layer >= 0, the tensor-core attention launch of that layer (every forward;
+ * later ones overwrite) writes to d_attn_trace (device, n_attn uint64 entries, or NULL with
+ * n_attn = 0) if its grid fits, per CTA at (CTA linear index) * 16 + i the global timer in ns at:
+ * entry (0), dependency on the previous kernel met (1), query tile staged (2), KV tile t done
+ * (3 + t, t < 6), split partials published to the cluster (10), output written (11); and the
+ * chain launch that starts with that layer's O projection writes d_chain_trace (NULL, or at
+ * least 148*16 + 256 entries) in the layout of nld_trace_chain.  Buffers are caller-owned and
+ * zeroed by the caller.  layer = -1 turns the hook off.  Synchronises and drops the captured
+ * graphs. */
+nld_status nld_debug_layer_trace(nld_ctx* ctx, int layer, unsigned long long* d_attn_trace, size_t n_attn,
+                                 unsigned long long* d_chain_trace, size_t n_chain);
 
 /* Test hook for failure detection: one launch of layer 0's four-phase chain over the current
  * batch (scratch buffers only, as nld_time_chain) with every bounded wait limited to timeout_ns

@@ -75,7 +75,7 @@ def load_library() -> ctypes.CDLL:
         "nld_debug_chain_tuning": ([P, I, I, I, I, I, I], I),
         "nld_debug_timeout_chain": ([P, ctypes.c_ulonglong], I),
         "nld_debug_attention_tuning": ([P, I, I], I),
-        "nld_debug_attention_trace": ([P, P, S], I),
+        "nld_debug_layer_trace": ([P, I, P, S, P, S], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),
         "nld_attention": ([P, P, P, I, I, P, I, I, I, I, I, I, I, P, P], I),
@@ -236,11 +236,12 @@ class Context:
                                                     int(boundary_prefetch), int(act_3d),
                                                     int(runahead_stages), int(warm_next)), self.h)
 
-    def nld_debug_attention_trace(self, trace=None) -> None:
-        """trace: int64 device tensor (16 entries per CTA) or None to turn the hook off."""
-        n = 0 if trace is None else trace.numel()
-        self._check(self.lib.nld_debug_attention_trace(self.h, _ptr(trace) if trace is not None else None, n),
-                    self.h)
+    def nld_debug_layer_trace(self, layer: int = -1, attn_trace=None, chain_trace=None) -> None:
+        """Timestamp one layer's attention and chain launches (int64 device tensors, zeroed by
+        the caller); layer -1 turns the hook off."""
+        self._check(self.lib.nld_debug_layer_trace(
+            self.h, int(layer), _ptr(attn_trace), 0 if attn_trace is None else attn_trace.numel(),
+            _ptr(chain_trace), 0 if chain_trace is None else chain_trace.numel()), self.h)
 
     def nld_debug_attention_tuning(self, rows_per_cta: int = 0, min_tiles_per_split: int = 0) -> None:
         self._check(self.lib.nld_debug_attention_tuning(self.h, int(rows_per_cta), int(min_tiles_per_split)),

@@ -122,7 +122,7 @@ NLD_DEV void trace_mark(const ChainArgs& A, int slot) {
 // chunk written.
 NLD_DEV void trace_iter(const ChainArgs& A, int kind, int it) {
   if (A.trace && blockIdx.x == 0 && it >= 0 && it < 64)
-    A.trace[148 * 16 + kind * 64 + it] = globaltimer_ns();
+    A.trace[kChainTraceEntries - 4 * 64 + kind * 64 + it] = globaltimer_ns();
 }
 
 // The accumulator of chunk c (16 tokens) of a tile.  With hi/lo activations (rows 2t, 2t+1 =

@@ -148,8 +148,10 @@ struct nld_ctx {
   int chain_boundary_pf = 16;   // weight boxes prefetched into L2 per CTA at a phase boundary
   int chain_pf_stages = 0;      // L2 run-ahead distance in stages (0 = off)
   int chain_warm_next = 0;      // boxes of the next chain's second phase each CTA warms in L2
-  unsigned long long* attn_trace = nullptr;   // profiling hook: attention timestamps (or null)
+  int trace_layer = -1;        // profiling hook: the layer whose attention and chain launches
+  unsigned long long* attn_trace = nullptr;   // write timestamps (or -1 / null: off)
   size_t attn_trace_n = 0;
+  unsigned long long* chain_trace = nullptr;
   // host-side sequence bookkeeping
   int batch = 0;
   bool started = false;
@@ -604,6 +606,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
 
   const int max_len = static_cast<int>(std::min<long long>(x->kv_cap, x->len_upper + f.m));
   AttnArgs aa{};
+  bool attn_traced = false;
   aa.q = x->qbuf;
   aa.out = x->attn;
   aa.m = f.m;
@@ -625,7 +628,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
               [](int S, int NW, int stages) { return attn_device_capacity(true, S, NW, stages); },
               x->attn_rows_cap, x->attn_min_tiles);
     const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
-    if (x->attn_trace && ctas * 16 <= x->attn_trace_n) aa.trace = x->attn_trace;
+    attn_traced = x->attn_trace && ctas * 16 <= x->attn_trace_n;
   } else {
     aa.G = aa.Hq / aa.Hkv;
   }
@@ -663,6 +666,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   for (int l = 0; l < L; ++l) {
     if (x->bf16) {
       aa.layer_row0 = l * x->n_pages * 2 * x->c.n_kv_heads * kPage;
+      aa.trace = (attn_traced && l == x->trace_layer) ? x->attn_trace : nullptr;
       CK(launch_attention_mma(x->stream, &x->tmKV, aa, f.B, pdl));
     } else {
       aa.pool = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
@@ -683,7 +687,8 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
       // the phase boundary instead of after a kernel boundary
       cur[n++] = proj(GW_LM, 0);
     }
-    TRY(chain(x, cur, n, M, pdl, x->bars + (1 + l) * kMaxPhases, nn ? nxt : nullptr, nn));
+    TRY(chain(x, cur, n, M, pdl, x->bars + (1 + l) * kMaxPhases, nn ? nxt : nullptr, nn,
+              l == x->trace_layer ? x->chain_trace : nullptr));
   }
   return NLD_OK;
 }
@@ -1671,13 +1676,19 @@ nld_status nld_debug_chain_tuning(nld_ctx* x, int stage_cap, int k_tiles_per_sta
   return NLD_OK;
 }
 
-nld_status nld_debug_attention_trace(nld_ctx* x, unsigned long long* d_trace, size_t n) {
+nld_status nld_debug_layer_trace(nld_ctx* x, int layer, unsigned long long* d_attn_trace, size_t n_attn,
+                                 unsigned long long* d_chain_trace, size_t n_chain) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
-  if ((d_trace == nullptr) != (n == 0)) return fail(x, NLD_ERR_ARG, "trace buffer and size: both or neither");
+  if (layer >= x->c.n_layers || (d_attn_trace == nullptr) != (n_attn == 0) ||
+      (d_chain_trace != nullptr && n_chain < kChainTraceEntries))
+    return fail(x, NLD_ERR_ARG, "layer < n_layers; attention buffer and size both or neither; chain buffer >= %d entries",
+                kChainTraceEntries);
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);   // captured graphs hold the old launch parameters
-  x->attn_trace = d_trace;
-  x->attn_trace_n = n;
+  x->trace_layer = layer < 0 ? -1 : layer;
+  x->attn_trace = layer < 0 ? nullptr : d_attn_trace;
+  x->attn_trace_n = layer < 0 ? 0 : n_attn;
+  x->chain_trace = layer < 0 ? nullptr : d_chain_trace;
   return NLD_OK;
 }
 

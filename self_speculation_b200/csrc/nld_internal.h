@@ -81,6 +81,10 @@ struct EpiArgs {
   int* err;
 };
 
+// Entries of a chain launch's profiling trace: 16 per CTA (grid <= 148), then CTA 0's
+// per-iteration pipeline stamps (4 kinds x 64).
+constexpr int kChainTraceEntries = 148 * 16 + 4 * 64;
+
 // One projection of a chain launch.
 constexpr int kMaxPhases = 4;
 struct alignas(64) PhaseArgs {

@@ -56,7 +56,7 @@ def test_null_arguments_rejected():
     assert lib.nld_prefill(None, None, 1, None, 1, None) == 1
     assert lib.nld_debug_chain_tuning(None, 0, 0, 16, 1, 0, 0) == 1
     assert lib.nld_debug_timeout_chain(None, 1000000) == 1
-    assert lib.nld_debug_attention_trace(None, None, 0) == 1
+    assert lib.nld_debug_layer_trace(None, -1, None, 0, None, 0) == 1
     assert lib.nld_selfspec_round(None, None, None, None) == 1
     assert lib.nld_sync(None) == 1
     assert lib.nld_attention(None, None, None, 1, 1, None, 1, 32, 32, 8, 128, 1, 32, None, None) == 1
