@@ -22,7 +22,8 @@ namespace nld {
 // accumulator values where the caller can (a split tile loads them before waiting for its
 // group's partials), so a chunk costs at most one memory round trip.
 struct EpiPre {
-  float a[32];   // EPI_RESID: residual h of the 16 tokens; EPI_QKV: RoPE (cos, sin) of each
+  float a[16];   // EPI_RESID: residual h of the 16 tokens; EPI_QKV: RoPE cos (even feature
+                 // rows) or sin (odd rows) of each token: the pair's other thread holds the other
 };
 
 NLD_DEV void qkv_row_info(const EpiArgs& e, int row, int& sec, int& head, int& lr, int& feat) {
@@ -56,11 +57,10 @@ NLD_DEV void epi_preload(const EpiArgs& e, int row_tile, int row_in_tile, int to
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int pos = s_rpos[col0 + j];
-      const float2 cs = (sec < 2 && pos >= 0)
-                            ? __ldg(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)])
-                            : make_float2(1.f, 0.f);
-      p.a[2 * j] = cs.x;
-      p.a[2 * j + 1] = cs.y;
+      p.a[j] = (sec < 2 && pos >= 0)
+                   ? __ldg(reinterpret_cast<const float*>(&e.rope[static_cast<size_t>(pos) * half + (lr >> 1)]) +
+                           (lr & 1))
+                   : ((lr & 1) ? 0.f : 1.f);
     }
   }
 }
@@ -134,9 +134,12 @@ NLD_DEV void epi_chunk(const EpiArgs& e, int row_tile, int row_in_tile, int lane
 #pragma unroll
       for (int j = 0; j < 16; ++j) pt[j] = __shfl_xor_sync(0xffffffffu, x[j], 1);
       if (sec < 2) {
+        // rows 2i and 2i+1 (lanes l, l^1) rotate the same pair; each thread holds one of the
+        // pair's (cos, sin) and takes the other from its partner
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float c = pre.a[2 * j], sn = pre.a[2 * j + 1];
+          const float other = __shfl_xor_sync(0xffffffffu, pre.a[j], 1);
+          const float c = (lr & 1) ? other : pre.a[j], sn = (lr & 1) ? pre.a[j] : other;
           x[j] = (lr & 1) ? (x[j] * c + pt[j] * sn) : (x[j] * c - pt[j] * sn);
         }
       }

@@ -67,6 +67,10 @@ struct GemmTail {
   int pad;
   float red_f[2][80];   // per epilogue half (4 x 16 partials + 16 results)
   int red_i[2][80];
+  // the producer's queued activation loads (one thread; in shared memory, the dynamically
+  // indexed arrays stay out of local memory, which goes to L2 with the unified L1 given to the
+  // ring)
+  int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages], q_nk[kMaxStages];
   // followed in shared memory by the tile's per-column data: inv[NT], pos[NT], pg[NT], rpos[NT]
 };
 
@@ -254,7 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------- TMA producer --
       const uint64_t pol = l2_policy_evict_first();
-      int q_stage[kMaxStages], q_k[kMaxStages], q_tt[kMaxStages], q_nk[kMaxStages];
+      int* q_stage = tail->q_stage;
+      int* q_k = tail->q_k;
+      int* q_tt = tail->q_tt;
+      int* q_nk = tail->q_nk;
       int it = 0;
       int n_issued = 0;   // stages whose loads were issued
       bool ok = true;
