@@ -314,11 +314,11 @@ nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_s
                                   int boundary_prefetch, int act_3d, int runahead_stages,
                                   int warm_next);
 
-/* Profiling hook: attention planning.  rows_per_cta (16..128) caps the query rows (positions x
+/* Profiling hook: attention planning.  rows_per_cta (16..144) caps the query rows (positions x
  * query heads of one kv head) a CTA holds, so smaller values give more, lighter CTAs;
  * min_tiles_per_split (1..8) is the fewest 64-key tiles a KV split takes (more splits merge more
  * partials).  0 for either restores the planner's choice (the default): 64 rows and single-tile
- * splits when a few sequences leave most SMs idle, else 128 rows and 2 tiles.  Synchronises and
+ * splits when a few sequences leave most SMs idle, else 144 rows and 2 tiles.  Synchronises and
  * drops the captured graphs. */
 nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
 

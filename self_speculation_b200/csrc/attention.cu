@@ -29,8 +29,10 @@ namespace {
 constexpr int kMaxAttStages = 3;   // K/V ring depth: 2 or 3 (AttnArgs::stages)
 constexpr int kHalfTile = kPage * 64 * 2;        // 8 KB: 64 keys x 64 dims bf16
 constexpr int kKVTile = 2 * kHalfTile;           // 16 KB: 64 keys x 128 dims
-constexpr int kMaxAttWarps = 8;   // rows = positions x G <= 128 (the planner's query tile); at
-                                  // most two warps per SM sub-partition, so 255 registers each
+constexpr int kMaxAttWarps = 9;   // rows = positions x G <= 144 (the planner's query tile).  Up
+                                  // to 8 warps (two per SM sub-partition) a thread gets 255
+                                  // registers; the 9-warp form (a 33-position query tile of 4
+                                  // heads, many sequences) gets 168
 
 NLD_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -101,8 +103,8 @@ NLD_DEV bool key_visible(int key, int v1, int l2, int h2) { return key <= v1 || 
 // so only the bf16 K/V cache rounds; the output is written as (hi, lo) bf16 row pairs, the
 // operand layout of the O projection.  Otherwise (the stand-alone entry point) q and the output
 // are plain bf16 and P is rounded to bf16 for its MMA.
-template <bool kHiLo>
-__global__ void __launch_bounds__(32 * kMaxAttWarps, 1)
+template <bool kHiLo, int kMaxW>
+__global__ void __launch_bounds__(32 * kMaxW, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -569,6 +571,15 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const AttnArgs a) {
 
 cudaError_t gemm_tc_init_attributes();
 
+namespace {
+using AttnKernel = void (*)(const CUtensorMap, const AttnArgs);
+// The instantiation for a launch: its operand form and its launch bound (<= 8 or 9 warps).
+AttnKernel attn_kernel_for(bool hilo, int NW) {
+  if (NW > 8) return hilo ? attn_mma_kernel<true, 9> : attn_mma_kernel<false, 9>;
+  return hilo ? attn_mma_kernel<true, 8> : attn_mma_kernel<false, 8>;
+}
+}  // namespace
+
 // Shared-memory opt-ins of the large-smem kernels (host, once per process and device).
 cudaError_t init_kernel_attributes() {
   cudaError_t e = gemm_tc_init_attributes();
@@ -577,14 +588,15 @@ cudaError_t init_kernel_attributes() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel<false>)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(attn_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                optin - static_cast<int>(fa.sharedSizeBytes))) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncGetAttributes(&fa, attn_mma_kernel<true>)) != cudaSuccess) return e;
-  return cudaFuncSetAttribute(attn_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              optin - static_cast<int>(fa.sharedSizeBytes));
+  for (int v = 0; v < 4; ++v) {
+    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8);
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  optin - static_cast<int>(fa.sharedSizeBytes))) != cudaSuccess)
+      return e;
+  }
+  return cudaSuccess;
 }
 
 // Dynamic shared memory of a launch: the K/V ring and the query tile (hi and lo halves with
@@ -610,8 +622,7 @@ int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t e = hilo ? cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<true>, &cfg)
-                             : cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<false>, &cfg);
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, attn_kernel_for(hilo, NW), &cfg);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return sms / S;
@@ -641,8 +652,7 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   if (pdl) attrs[na++] = attr[0];
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  if (a.hilo) return cudaLaunchKernelEx(&cfg, attn_mma_kernel<true>, *tmKV, a);
-  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<false>, *tmKV, a);
+  return cudaLaunchKernelEx(&cfg, attn_kernel_for(a.hilo != 0, a.NW), *tmKV, a);
 }
 
 cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,

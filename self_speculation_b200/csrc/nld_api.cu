@@ -477,7 +477,7 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
 // Clusters of S attention CTAs (NW warps, `stages` ring stages) resident at once.
 using AttnCapacity = std::function<int(int S, int NW, int stages)>;
 
-// rows_cap: query rows (positions x heads) per CTA at most (16..128: 8 warps); min_tiles: KV
+// rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
 // tiles a split takes at least; 0 = the planner's choice for either.
 void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
                int rows_cap = 0, int min_tiles = 0) {
@@ -491,10 +491,10 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // idle, so the query positions are cut into tiles of <= 64 rows (one warp per SM
   // sub-partition: a KV tile then costs a quarter of the MMA time of an 8-warp CTA), the keys
   // into splits of single tiles, and the ring holds 2 stages (about 100 KB, two CTAs per SM).
-  // Otherwise tiles of up to 128 rows read each K/V tile once for as many query rows as
-  // possible, through a 3-stage ring.
-  const bool latency = batch * Hkv * q_tiles_for(128) * 8 < 2 * sms;
-  if (rows_cap <= 0) rows_cap = latency ? 64 : 128;
+  // Otherwise tiles of up to 144 rows (a 33-position verify block of 4 heads in one 9-warp
+  // CTA) read each K/V tile once for as many query rows as possible, through a 3-stage ring.
+  const bool latency = batch * Hkv * q_tiles_for(144) * 8 < 2 * sms;
+  if (rows_cap <= 0) rows_cap = latency ? 64 : 144;
   if (min_tiles <= 0) min_tiles = latency ? 1 : 2;
   a.min_tiles = min_tiles;
   a.stages = latency ? 2 : 3;
@@ -520,9 +520,9 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
 
 // The device's cluster capacity for the attention kernel (occupancy query, cached).
 int attn_device_capacity(bool hilo, int S, int NW, int stages) {
-  static int cache[16][9][9][2][4];   // [device][S][NW][hilo][stages]; 0 = not yet queried
+  static int cache[16][9][10][2][4];   // [device][S][NW][hilo][stages]; 0 = not yet queried
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 16 || S < 1 || S > 8 || NW < 1 || NW > 8 || stages < 2 ||
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 16 || S < 1 || S > 8 || NW < 1 || NW > 9 || stages < 2 ||
       stages > 3) {
     cudaGetLastError();
     return 1;
@@ -1694,9 +1694,9 @@ nld_status nld_debug_layer_trace(nld_ctx* x, int layer, unsigned long long* d_at
 
 nld_status nld_debug_attention_tuning(nld_ctx* x, int rows_per_cta, int min_tiles_per_split) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
-  if ((rows_per_cta != 0 && (rows_per_cta < 16 || rows_per_cta > 128)) || min_tiles_per_split < 0 ||
+  if ((rows_per_cta != 0 && (rows_per_cta < 16 || rows_per_cta > 144)) || min_tiles_per_split < 0 ||
       min_tiles_per_split > 8)
-    return fail(x, NLD_ERR_ARG, "rows per CTA 0 or 16..128, KV tiles per split 0..8");
+    return fail(x, NLD_ERR_ARG, "rows per CTA 0 or 16..144, KV tiles per split 0..8");
   CK(cudaStreamSynchronize(x->stream));
   drop_graphs(x);
   x->attn_rows_cap = rows_per_cta;

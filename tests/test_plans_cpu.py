@@ -1,7 +1,7 @@
 """Host logic of the launch planners, on CPU through the pure-host hooks nld_plan_chain and
 nld_plan_attention: every plan the library can make for the benchmark and test shapes keeps
 the kernels' limits (227 KB of shared memory, TMEM columns a power of two covering the
-double-buffered accumulator, split-K factors that give every rank work, <= 8 attention warps,
+double-buffered accumulator, split-K factors that give every rank work, <= 9 attention warps,
 <= 8 KV splits, no KV split left without a tile), and the plans at the benchmarked decode shape
 are the ones the committed launch list records (layer chain 132 CTAs in clusters of 4, layer-0
 QKV 96 CTAs in clusters of 2, attention in query tiles of <= 64 rows and single-tile KV
@@ -128,7 +128,7 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
                 assert A["G"] * cfg.n_kv_heads == cfg.n_q_heads, where
                 assert 1 <= A["QT"] <= m and A["QT"] * A["q_tiles"] >= m, where
                 assert A["rows"] == A["QT"] * A["G"] and A["rows"] <= 16 * A["NW"], where
-                assert 1 <= A["NW"] <= 8, where
+                assert 1 <= A["NW"] <= 9 and A["rows"] <= 144, where
                 assert 1 <= A["S"] <= 8, where
                 assert A["S"] <= -(-max_len // 64), where   # every split has a KV tile
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
@@ -144,9 +144,9 @@ def test_attention_plan_of_the_benchmarked_round():
         d = plan_attention(1, 32, 32, 8, keys)
         assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"]) == (4, 11, 3, 3, S)
         assert (d["QT"], d["q_tiles"], d["NW"], d["S"]) == (16, 2, 4, S)
-    # many sequences: whole 128-row query tiles, no split
+    # many sequences: the whole 33-position verify block of 4 heads in one 9-warp CTA, no split
     b = plan_attention(64, 33, 32, 8, 4096 + 33)
-    assert (b["QT"], b["NW"], b["S"]) == (17, 5, 1)
+    assert (b["QT"], b["q_tiles"], b["NW"], b["S"]) == (33, 1, 9, 1)
 
 
 def test_plan_hooks_reject_bad_sizes():
