@@ -350,8 +350,9 @@ def run_ours(args, world, rank, local):
 
     # two forwards (draft, verify), each: embed, QKV chain of layer 0, per layer one attention
     # and one chain (O, gate/up, down, then the next QKV or, last, the LM head); then finalize
-    # for draft, verify and commit
-    per_round = 2 * (1 + 1 + 2 * cfg.n_layers) + 3 + (2 * cfg.n_layers if args.lora else 0)
+    # for draft, verify and commit; with an adapter the draft forward has one more launch per
+    # layer (z = scale A att; B is folded into the chain's O projection)
+    per_round = 2 * (1 + 1 + 2 * cfg.n_layers) + 3 + (cfg.n_layers if args.lora else 0)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,

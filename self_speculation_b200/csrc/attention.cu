@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
     const int p = r / a.G, gq = r - p * a.G;
     const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
     const size_t orow = kHiLo ? 2 * tok + part : tok;
-    return static_cast<__nv_bfloat16*>(a.out) + ((orow * a.Hq) + g * a.G + gq) * 128;
+    return static_cast<__nv_bfloat16*>(a.out) + orow * a.out_ld + static_cast<size_t>(g * a.G + gq) * 128;
   };
   // store the pair (x0, x1) at column d of output row r
   auto store2 = [&](int r, int d, float x0, float x1) {

@@ -393,9 +393,23 @@ cudaError_t launch_finalize(cudaStream_t st, const FinalizeArgs& a, int batch, b
 constexpr int kLoraJ = 16, kLoraT = 32, kLoraThreads = 256;
 template <typename T> struct LoraCols { static constexpr int n = 512 / sizeof(T); };
 
+// With a counter array (the folded form, bf16 (hi, lo) forwards only): the CTA that completes a
+// (16 adapter rows, 32 tokens) block last sums its slices in slice order (deterministic), scales
+// by `scale` and writes z as (hi, lo) bf16 pairs into columns qd + j of rows 2t, 2t+1 of zout
+// (pitch ld), zero for rows that are not drafter rows (as lora_up skips them).
+struct LoraFinal {
+  int* cnt;           // [gridDim.x * gridDim.z] zero counters, left zero
+  __nv_bfloat16* zout;
+  size_t ld;
+  float scale;
+  int m, causal_rows;
+  const int* causal_seq;
+};
+
 template <typename T, bool kHiLo>
-__global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, const T* att, float* zp,
-                                                                 int M, int qd, int r) {
+__global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, const T* att, size_t att_ld,
+                                                                 float* zp, int M, int qd, int r,
+                                                                 const LoraFinal fin) {
   constexpr int C = LoraCols<T>::n, LD = C + 2, V = 16 / sizeof(T);
   constexpr int kXRows = kHiLo ? 2 * kLoraT : kLoraT;   // with hi/lo: rows 2t, 2t+1 per token
   __shared__ __align__(16) T sA[kLoraJ][LD];
@@ -417,7 +431,7 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
       } else if (((row - kLoraJ) >> (kHiLo ? 1 : 0)) + t0 < M) {
         // att row index: token t0 + i (plain) or row 2 t0 + i of the (hi, lo) pairs
         const size_t arow = (kHiLo ? 2 * static_cast<size_t>(t0) : static_cast<size_t>(t0)) + (row - kLoraJ);
-        v[u] = *reinterpret_cast<const uint4*>(att + arow * qd + c);
+        v[u] = *reinterpret_cast<const uint4*>(att + arow * att_ld + c);
       }
     }
   }
@@ -468,6 +482,29 @@ __global__ void __launch_bounds__(kLoraThreads) lora_down_kernel(const T* A, con
     if (j < r) out[j] = a0;
     if (j + 1 < r) out[j + 1] = a1;
   }
+  if (fin.cnt == nullptr) return;
+  // folded form: the block's last slice CTA (release/acquire through the counter) sums
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  int* cnt = fin.cnt + blockIdx.x * gridDim.z + blockIdx.z;
+  if (threadIdx.x == 0) s_last = (atomicAdd(cnt, 1) == static_cast<int>(gridDim.y) - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < kLoraJ * kLoraT; e += kLoraThreads) {
+    const int jj = j0 + e % kLoraJ, tt = t0 + e / kLoraJ;
+    if (jj >= r || tt >= M) continue;
+    float acc = 0.f;
+    for (int ks = 0; ks < static_cast<int>(gridDim.y); ++ks)   // slice order; other CTAs' writes: not L1
+      acc += __ldcg(zp + (static_cast<size_t>(ks) * M + tt) * r + jj);
+    const bool drafter = (tt % fin.m) >= fin.causal_rows && !(fin.causal_seq && fin.causal_seq[tt / fin.m]);
+    __nv_bfloat16 hi, lo;
+    split_bf16(drafter ? fin.scale * acc : 0.f, hi, lo);
+    fin.zout[(2 * static_cast<size_t>(tt)) * fin.ld + qd + jj] = hi;
+    fin.zout[(2 * static_cast<size_t>(tt) + 1) * fin.ld + qd + jj] = lo;
+  }
+  if (threadIdx.x == 0) *cnt = 0;   // every CTA of the block has arrived
 }
 
 // h[t][i] += scale * sum_j B[i][j] z[t][j], z = the activation-type rounding of the summed
@@ -577,26 +614,45 @@ cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const voi
   if (bf16 && hilo) {
     using T = __nv_bfloat16;
     e = cudaLaunchKernelEx(&c1, lora_down_kernel<T, true>, static_cast<const T*>(A), static_cast<const T*>(att),
-                           zp, M, qd, r);
+                           static_cast<size_t>(qd), zp, M, qd, r, LoraFinal{});
     if (e == cudaSuccess)
       e = cudaLaunchKernelEx(&c2, lora_up_kernel<T, true>, static_cast<const T*>(B), static_cast<const float*>(zp),
                              h, M, d, r, n_ks, scale, m, causal_rows, causal_seq);
   } else if (bf16) {
     using T = __nv_bfloat16;
     e = cudaLaunchKernelEx(&c1, lora_down_kernel<T, false>, static_cast<const T*>(A), static_cast<const T*>(att),
-                           zp, M, qd, r);
+                           static_cast<size_t>(qd), zp, M, qd, r, LoraFinal{});
     if (e == cudaSuccess)
       e = cudaLaunchKernelEx(&c2, lora_up_kernel<T, false>, static_cast<const T*>(B), static_cast<const float*>(zp),
                              h, M, d, r, n_ks, scale, m, causal_rows, causal_seq);
   } else {
     e = cudaLaunchKernelEx(&c1, lora_down_kernel<float, false>, static_cast<const float*>(A),
-                           static_cast<const float*>(att), zp, M, qd, r);
+                           static_cast<const float*>(att), static_cast<size_t>(qd), zp, M, qd, r, LoraFinal{});
     if (e == cudaSuccess)
       e = cudaLaunchKernelEx(&c2, lora_up_kernel<float, false>, static_cast<const float*>(B),
                              static_cast<const float*>(zp), h, M, d, r, n_ks, scale, m, causal_rows,
                              causal_seq);
   }
   return e;
+}
+
+cudaError_t launch_lora_z(cudaStream_t st, const void* A, const void* att, size_t att_ld, float* zp,
+                          int* cnt, void* zout, size_t ld, int M, int qd, int r, float scale, int m,
+                          int causal_rows, const int* causal_seq, bool pdl) {
+  if (r < 8 || r > 256 || r % 8 || M < 1 || !cnt || !zout) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c1 = {};
+  c1.gridDim = dim3((r + kLoraJ - 1) / kLoraJ, lora_n_ks(qd, true), (M + kLoraT - 1) / kLoraT);
+  c1.blockDim = dim3(kLoraThreads);
+  c1.stream = st;
+  c1.attrs = attr;
+  c1.numAttrs = pdl ? 1 : 0;
+  using T = __nv_bfloat16;
+  const LoraFinal fin{cnt, static_cast<T*>(zout), ld, scale, m, causal_rows, causal_seq};
+  return cudaLaunchKernelEx(&c1, lora_down_kernel<T, true>, static_cast<const T*>(A), static_cast<const T*>(att),
+                            att_ld, zp, M, qd, r, fin);
 }
 
 // -------------------------------------------------------------------------------- repack --

@@ -75,8 +75,10 @@ bool make_map_tiled(CUtensorMap* map, const void* base, int n_rows, int K) {
   return make_map_bf16(map, base, kTileK, row_tiles * (K / kTileK) * kTileRows, kTileRows);
 }
 
-enum XBuf { XB_HB = 0, XB_ATTN = 1, XB_U = 2 };
-enum GemmWhich { GW_QKV = 0, GW_O = 1, GW_GU = 2, GW_D = 3, GW_LM = 4 };
+enum XBuf { XB_HB = 0, XB_ATTN = 1, XB_U = 2, XB_ATTZ = 3 };
+// GW_OL: the O projection of a drafter forward with the adapter folded in ([W_o | B] over
+// [att ; scale * A att], bf16 configuration)
+enum GemmWhich { GW_QKV = 0, GW_O = 1, GW_GU = 2, GW_D = 3, GW_LM = 4, GW_OL = 5 };
 enum LmKind { LM_NONE = 0, LM_ARGMAX = 1, LM_LOGITS = 2 };
 
 std::string g_static_err;
@@ -103,6 +105,12 @@ struct nld_ctx {
   float lora_scale = 0.f;
   std::vector<void*> lora_A, lora_B;
   float* lora_zp = nullptr;
+  // folded adapter (bf16): attention output rows with r_pad more columns for z = scale A att,
+  // [W_o | B] per layer (pre-tiled, K = qd + r_pad), block counters of the z kernel
+  int lora_rpad = 0;
+  void* attz = nullptr;
+  std::vector<void*> wol;
+  int* lora_cnt = nullptr;
   // KV cache
   void* pool = nullptr;
   int* page_table = nullptr;
@@ -276,8 +284,9 @@ const CUtensorMap* xmap(nld_ctx* x, int buf, int rows, int kps, int* is3d) {
     return &it->second.first;
   }
   CUtensorMap m;
-  const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : x->ubuf);
-  const int inner = buf == XB_HB ? x->c.d_model : (buf == XB_ATTN ? x->qd : x->c.ffn_dim);
+  const void* base = buf == XB_HB ? x->hb : (buf == XB_ATTN ? x->attn : (buf == XB_ATTZ ? x->attz : x->ubuf));
+  const int inner = buf == XB_HB ? x->c.d_model
+                                 : (buf == XB_ATTN ? x->qd : (buf == XB_ATTZ ? x->qd + x->lora_rpad : x->c.ffn_dim));
   // bf16 activations are (hi, lo) row pairs: 2 M_max rows
   int d3 = 0;
   if (x->chain_x3d && make_map_act3d(&m, base, inner, 2ull * x->M_max, rows, kps)) {
@@ -304,6 +313,7 @@ WInfo winfo(nld_ctx* x, int which, int layer) {
     case GW_O: w = {x->c.d_model, x->qd, XB_ATTN, x->wo[layer], x->bf16 ? &x->tmWo[layer] : nullptr}; break;
     case GW_GU: w = {x->gu_rows, x->c.d_model, XB_HB, x->wgu[layer], x->bf16 ? &x->tmWgu[layer] : nullptr}; break;
     case GW_D: w = {x->c.d_model, x->c.ffn_dim, XB_U, x->wd[layer], x->bf16 ? &x->tmWd[layer] : nullptr}; break;
+    case GW_OL: w = {x->c.d_model, x->qd + x->lora_rpad, XB_ATTZ, x->wol[layer], &x->tmWo[layer]}; break;
     default: w = {x->c.vocab, x->c.d_model, XB_HB, x->wlm, x->bf16 ? &x->tmWlm : nullptr}; break;
   }
   return w;
@@ -608,7 +618,13 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   AttnArgs aa{};
   bool attn_traced = false;
   aa.q = x->qbuf;
-  aa.out = x->attn;
+  // drafter forwards of a context with an adapter: on the tensor-core path the adapter is folded
+  // into the O projection; the attention writes rows with room for z
+  const bool lora_fwd = x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF ||
+                                          f.mode == FWD_NLDIFF || f.mode == FWD_QUAD);
+  const bool folded = lora_fwd && x->bf16;
+  aa.out = folded ? x->attz : x->attn;
+  aa.out_ld = static_cast<size_t>(x->qd) + (folded ? x->lora_rpad : 0);
   aa.m = f.m;
   aa.Hq = x->c.n_q_heads;
   aa.Hkv = x->c.n_kv_heads;
@@ -639,7 +655,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   auto proj = [&](int which, int layer) {
     ProjRef r{which, layer, base_epi(x, M, f.m)};
     r.e.quad_k = f.quad_k;
-    static const int kinds[5] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD};
+    static const int kinds[6] = {EPI_QKV, EPI_RESID, EPI_SWIGLU, EPI_RESID, EPI_LMHEAD, EPI_RESID};
     r.e.kind = kinds[which];
     if (which == GW_QKV)
       r.e.kv_layer = static_cast<char*>(x->pool) + static_cast<size_t>(layer) * x->layer_elems * x->el;
@@ -651,7 +667,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   };
   auto layer_chain = [&](int l, ProjRef* out) {
     int n = 0;
-    out[n++] = proj(GW_O, l);
+    out[n++] = proj(folded ? GW_OL : GW_O, l);
     out[n++] = proj(GW_GU, l);
     out[n++] = proj(GW_D, l);
     if (l + 1 < L) out[n++] = proj(GW_QKV, l + 1);
@@ -672,9 +688,13 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
       aa.pool = static_cast<char*>(x->pool) + static_cast<size_t>(l) * x->layer_elems * x->el;
       CK(launch_attention_simt(x->stream, aa, f.B, true, x->kv_cap, pdl));
     }
-    // LoRA drafter: the block-bidirectional rows (the fused fill's causal rows excluded)
-    if (x->lora_r > 0 && (f.mode == FWD_DRAFT || f.mode == FWD_DIFFUSE || f.mode == FWD_FILLDIFF ||
-                          f.mode == FWD_NLDIFF || f.mode == FWD_QUAD))
+    // LoRA drafter: the block-bidirectional rows (the fused fill's causal rows excluded).  Folded
+    // (bf16): one launch writes z = scale * A att beside the attention output, and the chain's
+    // O projection takes B as r_pad more K columns; fp32: z, then h += scale * B z
+    if (folded)
+      CK(launch_lora_z(x->stream, x->lora_A[l], x->attz, aa.out_ld, x->lora_zp, x->lora_cnt, x->attz, aa.out_ld,
+                       M, x->qd, x->lora_r, x->lora_scale, f.m, f.causal_rows, f.causal_seq, pdl));
+    else if (lora_fwd)
       CK(launch_lora(x->stream, x->lora_A[l], x->lora_B[l], x->attn, x->lora_zp, x->h, M, x->qd,
                      x->c.d_model, x->lora_r, x->lora_scale, f.m, f.causal_rows, f.causal_seq,
                      x->bf16, x->bf16, pdl));
@@ -991,6 +1011,55 @@ nld_status nld_init_lora(nld_ctx* x, int rank, float scale, const void* const* t
   for (int l = 0; l < L; ++l) {
     CK(cudaMemcpyAsync(x->lora_A[l], tensors[2 * l], static_cast<size_t>(rank) * x->qd * el, kind, x->stream));
     CK(cudaMemcpyAsync(x->lora_B[l], tensors[2 * l + 1], static_cast<size_t>(d) * rank * el, kind, x->stream));
+  }
+  if (x->bf16) {
+    // the folded adapter: [W_o | B] per layer as pre-tiled blocks (row tile, k tile), K = qd +
+    // r_pad (B's columns zero-padded to a whole k tile), and the attention output buffer with
+    // r_pad more columns per (hi, lo) row for z
+    const int rpad = (rank + kTileK - 1) / kTileK * kTileK;
+    const int KT = x->qd / kTileK, KB = rpad / kTileK, KTL = KT + KB, RT = d / kTileRows;
+    const size_t blk = static_cast<size_t>(kTileRows) * kTileK * el;   // 16 KB
+    if (x->wol.empty()) {
+      std::vector<void*> wol(L, nullptr);
+      void* attz = nullptr;
+      int* cnt = nullptr;
+      for (int l = 0; l < L; ++l)
+        if ((s = dalloc(x, &wol[l], static_cast<size_t>(RT) * KTL * blk)) != NLD_OK) return s;
+      const size_t zrows = 2ull * x->M_max;
+      if ((s = dalloc(x, &attz, zrows * (x->qd + rpad) * el)) != NLD_OK) return s;
+      const size_t ncnt = static_cast<size_t>((256 + 15) / 16) * ((x->M_max + 31) / 32);
+      if ((s = dalloc(x, &cnt, ncnt * sizeof(int))) != NLD_OK) return s;
+      CK(cudaMemsetAsync(attz, 0, zrows * (x->qd + rpad) * el, x->stream));
+      CK(cudaMemsetAsync(cnt, 0, ncnt * sizeof(int), x->stream));
+      x->wol.swap(wol);
+      x->attz = attz;
+      x->lora_cnt = cnt;
+      x->lora_rpad = rpad;
+      x->tmX.clear();
+    }
+    void* stage = nullptr;
+    void* tiled = nullptr;
+    CK(cudaMalloc(&stage, static_cast<size_t>(d) * rpad * el));
+    if (cudaMalloc(&tiled, static_cast<size_t>(RT) * KB * blk) != cudaSuccess) {
+      cudaFree(stage);
+      return fail(x, NLD_ERR_CUDA, "out of device memory (adapter staging)");
+    }
+    cudaError_t e = cudaMemsetAsync(stage, 0, static_cast<size_t>(d) * rpad * el, x->stream);
+    for (int l = 0; l < L && e == cudaSuccess; ++l) {
+      e = cudaMemcpy2DAsync(x->wol[l], KTL * blk, x->wo[l], KT * blk, KT * blk, RT, cudaMemcpyDeviceToDevice,
+                            x->stream);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(stage, rpad * el, x->lora_B[l], rank * el, rank * el, d, cudaMemcpyDeviceToDevice,
+                              x->stream);
+      if (e == cudaSuccess) e = launch_repack(x->stream, tiled, stage, nullptr, d, rpad, nullptr, true, true);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(static_cast<char*>(x->wol[l]) + KT * blk, KTL * blk, tiled, KB * blk, KB * blk, RT,
+                              cudaMemcpyDeviceToDevice, x->stream);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(x->stream);
+    cudaFree(stage);
+    cudaFree(tiled);
+    if (e != cudaSuccess) return fail(x, NLD_ERR_CUDA, "folding the adapter failed: %s", cudaGetErrorString(e));
   }
   CK(cudaStreamSynchronize(x->stream));
   x->lora_r = rank;
@@ -2016,6 +2085,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
     return fail(nullptr, NLD_ERR_CUDA, "tensor map encode failed (pool)");
   a.q = d_q;
   a.out = d_out;
+  a.out_ld = static_cast<size_t>(n_q_heads) * 128;
   a.m = m;
   a.Hq = n_q_heads;
   a.Hkv = n_kv_heads;

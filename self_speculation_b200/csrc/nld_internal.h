@@ -141,7 +141,8 @@ struct alignas(64) ChainArgs {
 
 struct AttnArgs {
   const void* q;        // [M, Hq, hd]
-  void* out;            // [M, Hq, hd]
+  void* out;            // [M, Hq, hd] rows out_ld elements apart (tensor-core path)
+  size_t out_ld;
   const void* pool;     // SIMT path: pool base of this layer
   int m, Hq, Hkv, G, hd;
   const int* lens;
@@ -216,6 +217,13 @@ cudaError_t launch_fill_i32(cudaStream_t st, int* p, int value, int n);
 // attention output, and z stays fp32; otherwise z is rounded to the activation type.
 // A [r, qd], B [d, r] row-major; 8 <= r <= 256, r % 8 == 0; qd a multiple of 8.
 int lora_n_ks(int qd, bool bf16);
+// The drafter's z = scale * A att of the bf16 (hi, lo) forward, written as (hi, lo) bf16 into
+// columns qd..qd+r of the rows of zout (row pitch ld; rows 2t, 2t+1), where the O projection of
+// the layer chain reads it as r more K columns against scale-free B (the folded adapter).
+// cnt: [ceil(r/16) * ceil(M/32)] zero counters (left zero).
+cudaError_t launch_lora_z(cudaStream_t st, const void* A, const void* att, size_t att_ld, float* zp,
+                          int* cnt, void* zout, size_t ld, int M, int qd, int r, float scale, int m,
+                          int causal_rows, const int* causal_seq, bool pdl);
 cudaError_t launch_lora(cudaStream_t st, const void* A, const void* B, const void* att, float* zp,
                         float* h, int M, int qd, int d, int r, float scale, int m, int causal_rows,
                         const int* causal_seq, bool bf16, bool hilo, bool pdl);
