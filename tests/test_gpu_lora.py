@@ -4,9 +4,11 @@ block-bidirectional forwards only (Nemotron-Labs-Diffusion notes, ranhao.site, s
 fp32 tiny model (rank 8): draft logits within 1e-4 of the fp64 oracle with the same adapter,
 verify and AR logits equal to the adapter-free oracle's, token-exact self-speculation (with
 the oracle's per-round acceptance counts, which depend on the drafts) and diffusion (unfused
-and fused fill).  bf16 small model (rank 128, the pages' rank): draft logits within 2e-2 of
-the rounding-matched oracle.  Host logic: rank changes are refused, rank 0 switches the
-adapter off and the forwards return to the adapter-free results bit for bit.
+and fused fill).  bf16 (the adapter folded into the layer chain: z = scale * A att beside the
+attention output, B as more K columns of the O projection): draft and diffusion logits of the
+small model (rank 128, the pages' rank; rank 16, zero-padded to a whole k tile) and draft
+logits at the 8B layer shape within 2e-2 of the oracle.  Host logic: rank changes are refused,
+rank 0 switches the adapter off and the forwards return to the adapter-free results bit for bit.
 """
 import pytest
 import torch
@@ -164,3 +166,19 @@ def test_rank_rules_and_switch_off_bit_exact():
     # the same rank loads again: back to the adapter's logits
     ctx.nld_init_lora(16, 4.0, flat)
     assert torch.equal(gpu_logits(ctx, 1, 1, k), on)
+
+
+def test_draft_logits_bf16_rank128_8b_layer_shape():
+    # the bench's adapter shape: K = 4096 + 128 over split 4 (17 / 17 / 17 / 15 k tiles)
+    cfg = synth.LLAMA8B.replace(n_layers=2, max_seq=512)
+    ctx, om, W = make_pair(cfg, device_weights=True)
+    A, B = _adapter(cfg, 128, seed=5, std=0.02)
+    _load(ctx, om, A, B, 1.0)
+    p = synth.prompt_tokens(1, 100, cfg.vocab, seed=11)
+    ctx.nld_prefill(p.cuda())
+    st = odec.prefill(om, p, cfg.max_seq + 64)
+    k = cfg.block_k
+    gl = gpu_logits(ctx, 1, 1, k)
+    ol = odec.draft_forward(om, st, k)
+    assert (gl.double() - ol.double()).abs().max().item() < 2e-2
+    ctx.close()
