@@ -537,6 +537,8 @@ int attn_device_capacity(bool hilo, int S, int NW, int stages) {
     cudaGetLastError();
     return 1;
   }
+  static std::mutex mu;   // the stand-alone attention may be called from several threads
+  std::lock_guard<std::mutex> lock(mu);
   int& c = cache[dev][S][NW][hilo ? 1 : 0][stages];
   if (c == 0) c = attn_mma_max_clusters(S, NW, hilo, stages, device_sms());
   return c;
