@@ -211,7 +211,9 @@ nld_status nld_diffuse_block_step(nld_ctx* ctx, float threshold, int32_t* d_bloc
  * outputs as nld_diffuse_block_step; *h_filled_out = 1 when this call performed a deferred
  * fill (len += k, pending = b_k happened here).  A fill still deferred runs alone at the start
  * of the next nld_diffuse_block_step, nld_ar_step, nld_selfspec_* or nld_debug_logits call
- * (nld_debug_state reports the state before it).  Needs 2k <= 64 and batch*2k token rows
+ * (nld_debug_state reports the state before it).  Past 256 token rows (batch*2k) the merged
+ * forward is compute-bound and no cheaper than two, so the call then runs the fill and the step
+ * as two forwards (same outputs and state).  Needs 2k <= 64 and batch*2k token rows
  * (NLD_ERR_UNSUPPORTED otherwise). */
 nld_status nld_diffuse_block_step_fused(nld_ctx* ctx, float threshold, int32_t* d_block_out,
                                         float* d_conf_out, int32_t* d_ncommit_out,

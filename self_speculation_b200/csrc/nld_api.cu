@@ -1559,14 +1559,23 @@ nld_status nld_diffuse_block_step(nld_ctx* x, float threshold, int32_t* d_block_
   return NLD_OK;
 }
 
+// Largest forward (batch x 2k token rows) that runs the fused fill as one forward.
+constexpr int kFusedFillRows = 256;
+
 nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_block_out,
                                         float* d_conf_out, int32_t* d_ncommit_out, int32_t* h_filled_out) {
   TRY(need_started(x));
   TRY(flush_nl(x));
   const int k = x->c.block_k;
-  const bool fused = x->fill_pending;
-  if (fused && (2 * k > 64 || x->batch * 2 * k > x->M_max))
+  const bool filling = x->fill_pending;
+  if (filling && (2 * k > 64 || x->batch * 2 * k > x->M_max))
     return fail(x, NLD_ERR_UNSUPPORTED, "fused fill needs 2k <= 64 and batch*2k <= %d rows", x->M_max);
+  // The 2k-row forward saves a weight stream while the forward is bound by HBM; past
+  // kFusedFillRows token rows the (hi, lo) products make it compute-bound and it costs as much
+  // as the two forwards it replaces, so the fill then runs alone first (same results: the two
+  // forms are equal in exact arithmetic)
+  const bool fused = filling && x->batch * 2 * k <= kFusedFillRows;
+  if (filling && !fused) TRY(run_fill(x));
   TRY(ensure_capacity(x, fused ? 2 * k : k));
   int open = 1;
   TRY(run_denoise(x, fused, threshold, d_block_out, d_conf_out, d_ncommit_out, &open));
@@ -1575,7 +1584,7 @@ nld_status nld_diffuse_block_step_fused(nld_ctx* x, float threshold, int32_t* d_
     x->fill_pending = false;
   }
   if (open == 0) x->fill_pending = true;   // this block's fill joins the next step
-  if (h_filled_out) *h_filled_out = fused ? 1 : 0;
+  if (h_filled_out) *h_filled_out = filling ? 1 : 0;
   x->verify_fresh = false;
   x->quad_ready = false;
   return NLD_OK;
