@@ -324,6 +324,12 @@ nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_s
  * drops the captured graphs. */
 nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
 
+/* Profiling hook, process-wide: which kernel serves the tensor-core attention (query tiles of
+ * <= 128 rows): 0 = mma.sync (the default), 1 = tcgen05 (S and O accumulated in tensor memory).
+ * Applies to launches planned afterwards (a context's captured graphs keep their kernel until
+ * they are dropped, e.g. by nld_debug_attention_tuning).  NLD_ERR_ARG for other values. */
+nld_status nld_debug_attention_kernel(int tcgen05);
+
 /* Profiling hook: timestamps of one layer inside the model's own forwards (graph launches
  * included).  While layer >= 0, the tensor-core attention launch of that layer (every forward;
  * later ones overwrite) writes to d_attn_trace (device, n_attn uint64 entries, or NULL with

@@ -96,6 +96,22 @@ NLD_DEV void row_keys(int len, int p, int bs, int m, int c, int quad_k, int& v1,
 }
 NLD_DEV bool key_visible(int key, int v1, int l2, int h2) { return key <= v1 || (key >= l2 && key <= h2); }
 
+// 16 consecutive fp32 columns of TMEM from registers (lane = thread); visible to later tcgen05
+// operations after tmem_st_wait().
+NLD_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+NLD_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 }  // namespace
 
 // kHiLo (the model's forwards): q arrives in fp32 and is split into bf16 hi and lo halves, the
@@ -502,6 +518,472 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
   cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
+// ------------------------------------------------------------------ tcgen05 attention --
+// The same attention on the 5th-generation tensor cores, for query tiles of <= 128 rows: one
+// CTA per (KV split, kv head, sequence x query tile), TMEM lane r = query row r.  Per KV tile of
+// 64 keys, S = Q K^T (M 128, N 64, K 128) goes to one of two TMEM S buffers.  Eight softmax
+// warps take two threads per row, one per half of the tile's keys; each half keeps its own
+// online softmax (reference max, row sum) and its own O accumulator in TMEM, so the two never
+// exchange anything inside the KV loop: a thread reads its 32 scores, masks and scales them,
+// writes P as bf16 (with hi/lo: its lo half too) into shared memory in the 128-byte-swizzled
+// K-major form the MMA reads, and O_h += P_h V_h (M 128, N 128, K 32) takes V straight from the
+// TMA tile as an MN-major operand.  A half's reference max moves only when a tile's max exceeds
+// it by more than 2^8 (so P <= 256), which rescales that half's O row in TMEM.  After the loop
+// the two halves of a row combine like two KV splits, then splits merge over the cluster as in
+// attn_mma_kernel.  One thread loads K/V by TMA into a 3-stage ring, another issues the MMAs; P
+// is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.
+constexpr int kTcSoftmax = 256;                 // 8 warps: half h = warp / 4, rows of warp % 4
+constexpr int kTcThreads = kTcSoftmax + 64;     // + the MMA warp + the TMA warp
+constexpr int kTcStages = 3;
+constexpr float kTcRescale = 8.f;               // log2 units
+constexpr int kTcBarBytes = 256;
+
+// Shared-memory descriptor of an MN-major operand in 128-byte-swizzled atoms (64 elements of
+// MN x 8 of K, 1024 bytes): `lbo` = bytes from one 64-element MN block to the next, `sbo` =
+// bytes from one group of 8 K rows to the next.
+NLD_DEV uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+template <bool kHiLo>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  constexpr int kQ = kHiLo ? 2 : 1;                // operand halves (hi, lo)
+  constexpr int NS = kTcStages;
+  uint8_t* sQ = smem;                              // [kQ][2 dim boxes][128 rows][128 B]
+  uint8_t* sK = sQ + kQ * 32768;                   // [NS][2 dim boxes][64 keys][128 B]
+  uint8_t* sV = sK + NS * kKVTile;                 // same
+  uint8_t* sP = sV + NS * kKVTile;                 // [2 buffers][kQ][128 rows][64 keys = 128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kQ * 16384);
+  uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
+  uint64_t* empty = bars + NS;        // [NS] K/V stage free (the tile's P V MMAs completed)
+  uint64_t* s_full = bars + 2 * NS;   // [2] S buffer written (MMA commit)
+  uint64_t* s_free = s_full + 2;      // [2] S buffer read (256 softmax threads)
+  uint64_t* p_full = s_full + 4;      // [2] P buffer written (256 softmax threads)
+  uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
+  uint64_t* fin = s_full + 8;         // the MMA thread's outstanding MMAs on an early exit
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 9);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 10);
+  constexpr uint64_t kWait = 2000000000ull;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int split = blockIdx.x;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z / a.q_tiles;
+  const int qt = blockIdx.z - b * a.q_tiles;
+  const bool softmax_thr = tid < kTcSoftmax;
+  const bool mma_thr = tid == kTcSoftmax;
+  const bool tma_thr = tid == kTcSoftmax + 32;
+  auto stamp = [&](int i) {
+    if (a.trace && tid == 0)
+      a.trace[((static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 16 + i] =
+          globaltimer_ns();
+  };
+  stamp(0);
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kTcSoftmax);
+      mbar_init(&p_full[i], kTcSoftmax);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(fin, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmKV);
+  }
+  if (warp == kTcSoftmax / 32) {
+    tmem_alloc(s_tmem, 512);   // S buffers: columns 0..127, O_0: 128..255, O_1: 256..383
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  int len = a.lens[b];
+  const int p0 = qt * a.QT;
+  const int np = min(a.QT, a.m - p0);
+  if (len < 0 || len + a.m > a.pps * kPage) {
+    if (tid == 0) set_err(a.err, NLD_DEVERR_KV_OVERFLOW);
+    len = max(0, min(len, a.pps * kPage - a.m));
+  }
+  const int crow = (a.causal_seq && a.causal_seq[b]) ? a.m : a.causal_rows;
+  int kv_end;
+  {
+    int v1, l2, h2;
+    row_keys(len, p0 + np - 1, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
+    kv_end = max(v1, h2) + 1;
+  }
+  const int n_tiles = (kv_end + kPage - 1) / kPage;
+  const int per = max(a.min_tiles, (n_tiles + a.S - 1) / a.S);
+  const int t_lo = split * per;
+  const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
+
+  int n_issued = 0;   // K/V tiles requested (TMA thread)
+  auto issue = [&](int i) {
+    ++n_issued;
+    const int stage = i % NS;
+    const int kt = t_lo + i;
+    const int page = a.page_table[b * a.pps + kt];
+    const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
+    const int row0v = row0 + a.Hkv * kPage;
+    mbar_arrive_expect_tx(&full[stage], 2 * kKVTile);
+    tma_load_2d(sK + stage * kKVTile, &tmKV, &full[stage], 0, row0);
+    tma_load_2d(sK + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0);
+    tma_load_2d(sV + stage * kKVTile, &tmKV, &full[stage], 0, row0v);
+    tma_load_2d(sV + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0v);
+  };
+  // the K/V tiles wholly in the cached prefix are requested before the dependency wait
+  int n_pre = 0;
+  if (tma_thr)
+    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
+  pdl_wait();
+  stamp(1);
+  if (tma_thr)
+    for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
+
+  // query rows -> shared memory: thread (h, r) stages dims 64h..64h+63 of row r (position
+  // r / G, head r % G) as box h, 16-byte piece u at (u ^ (r & 7)); padding rows are zero
+  const int hk = tid >> 7;            // softmax threads: key half and dim box
+  const int r = tid & 127;
+  const int prow = r / a.G, gq = r - prow * a.G;
+  const bool row_ok = softmax_thr && r < a.rows && prow < np;
+  if (softmax_thr) {
+    const size_t tok = static_cast<size_t>(b) * a.m + p0 + prow;
+    const size_t qoff = ((tok * a.Hq) + g * a.G + gq) * 128 + hk * 64;
+    uint4 hv[8], lv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      hv[u] = lv[u] = make_uint4(0, 0, 0, 0);
+      if (row_ok) {
+        if constexpr (kHiLo) {
+          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + qoff + u * 8);
+          const float4 x0 = src[0], x1 = src[1];
+          const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          split8(xs, hv[u], lv[u]);
+        } else {
+          hv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qoff + u * 8);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t off = hk * 16384 + r * 128 + ((u ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(sQ + off) = hv[u];
+      if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQ + 32768 + off) = lv[u];
+    }
+  }
+  fence_proxy_async();   // the tensor core reads these through the async proxy
+  __syncthreads();
+  stamp(2);
+  pdl_launch_dependents();
+
+  float m_ref = -INFINITY, l_sum = 0.f;
+  bool aborted = false;
+  if (tma_thr) {
+    // ------------------------------------------------------------------ TMA thread --
+    // tile i reuses the stage of tile i - NS once that tile's P V MMAs have completed
+    for (int i = NS; i < ntile; ++i) {
+      if (*s_abort || !mbar_wait(&empty[i % NS], static_cast<uint32_t>(i / NS - 1) & 1u, kWait)) {
+        aborted = true;
+        break;
+      }
+      issue(i);
+    }
+    if (aborted) {
+      *s_abort = 1;
+      set_err(a.err, NLD_DEVERR_TIMEOUT);
+    }
+  } else if (mma_thr) {
+    // ------------------------------------------------------------------ MMA thread --
+    const uint32_t idS = idesc_bf16_f32(128, 64);
+    const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
+    auto pv_step = [&](int i) -> bool {
+      const int pb = i & 1, st = i % NS;
+      if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(i >> 1) & 1u, kWait)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < kQ; ++q)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int ks = h * 2 + kk;   // 16-key step of the tile
+            tc_mma_f16(tmem + 128 + h * 128, sdesc_k_sw128(smem_u32(sP + (pb * kQ + q) * 16384)) + 2 * ks,
+                       sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
+                       (i > 0 || q > 0 || kk > 0) ? 1u : 0u);
+          }
+      tc_commit(&pv_done[pb]);
+      tc_commit(&empty[st]);
+      return true;
+    };
+    for (int j = 0; j < ntile && !aborted; ++j) {
+      const int st = j % NS, sb = j & 1;
+      if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
+          (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait))) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < kQ; ++q)
+#pragma unroll
+        for (int box = 0; box < 2; ++box)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_f16(tmem + sb * 64, sdesc_k_sw128(smem_u32(sQ + q * 32768 + box * 16384)) + 2 * kk,
+                       sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
+                       (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
+      tc_commit(&s_full[sb]);
+      if (j >= 1 && !pv_step(j - 1)) aborted = true;
+    }
+    if (!aborted && ntile > 0 && !pv_step(ntile - 1)) aborted = true;
+    if (aborted) {
+      *s_abort = 1;
+      set_err(a.err, NLD_DEVERR_TIMEOUT);
+    }
+    // every MMA this thread issued has completed before the tensor memory is released
+    tc_commit(fin);
+    mbar_wait(fin, 0, kWait);
+  } else if (softmax_thr) {
+    // ------------------------------------------- softmax: row r, keys 32hk..32hk+31 --
+    int v1 = -1, l2 = 0x7fffffff, h2 = -1;
+    if (row_ok) row_keys(len, p0 + prow, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t o_col = 128 + hk * 128;
+    for (int j = 0; j < ntile; ++j) {
+      const int sb = j & 1;
+      // tcgen05.ld/st are warp-collective: every exit of this loop is taken by the whole warp
+      const bool ok = !*s_abort && mbar_wait(&s_full[sb], static_cast<uint32_t>(j >> 1) & 1u, kWait);
+      if (!__all_sync(0xffffffffu, ok)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      float sv[32];
+      {
+        uint32_t raw[2][16];
+        tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32, raw[0]);
+        tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32 + 16, raw[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sv[c * 16 + i] = __uint_as_float(raw[c][i]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+      const int k0 = (t_lo + j) * kPage + hk * 32;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float x = key_visible(k0 + k, v1, l2, h2) ? sv[k] * a.scale_log2 : -INFINITY;
+        sv[k] = x;
+        mx = fmaxf(mx, x);
+      }
+      const bool move = mx > m_ref + kTcRescale;
+      const bool scale_o = move && j >= 1 && m_ref != -INFINITY;
+      if (__any_sync(0xffffffffu, scale_o)) {
+        // this half's O row holds tiles < j once O += P V of tile j - 1 has completed; the warp
+        // rescales its 32 rows together (factor 1 for rows that keep their max)
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, kWait))) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const float alpha = scale_o ? exp2f(m_ref - mx) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float o[16];
+          tmem_ld16(tmem + lane_base + o_col + c * 16, o);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] *= alpha;
+          tmem_st16(tmem + lane_base + o_col + c * 16, o);
+        }
+        tmem_st_wait();
+        l_sum *= alpha;
+      }
+      if (move) m_ref = mx;
+      // P buffer sb is free once O += P V of tile j - 2 has completed
+      if (!__all_sync(0xffffffffu, j < 2 || mbar_wait(&pv_done[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait))) {
+        aborted = true;
+        break;
+      }
+      const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // P row r, keys 32hk..: pieces 4hk..4hk+3 of 8 keys, piece p at (p ^ (r & 7)) of the row
+      uint8_t* prow_p = sP + sb * kQ * 16384 + r * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float pv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pv[i] = exp2f(sv[q * 8 + i] - base);
+          l_sum += pv[i];
+        }
+        uint4 ph, pl;
+        if constexpr (kHiLo) {
+          split8(pv, ph, pl);
+        } else {
+          ph = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]), pack_bf16(pv[4], pv[5]),
+                          pack_bf16(pv[6], pv[7]));
+        }
+        const uint32_t off = (((hk * 4 + q) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow_p + off) = ph;
+        if constexpr (kHiLo) *reinterpret_cast<uint4*>(prow_p + 16384 + off) = pl;
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&p_full[sb]);
+      if (j < 6 && tid == 0) stamp(3 + j);
+    }
+    if (!aborted && ntile > 0 &&
+        !__all_sync(0xffffffffu, mbar_wait(&pv_done[(ntile - 1) & 1], static_cast<uint32_t>((ntile - 1) >> 1) & 1u, kWait)))
+      aborted = true;
+    if (aborted) {
+      *s_abort = 1;
+      set_err(a.err, NLD_DEVERR_TIMEOUT);
+    }
+    tc_fence_after();
+  }
+
+  // output row rr of this CTA (part 1: the lo row of a (hi, lo) pair)
+  auto out_ptr = [&](int rr, int part) -> __nv_bfloat16* {
+    const int p = rr / a.G, gh = rr - p * a.G;
+    const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
+    const size_t orow = kHiLo ? 2 * tok + part : tok;
+    return static_cast<__nv_bfloat16*>(a.out) + orow * a.out_ld + static_cast<size_t>(g * a.G + gh) * 128;
+  };
+  auto store2 = [&](int rr, int d, float x0, float x1) {
+    if constexpr (kHiLo) {
+      uint32_t hi, lo;
+      pack_bf16_hilo(x0, x1, hi, lo);
+      *reinterpret_cast<uint32_t*>(out_ptr(rr, 0) + d) = hi;
+      *reinterpret_cast<uint32_t*>(out_ptr(rr, 1) + d) = lo;
+    } else {
+      *reinterpret_cast<uint32_t*>(out_ptr(rr, 0) + d) = pack_bf16(x0, x1);
+    }
+  };
+
+  // the two key halves of a row combine: thread (h, r) takes dims 64h..64h+63 of both O_0 and
+  // O_1, weighted by 2^(m_h - M) with M the larger reference max
+  __syncthreads();   // every MMA and every TMA load of this CTA has completed
+  float2* sMLh = reinterpret_cast<float2*>(sP);          // [2][128] (m, l) per key half
+  float* sO = reinterpret_cast<float*>(smem);            // [128][128] partials (over Q, K)
+  float* sML = sO + 128 * 128;                           // [128][2]
+  const bool have = ntile > 0 && !*s_abort;
+  // after a timeout anywhere, the loads still in flight land before the ring is overlaid
+  if (tma_thr && !have)
+    for (int t = max(0, n_issued - NS); t < n_issued; ++t)
+      mbar_wait(&full[t % NS], static_cast<uint32_t>(t / NS) & 1u, kWait);
+  if (softmax_thr) sMLh[hk * 128 + r] = make_float2(have ? m_ref : -INFINITY, have ? l_sum : 0.f);
+  __syncthreads();
+  if (softmax_thr) {
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float2 ml0 = sMLh[r], ml1 = sMLh[128 + r];
+    const float M = fmaxf(ml0.x, ml1.x);
+    const float w0 = (ml0.x == -INFINITY) ? 0.f : exp2f(ml0.x - M);
+    const float w1 = (ml1.x == -INFINITY) ? 0.f : exp2f(ml1.x - M);
+    const float L = ml0.y * w0 + ml1.y * w1;
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float o0[16], o1[16];
+      const uint32_t col = hk * 64 + c * 16;
+      if (have) {
+        tmem_ld16(tmem + lane_base + 128 + col, o0);
+        tmem_ld16(tmem + lane_base + 256 + col, o1);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o0[i] = o1[i] = 0.f;
+      }
+      float o[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[i] = o0[i] * w0 + o1[i] * w1;
+      if (a.S == 1) {
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) store2(r, col + i, o[i] * inv, o[i + 1] * inv);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(sO + r * 128 + col + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+      }
+    }
+    if (a.S > 1 && hk == 0) *reinterpret_cast<float2*>(sML + r * 2) = make_float2(M, L);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTcSoftmax / 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (a.S == 1) {
+    stamp(11);
+    return;
+  }
+  cluster_sync();
+  stamp(10);
+  const int S = a.S;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int per_rank = (a.rows + S - 1) / S;
+  const int r0 = rank * per_rank, r1 = min(a.rows, r0 + per_rank);
+  const uint32_t o_base = smem_u32(sO), ml_base = smem_u32(sML);
+  uint32_t o_peer[8], ml_peer[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
+    ml_peer[q] = (q < S) ? dsmem_addr(ml_base, q) : 0u;
+  }
+  for (int e = tid; e < (r1 - r0) * 32; e += kTcThreads) {
+    const int rr = r0 + (e >> 5), d4 = e & 31;
+    if (rr / a.G >= np) continue;
+    float2 ml[8];
+    float4 ov[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + rr * 8) : make_float2(-INFINITY, 0.f);
+      ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + (rr * 128 + d4 * 4) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) M = fmaxf(M, ml[q].x);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < S && ml[q].x != -INFINITY) {
+        const float w = exp2f(ml[q].x - M);
+        L += w * ml[q].y;
+        acc.x += w * ov[q].x;
+        acc.y += w * ov[q].y;
+        acc.z += w * ov[q].z;
+        acc.w += w * ov[q].w;
+      }
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    store2(rr, d4 * 4, acc.x * inv, acc.y * inv);
+    store2(rr, d4 * 4 + 2, acc.z * inv, acc.w * inv);
+  }
+  stamp(11);
+  cluster_sync();   // peers may still be reading this CTA's shared memory
+}
+
 // Plain per-(token, head) attention for any head_dim <= 128 and either storage type; used by
 // the fp32 configuration.  Scores go to shared memory (max_kv floats), two-pass softmax.
 template <typename T>
@@ -573,8 +1055,10 @@ cudaError_t gemm_tc_init_attributes();
 
 namespace {
 using AttnKernel = void (*)(const CUtensorMap, const AttnArgs);
-// The instantiation for a launch: its operand form and its launch bound (<= 8 or 9 warps).
-AttnKernel attn_kernel_for(bool hilo, int NW) {
+// The instantiation for a launch: tcgen05 or mma.sync, its operand form and (mma.sync) its
+// launch bound (<= 8 or 9 warps).
+AttnKernel attn_kernel_for(bool hilo, int NW, bool tc) {
+  if (tc) return hilo ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   if (NW > 8) return hilo ? attn_mma_kernel<true, 9> : attn_mma_kernel<false, 9>;
   return hilo ? attn_mma_kernel<true, 8> : attn_mma_kernel<false, 8>;
 }
@@ -588,8 +1072,8 @@ cudaError_t init_kernel_attributes() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  for (int v = 0; v < 4; ++v) {
-    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8);
+  for (int v = 0; v < 6; ++v) {
+    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8, v >= 4);
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -608,12 +1092,21 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
   return 1024 + std::max(ring_q, partials) + kMaxAttStages * sizeof(uint64_t);
 }
 
-// Clusters of S CTAs (NW warps, the shared memory above) that can be resident at once.
-int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms) {
+// Dynamic shared memory of a tcgen05 attention launch: the query tile (hi and lo halves with
+// hilo), the K and V rings, two P buffers (hi, lo) and the barriers; the split partials overlay
+// the first three after the KV loop.
+size_t attn_tc_smem_bytes(bool hilo) {
+  const size_t kq = hilo ? 2 : 1;
+  return 1024 + kq * 32768 + 2 * static_cast<size_t>(kTcStages) * kKVTile + 2 * kq * 16384 + kTcBarBytes;
+}
+
+// Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
+// resident at once.
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, bool tc) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S * (sms / S));
-  cfg.blockDim = dim3(32 * NW);
-  cfg.dynamicSmemBytes = attn_mma_smem_bytes(NW, hilo, stages);
+  cfg.blockDim = dim3(tc ? kTcThreads : 32 * NW);
+  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(hilo) : attn_mma_smem_bytes(NW, hilo, stages);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
@@ -622,7 +1115,7 @@ int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, attn_kernel_for(hilo, NW), &cfg);
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, attn_kernel_for(hilo, NW, tc), &cfg);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return sms / S;
@@ -632,12 +1125,14 @@ int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms) {
 
 cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
                                  int batch, bool pdl) {
-  if (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages)
-    return cudaErrorInvalidValue;   // launch bound, ring depth
+  const bool tc = a.tc != 0;
+  if (tc ? (a.rows < 1 || a.rows > 128 || a.S < 1 || a.S > 8)
+         : (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages))
+    return cudaErrorInvalidValue;   // tile rows / launch bound, ring depth
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
-  cfg.blockDim = dim3(32 * a.NW);
-  cfg.dynamicSmemBytes = attn_mma_smem_bytes(a.NW, a.hilo != 0, a.stages);
+  cfg.blockDim = dim3(tc ? kTcThreads : 32 * a.NW);
+  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(a.hilo != 0) : attn_mma_smem_bytes(a.NW, a.hilo != 0, a.stages);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -652,7 +1147,7 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   if (pdl) attrs[na++] = attr[0];
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_kernel_for(a.hilo != 0, a.NW), *tmKV, a);
+  return cudaLaunchKernelEx(&cfg, attn_kernel_for(a.hilo != 0, a.NW, tc), *tmKV, a);
 }
 
 cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,

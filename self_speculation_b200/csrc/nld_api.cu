@@ -17,6 +17,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <atomic>
 #include <functional>
 #include <string>
 #include <tuple>
@@ -28,7 +29,8 @@ using namespace nld;
 
 namespace nld {
 size_t attn_mma_smem_bytes(int NW, bool hilo, int stages);
-int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms);
+size_t attn_tc_smem_bytes(bool hilo);
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, bool tc);
 cudaError_t init_kernel_attributes();
 }
 
@@ -484,13 +486,18 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
   return NLD_OK;
 }
 
-// Clusters of S attention CTAs (NW warps, `stages` ring stages) resident at once.
-using AttnCapacity = std::function<int(int S, int NW, int stages)>;
+// Clusters of S attention CTAs (NW warps, `stages` ring stages; or the tcgen05 kernel) resident
+// at once.
+using AttnCapacity = std::function<int(int S, int NW, int stages, bool tc)>;
+
+// Which attention kernel serves query tiles of <= 128 rows (profiling hook): 0 mma.sync,
+// 1 tcgen05.
+std::atomic<int> g_attn_tc{0};
 
 // rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
 // tiles a split takes at least; 0 = the planner's choice for either.
 void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
-               int rows_cap = 0, int min_tiles = 0) {
+               int rows_cap = 0, int min_tiles = 0, bool tc = false) {
   a.G = Hq / Hkv;
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   auto q_tiles_for = [&](int c) {
@@ -503,11 +510,14 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // into splits of single tiles, and the ring holds 2 stages (about 100 KB, two CTAs per SM).
   // Otherwise tiles of up to 144 rows (a 33-position verify block of 4 heads in one 9-warp
   // CTA) read each K/V tile once for as many query rows as possible, through a 3-stage ring.
+  // The tcgen05 kernel takes query tiles of up to 128 rows (one MMA tile) in either regime.
   const bool latency = batch * Hkv * q_tiles_for(144) * 8 < 2 * sms;
-  if (rows_cap <= 0) rows_cap = latency ? 64 : 144;
+  if (rows_cap <= 0) rows_cap = tc ? 128 : (latency ? 64 : 144);
+  if (tc) rows_cap = std::min(rows_cap, 128);
   if (min_tiles <= 0) min_tiles = latency ? 1 : 2;
   a.min_tiles = min_tiles;
-  a.stages = latency ? 2 : 3;
+  a.stages = (latency || tc) ? 2 : 3;
+  a.tc = tc ? 1 : 0;
   // query positions per CTA: as many as rows_cap allows, spread evenly over the query tiles
   const int nq = q_tiles_for(rows_cap);
   a.QT = (m + nq - 1) / nq;
@@ -522,15 +532,15 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   a.S = 1;
   if (units < 2 * sms) {
     int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / min_tiles)}));
-    while (s_max > 1 && units > cap(s_max, a.NW, a.stages)) --s_max;
+    while (s_max > 1 && units > cap(s_max, a.NW, a.stages, tc)) --s_max;
     const int per = std::max(min_tiles, (n_tiles + s_max - 1) / s_max);
     a.S = std::max(1, (n_tiles + per - 1) / per);
   }
 }
 
 // The device's cluster capacity for the attention kernel (occupancy query, cached).
-int attn_device_capacity(bool hilo, int S, int NW, int stages) {
-  static int cache[16][9][10][2][4];   // [device][S][NW][hilo][stages]; 0 = not yet queried
+int attn_device_capacity(bool hilo, int S, int NW, int stages, bool tc) {
+  static int cache[16][9][10][2][4][2];   // [device][S][NW][hilo][stages][tc]; 0 = not yet queried
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 16 || S < 1 || S > 8 || NW < 1 || NW > 9 || stages < 2 ||
       stages > 3) {
@@ -539,8 +549,8 @@ int attn_device_capacity(bool hilo, int S, int NW, int stages) {
   }
   static std::mutex mu;   // the stand-alone attention may be called from several threads
   std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][S][NW][hilo ? 1 : 0][stages];
-  if (c == 0) c = attn_mma_max_clusters(S, NW, hilo, stages, device_sms());
+  int& c = cache[dev][S][NW][hilo ? 1 : 0][stages][tc ? 1 : 0];
+  if (c == 0) c = attn_mma_max_clusters(S, NW, hilo, stages, device_sms(), tc);
   return c;
 }
 
@@ -643,8 +653,8 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.quad_k = f.quad_k;
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa,
-              [](int S, int NW, int stages) { return attn_device_capacity(true, S, NW, stages); },
-              x->attn_rows_cap, x->attn_min_tiles);
+              [](int S, int NW, int stages, bool tc) { return attn_device_capacity(true, S, NW, stages, tc); },
+              x->attn_rows_cap, x->attn_min_tiles, g_attn_tc.load() != 0);
     const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
     attn_traced = x->attn_trace && ctas * 16 <= x->attn_trace_n;
   } else {
@@ -1772,6 +1782,12 @@ nld_status nld_debug_layer_trace(nld_ctx* x, int layer, unsigned long long* d_at
   return NLD_OK;
 }
 
+nld_status nld_debug_attention_kernel(int tcgen05) {
+  if (tcgen05 != 0 && tcgen05 != 1) return fail(nullptr, NLD_ERR_ARG, "0 (mma.sync) or 1 (tcgen05)");
+  g_attn_tc.store(tcgen05);
+  return NLD_OK;
+}
+
 nld_status nld_debug_attention_tuning(nld_ctx* x, int rows_per_cta, int min_tiles_per_split) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if ((rows_per_cta != 0 && (rows_per_cta < 16 || rows_per_cta > 144)) || min_tiles_per_split < 0 ||
@@ -1850,8 +1866,9 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
   AttnArgs a{};
   // pure host: clusters of S resident at once as if every SM held as many CTAs as its 228 KB of
   // shared memory allows (one block reserves 1 KB)
-  attn_plan(batch, m, Hq, Hkv, max_len, sms, a, [sms](int S, int NW, int stages) {
-    const int per_sm = static_cast<int>(233472 / (attn_mma_smem_bytes(NW, true, stages) + 1024));
+  attn_plan(batch, m, Hq, Hkv, max_len, sms, a, [sms](int S, int NW, int stages, bool tc) {
+    const size_t smem = tc ? attn_tc_smem_bytes(true) : attn_mma_smem_bytes(NW, true, stages);
+    const int per_sm = static_cast<int>(233472 / (smem + 1024));
     return std::max(1, sms * per_sm / S);
   });
   out6[0] = a.G;
@@ -2089,7 +2106,8 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   }
   AttnArgs a{};
   attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
-            [](int S, int NW, int stages) { return attn_device_capacity(false, S, NW, stages); });
+            [](int S, int NW, int stages, bool tc) { return attn_device_capacity(false, S, NW, stages, tc); },
+            0, 0, g_attn_tc.load() != 0);
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))

@@ -19,6 +19,17 @@ HQ, HKV, HD = 32, 8, 128
 TOL = 2e-2
 
 
+@pytest.fixture(autouse=True, params=["mma_sync", "tcgen05"])
+def attention_kernel(request):
+    """Every case runs on both tensor-core attention kernels (the process-wide switch is put
+    back to the default afterwards)."""
+    import self_speculation_b200 as nb
+    lib = nb.load_library()
+    assert lib.nld_debug_attention_kernel(1 if request.param == "tcgen05" else 0) == 0
+    yield request.param
+    assert lib.nld_debug_attention_kernel(0) == 0
+
+
 def _setup(lens, m, seed=2, shuffle_seed=0):
     import self_speculation_b200 as nb
     B = len(lens)
