@@ -525,18 +525,41 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // warps take two threads per row, one per half of the tile's keys; each half keeps its own
 // online softmax (reference max, row sum) and its own O accumulator in TMEM, so the two never
 // exchange anything inside the KV loop: a thread reads its 32 scores, masks and scales them,
-// writes P as bf16 (with hi/lo: its lo half too) into shared memory in the 128-byte-swizzled
-// K-major form the MMA reads, and O_h += P_h V_h (M 128, N 128, K 32) takes V straight from the
-// TMA tile as an MN-major operand.  A half's reference max moves only when a tile's max exceeds
-// it by more than 2^8 (so P <= 256), which rescales that half's O row in TMEM.  After the loop
-// the two halves of a row combine like two KV splits, then splits merge over the cluster as in
-// attn_mma_kernel.  One thread loads K/V by TMA into a 3-stage ring, another issues the MMAs; P
-// is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.
+// writes P as packed bf16 pairs (with hi/lo: its lo half too) into TMEM, and O_h += P_h V_h
+// (M 128, N 128, K 32) takes P from TMEM as the A operand and V straight from the TMA tile as an
+// MN-major operand.  A half's reference max moves only when a tile's max exceeds it by more than
+// 2^8 (so P <= 256), which rescales that half's O row in TMEM.  After the loop the two halves of
+// a row combine like two KV splits, then splits merge over the cluster as in attn_mma_kernel.
+// One thread loads K/V by TMA into a 5-stage (bf16 Q: 6-stage) ring, another issues the MMAs;
+// P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.  TMEM columns:
+// S buffers 0..127, O_0 128..255, O_1 256..383, P buffers 384..511 (per buffer, key half h at
+// 32h: hi pairs, then lo pairs).
 constexpr int kTcSoftmax = 256;                 // 8 warps: half h = warp / 4, rows of warp % 4
 constexpr int kTcThreads = kTcSoftmax + 64;     // + the MMA warp + the TMA warp
-constexpr int kTcStages = 3;
+constexpr int kTcMaxStages = 6;
+__host__ __device__ constexpr int tc_stages(bool hilo) { return hilo ? 5 : 6; }
+// S of tile j + 2 is issued before O += P V of tile j, so its K/V stage must not wait for that
+static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
 constexpr int kTcBarBytes = 256;
+
+// 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0).
+NLD_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate; A's row i is TMEM lane i,
+// two bf16 of K per 32-bit column.
+NLD_DEV void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 // Shared-memory descriptor of an MN-major operand in 128-byte-swizzled atoms (64 elements of
 // MN x 8 of K, 1024 bytes): `lbo` = bytes from one 64-element MN block to the next, `sbo` =
@@ -558,17 +581,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kQ = kHiLo ? 2 : 1;                // operand halves (hi, lo)
-  constexpr int NS = kTcStages;
+  constexpr int NS = tc_stages(kHiLo);
   uint8_t* sQ = smem;                              // [kQ][2 dim boxes][128 rows][128 B]
   uint8_t* sK = sQ + kQ * 32768;                   // [NS][2 dim boxes][64 keys][128 B]
   uint8_t* sV = sK + NS * kKVTile;                 // same
-  uint8_t* sP = sV + NS * kKVTile;                 // [2 buffers][kQ][128 rows][64 keys = 128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kQ * 16384);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile);
   uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
-  uint64_t* empty = bars + NS;        // [NS] K/V stage free (the tile's P V MMAs completed)
-  uint64_t* s_full = bars + 2 * NS;   // [2] S buffer written (MMA commit)
+  uint64_t* empty = bars + kTcMaxStages;   // [NS] K/V stage free (the tile's P V MMAs completed)
+  uint64_t* s_full = bars + 2 * kTcMaxStages;   // [2] S buffer written (MMA commit)
   uint64_t* s_free = s_full + 2;      // [2] S buffer read (256 softmax threads)
-  uint64_t* p_full = s_full + 4;      // [2] P buffer written (256 softmax threads)
+  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (256 softmax threads)
   uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
   uint64_t* fin = s_full + 8;         // the MMA thread's outstanding MMAs on an early exit
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 9);
@@ -607,7 +629,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tmKV);
   }
   if (warp == kTcSoftmax / 32) {
-    tmem_alloc(s_tmem, 512);   // S buffers: columns 0..127, O_0: 128..255, O_1: 256..383
+    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O_0: 128..255, O_1: 256..383, P: 384..511
     tmem_relinquish();
   }
   tc_fence_before();
@@ -723,22 +745,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int q = 0; q < kQ; ++q)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
-            const int ks = h * 2 + kk;   // 16-key step of the tile
-            tc_mma_f16(tmem + 128 + h * 128, sdesc_k_sw128(smem_u32(sP + (pb * kQ + q) * 16384)) + 2 * ks,
-                       sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
-                       (i > 0 || q > 0 || kk > 0) ? 1u : 0u);
+            const int ks = h * 2 + kk;   // 16-key step of the tile: 8 TMEM columns of P
+            tc_mma_f16_ts(tmem + 128 + h * 128, tmem + 384 + pb * 64 + h * 32 + q * 16 + kk * 8,
+                          sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
+                          (i > 0 || q > 0 || kk > 0) ? 1u : 0u);
           }
       tc_commit(&pv_done[pb]);
       tc_commit(&empty[st]);
       return true;
     };
-    for (int j = 0; j < ntile && !aborted; ++j) {
+    // S of tile j into S buffer j & 1 (free once the softmax read S of tile j - 2)
+    auto s_step = [&](int j) -> bool {
       const int st = j % NS, sb = j & 1;
       if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
-          (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait))) {
-        aborted = true;
-        break;
-      }
+          (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
+        return false;
       tc_fence_after();
 #pragma unroll
       for (int q = 0; q < kQ; ++q)
@@ -750,9 +771,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
                        (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&s_full[sb]);
-      if (j >= 1 && !pv_step(j - 1)) aborted = true;
+      return true;
+    };
+    // S runs two tiles ahead of the softmax: S of tile j + 2 goes as soon as the softmax has
+    // read S of tile j, before O += P V of tile j
+    for (int j = 0; j < min(2, ntile) && !aborted; ++j)
+      if (!s_step(j)) aborted = true;
+    for (int j = 0; j < ntile && !aborted; ++j) {
+      if (j + 2 < ntile && !s_step(j + 2)) {
+        aborted = true;
+        break;
+      }
+      if (!pv_step(j)) aborted = true;
     }
-    if (!aborted && ntile > 0 && !pv_step(ntile - 1)) aborted = true;
     if (aborted) {
       *s_abort = 1;
       set_err(a.err, NLD_DEVERR_TIMEOUT);
@@ -789,13 +820,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&s_free[sb]);
       const int k0 = (t_lo + j) * kPage + hk * 32;
-      float mx = -INFINITY;
+      if (k0 + 31 <= v1) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float x = key_visible(k0 + k, v1, l2, h2) ? sv[k] * a.scale_log2 : -INFINITY;
-        sv[k] = x;
-        mx = fmaxf(mx, x);
+        for (int k = 0; k < 32; ++k) sv[k] *= a.scale_log2;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) sv[k] = key_visible(k0 + k, v1, l2, h2) ? sv[k] * a.scale_log2 : -INFINITY;
       }
+      // max as a tree (independent pairs: short dependency chains)
+      float mt[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) mt[k] = fmaxf(sv[k], sv[k + 16]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int k = 0; k < w; ++k) mt[k] = fmaxf(mt[k], mt[k + w]);
+      const float mx = mt[0];
       const bool move = mx > m_ref + kTcRescale;
       const bool scale_o = move && j >= 1 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, scale_o)) {
@@ -825,28 +865,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // P row r, keys 32hk..: pieces 4hk..4hk+3 of 8 keys, piece p at (p ^ (r & 7)) of the row
-      uint8_t* prow_p = sP + sb * kQ * 16384 + r * 128;
+      // P row r, keys 32hk..32hk+31 as 16 bf16 pairs (lower key in the low half), hi then lo
+      float ph[16], pl[16];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float pv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          pv[i] = exp2f(sv[q * 8 + i] - base);
-          l_sum += pv[i];
-        }
-        uint4 ph, pl;
+      for (int c = 0; c < 16; ++c) {
+        const float p0 = ex2_approx(sv[2 * c] - base), p1 = ex2_approx(sv[2 * c + 1] - base);
+        ls[c & 3] += p0 + p1;
+        uint32_t hi, lo;
         if constexpr (kHiLo) {
-          split8(pv, ph, pl);
+          pack_bf16_hilo(p0, p1, hi, lo);
         } else {
-          ph = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]), pack_bf16(pv[4], pv[5]),
-                          pack_bf16(pv[6], pv[7]));
+          hi = pack_bf16(p0, p1);
+          lo = 0u;
         }
-        const uint32_t off = (((hk * 4 + q) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow_p + off) = ph;
-        if constexpr (kHiLo) *reinterpret_cast<uint4*>(prow_p + 16384 + off) = pl;
+        ph[c] = __uint_as_float(hi);
+        pl[c] = __uint_as_float(lo);
       }
-      fence_proxy_async();
+      l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      const uint32_t p_col = 384 + sb * 64 + hk * 32;
+      tmem_st16(tmem + lane_base + p_col, ph);
+      if constexpr (kHiLo) tmem_st16(tmem + lane_base + p_col + 16, pl);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[sb]);
       if (j < 6 && tid == 0) stamp(3 + j);
@@ -882,9 +922,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // the two key halves of a row combine: thread (h, r) takes dims 64h..64h+63 of both O_0 and
   // O_1, weighted by 2^(m_h - M) with M the larger reference max
   __syncthreads();   // every MMA and every TMA load of this CTA has completed
-  float2* sMLh = reinterpret_cast<float2*>(sP);          // [2][128] (m, l) per key half
   float* sO = reinterpret_cast<float*>(smem);            // [128][128] partials (over Q, K)
   float* sML = sO + 128 * 128;                           // [128][2]
+  float2* sMLh = reinterpret_cast<float2*>(sML + 256);   // [2][128] (m, l) per key half
   const bool have = ntile > 0 && !*s_abort;
   // after a timeout anywhere, the loads still in flight land before the ring is overlaid
   if (tma_thr && !have)
@@ -1093,11 +1133,11 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
 }
 
 // Dynamic shared memory of a tcgen05 attention launch: the query tile (hi and lo halves with
-// hilo), the K and V rings, two P buffers (hi, lo) and the barriers; the split partials overlay
-// the first three after the KV loop.
+// hilo), the K and V rings and the barriers; the split partials overlay the first two after the
+// KV loop.
 size_t attn_tc_smem_bytes(bool hilo) {
   const size_t kq = hilo ? 2 : 1;
-  return 1024 + kq * 32768 + 2 * static_cast<size_t>(kTcStages) * kKVTile + 2 * kq * 16384 + kTcBarBytes;
+  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
