@@ -297,10 +297,11 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
                           int hilo, int* out20);
 
 /* Test hook, pure host: the attention launch plan for batch sequences of m rows, Hq/Hkv heads,
- * keys up to max_len, on sms SMs.  out6 = {G = Hq/Hkv, query positions per CTA, query tiles,
- * rows per CTA (positions x G), warps per CTA, KV splits (= cluster size)}.  NLD_ERR_ARG on
- * bad sizes. */
-nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out6);
+ * keys up to max_len, on sms SMs, under the current nld_debug_attention_kernel setting.
+ * out7 = {G = Hq/Hkv, query positions per CTA, query tiles, rows per CTA (positions x G), warps
+ * per CTA (mma.sync kernel), KV splits (= cluster size), kernel (1 tcgen05, 0 mma.sync)}.
+ * NLD_ERR_ARG on bad sizes. */
+nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out7);
 
 /* Profiling hook: tuning of the projection chains' pipeline.  stage_cap = 0 lets the planner
  * use as many shared-memory stages as fit, else at most stage_cap (3..8); k_tiles_per_stage =
@@ -324,11 +325,14 @@ nld_status nld_debug_chain_tuning(nld_ctx* ctx, int stage_cap, int k_tiles_per_s
  * drops the captured graphs. */
 nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_tiles_per_split);
 
-/* Profiling hook, process-wide: which kernel serves the tensor-core attention (query tiles of
- * <= 128 rows): 0 = mma.sync (the default), 1 = tcgen05 (S and O accumulated in tensor memory).
+/* Profiling hook, process-wide: which kernel serves the tensor-core attention.  0 (the
+ * default) = the planner's choice: the tcgen05 kernel (S, P and O in tensor memory, query tiles
+ * of <= 128 rows) for query tiles of >= 64 rows (>= 96 with many sequences) unless, with many
+ * sequences, 128-row tiles would cut a query block that one mma.sync CTA of <= 144 rows takes
+ * whole; the mma.sync kernel otherwise; 1 = tcgen05 always; 2 = mma.sync always.
  * Applies to launches planned afterwards (a context's captured graphs keep their kernel until
  * they are dropped, e.g. by nld_debug_attention_tuning).  NLD_ERR_ARG for other values. */
-nld_status nld_debug_attention_kernel(int tcgen05);
+nld_status nld_debug_attention_kernel(int kernel);
 
 /* Profiling hook: timestamps of one layer inside the model's own forwards (graph launches
  * included).  While layer >= 0, the tensor-core attention launch of that layer (every forward;

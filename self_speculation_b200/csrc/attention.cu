@@ -111,6 +111,14 @@ NLD_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
       : "memory");
 }
 NLD_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Wait for this thread's outstanding tcgen05.ld, with r as in-out operands so that no use of
+// the loaded registers is scheduled before the wait.
+NLD_DEV void tmem_ld_wait_regs(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15])::"memory");
+}
 
 }  // namespace
 
@@ -679,35 +687,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tma_thr)
     for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
 
-  // query rows -> shared memory: thread (h, r) stages dims 64h..64h+63 of row r (position
-  // r / G, head r % G) as box h, 16-byte piece u at (u ^ (r & 7)); padding rows are zero
-  const int hk = tid >> 7;            // softmax threads: key half and dim box
-  const int r = tid & 127;
-  const int prow = r / a.G, gq = r - prow * a.G;
+  const int hk = tid >> 7;            // softmax threads: key half
+  const int r = tid & 127;            // and query row (position r / G, head r % G)
+  const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
+  // query rows -> shared memory, coalesced: piece e = tid + 256u of the tile's 128 rows x 16
+  // pieces of 8 dims (row e / 16, piece c = e % 16) goes to box c / 8 at piece (c % 8) ^ (row % 8);
+  // padding rows are zero
   if (softmax_thr) {
-    const size_t tok = static_cast<size_t>(b) * a.m + p0 + prow;
-    const size_t qoff = ((tok * a.Hq) + g * a.G + gq) * 128 + hk * 64;
     uint4 hv[8], lv[8];
+    int offs[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
+      const int e = tid + u * kTcSoftmax;
+      const int row = e >> 4, c = e & 15;
+      const int p = row / a.G, gh = row - p * a.G;
+      offs[u] = (c >> 3) * 16384 + row * 128 + (((c & 7) ^ (row & 7)) << 4);
       hv[u] = lv[u] = make_uint4(0, 0, 0, 0);
-      if (row_ok) {
+      if (row < a.rows && p < np) {
+        const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
+        const size_t qoff = ((tok * a.Hq) + g * a.G + gh) * 128 + c * 8;
         if constexpr (kHiLo) {
-          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + qoff + u * 8);
+          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + qoff);
           const float4 x0 = src[0], x1 = src[1];
           const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
           split8(xs, hv[u], lv[u]);
         } else {
-          hv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qoff + u * 8);
+          hv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qoff);
         }
       }
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const uint32_t off = hk * 16384 + r * 128 + ((u ^ (r & 7)) << 4);
-      *reinterpret_cast<uint4*>(sQ + off) = hv[u];
-      if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQ + 32768 + off) = lv[u];
+      *reinterpret_cast<uint4*>(sQ + offs[u]) = hv[u];
+      if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQ + 32768 + offs[u]) = lv[u];
     }
   }
   fence_proxy_async();   // the tensor core reads these through the async proxy
@@ -811,7 +824,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t raw[2][16];
         tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32, raw[0]);
         tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32 + 16, raw[1]);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(raw[0]);
+        tmem_ld_wait_regs(raw[1]);
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -920,7 +934,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   // the two key halves of a row combine: thread (h, r) takes dims 64h..64h+63 of both O_0 and
-  // O_1, weighted by 2^(m_h - M) with M the larger reference max
+  // O_1, weighted by 2^(m_h - M) with M the larger reference max, into the CTA's partial (O
+  // unnormalised, (M, L)) in shared memory; float4 slot s of row r sits at slot s ^ (r % 32)
   __syncthreads();   // every MMA and every TMA load of this CTA has completed
   float* sO = reinterpret_cast<float*>(smem);            // [128][128] partials (over Q, K)
   float* sML = sO + 128 * 128;                           // [128][2]
@@ -938,34 +953,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float M = fmaxf(ml0.x, ml1.x);
     const float w0 = (ml0.x == -INFINITY) ? 0.f : exp2f(ml0.x - M);
     const float w1 = (ml1.x == -INFINITY) ? 0.f : exp2f(ml1.x - M);
-    const float L = ml0.y * w0 + ml1.y * w1;
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float o0[16], o1[16];
-      const uint32_t col = hk * 64 + c * 16;
+    for (int c = 0; c < 2; ++c) {
+      uint32_t o0[2][16], o1[2][16];
+      const uint32_t col = hk * 64 + c * 32;
       if (have) {
-        tmem_ld16(tmem + lane_base + 128 + col, o0);
-        tmem_ld16(tmem + lane_base + 256 + col, o1);
+        tmem_ld16_nowait(tmem + lane_base + 128 + col, o0[0]);
+        tmem_ld16_nowait(tmem + lane_base + 128 + col + 16, o0[1]);
+        tmem_ld16_nowait(tmem + lane_base + 256 + col, o1[0]);
+        tmem_ld16_nowait(tmem + lane_base + 256 + col + 16, o1[1]);
+        tmem_ld_wait_regs(o0[0]);
+        tmem_ld_wait_regs(o0[1]);
+        tmem_ld_wait_regs(o1[0]);
+        tmem_ld_wait_regs(o1[1]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o0[i] = o1[i] = 0.f;
+        for (int i = 0; i < 16; ++i) o0[0][i] = o0[1][i] = o1[0][i] = o1[1][i] = 0u;
       }
-      float o[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = o0[i] * w0 + o1[i] * w1;
-      if (a.S == 1) {
-        if (row_ok) {
+      for (int i = 0; i < 32; i += 4) {
+        float o[4];
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) store2(r, col + i, o[i] * inv, o[i + 1] * inv);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4*>(sO + r * 128 + col + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        for (int t = 0; t < 4; ++t)
+          o[t] = __uint_as_float(o0[(i + t) >> 4][(i + t) & 15]) * w0 + __uint_as_float(o1[(i + t) >> 4][(i + t) & 15]) * w1;
+        const int slot = ((col + i) >> 2) ^ (r & 31);
+        *reinterpret_cast<float4*>(sO + r * 128 + slot * 4) = make_float4(o[0], o[1], o[2], o[3]);
       }
     }
-    if (a.S > 1 && hk == 0) *reinterpret_cast<float2*>(sML + r * 2) = make_float2(M, L);
+    if (hk == 0) *reinterpret_cast<float2*>(sML + r * 2) = make_float2(M, ml0.y * w0 + ml1.y * w1);
   }
   tc_fence_before();
   __syncthreads();
@@ -973,13 +988,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (a.S == 1) {
-    stamp(11);
-    return;
-  }
-  cluster_sync();
-  stamp(10);
+  // the S splits' partials merge: rank q of the cluster writes rows [q rows/S, (q+1) rows/S),
+  // one warp per row, each thread 4 dims (coalesced output)
   const int S = a.S;
+  if (S > 1) cluster_sync();
+  stamp(10);
   const int rank = static_cast<int>(cluster_ctarank());
   const int per_rank = (a.rows + S - 1) / S;
   const int r0 = rank * per_rank, r1 = min(a.rows, r0 + per_rank);
@@ -993,12 +1006,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   for (int e = tid; e < (r1 - r0) * 32; e += kTcThreads) {
     const int rr = r0 + (e >> 5), d4 = e & 31;
     if (rr / a.G >= np) continue;
+    const uint32_t o_off = (rr * 128 + ((d4 ^ (rr & 31)) << 2)) * 4;
     float2 ml[8];
     float4 ov[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + rr * 8) : make_float2(-INFINITY, 0.f);
-      ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + (rr * 128 + d4 * 4) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + o_off) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     float M = -INFINITY;
 #pragma unroll
@@ -1021,7 +1035,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     store2(rr, d4 * 4 + 2, acc.z * inv, acc.w * inv);
   }
   stamp(11);
-  cluster_sync();   // peers may still be reading this CTA's shared memory
+  if (S > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
 // Plain per-(token, head) attention for any head_dim <= 128 and either storage type; used by

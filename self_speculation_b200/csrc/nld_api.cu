@@ -490,14 +490,14 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
 // at once.
 using AttnCapacity = std::function<int(int S, int NW, int stages, bool tc)>;
 
-// Which attention kernel serves query tiles of <= 128 rows (profiling hook): 0 mma.sync,
-// 1 tcgen05.
-std::atomic<int> g_attn_tc{0};
+// Which kernel serves the tensor-core attention (profiling hook): 0 the planner's choice,
+// 1 tcgen05, 2 mma.sync.
+std::atomic<int> g_attn_kernel{0};
 
 // rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
 // tiles a split takes at least; 0 = the planner's choice for either.
 void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
-               int rows_cap = 0, int min_tiles = 0, bool tc = false) {
+               int rows_cap = 0, int min_tiles = 0, int kernel = 0) {
   a.G = Hq / Hkv;
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   auto q_tiles_for = [&](int c) {
@@ -510,8 +510,16 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // into splits of single tiles, and the ring holds 2 stages (about 100 KB, two CTAs per SM).
   // Otherwise tiles of up to 144 rows (a 33-position verify block of 4 heads in one 9-warp
   // CTA) read each K/V tile once for as many query rows as possible, through a 3-stage ring.
-  // The tcgen05 kernel takes query tiles of up to 128 rows (one MMA tile) in either regime.
+  // The tcgen05 kernel takes query tiles of up to 128 rows (one MMA tile, in either regime),
+  // and a KV tile costs it the same whatever the rows, so it serves tiles of >= 64 rows (>= 96
+  // with many sequences) unless an explicit tile above 128 rows is asked for or, with many
+  // sequences, 128-row tiles would cut a query block that one 144-row mma.sync CTA takes whole
+  // (a 33-position verify block of 4 heads: two CTAs would each stream all its keys).
   const bool latency = batch * Hkv * q_tiles_for(144) * 8 < 2 * sms;
+  const int tc_rows = ((m + q_tiles_for(128) - 1) / q_tiles_for(128)) * a.G;
+  const bool tc = kernel == 1 ||
+                  (kernel == 0 && rows_cap <= 128 && tc_rows >= (latency ? 64 : 96) &&
+                   (latency || q_tiles_for(128) <= q_tiles_for(144)));
   if (rows_cap <= 0) rows_cap = tc ? 128 : (latency ? 64 : 144);
   if (tc) rows_cap = std::min(rows_cap, 128);
   if (min_tiles <= 0) min_tiles = latency ? 1 : 2;
@@ -654,7 +662,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa,
               [](int S, int NW, int stages, bool tc) { return attn_device_capacity(true, S, NW, stages, tc); },
-              x->attn_rows_cap, x->attn_min_tiles, g_attn_tc.load() != 0);
+              x->attn_rows_cap, x->attn_min_tiles, g_attn_kernel.load());
     const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
     attn_traced = x->attn_trace && ctas * 16 <= x->attn_trace_n;
   } else {
@@ -1782,9 +1790,9 @@ nld_status nld_debug_layer_trace(nld_ctx* x, int layer, unsigned long long* d_at
   return NLD_OK;
 }
 
-nld_status nld_debug_attention_kernel(int tcgen05) {
-  if (tcgen05 != 0 && tcgen05 != 1) return fail(nullptr, NLD_ERR_ARG, "0 (mma.sync) or 1 (tcgen05)");
-  g_attn_tc.store(tcgen05);
+nld_status nld_debug_attention_kernel(int kernel) {
+  if (kernel < 0 || kernel > 2) return fail(nullptr, NLD_ERR_ARG, "0 (planner), 1 (tcgen05) or 2 (mma.sync)");
+  g_attn_kernel.store(kernel);
   return NLD_OK;
 }
 
@@ -1859,8 +1867,8 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
   return NLD_OK;
 }
 
-nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out6) {
-  if (!out6) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
+nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out7) {
+  if (!out7) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
   if (batch < 1 || m < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_len < 1 || sms < 1)
     return fail(nullptr, NLD_ERR_ARG, "bad attention plan sizes");
   AttnArgs a{};
@@ -1870,13 +1878,9 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
     const size_t smem = tc ? attn_tc_smem_bytes(true) : attn_mma_smem_bytes(NW, true, stages);
     const int per_sm = static_cast<int>(233472 / (smem + 1024));
     return std::max(1, sms * per_sm / S);
-  });
-  out6[0] = a.G;
-  out6[1] = a.QT;
-  out6[2] = a.q_tiles;
-  out6[3] = a.rows;
-  out6[4] = a.NW;
-  out6[5] = a.S;
+  }, 0, 0, g_attn_kernel.load());
+  const int v[7] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc};
+  for (int i = 0; i < 7; ++i) out7[i] = v[i];
   return NLD_OK;
 }
 
@@ -2107,7 +2111,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   AttnArgs a{};
   attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
             [](int S, int NW, int stages, bool tc) { return attn_device_capacity(false, S, NW, stages, tc); },
-            0, 0, g_attn_tc.load() != 0);
+            0, 0, g_attn_kernel.load());
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))

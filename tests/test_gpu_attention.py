@@ -25,7 +25,7 @@ def attention_kernel(request):
     back to the default afterwards)."""
     import self_speculation_b200 as nb
     lib = nb.load_library()
-    assert lib.nld_debug_attention_kernel(1 if request.param == "tcgen05" else 0) == 0
+    assert lib.nld_debug_attention_kernel(1 if request.param == "tcgen05" else 2) == 0
     yield request.param
     assert lib.nld_debug_attention_kernel(0) == 0
 

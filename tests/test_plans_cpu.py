@@ -7,6 +7,7 @@ are the ones the committed launch list records (layer chain 132 CTAs in clusters
 QKV 96 CTAs in clusters of 2, attention in query tiles of <= 64 rows and single-tile KV
 splits)."""
 import ctypes
+import itertools
 
 import pytest
 
@@ -35,11 +36,16 @@ def plan_chain(M, phases, clusters=B200_CLUSTERS, hilo=1):
                 split=[(o[10 + 2 * p], o[11 + 2 * p]) for p in range(n)])
 
 
-def plan_attention(batch, m, Hq, Hkv, max_len, sms=148):
+def plan_attention(batch, m, Hq, Hkv, max_len, sms=148, kernel=0):
+    """kernel: 0 the planner's choice, 1 tcgen05, 2 mma.sync (the process-wide setting is put back)."""
     lib = nb.load_library()
-    out = (ctypes.c_int * 6)()
-    assert lib.nld_plan_attention(batch, m, Hq, Hkv, max_len, sms, out) == 0
-    return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S"], list(out)))
+    out = (ctypes.c_int * 7)()
+    assert lib.nld_debug_attention_kernel(kernel) == 0
+    try:
+        assert lib.nld_plan_attention(batch, m, Hq, Hkv, max_len, sms, out) == 0
+    finally:
+        assert lib.nld_debug_attention_kernel(0) == 0
+    return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S", "tc"], list(out)))
 
 
 def chains(cfg):
@@ -122,13 +128,16 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
             m = M // B
             if m > 2 * cfg.block_k + 1:
                 continue
-            for max_len in (m, 64, 900, 4096 + m, 32768):
-                A = plan_attention(B, m, cfg.n_q_heads, cfg.n_kv_heads, max_len)
-                where = (name, B, m, max_len)
+            for max_len, kernel in itertools.product((m, 64, 900, 4096 + m, 32768), (0, 1, 2)):
+                A = plan_attention(B, m, cfg.n_q_heads, cfg.n_kv_heads, max_len, kernel=kernel)
+                where = (name, B, m, max_len, kernel)
                 assert A["G"] * cfg.n_kv_heads == cfg.n_q_heads, where
                 assert 1 <= A["QT"] <= m and A["QT"] * A["q_tiles"] >= m, where
                 assert A["rows"] == A["QT"] * A["G"] and A["rows"] <= 16 * A["NW"], where
                 assert 1 <= A["NW"] <= 9 and A["rows"] <= 144, where
+                assert A["tc"] == {1: 1, 2: 0}.get(kernel, A["tc"]), where
+                if A["tc"]:
+                    assert A["rows"] <= 128, where   # one tcgen05 MMA tile
                 assert 1 <= A["S"] <= 8, where
                 assert A["S"] <= -(-max_len // 64), where   # every split has a KV tile
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
@@ -136,17 +145,32 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
 
 
 def test_attention_plan_of_the_benchmarked_round():
-    # verify forward (m = 33: 3 query tiles of 11 positions x 4 heads, 3 warps) and draft forward
-    # (m = 32: 2 tiles of 16 positions, 4 warps); 545 keys = 9 tiles in 5 splits of <= 2 tiles,
-    # 865 keys = 14 tiles in 7 splits
-    for keys, S in ((545, 5), (865, 7)):
+    # tcgen05 (the planner's choice): verify forward (m = 33: 2 query tiles of 17 positions x 4
+    # heads) and draft forward (m = 32: one 128-row tile); 545 keys = 9 tiles in 5 splits of <= 2
+    # tiles, 865 keys = 14 tiles in 7 splits, 1400 keys = 22 tiles in 8 splits
+    for keys, S in ((545, 5), (865, 7), (1400, 8)):
         v = plan_attention(1, 33, 32, 8, keys)
         d = plan_attention(1, 32, 32, 8, keys)
-        assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"]) == (4, 11, 3, 3, S)
-        assert (d["QT"], d["q_tiles"], d["NW"], d["S"]) == (16, 2, 4, S)
-    # many sequences: the whole 33-position verify block of 4 heads in one 9-warp CTA, no split
+        assert (v["G"], v["QT"], v["q_tiles"], v["rows"], v["S"], v["tc"]) == (4, 17, 2, 68, S, 1)
+        assert (d["QT"], d["q_tiles"], d["rows"], d["S"], d["tc"]) == (32, 1, 128, S, 1)
+    # mma.sync: 3 query tiles of 11 positions (3 warps) and 2 tiles of 16 positions (4 warps)
+    for keys, S in ((545, 5), (865, 7)):
+        v = plan_attention(1, 33, 32, 8, keys, kernel=2)
+        d = plan_attention(1, 32, 32, 8, keys, kernel=2)
+        assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"], v["tc"]) == (4, 11, 3, 3, S, 0)
+        assert (d["QT"], d["q_tiles"], d["NW"], d["S"], d["tc"]) == (16, 2, 4, S, 0)
+    # many sequences: the whole 33-position verify block of 4 heads in one 9-warp mma.sync CTA,
+    # no split (128-row tcgen05 tiles would take two CTAs); a 32-position block stays on tcgen05
     b = plan_attention(64, 33, 32, 8, 4096 + 33)
-    assert (b["QT"], b["q_tiles"], b["NW"], b["S"]) == (33, 1, 9, 1)
+    assert (b["QT"], b["q_tiles"], b["NW"], b["S"], b["tc"]) == (33, 1, 9, 1, 0)
+    b = plan_attention(64, 32, 32, 8, 4096 + 32)
+    assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"]) == (32, 1, 128, 1, 1)
+    # small query tiles (a 4-row single-token decode, 64-row blocks of many sequences) cost the
+    # tcgen05 kernel a whole 128-row tile per KV tile: they stay on mma.sync
+    assert plan_attention(1, 1, 32, 8, 4096)["tc"] == 0
+    assert plan_attention(64, 1, 32, 8, 4096)["tc"] == 0
+    assert plan_attention(16, 16, 32, 8, 2048)["tc"] == 0
+    assert plan_attention(1, 16, 32, 8, 2048)["tc"] == 1
 
 
 def test_plan_hooks_reject_bad_sizes():
@@ -159,4 +183,4 @@ def test_plan_hooks_reject_bad_sizes():
     assert lib.nld_plan_chain(0, 1, rows, (ctypes.c_int * 1)(4096), mc, 1, out) == 1
     none = (ctypes.c_int * 9)(*([0] * 9))
     assert lib.nld_plan_chain(33, 1, rows, (ctypes.c_int * 1)(4096), none, 1, out) == 8   # unsupported
-    assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 6)()) == 1
+    assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 7)()) == 1
