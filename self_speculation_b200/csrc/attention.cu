@@ -529,33 +529,42 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // ------------------------------------------------------------------ tcgen05 attention --
 // The same attention on the 5th-generation tensor cores, for query tiles of <= 128 rows: one
 // CTA per (KV split, kv head, sequence x query tile), TMEM lane r = query row r.  Per KV tile of
-// 64 keys, S = Q K^T (M 128, N 64, K 128) goes to one of two TMEM S buffers.  Eight softmax
-// warps take two threads per row, one per half of the tile's keys; each half keeps its own
-// online softmax (reference max, row sum) and its own O accumulator in TMEM, so the two never
-// exchange anything inside the KV loop: a thread reads its 32 scores, masks and scales them,
-// writes P as packed bf16 pairs (with hi/lo: its lo half too) into TMEM, and O_h += P_h V_h
-// (M 128, N 128, K 32) takes P from TMEM as the A operand and V straight from the TMA tile as an
-// MN-major operand.  A half's reference max moves only when a tile's max exceeds it by more than
-// 2^8 (so P <= 256), which rescales that half's O row in TMEM.  After the loop the two halves of
-// a row combine like two KV splits, then splits merge over the cluster as in attn_mma_kernel.
-// One thread loads K/V by TMA into a 5-stage (bf16 Q: 6-stage) ring, another issues the MMAs;
-// P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.  TMEM columns:
-// S buffers 0..127, O_0 128..255, O_1 256..383, P buffers 384..511 (per buffer, key half h at
-// 32h: hi pairs, then lo pairs).
-constexpr int kTcSoftmax = 256;                 // 8 warps: half h = warp / 4, rows of warp % 4
+// 64 keys, S = Q K^T (M 128, N 64, K 128) goes to one of two TMEM S buffers, issued two tiles
+// ahead of the softmax.  Sixteen softmax warps take four threads per row, one per 16-key quarter
+// of each tile (warps w, w+4, w+8, w+12 share TMEM lane quarter w % 4 and an SM sub-partition):
+// a thread reads its 16 scores, the four threads of a row exchange their maxima through shared
+// memory (an mbarrier per lane quarter and tile parity), and each writes P as packed bf16 pairs
+// (with hi/lo: its lo half too) into TMEM.  O += P V (M 128, N 128, K 64) takes P from TMEM as
+// the A operand and V straight from the TMA tile as an MN-major operand.  A row's reference max
+// moves only when a tile's max exceeds it by more than 2^8 (so P <= 256), which rescales its O
+// row in TMEM (each thread its 32 columns).  Splits merge over the cluster as in
+// attn_mma_kernel.  One thread loads K/V by TMA into a 4-stage (bf16 Q: 5-stage) ring, another
+// issues the MMAs; P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.
+// TMEM columns: S buffers 0..127, O 128..255, P buffers 384..511 (per buffer: 32 columns of hi
+// pairs, then 32 of lo pairs; key quarter q at 8q).
+constexpr int kTcSoftmax = 512;                 // 16 warps: key quarter warp / 4, rows of warp % 4
 constexpr int kTcThreads = kTcSoftmax + 64;     // + the MMA warp + the TMA warp
-constexpr int kTcMaxStages = 6;
-__host__ __device__ constexpr int tc_stages(bool hilo) { return hilo ? 5 : 6; }
+constexpr int kTcMaxStages = 5;
+__host__ __device__ constexpr int tc_stages(bool hilo) { return hilo ? 4 : 5; }
 // S of tile j + 2 is issued before O += P V of tile j, so its K/V stage must not wait for that
 static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
 constexpr int kTcBarBytes = 256;
+constexpr int kTcXchgBytes = 2 * 4 * 128 * 4;   // row-max exchange: [tile parity][quarter][row]
 
 // 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0).
 NLD_DEV float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 8 consecutive 32-bit TMEM columns from registers (lane = thread); visible to later tcgen05
+// operations after tmem_st_wait().
+NLD_DEV void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate; A's row i is TMEM lane i,
@@ -593,16 +602,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sQ = smem;                              // [kQ][2 dim boxes][128 rows][128 B]
   uint8_t* sK = sQ + kQ * 32768;                   // [NS][2 dim boxes][64 keys][128 B]
   uint8_t* sV = sK + NS * kKVTile;                 // same
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile);
+  float* xmax = reinterpret_cast<float*>(sV + NS * kKVTile);   // [2][4][128] row maxima
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile + kTcXchgBytes);
   uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
   uint64_t* empty = bars + kTcMaxStages;   // [NS] K/V stage free (the tile's P V MMAs completed)
   uint64_t* s_full = bars + 2 * kTcMaxStages;   // [2] S buffer written (MMA commit)
-  uint64_t* s_free = s_full + 2;      // [2] S buffer read (256 softmax threads)
-  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (256 softmax threads)
+  // the softmax warps arrive on their barriers once per warp (lane 0, after the warp's threads
+  // synchronise): one arrival per thread would queue 512 arrivals per barrier and tile
+  uint64_t* s_free = s_full + 2;      // [2] S buffer read (16 softmax warps)
+  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (16 softmax warps)
   uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
   uint64_t* fin = s_full + 8;         // the MMA thread's outstanding MMAs on an early exit
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 9);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 10);
+  uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (4 warps)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 17);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 18);
   constexpr uint64_t kWait = 2000000000ull;
 
   const int tid = threadIdx.x;
@@ -627,17 +640,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kTcSoftmax);
-      mbar_init(&p_full[i], kTcSoftmax);
+      mbar_init(&s_free[i], kTcSoftmax / 32);
+      mbar_init(&p_full[i], kTcSoftmax / 32);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(fin, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 4);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmKV);
   }
   if (warp == kTcSoftmax / 32) {
-    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O_0: 128..255, O_1: 256..383, P: 384..511
+    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O: 128..255, P: 384..511
     tmem_relinquish();
   }
   tc_fence_before();
@@ -687,18 +701,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tma_thr)
     for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
 
-  const int hk = tid >> 7;            // softmax threads: key half
+  const int kq = tid >> 7;            // softmax threads: key quarter
   const int r = tid & 127;            // and query row (position r / G, head r % G)
   const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
-  // query rows -> shared memory, coalesced: piece e = tid + 256u of the tile's 128 rows x 16
+  // query rows -> shared memory, coalesced: piece e = tid + 512u of the tile's 128 rows x 16
   // pieces of 8 dims (row e / 16, piece c = e % 16) goes to box c / 8 at piece (c % 8) ^ (row % 8);
   // padding rows are zero
+  constexpr int kQPer = 2048 / kTcSoftmax;
   if (softmax_thr) {
-    uint4 hv[8], lv[8];
-    int offs[8];
+    uint4 hv[kQPer], lv[kQPer];
+    int offs[kQPer];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kQPer; ++u) {
       const int e = tid + u * kTcSoftmax;
       const int row = e >> 4, c = e & 15;
       const int p = row / a.G, gh = row - p * a.G;
@@ -718,7 +733,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kQPer; ++u) {
       *reinterpret_cast<uint4*>(sQ + offs[u]) = hv[u];
       if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQ + 32768 + offs[u]) = lv[u];
     }
@@ -753,16 +768,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(i >> 1) & 1u, kWait)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int q = 0; q < kQ; ++q)
 #pragma unroll
-        for (int q = 0; q < kQ; ++q)
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const int ks = h * 2 + kk;   // 16-key step of the tile: 8 TMEM columns of P
-            tc_mma_f16_ts(tmem + 128 + h * 128, tmem + 384 + pb * 64 + h * 32 + q * 16 + kk * 8,
-                          sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
-                          (i > 0 || q > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int ks = 0; ks < 4; ++ks)   // 16-key step of the tile: 8 TMEM columns of P
+          tc_mma_f16_ts(tmem + 128, tmem + 384 + pb * 64 + q * 32 + ks * 8,
+                        sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
+                        (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
       tc_commit(&pv_done[pb]);
       tc_commit(&empty[st]);
       return true;
@@ -805,11 +816,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_commit(fin);
     mbar_wait(fin, 0, kWait);
   } else if (softmax_thr) {
-    // ------------------------------------------- softmax: row r, keys 32hk..32hk+31 --
+    // ------------------------------------------- softmax: row r, keys 16kq..16kq+15 --
     int v1 = -1, l2 = 0x7fffffff, h2 = -1;
     if (row_ok) row_keys(len, p0 + prow, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t o_col = 128 + hk * 128;
+    const int lq = warp & 3;   // TMEM lane quarter
+    const uint32_t lane_base = static_cast<uint32_t>(lq * 32) << 16;
+    const uint32_t o_col = 128 + kq * 32;   // this thread's 32 columns of O
+    const float c = a.scale_log2;
     for (int j = 0; j < ntile; ++j) {
       const int sb = j & 1;
       // tcgen05.ld/st are warp-collective: every exit of this loop is taken by the whole warp
@@ -819,55 +832,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[32];
-      {
-        uint32_t raw[2][16];
-        tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32, raw[0]);
-        tmem_ld16_nowait(tmem + lane_base + sb * 64 + hk * 32 + 16, raw[1]);
-        tmem_ld_wait_regs(raw[0]);
-        tmem_ld_wait_regs(raw[1]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) sv[c * 16 + i] = __uint_as_float(raw[c][i]);
-      }
+      uint32_t raw[16];
+      tmem_ld16_nowait(tmem + lane_base + sb * 64 + kq * 16, raw);
+      tmem_ld_wait_regs(raw);
       tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-      const int k0 = (t_lo + j) * kPage + hk * 32;
-      if (k0 + 31 <= v1) {
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&s_free[sb]);
+      float sv[16];
+      const int k0 = (t_lo + j) * kPage + kq * 16;
+      if (k0 + 15 <= v1) {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) sv[k] *= a.scale_log2;
+        for (int k = 0; k < 16; ++k) sv[k] = __uint_as_float(raw[k]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) sv[k] = key_visible(k0 + k, v1, l2, h2) ? sv[k] * a.scale_log2 : -INFINITY;
+        for (int k = 0; k < 16; ++k) sv[k] = key_visible(k0 + k, v1, l2, h2) ? __uint_as_float(raw[k]) : -INFINITY;
       }
-      // max as a tree (independent pairs: short dependency chains)
-      float mt[16];
+      // the row's max over the tile: a tree over this thread's 16 scores, then the four
+      // quarters' through shared memory (scores unscaled: the scale is positive)
+      float mt[8];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) mt[k] = fmaxf(sv[k], sv[k + 16]);
+      for (int k = 0; k < 8; ++k) mt[k] = fmaxf(sv[k], sv[k + 8]);
 #pragma unroll
-      for (int w = 8; w > 0; w >>= 1)
+      for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
         for (int k = 0; k < w; ++k) mt[k] = fmaxf(mt[k], mt[k + w]);
-      const float mx = mt[0];
+      float* xm = xmax + sb * 512;
+      xm[kq * 128 + r] = mt[0];
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&xbar[sb * 4 + lq]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&xbar[sb * 4 + lq], static_cast<uint32_t>(j >> 1) & 1u, kWait))) {
+        aborted = true;
+        break;
+      }
+      const float mx = fmaxf(fmaxf(xm[r], xm[128 + r]), fmaxf(xm[256 + r], xm[384 + r])) * c;
       const bool move = mx > m_ref + kTcRescale;
       const bool scale_o = move && j >= 1 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, scale_o)) {
-        // this half's O row holds tiles < j once O += P V of tile j - 1 has completed; the warp
-        // rescales its 32 rows together (factor 1 for rows that keep their max)
+        // the O row holds tiles < j once O += P V of tile j - 1 has completed; the warp rescales
+        // its 32 rows x 32 columns together (factor 1 for rows that keep their max)
         if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, kWait))) {
           aborted = true;
           break;
         }
         tc_fence_after();
         const float alpha = scale_o ? exp2f(m_ref - mx) : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
           float o[16];
-          tmem_ld16(tmem + lane_base + o_col + c * 16, o);
+          tmem_ld16(tmem + lane_base + o_col + cc * 16, o);
 #pragma unroll
           for (int i = 0; i < 16; ++i) o[i] *= alpha;
-          tmem_st16(tmem + lane_base + o_col + c * 16, o);
+          tmem_st16(tmem + lane_base + o_col + cc * 16, o);
         }
         tmem_st_wait();
         l_sum *= alpha;
@@ -878,31 +893,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         aborted = true;
         break;
       }
-      const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // P row r, keys 32hk..32hk+31 as 16 bf16 pairs (lower key in the low half), hi then lo
-      float ph[16], pl[16];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      // P row r, keys 16kq..16kq+15 as 8 bf16 pairs (lower key in the low half), hi then lo
+      uint32_t ph[8], pl[8];
+      float ls[2] = {0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float p0 = ex2_approx(sv[2 * c] - base), p1 = ex2_approx(sv[2 * c + 1] - base);
-        ls[c & 3] += p0 + p1;
-        uint32_t hi, lo;
+      for (int k = 0; k < 8; ++k) {
+        const float q0 = ex2_approx(fmaf(sv[2 * k], c, nb)), q1 = ex2_approx(fmaf(sv[2 * k + 1], c, nb));
+        ls[k & 1] += q0 + q1;
         if constexpr (kHiLo) {
-          pack_bf16_hilo(p0, p1, hi, lo);
+          pack_bf16_hilo(q0, q1, ph[k], pl[k]);
         } else {
-          hi = pack_bf16(p0, p1);
-          lo = 0u;
+          ph[k] = pack_bf16(q0, q1);
+          pl[k] = 0u;
         }
-        ph[c] = __uint_as_float(hi);
-        pl[c] = __uint_as_float(lo);
       }
-      l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      const uint32_t p_col = 384 + sb * 64 + hk * 32;
-      tmem_st16(tmem + lane_base + p_col, ph);
-      if constexpr (kHiLo) tmem_st16(tmem + lane_base + p_col + 16, pl);
+      l_sum += ls[0] + ls[1];
+      const uint32_t p_col = 384 + sb * 64 + kq * 8;
+      tmem_st8(tmem + lane_base + p_col, ph);
+      if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + 32, pl);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&p_full[sb]);
       if (j < 6 && tid == 0) stamp(3 + j);
     }
     if (!aborted && ntile > 0 &&
@@ -933,54 +946,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   };
 
-  // the two key halves of a row combine: thread (h, r) takes dims 64h..64h+63 of both O_0 and
-  // O_1, weighted by 2^(m_h - M) with M the larger reference max, into the CTA's partial (O
-  // unnormalised, (M, L)) in shared memory; float4 slot s of row r sits at slot s ^ (r % 32)
+  // the CTA's partial (O unnormalised, (m, L)) into shared memory: the four key quarters' row
+  // sums add up (one reference max per row), thread (q, r) moves columns 32q..32q+31 of O; float4
+  // slot s of row r sits at slot s ^ (r % 32)
   __syncthreads();   // every MMA and every TMA load of this CTA has completed
   float* sO = reinterpret_cast<float*>(smem);            // [128][128] partials (over Q, K)
   float* sML = sO + 128 * 128;                           // [128][2]
-  float2* sMLh = reinterpret_cast<float2*>(sML + 256);   // [2][128] (m, l) per key half
+  float* sLq = sML + 256;                                // [4][128] row sums per key quarter
   const bool have = ntile > 0 && !*s_abort;
   // after a timeout anywhere, the loads still in flight land before the ring is overlaid
   if (tma_thr && !have)
     for (int t = max(0, n_issued - NS); t < n_issued; ++t)
       mbar_wait(&full[t % NS], static_cast<uint32_t>(t / NS) & 1u, kWait);
-  if (softmax_thr) sMLh[hk * 128 + r] = make_float2(have ? m_ref : -INFINITY, have ? l_sum : 0.f);
+  if (softmax_thr) sLq[kq * 128 + r] = have ? l_sum : 0.f;
   __syncthreads();
   if (softmax_thr) {
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const float2 ml0 = sMLh[r], ml1 = sMLh[128 + r];
-    const float M = fmaxf(ml0.x, ml1.x);
-    const float w0 = (ml0.x == -INFINITY) ? 0.f : exp2f(ml0.x - M);
-    const float w1 = (ml1.x == -INFINITY) ? 0.f : exp2f(ml1.x - M);
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      uint32_t o0[2][16], o1[2][16];
-      const uint32_t col = hk * 64 + c * 32;
-      if (have) {
-        tmem_ld16_nowait(tmem + lane_base + 128 + col, o0[0]);
-        tmem_ld16_nowait(tmem + lane_base + 128 + col + 16, o0[1]);
-        tmem_ld16_nowait(tmem + lane_base + 256 + col, o1[0]);
-        tmem_ld16_nowait(tmem + lane_base + 256 + col + 16, o1[1]);
-        tmem_ld_wait_regs(o0[0]);
-        tmem_ld_wait_regs(o0[1]);
-        tmem_ld_wait_regs(o1[0]);
-        tmem_ld_wait_regs(o1[1]);
-      } else {
+    uint32_t o[2][16];
+    if (have) {
+      tmem_ld16_nowait(tmem + lane_base + 128 + kq * 32, o[0]);
+      tmem_ld16_nowait(tmem + lane_base + 128 + kq * 32 + 16, o[1]);
+      tmem_ld_wait_regs(o[0]);
+      tmem_ld_wait_regs(o[1]);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o0[0][i] = o0[1][i] = o1[0][i] = o1[1][i] = 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float o[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          o[t] = __uint_as_float(o0[(i + t) >> 4][(i + t) & 15]) * w0 + __uint_as_float(o1[(i + t) >> 4][(i + t) & 15]) * w1;
-        const int slot = ((col + i) >> 2) ^ (r & 31);
-        *reinterpret_cast<float4*>(sO + r * 128 + slot * 4) = make_float4(o[0], o[1], o[2], o[3]);
-      }
+      for (int i = 0; i < 16; ++i) o[0][i] = o[1][i] = 0u;
     }
-    if (hk == 0) *reinterpret_cast<float2*>(sML + r * 2) = make_float2(M, ml0.y * w0 + ml1.y * w1);
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const int slot = ((kq * 32 + i) >> 2) ^ (r & 31);
+      *reinterpret_cast<float4*>(sO + r * 128 + slot * 4) =
+          make_float4(__uint_as_float(o[i >> 4][i & 15]), __uint_as_float(o[i >> 4][(i & 15) + 1]),
+                      __uint_as_float(o[i >> 4][(i & 15) + 2]), __uint_as_float(o[i >> 4][(i & 15) + 3]));
+    }
+    if (kq == 0)
+      *reinterpret_cast<float2*>(sML + r * 2) =
+          make_float2(have ? m_ref : -INFINITY, (sLq[r] + sLq[128 + r]) + (sLq[256 + r] + sLq[384 + r]));
   }
   tc_fence_before();
   __syncthreads();
@@ -1147,11 +1148,11 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
 }
 
 // Dynamic shared memory of a tcgen05 attention launch: the query tile (hi and lo halves with
-// hilo), the K and V rings and the barriers; the split partials overlay the first two after the
-// KV loop.
+// hilo), the K and V rings, the row-max exchange and the barriers; the split partials overlay
+// the first two after the KV loop.
 size_t attn_tc_smem_bytes(bool hilo) {
   const size_t kq = hilo ? 2 : 1;
-  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + kTcBarBytes;
+  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + kTcXchgBytes + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
