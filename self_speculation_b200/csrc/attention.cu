@@ -542,15 +542,16 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // issues the MMAs; P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.
 // TMEM columns: S buffers 0..127, O 128..255, P buffers 384..511 (per buffer: 32 columns of hi
 // pairs, then 32 of lo pairs; key quarter q at 8q).
-constexpr int kTcSoftmax = 512;                 // 16 warps: key quarter warp / 4, rows of warp % 4
-constexpr int kTcThreads = kTcSoftmax + 64;     // + the MMA warp + the TMA warp
+// kRT softmax threads per row (2 or 4): 128 kRT softmax threads, + the MMA warp + the TMA warp
+__host__ __device__ constexpr int tc_threads(int rt) { return 128 * rt + 64; }
 constexpr int kTcMaxStages = 5;
 __host__ __device__ constexpr int tc_stages(bool hilo) { return hilo ? 4 : 5; }
 // S of tile j + 2 is issued before O += P V of tile j, so its K/V stage must not wait for that
 static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
 constexpr int kTcBarBytes = 256;
-constexpr int kTcXchgBytes = 2 * 4 * 128 * 4;   // row-max exchange: [tile parity][quarter][row]
+// row-max exchange: [tile parity][key part][row] floats
+__host__ __device__ constexpr int tc_xchg_bytes(int rt) { return 2 * rt * 128 * 4; }
 
 // 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0).
 NLD_DEV float ex2_approx(float x) {
@@ -591,9 +592,14 @@ NLD_DEV uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return d;
 }
 
-template <bool kHiLo>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <bool kHiLo, int kRT>
+__global__ void __launch_bounds__(tc_threads(kRT), 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
+  static_assert(kRT == 2 || kRT == 4, "2 or 4 softmax threads per row");
+  constexpr int kTcSoftmax = 128 * kRT;
+  constexpr int kTcThreads = tc_threads(kRT);
+  constexpr int kKT = 64 / kRT;    // keys of a tile per softmax thread
+  constexpr int kOC = 128 / kRT;   // O columns per softmax thread in the rescale and the combine
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -602,18 +608,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sQ = smem;                              // [kQ][2 dim boxes][128 rows][128 B]
   uint8_t* sK = sQ + kQ * 32768;                   // [NS][2 dim boxes][64 keys][128 B]
   uint8_t* sV = sK + NS * kKVTile;                 // same
-  float* xmax = reinterpret_cast<float*>(sV + NS * kKVTile);   // [2][4][128] row maxima
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile + kTcXchgBytes);
+  float* xmax = reinterpret_cast<float*>(sV + NS * kKVTile);   // [2][kRT][128] row maxima
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile + tc_xchg_bytes(kRT));
   uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
   uint64_t* empty = bars + kTcMaxStages;   // [NS] K/V stage free (the tile's P V MMAs completed)
   uint64_t* s_full = bars + 2 * kTcMaxStages;   // [2] S buffer written (MMA commit)
   // the softmax warps arrive on their barriers once per warp (lane 0, after the warp's threads
   // synchronise): one arrival per thread would queue 512 arrivals per barrier and tile
-  uint64_t* s_free = s_full + 2;      // [2] S buffer read (16 softmax warps)
-  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (16 softmax warps)
+  uint64_t* s_free = s_full + 2;      // [2] S buffer read (the softmax warps)
+  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (the softmax warps)
   uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
   uint64_t* fin = s_full + 8;         // the MMA thread's outstanding MMAs on an early exit
-  uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (4 warps)
+  uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (kRT warps)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 17);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 18);
   constexpr uint64_t kWait = 2000000000ull;
@@ -645,7 +651,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(fin, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 4);
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], kRT);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmKV);
@@ -701,11 +707,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tma_thr)
     for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
 
-  const int kq = tid >> 7;            // softmax threads: key quarter
+  const int kq = tid >> 7;            // softmax threads: key part (keys kKT kq .. of a tile)
   const int r = tid & 127;            // and query row (position r / G, head r % G)
   const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
-  // query rows -> shared memory, coalesced: piece e = tid + 512u of the tile's 128 rows x 16
+  // query rows -> shared memory, coalesced: piece e = tid + 128 kRT u of the tile's 128 rows x 16
   // pieces of 8 dims (row e / 16, piece c = e % 16) goes to box c / 8 at piece (c % 8) ^ (row % 8);
   // padding rows are zero
   constexpr int kQPer = 2048 / kTcSoftmax;
@@ -816,12 +822,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_commit(fin);
     mbar_wait(fin, 0, kWait);
   } else if (softmax_thr) {
-    // ------------------------------------------- softmax: row r, keys 16kq..16kq+15 --
+    // ------------------------------------- softmax: row r, keys kKT kq .. kKT kq + kKT - 1 --
     int v1 = -1, l2 = 0x7fffffff, h2 = -1;
     if (row_ok) row_keys(len, p0 + prow, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
     const int lq = warp & 3;   // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(lq * 32) << 16;
-    const uint32_t o_col = 128 + kq * 32;   // this thread's 32 columns of O
+    const uint32_t o_col = 128 + kq * kOC;   // this thread's columns of O
     const float c = a.scale_log2;
     for (int j = 0; j < ntile; ++j) {
       const int sb = j & 1;
@@ -832,31 +838,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t raw[16];
-      tmem_ld16_nowait(tmem + lane_base + sb * 64 + kq * 16, raw);
-      tmem_ld_wait_regs(raw);
+      uint32_t raw[kKT / 16][16];
+#pragma unroll
+      for (int u = 0; u < kKT / 16; ++u) tmem_ld16_nowait(tmem + lane_base + sb * 64 + kq * kKT + u * 16, raw[u]);
+#pragma unroll
+      for (int u = 0; u < kKT / 16; ++u) tmem_ld_wait_regs(raw[u]);
       tc_fence_before();
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&s_free[sb]);
-      float sv[16];
-      const int k0 = (t_lo + j) * kPage + kq * 16;
-      if (k0 + 15 <= v1) {
+      float sv[kKT];
+      const int k0 = (t_lo + j) * kPage + kq * kKT;
+      if (k0 + kKT - 1 <= v1) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) sv[k] = __uint_as_float(raw[k]);
+        for (int k = 0; k < kKT; ++k) sv[k] = __uint_as_float(raw[k >> 4][k & 15]);
       } else {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) sv[k] = key_visible(k0 + k, v1, l2, h2) ? __uint_as_float(raw[k]) : -INFINITY;
+        for (int k = 0; k < kKT; ++k)
+          sv[k] = key_visible(k0 + k, v1, l2, h2) ? __uint_as_float(raw[k >> 4][k & 15]) : -INFINITY;
       }
-      // the row's max over the tile: a tree over this thread's 16 scores, then the four
-      // quarters' through shared memory (scores unscaled: the scale is positive)
-      float mt[8];
+      // the row's max over the tile: a tree over this thread's scores, then the kRT parts'
+      // through shared memory (scores unscaled: the scale is positive)
+      float mt[kKT / 2];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mt[k] = fmaxf(sv[k], sv[k + 8]);
+      for (int k = 0; k < kKT / 2; ++k) mt[k] = fmaxf(sv[k], sv[k + kKT / 2]);
 #pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
+      for (int w = kKT / 4; w > 0; w >>= 1)
 #pragma unroll
         for (int k = 0; k < w; ++k) mt[k] = fmaxf(mt[k], mt[k + w]);
-      float* xm = xmax + sb * 512;
+      float* xm = xmax + sb * kRT * 128;
       xm[kq * 128 + r] = mt[0];
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&xbar[sb * 4 + lq]);
@@ -864,12 +873,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         aborted = true;
         break;
       }
-      const float mx = fmaxf(fmaxf(xm[r], xm[128 + r]), fmaxf(xm[256 + r], xm[384 + r])) * c;
+      float mx = xm[r];
+#pragma unroll
+      for (int q = 1; q < kRT; ++q) mx = fmaxf(mx, xm[q * 128 + r]);
+      mx *= c;
       const bool move = mx > m_ref + kTcRescale;
       const bool scale_o = move && j >= 1 && m_ref != -INFINITY;
       if (__any_sync(0xffffffffu, scale_o)) {
         // the O row holds tiles < j once O += P V of tile j - 1 has completed; the warp rescales
-        // its 32 rows x 32 columns together (factor 1 for rows that keep their max)
+        // its 32 rows x kOC columns together (factor 1 for rows that keep their max)
         if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, kWait))) {
           aborted = true;
           break;
@@ -877,7 +889,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         const float alpha = scale_o ? exp2f(m_ref - mx) : 1.f;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < kOC / 16; ++cc) {
           float o[16];
           tmem_ld16(tmem + lane_base + o_col + cc * 16, o);
 #pragma unroll
@@ -894,24 +906,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      // P row r, keys 16kq..16kq+15 as 8 bf16 pairs (lower key in the low half), hi then lo
-      uint32_t ph[8], pl[8];
-      float ls[2] = {0.f, 0.f};
+      // P row r, this thread's keys as kKT / 2 bf16 pairs (lower key in the low half), hi then lo
+      uint32_t ph[kKT / 16][8], pl[kKT / 16][8];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kKT / 2; ++k) {
         const float q0 = ex2_approx(fmaf(sv[2 * k], c, nb)), q1 = ex2_approx(fmaf(sv[2 * k + 1], c, nb));
-        ls[k & 1] += q0 + q1;
+        ls[k & 3] += q0 + q1;
         if constexpr (kHiLo) {
-          pack_bf16_hilo(q0, q1, ph[k], pl[k]);
+          pack_bf16_hilo(q0, q1, ph[k >> 3][k & 7], pl[k >> 3][k & 7]);
         } else {
-          ph[k] = pack_bf16(q0, q1);
-          pl[k] = 0u;
+          ph[k >> 3][k & 7] = pack_bf16(q0, q1);
+          pl[k >> 3][k & 7] = 0u;
         }
       }
-      l_sum += ls[0] + ls[1];
-      const uint32_t p_col = 384 + sb * 64 + kq * 8;
-      tmem_st8(tmem + lane_base + p_col, ph);
-      if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + 32, pl);
+      l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      const uint32_t p_col = 384 + sb * 64 + kq * (kKT / 2);
+#pragma unroll
+      for (int u = 0; u < kKT / 16; ++u) {
+        tmem_st8(tmem + lane_base + p_col + u * 8, ph[u]);
+        if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + 32 + u * 8, pl[u]);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -946,13 +961,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   };
 
-  // the CTA's partial (O unnormalised, (m, L)) into shared memory: the four key quarters' row
-  // sums add up (one reference max per row), thread (q, r) moves columns 32q..32q+31 of O; float4
-  // slot s of row r sits at slot s ^ (r % 32)
+  // the CTA's partial (O unnormalised, (m, L)) into shared memory: the kRT key parts' row sums
+  // add up (one reference max per row), thread (q, r) moves columns kOC q .. of O; float4 slot s
+  // of row r sits at slot s ^ (r % 32)
   __syncthreads();   // every MMA and every TMA load of this CTA has completed
   float* sO = reinterpret_cast<float*>(smem);            // [128][128] partials (over Q, K)
   float* sML = sO + 128 * 128;                           // [128][2]
-  float* sLq = sML + 256;                                // [4][128] row sums per key quarter
+  float* sLq = sML + 256;                                // [kRT][128] row sums per key part
   const bool have = ntile > 0 && !*s_abort;
   // after a timeout anywhere, the loads still in flight land before the ring is overlaid
   if (tma_thr && !have)
@@ -962,26 +977,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (softmax_thr) {
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t o[2][16];
-    if (have) {
-      tmem_ld16_nowait(tmem + lane_base + 128 + kq * 32, o[0]);
-      tmem_ld16_nowait(tmem + lane_base + 128 + kq * 32 + 16, o[1]);
-      tmem_ld_wait_regs(o[0]);
-      tmem_ld_wait_regs(o[1]);
-    } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o[0][i] = o[1][i] = 0u;
-    }
+    for (int cc = 0; cc < kOC / 32; ++cc) {
+      uint32_t o[2][16];
+      if (have) {
+        tmem_ld16_nowait(tmem + lane_base + 128 + kq * kOC + cc * 32, o[0]);
+        tmem_ld16_nowait(tmem + lane_base + 128 + kq * kOC + cc * 32 + 16, o[1]);
+        tmem_ld_wait_regs(o[0]);
+        tmem_ld_wait_regs(o[1]);
+      } else {
 #pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      const int slot = ((kq * 32 + i) >> 2) ^ (r & 31);
-      *reinterpret_cast<float4*>(sO + r * 128 + slot * 4) =
-          make_float4(__uint_as_float(o[i >> 4][i & 15]), __uint_as_float(o[i >> 4][(i & 15) + 1]),
-                      __uint_as_float(o[i >> 4][(i & 15) + 2]), __uint_as_float(o[i >> 4][(i & 15) + 3]));
+        for (int i = 0; i < 16; ++i) o[0][i] = o[1][i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const int slot = ((kq * kOC + cc * 32 + i) >> 2) ^ (r & 31);
+        *reinterpret_cast<float4*>(sO + r * 128 + slot * 4) =
+            make_float4(__uint_as_float(o[i >> 4][i & 15]), __uint_as_float(o[i >> 4][(i & 15) + 1]),
+                        __uint_as_float(o[i >> 4][(i & 15) + 2]), __uint_as_float(o[i >> 4][(i & 15) + 3]));
+      }
     }
-    if (kq == 0)
-      *reinterpret_cast<float2*>(sML + r * 2) =
-          make_float2(have ? m_ref : -INFINITY, (sLq[r] + sLq[128 + r]) + (sLq[256 + r] + sLq[384 + r]));
+    if (kq == 0) {
+      float L = 0.f;
+#pragma unroll
+      for (int q = 0; q < kRT; ++q) L += sLq[q * 128 + r];
+      *reinterpret_cast<float2*>(sML + r * 2) = make_float2(have ? m_ref : -INFINITY, L);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1112,8 +1133,9 @@ namespace {
 using AttnKernel = void (*)(const CUtensorMap, const AttnArgs);
 // The instantiation for a launch: tcgen05 or mma.sync, its operand form and (mma.sync) its
 // launch bound (<= 8 or 9 warps).
-AttnKernel attn_kernel_for(bool hilo, int NW, bool tc) {
-  if (tc) return hilo ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+AttnKernel attn_kernel_for(bool hilo, int NW, int tc) {
+  if (tc == 2) return hilo ? attn_tc_kernel<true, 2> : attn_tc_kernel<false, 2>;
+  if (tc) return hilo ? attn_tc_kernel<true, 4> : attn_tc_kernel<false, 4>;
   if (NW > 8) return hilo ? attn_mma_kernel<true, 9> : attn_mma_kernel<false, 9>;
   return hilo ? attn_mma_kernel<true, 8> : attn_mma_kernel<false, 8>;
 }
@@ -1127,8 +1149,8 @@ cudaError_t init_kernel_attributes() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  for (int v = 0; v < 6; ++v) {
-    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8, v >= 4);
+  for (int v = 0; v < 8; ++v) {   // mma.sync (hilo x 8/9 warps), tcgen05 (hilo x 2/4 per row)
+    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8, v >= 4 ? 2 * ((v >> 1) & 1) + 2 : 0);
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1150,18 +1172,18 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
 // Dynamic shared memory of a tcgen05 attention launch: the query tile (hi and lo halves with
 // hilo), the K and V rings, the row-max exchange and the barriers; the split partials overlay
 // the first two after the KV loop.
-size_t attn_tc_smem_bytes(bool hilo) {
+size_t attn_tc_smem_bytes(bool hilo, int rt) {
   const size_t kq = hilo ? 2 : 1;
-  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + kTcXchgBytes + kTcBarBytes;
+  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + tc_xchg_bytes(rt) + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
 // resident at once.
-int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, bool tc) {
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, int tc) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S * (sms / S));
-  cfg.blockDim = dim3(tc ? kTcThreads : 32 * NW);
-  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(hilo) : attn_mma_smem_bytes(NW, hilo, stages);
+  cfg.blockDim = dim3(tc ? tc_threads(tc) : 32 * NW);
+  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(hilo, tc) : attn_mma_smem_bytes(NW, hilo, stages);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
@@ -1180,14 +1202,15 @@ int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, bool tc
 
 cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const AttnArgs& a,
                                  int batch, bool pdl) {
-  const bool tc = a.tc != 0;
-  if (tc ? (a.rows < 1 || a.rows > 128 || a.S < 1 || a.S > 8)
-         : (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages))
-    return cudaErrorInvalidValue;   // tile rows / launch bound, ring depth
+  const int tc = a.tc;
+  if ((tc != 0 && tc != 2 && tc != 4) ||
+      (tc ? (a.rows < 1 || a.rows > 128 || a.S < 1 || a.S > 8)
+          : (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages)))
+    return cudaErrorInvalidValue;   // kernel form, tile rows / launch bound, ring depth
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.S, a.Hkv, batch * a.q_tiles);
-  cfg.blockDim = dim3(tc ? kTcThreads : 32 * a.NW);
-  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(a.hilo != 0) : attn_mma_smem_bytes(a.NW, a.hilo != 0, a.stages);
+  cfg.blockDim = dim3(tc ? tc_threads(tc) : 32 * a.NW);
+  cfg.dynamicSmemBytes = tc ? attn_tc_smem_bytes(a.hilo != 0, tc) : attn_mma_smem_bytes(a.NW, a.hilo != 0, a.stages);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

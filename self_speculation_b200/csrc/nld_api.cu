@@ -29,8 +29,8 @@ using namespace nld;
 
 namespace nld {
 size_t attn_mma_smem_bytes(int NW, bool hilo, int stages);
-size_t attn_tc_smem_bytes(bool hilo);
-int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, bool tc);
+size_t attn_tc_smem_bytes(bool hilo, int rt);
+int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, int tc);
 cudaError_t init_kernel_attributes();
 }
 
@@ -488,10 +488,10 @@ nld_status chain(nld_ctx* x, const ProjRef* pr, int nph, int M, bool pdl, unsign
 
 // Clusters of S attention CTAs (NW warps, `stages` ring stages; or the tcgen05 kernel) resident
 // at once.
-using AttnCapacity = std::function<int(int S, int NW, int stages, bool tc)>;
+using AttnCapacity = std::function<int(int S, int NW, int stages, int tc)>;
 
 // Which kernel serves the tensor-core attention (profiling hook): 0 the planner's choice,
-// 1 tcgen05, 2 mma.sync.
+// 1 tcgen05, 2 mma.sync, 3 / 4 tcgen05 with 2 / 4 softmax threads per row.
 std::atomic<int> g_attn_kernel{0};
 
 // rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
@@ -519,15 +519,17 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   const bool latency = batch * Hkv * q_tiles_for(144) * 8 < 2 * sms;
   const int tc_rows = ((m + q_tiles_for(128) - 1) / q_tiles_for(128)) * a.G;
   const int mma_rows = ((m + q_tiles_for(144) - 1) / q_tiles_for(144)) * a.G;
-  const bool tc = kernel == 1 ||
-                  (kernel == 0 && rows_cap <= 128 &&
-                   (latency ? tc_rows >= 64 : q_tiles_for(128) * 64 < q_tiles_for(144) * mma_rows));
+  const bool use_tc = kernel == 1 || kernel >= 3 ||
+                      (kernel == 0 && rows_cap <= 128 &&
+                       (latency ? tc_rows >= 64 : q_tiles_for(128) * 64 < q_tiles_for(144) * mma_rows));
+  // softmax threads per row (set below for the planner's choice)
+  int tc = !use_tc ? 0 : kernel == 3 ? 2 : 4;
   if (rows_cap <= 0) rows_cap = tc ? 128 : (latency ? 64 : 144);
   if (tc) rows_cap = std::min(rows_cap, 128);
   if (min_tiles <= 0) min_tiles = latency ? 1 : 2;
   a.min_tiles = min_tiles;
   a.stages = (latency || tc) ? 2 : 3;
-  a.tc = tc ? 1 : 0;
+  a.tc = tc;
   // query positions per CTA: as many as rows_cap allows, spread evenly over the query tiles
   const int nq = q_tiles_for(rows_cap);
   a.QT = (m + nq - 1) / nq;
@@ -546,20 +548,29 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
     const int per = std::max(min_tiles, (n_tiles + s_max - 1) / s_max);
     a.S = std::max(1, (n_tiles + per - 1) / per);
   }
+  // tcgen05 softmax threads per row: 4 (16 warps) shorten a CTA's fixed costs and each KV tile's
+  // latency chain, which short splits wait on; 2 (8 warps) issue fewer instructions per tile,
+  // which long splits are bound by (measured: 4 win at <= 17 tiles per CTA by up to 20 %, 2 at
+  // 65 and 257 tiles by 5-8 %, even at 33)
+  if (use_tc && (kernel == 0 || kernel == 1)) {
+    const int per = std::max(min_tiles, (n_tiles + a.S - 1) / a.S);
+    tc = per > 32 ? 2 : 4;
+    a.tc = tc;
+  }
 }
 
 // The device's cluster capacity for the attention kernel (occupancy query, cached).
-int attn_device_capacity(bool hilo, int S, int NW, int stages, bool tc) {
-  static int cache[16][9][10][2][4][2];   // [device][S][NW][hilo][stages][tc]; 0 = not yet queried
+int attn_device_capacity(bool hilo, int S, int NW, int stages, int tc) {
+  static int cache[16][9][10][2][4][3];   // [device][S][NW][hilo][stages][tc / 2]; 0 = not yet queried
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 16 || S < 1 || S > 8 || NW < 1 || NW > 9 || stages < 2 ||
-      stages > 3) {
+      stages > 3 || (tc != 0 && tc != 2 && tc != 4)) {
     cudaGetLastError();
     return 1;
   }
   static std::mutex mu;   // the stand-alone attention may be called from several threads
   std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][S][NW][hilo ? 1 : 0][stages][tc ? 1 : 0];
+  int& c = cache[dev][S][NW][hilo ? 1 : 0][stages][tc / 2];
   if (c == 0) c = attn_mma_max_clusters(S, NW, hilo, stages, device_sms(), tc);
   return c;
 }
@@ -663,7 +674,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   aa.quad_k = f.quad_k;
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa,
-              [](int S, int NW, int stages, bool tc) { return attn_device_capacity(true, S, NW, stages, tc); },
+              [](int S, int NW, int stages, int tc) { return attn_device_capacity(true, S, NW, stages, tc); },
               x->attn_rows_cap, x->attn_min_tiles, g_attn_kernel.load());
     const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
     attn_traced = x->attn_trace && ctas * 16 <= x->attn_trace_n;
@@ -1793,7 +1804,8 @@ nld_status nld_debug_layer_trace(nld_ctx* x, int layer, unsigned long long* d_at
 }
 
 nld_status nld_debug_attention_kernel(int kernel) {
-  if (kernel < 0 || kernel > 2) return fail(nullptr, NLD_ERR_ARG, "0 (planner), 1 (tcgen05) or 2 (mma.sync)");
+  if (kernel < 0 || kernel > 4)
+    return fail(nullptr, NLD_ERR_ARG, "0 (planner), 1 (tcgen05), 2 (mma.sync), 3 / 4 (tcgen05, 2 / 4 threads per row)");
   g_attn_kernel.store(kernel);
   return NLD_OK;
 }
@@ -1876,12 +1888,12 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
   AttnArgs a{};
   // pure host: clusters of S resident at once as if every SM held as many CTAs as its 228 KB of
   // shared memory allows (one block reserves 1 KB)
-  attn_plan(batch, m, Hq, Hkv, max_len, sms, a, [sms](int S, int NW, int stages, bool tc) {
-    const size_t smem = tc ? attn_tc_smem_bytes(true) : attn_mma_smem_bytes(NW, true, stages);
+  attn_plan(batch, m, Hq, Hkv, max_len, sms, a, [sms](int S, int NW, int stages, int tc) {
+    const size_t smem = tc ? attn_tc_smem_bytes(true, tc) : attn_mma_smem_bytes(NW, true, stages);
     const int per_sm = static_cast<int>(233472 / (smem + 1024));
     return std::max(1, sms * per_sm / S);
   }, 0, 0, g_attn_kernel.load());
-  const int v[7] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc};
+  const int v[7] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc ? 1 : 0};
   for (int i = 0; i < 7; ++i) out7[i] = v[i];
   return NLD_OK;
 }
@@ -2112,7 +2124,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   }
   AttnArgs a{};
   attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
-            [](int S, int NW, int stages, bool tc) { return attn_device_capacity(false, S, NW, stages, tc); },
+            [](int S, int NW, int stages, int tc) { return attn_device_capacity(false, S, NW, stages, tc); },
             0, 0, g_attn_kernel.load());
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;

@@ -65,6 +65,6 @@ def test_null_arguments_rejected():
     assert lib.nld_diffuse_step_nonlockstep(None, 0.9, None, None, None, None) == 1
     assert lib.nld_plan_chain(1, 1, None, None, None, 1, None) == 1
     assert lib.nld_plan_attention(1, 1, 8, 8, 1, 148, None) == 1
-    assert lib.nld_debug_attention_kernel(3) == 1
+    assert lib.nld_debug_attention_kernel(5) == 1
     assert lib.nld_debug_attention_kernel(-1) == 1
     assert lib.nld_debug_attention_kernel(0) == 0

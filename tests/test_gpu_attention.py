@@ -19,13 +19,13 @@ HQ, HKV, HD = 32, 8, 128
 TOL = 2e-2
 
 
-@pytest.fixture(autouse=True, params=["mma_sync", "tcgen05"])
+@pytest.fixture(autouse=True, params=["mma_sync", "tcgen05_2", "tcgen05_4"])
 def attention_kernel(request):
-    """Every case runs on both tensor-core attention kernels (the process-wide switch is put
-    back to the default afterwards)."""
+    """Every case runs on each tensor-core attention kernel: mma.sync, and tcgen05 with 2 or 4
+    softmax threads per row (the process-wide switch is put back to the default afterwards)."""
     import self_speculation_b200 as nb
     lib = nb.load_library()
-    assert lib.nld_debug_attention_kernel(1 if request.param == "tcgen05" else 2) == 0
+    assert lib.nld_debug_attention_kernel({"mma_sync": 2, "tcgen05_2": 3, "tcgen05_4": 4}[request.param]) == 0
     yield request.param
     assert lib.nld_debug_attention_kernel(0) == 0
 
