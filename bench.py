@@ -464,17 +464,17 @@ def _events_ms(fn, stream, reps, warm=3):
 
 
 def run_attention(args):
-    """Attention micro-workload: 32 q / 8 kv heads x 128, a block of 32 queries per sequence after
-    a cached prefix of 1k/4k/16k/32k, batch 1/8/32, modes block-bidirectional (block 32), strict
-    causal and block size 1.  Q/K/V ~ N(0,1) bf16 (seed 2) in a paged pool.  HBM bytes per call:
-    B*(L+32)*8*128*2*2 (K and V) + 2*B*32*32*128*2 (Q and O)."""
+    """Attention micro-workload: 32 q / 8 kv heads x 128, a block of m = 32 queries per sequence
+    (--attn-m) after a cached prefix of 1k/4k/16k/32k, batch 1/8/32, modes block-bidirectional
+    (block 32), strict causal and block size 1.  Q/K/V ~ N(0,1) bf16 (seed 2) in a paged pool.
+    HBM bytes per call: B*(L+m)*8*128*2*2 (K and V) + 2*B*m*32*128*2 (Q and O)."""
     import torch
 
     import self_speculation_b200 as nb
     from self_speculation_b200 import build as nbuild
     nbuild.build()
     hbm, peak_src = peaks()
-    Hq, Hkv, hd, m = 32, 8, 128, 32
+    Hq, Hkv, hd, m = 32, 8, 128, args.attn_m
     stream = torch.cuda.current_stream()
     points = []
     grid = [(L, B) for L in (1024, 4096, 16384, 32768) for B in (1, 8, 32)]
@@ -506,7 +506,7 @@ def run_attention(args):
         "metric": "attention HBM throughput (block-causal GQA over paged bf16 KV)",
         "value": best["GB/s"], "unit": "GB/s", "n_gpus": 1, "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "attention micro-workload: 32q/8kv x 128, 32 queries per sequence",
+        "config": {"workload": f"attention micro-workload: 32q/8kv x 128, {m} queries per sequence",
                    "l2": "not flushed: points under 126 MB are marked l2_resident"},
         "roofline": {"bound": "hbm", "achieved": best["GB/s"], "peak": hbm, "unit": "GB/s",
                      "frac": best["frac"], "traffic": None, "peak_kind": f"{peak_src} HBM copy"},
@@ -800,6 +800,8 @@ def main():
     ap.add_argument("--workload", choices=["selfspec8b", "attention", "diffusion8b", "sweep14b",
                                            "commit8b"],
                     default="selfspec8b")
+    ap.add_argument("--attn-m", type=int, default=32,
+                    help="queries per sequence of the attention workload (32; 1 = single-token decode)")
     ap.add_argument("--attn-point", default="",
                     help="attention workload: one point 'prefix,batch' instead of the whole grid")
     ap.add_argument("--probe", action="store_true",
