@@ -528,24 +528,25 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 
 // ------------------------------------------------------------------ tcgen05 attention --
 // The same attention on the 5th-generation tensor cores, for query tiles of <= 128 rows: one
-// CTA per (KV split, kv head, sequence x query tile), TMEM lane r = query row r.  Per KV tile of
-// 64 keys, S = Q K^T (M 128, N 64, K 128) goes to one of two TMEM S buffers, issued two tiles
-// ahead of the softmax.  Sixteen softmax warps take four threads per row, one per 16-key quarter
-// of each tile (warps w, w+4, w+8, w+12 share TMEM lane quarter w % 4 and an SM sub-partition):
-// a thread reads its 16 scores, the four threads of a row exchange their maxima through shared
-// memory (an mbarrier per lane quarter and tile parity), and each writes P as packed bf16 pairs
-// (with hi/lo: its lo half too) into TMEM.  O += P V (M 128, N 128, K 64) takes P from TMEM as
-// the A operand and V straight from the TMA tile as an MN-major operand.  A row's reference max
-// moves only when a tile's max exceeds it by more than 2^8 (so P <= 256), which rescales its O
-// row in TMEM (each thread its 32 columns).  Splits merge over the cluster as in
-// attn_mma_kernel.  One thread loads K/V by TMA into a 4-stage (bf16 Q: 5-stage) ring, another
-// issues the MMAs; P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.
-// TMEM columns: S buffers 0..127, O 128..255, P buffers 384..511 (per buffer: 32 columns of hi
-// pairs, then 32 of lo pairs; key quarter q at 8q).
+// CTA per (KV split, kv head, sequence x query tile), TMEM lane r = query row r.  The query tile
+// sits in TMEM (packed bf16 pairs, with hi/lo both halves) as the A operand of S = Q K^T (M 128,
+// N 64, K 128), which goes per KV tile of 64 keys to one of two TMEM S buffers, issued two tiles
+// ahead of the softmax.  kRT softmax threads per row (2: 8 warps, 4: 16 warps; warps w, w+4, ...
+// share TMEM lane quarter w % 4 and an SM sub-partition), one per 64/kRT-key part of each tile:
+// a thread reads its scores, the threads of a row exchange their maxima through shared memory
+// (an mbarrier per lane quarter and tile parity), and each writes P as packed bf16 pairs (with
+// hi/lo: its lo half too) into TMEM.  O += P V (M 128, N 128, K 64) takes P from TMEM as the A
+// operand and V straight from the TMA tile as an MN-major operand.  A row's reference max moves
+// only when a tile's max exceeds it by more than 2^8 (so P <= 256), which rescales its O row in
+// TMEM (each thread 128/kRT columns).  Splits merge over the cluster as in attn_mma_kernel.  One
+// thread loads K/V by TMA into a 6-stage ring (shared memory holds only the ring), another issues
+// the MMAs; P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.  TMEM
+// columns: S buffers 0..127, O 128..255, Q 256..383 (hi pairs, then lo pairs), P buffers
+// 384..511 (per buffer: 32 columns of hi pairs, then 32 of lo pairs; key part q at q 32/kRT).
 // kRT softmax threads per row (2 or 4): 128 kRT softmax threads, + the MMA warp + the TMA warp
 __host__ __device__ constexpr int tc_threads(int rt) { return 128 * rt + 64; }
-constexpr int kTcMaxStages = 5;
-__host__ __device__ constexpr int tc_stages(bool hilo) { return hilo ? 4 : 5; }
+constexpr int kTcMaxStages = 6;
+__host__ __device__ constexpr int tc_stages(bool) { return 6; }
 // S of tile j + 2 is issued before O += P V of tile j, so its K/V stage must not wait for that
 static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
@@ -605,8 +606,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kQ = kHiLo ? 2 : 1;                // operand halves (hi, lo)
   constexpr int NS = tc_stages(kHiLo);
-  uint8_t* sQ = smem;                              // [kQ][2 dim boxes][128 rows][128 B]
-  uint8_t* sK = sQ + kQ * 32768;                   // [NS][2 dim boxes][64 keys][128 B]
+  uint8_t* sK = smem;                              // [NS][2 dim boxes][64 keys][128 B]
   uint8_t* sV = sK + NS * kKVTile;                 // same
   float* xmax = reinterpret_cast<float*>(sV + NS * kKVTile);   // [2][kRT][128] row maxima
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile + tc_xchg_bytes(kRT));
@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     tma_prefetch_desc(&tmKV);
   }
   if (warp == kTcSoftmax / 32) {
-    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O: 128..255, P: 384..511
+    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O: 128..255, Q: 256..383, P: 384..511
     tmem_relinquish();
   }
   tc_fence_before();
@@ -711,40 +711,48 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   const int r = tid & 127;            // and query row (position r / G, head r % G)
   const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
-  // query rows -> shared memory, coalesced: piece e = tid + 128 kRT u of the tile's 128 rows x 16
-  // pieces of 8 dims (row e / 16, piece c = e % 16) goes to box c / 8 at piece (c % 8) ^ (row % 8);
-  // padding rows are zero
-  constexpr int kQPer = 2048 / kTcSoftmax;
+  // query rows -> TMEM, the A operand of S = Q K^T: thread (kq, r) writes dims kq kOC .. of row r
+  // as packed bf16 pairs at columns 256 + d / 2 (hi) and 320 + d / 2 (lo); padding rows are zero
   if (softmax_thr) {
-    uint4 hv[kQPer], lv[kQPer];
-    int offs[kQPer];
+    const uint32_t lane_q = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int gh = r - prow * a.G;
+    const size_t tok = static_cast<size_t>(b) * a.m + p0 + (row_ok ? prow : 0);
+    const size_t qoff = ((tok * a.Hq) + g * a.G + gh) * 128 + kq * kOC;
 #pragma unroll
-    for (int u = 0; u < kQPer; ++u) {
-      const int e = tid + u * kTcSoftmax;
-      const int row = e >> 4, c = e & 15;
-      const int p = row / a.G, gh = row - p * a.G;
-      offs[u] = (c >> 3) * 16384 + row * 128 + (((c & 7) ^ (row & 7)) << 4);
-      hv[u] = lv[u] = make_uint4(0, 0, 0, 0);
-      if (row < a.rows && p < np) {
-        const size_t tok = static_cast<size_t>(b) * a.m + p0 + p;
-        const size_t qoff = ((tok * a.Hq) + g * a.G + gh) * 128 + c * 8;
-        if constexpr (kHiLo) {
-          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + qoff);
-          const float4 x0 = src[0], x1 = src[1];
-          const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-          split8(xs, hv[u], lv[u]);
-        } else {
-          hv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qoff);
+    for (int cc = 0; cc < kOC / 32; ++cc) {
+      uint4 hv[4], lv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        hv[u] = lv[u] = make_uint4(0, 0, 0, 0);
+        if (row_ok) {
+          if constexpr (kHiLo) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + qoff + cc * 32 + u * 8);
+            const float4 x0 = src[0], x1 = src[1];
+            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            split8(xs, hv[u], lv[u]);
+          } else {
+            hv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qoff + cc * 32 + u * 8);
+          }
         }
       }
-    }
+      float hw[16], lw[16];
 #pragma unroll
-    for (int u = 0; u < kQPer; ++u) {
-      *reinterpret_cast<uint4*>(sQ + offs[u]) = hv[u];
-      if constexpr (kHiLo) *reinterpret_cast<uint4*>(sQ + 32768 + offs[u]) = lv[u];
+      for (int u = 0; u < 4; ++u) {
+        hw[4 * u] = __uint_as_float(hv[u].x);
+        hw[4 * u + 1] = __uint_as_float(hv[u].y);
+        hw[4 * u + 2] = __uint_as_float(hv[u].z);
+        hw[4 * u + 3] = __uint_as_float(hv[u].w);
+        lw[4 * u] = __uint_as_float(lv[u].x);
+        lw[4 * u + 1] = __uint_as_float(lv[u].y);
+        lw[4 * u + 2] = __uint_as_float(lv[u].z);
+        lw[4 * u + 3] = __uint_as_float(lv[u].w);
+      }
+      tmem_st16(tmem + lane_q + 256 + kq * (kOC / 2) + cc * 16, hw);
+      if constexpr (kHiLo) tmem_st16(tmem + lane_q + 320 + kq * (kOC / 2) + cc * 16, lw);
     }
+    tmem_st_wait();
   }
-  fence_proxy_async();   // the tensor core reads these through the async proxy
+  tc_fence_before();
   __syncthreads();
   stamp(2);
   pdl_launch_dependents();
@@ -797,9 +805,9 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         for (int box = 0; box < 2; ++box)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_f16(tmem + sb * 64, sdesc_k_sw128(smem_u32(sQ + q * 32768 + box * 16384)) + 2 * kk,
-                       sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
-                       (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_f16_ts(tmem + sb * 64, tmem + 256 + q * 64 + (box * 4 + kk) * 8,
+                          sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
+                          (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&s_full[sb]);
       return true;
     };
@@ -1169,12 +1177,11 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
   return 1024 + std::max(ring_q, partials) + kMaxAttStages * sizeof(uint64_t);
 }
 
-// Dynamic shared memory of a tcgen05 attention launch: the query tile (hi and lo halves with
-// hilo), the K and V rings, the row-max exchange and the barriers; the split partials overlay
-// the first two after the KV loop.
+// Dynamic shared memory of a tcgen05 attention launch: the K and V rings (the query tile lives in
+// TMEM), the row-max exchange and the barriers; the split partials overlay the rings after the
+// KV loop.
 size_t attn_tc_smem_bytes(bool hilo, int rt) {
-  const size_t kq = hilo ? 2 : 1;
-  return 1024 + kq * 32768 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + tc_xchg_bytes(rt) + kTcBarBytes;
+  return 1024 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + tc_xchg_bytes(rt) + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
