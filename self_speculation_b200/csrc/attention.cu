@@ -539,8 +539,9 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // operand and V straight from the TMA tile as an MN-major operand.  A row's reference max moves
 // only when a tile's max exceeds it by more than 2^8 (so P <= 256), which rescales its O row in
 // TMEM (each thread 128/kRT columns).  Splits merge over the cluster as in attn_mma_kernel.  One
-// thread loads K/V by TMA into a 6-stage ring (shared memory holds only the ring), another issues
-// the MMAs; P is double-buffered so the softmax of tile j overlaps O += P V of tile j - 1.  TMEM
+// thread issues the S MMAs; another, in another warp, loads K/V by TMA into a 6-stage ring
+// (shared memory holds only the ring) and issues the P V MMAs; P is double-buffered so the
+// softmax of tile j overlaps O += P V of tile j - 1.  TMEM
 // columns: S buffers 0..127, O 128..255, Q 256..383 (hi pairs, then lo pairs), P buffers
 // 384..511 (per buffer: 32 columns of hi pairs, then 32 of lo pairs; key part q at q 32/kRT).
 // kRT softmax threads per row (2 or 4): 128 kRT softmax threads, + the MMA warp + the TMA warp
@@ -618,7 +619,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   uint64_t* s_free = s_full + 2;      // [2] S buffer read (the softmax warps)
   uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (the softmax warps)
   uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
-  uint64_t* fin = s_full + 8;         // the MMA thread's outstanding MMAs on an early exit
+  uint64_t* fin = s_full + 8;         // every MMA of both issuing threads completed
   uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (kRT warps)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 17);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 18);
@@ -650,7 +651,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       mbar_init(&p_full[i], kTcSoftmax / 32);
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(fin, 1);
+    mbar_init(fin, 2);   // both issuing threads commit once
     for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], kRT);
     *s_abort = 0;
     fence_mbar_init();
@@ -759,74 +760,80 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
 
   float m_ref = -INFINITY, l_sum = 0.f;
   bool aborted = false;
+  // Two issuing threads, in different warps (SM sub-partitions): the MMA thread issues S = Q K^T,
+  // the TMA thread loads K/V and issues O += P V.  Their MMAs touch different TMEM (S buffers /
+  // O) and each commits only its own, so they need no ordering between them; splitting the
+  // issue halves the per-tile issue time of the one thread that used to issue both.
+  const uint32_t idS = idesc_bf16_f32(128, 64);
+  const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
+  // O += P V of tile i (P buffer i & 1, K/V stage i % NS); the stage frees when it completes
+  auto pv_step = [&](int i) -> bool {
+    const int pb = i & 1, st = i % NS;
+    if (*s_abort || !mbar_wait(&p_full[pb], static_cast<uint32_t>(i >> 1) & 1u, kWait)) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int q = 0; q < kQ; ++q)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)   // 16-key step of the tile: 8 TMEM columns of P
+        tc_mma_f16_ts(tmem + 128, tmem + 384 + pb * 64 + q * 32 + ks * 8,
+                      sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
+                      (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
+    tc_commit(&pv_done[pb]);
+    tc_commit(&empty[st]);
+    return true;
+  };
+  // S of tile j into S buffer j & 1 (free once the softmax read S of tile j - 2)
+  auto s_step = [&](int j) -> bool {
+    const int st = j % NS, sb = j & 1;
+    if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
+        (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
+      return false;
+    tc_fence_after();
+#pragma unroll
+    for (int q = 0; q < kQ; ++q)
+#pragma unroll
+      for (int box = 0; box < 2; ++box)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_f16_ts(tmem + sb * 64, tmem + 256 + q * 64 + (box * 4 + kk) * 8,
+                        sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
+                        (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
+    tc_commit(&s_full[sb]);
+    return true;
+  };
   if (tma_thr) {
-    // ------------------------------------------------------------------ TMA thread --
-    // tile i reuses the stage of tile i - NS once that tile's P V MMAs have completed
-    for (int i = NS; i < ntile; ++i) {
-      if (*s_abort || !mbar_wait(&empty[i % NS], static_cast<uint32_t>(i / NS - 1) & 1u, kWait)) {
-        aborted = true;
-        break;
-      }
-      issue(i);
-    }
-    if (aborted) {
-      *s_abort = 1;
-      set_err(a.err, NLD_DEVERR_TIMEOUT);
-    }
-  } else if (mma_thr) {
-    // ------------------------------------------------------------------ MMA thread --
-    const uint32_t idS = idesc_bf16_f32(128, 64);
-    const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
-    auto pv_step = [&](int i) -> bool {
-      const int pb = i & 1, st = i % NS;
-      if (!mbar_wait(&p_full[pb], static_cast<uint32_t>(i >> 1) & 1u, kWait)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < kQ; ++q)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)   // 16-key step of the tile: 8 TMEM columns of P
-          tc_mma_f16_ts(tmem + 128, tmem + 384 + pb * 64 + q * 32 + ks * 8,
-                        sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
-                        (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
-      tc_commit(&pv_done[pb]);
-      tc_commit(&empty[st]);
-      return true;
-    };
-    // S of tile j into S buffer j & 1 (free once the softmax read S of tile j - 2)
-    auto s_step = [&](int j) -> bool {
-      const int st = j % NS, sb = j & 1;
-      if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
-          (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
-        return false;
-      tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < kQ; ++q)
-#pragma unroll
-        for (int box = 0; box < 2; ++box)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_f16_ts(tmem + sb * 64, tmem + 256 + q * 64 + (box * 4 + kk) * 8,
-                          sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
-                          (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(&s_full[sb]);
-      return true;
-    };
-    // S runs two tiles ahead of the softmax: S of tile j + 2 goes as soon as the softmax has
-    // read S of tile j, before O += P V of tile j
-    for (int j = 0; j < min(2, ntile) && !aborted; ++j)
-      if (!s_step(j)) aborted = true;
+    // --------------------------------------------------------- TMA + P V thread --
+    // O += P V of tile j as soon as its P is written; then tile j + NS reuses tile j's stage
+    // once those MMAs have completed
     for (int j = 0; j < ntile && !aborted; ++j) {
-      if (j + 2 < ntile && !s_step(j + 2)) {
+      if (!pv_step(j)) {
         aborted = true;
         break;
       }
-      if (!pv_step(j)) aborted = true;
+      if (j + NS < ntile) {
+        if (!mbar_wait(&empty[j % NS], static_cast<uint32_t>(j / NS) & 1u, kWait)) {
+          aborted = true;
+          break;
+        }
+        issue(j + NS);
+      }
     }
     if (aborted) {
       *s_abort = 1;
       set_err(a.err, NLD_DEVERR_TIMEOUT);
     }
     // every MMA this thread issued has completed before the tensor memory is released
+    tc_commit(fin);
+    mbar_wait(fin, 0, kWait);
+  } else if (mma_thr) {
+    // ---------------------------------------------------------------- S thread --
+    // S runs up to two tiles ahead of the softmax
+    for (int j = 0; j < ntile && !aborted; ++j)
+      if (!s_step(j)) aborted = true;
+    if (aborted) {
+      *s_abort = 1;
+      set_err(a.err, NLD_DEVERR_TIMEOUT);
+    }
     tc_commit(fin);
     mbar_wait(fin, 0, kWait);
   } else if (softmax_thr) {
