@@ -546,9 +546,11 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // 384..511 (per buffer: 32 columns of hi pairs, then 32 of lo pairs; key part q at q 32/kRT).
 // kRT softmax threads per row (2 or 4): 128 kRT softmax threads, + the MMA warp + the TMA warp
 __host__ __device__ constexpr int tc_threads(int rt) { return 128 * rt + 64; }
-constexpr int kTcMaxStages = 6;
-__host__ __device__ constexpr int tc_stages(bool) { return 6; }
-// S of tile j + 2 is issued before O += P V of tile j, so its K/V stage must not wait for that
+constexpr int kTcMaxStages = 3;
+constexpr int kTcTile = 128;                     // keys per KV tile (two pages): S has N = 128
+constexpr int kTcStage = 2 * kKVTile;           // 32 KB: K (or V) of one tile
+__host__ __device__ constexpr int tc_stages(bool) { return 3; }
+// S of tile j + 2 may be issued while tile j's stage is held: three stages at least
 static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
 constexpr int kTcBarBytes = 256;
@@ -600,25 +602,25 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   static_assert(kRT == 2 || kRT == 4, "2 or 4 softmax threads per row");
   constexpr int kTcSoftmax = 128 * kRT;
   constexpr int kTcThreads = tc_threads(kRT);
-  constexpr int kKT = 64 / kRT;    // keys of a tile per softmax thread
+  constexpr int kKT = kTcTile / kRT;   // keys of a tile per softmax thread
   constexpr int kOC = 128 / kRT;   // O columns per softmax thread in the rescale and the combine
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kQ = kHiLo ? 2 : 1;                // operand halves (hi, lo)
   constexpr int NS = tc_stages(kHiLo);
-  uint8_t* sK = smem;                              // [NS][2 dim boxes][64 keys][128 B]
-  uint8_t* sV = sK + NS * kKVTile;                 // same
-  float* xmax = reinterpret_cast<float*>(sV + NS * kKVTile);   // [2][kRT][128] row maxima
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kKVTile + tc_xchg_bytes(kRT));
+  // a stage per tile: [2 dim boxes][128 keys (page 0 rows, then page 1 rows)][128 B]
+  uint8_t* sK = smem;                              // [NS] stages
+  uint8_t* sV = sK + NS * kTcStage;                // same
+  float* xmax = reinterpret_cast<float*>(sV + NS * kTcStage);   // [2][kRT][128] row maxima
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kTcStage + tc_xchg_bytes(kRT));
   uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
   uint64_t* empty = bars + kTcMaxStages;   // [NS] K/V stage free (the tile's P V MMAs completed)
   uint64_t* s_full = bars + 2 * kTcMaxStages;   // [2] S buffer written (MMA commit)
   // the softmax warps arrive on their barriers once per warp (lane 0, after the warp's threads
   // synchronise): one arrival per thread would queue 512 arrivals per barrier and tile
-  uint64_t* s_free = s_full + 2;      // [2] S buffer read (the softmax warps)
-  uint64_t* p_full = s_full + 4;      // [2] P buffer written into TMEM (the softmax warps)
-  uint64_t* pv_done = s_full + 6;     // [2] O += P V of the P buffer completed (MMA commit)
+  uint64_t* p_full = s_full + 4;      // [2] P written over S in the S buffer (the softmax warps)
+  uint64_t* pv_done = s_full + 6;     // [2] O += P V from the S buffer completed (MMA commit)
   uint64_t* fin = s_full + 8;         // every MMA of both issuing threads completed
   uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (kRT warps)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 17);
@@ -647,7 +649,6 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kTcSoftmax / 32);
       mbar_init(&p_full[i], kTcSoftmax / 32);
       mbar_init(&pv_done[i], 1);
     }
@@ -658,7 +659,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     tma_prefetch_desc(&tmKV);
   }
   if (warp == kTcSoftmax / 32) {
-    tmem_alloc(s_tmem, 512);   // S: columns 0..127, O: 128..255, Q: 256..383, P: 384..511
+    tmem_alloc(s_tmem, 512);   // S / P: columns 0..255, O: 256..383, Q: 384..511
     tmem_relinquish();
   }
   tc_fence_before();
@@ -680,8 +681,10 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     row_keys(len, p0 + np - 1, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
     kv_end = max(v1, h2) + 1;
   }
-  const int n_tiles = (kv_end + kPage - 1) / kPage;
-  const int per = max(a.min_tiles, (n_tiles + a.S - 1) / a.S);
+  // tiles of 128 keys (pages 2t, 2t + 1); the split plan counts pages (min_tiles)
+  const int n_pages = (kv_end + kPage - 1) / kPage;
+  const int n_tiles = (n_pages + 1) / 2;
+  const int per = max((a.min_tiles + 1) / 2, (n_tiles + a.S - 1) / a.S);
   const int t_lo = split * per;
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
 
@@ -689,20 +692,27 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   auto issue = [&](int i) {
     ++n_issued;
     const int stage = i % NS;
-    const int kt = t_lo + i;
-    const int page = a.page_table[b * a.pps + kt];
-    const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
-    const int row0v = row0 + a.Hkv * kPage;
-    mbar_arrive_expect_tx(&full[stage], 2 * kKVTile);
-    tma_load_2d(sK + stage * kKVTile, &tmKV, &full[stage], 0, row0);
-    tma_load_2d(sK + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0);
-    tma_load_2d(sV + stage * kKVTile, &tmKV, &full[stage], 0, row0v);
-    tma_load_2d(sV + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0v);
+    const int kt = 2 * (t_lo + i);
+    // a tile's second page past the keys reads the first page again: its keys are masked, and
+    // its V rows, multiplied by P = 0, must be finite
+    const int pg0 = a.page_table[b * a.pps + kt];
+    const int pg1 = a.page_table[b * a.pps + (kt + 1 < n_pages ? kt + 1 : kt)];
+    mbar_arrive_expect_tx(&full[stage], 2 * kTcStage);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row0 = a.layer_row0 + (((h ? pg1 : pg0) * 2) * a.Hkv + g) * kPage;
+      const int row0v = row0 + a.Hkv * kPage;
+#pragma unroll
+      for (int box = 0; box < 2; ++box) {
+        tma_load_2d(sK + stage * kTcStage + box * kKVTile + h * kHalfTile, &tmKV, &full[stage], box * 64, row0);
+        tma_load_2d(sV + stage * kTcStage + box * kKVTile + h * kHalfTile, &tmKV, &full[stage], box * 64, row0v);
+      }
+    }
   };
   // the K/V tiles wholly in the cached prefix are requested before the dependency wait
   int n_pre = 0;
   if (tma_thr)
-    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
+    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kTcTile <= len; ++n_pre) issue(n_pre);
   pdl_wait();
   stamp(1);
   if (tma_thr)
@@ -713,7 +723,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
   // query rows -> TMEM, the A operand of S = Q K^T: thread (kq, r) writes dims kq kOC .. of row r
-  // as packed bf16 pairs at columns 256 + d / 2 (hi) and 320 + d / 2 (lo); padding rows are zero
+  // as packed bf16 pairs at columns 384 + d / 2 (hi) and 448 + d / 2 (lo); padding rows are zero
   if (softmax_thr) {
     const uint32_t lane_q = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int gh = r - prow * a.G;
@@ -748,8 +758,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         lw[4 * u + 2] = __uint_as_float(lv[u].z);
         lw[4 * u + 3] = __uint_as_float(lv[u].w);
       }
-      tmem_st16(tmem + lane_q + 256 + kq * (kOC / 2) + cc * 16, hw);
-      if constexpr (kHiLo) tmem_st16(tmem + lane_q + 320 + kq * (kOC / 2) + cc * 16, lw);
+      tmem_st16(tmem + lane_q + 384 + kq * (kOC / 2) + cc * 16, hw);
+      if constexpr (kHiLo) tmem_st16(tmem + lane_q + 448 + kq * (kOC / 2) + cc * 16, lw);
     }
     tmem_st_wait();
   }
@@ -764,9 +774,11 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   // the TMA thread loads K/V and issues O += P V.  Their MMAs touch different TMEM (S buffers /
   // O) and each commits only its own, so they need no ordering between them; splitting the
   // issue halves the per-tile issue time of the one thread that used to issue both.
-  const uint32_t idS = idesc_bf16_f32(128, 64);
+  const uint32_t idS = idesc_bf16_f32(128, kTcTile);
   const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
-  // O += P V of tile i (P buffer i & 1, K/V stage i % NS); the stage frees when it completes
+  // O += P V of tile i (P over S in S buffer i & 1, K/V stage i % NS); the stage frees when it
+  // completes.  P of key part kq (keys kKT kq ..) sits in that part's S columns: kKT / 2 columns
+  // of hi pairs, then kKT / 2 of lo pairs
   auto pv_step = [&](int i) -> bool {
     const int pb = i & 1, st = i % NS;
     if (*s_abort || !mbar_wait(&p_full[pb], static_cast<uint32_t>(i >> 1) & 1u, kWait)) return false;
@@ -774,19 +786,22 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
 #pragma unroll
     for (int q = 0; q < kQ; ++q)
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)   // 16-key step of the tile: 8 TMEM columns of P
-        tc_mma_f16_ts(tmem + 128, tmem + 384 + pb * 64 + q * 32 + ks * 8,
-                      sdesc_mn_sw128(smem_u32(sV + st * kKVTile + ks * 2048), kHalfTile, 1024), idO,
-                      (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < kTcTile / 16; ++ks) {   // 16-key step: page ks / 4, rows 16 (ks % 4) ..
+        const int part = ks / (kKT / 16), u = ks % (kKT / 16);
+        tc_mma_f16_ts(tmem + 256, tmem + pb * 128 + part * kKT + q * (kKT / 2) + u * 8,
+                      sdesc_mn_sw128(smem_u32(sV + st * kTcStage + (ks >> 2) * kHalfTile + (ks & 3) * 2048), kKVTile,
+                                     1024),
+                      idO, (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
+      }
     tc_commit(&pv_done[pb]);
     tc_commit(&empty[st]);
     return true;
   };
-  // S of tile j into S buffer j & 1 (free once the softmax read S of tile j - 2)
+  // S of tile j into S buffer j & 1, free once O += P V of tile j - 2 (P over S there) completed
   auto s_step = [&](int j) -> bool {
     const int st = j % NS, sb = j & 1;
     if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
-        (j >= 2 && !mbar_wait(&s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
+        (j >= 2 && !mbar_wait(&pv_done[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
       return false;
     tc_fence_after();
 #pragma unroll
@@ -795,8 +810,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       for (int box = 0; box < 2; ++box)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_f16_ts(tmem + sb * 64, tmem + 256 + q * 64 + (box * 4 + kk) * 8,
-                        sdesc_k_sw128(smem_u32(sK + st * kKVTile + box * kHalfTile)) + 2 * kk, idS,
+          tc_mma_f16_ts(tmem + sb * 128, tmem + 384 + q * 64 + (box * 4 + kk) * 8,
+                        sdesc_k_sw128(smem_u32(sK + st * kTcStage + box * kKVTile)) + 2 * kk, idS,
                         (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
     tc_commit(&s_full[sb]);
     return true;
@@ -842,7 +857,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     if (row_ok) row_keys(len, p0 + prow, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
     const int lq = warp & 3;   // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(lq * 32) << 16;
-    const uint32_t o_col = 128 + kq * kOC;   // this thread's columns of O
+    const uint32_t o_col = 256 + kq * kOC;   // this thread's columns of O
     const float c = a.scale_log2;
     for (int j = 0; j < ntile; ++j) {
       const int sb = j & 1;
@@ -855,14 +870,11 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       tc_fence_after();
       uint32_t raw[kKT / 16][16];
 #pragma unroll
-      for (int u = 0; u < kKT / 16; ++u) tmem_ld16_nowait(tmem + lane_base + sb * 64 + kq * kKT + u * 16, raw[u]);
+      for (int u = 0; u < kKT / 16; ++u) tmem_ld16_nowait(tmem + lane_base + sb * 128 + kq * kKT + u * 16, raw[u]);
 #pragma unroll
       for (int u = 0; u < kKT / 16; ++u) tmem_ld_wait_regs(raw[u]);
-      tc_fence_before();
-      __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive(&s_free[sb]);
       float sv[kKT];
-      const int k0 = (t_lo + j) * kPage + kq * kKT;
+      const int k0 = (t_lo + j) * kTcTile + kq * kKT;
       if (k0 + kKT - 1 <= v1) {
 #pragma unroll
         for (int k = 0; k < kKT; ++k) sv[k] = __uint_as_float(raw[k >> 4][k & 15]);
@@ -915,11 +927,6 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         l_sum *= alpha;
       }
       if (move) m_ref = mx;
-      // P buffer sb is free once O += P V of tile j - 2 has completed
-      if (!__all_sync(0xffffffffu, j < 2 || mbar_wait(&pv_done[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait))) {
-        aborted = true;
-        break;
-      }
       const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref;
       // P row r, this thread's keys as kKT / 2 bf16 pairs (lower key in the low half), hi then lo
       uint32_t ph[kKT / 16][8], pl[kKT / 16][8];
@@ -936,11 +943,12 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         }
       }
       l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      const uint32_t p_col = 384 + sb * 64 + kq * (kKT / 2);
+      // P over this thread's own S columns (read above): kKT / 2 columns of hi pairs, then lo
+      const uint32_t p_col = sb * 128 + kq * kKT;
 #pragma unroll
       for (int u = 0; u < kKT / 16; ++u) {
         tmem_st8(tmem + lane_base + p_col + u * 8, ph[u]);
-        if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + 32 + u * 8, pl[u]);
+        if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + kKT / 2 + u * 8, pl[u]);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -996,8 +1004,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     for (int cc = 0; cc < kOC / 32; ++cc) {
       uint32_t o[2][16];
       if (have) {
-        tmem_ld16_nowait(tmem + lane_base + 128 + kq * kOC + cc * 32, o[0]);
-        tmem_ld16_nowait(tmem + lane_base + 128 + kq * kOC + cc * 32 + 16, o[1]);
+        tmem_ld16_nowait(tmem + lane_base + 256 + kq * kOC + cc * 32, o[0]);
+        tmem_ld16_nowait(tmem + lane_base + 256 + kq * kOC + cc * 32 + 16, o[1]);
         tmem_ld_wait_regs(o[0]);
         tmem_ld_wait_regs(o[1]);
       } else {
@@ -1188,7 +1196,7 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
 // TMEM), the row-max exchange and the barriers; the split partials overlay the rings after the
 // KV loop.
 size_t attn_tc_smem_bytes(bool hilo, int rt) {
-  return 1024 + 2 * static_cast<size_t>(tc_stages(hilo)) * kKVTile + tc_xchg_bytes(rt) + kTcBarBytes;
+  return 1024 + 2 * static_cast<size_t>(tc_stages(hilo)) * kTcStage + tc_xchg_bytes(rt) + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be

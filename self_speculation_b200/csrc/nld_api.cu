@@ -540,21 +540,24 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // only while the grid is short of two CTAs per SM, keep >= min_tiles KV tiles per split, take
   // no more splits than lets every cluster be resident at once (a second wave doubles the
   // latency), and launch no split that the tiles per split leave empty.
+  // The tcgen05 kernel's KV tiles are 128 keys (two pages): its splits are counted in those.
   const int units = batch * a.q_tiles * Hkv;
+  const int kt = use_tc ? (n_tiles + 1) / 2 : n_tiles;             // KV tiles of the kernel
+  const int min_kt = use_tc ? (min_tiles + 1) / 2 : min_tiles;
   a.S = 1;
   if (units < 2 * sms) {
-    int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, n_tiles / min_tiles)}));
+    int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, kt / min_kt)}));
     while (s_max > 1 && units > cap(s_max, a.NW, a.stages, tc)) --s_max;
-    const int per = std::max(min_tiles, (n_tiles + s_max - 1) / s_max);
-    a.S = std::max(1, (n_tiles + per - 1) / per);
+    const int per = std::max(min_kt, (kt + s_max - 1) / s_max);
+    a.S = std::max(1, (kt + per - 1) / per);
   }
   // tcgen05 softmax threads per row: 4 (16 warps) shorten a CTA's fixed costs and each KV tile's
   // latency chain, which short splits wait on; 2 (8 warps) issue fewer instructions per tile,
-  // which long splits are bound by (measured: 4 win at <= 17 tiles per CTA by up to 20 %, 2 at
-  // 65 and 257 tiles by 5-8 %, even at 33)
+  // which long splits are bound by (measured: 4 win at <= 17 pages per CTA by up to 20 %, 2 at
+  // 65 and 257 pages by 5-8 %, even at 33)
   if (use_tc && (kernel == 0 || kernel == 1)) {
-    const int per = std::max(min_tiles, (n_tiles + a.S - 1) / a.S);
-    tc = per > 32 ? 2 : 4;
+    const int per = std::max(min_kt, (kt + a.S - 1) / a.S);
+    tc = per > 16 ? 2 : 4;
     a.tc = tc;
   }
 }

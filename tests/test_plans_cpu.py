@@ -139,16 +139,17 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
                 if A["tc"]:
                     assert A["rows"] <= 128, where   # one tcgen05 MMA tile
                 assert 1 <= A["S"] <= 8, where
-                assert A["S"] <= -(-max_len // 64), where   # every split has a KV tile
+                # every split has a KV tile (tcgen05: tiles of 128 keys)
+                assert A["S"] <= -(-max_len // (128 if A["tc"] else 64)), where
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
                     assert A["S"] == 1, where
 
 
 def test_attention_plan_of_the_benchmarked_round():
-    # tcgen05 (the planner's choice): verify forward (m = 33: 2 query tiles of 17 positions x 4
-    # heads) and draft forward (m = 32: one 128-row tile); 545 keys = 9 tiles in 5 splits of <= 2
-    # tiles, 865 keys = 14 tiles in 7 splits, 1400 keys = 22 tiles in 8 splits
-    for keys, S in ((545, 5), (865, 7), (1400, 8)):
+    # tcgen05 (the planner's choice, KV tiles of 128 keys): verify forward (m = 33: 2 query tiles
+    # of 17 positions x 4 heads) and draft forward (m = 32: one 128-row tile); 545 keys = 5 tiles
+    # in 5 splits, 865 keys = 7 tiles in 7 splits, 1400 keys = 11 tiles in 6 splits of <= 2
+    for keys, S in ((545, 5), (865, 7), (1400, 6)):
         v = plan_attention(1, 33, 32, 8, keys)
         d = plan_attention(1, 32, 32, 8, keys)
         assert (v["G"], v["QT"], v["q_tiles"], v["rows"], v["S"], v["tc"]) == (4, 17, 2, 68, S, 1)
