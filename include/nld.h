@@ -328,7 +328,7 @@ nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_ti
 /* Profiling hook, process-wide: which kernel serves the tensor-core attention.  0 (the
  * default) = the planner's choice: the tcgen05 kernel (S, P and O in tensor memory, query tiles
  * of <= 128 rows) for query tiles of >= 64 rows with a few sequences, and with many sequences
- * where its query tiles x 64 rows stay below the rows of the mma.sync kernel's tiles (of <= 144
+ * where its query tiles x 56 rows stay below the rows of the mma.sync kernel's tiles (of <= 144
  * rows); the mma.sync kernel otherwise; 1 = tcgen05 always; 2 = mma.sync always; 3 / 4 =
  * tcgen05 always with 2 / 4 softmax threads per row (the planner's choice for 1 and 0).
  * Applies to launches planned afterwards (a context's captured graphs keep their kernel until

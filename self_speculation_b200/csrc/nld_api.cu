@@ -511,17 +511,17 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // Otherwise tiles of up to 144 rows (a 33-position verify block of 4 heads in one 9-warp
   // CTA) read each K/V tile once for as many query rows as possible, through a 3-stage ring.
   // The tcgen05 kernel takes query tiles of up to 128 rows (one MMA tile, in either regime),
-  // and a KV tile costs it about what a 64-row tile costs mma.sync, whatever its rows (mma.sync
+  // and a KV tile costs it about what a 56-row tile costs mma.sync, whatever its rows (mma.sync
   // scales with the rows).  So it serves tiles of >= 64 rows in the latency regime and, with
-  // many sequences, where its query tiles x 64 stay below the rows of mma.sync's tiles of up to
-  // 144 (a 32-position block of 4 heads: 64 < 128; a 33-position one in two tiles: 128 < 132),
+  // many sequences, where its query tiles x 56 stay below the rows of mma.sync's tiles of up to
+  // 144 (a 16-position block of 4 heads: 56 < 64; a 33-position one in two tiles: 112 < 132),
   // unless an explicit tile above 128 rows is asked for.
   const bool latency = batch * Hkv * q_tiles_for(144) * 8 < 2 * sms;
   const int tc_rows = ((m + q_tiles_for(128) - 1) / q_tiles_for(128)) * a.G;
   const int mma_rows = ((m + q_tiles_for(144) - 1) / q_tiles_for(144)) * a.G;
   const bool use_tc = kernel == 1 || kernel >= 3 ||
                       (kernel == 0 && rows_cap <= 128 &&
-                       (latency ? tc_rows >= 64 : q_tiles_for(128) * 64 < q_tiles_for(144) * mma_rows));
+                       (latency ? tc_rows >= 64 : q_tiles_for(128) * 56 < q_tiles_for(144) * mma_rows));
   // softmax threads per row (set below for the planner's choice)
   int tc = !use_tc ? 0 : kernel == 3 ? 2 : 4;
   if (rows_cap <= 0) rows_cap = tc ? 128 : (latency ? 64 : 144);

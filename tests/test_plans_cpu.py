@@ -161,18 +161,20 @@ def test_attention_plan_of_the_benchmarked_round():
         assert (v["G"], v["QT"], v["q_tiles"], v["NW"], v["S"], v["tc"]) == (4, 11, 3, 3, S, 0)
         assert (d["QT"], d["q_tiles"], d["NW"], d["S"], d["tc"]) == (16, 2, 4, S, 0)
     # many sequences: the 33-position verify block of 4 heads in two tcgen05 tiles of 17 and 16
-    # positions (2 x 64 < 132 rows of one 9-warp mma.sync CTA), a 32-position block in one
+    # positions (2 x 56 < 132 rows of one 9-warp mma.sync CTA), a 32-position block in one
     b = plan_attention(64, 33, 32, 8, 4096 + 33)
     assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"]) == (17, 2, 68, 1, 1)
     b = plan_attention(64, 33, 32, 8, 4096 + 33, kernel=2)
     assert (b["QT"], b["q_tiles"], b["NW"], b["S"], b["tc"]) == (33, 1, 9, 1, 0)
     b = plan_attention(64, 32, 32, 8, 4096 + 32)
     assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"]) == (32, 1, 128, 1, 1)
-    # small query tiles (a 4-row single-token decode, 64-row blocks of many sequences) cost the
-    # tcgen05 kernel a whole 128-row tile per KV tile: they stay on mma.sync
+    # small query tiles (a 4-row single-token decode, 32-row blocks of many sequences) cost the
+    # tcgen05 kernel a whole 128-row tile per KV tile: they stay on mma.sync; 64-row blocks go to
+    # tcgen05
     assert plan_attention(1, 1, 32, 8, 4096)["tc"] == 0
     assert plan_attention(64, 1, 32, 8, 4096)["tc"] == 0
-    assert plan_attention(16, 16, 32, 8, 2048)["tc"] == 0
+    assert plan_attention(16, 8, 32, 8, 2048)["tc"] == 0
+    assert plan_attention(16, 16, 32, 8, 2048)["tc"] == 1
     assert plan_attention(1, 16, 32, 8, 2048)["tc"] == 1
 
 
