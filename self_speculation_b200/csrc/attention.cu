@@ -530,28 +530,30 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
 // The same attention on the 5th-generation tensor cores, for query tiles of <= 128 rows: one
 // CTA per (KV split, kv head, sequence x query tile), TMEM lane r = query row r.  The query tile
 // sits in TMEM (packed bf16 pairs, with hi/lo both halves) as the A operand of S = Q K^T (M 128,
-// N 64, K 128), which goes per KV tile of 64 keys to one of two TMEM S buffers, issued two tiles
-// ahead of the softmax.  kRT softmax threads per row (2: 8 warps, 4: 16 warps; warps w, w+4, ...
-// share TMEM lane quarter w % 4 and an SM sub-partition), one per 64/kRT-key part of each tile:
-// a thread reads its scores, the threads of a row exchange their maxima through shared memory
-// (an mbarrier per lane quarter and tile parity), and each writes P as packed bf16 pairs (with
-// hi/lo: its lo half too) into TMEM.  O += P V (M 128, N 128, K 64) takes P from TMEM as the A
-// operand and V straight from the TMA tile as an MN-major operand.  A row's reference max moves
-// only when a tile's max exceeds it by more than 2^8 (so P <= 256), which rescales its O row in
-// TMEM (each thread 128/kRT columns).  Splits merge over the cluster as in attn_mma_kernel.  One
-// thread issues the S MMAs; another, in another warp, loads K/V by TMA into a 6-stage ring
-// (shared memory holds only the ring) and issues the P V MMAs; P is double-buffered so the
-// softmax of tile j overlaps O += P V of tile j - 1.  TMEM
-// columns: S buffers 0..127, O 128..255, Q 256..383 (hi pairs, then lo pairs), P buffers
-// 384..511 (per buffer: 32 columns of hi pairs, then 32 of lo pairs; key part q at q 32/kRT).
+// N = kTile, K 128), which goes per KV tile of kTile = 64 or 128 keys (one or two pages) to one
+// of two TMEM S buffers, issued up to two tiles ahead of the softmax.  kRT softmax threads per
+// row (2: 8 warps, 4: 16 warps; warps w, w+4, ... share TMEM lane quarter w % 4 and an SM
+// sub-partition), one per kTile/kRT-key part of each tile: a thread reads its scores, the
+// threads of a row exchange their maxima through shared memory (an mbarrier per lane quarter
+// and tile parity), and each writes P as packed bf16 pairs (with hi/lo: its lo half too) into
+// TMEM.  O += P V (M 128, N 128, K kTile) takes P from TMEM as the A operand and V straight from
+// the TMA tile as an MN-major operand.  A row's reference max moves only when a tile's max
+// exceeds it by more than 2^8 (so P <= 256), which rescales its O row in TMEM (each thread
+// 128/kRT columns).  Splits merge over the cluster as in attn_mma_kernel.  One thread issues
+// the S MMAs; another, in another warp, loads K/V by TMA into a 192 KB ring (shared memory holds
+// only the ring) and issues the P V MMAs.  TMEM columns: S buffers [0, 2 kTile), O, Q (hi pairs,
+// then lo pairs); with 64-key tiles two P buffers of their own after Q, with 128-key tiles P
+// over S in its buffer.
 // kRT softmax threads per row (2 or 4): 128 kRT softmax threads, + the MMA warp + the TMA warp
 __host__ __device__ constexpr int tc_threads(int rt) { return 128 * rt + 64; }
-constexpr int kTcMaxStages = 3;
-constexpr int kTcTile = 128;                     // keys per KV tile (two pages): S has N = 128
-constexpr int kTcStage = 2 * kKVTile;           // 32 KB: K (or V) of one tile
-__host__ __device__ constexpr int tc_stages(bool) { return 3; }
+// KV tiles of kTile = 64 keys (one page) or 128 (two pages: S with N = 128, half the S MMAs
+// per key); a ring stage holds K (and one V) of a tile, [2 dim boxes][kTile keys][128 B]; the
+// ring takes 192 KB either way
+constexpr int kTcMaxStages = 6;
+__host__ __device__ constexpr int tc_stage_bytes(int tile) { return tile * 256; }
+__host__ __device__ constexpr int tc_stages(int tile) { return tile == 64 ? 6 : 3; }
 // S of tile j + 2 may be issued while tile j's stage is held: three stages at least
-static_assert(tc_stages(true) >= 3 && tc_stages(false) >= 3 && tc_stages(false) <= kTcMaxStages, "ring depth");
+static_assert(tc_stages(64) >= 3 && tc_stages(128) >= 3 && tc_stages(64) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
 constexpr int kTcBarBytes = 256;
 // row-max exchange: [tile parity][key part][row] floats
@@ -596,30 +598,42 @@ NLD_DEV uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return d;
 }
 
-template <bool kHiLo, int kRT>
+template <bool kHiLo, int kRT, int kTile>
 __global__ void __launch_bounds__(tc_threads(kRT), 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const AttnArgs a) {
   static_assert(kRT == 2 || kRT == 4, "2 or 4 softmax threads per row");
+  static_assert(kTile == 64 || kTile == 128, "KV tiles of one or two pages");
+  constexpr int kPg = kTile / kPage;              // pages per tile
+  constexpr int kStage = tc_stage_bytes(kTile);   // K (or V) of one tile
+  constexpr int kBox = kStage / 2;                // one 64-dim box of a tile: kTile rows x 128 B
+  // TMEM columns: S buffers [0, 2 kTile) (P over S), O [2 kTile, 2 kTile + 128), Q after O
+  constexpr uint32_t kOCol = 2 * kTile, kQCol = 2 * kTile + 128;
+  // 128-key tiles write P over S (TMEM is full); 64-key tiles keep two P buffers of their own
+  // after Q (columns 384..511: per buffer 32 columns of hi pairs, then 32 of lo pairs), so S of
+  // tile j + 2 only waits for the softmax to have read S of tile j
+  constexpr bool kAlias = kTile == 128;
+  constexpr uint32_t kPCol = 2 * kTile + 256;
   constexpr int kTcSoftmax = 128 * kRT;
   constexpr int kTcThreads = tc_threads(kRT);
-  constexpr int kKT = kTcTile / kRT;   // keys of a tile per softmax thread
+  constexpr int kKT = kTile / kRT;   // keys of a tile per softmax thread
   constexpr int kOC = 128 / kRT;   // O columns per softmax thread in the rescale and the combine
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kQ = kHiLo ? 2 : 1;                // operand halves (hi, lo)
-  constexpr int NS = tc_stages(kHiLo);
+  constexpr int NS = tc_stages(kTile);
   // a stage per tile: [2 dim boxes][128 keys (page 0 rows, then page 1 rows)][128 B]
   uint8_t* sK = smem;                              // [NS] stages
-  uint8_t* sV = sK + NS * kTcStage;                // same
-  float* xmax = reinterpret_cast<float*>(sV + NS * kTcStage);   // [2][kRT][128] row maxima
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kTcStage + tc_xchg_bytes(kRT));
+  uint8_t* sV = sK + NS * kStage;                  // same
+  float* xmax = reinterpret_cast<float*>(sV + NS * kStage);   // [2][kRT][128] row maxima
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * kStage + tc_xchg_bytes(kRT));
   uint64_t* full = bars;              // [NS] K/V tile landed (TMA transaction bytes)
   uint64_t* empty = bars + kTcMaxStages;   // [NS] K/V stage free (the tile's P V MMAs completed)
   uint64_t* s_full = bars + 2 * kTcMaxStages;   // [2] S buffer written (MMA commit)
   // the softmax warps arrive on their barriers once per warp (lane 0, after the warp's threads
   // synchronise): one arrival per thread would queue 512 arrivals per barrier and tile
-  uint64_t* p_full = s_full + 4;      // [2] P written over S in the S buffer (the softmax warps)
+  uint64_t* s_free = s_full + 2;      // [2] S buffer read (the softmax warps; 64-key tiles)
+  uint64_t* p_full = s_full + 4;      // [2] P written (the softmax warps)
   uint64_t* pv_done = s_full + 6;     // [2] O += P V from the S buffer completed (MMA commit)
   uint64_t* fin = s_full + 8;         // every MMA of both issuing threads completed
   uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (kRT warps)
@@ -649,6 +663,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kTcSoftmax / 32);
       mbar_init(&p_full[i], kTcSoftmax / 32);
       mbar_init(&pv_done[i], 1);
     }
@@ -659,7 +674,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     tma_prefetch_desc(&tmKV);
   }
   if (warp == kTcSoftmax / 32) {
-    tmem_alloc(s_tmem, 512);   // S / P: columns 0..255, O: 256..383, Q: 384..511
+    tmem_alloc(s_tmem, 512);   // S / P, O, Q (kOCol, kQCol)
     tmem_relinquish();
   }
   tc_fence_before();
@@ -681,10 +696,10 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     row_keys(len, p0 + np - 1, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
     kv_end = max(v1, h2) + 1;
   }
-  // tiles of 128 keys (pages 2t, 2t + 1); the split plan counts pages (min_tiles)
+  // tiles of kTile keys (pages kPg t ..); the split plan's min_tiles counts pages
   const int n_pages = (kv_end + kPage - 1) / kPage;
-  const int n_tiles = (n_pages + 1) / 2;
-  const int per = max((a.min_tiles + 1) / 2, (n_tiles + a.S - 1) / a.S);
+  const int n_tiles = (n_pages + kPg - 1) / kPg;
+  const int per = max((a.min_tiles + kPg - 1) / kPg, (n_tiles + a.S - 1) / a.S);
   const int t_lo = split * per;
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
 
@@ -692,27 +707,26 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   auto issue = [&](int i) {
     ++n_issued;
     const int stage = i % NS;
-    const int kt = 2 * (t_lo + i);
-    // a tile's second page past the keys reads the first page again: its keys are masked, and
-    // its V rows, multiplied by P = 0, must be finite
-    const int pg0 = a.page_table[b * a.pps + kt];
-    const int pg1 = a.page_table[b * a.pps + (kt + 1 < n_pages ? kt + 1 : kt)];
-    mbar_arrive_expect_tx(&full[stage], 2 * kTcStage);
+    const int kt = kPg * (t_lo + i);
+    mbar_arrive_expect_tx(&full[stage], 2 * kStage);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row0 = a.layer_row0 + (((h ? pg1 : pg0) * 2) * a.Hkv + g) * kPage;
+    for (int h = 0; h < kPg; ++h) {
+      // a tile's second page past the keys reads the first page again: its keys are masked, and
+      // its V rows, multiplied by P = 0, must be finite
+      const int page = a.page_table[b * a.pps + (kt + h < n_pages ? kt + h : kt)];
+      const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
       const int row0v = row0 + a.Hkv * kPage;
 #pragma unroll
       for (int box = 0; box < 2; ++box) {
-        tma_load_2d(sK + stage * kTcStage + box * kKVTile + h * kHalfTile, &tmKV, &full[stage], box * 64, row0);
-        tma_load_2d(sV + stage * kTcStage + box * kKVTile + h * kHalfTile, &tmKV, &full[stage], box * 64, row0v);
+        tma_load_2d(sK + stage * kStage + box * kBox + h * kHalfTile, &tmKV, &full[stage], box * 64, row0);
+        tma_load_2d(sV + stage * kStage + box * kBox + h * kHalfTile, &tmKV, &full[stage], box * 64, row0v);
       }
     }
   };
   // the K/V tiles wholly in the cached prefix are requested before the dependency wait
   int n_pre = 0;
   if (tma_thr)
-    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kTcTile <= len; ++n_pre) issue(n_pre);
+    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kTile <= len; ++n_pre) issue(n_pre);
   pdl_wait();
   stamp(1);
   if (tma_thr)
@@ -723,7 +737,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   const int prow = r / a.G;
   const bool row_ok = softmax_thr && r < a.rows && prow < np;
   // query rows -> TMEM, the A operand of S = Q K^T: thread (kq, r) writes dims kq kOC .. of row r
-  // as packed bf16 pairs at columns 384 + d / 2 (hi) and 448 + d / 2 (lo); padding rows are zero
+  // as packed bf16 pairs at columns kQCol + d / 2 (hi) and kQCol + 64 + d / 2 (lo); padding rows
+  // are zero
   if (softmax_thr) {
     const uint32_t lane_q = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int gh = r - prow * a.G;
@@ -758,8 +773,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         lw[4 * u + 2] = __uint_as_float(lv[u].z);
         lw[4 * u + 3] = __uint_as_float(lv[u].w);
       }
-      tmem_st16(tmem + lane_q + 384 + kq * (kOC / 2) + cc * 16, hw);
-      if constexpr (kHiLo) tmem_st16(tmem + lane_q + 448 + kq * (kOC / 2) + cc * 16, lw);
+      tmem_st16(tmem + lane_q + kQCol + kq * (kOC / 2) + cc * 16, hw);
+      if constexpr (kHiLo) tmem_st16(tmem + lane_q + kQCol + 64 + kq * (kOC / 2) + cc * 16, lw);
     }
     tmem_st_wait();
   }
@@ -774,7 +789,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   // the TMA thread loads K/V and issues O += P V.  Their MMAs touch different TMEM (S buffers /
   // O) and each commits only its own, so they need no ordering between them; splitting the
   // issue halves the per-tile issue time of the one thread that used to issue both.
-  const uint32_t idS = idesc_bf16_f32(128, kTcTile);
+  const uint32_t idS = idesc_bf16_f32(128, kTile);
   const uint32_t idO = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) MN-major
   // O += P V of tile i (P over S in S buffer i & 1, K/V stage i % NS); the stage frees when it
   // completes.  P of key part kq (keys kKT kq ..) sits in that part's S columns: kKT / 2 columns
@@ -786,11 +801,12 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
 #pragma unroll
     for (int q = 0; q < kQ; ++q)
 #pragma unroll
-      for (int ks = 0; ks < kTcTile / 16; ++ks) {   // 16-key step: page ks / 4, rows 16 (ks % 4) ..
+      for (int ks = 0; ks < kTile / 16; ++ks) {   // 16-key step: page ks / 4, rows 16 (ks % 4) ..
         const int part = ks / (kKT / 16), u = ks % (kKT / 16);
-        tc_mma_f16_ts(tmem + 256, tmem + pb * 128 + part * kKT + q * (kKT / 2) + u * 8,
-                      sdesc_mn_sw128(smem_u32(sV + st * kTcStage + (ks >> 2) * kHalfTile + (ks & 3) * 2048), kKVTile,
-                                     1024),
+        tc_mma_f16_ts(tmem + kOCol,
+                      kAlias ? tmem + pb * kTile + part * kKT + q * (kKT / 2) + u * 8
+                             : tmem + kPCol + pb * 64 + q * 32 + ks * 8,
+                      sdesc_mn_sw128(smem_u32(sV + st * kStage + (ks >> 2) * kHalfTile + (ks & 3) * 2048), kBox, 1024),
                       idO, (i > 0 || q > 0 || ks > 0) ? 1u : 0u);
       }
     tc_commit(&pv_done[pb]);
@@ -801,7 +817,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   auto s_step = [&](int j) -> bool {
     const int st = j % NS, sb = j & 1;
     if (*s_abort || !mbar_wait(&full[st], static_cast<uint32_t>(j / NS) & 1u, kWait) ||
-        (j >= 2 && !mbar_wait(&pv_done[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
+        (j >= 2 && !mbar_wait(kAlias ? &pv_done[sb] : &s_free[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait)))
       return false;
     tc_fence_after();
 #pragma unroll
@@ -810,8 +826,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       for (int box = 0; box < 2; ++box)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_f16_ts(tmem + sb * 128, tmem + 384 + q * 64 + (box * 4 + kk) * 8,
-                        sdesc_k_sw128(smem_u32(sK + st * kTcStage + box * kKVTile)) + 2 * kk, idS,
+          tc_mma_f16_ts(tmem + sb * kTile, tmem + kQCol + q * 64 + (box * 4 + kk) * 8,
+                        sdesc_k_sw128(smem_u32(sK + st * kStage + box * kBox)) + 2 * kk, idS,
                         (q > 0 || box > 0 || kk > 0) ? 1u : 0u);
     tc_commit(&s_full[sb]);
     return true;
@@ -857,7 +873,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     if (row_ok) row_keys(len, p0 + prow, a.block_size, a.m, crow, a.quad_k, v1, l2, h2);
     const int lq = warp & 3;   // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(lq * 32) << 16;
-    const uint32_t o_col = 256 + kq * kOC;   // this thread's columns of O
+    const uint32_t o_col = kOCol + kq * kOC;   // this thread's columns of O
     const float c = a.scale_log2;
     for (int j = 0; j < ntile; ++j) {
       const int sb = j & 1;
@@ -870,11 +886,16 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       tc_fence_after();
       uint32_t raw[kKT / 16][16];
 #pragma unroll
-      for (int u = 0; u < kKT / 16; ++u) tmem_ld16_nowait(tmem + lane_base + sb * 128 + kq * kKT + u * 16, raw[u]);
+      for (int u = 0; u < kKT / 16; ++u) tmem_ld16_nowait(tmem + lane_base + sb * kTile + kq * kKT + u * 16, raw[u]);
 #pragma unroll
       for (int u = 0; u < kKT / 16; ++u) tmem_ld_wait_regs(raw[u]);
+      if constexpr (!kAlias) {
+        tc_fence_before();
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(&s_free[sb]);
+      }
       float sv[kKT];
-      const int k0 = (t_lo + j) * kTcTile + kq * kKT;
+      const int k0 = (t_lo + j) * kTile + kq * kKT;
       if (k0 + kKT - 1 <= v1) {
 #pragma unroll
         for (int k = 0; k < kKT; ++k) sv[k] = __uint_as_float(raw[k >> 4][k & 15]);
@@ -943,12 +964,21 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
         }
       }
       l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // P over this thread's own S columns (read above): kKT / 2 columns of hi pairs, then lo
-      const uint32_t p_col = sb * 128 + kq * kKT;
+      // P: 128-key tiles over this thread's own S columns (read above), kKT / 2 columns of hi
+      // pairs then lo; 64-key tiles into P buffer sb
+      // 64-key tiles: P buffer sb is free once O += P V of tile j - 2 has completed
+      if constexpr (!kAlias) {
+        if (!__all_sync(0xffffffffu, j < 2 || mbar_wait(&pv_done[sb], static_cast<uint32_t>((j - 2) >> 1) & 1u, kWait))) {
+          aborted = true;
+          break;
+        }
+      }
+      const uint32_t p_col = kAlias ? sb * kTile + kq * kKT : kPCol + sb * 64 + kq * (kKT / 2);
+      const uint32_t p_lo = kAlias ? kKT / 2 : 32;   // lo pairs after the hi pairs
 #pragma unroll
       for (int u = 0; u < kKT / 16; ++u) {
         tmem_st8(tmem + lane_base + p_col + u * 8, ph[u]);
-        if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + kKT / 2 + u * 8, pl[u]);
+        if constexpr (kHiLo) tmem_st8(tmem + lane_base + p_col + p_lo + u * 8, pl[u]);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -1004,8 +1034,8 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
     for (int cc = 0; cc < kOC / 32; ++cc) {
       uint32_t o[2][16];
       if (have) {
-        tmem_ld16_nowait(tmem + lane_base + 256 + kq * kOC + cc * 32, o[0]);
-        tmem_ld16_nowait(tmem + lane_base + 256 + kq * kOC + cc * 32 + 16, o[1]);
+        tmem_ld16_nowait(tmem + lane_base + kOCol + kq * kOC + cc * 32, o[0]);
+        tmem_ld16_nowait(tmem + lane_base + kOCol + kq * kOC + cc * 32 + 16, o[1]);
         tmem_ld_wait_regs(o[0]);
         tmem_ld_wait_regs(o[1]);
       } else {
@@ -1156,9 +1186,13 @@ namespace {
 using AttnKernel = void (*)(const CUtensorMap, const AttnArgs);
 // The instantiation for a launch: tcgen05 or mma.sync, its operand form and (mma.sync) its
 // launch bound (<= 8 or 9 warps).
-AttnKernel attn_kernel_for(bool hilo, int NW, int tc) {
-  if (tc == 2) return hilo ? attn_tc_kernel<true, 2> : attn_tc_kernel<false, 2>;
-  if (tc) return hilo ? attn_tc_kernel<true, 4> : attn_tc_kernel<false, 4>;
+AttnKernel attn_kernel_for(bool hilo, int NW, int tc, int tile) {
+  if (tc && tile == 64) {
+    if (tc == 2) return hilo ? attn_tc_kernel<true, 2, 64> : attn_tc_kernel<false, 2, 64>;
+    return hilo ? attn_tc_kernel<true, 4, 64> : attn_tc_kernel<false, 4, 64>;
+  }
+  if (tc == 2) return hilo ? attn_tc_kernel<true, 2, 128> : attn_tc_kernel<false, 2, 128>;
+  if (tc) return hilo ? attn_tc_kernel<true, 4, 128> : attn_tc_kernel<false, 4, 128>;
   if (NW > 8) return hilo ? attn_mma_kernel<true, 9> : attn_mma_kernel<false, 9>;
   return hilo ? attn_mma_kernel<true, 8> : attn_mma_kernel<false, 8>;
 }
@@ -1172,8 +1206,9 @@ cudaError_t init_kernel_attributes() {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  for (int v = 0; v < 8; ++v) {   // mma.sync (hilo x 8/9 warps), tcgen05 (hilo x 2/4 per row)
-    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8, v >= 4 ? 2 * ((v >> 1) & 1) + 2 : 0);
+  // mma.sync (hilo x 8/9 warps), tcgen05 (hilo x 2/4 per row x 64/128-key tiles)
+  for (int v = 0; v < 12; ++v) {
+    const AttnKernel k = attn_kernel_for(v & 1, (v & 2) ? 9 : 8, v >= 4 ? 2 * ((v >> 1) & 1) + 2 : 0, v >= 8 ? 64 : 128);
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1195,8 +1230,9 @@ size_t attn_mma_smem_bytes(int NW, bool hilo, int stages) {
 // Dynamic shared memory of a tcgen05 attention launch: the K and V rings (the query tile lives in
 // TMEM), the row-max exchange and the barriers; the split partials overlay the rings after the
 // KV loop.
-size_t attn_tc_smem_bytes(bool hilo, int rt) {
-  return 1024 + 2 * static_cast<size_t>(tc_stages(hilo)) * kTcStage + tc_xchg_bytes(rt) + kTcBarBytes;
+size_t attn_tc_smem_bytes(bool, int rt) {
+  // the same ring bytes for either tile size
+  return 1024 + 2 * static_cast<size_t>(tc_stages(128)) * tc_stage_bytes(128) + tc_xchg_bytes(rt) + kTcBarBytes;
 }
 
 // Clusters of S CTAs (NW warps, the shared memory above; or the tcgen05 kernel) that can be
@@ -1214,7 +1250,7 @@ int attn_mma_max_clusters(int S, int NW, bool hilo, int stages, int sms, int tc)
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, attn_kernel_for(hilo, NW, tc), &cfg);
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, attn_kernel_for(hilo, NW, tc, 128), &cfg);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return sms / S;
@@ -1226,7 +1262,7 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
                                  int batch, bool pdl) {
   const int tc = a.tc;
   if ((tc != 0 && tc != 2 && tc != 4) ||
-      (tc ? (a.rows < 1 || a.rows > 128 || a.S < 1 || a.S > 8)
+      (tc ? (a.rows < 1 || a.rows > 128 || a.S < 1 || a.S > 8 || (a.tc_tile != 64 && a.tc_tile != 128))
           : (a.NW < 1 || a.NW > kMaxAttWarps || a.stages < 2 || a.stages > kMaxAttStages)))
     return cudaErrorInvalidValue;   // kernel form, tile rows / launch bound, ring depth
   cudaLaunchConfig_t cfg = {};
@@ -1247,7 +1283,7 @@ cudaError_t launch_attention_mma(cudaStream_t st, const CUtensorMap* tmKV, const
   if (pdl) attrs[na++] = attr[0];
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_kernel_for(a.hilo != 0, a.NW, tc), *tmKV, a);
+  return cudaLaunchKernelEx(&cfg, attn_kernel_for(a.hilo != 0, a.NW, tc, a.tc_tile), *tmKV, a);
 }
 
 cudaError_t launch_attention_simt(cudaStream_t st, const AttnArgs& a, int batch, bool f32,

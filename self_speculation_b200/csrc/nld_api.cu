@@ -540,24 +540,36 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // only while the grid is short of two CTAs per SM, keep >= min_tiles KV tiles per split, take
   // no more splits than lets every cluster be resident at once (a second wave doubles the
   // latency), and launch no split that the tiles per split leave empty.
-  // The tcgen05 kernel's KV tiles are 128 keys (two pages): its splits are counted in those.
+  // The tcgen05 kernel's KV tiles: 64 keys where a split holds a few pages (its short chain of
+  // tiles is the latency: the batch-1 round), 128 where splits are long (S with N = 128: half
+  // the S MMAs per key); its splits are counted in those tiles.
   const int units = batch * a.q_tiles * Hkv;
-  const int kt = use_tc ? (n_tiles + 1) / 2 : n_tiles;             // KV tiles of the kernel
-  const int min_kt = use_tc ? (min_tiles + 1) / 2 : min_tiles;
-  a.S = 1;
-  if (units < 2 * sms) {
-    int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, kt / min_kt)}));
-    while (s_max > 1 && units > cap(s_max, a.NW, a.stages, tc)) --s_max;
-    const int per = std::max(min_kt, (kt + s_max - 1) / s_max);
-    a.S = std::max(1, (kt + per - 1) / per);
+  auto split_plan = [&](int pg, int* per_pages) {
+    const int kt = (n_tiles + pg - 1) / pg;                       // KV tiles of the kernel
+    const int min_kt = (min_tiles + pg - 1) / pg;
+    int S = 1;
+    if (units < 2 * sms) {
+      int s_max = std::max(1, std::min({8, (2 * sms + units - 1) / units, std::max(1, kt / min_kt)}));
+      while (s_max > 1 && units > cap(s_max, a.NW, a.stages, tc)) --s_max;
+      const int per = std::max(min_kt, (kt + s_max - 1) / s_max);
+      S = std::max(1, (kt + per - 1) / per);
+    }
+    *per_pages = std::max(min_kt, (kt + S - 1) / S) * pg;
+    return S;
+  };
+  int per_pages = 0;
+  a.S = split_plan(1, &per_pages);
+  a.tc_tile = 64;
+  if (use_tc && per_pages > 4) {
+    a.tc_tile = 128;
+    a.S = split_plan(2, &per_pages);
   }
   // tcgen05 softmax threads per row: 4 (16 warps) shorten a CTA's fixed costs and each KV tile's
   // latency chain, which short splits wait on; 2 (8 warps) issue fewer instructions per tile,
   // which long splits are bound by (measured: 4 win at <= 17 pages per CTA by up to 20 %, 2 at
   // 65 and 257 pages by 5-8 %, even at 33)
   if (use_tc && (kernel == 0 || kernel == 1)) {
-    const int per = std::max(min_kt, (kt + a.S - 1) / a.S);
-    tc = per > 16 ? 2 : 4;
+    tc = per_pages > 32 ? 2 : 4;
     a.tc = tc;
   }
 }
@@ -1884,8 +1896,8 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
   return NLD_OK;
 }
 
-nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out7) {
-  if (!out7) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
+nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out8) {
+  if (!out8) return fail(nullptr, NLD_ERR_ARG, "NULL argument");
   if (batch < 1 || m < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_len < 1 || sms < 1)
     return fail(nullptr, NLD_ERR_ARG, "bad attention plan sizes");
   AttnArgs a{};
@@ -1896,8 +1908,8 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
     const int per_sm = static_cast<int>(233472 / (smem + 1024));
     return std::max(1, sms * per_sm / S);
   }, 0, 0, g_attn_kernel.load());
-  const int v[7] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc ? 1 : 0};
-  for (int i = 0; i < 7; ++i) out7[i] = v[i];
+  const int v[8] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc ? 1 : 0, a.tc ? a.tc_tile : 64};
+  for (int i = 0; i < 8; ++i) out8[i] = v[i];
   return NLD_OK;
 }
 

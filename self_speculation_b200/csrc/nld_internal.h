@@ -158,6 +158,7 @@ struct AttnArgs {
   int stages;           // K/V ring depth of the tensor-core path (2 or 3)
   int tc;               // 2 / 4: the tcgen05 kernel (query tiles of <= 128 rows) with 2 / 4
                         // softmax threads per row; 0: mma.sync
+  int tc_tile;          // tcgen05: keys per KV tile, 64 or 128
   float scale_log2;     // log2(e) / sqrt(hd)
   int hilo;             // tensor-core path: q fp32 [M, Hq, hd], out (hi, lo) bf16 rows [2M, Hq, hd]
   int quad_k;           // quadratic self-speculation forward with block k (0 = off): rows 0..k are

@@ -39,13 +39,13 @@ def plan_chain(M, phases, clusters=B200_CLUSTERS, hilo=1):
 def plan_attention(batch, m, Hq, Hkv, max_len, sms=148, kernel=0):
     """kernel: 0 the planner's choice, 1 tcgen05, 2 mma.sync (the process-wide setting is put back)."""
     lib = nb.load_library()
-    out = (ctypes.c_int * 7)()
+    out = (ctypes.c_int * 8)()
     assert lib.nld_debug_attention_kernel(kernel) == 0
     try:
         assert lib.nld_plan_attention(batch, m, Hq, Hkv, max_len, sms, out) == 0
     finally:
         assert lib.nld_debug_attention_kernel(0) == 0
-    return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S", "tc"], list(out)))
+    return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S", "tc", "tile"], list(out)))
 
 
 def chains(cfg):
@@ -139,21 +139,22 @@ def test_attention_plans_keep_kernel_limits(name, cfg):
                 if A["tc"]:
                     assert A["rows"] <= 128, where   # one tcgen05 MMA tile
                 assert 1 <= A["S"] <= 8, where
-                # every split has a KV tile (tcgen05: tiles of 128 keys)
-                assert A["S"] <= -(-max_len // (128 if A["tc"] else 64)), where
+                assert A["tile"] in ((64, 128) if A["tc"] else (64,)), where
+                assert A["S"] <= -(-max_len // A["tile"]), where   # every split has a KV tile
                 if B * A["q_tiles"] * cfg.n_kv_heads >= 2 * 148:
                     assert A["S"] == 1, where
 
 
 def test_attention_plan_of_the_benchmarked_round():
-    # tcgen05 (the planner's choice, KV tiles of 128 keys): verify forward (m = 33: 2 query tiles
-    # of 17 positions x 4 heads) and draft forward (m = 32: one 128-row tile); 545 keys = 5 tiles
-    # in 5 splits, 865 keys = 7 tiles in 7 splits, 1400 keys = 11 tiles in 6 splits of <= 2
-    for keys, S in ((545, 5), (865, 7), (1400, 6)):
+    # tcgen05 (the planner's choice; KV tiles of 64 keys at batch 1): verify forward (m = 33: 2
+    # query tiles of 17 positions x 4 heads) and draft forward (m = 32: one 128-row tile); 545
+    # keys = 9 tiles in 5 splits of <= 2, 865 keys = 14 tiles in 7 splits, 1400 keys = 22 tiles
+    # in 8 splits of <= 3
+    for keys, S in ((545, 5), (865, 7), (1400, 8)):
         v = plan_attention(1, 33, 32, 8, keys)
         d = plan_attention(1, 32, 32, 8, keys)
-        assert (v["G"], v["QT"], v["q_tiles"], v["rows"], v["S"], v["tc"]) == (4, 17, 2, 68, S, 1)
-        assert (d["QT"], d["q_tiles"], d["rows"], d["S"], d["tc"]) == (32, 1, 128, S, 1)
+        assert (v["G"], v["QT"], v["q_tiles"], v["rows"], v["S"], v["tc"], v["tile"]) == (4, 17, 2, 68, S, 1, 64)
+        assert (d["QT"], d["q_tiles"], d["rows"], d["S"], d["tc"], d["tile"]) == (32, 1, 128, S, 1, 64)
     # mma.sync: 3 query tiles of 11 positions (3 warps) and 2 tiles of 16 positions (4 warps)
     for keys, S in ((545, 5), (865, 7)):
         v = plan_attention(1, 33, 32, 8, keys, kernel=2)
@@ -167,7 +168,7 @@ def test_attention_plan_of_the_benchmarked_round():
     b = plan_attention(64, 33, 32, 8, 4096 + 33, kernel=2)
     assert (b["QT"], b["q_tiles"], b["NW"], b["S"], b["tc"]) == (33, 1, 9, 1, 0)
     b = plan_attention(64, 32, 32, 8, 4096 + 32)
-    assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"]) == (32, 1, 128, 1, 1)
+    assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"], b["tile"]) == (32, 1, 128, 1, 1, 128)
     # small query tiles (a 4-row single-token decode, 32-row blocks of many sequences) cost the
     # tcgen05 kernel a whole 128-row tile per KV tile: they stay on mma.sync; 64-row blocks go to
     # tcgen05
@@ -188,4 +189,4 @@ def test_plan_hooks_reject_bad_sizes():
     assert lib.nld_plan_chain(0, 1, rows, (ctypes.c_int * 1)(4096), mc, 1, out) == 1
     none = (ctypes.c_int * 9)(*([0] * 9))
     assert lib.nld_plan_chain(33, 1, rows, (ctypes.c_int * 1)(4096), none, 1, out) == 8   # unsupported
-    assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 7)()) == 1
+    assert lib.nld_plan_attention(1, 33, 32, 7, 100, 148, (ctypes.c_int * 8)()) == 1
