@@ -300,7 +300,7 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
  * keys up to max_len, on sms SMs, under the current nld_debug_attention_kernel setting.
  * out8 = {G = Hq/Hkv, query positions per CTA, query tiles, rows per CTA (positions x G), warps
  * per CTA (mma.sync kernel), KV splits (= cluster size), kernel (1 tcgen05, 0 mma.sync), keys
- * per KV tile (64; 128 for tcgen05 splits of more than 4 pages)}.  NLD_ERR_ARG on bad sizes. */
+ * per KV tile (64; 128 for tcgen05 splits of more than 16 pages)}.  NLD_ERR_ARG on bad sizes. */
 nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out8);
 
 /* Profiling hook: tuning of the projection chains' pipeline.  stage_cap = 0 lets the planner

@@ -540,8 +540,8 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // only while the grid is short of two CTAs per SM, keep >= min_tiles KV tiles per split, take
   // no more splits than lets every cluster be resident at once (a second wave doubles the
   // latency), and launch no split that the tiles per split leave empty.
-  // The tcgen05 kernel's KV tiles: 64 keys where a split holds a few pages (its short chain of
-  // tiles is the latency: the batch-1 round), 128 where splits are long (S with N = 128: half
+  // The tcgen05 kernel's KV tiles: 64 keys where a split holds up to 16 pages (its chain of
+  // tiles is the latency: the batch-1 round), 128 where splits are longer (S with N = 128: half
   // the S MMAs per key); its splits are counted in those tiles.
   const int units = batch * a.q_tiles * Hkv;
   auto split_plan = [&](int pg, int* per_pages) {
@@ -560,7 +560,7 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   int per_pages = 0;
   a.S = split_plan(1, &per_pages);
   a.tc_tile = 64;
-  if (use_tc && per_pages > 4) {
+  if (use_tc && per_pages > 16) {
     a.tc_tile = 128;
     a.S = split_plan(2, &per_pages);
   }
