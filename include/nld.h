@@ -297,10 +297,12 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
                           int hilo, int* out20);
 
 /* Test hook, pure host: the attention launch plan for batch sequences of m rows, Hq/Hkv heads,
- * keys up to max_len, on sms SMs, under the current nld_debug_attention_kernel setting.
+ * keys up to max_len, on sms SMs, under the current nld_debug_attention_kernel and
+ * nld_debug_attention_tile settings.
  * out8 = {G = Hq/Hkv, query positions per CTA, query tiles, rows per CTA (positions x G), warps
  * per CTA (mma.sync kernel), KV splits (= cluster size), kernel (1 tcgen05, 0 mma.sync), keys
- * per KV tile (64; 128 for tcgen05 splits of more than 16 pages)}.  NLD_ERR_ARG on bad sizes. */
+ * per KV tile (64; 128 for tcgen05 splits of more than 16 pages, or as nld_debug_attention_tile
+ * sets)}.  NLD_ERR_ARG on bad sizes. */
 nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out8);
 
 /* Profiling hook: tuning of the projection chains' pipeline.  stage_cap = 0 lets the planner
@@ -334,6 +336,14 @@ nld_status nld_debug_attention_tuning(nld_ctx* ctx, int rows_per_cta, int min_ti
  * Applies to launches planned afterwards (a context's captured graphs keep their kernel until
  * they are dropped, e.g. by nld_debug_attention_tuning).  NLD_ERR_ARG for other values. */
 nld_status nld_debug_attention_kernel(int kernel);
+
+/* Test and profiling hook, process-wide: keys per KV tile of the tcgen05 attention kernel.  0
+ * (the default) = the planner's choice: 64-key tiles, whose P has TMEM columns of its own, while
+ * a KV split holds at most 16 pages of 64 keys, else 128-key tiles, whose P is written over S;
+ * 64 or 128 = that tile whatever the split length (the KV splits are then planned in those
+ * tiles).  Either tile is correct for every input.  Applies to launches planned afterwards, as
+ * nld_debug_attention_kernel.  NLD_ERR_ARG for other values. */
+nld_status nld_debug_attention_tile(int keys);
 
 /* Profiling hook: timestamps of one layer inside the model's own forwards (graph launches
  * included).  While layer >= 0, the tensor-core attention launch of that layer (every forward;

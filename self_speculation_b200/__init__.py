@@ -76,6 +76,7 @@ def load_library() -> ctypes.CDLL:
         "nld_debug_timeout_chain": ([P, ctypes.c_ulonglong], I),
         "nld_debug_attention_tuning": ([P, I, I], I),
         "nld_debug_attention_kernel": ([I], I),
+        "nld_debug_attention_tile": ([I], I),
         "nld_debug_layer_trace": ([P, I, P, S, P, S], I),
         "nld_stream": ([P], P),
         "nld_last_error": ([P], ctypes.c_char_p),

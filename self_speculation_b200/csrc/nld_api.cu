@@ -493,11 +493,15 @@ using AttnCapacity = std::function<int(int S, int NW, int stages, int tc)>;
 // Which kernel serves the tensor-core attention (profiling hook): 0 the planner's choice,
 // 1 tcgen05, 2 mma.sync, 3 / 4 tcgen05 with 2 / 4 softmax threads per row.
 std::atomic<int> g_attn_kernel{0};
+// Keys per KV tile of the tcgen05 kernel (profiling and test hook): 0 the planner's choice, 64
+// or 128.
+std::atomic<int> g_attn_tile{0};
 
 // rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
-// tiles a split takes at least; 0 = the planner's choice for either.
+// tiles a split takes at least; 0 = the planner's choice for either.  tile: keys per tcgen05 KV
+// tile, 0 = the planner's choice.
 void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
-               int rows_cap = 0, int min_tiles = 0, int kernel = 0) {
+               int rows_cap = 0, int min_tiles = 0, int kernel = 0, int tile = 0) {
   a.G = Hq / Hkv;
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   auto q_tiles_for = [&](int c) {
@@ -560,7 +564,7 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   int per_pages = 0;
   a.S = split_plan(1, &per_pages);
   a.tc_tile = 64;
-  if (use_tc && per_pages > 16) {
+  if (use_tc && (tile == 128 || (tile == 0 && per_pages > 16))) {
     a.tc_tile = 128;
     a.S = split_plan(2, &per_pages);
   }
@@ -690,7 +694,7 @@ nld_status launch_forward(nld_ctx* x, const FwdSpec& f) {
   if (x->bf16) {
     attn_plan(f.B, f.m, aa.Hq, aa.Hkv, max_len, x->sms, aa,
               [](int S, int NW, int stages, int tc) { return attn_device_capacity(true, S, NW, stages, tc); },
-              x->attn_rows_cap, x->attn_min_tiles, g_attn_kernel.load());
+              x->attn_rows_cap, x->attn_min_tiles, g_attn_kernel.load(), g_attn_tile.load());
     const size_t ctas = static_cast<size_t>(aa.S) * aa.Hkv * f.B * aa.q_tiles;
     attn_traced = x->attn_trace && ctas * 16 <= x->attn_trace_n;
   } else {
@@ -1825,6 +1829,13 @@ nld_status nld_debug_attention_kernel(int kernel) {
   return NLD_OK;
 }
 
+nld_status nld_debug_attention_tile(int keys) {
+  if (keys != 0 && keys != 64 && keys != 128)
+    return fail(nullptr, NLD_ERR_ARG, "keys per tcgen05 KV tile: 0 (planner), 64 or 128");
+  g_attn_tile.store(keys);
+  return NLD_OK;
+}
+
 nld_status nld_debug_attention_tuning(nld_ctx* x, int rows_per_cta, int min_tiles_per_split) {
   if (!x) return fail(nullptr, NLD_ERR_ARG, "ctx is NULL");
   if ((rows_per_cta != 0 && (rows_per_cta < 16 || rows_per_cta > 144)) || min_tiles_per_split < 0 ||
@@ -1907,7 +1918,7 @@ nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, in
     const size_t smem = tc ? attn_tc_smem_bytes(true, tc) : attn_mma_smem_bytes(NW, true, stages);
     const int per_sm = static_cast<int>(233472 / (smem + 1024));
     return std::max(1, sms * per_sm / S);
-  }, 0, 0, g_attn_kernel.load());
+  }, 0, 0, g_attn_kernel.load(), g_attn_tile.load());
   const int v[8] = {a.G, a.QT, a.q_tiles, a.rows, a.NW, a.S, a.tc ? 1 : 0, a.tc ? a.tc_tile : 64};
   for (int i = 0; i < 8; ++i) out8[i] = v[i];
   return NLD_OK;
@@ -2140,7 +2151,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   AttnArgs a{};
   attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
             [](int S, int NW, int stages, int tc) { return attn_device_capacity(false, S, NW, stages, tc); },
-            0, 0, g_attn_kernel.load());
+            0, 0, g_attn_kernel.load(), g_attn_tile.load());
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))

@@ -68,3 +68,6 @@ def test_null_arguments_rejected():
     assert lib.nld_debug_attention_kernel(5) == 1
     assert lib.nld_debug_attention_kernel(-1) == 1
     assert lib.nld_debug_attention_kernel(0) == 0
+    assert lib.nld_debug_attention_tile(32) == 1
+    assert lib.nld_debug_attention_tile(256) == 1
+    assert lib.nld_debug_attention_tile(0) == 0

@@ -19,15 +19,23 @@ HQ, HKV, HD = 32, 8, 128
 TOL = 2e-2
 
 
-@pytest.fixture(autouse=True, params=["mma_sync", "tcgen05_2", "tcgen05_4"])
+KERNELS = {"mma_sync": (2, 0), "tcgen05_2_k64": (3, 64), "tcgen05_2_k128": (3, 128),
+           "tcgen05_4_k64": (4, 64), "tcgen05_4_k128": (4, 128)}
+
+
+@pytest.fixture(autouse=True, params=list(KERNELS))
 def attention_kernel(request):
     """Every case runs on each tensor-core attention kernel: mma.sync, and tcgen05 with 2 or 4
-    softmax threads per row (the process-wide switch is put back to the default afterwards)."""
+    softmax threads per row and KV tiles of 64 keys (P in TMEM columns of its own) or 128 (P
+    over S), whatever the split lengths (the process-wide switches are put back afterwards)."""
     import self_speculation_b200 as nb
     lib = nb.load_library()
-    assert lib.nld_debug_attention_kernel({"mma_sync": 2, "tcgen05_2": 3, "tcgen05_4": 4}[request.param]) == 0
+    kernel, tile = KERNELS[request.param]
+    assert lib.nld_debug_attention_kernel(kernel) == 0
+    assert lib.nld_debug_attention_tile(tile) == 0
     yield request.param
     assert lib.nld_debug_attention_kernel(0) == 0
+    assert lib.nld_debug_attention_tile(0) == 0
 
 
 def _setup(lens, m, seed=2, shuffle_seed=0):

@@ -58,6 +58,33 @@ def test_forward_logits_all_modes(B, P):
     _check_logits(ga, odec.ar_forward(om, st2))
 
 
+@pytest.mark.parametrize("kernel,tile", [(3, 64), (3, 128), (4, 64), (4, 128)])
+@pytest.mark.parametrize("B,P", [(1, 100), (3, 77)])
+def test_draft_verify_logits_each_tcgen05_attention_form(kernel, tile, B, P):
+    """The model's own attention launches (fp32 q and P as (hi, lo) operands) on the tcgen05
+    kernel with 2 / 4 softmax threads per row and 64- / 128-key KV tiles, whatever the planner
+    would pick: draft and verify logits within the bar."""
+    import self_speculation_b200 as nb
+    lib = nb.load_library()
+    assert lib.nld_debug_attention_kernel(kernel) == 0
+    assert lib.nld_debug_attention_tile(tile) == 0
+    try:
+        ctx, om, _ = make_pair(CFG)
+        p = synth.prompt_tokens(B, P, CFG.vocab, seed=4)
+        ctx.nld_prefill(p.cuda())
+        st = odec.prefill(om, p, CFG.max_seq + 64)
+        k = CFG.block_k
+        gl = gpu_logits(ctx, 1, B, k)
+        _check_logits(gl, odec.draft_forward(om, st, k))
+        _, _, draft, _ = gpu_state(ctx, B)
+        gv = gpu_logits(ctx, 2, B, k + 1)
+        _check_logits(gv, odec.verify_forward(om, st, draft))
+        del ctx
+    finally:
+        assert lib.nld_debug_attention_kernel(0) == 0
+        assert lib.nld_debug_attention_tile(0) == 0
+
+
 def test_rounds_commit_bit_exact_given_argmaxes():
     """Teacher-forced over several rounds: the oracle replays each round's commit on the GPU's
     draft and verify argmaxes; tokens, counts, lengths and pending tokens must match exactly,

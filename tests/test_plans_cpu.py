@@ -36,15 +36,18 @@ def plan_chain(M, phases, clusters=B200_CLUSTERS, hilo=1):
                 split=[(o[10 + 2 * p], o[11 + 2 * p]) for p in range(n)])
 
 
-def plan_attention(batch, m, Hq, Hkv, max_len, sms=148, kernel=0):
-    """kernel: 0 the planner's choice, 1 tcgen05, 2 mma.sync (the process-wide setting is put back)."""
+def plan_attention(batch, m, Hq, Hkv, max_len, sms=148, kernel=0, tile=0):
+    """kernel: 0 the planner's choice, 1 tcgen05, 2 mma.sync; tile: keys per tcgen05 KV tile, 0
+    the planner's choice (the process-wide settings are put back)."""
     lib = nb.load_library()
     out = (ctypes.c_int * 8)()
     assert lib.nld_debug_attention_kernel(kernel) == 0
+    assert lib.nld_debug_attention_tile(tile) == 0
     try:
         assert lib.nld_plan_attention(batch, m, Hq, Hkv, max_len, sms, out) == 0
     finally:
         assert lib.nld_debug_attention_kernel(0) == 0
+        assert lib.nld_debug_attention_tile(0) == 0
     return dict(zip(["G", "QT", "q_tiles", "rows", "NW", "S", "tc", "tile"], list(out)))
 
 
@@ -178,6 +181,14 @@ def test_attention_plan_of_the_benchmarked_round():
     assert (b["S"], b["tc"], b["tile"]) == (2, 1, 128)
     b = plan_attention(1, 32, 32, 8, 16416)
     assert (b["S"], b["tc"], b["tile"]) == (8, 1, 128)
+    # a forced tile plans the splits in its own tiles: 545 keys = 9 pages = 5 tiles of 128 keys
+    # (5 splits of one); 4128 keys at batch 8 in 64-key tiles: 2 splits of 33
+    b = plan_attention(1, 32, 32, 8, 545, tile=128)
+    assert (b["S"], b["tc"], b["tile"]) == (5, 1, 128)
+    b = plan_attention(8, 32, 32, 8, 4128, tile=64)
+    assert (b["S"], b["tc"], b["tile"]) == (2, 1, 64)
+    # the tile is the tcgen05 kernel's: mma.sync plans keep 64-key pages
+    assert plan_attention(1, 1, 32, 8, 4096, tile=128)["tile"] == 64
     # small query tiles (a 4-row single-token decode, 32-row blocks of many sequences) cost the
     # tcgen05 kernel a whole 128-row tile per KV tile: they stay on mma.sync; 64-row blocks go to
     # tcgen05
