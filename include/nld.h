@@ -350,7 +350,9 @@ nld_status nld_debug_attention_tile(int keys);
  * later ones overwrite) writes to d_attn_trace (device, n_attn uint64 entries, or NULL with
  * n_attn = 0) if its grid fits, per CTA at (CTA linear index) * 16 + i the global timer in ns at:
  * entry (0), dependency on the previous kernel met (1), query tile staged (2), KV tile t done
- * (3 + t, t < 6), split partials published to the cluster (10), output written (11); and the
+ * (3 + t, t < 6), split partials published to the cluster (10), output written (11); the tcgen05
+ * kernel also at: last P V completed (12), partial in shared memory (13), first merged output
+ * row computed (14); and the
  * chain launch that starts with that layer's O projection writes d_chain_trace (NULL, or at
  * least 148*16 + 256 entries) in the layout of nld_trace_chain.  Buffers are caller-owned and
  * zeroed by the caller.  layer = -1 turns the hook off.  Synchronises and drops the captured

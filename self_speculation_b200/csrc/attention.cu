@@ -192,10 +192,8 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
   __syncthreads();
 
-  auto issue = [&](int i) {
+  auto issue_page = [&](int i, int page) {
     const int stage = i % NS;
-    const int kt = t_lo + i;
-    const int page = a.page_table[b * a.pps + kt];
     const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
     const int row0v = row0 + a.Hkv * kPage;
     mbar_arrive_expect_tx(&full[stage], 2 * kKVTile);
@@ -204,15 +202,29 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
     tma_load_2d(sV + stage * kKVTile, &tmKV, &full[stage], 0, row0v);
     tma_load_2d(sV + stage * kKVTile + kHalfTile, &tmKV, &full[stage], 64, row0v);
   };
+  auto issue = [&](int i) { issue_page(i, a.page_table[b * a.pps + t_lo + i]); };
+  // the first tiles: page ids all requested at once, before the dependency wait (the page table
+  // does not change within a forward), so the tiles requested after it (the block's own keys)
+  // wait on no global load; the tiles wholly in the cached prefix are requested before it
+  const int n0 = min(NS, ntile);
   int n_pre = 0;
+  while (n_pre < n0 && (t_lo + n_pre + 1) * kPage <= len) ++n_pre;
+  int pg[kMaxAttStages];
+#pragma unroll
+  for (int u = 0; u < kMaxAttStages; ++u) pg[u] = (tid == 0 && u < n0) ? a.page_table[b * a.pps + t_lo + u] : 0;
   if (tid == 0) {
-    for (; n_pre < min(NS, ntile) && (t_lo + n_pre + 1) * kPage <= len; ++n_pre) issue(n_pre);
+#pragma unroll
+    for (int u = 0; u < kMaxAttStages; ++u)
+      if (u < n_pre) issue_page(u, pg[u]);
   }
   __syncwarp();
   pdl_wait();
   stamp(1);
-  if (tid == 0)
-    for (int i = n_pre; i < min(NS, ntile); ++i) issue(i);
+  if (tid == 0) {
+#pragma unroll
+    for (int u = 0; u < kMaxAttStages; ++u)
+      if (u >= n_pre && u < n0) issue_page(u, pg[u]);
+  }
   __syncwarp();
 
   // Q tile -> shared memory (row = position*G + head, 16-byte chunks XOR-swizzled by row); each
@@ -483,25 +495,27 @@ __global__ void __launch_bounds__(32 * kMaxW, 1)
   const int per_rank = (a.rows + S - 1) / S;
   const int r0 = rank * per_rank, r1 = min(a.rows, r0 + per_rank);
   const uint32_t o_base = smem_u32(sO), ml_base = smem_u32(sML);
-  uint32_t o_peer[8], ml_peer[8];
+  uint32_t o_peer[8];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
-    ml_peer[q] = (q < S) ? dsmem_addr(ml_base, q) : 0u;
-  }
-  for (int e = tid; e < (r1 - r0) * 32; e += nthr) {
+  for (int q = 0; q < 8; ++q) o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
+  // a warp merges one row: lane q < S reads split q's (m, l) of it and the warp shares them (the
+  // cluster's shared-memory reads, which bound the merge, drop by a third)
+  const uint32_t ml_lane = ((tid & 31) < S) ? dsmem_addr(ml_base, tid & 31) : 0u;
+  for (int e = tid; e < (r1 - r0) * 32; e += nthr) {   // warp-uniform: nthr is whole warps
     const int r = r0 + (e >> 5), d4 = e & 31;
     const int p = r / a.G;
     if (p >= np) continue;
     // every split published (m, l) and O for every row (zeros and -inf where it saw no key),
     // so all loads are issued before any is used
+    const float2 mine = (d4 < S) ? ld_dsmem_f2(ml_lane + r * 8) : make_float2(-INFINITY, 0.f);
     float2 ml[8];
     float4 ov[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + r * 8) : make_float2(-INFINITY, 0.f);
+    for (int q = 0; q < 8; ++q)
       ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + (r * 128 + d4 * 4) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      ml[q] = make_float2(__shfl_sync(0xffffffffu, mine.x, q), __shfl_sync(0xffffffffu, mine.y, q));
     float M = -INFINITY;
 #pragma unroll
     for (int q = 0; q < 8; ++q) M = fmaxf(M, ml[q].x);
@@ -555,7 +569,7 @@ __host__ __device__ constexpr int tc_stages(int tile) { return tile == 64 ? 6 : 
 // S of tile j + 2 may be issued while tile j's stage is held: three stages at least
 static_assert(tc_stages(64) >= 3 && tc_stages(128) >= 3 && tc_stages(64) <= kTcMaxStages, "ring depth");
 constexpr float kTcRescale = 8.f;               // log2 units
-constexpr int kTcBarBytes = 256;
+constexpr int kTcBarBytes = 320;
 // row-max exchange: [tile parity][key part][row] floats
 __host__ __device__ constexpr int tc_xchg_bytes(int rt) { return 2 * rt * 128 * 4; }
 
@@ -639,6 +653,9 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   uint64_t* xbar = s_full + 9;        // [2][4] row maxima of a lane quarter written (kRT warps)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_full + 17);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_full + 18);
+  int* s_pg = reinterpret_cast<int*>(s_full + 19);   // [NS kPg] page ids of the first NS tiles
+  static_assert(NS * kPg <= kTcMaxStages, "page ids of the first tiles");
+  static_assert(2 * kTcMaxStages * 8 + 19 * 8 + kTcMaxStages * 4 <= kTcBarBytes, "barrier bytes");
   constexpr uint64_t kWait = 2000000000ull;
 
   const int tid = threadIdx.x;
@@ -704,16 +721,30 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   const int ntile = max(0, min(n_tiles, t_lo + per) - t_lo);
 
   int n_issued = 0;   // K/V tiles requested (TMA thread)
+  // a tile's second page past the keys reads the first page again: its keys are masked, and its
+  // V rows, multiplied by P = 0, must be finite
+  auto page_of = [&](int i, int h) {
+    const int kt = kPg * (t_lo + i);
+    return a.page_table[b * a.pps + (kt + h < n_pages ? kt + h : kt)];
+  };
+  // the page ids of the first NS tiles, all requested at once: the page table does not change
+  // within a forward, so they are read before the dependency wait, and the tiles requested
+  // after it (the block's own keys) wait on no global load
+  if (tma_thr) {
+    const int n0 = min(NS, ntile);
+    int pg[NS * kPg];
+#pragma unroll
+    for (int u = 0; u < NS * kPg; ++u) pg[u] = (u / kPg < n0) ? page_of(u / kPg, u % kPg) : 0;
+#pragma unroll
+    for (int u = 0; u < NS * kPg; ++u) s_pg[u] = pg[u];
+  }
   auto issue = [&](int i) {
     ++n_issued;
     const int stage = i % NS;
-    const int kt = kPg * (t_lo + i);
     mbar_arrive_expect_tx(&full[stage], 2 * kStage);
 #pragma unroll
     for (int h = 0; h < kPg; ++h) {
-      // a tile's second page past the keys reads the first page again: its keys are masked, and
-      // its V rows, multiplied by P = 0, must be finite
-      const int page = a.page_table[b * a.pps + (kt + h < n_pages ? kt + h : kt)];
+      const int page = i < NS ? s_pg[i * kPg + h] : page_of(i, h);
       const int row0 = a.layer_row0 + ((page * 2) * a.Hkv + g) * kPage;
       const int row0v = row0 + a.Hkv * kPage;
 #pragma unroll
@@ -994,6 +1025,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       set_err(a.err, NLD_DEVERR_TIMEOUT);
     }
     tc_fence_after();
+    stamp(12);
   }
 
   // output row rr of this CTA (part 1: the lo row of a (hi, lo) pair)
@@ -1059,6 +1091,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   }
   tc_fence_before();
   __syncthreads();
+  stamp(13);
   if (warp == kTcSoftmax / 32) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -1072,23 +1105,24 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
   const int per_rank = (a.rows + S - 1) / S;
   const int r0 = rank * per_rank, r1 = min(a.rows, r0 + per_rank);
   const uint32_t o_base = smem_u32(sO), ml_base = smem_u32(sML);
-  uint32_t o_peer[8], ml_peer[8];
+  uint32_t o_peer[8];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
-    ml_peer[q] = (q < S) ? dsmem_addr(ml_base, q) : 0u;
-  }
-  for (int e = tid; e < (r1 - r0) * 32; e += kTcThreads) {
+  for (int q = 0; q < 8; ++q) o_peer[q] = (q < S) ? dsmem_addr(o_base, q) : 0u;
+  // a warp merges one row: lane q < S reads split q's (m, L) of it and the warp shares them (the
+  // cluster's shared-memory reads, which bound the merge, drop by a third)
+  const uint32_t ml_lane = ((tid & 31) < S) ? dsmem_addr(ml_base, tid & 31) : 0u;
+  for (int e = tid; e < (r1 - r0) * 32; e += kTcThreads) {   // warp-uniform
     const int rr = r0 + (e >> 5), d4 = e & 31;
     if (rr / a.G >= np) continue;
     const uint32_t o_off = (rr * 128 + ((d4 ^ (rr & 31)) << 2)) * 4;
+    const float2 mine = (d4 < S) ? ld_dsmem_f2(ml_lane + rr * 8) : make_float2(-INFINITY, 0.f);
     float2 ml[8];
     float4 ov[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      ml[q] = (q < S) ? ld_dsmem_f2(ml_peer[q] + rr * 8) : make_float2(-INFINITY, 0.f);
-      ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + o_off) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int q = 0; q < 8; ++q) ov[q] = (q < S) ? ld_dsmem_f4(o_peer[q] + o_off) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      ml[q] = make_float2(__shfl_sync(0xffffffffu, mine.x, q), __shfl_sync(0xffffffffu, mine.y, q));
     float M = -INFINITY;
 #pragma unroll
     for (int q = 0; q < 8; ++q) M = fmaxf(M, ml[q].x);
@@ -1106,6 +1140,7 @@ __global__ void __launch_bounds__(tc_threads(kRT), 1)
       }
     }
     const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    if (e == tid) stamp(14);
     store2(rr, d4 * 4, acc.x * inv, acc.y * inv);
     store2(rr, d4 * 4 + 2, acc.z * inv, acc.w * inv);
   }
