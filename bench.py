@@ -783,6 +783,61 @@ def run_probe(args):
                                            "epi_tiles": [rel(it[3][8 * i:8 * i + 8]) for i in range(8)]}}))
 
 
+def run_layer_trace(args):
+    """Timeline of one layer inside a live self-speculation round (8B shape, batch 1, prompt 512,
+    the graphs the bench replays): the global timer at each stamp of nld_debug_layer_trace, per
+    CTA of that layer's last attention launch in the round (the verify forward's) and of the
+    chain launch after it, as min / median / max over CTAs in microseconds after the attention's
+    dependency on the previous chain is met (no JSON bench line)."""
+    import torch
+
+    import self_speculation_b200 as nb
+    import synth
+    from self_speculation_b200 import build as nbuild
+    nbuild.build()
+    cfg = synth.LLAMA8B.replace(max_seq=2048)
+    st = torch.cuda.Stream()
+    ctx = nb.Context(cfg, stream=st.cuda_stream)
+    ctx.nld_init_weights(synth.model_weights(cfg, 0, device="cuda"), on_device=True)
+    torch.cuda.empty_cache()
+    ctx.nld_prefill(synth.prompt_tokens(1, PROMPT, cfg.vocab, seed=1).cuda())
+    toks = torch.empty(1, K_BLOCK + 1, dtype=torch.int32, device="cuda")
+    nc = torch.empty(1, dtype=torch.int32, device="cuda")
+    for _ in range(args.warmup):
+        ctx.nld_selfspec_round(toks, nc, None)
+    ctx.nld_sync()
+    at = torch.zeros(4096 * 16, dtype=torch.int64, device="cuda")
+    ch = torch.zeros(148 * 16 + 256, dtype=torch.int64, device="cuda")
+    ctx.nld_debug_layer_trace(args.layer_trace, at, ch)
+    ctx.nld_selfspec_round(toks, nc, None)
+    ctx.nld_sync()
+    ctx.nld_debug_layer_trace(-1)
+    a = at.view(-1, 16).cpu().double()
+    # the draft forward's launch of the layer wrote first: keep the CTAs that entered with the
+    # round's last launch, and per stamp the values it wrote
+    a = a[a[:, 0] > a[:, 0].max() - 100e3]
+    t0 = a[:, 1][a[:, 1] > 0].min()
+
+    def stats(col):
+        col = col[col > t0 - 100e3]
+        if len(col) == 0:
+            return None
+        v = (col - t0) / 1e3
+        return [round(float(v.min()), 2), round(float(v.median()), 2), round(float(v.max()), 2)]
+    attn_names = {0: "entry", 1: "dependency_met", 2: "query_staged", 3: "kv_tile0", 4: "kv_tile1",
+                  12: "last_pv_done", 13: "partial_written", 10: "cluster_published",
+                  14: "first_row_merged", 11: "output_written"}
+    c = ch[:148 * 16].view(148, 16).cpu().double()
+    c = c[c[:, 0] > 0]
+    chain_names = ["start", "setup"] + [f"{k}{p}" for p in ("O", "GU", "D", "QKV")
+                                        for k in ("w0_", "epi_go_", "epi_done_")] + ["mma_last", "exit"]
+    print(json.dumps({
+        "layer": args.layer_trace, "attention_ctas": int(a.shape[0]), "chain_ctas": int(c.shape[0]),
+        "attention_us_min_med_max": {nm: stats(a[:, i]) for i, nm in attn_names.items()},
+        "chain_us_min_med_max": {nm: stats(c[:, i]) for i, nm in enumerate(chain_names)}}), flush=True)
+    ctx.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -806,12 +861,17 @@ def main():
                     help="attention workload: one point 'prefix,batch' instead of the whole grid")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
+    ap.add_argument("--layer-trace", type=int, default=-1,
+                    help="timeline of this layer's verify attention and the chain after it in a "
+                         "live round (no JSON bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
     if args.probe:
         run_probe(args)
+    elif args.layer_trace >= 0:
+        run_layer_trace(args)
     elif args.workload == "attention":
         run_attention(args)
     elif args.workload == "diffusion8b":
