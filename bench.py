@@ -476,6 +476,9 @@ def run_attention(args):
     hbm, peak_src = peaks()
     Hq, Hkv, hd, m = 32, 8, 128, args.attn_m
     stream = torch.cuda.current_stream()
+    lib = nb.load_library()
+    if lib.nld_debug_attention_tile(args.attn_tile) != 0:
+        raise SystemExit("--attn-tile takes 0, 64 or 128")
     points = []
     grid = [(L, B) for L in (1024, 4096, 16384, 32768) for B in (1, 8, 32)]
     if args.attn_point:
@@ -507,6 +510,7 @@ def run_attention(args):
         "value": best["GB/s"], "unit": "GB/s", "n_gpus": 1, "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"attention micro-workload: 32q/8kv x 128, {m} queries per sequence",
+                   "tcgen05_kv_tile": args.attn_tile or "planner",
                    "l2": "not flushed: points under 126 MB are marked l2_resident"},
         "roofline": {"bound": "hbm", "achieved": best["GB/s"], "peak": hbm, "unit": "GB/s",
                      "frac": best["frac"], "traffic": None, "peak_kind": f"{peak_src} HBM copy"},
@@ -859,6 +863,8 @@ def main():
                     help="queries per sequence of the attention workload (32; 1 = single-token decode)")
     ap.add_argument("--attn-point", default="",
                     help="attention workload: one point 'prefix,batch' instead of the whole grid")
+    ap.add_argument("--attn-tile", type=int, default=0,
+                    help="attention workload: keys per tcgen05 KV tile (0 = the planner's choice, 64, 128)")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
     ap.add_argument("--layer-trace", type=int, default=-1,

@@ -301,7 +301,7 @@ nld_status nld_plan_chain(int M, int nph, const int* n_rows, const int* K, const
  * nld_debug_attention_tile settings.
  * out8 = {G = Hq/Hkv, query positions per CTA, query tiles, rows per CTA (positions x G), warps
  * per CTA (mma.sync kernel), KV splits (= cluster size), kernel (1 tcgen05, 0 mma.sync), keys
- * per KV tile (64; 128 for tcgen05 splits of more than 16 pages, or as nld_debug_attention_tile
+ * per KV tile (64; 128 for tcgen05 splits of more than 3 pages, or as nld_debug_attention_tile
  * sets)}.  NLD_ERR_ARG on bad sizes. */
 nld_status nld_plan_attention(int batch, int m, int Hq, int Hkv, int max_len, int sms, int* out8);
 
@@ -339,7 +339,7 @@ nld_status nld_debug_attention_kernel(int kernel);
 
 /* Test and profiling hook, process-wide: keys per KV tile of the tcgen05 attention kernel.  0
  * (the default) = the planner's choice: 64-key tiles, whose P has TMEM columns of its own, while
- * a KV split holds at most 16 pages of 64 keys, else 128-key tiles, whose P is written over S;
+ * a KV split holds at most 3 pages of 64 keys, else 128-key tiles, whose P is written over S;
  * 64 or 128 = that tile whatever the split length (the KV splits are then planned in those
  * tiles).  Either tile is correct for every input.  Applies to launches planned afterwards, as
  * nld_debug_attention_kernel.  NLD_ERR_ARG for other values. */

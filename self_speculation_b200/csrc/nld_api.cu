@@ -544,9 +544,10 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // only while the grid is short of two CTAs per SM, keep >= min_tiles KV tiles per split, take
   // no more splits than lets every cluster be resident at once (a second wave doubles the
   // latency), and launch no split that the tiles per split leave empty.
-  // The tcgen05 kernel's KV tiles: 64 keys where a split holds up to 16 pages (its chain of
-  // tiles is the latency: the batch-1 round), 128 where splits are longer (S with N = 128: half
-  // the S MMAs per key); its splits are counted in those tiles.
+  // The tcgen05 kernel's KV tiles: 64 keys where a split holds up to 3 pages (a chain of one to
+  // three short tiles is the latency: the batch-1 round at short prefixes), 128 where splits are
+  // longer (S with N = 128: half the S MMAs per key); its splits are counted in those tiles
+  // (measured: 64 win at <= 2 pages per split, even at 3, 128 win from 4 by 0.5-5 %).
   const int units = batch * a.q_tiles * Hkv;
   auto split_plan = [&](int pg, int* per_pages) {
     const int kt = (n_tiles + pg - 1) / pg;                       // KV tiles of the kernel
@@ -564,7 +565,7 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   int per_pages = 0;
   a.S = split_plan(1, &per_pages);
   a.tc_tile = 64;
-  if (use_tc && (tile == 128 || (tile == 0 && per_pages > 16))) {
+  if (use_tc && (tile == 128 || (tile == 0 && per_pages > 3))) {
     a.tc_tile = 128;
     a.S = split_plan(2, &per_pages);
   }

@@ -172,11 +172,15 @@ def test_attention_plan_of_the_benchmarked_round():
     assert (b["QT"], b["q_tiles"], b["NW"], b["S"], b["tc"]) == (33, 1, 9, 1, 0)
     b = plan_attention(64, 32, 32, 8, 4096 + 32)
     assert (b["QT"], b["q_tiles"], b["rows"], b["S"], b["tc"], b["tile"]) == (32, 1, 128, 1, 1, 128)
-    # the tcgen05 KV tile: 64 keys while a split holds <= 16 pages, else 128 (4128 keys = 65
-    # pages: 8 splits of 9 pages at batch 1, 2 splits of 33 at batch 8; 16416 keys at batch 1:
-    # 8 splits of 33 pages)
+    # the tcgen05 KV tile: 64 keys while a split holds <= 3 pages, else 128 (1056 keys = 17
+    # pages: 6 splits of 3 at batch 1; 4128 keys = 65 pages = 33 tiles of 128 keys: 7 splits of
+    # 5 at batch 1, 2 splits of 17 at batch 8; 16416 keys at batch 1: 8 splits of 17 tiles)
+    b = plan_attention(1, 32, 32, 8, 1056)
+    assert (b["S"], b["tc"], b["tile"]) == (6, 1, 64)
+    b = plan_attention(8, 32, 32, 8, 1056)
+    assert (b["tc"], b["tile"]) == (1, 128)
     b = plan_attention(1, 32, 32, 8, 4128)
-    assert (b["S"], b["tc"], b["tile"]) == (8, 1, 64)
+    assert (b["S"], b["tc"], b["tile"]) == (7, 1, 128)
     b = plan_attention(8, 32, 32, 8, 4128)
     assert (b["S"], b["tc"], b["tile"]) == (2, 1, 128)
     b = plan_attention(1, 32, 32, 8, 16416)
