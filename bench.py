@@ -478,7 +478,7 @@ def run_attention(args):
     stream = torch.cuda.current_stream()
     lib = nb.load_library()
     if lib.nld_debug_attention_tile(args.attn_tile) != 0:
-        raise SystemExit("--attn-tile takes 0, 64 or 128")
+        raise SystemExit("nld_debug_attention_tile refused the tile")
     points = []
     grid = [(L, B) for L in (1024, 4096, 16384, 32768) for B in (1, 8, 32)]
     if args.attn_point:
@@ -863,7 +863,7 @@ def main():
                     help="queries per sequence of the attention workload (32; 1 = single-token decode)")
     ap.add_argument("--attn-point", default="",
                     help="attention workload: one point 'prefix,batch' instead of the whole grid")
-    ap.add_argument("--attn-tile", type=int, default=0,
+    ap.add_argument("--attn-tile", type=int, default=0, choices=[0, 64, 128],
                     help="attention workload: keys per tcgen05 KV tile (0 = the planner's choice, 64, 128)")
     ap.add_argument("--probe", action="store_true",
                     help="small kernel-probe case for profiler captures (no JSON bench line)")
