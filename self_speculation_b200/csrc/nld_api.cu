@@ -499,9 +499,10 @@ std::atomic<int> g_attn_tile{0};
 
 // rows_cap: query rows (positions x heads) per CTA at most (16..144: 9 warps); min_tiles: KV
 // tiles a split takes at least; 0 = the planner's choice for either.  tile: keys per tcgen05 KV
-// tile, 0 = the planner's choice.
+// tile, 0 = the planner's choice.  hilo: q and P as (hi, lo) operand pairs (the model's
+// forwards) rather than bf16 q (the stand-alone call).
 void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs& a, const AttnCapacity& cap,
-               int rows_cap = 0, int min_tiles = 0, int kernel = 0, int tile = 0) {
+               int rows_cap = 0, int min_tiles = 0, int kernel = 0, int tile = 0, bool hilo = true) {
   a.G = Hq / Hkv;
   const int n_tiles = std::max(1, (max_len + kPage - 1) / kPage);
   auto q_tiles_for = [&](int c) {
@@ -572,9 +573,12 @@ void attn_plan(int batch, int m, int Hq, int Hkv, int max_len, int sms, AttnArgs
   // tcgen05 softmax threads per row: 4 (16 warps) shorten a CTA's fixed costs and each KV tile's
   // latency chain, which short splits wait on; 2 (8 warps) issue fewer instructions per tile,
   // which long splits are bound by (measured: 4 win at <= 17 pages per CTA by up to 20 %, 2 at
-  // 65 and 257 pages by 5-8 %, even at 33)
+  // 65 and 257 pages by 5-8 %, even at 33).  With bf16 q (half the MMAs and P stores of a
+  // tile) and at most half the SMs busy, 2 win from 8 pages (4k keys at batch 1: 18.6 vs 20.4
+  // us); the model's (hi, lo) forwards keep 4 there (14B round at a 4k prefix: 4 win by 4 %).
   if (use_tc && (kernel == 0 || kernel == 1)) {
     tc = per_pages > 32 ? 2 : 4;
+    if (!hilo && per_pages >= 8 && 2 * units * a.S <= sms) tc = 2;
     a.tc = tc;
   }
 }
@@ -2152,7 +2156,7 @@ nld_status nld_attention(const void* d_q, const void* d_kv_pool, const int32_t* 
   AttnArgs a{};
   attn_plan(batch, m, n_q_heads, n_kv_heads, max_len, device_sms(), a,
             [](int S, int NW, int stages, int tc) { return attn_device_capacity(false, S, NW, stages, tc); },
-            0, 0, g_attn_kernel.load(), g_attn_tile.load());
+            0, 0, g_attn_kernel.load(), g_attn_tile.load(), false);
   if (static_cast<long long>(batch) * a.q_tiles > 65535) return fail(nullptr, NLD_ERR_ARG, "batch*query tiles too large");
   CUtensorMap map;
   if (!make_map_bf16(&map, d_kv_pool, 128, static_cast<uint64_t>(n_pages) * 2 * n_kv_heads * kPage, kPage))
