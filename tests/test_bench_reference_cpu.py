@@ -40,3 +40,16 @@ def test_reference_line_keys_and_values():
 
 def test_reference_other_ranks_print_nothing():
     assert _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_profiling_options_parse_and_reject_bad_values():
+    """The profiling options are declared, and a KV tile the attention kernel does not have is
+    refused before anything runs."""
+    r = subprocess.run([sys.executable, "bench.py", "--help"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0
+    for opt in ("--layer-trace", "--attn-tile", "--attn-point", "--attn-m", "--probe"):
+        assert opt in r.stdout, opt
+    r = subprocess.run([sys.executable, "bench.py", "--workload", "attention", "--attn-tile", "32"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2 and "invalid choice" in r.stderr
